@@ -1,0 +1,386 @@
+"""Pins of the CPU oracle to facts outside itself (no GPU needed).
+
+Each test ties one part of the oracle to something the pages or mathematics
+fix: a worked example, a library routine that computes the same definition,
+a closed form, brute force over a tiny id range, or published test values.
+"""
+import json
+import math
+import os
+from fractions import Fraction
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import Oracle, init_row, pack_keys, splitmix64_outputs
+from tests.conftest import GOLDEN
+
+SCALE = np.float32(0.05) * np.float32(2.0 ** -23)
+
+
+def _golden(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        return json.load(f) if name.endswith(".json") else f.read()
+
+
+def _ulp(x):
+    x = np.abs(np.asarray(x, np.float32))
+    return np.spacing(x)
+
+
+# --- splitmix64 / row initialisation -------------------------------------------------
+
+def test_splitmix64_published_values():
+    txt = _golden("splitmix64_seed0.txt")
+    want = [int(l, 16) for l in txt.splitlines() if l.strip() and not l.startswith("#")]
+    assert splitmix64_outputs(0, len(want)) == want
+
+
+def test_init_row_range_grid_and_moments():
+    keys = np.arange(4000, dtype=np.int64) * 7919 + 12345
+    rows = np.stack([init_row(int(k), 32) for k in keys])
+    assert rows.min() >= -0.05 and rows.max() < 0.05
+    # every value is the fp32 product of an integer in [-2^23, 2^23) and the step
+    u = np.round(rows.astype(np.float64) / float(SCALE))
+    assert np.array_equal(u.astype(np.float32) * SCALE, rows)
+    assert u.min() >= -(2 ** 23) and u.max() < 2 ** 23
+    # uniform on [-0.05, 0.05): mean 0, variance 0.05^2/3 (128k samples)
+    assert abs(rows.mean()) < 3 * 0.05 / math.sqrt(3 * rows.size) * 1.5
+    assert abs(rows.var() / (0.05 ** 2 / 3) - 1) < 0.02
+    # elements within a row and across keys are not visibly correlated
+    c = np.corrcoef(rows[:, 0], rows[:, 1])[0, 1]
+    assert abs(c) < 0.05
+
+
+def test_init_row_uses_successive_outputs_of_the_key_stream():
+    # element j is the (j+1)-th output of the generator seeded with the key;
+    # a shifted or reused output would break this
+    for key in (0, 1, 2 ** 40 + 3, (5 << 48) | 77):
+        outs = splitmix64_outputs(key, 8)
+        row = init_row(key, 8)
+        for j, z in enumerate(outs):
+            u = np.int64(z >> 40) - 2 ** 23
+            assert row[j] == np.float32(u) * SCALE
+
+
+def test_init_independent_of_insertion_order():
+    keys = np.array([9, 3, 77, 2 ** 47, 5], np.int64)
+    a, b = Oracle(8), Oracle(8)
+    a.lookup_or_insert(keys)
+    b.lookup_or_insert(keys[::-1])
+    ra, _ = a.get_rows(keys)
+    rb, _ = b.get_rows(keys)
+    assert np.array_equal(ra, rb)
+
+
+# --- key -> row mapping ---------------------------------------------------------------
+
+def test_mapping_is_first_occurrence_order_brute_force():
+    rng = np.random.default_rng(5)
+    o = Oracle(4)
+    seen = []
+    for step in range(6):
+        keys = rng.integers(0, 50, size=int(rng.integers(0, 40)), dtype=np.int64)
+        off, rc = o.lookup_or_insert(keys)
+        assert rc == 0
+        seen.extend(keys.tolist())
+        # independent computation: distinct keys ordered by first index in the
+        # concatenated stream (np.unique + argsort of first indices)
+        allk = np.array(seen, np.int64)
+        uniq, first = np.unique(allk, return_index=True)
+        order = uniq[np.argsort(first)]
+        rank = {int(k): r for r, k in enumerate(order)}
+        assert off.tolist() == [rank[int(k)] for k in keys]
+        assert o.size == len(order)
+
+
+def test_modulo_collision_ids_get_distinct_rows():
+    g = _golden("modulo_collision.json")
+    a, b = g["ids"]
+    assert a % g["modulus"] == g["residue"] == b % g["modulus"]
+    o = Oracle(16)
+    off, _ = o.lookup_or_insert(np.array([a, b, a], np.int64))
+    assert off[0] != off[1] and off[2] == off[0]
+    rows, _ = o.get_rows(np.array([a, b], np.int64))
+    assert not np.array_equal(rows[0], rows[1])
+
+
+def test_pack_keys_layout_and_validation():
+    t = np.array([0, 1, 25, 32767, -1, 3], np.int32)
+    i = np.array([5, 5, 2 ** 48 - 1, 0, 1, 2 ** 48], np.int64)
+    k, rc = pack_keys(t, i)
+    assert k[0] == 5 and k[1] == (1 << 48) + 5
+    assert k[2] == (25 << 48) + 2 ** 48 - 1 and k[3] == 32767 << 48
+    assert k[4] == -1 and k[5] == -1 and rc != 0
+    assert np.all(k[:4] >= 0)
+
+
+# --- forward -----------------------------------------------------------------------
+
+def test_forward_matches_torch_embedding_bag_sum():
+    d = 12
+    o = Oracle(d)
+    o.lookup_or_insert(np.arange(64, dtype=np.int64))  # key k -> row k
+    _, rows = o.export()
+    weight = torch.from_numpy(rows[:, :d].copy())
+    rng = np.random.default_rng(1)
+    lens = rng.integers(0, 9, size=37)
+    lens[[0, 5, 36]] = 0  # empty bags, including the first and the last
+    offs = np.concatenate([[0], np.cumsum(lens)]).astype(np.int64)
+    keys = rng.integers(0, 64, size=int(offs[-1]), dtype=np.int64)
+    pooled, rc = o.forward(keys, offs)
+    assert rc == 0
+    ref = torch.nn.functional.embedding_bag(torch.from_numpy(keys), weight,
+                                            torch.from_numpy(offs[:-1]), mode="sum").numpy()
+    assert np.all(pooled[lens == 0] == 0)
+    np.testing.assert_allclose(pooled, ref, rtol=1e-6, atol=1e-7)
+
+
+def test_merged_tables_equal_separate_tables():
+    g = _golden("dlrm_shape_example.json")
+    bsz, d, T = g["batch"], g["dim"], g["tables"]
+    rng = np.random.default_rng(3)
+    raw = rng.integers(0, 6, size=(bsz, T)).astype(np.int64)  # same raw ids recur across tables
+    tids = np.broadcast_to(np.arange(T, dtype=np.int32), (bsz, T)).copy()
+    keys, rc = pack_keys(tids.reshape(-1), raw.reshape(-1))
+    assert rc == 0
+    merged = Oracle(d)
+    out, _ = merged.forward(keys, np.arange(bsz * T + 1, dtype=np.int64))
+    out = out.reshape(bsz, T, d)
+    for t in range(T):
+        sep = Oracle(d)
+        kt, _ = pack_keys(np.full(bsz, t, np.int32), raw[:, t])
+        ot, _ = sep.forward(kt, np.arange(bsz + 1, dtype=np.int64))
+        assert list(ot.shape) == g["per_table_shape"]
+        assert np.array_equal(out[:, t, :], ot)
+    # equal raw ids in different tables are different rows
+    assert merged.size == len({(t, int(raw[s, t])) for s in range(bsz) for t in range(T)})
+
+
+# --- backward ----------------------------------------------------------------------
+
+def test_worked_sgd_example():
+    g = _golden("worked_sgd_example.json")
+    n, d, lr, ids = g["num_embeddings"], g["dim"], g["lr"], g["ids"]
+    o = Oracle(d, "sgd")
+    o.lookup_or_insert(np.arange(n, dtype=np.int64))
+    _, before = o.export()
+    keys = np.array(ids, np.int64)
+    offs = np.arange(len(ids) + 1, dtype=np.int64)
+    vecs, _ = o.forward(keys, offs)
+    grad = 2.0 * vecs                     # dL/de for L = sum e^2
+    assert o.backward_update(keys, offs, grad, lr) == 0
+    _, after = o.export()
+    for r in range(n):
+        if r in ids:
+            want = np.float32(g["touched_factor"]) * before[r]
+            assert np.all(np.abs(after[r] - want) <= 2 * _ulp(want))
+        else:
+            assert np.array_equal(after[r], before[r])
+    # the same step through torch nn.Embedding + optim.SGD
+    emb = torch.nn.Embedding(n, d)
+    with torch.no_grad():
+        emb.weight.copy_(torch.from_numpy(before))
+    opt = torch.optim.SGD(emb.parameters(), lr=lr)
+    loss = (emb(torch.tensor(ids)) ** 2).sum()
+    opt.zero_grad()
+    loss.backward()
+    opt.step()
+    w = emb.weight.detach().numpy()
+    assert np.all(np.abs(after - w) <= _ulp(w))
+
+
+@pytest.mark.parametrize("opt", ["sgd", "adagrad"])
+def test_dense_table_equivalence(opt):
+    """Sparse touched-rows-only steps equal dense torch steps over keys [0, 64):
+    a dense SGD/Adagrad step with zero gradient leaves a row unchanged."""
+    d, V, lr, eps = 8, 64, 0.05, 1e-8
+    o = Oracle(d, opt, eps=eps)
+    o.lookup_or_insert(np.arange(V, dtype=np.int64))
+    _, rows = o.export()
+    W = torch.nn.Parameter(torch.from_numpy(rows[:, :d].copy()))
+    topt = (torch.optim.SGD([W], lr=lr) if opt == "sgd"
+            else torch.optim.Adagrad([W], lr=lr, eps=eps, initial_accumulator_value=0.0))
+    rng = np.random.default_rng(11)
+    for step in range(5):
+        lens = rng.integers(0, 6, size=23)
+        offs = np.concatenate([[0], np.cumsum(lens)]).astype(np.int64)
+        keys = rng.integers(0, 20 if step % 2 else V, size=int(offs[-1]), dtype=np.int64)
+        grad = rng.standard_normal((23, d)).astype(np.float32)
+        pooled, _ = o.forward(keys, offs)
+        assert o.backward_update(keys, offs, grad, lr) == 0
+        out = torch.nn.functional.embedding_bag(torch.from_numpy(keys), W,
+                                                torch.from_numpy(offs[:-1]), mode="sum")
+        np.testing.assert_allclose(pooled, out.detach().numpy(), rtol=1e-6, atol=1e-7)
+        topt.zero_grad()
+        (out * torch.from_numpy(grad)).sum().backward()
+        topt.step()
+    _, rows = o.export()
+    np.testing.assert_allclose(rows[:, :d], W.detach().numpy(), rtol=1e-5, atol=1e-7)
+    if opt == "adagrad":
+        G = topt.state[W]["sum"].numpy()
+        np.testing.assert_allclose(rows[:, d:], G, rtol=1e-5, atol=1e-7)
+
+
+def test_lazy_adam_matches_torch_sparse_adam():
+    d, V, lr, eps, b1, b2 = 8, 64, 1e-2, 1e-8, 0.9, 0.999
+    o = Oracle(d, "adam", eps=eps, beta1=b1, beta2=b2)
+    o.lookup_or_insert(np.arange(V, dtype=np.int64))
+    _, rows = o.export()
+    bag = torch.nn.EmbeddingBag(V, d, mode="sum", sparse=True)
+    with torch.no_grad():
+        bag.weight.copy_(torch.from_numpy(rows[:, :d]))
+    topt = torch.optim.SparseAdam(bag.parameters(), lr=lr, betas=(b1, b2), eps=eps)
+    rng = np.random.default_rng(12)
+    for step in range(6):
+        lens = rng.integers(1, 5, size=17)
+        offs = np.concatenate([[0], np.cumsum(lens)]).astype(np.int64)
+        keys = rng.integers(0, 30 if step % 2 else V, size=int(offs[-1]), dtype=np.int64)
+        grad = rng.standard_normal((17, d)).astype(np.float32)
+        o.forward(keys, offs)
+        assert o.backward_update(keys, offs, grad, lr) == 0
+        out = bag(torch.from_numpy(keys), torch.from_numpy(offs[:-1]))
+        topt.zero_grad()
+        (out * torch.from_numpy(grad)).sum().backward()
+        topt.step()
+    _, rows = o.export()
+    np.testing.assert_allclose(rows[:, :d], bag.weight.detach().numpy(), rtol=1e-5, atol=1e-6)
+    # SparseAdam moves the moments as m + (1-b1)(g-m) and v + (1-b2)(g^2-v):
+    # the same values in exact arithmetic, rounded differently (the cancellation
+    # in g^2 - v costs a few more ulps), hence the looser bound on the moments
+    st = topt.state[bag.weight]
+    np.testing.assert_allclose(rows[:, d:2 * d], st["exp_avg"].numpy(), rtol=5e-5, atol=1e-7)
+    np.testing.assert_allclose(rows[:, 2 * d:], st["exp_avg_sq"].numpy(), rtol=5e-5, atol=1e-7)
+
+
+def test_touched_rows_only():
+    d = 16
+    for opt in ("sgd", "adagrad", "adam", "adagrad_rowwise"):
+        o = Oracle(d, opt)
+        allk = np.arange(100, dtype=np.int64) * 3
+        o.lookup_or_insert(allk)
+        _, before = o.export()
+        keys = np.array([3, 3, 30, 297], np.int64)
+        offs = np.array([0, 2, 4], np.int64)
+        o.forward(keys, offs)
+        o.backward_update(keys, offs, np.ones((2, d), np.float32), 0.1)
+        _, after = o.export()
+        touched = {1, 10, 99}
+        for r in range(100):
+            assert np.array_equal(after[r], before[r]) == (r not in touched), (opt, r)
+
+
+def test_coalesce_is_the_exact_sum_rounded_once():
+    """g_k = fl(exact sum of the occurrence gradients): checked through the
+    Adagrad accumulator, G = fl(g*g) after one step from G = 0.  The grads are
+    chosen so that a running fp32 sum would round differently."""
+    d = 4
+    o = Oracle(d, "adagrad")
+    key = np.array([42], np.int64)
+    o.lookup_or_insert(key)
+    occ = 257
+    keys = np.full(occ, 42, np.int64)
+    offs = np.arange(occ + 1, dtype=np.int64)
+    g = np.zeros((occ, d), np.float32)
+    g[0] = [1.0, -1.0, 3.0, 0.5]
+    g[1:] = np.float32(2.0 ** -25)          # each one alone is lost in fp32 next to 1.0
+    g[1:, 2] = np.float32(-1e-3)
+    o.backward_update(keys, offs, g, 0.0)
+    rows, _ = o.get_rows(key)
+    for j in range(d):
+        exact = sum((Fraction(float(x)) for x in g[:, j]), Fraction(0))
+        gj = np.float32(float(exact))        # round once
+        assert rows[0, d + j] == gj * gj, j
+    # and a running fp32 sum would have given another value in column 0
+    run = np.float32(0)
+    for x in g[:, 0]:
+        run = np.float32(run + x)
+    assert run != np.float32(float(sum(Fraction(float(x)) for x in g[:, 0])))
+
+
+def test_adagrad_closed_form():
+    d, lr, eps, T = 4, 0.01, 1e-8, 50
+    o = Oracle(d, "adagrad", eps=eps)
+    key = np.array([7], np.int64)
+    o.lookup_or_insert(key)
+    w0, _ = o.get_rows(key)
+    gval = np.array([0.5, -0.25, 2.0, 1.0], np.float32)
+    for _ in range(T):
+        o.backward_update(key, np.array([0, 1], np.int64), gval[None, :], lr)
+    rows, _ = o.get_rows(key)
+    # G_t = t g^2 ; w_T = w_0 - sum_t lr g / (sqrt(t) |g| + eps)
+    for j in range(d):
+        g = float(gval[j])
+        want_w = float(w0[0, j]) - sum(lr * g / (math.sqrt(t) * abs(g) + eps) for t in range(1, T + 1))
+        assert rows[0, d + j] == np.float32(T * g * g)
+        assert abs(rows[0, j] - want_w) <= 1e-5 * abs(want_w) + 1e-7
+
+
+def test_adam_closed_form_constant_gradient():
+    """With a constant gradient, bias-corrected moments equal g and g^2, so each
+    step moves the weight by lr * g / (|g| + eps)."""
+    d, lr, eps, T = 4, 1e-3, 1e-8, 40
+    o = Oracle(d, "adam", eps=eps, beta1=0.9, beta2=0.999)
+    key = np.array([11], np.int64)
+    o.lookup_or_insert(key)
+    w0, _ = o.get_rows(key)
+    gval = np.array([0.5, -0.25, 2.0, -1.0], np.float32)
+    for _ in range(T):
+        o.backward_update(key, np.array([0, 1], np.int64), gval[None, :], lr)
+    rows, _ = o.get_rows(key)
+    for j in range(d):
+        g = float(gval[j])
+        want = float(w0[0, j]) - T * lr * g / (abs(g) + eps)
+        assert abs(rows[0, j] - want) <= 1e-4 * T * lr
+        assert abs(rows[0, d + j] - (1 - 0.9 ** T) * g) <= 1e-5 * abs(g)
+        assert abs(rows[0, 2 * d + j] - (1 - 0.999 ** T) * g * g) <= 1e-5 * g * g
+
+
+def test_rowwise_adagrad_single_accumulator():
+    d, lr, eps = 8, 0.1, 1e-8
+    o = Oracle(d, "adagrad_rowwise", eps=eps)
+    assert o.stride == d + 1
+    key = np.array([5], np.int64)
+    o.lookup_or_insert(key)
+    w0, _ = o.get_rows(key)
+    g = np.arange(1, d + 1, dtype=np.float32)[None, :]
+    o.backward_update(key, np.array([0, 1], np.int64), g, lr)
+    rows, _ = o.get_rows(key)
+    G = float(np.mean(g.astype(np.float64) ** 2))     # 25.5
+    assert rows[0, d] == np.float32(G)
+    want = w0[0, :d].astype(np.float64) - lr * g[0] / (math.sqrt(G) + eps)
+    np.testing.assert_allclose(rows[0, :d], want, rtol=1e-6)
+
+
+# --- error handling and degenerate cases ------------------------------------------
+
+def test_missing_and_negative_keys_are_reported_and_skipped():
+    o = Oracle(4, "sgd")
+    o.lookup_or_insert(np.array([1, 2], np.int64))
+    _, before = o.export()
+    rc = o.backward_update(np.array([1, 99], np.int64), np.array([0, 1, 2], np.int64),
+                           np.ones((2, 4), np.float32), 0.5)
+    assert rc == 5
+    _, after = o.export()
+    assert not np.array_equal(after[0], before[0]) and np.array_equal(after[1], before[1])
+    assert o.size == 2
+    off, rc = o.lookup_or_insert(np.array([-3, 2], np.int64))
+    assert rc == 1 and off.tolist() == [-1, 1]
+
+
+def test_empty_batch_and_empty_bags():
+    o = Oracle(4, "adam")
+    out, rc = o.forward(np.zeros(0, np.int64), np.array([0], np.int64))
+    assert out.shape == (0, 4) and rc == 0
+    out, rc = o.forward(np.zeros(0, np.int64), np.array([0, 0, 0], np.int64))
+    assert np.all(out == 0) and o.size == 0
+    assert o.backward_update(np.zeros(0, np.int64), np.array([0, 0], np.int64),
+                             np.ones((1, 4), np.float32), 0.1) == 0
+
+
+def test_bytes_per_row_arithmetic():
+    g = _golden("memory_arith.json")
+    for c in g["cases"]:
+        gb = c["rows"] * c["dim"] * c["bytes_per_float"] / 1e9
+        assert abs(gb - c["stated_gb"]) / c["stated_gb"] < 0.03
