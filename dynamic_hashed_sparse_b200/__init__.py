@@ -1,0 +1,30 @@
+"""B200 dynamic hashed embedding engine: IDMap + EmbeddingBlocks, lookup-or-
+insert + sum-pooling forward, coalesced sparse-gradient + fused optimizer
+backward, all in the CUDA kernels of libdhs.so (C ABI: include/dhs.h).
+
+This package is the thin Python binding of that library.
+"""
+from ._binding import (  # noqa: F401
+    DhsError,
+    OPT_CODES,
+    PHASES,
+    Table,
+    dhs_pack_keys,
+    dhs_status_str,
+    embbag_backward_update,
+    embbag_forward,
+    ht_counters,
+    ht_create,
+    ht_destroy,
+    ht_export,
+    ht_get_rows,
+    ht_lookup,
+    ht_lookup_or_insert,
+    ht_phase_times,
+    ht_reserve,
+    ht_row_stride,
+    ht_set_phase_timing,
+    ht_size,
+    ht_sync,
+    lib,
+)

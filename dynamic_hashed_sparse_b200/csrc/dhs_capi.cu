@@ -1,0 +1,819 @@
+// C ABI of the dynamic hashed embedding engine (see include/dhs.h).
+//
+// Host side: table lifecycle, growth of the IDMap (rehash of keys and
+// offsets only; rows never move) and of the EmbeddingBlocks (append), the
+// per-call workspace, and the launch sequence of each call.  Every step of
+// every call runs in the kernels of dhs_fwd.cuh / dhs_bwd.cuh; the host only
+// sizes, allocates and launches.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <new>
+#include <vector>
+
+#include "../../include/dhs.h"
+#include "dhs_bwd.cuh"
+#include "dhs_device.cuh"
+#include "dhs_fwd.cuh"
+#include "dhs_launch.h"
+
+using namespace dhs;
+
+namespace {
+
+constexpr long long kDefaultBlockRows = 1ll << 20;
+constexpr long long kDefaultMaxRows = 1ll << 31;
+constexpr long long kMaxRowsLimit = (1ll << 32) - 2;
+constexpr unsigned long long kInitialSlots = 1ull << 16;
+constexpr double kMaxLoad = 0.5;
+constexpr int kSegChunk = 256;
+constexpr int kSnapRing = 4;
+enum { PH_FWD_POOL = 0, PH_FWD_ASSIGN = 1, PH_BWD_PROBE = 2, PH_BWD_SORT = 3, PH_BWD_SEG = 4,
+       PH_LOOKUP_INSERT = 5, PH_GROW = 6 };
+
+struct Snap {
+  cudaEvent_t ev = nullptr;
+  unsigned long long* pinned = nullptr;  // row_count copied here
+  long long cum_n = 0;                   // inserted-key upper bound counter at record time
+  bool valid = false;
+};
+
+struct PhaseRec {
+  int phase;
+  cudaEvent_t a, b;
+};
+
+struct Buf {
+  void* p = nullptr;
+  size_t bytes = 0;
+};
+
+int pick_group(int dim) {
+  int need = (dim + 3) / 4;
+  int g = 1;
+  while (g < need && g < 32) g <<= 1;
+  return g;
+}
+
+// float4 columns per lane: 1, 2 or 4 (the kernels are instantiated for these)
+int pick_nv(int dim, int g) {
+  const int need = (dim / 4 + g - 1) / g;
+  int v = 1;
+  while (v < need) v <<= 1;
+  return v;
+}
+
+int log2_exact(long long x) {
+  int l = 0;
+  while ((1ll << l) < x) ++l;
+  return l;
+}
+
+}  // namespace
+
+struct dhs_table {
+  int device = 0;
+  int sm_count = 148;
+  int dim = 0, opt = 0, stride = 0;
+  float eps = 1e-8f, b1 = 0.9f, b2 = 0.999f;
+  long long adam_t = 0;
+  long long block_rows = kDefaultBlockRows;
+  int log2_br = 20;
+  long long max_rows = kDefaultMaxRows;
+  long long max_blocks = 0;
+  dhs_allocator alloc{};
+  bool custom_alloc = false;
+  cudaStream_t last_stream = nullptr;
+
+  Slot* slots = nullptr;
+  unsigned long long nslots = 0;
+  long long n_rehash = 0;
+  long long n_insert_calls = 0;
+
+  std::vector<float*> blocks_h;
+  float** blocks_d = nullptr;
+  DevState* st = nullptr;
+
+  // upper bound on the device row count after all enqueued work
+  long long rows_ub = 0;
+  long long cum_n = 0;  // sum of key counts of all insert calls
+  Snap snaps[kSnapRing];
+  int snap_next = 0;
+
+  // workspace, sized for ws_n positions
+  long long ws_n = -1;
+  Buf b_nbm, b_fbm, b_gcnt, b_gpref, b_slotpos, b_ka, b_va, b_kb, b_vb, b_hist, b_totals, b_ph,
+      b_pt, b_cflags;
+
+  bool timing = false;
+  std::vector<PhaseRec> recs;
+  std::vector<cudaEvent_t> ev_pool;
+};
+
+namespace {
+
+void* dalloc(dhs_table* t, size_t bytes, cudaStream_t s) {
+  if (bytes == 0) bytes = 16;
+  if (t->custom_alloc) return t->alloc.alloc(bytes, (dhs_stream)s, t->alloc.ctx);
+  void* p = nullptr;
+  if (cudaMallocAsync(&p, bytes, s) != cudaSuccess) {
+    cudaGetLastError();
+    return nullptr;
+  }
+  return p;
+}
+
+void dfree(dhs_table* t, void* p, size_t bytes, cudaStream_t s) {
+  if (!p) return;
+  if (t->custom_alloc)
+    t->alloc.free(p, bytes ? bytes : 16, (dhs_stream)s, t->alloc.ctx);
+  else
+    cudaFreeAsync(p, s);
+}
+
+dhs_status bget(dhs_table* t, Buf& b, size_t bytes, cudaStream_t s) {
+  if (b.bytes >= bytes && b.p) return DHS_OK;
+  dfree(t, b.p, b.bytes, s);
+  b.p = dalloc(t, bytes, s);
+  b.bytes = b.p ? bytes : 0;
+  return b.p ? DHS_OK : DHS_ERR_OOM;
+}
+
+void bfree(dhs_table* t, Buf& b, cudaStream_t s) {
+  dfree(t, b.p, b.bytes, s);
+  b.p = nullptr;
+  b.bytes = 0;
+}
+
+struct DeviceGuard {
+  int prev = -1;
+  explicit DeviceGuard(int dev) {
+    int cur = -1;
+    if (cudaGetDevice(&cur) == cudaSuccess && cur != dev) {
+      prev = cur;
+      cudaSetDevice(dev);
+    }
+  }
+  ~DeviceGuard() {
+    if (prev >= 0) cudaSetDevice(prev);
+  }
+};
+
+dhs_status last_launch() {
+  cudaError_t e = cudaGetLastError();
+  if (e == cudaSuccess) return DHS_OK;
+  return e == cudaErrorMemoryAllocation ? DHS_ERR_OOM : DHS_ERR_CUDA;
+}
+
+#define DHS_TRY(x)                  \
+  do {                              \
+    dhs_status _s = (x);            \
+    if (_s != DHS_OK) return _s;    \
+  } while (0)
+
+#define DHS_CUDA(x)                                         \
+  do {                                                      \
+    if ((x) != cudaSuccess) {                               \
+      cudaGetLastError();                                   \
+      return DHS_ERR_CUDA;                                  \
+    }                                                       \
+  } while (0)
+
+IdMap idmap(const dhs_table* t) { return IdMap{t->slots, t->nslots / 2 - 1}; }
+
+RowSpace rowspace(const dhs_table* t) {
+  return RowSpace{t->blocks_d, (unsigned long long)t->block_rows - 1, t->log2_br, t->stride};
+}
+
+// ---- phase timing ----
+cudaEvent_t ev_get(dhs_table* t) {
+  if (!t->ev_pool.empty()) {
+    cudaEvent_t e = t->ev_pool.back();
+    t->ev_pool.pop_back();
+    return e;
+  }
+  cudaEvent_t e = nullptr;
+  cudaEventCreate(&e);
+  return e;
+}
+
+struct PhaseScope {
+  dhs_table* t;
+  int phase;
+  cudaStream_t s;
+  cudaEvent_t a = nullptr;
+  PhaseScope(dhs_table* t_, int ph, cudaStream_t s_) : t(t_), phase(ph), s(s_) {
+    if (t->timing) {
+      a = ev_get(t);
+      cudaEventRecord(a, s);
+    }
+  }
+  ~PhaseScope() {
+    if (a) {
+      cudaEvent_t b = ev_get(t);
+      cudaEventRecord(b, s);
+      t->recs.push_back(PhaseRec{phase, a, b});
+    }
+  }
+};
+
+// ---- grid sizing ----
+template <typename K>
+int resident_blocks(K kernel, int threads, size_t smem, int sm_count) {
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, threads, smem) != cudaSuccess ||
+      per_sm < 1) {
+    cudaGetLastError();
+    per_sm = 1;
+  }
+  return per_sm * sm_count;
+}
+
+long long grid_for(long long units_per_block_needed, int resident) {
+  if (units_per_block_needed < 1) return 1;
+  return std::min<long long>(units_per_block_needed, resident);
+}
+
+// ---- row-count bookkeeping ----
+// Use the newest finished snapshot of the device row count to tighten the
+// host's upper bound; with `wait`, wait for the newest recorded snapshot.
+void refresh_ub(dhs_table* t, bool wait) {
+  for (int i = 0; i < kSnapRing; ++i) {
+    const int k = ((t->snap_next - 1 - i) % kSnapRing + kSnapRing) % kSnapRing;
+    Snap& sn = t->snaps[k];
+    if (!sn.valid) continue;
+    cudaError_t q = wait && i == 0 ? cudaEventSynchronize(sn.ev) : cudaEventQuery(sn.ev);
+    if (q == cudaSuccess) {
+      const long long ub = (long long)*sn.pinned + (t->cum_n - sn.cum_n);
+      if (ub < t->rows_ub) t->rows_ub = ub;
+      return;
+    }
+    cudaGetLastError();
+  }
+}
+
+void record_snapshot(dhs_table* t, cudaStream_t s) {
+  Snap& sn = t->snaps[t->snap_next];
+  if (sn.valid) cudaEventSynchronize(sn.ev);  // ring slot reuse: at most kSnapRing in flight
+  cudaMemcpyAsync(sn.pinned, &t->st->row_count, sizeof(unsigned long long), cudaMemcpyDeviceToHost, s);
+  cudaEventRecord(sn.ev, s);
+  sn.cum_n = t->cum_n;
+  sn.valid = true;
+  t->snap_next = (t->snap_next + 1) % kSnapRing;
+}
+
+__global__ void set_block_kernel(float** blocks_d, long long idx, float* ptr, DevState* st,
+                                 unsigned long long n_blocks) {
+  blocks_d[idx] = ptr;
+  st->n_blocks = n_blocks;
+}
+
+dhs_status grow_map(dhs_table* t, unsigned long long want_slots, cudaStream_t s) {
+  PhaseScope ph(t, PH_GROW, s);
+  unsigned long long ns = std::max<unsigned long long>(t->nslots * 2, kInitialSlots);
+  while (ns < want_slots) ns <<= 1;
+  Slot* fresh = (Slot*)dalloc(t, ns * sizeof(Slot), s);
+  if (!fresh) return DHS_ERR_OOM;
+  const int thr = 256;
+  const long long g = std::min<long long>((long long)((ns + thr - 1) / thr), (long long)t->sm_count * 16);
+  fill_empty_kernel<<<(unsigned)g, thr, 0, s>>>(fresh, ns);
+  if (t->slots) {
+    IdMap to{fresh, ns / 2 - 1};
+    const long long g2 = std::min<long long>((long long)((t->nslots + thr - 1) / thr), (long long)t->sm_count * 16);
+    rehash_kernel<<<(unsigned)g2, thr, 0, s>>>(t->slots, t->nslots, to, t->st);
+    dfree(t, t->slots, t->nslots * sizeof(Slot), s);
+    t->n_rehash++;
+  }
+  t->slots = fresh;
+  t->nslots = ns;
+  return last_launch();
+}
+
+// Make room for up to `n` new keys: IDMap load <= kMaxLoad and blocks
+// covering the row upper bound.
+dhs_status ensure_capacity(dhs_table* t, long long n, cudaStream_t s) {
+  refresh_ub(t, false);
+  long long need = t->rows_ub + n;
+  if (need > t->max_rows) {
+    refresh_ub(t, true);
+    need = t->rows_ub + n;
+    if (need > t->max_rows) return DHS_ERR_TABLE_FULL;
+  }
+  if ((double)need > kMaxLoad * (double)t->nslots) {
+    refresh_ub(t, true);
+    need = t->rows_ub + n;
+    if ((double)need > kMaxLoad * (double)t->nslots)
+      DHS_TRY(grow_map(t, (unsigned long long)std::ceil((double)need / kMaxLoad), s));
+  }
+  long long have = (long long)t->blocks_h.size() * t->block_rows;
+  if (need > have) {
+    refresh_ub(t, true);
+    need = t->rows_ub + n;
+  }
+  while (need > have) {
+    if ((long long)t->blocks_h.size() >= t->max_blocks) return DHS_ERR_TABLE_FULL;
+    const size_t bytes = (size_t)t->block_rows * t->stride * sizeof(float);
+    float* b = (float*)dalloc(t, bytes, s);
+    if (!b) return DHS_ERR_OOM;
+    t->blocks_h.push_back(b);
+    set_block_kernel<<<1, 1, 0, s>>>(t->blocks_d, (long long)t->blocks_h.size() - 1, b, t->st,
+                                     (unsigned long long)t->blocks_h.size());
+    DHS_TRY(last_launch());
+    have += t->block_rows;
+  }
+  return DHS_OK;
+}
+
+dhs_status ensure_ws(dhs_table* t, long long n, cudaStream_t s) {
+  if (n <= t->ws_n) return DHS_OK;
+  long long cap = std::max<long long>(n, t->ws_n > 0 ? t->ws_n + t->ws_n / 2 : 0);
+  cap = std::max<long long>(cap, 4096);
+  const long long nwords = (cap + 31) / 32 + 32;
+  const long long ngroups = (cap + 1023) / 1024 + 1;
+  const long long ntiles = (cap + kRadixTile - 1) / kRadixTile;
+  const long long nchunks = (cap + kSegChunk - 1) / kSegChunk;
+  const int G = pick_group(t->dim), NV = pick_nv(t->dim, G);
+  const long long pstride = (long long)NV * G * 4;
+  DHS_TRY(bget(t, t->b_nbm, nwords * 4, s));
+  DHS_TRY(bget(t, t->b_fbm, nwords * 4, s));
+  DHS_TRY(bget(t, t->b_gcnt, ngroups * 4, s));
+  DHS_TRY(bget(t, t->b_gpref, ngroups * 4, s));
+  DHS_TRY(bget(t, t->b_slotpos, cap * 4, s));
+  DHS_TRY(bget(t, t->b_ka, cap * 4, s));
+  DHS_TRY(bget(t, t->b_va, cap * 4, s));
+  DHS_TRY(bget(t, t->b_kb, cap * 4, s));
+  DHS_TRY(bget(t, t->b_vb, cap * 4, s));
+  DHS_TRY(bget(t, t->b_hist, (size_t)kRadixBins * ntiles * 4, s));
+  DHS_TRY(bget(t, t->b_totals, kRadixBins * 4, s));
+  DHS_TRY(bget(t, t->b_ph, (size_t)nchunks * pstride * 8, s));
+  DHS_TRY(bget(t, t->b_pt, (size_t)nchunks * pstride * 8, s));
+  DHS_TRY(bget(t, t->b_cflags, nchunks, s));
+  DHS_CUDA(cudaMemsetAsync(t->b_nbm.p, 0, t->b_nbm.bytes, s));
+  t->ws_n = cap;
+  return DHS_OK;
+}
+
+dhs_status check_table(const dhs_table* t) { return t ? DHS_OK : DHS_ERR_INVALID_ARG; }
+
+// ---- kernel dispatch on the row width ----
+dhs_status dispatch_pool(dhs_table* t, const long long* keys, long long n, const long long* bo,
+                         long long nb, float* out, cudaStream_t s) {
+  const int G = pick_group(t->dim), NV = pick_nv(t->dim, G);
+  const cudaError_t e = launch_probe_pool(G, NV, t->sm_count, idmap(t), rowspace(t), t->dim, keys, n,
+                                          bo, nb, out, (unsigned*)t->b_nbm.p,
+                                          (unsigned*)t->b_slotpos.p, t->st, s);
+  if (e != cudaSuccess) cudaGetLastError();
+  return e == cudaSuccess ? DHS_OK : DHS_ERR_CUDA;
+}
+
+dhs_status dispatch_seg(dhs_table* t, const unsigned* sk, const unsigned* sv, long long n,
+                        const float* grad, long long nb, const OptArgs& oa, cudaStream_t s) {
+  const int G = pick_group(t->dim), NV = pick_nv(t->dim, G);
+  const cudaError_t e = launch_seg(G, NV, t->sm_count, sk, sv, n, grad, nb, t->dim, rowspace(t), oa,
+                                   (double*)t->b_ph.p, (double*)t->b_pt.p,
+                                   (unsigned char*)t->b_cflags.p, kSegChunk, t->st, s);
+  if (e != cudaSuccess) cudaGetLastError();
+  return e == cudaSuccess ? DHS_OK : DHS_ERR_CUDA;
+}
+
+// offset assignment + row init for the new keys of an insert call
+dhs_status launch_assign(dhs_table* t, long long n, cudaStream_t s) {
+  const long long nwords = (n + 31) / 32;
+  const long long ngroups = (n + 1023) / 1024;
+  fwd_mark_kernel<<<(unsigned)((nwords + 255) / 256), 256, 0, s>>>(
+      t->slots, (unsigned*)t->b_nbm.p, (unsigned*)t->b_fbm.p, (unsigned*)t->b_gcnt.p,
+      (unsigned*)t->b_gpref.p, (const unsigned*)t->b_slotpos.p, nwords, ngroups, t->st);
+  DHS_TRY(last_launch());
+  fwd_assign_kernel<<<(unsigned)((ngroups + kAssignWarps - 1) / kAssignWarps), kAssignWarps * 32, 0, s>>>(
+      t->slots, rowspace(t), t->dim, (const unsigned*)t->b_fbm.p, (const unsigned*)t->b_gpref.p,
+      (const unsigned*)t->b_slotpos.p, nwords, ngroups, t->st);
+  return last_launch();
+}
+
+int state_floats(int opt, int dim) {
+  switch (opt) {
+    case DHS_SGD: return 0;
+    case DHS_ADAGRAD: return dim;
+    case DHS_ADAM: return 2 * dim;
+    case DHS_ADAGRAD_ROWWISE: return 4;  // accumulator + 3 pad floats (16-byte rows)
+  }
+  return -1;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* dhs_status_str(dhs_status s) {
+  switch (s) {
+    case DHS_OK: return "ok";
+    case DHS_ERR_INVALID_ARG: return "invalid argument";
+    case DHS_ERR_OOM: return "out of device memory";
+    case DHS_ERR_CUDA: return "CUDA error";
+    case DHS_ERR_TABLE_FULL: return "table full";
+    case DHS_ERR_NOT_FOUND: return "key not found";
+    case DHS_ERR_UNSUPPORTED: return "unsupported";
+  }
+  return "unknown status";
+}
+
+dhs_status dhs_pack_keys(const int32_t* d_table_ids, const int64_t* d_ids, int64_t n,
+                         int64_t* d_keys_out, dhs_stream stream) {
+  if (n < 0 || (n > 0 && (!d_table_ids || !d_ids || !d_keys_out))) return DHS_ERR_INVALID_ARG;
+  if (n == 0) return DHS_OK;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const long long grid = std::min<long long>((n + 255) / 256, (long long)sms * 8);
+  pack_keys_kernel<<<(unsigned)grid, 256, 0, (cudaStream_t)stream>>>(
+      d_table_ids, (const long long*)d_ids, n, (long long*)d_keys_out);
+  return last_launch();
+}
+
+dhs_status ht_create(int32_t dim, dhs_optimizer opt, int64_t block_rows, int64_t max_rows,
+                     const dhs_opt_params* params, const dhs_allocator* alloc, dhs_table** out) {
+  if (!out) return DHS_ERR_INVALID_ARG;
+  *out = nullptr;
+  if (dim < 4 || dim > 512 || dim % 4) return DHS_ERR_INVALID_ARG;
+  if (state_floats(opt, dim) < 0) return DHS_ERR_INVALID_ARG;
+  if (block_rows == 0) block_rows = kDefaultBlockRows;
+  if (block_rows < 1 || (block_rows & (block_rows - 1)) || block_rows > (1ll << 30))
+    return DHS_ERR_INVALID_ARG;
+  if (max_rows == 0) max_rows = kDefaultMaxRows;
+  if (max_rows < 1 || max_rows > kMaxRowsLimit) return DHS_ERR_INVALID_ARG;
+  if (alloc && (!alloc->alloc || !alloc->free)) return DHS_ERR_INVALID_ARG;
+  if (params && !(params->eps >= 0.f && params->beta1 >= 0.f && params->beta1 < 1.f &&
+                  params->beta2 >= 0.f && params->beta2 < 1.f))
+    return DHS_ERR_INVALID_ARG;
+
+  dhs_table* t = new (std::nothrow) dhs_table();
+  if (!t) return DHS_ERR_OOM;
+  if (cudaGetDevice(&t->device) != cudaSuccess) {
+    cudaGetLastError();
+    delete t;
+    return DHS_ERR_CUDA;
+  }
+  cudaDeviceGetAttribute(&t->sm_count, cudaDevAttrMultiProcessorCount, t->device);
+  t->dim = dim;
+  t->opt = opt;
+  t->stride = dim + state_floats(opt, dim);
+  if (params) {
+    t->eps = params->eps;
+    t->b1 = params->beta1;
+    t->b2 = params->beta2;
+  }
+  t->block_rows = block_rows;
+  t->log2_br = log2_exact(block_rows);
+  t->max_rows = max_rows;
+  t->max_blocks = (max_rows + block_rows - 1) / block_rows;
+  if (alloc) {
+    t->alloc = *alloc;
+    t->custom_alloc = true;
+  }
+  cudaStream_t s = nullptr;
+  dhs_status rc = DHS_OK;
+  t->st = (DevState*)dalloc(t, sizeof(DevState), s);
+  t->blocks_d = (float**)dalloc(t, sizeof(float*) * t->max_blocks, s);
+  if (!t->st || !t->blocks_d) rc = DHS_ERR_OOM;
+  if (rc == DHS_OK && cudaMemsetAsync(t->st, 0, sizeof(DevState), s) != cudaSuccess) rc = DHS_ERR_CUDA;
+  if (rc == DHS_OK && cudaMemsetAsync(t->blocks_d, 0, sizeof(float*) * t->max_blocks, s) != cudaSuccess)
+    rc = DHS_ERR_CUDA;
+  for (int i = 0; rc == DHS_OK && i < kSnapRing; ++i) {
+    if (cudaEventCreateWithFlags(&t->snaps[i].ev, cudaEventDisableTiming) != cudaSuccess ||
+        cudaHostAlloc((void**)&t->snaps[i].pinned, sizeof(unsigned long long), cudaHostAllocDefault) != cudaSuccess)
+      rc = DHS_ERR_CUDA;
+  }
+  if (rc == DHS_OK) rc = grow_map(t, kInitialSlots, s);
+  if (rc == DHS_OK && cudaStreamSynchronize(s) != cudaSuccess) rc = DHS_ERR_CUDA;
+  if (rc != DHS_OK) {
+    cudaGetLastError();
+    ht_destroy(t);
+    return rc;
+  }
+  t->last_stream = s;
+  *out = t;
+  return DHS_OK;
+}
+
+dhs_status ht_destroy(dhs_table* t) {
+  if (!t) return DHS_OK;
+  DeviceGuard g(t->device);
+  cudaStream_t s = t->last_stream;
+  cudaStreamSynchronize(s);
+  cudaDeviceSynchronize();
+  s = nullptr;
+  for (float* b : t->blocks_h) dfree(t, b, (size_t)t->block_rows * t->stride * sizeof(float), s);
+  t->blocks_h.clear();
+  dfree(t, t->slots, t->nslots * sizeof(Slot), s);
+  dfree(t, t->blocks_d, sizeof(float*) * t->max_blocks, s);
+  dfree(t, t->st, sizeof(DevState), s);
+  Buf* bufs[] = {&t->b_nbm, &t->b_fbm, &t->b_gcnt, &t->b_gpref, &t->b_slotpos, &t->b_ka, &t->b_va,
+                 &t->b_kb, &t->b_vb, &t->b_hist, &t->b_totals, &t->b_ph, &t->b_pt, &t->b_cflags};
+  for (Buf* b : bufs) bfree(t, *b, s);
+  cudaStreamSynchronize(s);
+  for (auto& sn : t->snaps) {
+    if (sn.ev) cudaEventDestroy(sn.ev);
+    if (sn.pinned) cudaFreeHost(sn.pinned);
+  }
+  for (auto& r : t->recs) {
+    cudaEventDestroy(r.a);
+    cudaEventDestroy(r.b);
+  }
+  for (cudaEvent_t e : t->ev_pool) cudaEventDestroy(e);
+  cudaGetLastError();
+  delete t;
+  return DHS_OK;
+}
+
+dhs_status ht_reserve(dhs_table* t, int64_t n_keys, dhs_stream stream) {
+  DHS_TRY(check_table(t));
+  if (n_keys < 0) return DHS_ERR_INVALID_ARG;
+  DeviceGuard g(t->device);
+  cudaStream_t s = (cudaStream_t)stream;
+  t->last_stream = s;
+  if ((double)n_keys > kMaxLoad * (double)t->nslots)
+    DHS_TRY(grow_map(t, (unsigned long long)std::ceil((double)n_keys / kMaxLoad), s));
+  return DHS_OK;
+}
+
+dhs_status ht_lookup_or_insert(dhs_table* t, const int64_t* d_keys, int64_t n,
+                               int64_t* d_offsets_out, dhs_stream stream) {
+  DHS_TRY(check_table(t));
+  if (n < 0 || n >= (1ll << 31) || (n > 0 && (!d_keys || !d_offsets_out))) return DHS_ERR_INVALID_ARG;
+  if (n == 0) return DHS_OK;
+  DeviceGuard g(t->device);
+  cudaStream_t s = (cudaStream_t)stream;
+  t->last_stream = s;
+  DHS_TRY(ensure_capacity(t, n, s));
+  DHS_TRY(ensure_ws(t, n, s));
+  {
+    PhaseScope ph(t, PH_LOOKUP_INSERT, s);
+    fwd_probe_offsets_kernel<<<(unsigned)((n + kFwdThreads - 1) / kFwdThreads), kFwdThreads, 0, s>>>(
+        idmap(t), (const long long*)d_keys, n, (long long*)d_offsets_out, (unsigned*)t->b_nbm.p,
+        (unsigned*)t->b_slotpos.p, t->st);
+    DHS_TRY(last_launch());
+    DHS_TRY(launch_assign(t, n, s));
+    const long long grid = std::min<long long>((n + 255) / 256, (long long)t->sm_count * 8);
+    fwd_fixup_kernel<<<(unsigned)grid, 256, 0, s>>>(t->slots, (long long*)d_offsets_out, n);
+    DHS_TRY(last_launch());
+  }
+  t->rows_ub += n;
+  t->cum_n += n;
+  t->n_insert_calls++;
+  record_snapshot(t, s);
+  return DHS_OK;
+}
+
+dhs_status ht_lookup(dhs_table* t, const int64_t* d_keys, int64_t n, int64_t* d_offsets_out,
+                     dhs_stream stream) {
+  DHS_TRY(check_table(t));
+  if (n < 0 || (n > 0 && (!d_keys || !d_offsets_out))) return DHS_ERR_INVALID_ARG;
+  if (n == 0) return DHS_OK;
+  DeviceGuard g(t->device);
+  cudaStream_t s = (cudaStream_t)stream;
+  t->last_stream = s;
+  const long long grid = std::min<long long>((n + 255) / 256, (long long)t->sm_count * 16);
+  lookup_kernel<<<(unsigned)grid, 256, 0, s>>>(idmap(t), (const long long*)d_keys, n, (long long*)d_offsets_out);
+  return last_launch();
+}
+
+dhs_status embbag_forward(dhs_table* t, const int64_t* d_keys, int64_t n_keys,
+                          const int64_t* d_bag_offsets, int64_t n_bags, float* d_pooled_out,
+                          dhs_stream stream) {
+  DHS_TRY(check_table(t));
+  if (n_keys < 0 || n_keys >= (1ll << 31) || n_bags < 0 || n_bags >= (1ll << 31))
+    return DHS_ERR_INVALID_ARG;
+  if (n_bags == 0) return n_keys == 0 ? DHS_OK : DHS_ERR_INVALID_ARG;
+  if (!d_bag_offsets || !d_pooled_out || (n_keys > 0 && !d_keys)) return DHS_ERR_INVALID_ARG;
+  DeviceGuard g(t->device);
+  cudaStream_t s = (cudaStream_t)stream;
+  t->last_stream = s;
+  if (n_keys > 0) DHS_TRY(ensure_capacity(t, n_keys, s));
+  DHS_TRY(ensure_ws(t, n_keys, s));
+  {
+    PhaseScope ph(t, PH_FWD_POOL, s);
+    DHS_TRY(dispatch_pool(t, (const long long*)d_keys, n_keys, (const long long*)d_bag_offsets,
+                          n_bags, d_pooled_out, s));
+  }
+  if (n_keys > 0) {
+    PhaseScope ph(t, PH_FWD_ASSIGN, s);
+    DHS_TRY(launch_assign(t, n_keys, s));
+  }
+  t->n_insert_calls++;
+  if (n_keys > 0) {
+    t->rows_ub += n_keys;
+    t->cum_n += n_keys;
+    record_snapshot(t, s);
+  }
+  return DHS_OK;
+}
+
+dhs_status embbag_backward_update(dhs_table* t, const int64_t* d_keys, int64_t n_keys,
+                                  const int64_t* d_bag_offsets, int64_t n_bags,
+                                  const float* d_grad, float lr, dhs_stream stream) {
+  DHS_TRY(check_table(t));
+  if (n_keys < 0 || n_keys >= (1ll << 31) || n_bags < 0 || n_bags >= (1ll << 31))
+    return DHS_ERR_INVALID_ARG;
+  if (n_bags == 0 && n_keys != 0) return DHS_ERR_INVALID_ARG;
+  if (n_bags > 0 && (!d_bag_offsets || !d_grad)) return DHS_ERR_INVALID_ARG;
+  if (n_keys > 0 && !d_keys) return DHS_ERR_INVALID_ARG;
+  if (!std::isfinite(lr)) return DHS_ERR_INVALID_ARG;
+  DeviceGuard g(t->device);
+  cudaStream_t s = (cudaStream_t)stream;
+  t->last_stream = s;
+  t->adam_t += 1;
+  if (n_keys == 0) return DHS_OK;
+  DHS_TRY(ensure_ws(t, n_keys, s));
+
+  // rows of the table are < rows_ub; rows_ub itself marks a missing key
+  refresh_ub(t, false);
+  const unsigned sentinel = (unsigned)t->rows_ub;
+  int bits = 0;
+  while (bits < 32 && (1ull << bits) <= (unsigned long long)sentinel) ++bits;
+  const int passes = std::max(1, (bits + 7) / 8);
+
+  unsigned* ka = (unsigned*)t->b_ka.p;
+  unsigned* va = (unsigned*)t->b_va.p;
+  unsigned* kb = (unsigned*)t->b_kb.p;
+  unsigned* vb = (unsigned*)t->b_vb.p;
+  {
+    PhaseScope ph(t, PH_BWD_PROBE, s);
+    static int resident = 0;
+    if (!resident) resident = resident_blocks(bwd_probe_kernel, 256, 0, t->sm_count);
+    const long long warps = (n_bags + 31) / 32;
+    const long long grid = grid_for((warps + 7) / 8, resident);
+    bwd_probe_kernel<<<(unsigned)grid, 256, 0, s>>>(idmap(t), (const long long*)d_keys, n_keys,
+                                                    (const long long*)d_bag_offsets, n_bags, ka, va,
+                                                    sentinel, t->st);
+    DHS_TRY(last_launch());
+  }
+  {
+    PhaseScope ph(t, PH_BWD_SORT, s);
+    const long long ntiles = (n_keys + kRadixTile - 1) / kRadixTile;
+    for (int p = 0; p < passes; ++p) {
+      const int shift = 8 * p;
+      radix_hist_kernel<<<(unsigned)ntiles, kRadixThreads, 0, s>>>(ka, n_keys, shift,
+                                                                   (unsigned*)t->b_hist.p, ntiles);
+      radix_scan_kernel<<<kRadixBins, 256, 0, s>>>((unsigned*)t->b_hist.p, ntiles,
+                                                   (unsigned*)t->b_totals.p);
+      radix_scatter_kernel<<<(unsigned)ntiles, kRadixThreads, 0, s>>>(
+          ka, va, kb, vb, n_keys, shift, (const unsigned*)t->b_hist.p,
+          (const unsigned*)t->b_totals.p, ntiles);
+      DHS_TRY(last_launch());
+      std::swap(ka, kb);
+      std::swap(va, vb);
+    }
+  }
+  {
+    PhaseScope ph(t, PH_BWD_SEG, s);
+    OptArgs oa;
+    oa.opt = t->opt;
+    oa.lr = lr;
+    oa.eps = t->eps;
+    oa.b1 = t->b1;
+    oa.b2 = t->b2;
+    oa.c1 = (float)(1.0 - (double)t->b1);
+    oa.c2 = (float)(1.0 - (double)t->b2);
+    oa.bc1 = (float)(1.0 - std::pow((double)t->b1, (double)t->adam_t));
+    oa.bc2 = (float)(1.0 - std::pow((double)t->b2, (double)t->adam_t));
+    DHS_TRY(dispatch_seg(t, ka, va, n_keys, d_grad, n_bags, oa, s));
+    const int G = pick_group(t->dim), NV = pick_nv(t->dim, G);
+    const int pstride = NV * G * 4;
+    const long long nchunks = (n_keys + kSegChunk - 1) / kSegChunk;
+    const size_t smem = (size_t)std::max(256, t->dim) * sizeof(double);
+    const long long grid = std::min<long long>(nchunks, (long long)t->sm_count * 8);
+    bwd_combine_kernel<<<(unsigned)grid, 256, smem, s>>>(ka, n_keys, t->dim, rowspace(t), oa,
+                                                        (const double*)t->b_ph.p, (const double*)t->b_pt.p,
+                                                        (const unsigned char*)t->b_cflags.p, kSegChunk,
+                                                        pstride, t->st);
+    DHS_TRY(last_launch());
+  }
+  return DHS_OK;
+}
+
+dhs_status ht_get_rows(dhs_table* t, const int64_t* d_keys, int64_t n, float* d_rows_out,
+                       dhs_stream stream) {
+  DHS_TRY(check_table(t));
+  if (n < 0 || (n > 0 && (!d_keys || !d_rows_out))) return DHS_ERR_INVALID_ARG;
+  if (n == 0) return DHS_OK;
+  DeviceGuard g(t->device);
+  cudaStream_t s = (cudaStream_t)stream;
+  t->last_stream = s;
+  const long long grid = std::min<long long>((n + 7) / 8, (long long)t->sm_count * 16);
+  get_rows_kernel<<<(unsigned)grid, 256, 0, s>>>(idmap(t), rowspace(t), (const long long*)d_keys, n, d_rows_out);
+  return last_launch();
+}
+
+int64_t ht_row_stride(const dhs_table* t) { return t ? t->stride : -1; }
+
+dhs_status ht_sync(dhs_table* t) {
+  DHS_TRY(check_table(t));
+  DeviceGuard g(t->device);
+  DHS_CUDA(cudaStreamSynchronize(t->last_stream));
+  DHS_CUDA(cudaDeviceSynchronize());
+  unsigned err = 0;
+  DHS_CUDA(cudaMemcpy(&err, &t->st->err, sizeof(unsigned), cudaMemcpyDeviceToHost));
+  if (err) {
+    const unsigned zero = 0;
+    DHS_CUDA(cudaMemcpy(&t->st->err, &zero, sizeof(unsigned), cudaMemcpyHostToDevice));
+  }
+  return (dhs_status)err;
+}
+
+dhs_status ht_size(dhs_table* t, int64_t* n_rows) {
+  DHS_TRY(check_table(t));
+  if (!n_rows) return DHS_ERR_INVALID_ARG;
+  const dhs_status rc = ht_sync(t);
+  if (rc == DHS_ERR_CUDA) return rc;
+  DeviceGuard g(t->device);
+  unsigned long long r = 0;
+  DHS_CUDA(cudaMemcpy(&r, &t->st->row_count, sizeof(r), cudaMemcpyDeviceToHost));
+  *n_rows = (int64_t)r;
+  t->rows_ub = (long long)r;
+  return rc;
+}
+
+dhs_status ht_counters(dhs_table* t, int64_t out[8]) {
+  DHS_TRY(check_table(t));
+  if (!out) return DHS_ERR_INVALID_ARG;
+  DeviceGuard g(t->device);
+  DHS_CUDA(cudaStreamSynchronize(t->last_stream));
+  DHS_CUDA(cudaDeviceSynchronize());
+  DevState h;
+  DHS_CUDA(cudaMemcpy(&h, t->st, sizeof(h), cudaMemcpyDeviceToHost));
+  out[0] = (int64_t)h.row_count;
+  out[1] = (int64_t)h.sum_new;
+  out[2] = (int64_t)h.sum_unique;
+  out[3] = t->n_insert_calls;
+  out[4] = t->adam_t;
+  out[5] = (int64_t)t->nslots;
+  out[6] = (int64_t)t->blocks_h.size();
+  out[7] = t->n_rehash;
+  return DHS_OK;
+}
+
+dhs_status ht_export(dhs_table* t, int64_t* h_keys, float* h_rows) {
+  DHS_TRY(check_table(t));
+  int64_t rows = 0;
+  const dhs_status rc = ht_size(t, &rows);
+  if (rc == DHS_ERR_CUDA) return rc;
+  DeviceGuard g(t->device);
+  cudaStream_t s = t->last_stream;
+  if (h_keys && rows > 0) {
+    long long* kb = (long long*)dalloc(t, sizeof(long long) * rows, s);
+    if (!kb) return DHS_ERR_OOM;
+    const long long grid = std::min<long long>((long long)((t->nslots + 255) / 256), (long long)t->sm_count * 16);
+    keys_by_row_kernel<<<(unsigned)grid, 256, 0, s>>>(t->slots, t->nslots, kb, (unsigned long long)rows);
+    dhs_status lr = last_launch();
+    if (lr == DHS_OK && cudaMemcpyAsync(h_keys, kb, sizeof(long long) * rows, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+      lr = DHS_ERR_CUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess) lr = DHS_ERR_CUDA;
+    dfree(t, kb, sizeof(long long) * rows, s);
+    cudaStreamSynchronize(s);
+    DHS_TRY(lr);
+  }
+  if (h_rows) {
+    for (long long r0 = 0; r0 < rows; r0 += t->block_rows) {
+      const long long cnt = std::min<long long>(t->block_rows, rows - r0);
+      DHS_CUDA(cudaMemcpy(h_rows + r0 * t->stride, t->blocks_h[r0 >> t->log2_br],
+                          sizeof(float) * cnt * t->stride, cudaMemcpyDeviceToHost));
+    }
+  }
+  return rc;
+}
+
+dhs_status ht_set_phase_timing(dhs_table* t, int enable) {
+  DHS_TRY(check_table(t));
+  t->timing = enable != 0;
+  return DHS_OK;
+}
+
+dhs_status ht_phase_times(dhs_table* t, double* ms_out, int64_t* count_out, int n) {
+  DHS_TRY(check_table(t));
+  if (n < 0 || (n > 0 && (!ms_out || !count_out))) return DHS_ERR_INVALID_ARG;
+  DeviceGuard g(t->device);
+  for (int i = 0; i < n; ++i) {
+    ms_out[i] = 0.0;
+    count_out[i] = 0;
+  }
+  dhs_status rc = DHS_OK;
+  for (auto& r : t->recs) {
+    if (cudaEventSynchronize(r.b) != cudaSuccess) rc = DHS_ERR_CUDA;
+    float ms = 0.f;
+    if (cudaEventElapsedTime(&ms, r.a, r.b) != cudaSuccess) rc = DHS_ERR_CUDA;
+    if (r.phase < n) {
+      ms_out[r.phase] += ms;
+      count_out[r.phase] += 1;
+    }
+    t->ev_pool.push_back(r.a);
+    t->ev_pool.push_back(r.b);
+  }
+  t->recs.clear();
+  cudaGetLastError();
+  return rc;
+}
+
+}  // extern "C"

@@ -1,0 +1,443 @@
+// Forward kernels: lookup-or-insert, gather, in-order sum pooling, and the
+// deterministic offset assignment of new keys.
+//
+// Pooling semantics: nn.EmbeddingBag(mode="sum") (DLRM practice article,
+// section 2.1) over row lookups (RecIS background article, nn.Embedding
+// section): pooled[b] = sum of the bag's rows, added in bag order in fp32.
+//
+// New keys are numbered by their first position in the batch.  The probe
+// leaves PENDING | min position in the claimed slot; a bitmap over batch
+// positions then marks each new key's first position, a prefix count over
+// that bitmap gives its rank, and rank + row count is its row.  No kernel
+// waits on another thread, and the map from keys to rows depends only on the
+// key stream.
+#pragma once
+
+#include "dhs_device.cuh"
+
+namespace dhs {
+
+constexpr int kFwdThreads = 256;
+
+// Bag ends of one chunk of G bags, held one per lane of the group and made
+// safe to use: clamped into [start, n_keys] and non-decreasing.  Malformed
+// offsets latch kErrInvalid.
+template <int G>
+__device__ __forceinline__ long long load_bag_ends(const long long* __restrict__ bag_off,
+                                                   long long b0, int nb, long long n_keys,
+                                                   long long n_bags, long long& start,
+                                                   unsigned gmask, int gl, DevState* st) {
+  long long s = __ldg(bag_off + b0);
+  bool bad = false;
+  if (b0 == 0 && s != 0) bad = true;
+  if (s < 0 || s > n_keys) {
+    bad = true;
+    s = s < 0 ? 0 : n_keys;
+  }
+  long long e = (gl < nb) ? __ldg(bag_off + b0 + gl + 1) : n_keys;
+  if (gl < nb) {
+    if (e < s || e > n_keys) bad = true;
+    if (b0 + gl + 1 == n_bags && e != n_keys) bad = true;
+  }
+  e = e < s ? s : (e > n_keys ? n_keys : e);
+  // running max so that ends never decrease along the chunk
+#pragma unroll
+  for (int o = 1; o < G; o <<= 1) {
+    const long long x = __shfl_up_sync(gmask, e, o, G);
+    if (gl >= o && x > e) {
+      e = x;
+      bad = true;
+    }
+  }
+  if (gl >= nb) e = LLONG_MAX;
+  if (bad) latch(st, kErrInvalid);
+  start = s;
+  return e;
+}
+
+// Fused lookup-or-insert + gather + sum pooling.  A group of G lanes owns a
+// chunk of G consecutive bags; it probes the chunk's ids G at a time (one id
+// per lane), then walks those ids in order, each lane loading NV float4
+// columns of the row (16-byte vector loads), U rows in flight, and adds them
+// into the current bag's accumulator.  A new key's row is not read: its
+// initial value is computed from the key, exactly as the assignment kernel
+// will store it.
+template <int G, int NV>
+__global__ void __launch_bounds__(kFwdThreads)
+fwd_probe_pool_kernel(IdMap m, RowSpace rs, int dim, const long long* __restrict__ keys,
+                      long long n_keys, const long long* __restrict__ bag_off, long long n_bags,
+                      float* __restrict__ out, unsigned* __restrict__ nbm,
+                      unsigned* __restrict__ slotpos, DevState* st) {
+  constexpr int U = G < 8 ? G : 8;
+  const int lane = threadIdx.x & 31;
+  const int gl = lane & (G - 1);
+  const int gw = lane / G;
+  const unsigned gmask = (G == 32) ? 0xffffffffu : (((1u << G) - 1u) << (gw * G));
+  const long long gid = ((long long)blockIdx.x * kFwdThreads + threadIdx.x) / G;
+  const long long ngroups = ((long long)gridDim.x * kFwdThreads) / G;
+  const long long nchunks = (n_bags + G - 1) / G;
+  const int d4 = dim >> 2;
+
+  for (long long c = gid; c < nchunks; c += ngroups) {
+    const long long b0 = c * G;
+    const int nb = (int)min((long long)G, n_bags - b0);
+    long long s;
+    const long long e = load_bag_ends<G>(bag_off, b0, nb, n_keys, n_bags, s, gmask, gl, st);
+    const long long E = __shfl_sync(gmask, e, nb - 1, G);
+    int cur = 0;
+    long long cur_end = __shfl_sync(gmask, e, 0, G);
+    float4 acc[NV];
+#pragma unroll
+    for (int q = 0; q < NV; ++q) acc[q] = make_float4(0.f, 0.f, 0.f, 0.f);
+
+    for (long long ws = s; ws < E; ws += G) {
+      const int cnt = (int)min((long long)G, E - ws);
+      // ---- probe: one id per lane ----
+      int kind = kBad;
+      unsigned long long ref = 0, key = 0;
+      if (gl < cnt) {
+        const long long p = ws + gl;
+        const long long k = __ldg(keys + p);
+        key = (unsigned long long)k;
+        if (k < 0) {
+          latch(st, kErrInvalid);
+        } else {
+          kind = probe_claim(m, key, (unsigned)p, ref, st);
+          if (kind == kNew) slotpos[p] = (unsigned)ref;
+        }
+      }
+      // mark the positions that carry a key new in this call (<= 2 words per window)
+      {
+        const unsigned bal = __ballot_sync(gmask, kind == kNew);
+        const unsigned mine = (G == 32) ? bal : ((bal >> (gw * G)) & ((1u << G) - 1u));
+        if (gl == 0 && mine) {
+          const unsigned long long p0 = (unsigned long long)ws;
+          const unsigned sh = (unsigned)(p0 & 31);
+          atomicOr(&nbm[p0 >> 5], mine << sh);
+          if (sh && (sh + G > 32)) {
+            const unsigned hi = mine >> (32 - sh);
+            if (hi) atomicOr(&nbm[(p0 >> 5) + 1], hi);
+          }
+        }
+      }
+      // ---- gather + pool, in id order ----
+      for (int t0 = 0; t0 < cnt; t0 += U) {
+        float4 v[U][NV];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+          const int t = t0 + u;
+          const int src = t & (G - 1);
+          const int kt = __shfl_sync(gmask, kind, src, G);
+          const unsigned long long rt = __shfl_sync(gmask, ref, src, G);
+          const unsigned long long keyt = __shfl_sync(gmask, key, src, G);
+          const float* rowp = (t < cnt && kt == kHit) ? rs.row(rt) : nullptr;
+#pragma unroll
+          for (int q = 0; q < NV; ++q) {
+            const int c4 = gl + q * G;
+            float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (t < cnt && c4 < d4) {
+              if (kt == kHit)
+                x = __ldg(reinterpret_cast<const float4*>(rowp) + c4);
+              else if (kt == kNew)
+                x = init_weight4(keyt, c4 * 4);
+            }
+            v[u][q] = x;
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+          const int t = t0 + u;
+          if (t < cnt) {
+            const long long pos = ws + t;
+            while (pos >= cur_end) {
+              float4* o = reinterpret_cast<float4*>(out + (b0 + cur) * (long long)dim);
+#pragma unroll
+              for (int q = 0; q < NV; ++q) {
+                const int c4 = gl + q * G;
+                if (c4 < d4) o[c4] = acc[q];
+                acc[q] = make_float4(0.f, 0.f, 0.f, 0.f);
+              }
+              ++cur;
+              cur_end = __shfl_sync(gmask, e, cur & (G - 1), G);
+            }
+#pragma unroll
+            for (int q = 0; q < NV; ++q) acc[q] = f4add(acc[q], v[u][q]);
+          }
+        }
+      }
+    }
+    // the bag in progress and any empty bags after it
+    while (cur < nb) {
+      float4* o = reinterpret_cast<float4*>(out + (b0 + cur) * (long long)dim);
+#pragma unroll
+      for (int q = 0; q < NV; ++q) {
+        const int c4 = gl + q * G;
+        if (c4 < d4) o[c4] = acc[q];
+        acc[q] = make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+      ++cur;
+    }
+  }
+}
+
+#ifndef DHS_TEMPLATES_ONLY
+// Lookup-or-insert without pooling: thread per position.  offsets_out holds
+// the row offset of a hit, -(2 + slot) for a key new in this call (resolved by
+// fwd_fixup_kernel) and -1 for a negative key.
+__global__ void __launch_bounds__(kFwdThreads)
+fwd_probe_offsets_kernel(IdMap m, const long long* __restrict__ keys, long long n,
+                         long long* __restrict__ offsets_out, unsigned* __restrict__ nbm,
+                         unsigned* __restrict__ slotpos, DevState* st) {
+  const long long p = (long long)blockIdx.x * kFwdThreads + threadIdx.x;
+  bool is_new = false;
+  if (p < n) {
+    const long long k = __ldg(keys + p);
+    long long o = -1;
+    if (k < 0) {
+      latch(st, kErrInvalid);
+    } else {
+      unsigned long long ref;
+      const int kind = probe_claim(m, (unsigned long long)k, (unsigned)p, ref, st);
+      if (kind == kHit) {
+        o = (long long)ref;
+      } else if (kind == kNew) {
+        o = -2 - (long long)ref;
+        slotpos[p] = (unsigned)ref;
+        is_new = true;
+      }
+    }
+    offsets_out[p] = o;
+  }
+  // positions of a warp are one aligned 32-bit word of the bitmap
+  const unsigned bal = __ballot_sync(0xffffffffu, is_new);
+  if ((threadIdx.x & 31) == 0 && bal) nbm[p >> 5] = bal;
+}
+
+__global__ void fwd_fixup_kernel(const Slot* __restrict__ slots, long long* __restrict__ offsets,
+                                 long long n) {
+  for (long long p = (long long)blockIdx.x * blockDim.x + threadIdx.x; p < n;
+       p += (long long)gridDim.x * blockDim.x) {
+    const long long o = offsets[p];
+    if (o <= -2) offsets[p] = (long long)slots[-2 - o].val;
+  }
+}
+
+// First-occurrence marking.  Thread per bitmap word (32 positions), warp per
+// group of 1024 positions.  A new position is a first occurrence iff its
+// slot holds PENDING | that position.  Writes the first-occurrence word,
+// clears the new-position word for the next call, and writes the group's
+// count.  The last block to finish scans the group counts, reserves the new
+// rows (row_base = row_count, row_count += M) and resets the ticket.
+__global__ void __launch_bounds__(256)
+fwd_mark_kernel(const Slot* __restrict__ slots, unsigned* __restrict__ nbm,
+                unsigned* __restrict__ fbm, unsigned* __restrict__ gcnt,
+                unsigned* __restrict__ gpref, const unsigned* __restrict__ slotpos,
+                long long nwords, long long ngroups, DevState* st) {
+  const long long w = (long long)blockIdx.x * 256 + threadIdx.x;
+  unsigned word = 0;
+  if (w < nwords) {
+    word = nbm[w];
+    if (word) nbm[w] = 0u;
+  }
+  unsigned fw = 0;
+  while (word) {
+    const int b = __ffs(word) - 1;
+    word &= word - 1;
+    const unsigned long long p = (unsigned long long)(w * 32 + b);
+    const unsigned s = slotpos[p];
+    const unsigned long long v = __ldcg(&slots[s].val);
+    if ((v & ~kPending) == p) fw |= 1u << b;
+  }
+  if (w < nwords) fbm[w] = fw;
+  const unsigned c = warp_sum_u32(__popc(fw));
+  const long long g = w >> 5;
+  if ((threadIdx.x & 31) == 0 && g < ngroups) gcnt[g] = c;
+
+  __shared__ bool is_last;
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) is_last = (atomicAdd(&st->ticket, 1u) == gridDim.x - 1);
+  __syncthreads();
+  if (!is_last) return;
+  __threadfence();
+
+  // exclusive scan of gcnt[0, ngroups) by this block, 256 entries per pass
+  __shared__ unsigned wsum[8];
+  __shared__ unsigned long long carry_s;
+  if (threadIdx.x == 0) carry_s = 0;
+  __syncthreads();
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  for (long long base = 0; base < ngroups; base += 256) {
+    const long long i = base + threadIdx.x;
+    const unsigned x = (i < ngroups) ? __ldcg(gcnt + i) : 0u;
+    unsigned inc = x;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const unsigned y = __shfl_up_sync(0xffffffffu, inc, o);
+      if (lane >= o) inc += y;
+    }
+    if (lane == 31) wsum[wid] = inc;
+    __syncthreads();
+    unsigned wpre = 0, tot = 0;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      if (k < wid) wpre += wsum[k];
+      tot += wsum[k];
+    }
+    const unsigned long long carry = carry_s;
+    if (i < ngroups) gpref[i] = (unsigned)(carry + wpre + inc - x);
+    __syncthreads();
+    if (threadIdx.x == 0) carry_s = carry + tot;
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) {
+    const unsigned long long M = carry_s;
+    const unsigned long long base = st->row_count;
+    st->row_base = base;
+    st->row_count = base + M;
+    st->m_last = M;
+    st->sum_new += M;
+    st->ticket = 0u;
+    __threadfence();
+  }
+}
+
+// Offset assignment + row initialisation.  Warp per group of 1024 positions:
+// the group's new keys have consecutive ranks, so their rows are one
+// contiguous run (split only at a block edge).  Each new key's slot gets its
+// row offset; the run is then written with coalesced 16-byte stores (initial
+// weights from splitmix64(key), optimizer state zero).
+constexpr int kAssignWarps = 4;
+
+__global__ void __launch_bounds__(kAssignWarps * 32)
+fwd_assign_kernel(Slot* __restrict__ slots, RowSpace rs, int dim,
+                  const unsigned* __restrict__ fbm, const unsigned* __restrict__ gpref,
+                  const unsigned* __restrict__ slotpos, long long nwords, long long ngroups,
+                  DevState* st) {
+  __shared__ unsigned long long skey[kAssignWarps][1024];
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  const long long g = (long long)blockIdx.x * kAssignWarps + wid;
+  if (g >= ngroups) return;
+  const long long w = g * 32 + lane;
+  unsigned fw = (w < nwords) ? fbm[w] : 0u;
+  const unsigned c = __popc(fw);
+  unsigned inc = c;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const unsigned y = __shfl_up_sync(0xffffffffu, inc, o);
+    if (lane >= o) inc += y;
+  }
+  const unsigned total = __shfl_sync(0xffffffffu, inc, 31);
+  if (total == 0) return;
+  const unsigned long long row0 = st->row_base + gpref[g];
+  const unsigned long long limit = st->n_blocks << rs.log2_br;
+  unsigned j = inc - c;
+  while (fw) {
+    const int b = __ffs(fw) - 1;
+    fw &= fw - 1;
+    const unsigned long long p = (unsigned long long)(w * 32 + b);
+    const unsigned s = slotpos[p];
+    const unsigned long long row = row0 + j;
+    skey[wid][j] = slots[s].key;
+    if (row < limit) {
+      slots[s].val = row;
+    } else {
+      latch(st, kErrFull);
+      slots[s].val = kPending;  // unusable; the table is reported full
+    }
+    ++j;
+  }
+  __syncwarp();
+  const int s4 = rs.stride >> 2, d4 = dim >> 2;
+  const long long work = (long long)total * s4;
+  for (long long idx = lane; idx < work; idx += 32) {
+    const unsigned r = (unsigned)(idx / s4);
+    const int c4 = (int)(idx - (long long)r * s4);
+    const unsigned long long row = row0 + r;
+    if (row >= limit) continue;
+    const float4 x = (c4 < d4) ? init_weight4(skey[wid][r], c4 * 4) : make_float4(0.f, 0.f, 0.f, 0.f);
+    reinterpret_cast<float4*>(rs.row(row))[c4] = x;
+  }
+}
+
+// ---- IDMap maintenance and read-only access ----
+
+__global__ void fill_empty_kernel(Slot* __restrict__ slots, unsigned long long n) {
+  for (unsigned long long i = (unsigned long long)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+       i += (unsigned long long)gridDim.x * blockDim.x)
+    reinterpret_cast<ulonglong2*>(slots)[i] = make_ulonglong2(kEmptyKey, kEmptyKey);
+}
+
+// Re-insert every key of `from` into the empty map `to` (keys are distinct,
+// offsets keep their values: rows never move).
+__global__ void rehash_kernel(const Slot* __restrict__ from, unsigned long long n_from, IdMap to,
+                              DevState* st) {
+  for (unsigned long long i = (unsigned long long)blockIdx.x * blockDim.x + threadIdx.x;
+       i < n_from; i += (unsigned long long)gridDim.x * blockDim.x) {
+    const ulonglong2 sv = reinterpret_cast<const ulonglong2*>(from)[i];
+    if (sv.x == kEmptyKey) continue;
+    unsigned long long w = hash_key(sv.x) & to.win_mask;
+    bool done = false;
+    for (unsigned long long step = 0; step <= to.win_mask && !done; ++step) {
+      Slot* ws = to.slots + 2 * w;
+      for (int j = 0; j < 2 && !done; ++j) {
+        if (atomicCAS(&ws[j].key, kEmptyKey, sv.x) == kEmptyKey) {
+          ws[j].val = sv.y;
+          done = true;
+        }
+      }
+      w = (w + 1) & to.win_mask;
+    }
+    if (!done) latch(st, kErrFull);
+  }
+}
+
+__global__ void lookup_kernel(IdMap m, const long long* __restrict__ keys, long long n,
+                              long long* __restrict__ out) {
+  for (long long p = (long long)blockIdx.x * blockDim.x + threadIdx.x; p < n;
+       p += (long long)gridDim.x * blockDim.x) {
+    const long long k = __ldg(keys + p);
+    out[p] = k < 0 ? -1 : probe_find(m, (unsigned long long)k);
+  }
+}
+
+// Full rows of the given keys; warp per key, NaN for an absent key.
+__global__ void get_rows_kernel(IdMap m, RowSpace rs, const long long* __restrict__ keys,
+                                long long n, float* __restrict__ out) {
+  const int lane = threadIdx.x & 31;
+  const long long nw = ((long long)gridDim.x * blockDim.x) >> 5;
+  for (long long i = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5; i < n; i += nw) {
+    const long long k = __ldg(keys + i);
+    const long long off = k < 0 ? -1 : probe_find(m, (unsigned long long)k);
+    const int s4 = rs.stride >> 2;
+    float4* o = reinterpret_cast<float4*>(out + i * (long long)rs.stride);
+    const float nan = __int_as_float(0x7fc00000);
+    for (int c4 = lane; c4 < s4; c4 += 32)
+      o[c4] = off < 0 ? make_float4(nan, nan, nan, nan)
+                      : reinterpret_cast<const float4*>(rs.row((unsigned long long)off))[c4];
+  }
+}
+
+// keys_by_row[val] = key for every occupied slot (export in row order).
+__global__ void keys_by_row_kernel(const Slot* __restrict__ slots, unsigned long long n,
+                                   long long* __restrict__ keys_by_row, unsigned long long rows) {
+  for (unsigned long long i = (unsigned long long)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+       i += (unsigned long long)gridDim.x * blockDim.x) {
+    const ulonglong2 sv = reinterpret_cast<const ulonglong2*>(slots)[i];
+    if (sv.x != kEmptyKey && sv.y < rows) keys_by_row[sv.y] = (long long)sv.x;
+  }
+}
+
+__global__ void pack_keys_kernel(const int* __restrict__ tids, const long long* __restrict__ ids,
+                                 long long n, long long* __restrict__ keys) {
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+       i += (long long)gridDim.x * blockDim.x) {
+    const long long t = tids[i], id = ids[i];
+    const bool ok = t >= 0 && t < (1 << 15) && id >= 0 && id < (1ll << 48);
+    keys[i] = ok ? ((t << 48) | id) : -1;
+  }
+}
+
+#endif  // DHS_TEMPLATES_ONLY
+
+}  // namespace dhs

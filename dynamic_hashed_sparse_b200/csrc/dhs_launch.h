@@ -1,0 +1,25 @@
+// Host-side launchers of the width-templated kernels (one translation unit
+// each, so that they compile in parallel).
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include "dhs_device.cuh"
+
+namespace dhs {
+
+struct OptArgs;
+
+// fwd_probe_pool_kernel<G, NV>; returns a cudaError_t of the launch.
+cudaError_t launch_probe_pool(int G, int NV, int sm_count, IdMap m, RowSpace rs, int dim,
+                              const long long* keys, long long n_keys, const long long* bag_off,
+                              long long n_bags, float* out, unsigned* nbm, unsigned* slotpos,
+                              DevState* st, cudaStream_t s);
+
+// bwd_seg_kernel<G, NV>
+cudaError_t launch_seg(int G, int NV, int sm_count, const unsigned* skey, const unsigned* sval,
+                       long long n, const float* grad, long long n_bags, int dim, RowSpace rs,
+                       const OptArgs& oa, double* part_head, double* part_tail,
+                       unsigned char* cflags, int chunk, DevState* st, cudaStream_t s);
+
+}  // namespace dhs

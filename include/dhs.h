@@ -1,0 +1,207 @@
+/*
+ * dhs.h - C ABI of the B200 dynamic hashed embedding engine (libdhs.so).
+ *
+ * One hot path, on one GPU: a two-level dynamic hash table (an IDMap from a
+ * feature id to a row offset, plus chunked EmbeddingBlocks that hold each
+ * row's parameters and optimizer state and grow by appending blocks), with a
+ * lookup-or-insert + sum-pooling forward and a coalesced sparse-gradient +
+ * fused row-optimizer backward.
+ *
+ * Sources of the operations (page title, then section):
+ *   [RecIS]  "RecIS: Alibaba's open-source unified training framework for
+ *            recommender systems" (pomoai.com hub page), section on the
+ *            Embedding Engine: IDMap (id -> offset) as the first level,
+ *            EmbeddingBlocks (parameters and optimizer state, contiguous,
+ *            sharded, growing without reallocation) as the second; merging
+ *            tables with the same attributes; and the code-layout section:
+ *            fused sparse-gradient update kernel with fewer atomics,
+ *            vectorised embedding lookup.
+ *   [BG]     "Alibaba RecIS: background and difficulties of search/ads/
+ *            recommendation training" (muyuuuu.github.io), nn.Embedding
+ *            section: a lookup reads one row, the backward updates only that
+ *            row; worked SGD example with a 10 x 4 table.
+ *   [DLRM-P] "DLRM model: core value and industrial deployment" (mokono.cn),
+ *            section 2.1: nn.EmbeddingBag(mode="sum") for variable-length
+ *            inputs with sparse gradients.
+ *   [DLRM-E] "DLRM: Meta splits industrial recommendation into 4 standard
+ *            blocks" (estelledc.github.io), module 2 (one table per
+ *            categorical field) and pitfall 4 (sparse optimizer: only the
+ *            touched rows are updated).
+ *
+ * Conventions for every call:
+ *   - Pointers named d_* are DEVICE pointers on the table's device; pointers
+ *     named h_* are HOST pointers.  The caller owns every buffer it passes;
+ *     the library owns the table (IDMap, blocks, workspace).
+ *   - Calls taking a stream are asynchronous and ordered on that stream
+ *     (NULL = the legacy default stream).  A table is used by one host thread
+ *     at a time, and its calls must be ordered (one stream, or the caller's
+ *     own events).
+ *   - Keys are int64 >= 0; with merged tables key = table_id << 48 | id
+ *     (dhs_pack_keys).  -1 is reserved.
+ *   - Argument errors are returned at once and nothing is launched.  Errors
+ *     found by a kernel (a negative key, a key missing in the backward, a
+ *     full table) are latched in a device word; the call's own work goes on
+ *     for the valid inputs, and the first latched error is returned by the
+ *     next ht_sync / ht_size / ht_export.
+ *   - Floating point: fp32 storage; forward sums in fp32 in bag order;
+ *     backward gradient sums in fp64, rounded once to fp32; optimizer
+ *     arithmetic in fp32, each operation rounded (no contraction).
+ */
+#ifndef DHS_H_
+#define DHS_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t / CUstream. */
+typedef struct CUstream_st* dhs_stream;
+
+typedef struct dhs_table dhs_table; /* opaque, library-owned */
+
+typedef enum {
+  DHS_OK = 0,
+  DHS_ERR_INVALID_ARG = 1, /* bad argument, negative key, malformed bag offsets */
+  DHS_ERR_OOM = 2,         /* device allocation failed */
+  DHS_ERR_CUDA = 3,        /* a CUDA runtime call failed */
+  DHS_ERR_TABLE_FULL = 4,  /* row limit (max_rows) or IDMap probe bound reached */
+  DHS_ERR_NOT_FOUND = 5,   /* backward saw a key that is not in the table */
+  DHS_ERR_UNSUPPORTED = 6  /* configuration this build does not handle */
+} dhs_status;
+
+typedef enum {
+  DHS_SGD = 0,             /* w -= lr*g                                         */
+  DHS_ADAGRAD = 1,         /* per-element G += g*g; w -= lr*g/(sqrt(G)+eps)     */
+  DHS_ADAM = 2,            /* lazy Adam: m, v per element beside the row        */
+  DHS_ADAGRAD_ROWWISE = 3  /* one accumulator per row: G += mean(g^2)           */
+} dhs_optimizer;
+
+typedef struct {
+  float eps;   /* default 1e-8 */
+  float beta1; /* Adam, default 0.9 */
+  float beta2; /* Adam, default 0.999 */
+} dhs_opt_params;
+
+/* Optional device allocator (e.g. a framework's caching allocator).  alloc
+ * returns device memory usable on `stream` or NULL; free releases a block
+ * returned by alloc once the work on `stream` that uses it is done.  With
+ * NULL the library uses cudaMallocAsync / cudaFreeAsync on the call's stream. */
+typedef struct {
+  void* (*alloc)(size_t bytes, dhs_stream stream, void* ctx);
+  void (*free)(void* ptr, size_t bytes, dhs_stream stream, void* ctx);
+  void* ctx;
+} dhs_allocator;
+
+/* Human-readable name of a status code (static string). */
+const char* dhs_status_str(dhs_status s);
+
+/* key[i] = table_ids[i] << 48 | ids[i]  ([RecIS] Embedding Engine: tables with
+ * the same attributes merged into one map).  An entry with table_id outside
+ * [0, 2^15) or id outside [0, 2^48) gives key -1, which a table call then
+ * reports as DHS_ERR_INVALID_ARG.  d_table_ids int32[n], d_ids int64[n],
+ * d_keys_out int64[n]; n = 0 is a no-op. */
+dhs_status dhs_pack_keys(const int32_t* d_table_ids, const int64_t* d_ids, int64_t n,
+                         int64_t* d_keys_out, dhs_stream stream);
+
+/* Create an empty table on the current CUDA device ([RecIS] Embedding
+ * Engine).  dim: embedding width, a multiple of 4 in [4, 512].  opt: the
+ * optimizer whose state lives beside each row.  block_rows: rows per
+ * EmbeddingBlock, a power of two (0 = 2^20).  max_rows: row limit (0 = 2^31;
+ * at most 2^32 - 2).  params / alloc may be NULL (defaults).  The row stride
+ * is dim * (1 + s) floats, s = 0 (SGD), 1 (Adagrad), 2 (Adam), or dim + 1
+ * for row-wise Adagrad.  On success *out is a new handle. */
+dhs_status ht_create(int32_t dim, dhs_optimizer opt, int64_t block_rows, int64_t max_rows,
+                     const dhs_opt_params* params, const dhs_allocator* alloc,
+                     dhs_table** out);
+
+/* Wait for the table's work and release everything it owns.  NULL is a no-op. */
+dhs_status ht_destroy(dhs_table* t);
+
+/* Grow the IDMap now so that it holds n_keys keys without rehashing (e.g.
+ * before a large pre-population).  Rows are untouched. */
+dhs_status ht_reserve(dhs_table* t, int64_t n_keys, dhs_stream stream);
+
+/* Lookup-or-insert ([RecIS] IDMap: id -> offset; [BG] row lookup).
+ * d_offsets_out[i] = row offset of d_keys[i].  A key seen for the first time
+ * gets the next free row; new keys of one call are numbered in the order of
+ * their first position in d_keys, starting at the row count before the call,
+ * and their rows are initialised from splitmix64(key) (values in
+ * [-0.05, 0.05), optimizer state 0).  Rows never move.  A negative key gives
+ * offset -1 and latches DHS_ERR_INVALID_ARG. */
+dhs_status ht_lookup_or_insert(dhs_table* t, const int64_t* d_keys, int64_t n,
+                               int64_t* d_offsets_out, dhs_stream stream);
+
+/* Read-only lookup (no insert): offset, or -1 for an absent or negative key. */
+dhs_status ht_lookup(dhs_table* t, const int64_t* d_keys, int64_t n, int64_t* d_offsets_out,
+                     dhs_stream stream);
+
+/* Forward ([DLRM-P] 2.1 EmbeddingBag sum; [BG] row lookup; [RecIS] vectorised
+ * lookup): lookup-or-insert of every key, then
+ *   d_pooled_out[b, :] = sum of rows of d_keys[d_bag_offsets[b] ..
+ *                        d_bag_offsets[b+1]) in that order, fp32.
+ * d_keys int64[n_keys]; d_bag_offsets int64[n_bags + 1], non-decreasing,
+ * [0] = 0, [n_bags] = n_keys (checked on the device); d_pooled_out
+ * float[n_bags, dim] row-major.  An empty bag gives a zero row.  New keys get
+ * rows exactly as in ht_lookup_or_insert. */
+dhs_status embbag_forward(dhs_table* t, const int64_t* d_keys, int64_t n_keys,
+                          const int64_t* d_bag_offsets, int64_t n_bags, float* d_pooled_out,
+                          dhs_stream stream);
+
+/* Backward + update ([RecIS] fused sparse-gradient update with fewer
+ * atomics; [DLRM-E] pitfall 4 sparse optimizer; [BG] only touched rows change).
+ * For each distinct key k of d_keys:
+ *   g_k = sum over the positions i holding k of d_grad[bag(i), :]
+ * (fp64 sum, rounded once), then one step of the table's optimizer on row k
+ * with learning rate lr.  Rows not in d_keys are not read or written.  The
+ * Adam step count advances by one per call.  Keys must be in the table
+ * (missing ones are skipped and latch DHS_ERR_NOT_FOUND).
+ * d_grad float[n_bags, dim] row-major; the other arguments as in
+ * embbag_forward. */
+dhs_status embbag_backward_update(dhs_table* t, const int64_t* d_keys, int64_t n_keys,
+                                  const int64_t* d_bag_offsets, int64_t n_bags,
+                                  const float* d_grad, float lr, dhs_stream stream);
+
+/* Copy the full rows (dim weights, then the state) of the given keys into
+ * d_rows_out float[n, ht_row_stride(t)]; an absent key gives a NaN row. */
+dhs_status ht_get_rows(dhs_table* t, const int64_t* d_keys, int64_t n, float* d_rows_out,
+                       dhs_stream stream);
+
+/* Floats per row (weights + optimizer state), or -1 for a NULL handle. */
+int64_t ht_row_stride(const dhs_table* t);
+
+/* Wait for all the table's work; return the first latched device error (and
+ * clear it), else DHS_OK. */
+dhs_status ht_sync(dhs_table* t);
+
+/* *n_rows = number of keys (= rows) in the table.  Synchronises like ht_sync
+ * and returns its status. */
+dhs_status ht_size(dhs_table* t, int64_t* n_rows);
+
+/* Synchronous export in row order: h_keys[r] = the key whose offset is r,
+ * h_rows[r * stride ..] = its row (weights then state).  Buffers hold at
+ * least ht_size rows; either pointer may be NULL. */
+dhs_status ht_export(dhs_table* t, int64_t* h_keys, float* h_rows);
+
+/* Counters since creation (synchronises): out[0] rows, out[1] keys inserted
+ * by forward / lookup-or-insert calls, out[2] sum over backward calls of the
+ * distinct keys updated, out[3] forward-type calls, out[4] backward calls,
+ * out[5] IDMap slots, out[6] blocks allocated, out[7] IDMap rehashes. */
+dhs_status ht_counters(dhs_table* t, int64_t out[8]);
+
+/* Per-phase device time, measured with CUDA events recorded on the call's
+ * stream around each phase while enabled.  Phases: 0 forward probe + pool,
+ * 1 forward offset assignment + row init, 2 backward probe, 3 backward sort,
+ * 4 backward segment reduce + update, 5 lookup-or-insert, 6 IDMap growth.
+ * ht_phase_times synchronises, writes ms_out[p] = total ms and
+ * count_out[p] = number of timed launches of phase p (p < n), then clears. */
+dhs_status ht_set_phase_timing(dhs_table* t, int enable);
+dhs_status ht_phase_times(dhs_table* t, double* ms_out, int64_t* count_out, int n);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DHS_H_ */
