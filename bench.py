@@ -1,0 +1,481 @@
+"""Benchmark of the hashed embedding training step (lookup-or-insert + sum-pool
+forward, coalesced sparse-gradient + fused optimizer backward) on B200.
+
+One step = key packing, embbag_forward and embbag_backward_update over one
+batch of the 26-table DLRM-style merged workload (65,536 samples x 26 ids,
+pooling 1, dim 128 fp32, Adagrad, Zipf 1.05 ids; synthetic, seeded).  The
+table starts empty: warm-up steps are the stream's first steps, timed steps
+the ones after.  Prints one JSON line.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl dhs|reference]
+
+--impl reference times the CPU oracle (single core) on a bounded sample of
+the same workload.  Under torchrun each rank runs an independent replica
+(its own table and seed): the path does not shard, so there is no data-path
+collective; value is the ids of all ranks over the slowest rank's time.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from workloads import gen  # noqa: E402
+
+METRIC = "IDs/sec & HBM GB/s (% of peak): hashed lookup+bag-sum fwd, sparse update bwd"
+UNIT = "IDs/s"
+WORKLOAD = "dlrm_merged_26"
+
+
+# ---------------------------------------------------------------------------
+# algorithmic bytes (compulsory traffic: each datum once)
+# ---------------------------------------------------------------------------
+def stride_floats(dim: int, opt: str) -> int:
+    return dim + {"sgd": 0, "adagrad": dim, "adam": 2 * dim, "adagrad_rowwise": 4}[opt]
+
+
+def alg_bytes(n: int, b: int, u: int, m: int, dim: int, opt: str) -> dict:
+    """Per step.  n ids, b bags, u distinct keys, m of them new."""
+    R = 4 * dim
+    S = 4 * stride_floats(dim, opt)
+    pack = 4 * n + 8 * n + 8 * n
+    fwd_pool = 8 * n + 8 * (b + 1) + 16 * u + 16 * m + R * (u - m) + 4 * dim * b
+    fwd_assign = S * m + 16 * m
+    bwd = 8 * n + 8 * (b + 1) + 16 * u + 4 * dim * b + 2 * S * u
+    return dict(pack=pack, fwd_pool=fwd_pool, fwd_assign=fwd_assign,
+                fwd=pack + fwd_pool + fwd_assign, bwd=bwd,
+                bwd_seg=4 * dim * b + 2 * S * u + 8 * n)
+
+
+def load_peaks() -> dict:
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return dict(hbm_gbs=float(d["hbm_gbs"]), source="measured")
+    return dict(hbm_gbs=6650.0, source="fallback")
+
+
+def load_traffic(kernel: str):
+    """DRAM bytes per launch of `kernel` from the committed ncu summary, if it
+    was taken on the current kernel sources (else None)."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    ent = d.get(kernel)
+    if not ent:
+        return None
+    from dynamic_hashed_sparse_b200 import build as B
+    if ent.get("source_digest") != B._digest():
+        return None
+    return ent
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            time.sleep(0.2)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self) -> dict:
+        rows = []
+        try:
+            with open(self.path) as f:
+                for line in f:
+                    parts = [x.strip() for x in line.split(",")]
+                    if len(parts) >= 9:
+                        rows.append(parts)
+        except OSError:
+            pass
+        finally:
+            if self.path and os.path.exists(self.path):
+                os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ---------------------------------------------------------------------------
+# distributed plumbing (independent replicas; max over ranks)
+# ---------------------------------------------------------------------------
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def init_dist(world: int, backend: str):
+    if world <= 1:
+        return None
+    import datetime
+
+    import torch.distributed as dist
+    dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+    return dist
+
+
+def max_over_ranks(x: float, dist, device=None) -> float:
+    if dist is None:
+        return x
+    import torch
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(x: float, dist, device=None) -> float:
+    if dist is None:
+        return x
+    import torch
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+def barrier(dist, device=None):
+    if dist is not None:
+        import torch
+        t = torch.zeros(1, device=device)
+        dist.all_reduce(t)
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle timing (reference arm and cpu_baseline)
+# ---------------------------------------------------------------------------
+def time_oracle(w, steps, frac: float, timed_from: int = 0):
+    """Run the oracle on the first `steps` steps of the workload, each batch cut
+    to its first `frac` of bags, timing the steps from `timed_from` on;
+    returns (timed ids, seconds)."""
+    from oracle import Oracle, pack_keys
+    o = Oracle(w.dim, w.optimizer, eps=w.eps, beta1=w.beta1, beta2=w.beta2)
+    ids = 0
+    secs = 0.0
+    try:
+        for s in range(steps):
+            b = w.batch(s)
+            nb = max(1, int(b.n_bags * frac))
+            offs = b.bag_offsets[: nb + 1]
+            n = int(offs[-1])
+            grad = w.grads(s, nb)  # the first nb rows of the step's gradients
+            t0 = time.perf_counter()
+            keys, _ = pack_keys(b.table_ids[:n], b.ids[:n])
+            o.forward(keys, offs)
+            o.backward_update(keys, offs, grad, w.lr)
+            if s >= timed_from:
+                secs += time.perf_counter() - t0
+                ids += n
+    finally:
+        o.close()
+    return ids, secs
+
+
+def cpu_cores_used() -> int:
+    return 1
+
+
+def run_reference(args):
+    world, rank, _ = dist_env()
+    if rank != 0:
+        return 0
+    w = gen.full(args.workload)
+    frac = args.ref_frac
+    ids, secs = time_oracle(w, args.warmup + args.steps, frac, timed_from=args.warmup)
+    value = ids / secs if secs > 0 else 0.0
+    sample = (f"steps {args.warmup}..{args.warmup + args.steps - 1} of {w.name} timed after "
+              f"{args.warmup} untimed, first {frac:.4f} of each batch's bags ({ids} timed ids), "
+              f"oracle single-threaded")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * secs / max(1, args.steps),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f32", "data": "synthetic",
+        "config": workload_config(w),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cpu_cores_used(), "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def workload_config(w) -> dict:
+    p = w.params
+    return {"workload": f"{w.name}: {p.get('tables', 1)} tables merged in one IDMap, batch {p.get('batch')} "
+                        f"samples x {p.get('tables')} ids (pooling 1), dim {w.dim} fp32, {w.optimizer} "
+                        f"lr {w.lr} eps {w.eps}, Zipf alpha {p.get('alpha')} per table, cardinalities "
+                        f"log-uniform in [1e3, 1e7]",
+            "ids_per_step": int(p.get("batch", 0)) * int(p.get("tables", 1)),
+            "batch": int(p.get("batch", 0)),
+            "bags_per_step": int(p.get("batch", 0)) * int(p.get("tables", 1)),
+            "dim": w.dim, "optimizer": w.optimizer,
+            "l2": "inputs larger than L2 (per-step gradients 872 MB, keys 13.6 MB; 126 MB L2)",
+            "table": "starts empty; warm-up = the stream's first steps"}
+
+
+# ---------------------------------------------------------------------------
+# the device run
+# ---------------------------------------------------------------------------
+def run_dhs(args):
+    import torch
+    world, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    dist = init_dist(world, "nccl")
+    import dynamic_hashed_sparse_b200 as dhs
+
+    if args.workload == WORKLOAD:
+        w = gen.DlrmMerged(seed=1002 + 7919 * rank, batch=args.batch or 65536)
+    else:
+        w = gen.full(args.workload)
+    total = args.warmup + args.steps
+    # inputs for every step, resident in HBM before the timed region
+    batches = []
+    for s in range(total):
+        b = w.batch(s)
+        batches.append((torch.from_numpy(b.table_ids).to(device), torch.from_numpy(b.ids).to(device),
+                        torch.from_numpy(b.bag_offsets).to(device), b.n, b.n_bags))
+    n_grad = min(total, args.grad_buffers)
+    grads = [w.torch_grads(s, batches[s][4], device) for s in range(n_grad)]
+    pooled = torch.empty((batches[0][4], w.dim), dtype=torch.float32, device=device)
+    keys = torch.empty(batches[0][3], dtype=torch.int64, device=device)
+
+    t = dhs.ht_create(w.dim, w.optimizer, block_rows=w.block_rows, eps=w.eps, beta1=w.beta1, beta2=w.beta2)
+    stream = torch.cuda.current_stream()
+
+    def step(s):
+        tids, ids, offs, n, nb = batches[s]
+        k = keys[:n]
+        dhs.dhs_pack_keys(tids, ids, out=k)
+        dhs.embbag_forward(t, k, offs, out=pooled[:nb])
+        dhs.embbag_backward_update(t, k, offs, grads[s % n_grad], w.lr)
+
+    for s in range(args.warmup):
+        step(s)
+    torch.cuda.synchronize()
+    c0 = dhs.ht_counters(t)
+    dhs.ht_phase_times(t)  # clear
+    dhs.ht_set_phase_timing(t, True)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(dist, device)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        e0.record(stream)
+        for s in range(args.warmup, total):
+            step(s)
+        e1.record(stream)
+        torch.cuda.synchronize()
+    barrier(dist, device)
+    dhs.ht_set_phase_timing(t, False)
+    ms_local = e0.elapsed_time(e1)
+    phases = dhs.ht_phase_times(t)
+    c1 = dhs.ht_counters(t)
+    status = dhs.ht_sync(t)
+    if status != 0:
+        raise RuntimeError(f"device status {status} ({dhs.dhs_status_str(status)}) after the timed steps")
+
+    K = args.steps
+    n_ids = sum(batches[s][3] for s in range(args.warmup, total))
+    n_bags = sum(batches[s][4] for s in range(args.warmup, total))
+    U = c1["unique_updated"] - c0["unique_updated"]
+    M = c1["inserted"] - c0["inserted"]
+    launches = c1["launches"] - c0["launches"] + K  # + one key-packing kernel per step
+    ms = max_over_ranks(ms_local, dist, device)
+    ids_all = sum_over_ranks(float(n_ids), dist, device)
+    value = ids_all / (ms / 1e3)
+
+    ab = alg_bytes(n_ids, n_bags, U, M, w.dim, w.optimizer)
+    peaks = load_peaks()
+    ph_ms = {k: v[0] for k, v in phases.items()}
+    ph_cnt = {k: v[1] for k, v in phases.items()}
+    fwd_ms = ph_ms["fwd_probe_pool"] + ph_ms["fwd_assign"]
+    bwd_ms = ph_ms["bwd_probe"] + ph_ms["bwd_sort"] + ph_ms["bwd_seg_update"]
+    dom = max(("fwd_probe_pool", "bwd_seg_update"), key=lambda k: ph_ms[k])
+    dom_kernel = {"fwd_probe_pool": "fwd_probe_pool_kernel", "bwd_seg_update": "bwd_seg_kernel"}[dom]
+    dom_bytes = ab["fwd_pool"] if dom == "fwd_probe_pool" else ab["bwd_seg"]
+    dom_launch_ms = ph_ms[dom] / max(1, ph_cnt[dom])
+    dom_bytes_per_launch = dom_bytes / max(1, ph_cnt[dom])
+    achieved = dom_bytes_per_launch / (dom_launch_ms / 1e3) / 1e9
+    traffic = load_traffic(dom_kernel)
+    roofline = {
+        "bound": "hbm", "kernel": dom_kernel, "achieved": achieved, "peak": peaks["hbm_gbs"],
+        "peak_source": peaks["source"], "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
+        "traffic": (traffic["dram_bytes_per_launch"] * dom_bytes_per_launch / traffic["alg_bytes_per_launch"]
+                    if traffic and traffic.get("alg_bytes_per_launch") else None),
+        "alg_bytes_per_launch": dom_bytes_per_launch, "launch_ms": dom_launch_ms,
+    }
+
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
+        "ms_per_step": ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "timing_valid": args.warmup >= 3,
+        "dtype": "f32", "data": "synthetic", "config": workload_config(w),
+        "fwd": {"ids_per_s": n_ids / (fwd_ms / 1e3) if fwd_ms else None, "ms_per_step": fwd_ms / K,
+                "gbs": ab["fwd"] / (fwd_ms / 1e3) / 1e9 if fwd_ms else None,
+                "frac_of_peak": ab["fwd"] / (fwd_ms / 1e3) / 1e9 / peaks["hbm_gbs"] if fwd_ms else None},
+        "bwd": {"ids_per_s": n_ids / (bwd_ms / 1e3) if bwd_ms else None, "ms_per_step": bwd_ms / K,
+                "gbs": ab["bwd"] / (bwd_ms / 1e3) / 1e9 if bwd_ms else None,
+                "frac_of_peak": ab["bwd"] / (bwd_ms / 1e3) / 1e9 / peaks["hbm_gbs"] if bwd_ms else None},
+        "step_gbs": (ab["fwd"] + ab["bwd"]) / (ms_local / 1e3) / 1e9,
+        "phases_ms_per_step": {k: v / K for k, v in ph_ms.items() if ph_cnt[k]},
+        "per_step": {"ids": n_ids / K, "bags": n_bags / K, "unique": U / K, "new": M / K},
+        "roofline": roofline,
+        "gpu_launches": launches,
+        "table": {"rows": c1["rows"], "slots": c1["slots"], "blocks": c1["blocks"], "rehashes": c1["rehashes"]},
+    }
+    line["clocks"] = clk.summary()
+    t.close()
+    del grads, batches
+    torch.cuda.empty_cache()
+
+    if not args.no_e2e:
+        line["e2e"] = run_e2e(args, w, device, dist)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        ids, secs = time_oracle(gen.full(args.workload), args.cpu_steps, 1.0)
+        line["cpu_baseline"] = {"value": ids / secs, "unit": UNIT, "cores": cpu_cores_used(), "kind": "oracle",
+                                "sample": f"steps 0..{args.cpu_steps - 1} of {w.name}, full batches "
+                                          f"({ids} ids, {secs:.1f} s), oracle single-threaded"}
+    if dist is not None:
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_e2e(args, w, device, dist):
+    """The same step through the public API with host inputs: per step, copy
+    the ids, table ids, bag offsets and gradients from pinned host memory,
+    run the step, and copy the pooled output back; all inside the timed
+    region."""
+    import torch
+
+    import dynamic_hashed_sparse_b200 as dhs
+    total = args.warmup + args.steps
+    hb = []
+    for s in range(total):
+        b = w.batch(s)
+        hb.append((torch.from_numpy(b.table_ids).pin_memory(), torch.from_numpy(b.ids).pin_memory(),
+                   torch.from_numpy(b.bag_offsets).pin_memory(), b.n, b.n_bags))
+    nb0 = hb[0][4]
+    n_grad = 2
+    hgrads = [w.torch_grads(s, nb0, device).cpu().pin_memory() for s in range(n_grad)]
+    hpooled = torch.empty((nb0, w.dim), dtype=torch.float32).pin_memory()
+    n0 = hb[0][3]
+    d_tids = torch.empty(n0, dtype=torch.int32, device=device)
+    d_ids = torch.empty(n0, dtype=torch.int64, device=device)
+    d_keys = torch.empty(n0, dtype=torch.int64, device=device)
+    d_offs = torch.empty(nb0 + 1, dtype=torch.int64, device=device)
+    d_grad = torch.empty((nb0, w.dim), dtype=torch.float32, device=device)
+    d_pooled = torch.empty((nb0, w.dim), dtype=torch.float32, device=device)
+    t = dhs.ht_create(w.dim, w.optimizer, block_rows=w.block_rows, eps=w.eps, beta1=w.beta1, beta2=w.beta2)
+    h2d = d2h = 0
+
+    def step(s):
+        nonlocal h2d, d2h
+        tids, ids, offs, n, nb = hb[s]
+        g = hgrads[s % n_grad]
+        d_tids[:n].copy_(tids, non_blocking=True)
+        d_ids[:n].copy_(ids, non_blocking=True)
+        d_offs[: nb + 1].copy_(offs, non_blocking=True)
+        d_grad[:nb].copy_(g[:nb], non_blocking=True)
+        k = d_keys[:n]
+        dhs.dhs_pack_keys(d_tids[:n], d_ids[:n], out=k)
+        dhs.embbag_forward(t, k, d_offs[: nb + 1], out=d_pooled[:nb])
+        dhs.embbag_backward_update(t, k, d_offs[: nb + 1], d_grad[:nb], w.lr)
+        hpooled[:nb].copy_(d_pooled[:nb], non_blocking=True)
+        h2d += tids.numel() * 4 + ids.numel() * 8 + (nb + 1) * 8 + nb * w.dim * 4
+        d2h += nb * w.dim * 4
+
+    for s in range(args.warmup):
+        step(s)
+    torch.cuda.synchronize()
+    h2d = d2h = 0
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(dist, device)
+    torch.cuda.synchronize()
+    e0.record()
+    for s in range(args.warmup, total):
+        step(s)
+    e1.record()
+    torch.cuda.synchronize()
+    ms = max_over_ranks(e0.elapsed_time(e1), dist, device)
+    ids = sum_over_ranks(float(sum(hb[s][3] for s in range(args.warmup, total))), dist, device)
+    status = dhs.ht_sync(t)
+    t.close()
+    if status != 0:
+        raise RuntimeError(f"device status {status} in the end-to-end run")
+    K = args.steps
+    return {"value": ids / (ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d // K,
+            "d2h_bytes_per_step": d2h // K, "ms_per_step": ms / K}
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=40)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="dhs", choices=["dhs", "reference"])
+    ap.add_argument("--workload", default=WORKLOAD, choices=list(gen.NAMES))
+    ap.add_argument("--grad-buffers", type=int, default=32)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-steps", type=int, default=5)
+    ap.add_argument("--ref-frac", type=float, default=1.0 / 16)
+    ap.add_argument("--batch", type=int, default=0,
+                    help="samples per step (default: the workload's 65,536); smaller only for profiling")
+    args = ap.parse_args(argv)
+    if args.warmup < 0 or args.steps < 1:
+        ap.error("--steps must be >= 1 and --warmup >= 0")
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_dhs(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -243,10 +243,10 @@ def ht_export(t: Table) -> Tuple[np.ndarray, np.ndarray, int]:
 
 
 def ht_counters(t: Table) -> dict:
-    out = np.zeros(8, np.int64)
+    out = np.zeros(10, np.int64)
     _check("ht_counters", _lib.ht_counters(t.handle, out.ctypes.data))
     names = ("rows", "inserted", "unique_updated", "insert_calls", "backward_calls", "slots",
-             "blocks", "rehashes")
+             "blocks", "rehashes", "launches", "last_inserted")
     return {k: int(v) for k, v in zip(names, out)}
 
 

@@ -92,6 +92,7 @@ struct dhs_table {
   unsigned long long nslots = 0;
   long long n_rehash = 0;
   long long n_insert_calls = 0;
+  long long n_launches = 0;  // kernels launched by this table's calls
 
   std::vector<float*> blocks_h;
   float** blocks_d = nullptr;
@@ -280,10 +281,12 @@ dhs_status grow_map(dhs_table* t, unsigned long long want_slots, cudaStream_t s)
   const int thr = 256;
   const long long g = std::min<long long>((long long)((ns + thr - 1) / thr), (long long)t->sm_count * 16);
   fill_empty_kernel<<<(unsigned)g, thr, 0, s>>>(fresh, ns);
+  t->n_launches++;
   if (t->slots) {
     IdMap to{fresh, ns / 2 - 1};
     const long long g2 = std::min<long long>((long long)((t->nslots + thr - 1) / thr), (long long)t->sm_count * 16);
     rehash_kernel<<<(unsigned)g2, thr, 0, s>>>(t->slots, t->nslots, to, t->st);
+    t->n_launches++;
     dfree(t, t->slots, t->nslots * sizeof(Slot), s);
     t->n_rehash++;
   }
@@ -321,6 +324,7 @@ dhs_status ensure_capacity(dhs_table* t, long long n, cudaStream_t s) {
     t->blocks_h.push_back(b);
     set_block_kernel<<<1, 1, 0, s>>>(t->blocks_d, (long long)t->blocks_h.size() - 1, b, t->st,
                                      (unsigned long long)t->blocks_h.size());
+    t->n_launches++;
     DHS_TRY(last_launch());
     have += t->block_rows;
   }
@@ -365,6 +369,7 @@ dhs_status dispatch_pool(dhs_table* t, const long long* keys, long long n, const
   const cudaError_t e = launch_probe_pool(G, NV, t->sm_count, idmap(t), rowspace(t), t->dim, keys, n,
                                           bo, nb, out, (unsigned*)t->b_nbm.p,
                                           (unsigned*)t->b_slotpos.p, t->st, s);
+  t->n_launches++;
   if (e != cudaSuccess) cudaGetLastError();
   return e == cudaSuccess ? DHS_OK : DHS_ERR_CUDA;
 }
@@ -375,6 +380,7 @@ dhs_status dispatch_seg(dhs_table* t, const unsigned* sk, const unsigned* sv, lo
   const cudaError_t e = launch_seg(G, NV, t->sm_count, sk, sv, n, grad, nb, t->dim, rowspace(t), oa,
                                    (double*)t->b_ph.p, (double*)t->b_pt.p,
                                    (unsigned char*)t->b_cflags.p, kSegChunk, t->st, s);
+  t->n_launches++;
   if (e != cudaSuccess) cudaGetLastError();
   return e == cudaSuccess ? DHS_OK : DHS_ERR_CUDA;
 }
@@ -386,6 +392,7 @@ dhs_status launch_assign(dhs_table* t, long long n, cudaStream_t s) {
   fwd_mark_kernel<<<(unsigned)((nwords + 255) / 256), 256, 0, s>>>(
       t->slots, (unsigned*)t->b_nbm.p, (unsigned*)t->b_fbm.p, (unsigned*)t->b_gcnt.p,
       (unsigned*)t->b_gpref.p, (const unsigned*)t->b_slotpos.p, nwords, ngroups, t->st);
+  t->n_launches += 2;
   DHS_TRY(last_launch());
   fwd_assign_kernel<<<(unsigned)((ngroups + kAssignWarps - 1) / kAssignWarps), kAssignWarps * 32, 0, s>>>(
       t->slots, rowspace(t), t->dim, (const unsigned*)t->b_fbm.p, (const unsigned*)t->b_gpref.p,
@@ -554,6 +561,7 @@ dhs_status ht_lookup_or_insert(dhs_table* t, const int64_t* d_keys, int64_t n,
     fwd_probe_offsets_kernel<<<(unsigned)((n + kFwdThreads - 1) / kFwdThreads), kFwdThreads, 0, s>>>(
         idmap(t), (const long long*)d_keys, n, (long long*)d_offsets_out, (unsigned*)t->b_nbm.p,
         (unsigned*)t->b_slotpos.p, t->st);
+    t->n_launches += 2;
     DHS_TRY(last_launch());
     DHS_TRY(launch_assign(t, n, s));
     const long long grid = std::min<long long>((n + 255) / 256, (long long)t->sm_count * 8);
@@ -577,6 +585,7 @@ dhs_status ht_lookup(dhs_table* t, const int64_t* d_keys, int64_t n, int64_t* d_
   t->last_stream = s;
   const long long grid = std::min<long long>((n + 255) / 256, (long long)t->sm_count * 16);
   lookup_kernel<<<(unsigned)grid, 256, 0, s>>>(idmap(t), (const long long*)d_keys, n, (long long*)d_offsets_out);
+  t->n_launches++;
   return last_launch();
 }
 
@@ -648,6 +657,7 @@ dhs_status embbag_backward_update(dhs_table* t, const int64_t* d_keys, int64_t n
     bwd_probe_kernel<<<(unsigned)grid, 256, 0, s>>>(idmap(t), (const long long*)d_keys, n_keys,
                                                     (const long long*)d_bag_offsets, n_bags, ka, va,
                                                     sentinel, t->st);
+    t->n_launches++;
     DHS_TRY(last_launch());
   }
   {
@@ -662,6 +672,7 @@ dhs_status embbag_backward_update(dhs_table* t, const int64_t* d_keys, int64_t n
       radix_scatter_kernel<<<(unsigned)ntiles, kRadixThreads, 0, s>>>(
           ka, va, kb, vb, n_keys, shift, (const unsigned*)t->b_hist.p,
           (const unsigned*)t->b_totals.p, ntiles);
+      t->n_launches += 3;
       DHS_TRY(last_launch());
       std::swap(ka, kb);
       std::swap(va, vb);
@@ -689,6 +700,7 @@ dhs_status embbag_backward_update(dhs_table* t, const int64_t* d_keys, int64_t n
                                                         (const double*)t->b_ph.p, (const double*)t->b_pt.p,
                                                         (const unsigned char*)t->b_cflags.p, kSegChunk,
                                                         pstride, t->st);
+    t->n_launches++;
     DHS_TRY(last_launch());
   }
   return DHS_OK;
@@ -704,6 +716,7 @@ dhs_status ht_get_rows(dhs_table* t, const int64_t* d_keys, int64_t n, float* d_
   t->last_stream = s;
   const long long grid = std::min<long long>((n + 7) / 8, (long long)t->sm_count * 16);
   get_rows_kernel<<<(unsigned)grid, 256, 0, s>>>(idmap(t), rowspace(t), (const long long*)d_keys, n, d_rows_out);
+  t->n_launches++;
   return last_launch();
 }
 
@@ -736,7 +749,7 @@ dhs_status ht_size(dhs_table* t, int64_t* n_rows) {
   return rc;
 }
 
-dhs_status ht_counters(dhs_table* t, int64_t out[8]) {
+dhs_status ht_counters(dhs_table* t, int64_t out[10]) {
   DHS_TRY(check_table(t));
   if (!out) return DHS_ERR_INVALID_ARG;
   DeviceGuard g(t->device);
@@ -752,6 +765,8 @@ dhs_status ht_counters(dhs_table* t, int64_t out[8]) {
   out[5] = (int64_t)t->nslots;
   out[6] = (int64_t)t->blocks_h.size();
   out[7] = t->n_rehash;
+  out[8] = t->n_launches;
+  out[9] = (int64_t)h.m_last;
   return DHS_OK;
 }
 

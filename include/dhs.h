@@ -188,8 +188,10 @@ dhs_status ht_export(dhs_table* t, int64_t* h_keys, float* h_rows);
 /* Counters since creation (synchronises): out[0] rows, out[1] keys inserted
  * by forward / lookup-or-insert calls, out[2] sum over backward calls of the
  * distinct keys updated, out[3] forward-type calls, out[4] backward calls,
- * out[5] IDMap slots, out[6] blocks allocated, out[7] IDMap rehashes. */
-dhs_status ht_counters(dhs_table* t, int64_t out[8]);
+ * out[5] IDMap slots, out[6] blocks allocated, out[7] IDMap rehashes,
+ * out[8] kernels launched by the table's calls, out[9] keys inserted by the
+ * last insert call. */
+dhs_status ht_counters(dhs_table* t, int64_t out[10]);
 
 /* Per-phase device time, measured with CUDA events recorded on the call's
  * stream around each phase while enabled.  Phases: 0 forward probe + pool,

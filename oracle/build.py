@@ -3,6 +3,7 @@
 Plain g++, no CUDA.  -ffp-contract=off keeps every fp32 operation rounded on
 its own, as the oracle's definitions state.
 """
+import hashlib
 import os
 import subprocess
 import sys
@@ -12,13 +13,21 @@ SRC = os.path.join(HERE, "oracle.cpp")
 LIB = os.path.join(HERE, "liboracle.so")
 
 
+def _digest() -> str:
+    with open(SRC, "rb") as f:
+        return hashlib.sha256(f.read() + open(__file__, "rb").read()).hexdigest()
+
+
 def build(force: bool = False) -> str:
-    if not force and os.path.exists(LIB) and os.path.getmtime(LIB) >= os.path.getmtime(SRC):
+    stamp = LIB + ".stamp"
+    if not force and os.path.exists(LIB) and os.path.exists(stamp) and open(stamp).read().strip() == _digest():
         return LIB
     cmd = ["g++", "-O2", "-std=c++17", "-ffp-contract=off", "-fno-fast-math", "-fPIC", "-shared",
            "-Wall", "-o", LIB + ".tmp", SRC]
     subprocess.run(cmd, check=True)
     os.replace(LIB + ".tmp", LIB)
+    with open(stamp, "w") as f:
+        f.write(_digest())
     return LIB
 
 

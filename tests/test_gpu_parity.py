@@ -94,7 +94,7 @@ def test_lookup_or_insert_maps_first_occurrence_across_calls_and_growth():
         seen = np.zeros(0, np.int64)
         for call, n in enumerate([1, 4096, 33333, 70001, 5, 0, 25000]):
             fresh = rng.integers(0, 1 << 62, size=n // 2 + 1, dtype=np.int64)
-            old = seen[rng.integers(0, max(1, seen.size), size=n - n // 2 - 1)] if seen.size else fresh[:0]
+            old = seen[rng.integers(0, max(1, seen.size), size=max(0, n - n // 2 - 1))] if seen.size else fresh[:0]
             keys = rng.permutation(np.concatenate([fresh, old, fresh[: n // 7]]))[:n]
             g = host(dhs.ht_lookup_or_insert(t, dev(keys)))
             r, _ = o.lookup_or_insert(keys)
