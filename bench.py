@@ -20,9 +20,7 @@ import argparse
 import json
 import os
 import statistics
-import subprocess
 import sys
-import tempfile
 import time
 
 import numpy as np
@@ -88,57 +86,73 @@ def load_traffic(kernel: str):
 # clocks during the timed region
 # ---------------------------------------------------------------------------
 class ClockSampler:
-    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    """SM clock and clock-event reasons of this process's GPU, sampled every
+    ~10 ms by a thread through NVML while the timed region runs (two cheap
+    queries per sample, so the sampling does not stall the driver)."""
 
-    def __init__(self, gpu_index: int):
-        self.gpu = gpu_index
-        self.proc = None
-        self.path = None
+    REASONS = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
+               ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
+               ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown"),
+               ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap"),
+               ("hw_power_brake", "nvmlClocksEventReasonHwPowerBrakeSlowdown"))
+
+    def __init__(self, cuda_index: int, period_s: float = 0.01):
+        self.idx = cuda_index
+        self.period = period_s
+        self.samples = []
+        self.max_mhz = None
+        self._stop = None
+        self._thread = None
+        self.err = None
+
+    def _handle(self, nv):
+        try:
+            import torch
+            p = torch.cuda.get_device_properties(self.idx)
+            bus = f"{p.pci_domain_id:08x}:{p.pci_bus_id:02x}:{p.pci_device_id:02x}.0"
+            return nv.nvmlDeviceGetHandleByPciBusId(bus)
+        except Exception:
+            return nv.nvmlDeviceGetHandleByIndex(self.idx)
+
+    def _run(self):
+        import pynvml as nv
+        try:
+            nv.nvmlInit()
+            h = self._handle(nv)
+            self.max_mhz = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+            bits = [(name, getattr(nv, attr, 0)) for name, attr in self.REASONS]
+            while not self._stop.is_set():
+                mhz = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+                self.samples.append((time.perf_counter(), mhz, [n for n, bit in bits if bit and r & bit]))
+                self._stop.wait(self.period)
+        except Exception as e:  # no NVML: the line says so
+            self.err = repr(e)
 
     def __enter__(self):
-        fd, self.path = tempfile.mkstemp(suffix=".csv")
-        os.close(fd)
-        try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
-                 "-lms", "100"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
-            time.sleep(0.3)
-        except OSError:
-            self.proc = None
+        import threading
+        self._stop = threading.Event()
+        self._thread = threading.Thread(target=self._run, daemon=True)
+        self._thread.start()
+        time.sleep(0.05)
+        self.t0 = time.perf_counter()
         return self
 
     def __exit__(self, *a):
-        if self.proc is not None:
-            time.sleep(0.2)
-            self.proc.terminate()
-            try:
-                self.proc.wait(timeout=5)
-            except subprocess.TimeoutExpired:
-                self.proc.kill()
+        self.t1 = time.perf_counter()
+        time.sleep(0.02)
+        self._stop.set()
+        self._thread.join(timeout=5)
 
     def summary(self) -> dict:
-        rows = []
-        try:
-            with open(self.path) as f:
-                for line in f:
-                    parts = [x.strip() for x in line.split(",")]
-                    if len(parts) >= 9:
-                        rows.append(parts)
-        except OSError:
-            pass
-        finally:
-            if self.path and os.path.exists(self.path):
-                os.unlink(self.path)
-        if not rows:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
-        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
-        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
-                "reasons": reasons, "samples": len(rows)}
+        inside = [x for x in self.samples if self.t0 <= x[0] <= self.t1]
+        if not inside and self.samples:  # region shorter than one period: nearest samples
+            inside = sorted(self.samples, key=lambda x: min(abs(x[0] - self.t0), abs(x[0] - self.t1)))[:2]
+        if not inside:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unsampled"], "samples": 0,
+                    "error": self.err}
+        return {"sm_mhz": statistics.median(x[1] for x in inside), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted({r for x in inside for r in x[2]}), "samples": len(inside)}
 
 
 # ---------------------------------------------------------------------------
@@ -256,7 +270,8 @@ def workload_config(w) -> dict:
             "bags_per_step": int(p.get("batch", 0)) * int(p.get("tables", 1)),
             "dim": w.dim, "optimizer": w.optimizer,
             "l2": "inputs larger than L2 (per-step gradients 872 MB, keys 13.6 MB; 126 MB L2)",
-            "table": "starts empty; warm-up = the stream's first steps"}
+            "table": "starts empty (capacity for 6M keys reserved before step 0 unless --reserve-keys "
+                     "says otherwise); warm-up = the stream's first steps"}
 
 
 # ---------------------------------------------------------------------------
@@ -287,6 +302,8 @@ def run_dhs(args):
     keys = torch.empty(batches[0][3], dtype=torch.int64, device=device)
 
     t = dhs.ht_create(w.dim, w.optimizer, block_rows=w.block_rows, eps=w.eps, beta1=w.beta1, beta2=w.beta2)
+    if args.reserve_keys:
+        dhs.ht_reserve(t, args.reserve_keys)
     stream = torch.cuda.current_stream()
 
     def step(s):
@@ -367,7 +384,12 @@ def run_dhs(args):
         "per_step": {"ids": n_ids / K, "bags": n_bags / K, "unique": U / K, "new": M / K},
         "roofline": roofline,
         "gpu_launches": launches,
-        "table": {"rows": c1["rows"], "slots": c1["slots"], "blocks": c1["blocks"], "rehashes": c1["rehashes"]},
+        "table": {"rows": c1["rows"], "slots": c1["slots"], "blocks": c1["blocks"], "rehashes": c1["rehashes"],
+                  "reserved_keys": args.reserve_keys,
+                  "timed_growth": {"rehashes": c1["rehashes"] - c0["rehashes"],
+                                   "blocks_appended": c1["blocks"] - c0["blocks"],
+                                   "device_allocs": c1["allocs"] - c0["allocs"],
+                                   "host_wait_ms": (c1["host_wait_ns"] - c0["host_wait_ns"]) / 1e6}},
     }
     line["clocks"] = clk.summary()
     t.close()
@@ -414,6 +436,8 @@ def run_e2e(args, w, device, dist):
     d_grad = torch.empty((nb0, w.dim), dtype=torch.float32, device=device)
     d_pooled = torch.empty((nb0, w.dim), dtype=torch.float32, device=device)
     t = dhs.ht_create(w.dim, w.optimizer, block_rows=w.block_rows, eps=w.eps, beta1=w.beta1, beta2=w.beta2)
+    if args.reserve_keys:
+        dhs.ht_reserve(t, args.reserve_keys)
     h2d = d2h = 0
 
     def step(s):
@@ -467,6 +491,8 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-steps", type=int, default=5)
     ap.add_argument("--ref-frac", type=float, default=1.0 / 16)
+    ap.add_argument("--reserve-keys", type=int, default=6_000_000,
+                    help="capacity reserved (ht_reserve) before step 0; 0 = grow on demand")
     ap.add_argument("--batch", type=int, default=0,
                     help="samples per step (default: the workload's 65,536); smaller only for profiling")
     args = ap.parse_args(argv)

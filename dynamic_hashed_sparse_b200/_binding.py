@@ -19,7 +19,7 @@ from . import build as _build
 
 STATUS = {
     0: "ok", 1: "invalid argument", 2: "out of device memory", 3: "CUDA error",
-    4: "table full", 5: "key not found", 6: "unsupported",
+    4: "table full", 5: "key not found", 6: "unsupported", 7: "internal wait bound exceeded",
 }
 OPT_CODES = {"sgd": 0, "adagrad": 1, "adam": 2, "adagrad_rowwise": 3}
 PHASES = ("fwd_probe_pool", "fwd_assign", "bwd_probe", "bwd_sort", "bwd_seg_update",
@@ -243,10 +243,11 @@ def ht_export(t: Table) -> Tuple[np.ndarray, np.ndarray, int]:
 
 
 def ht_counters(t: Table) -> dict:
-    out = np.zeros(10, np.int64)
+    out = np.zeros(14, np.int64)
     _check("ht_counters", _lib.ht_counters(t.handle, out.ctypes.data))
     names = ("rows", "inserted", "unique_updated", "insert_calls", "backward_calls", "slots",
-             "blocks", "rehashes", "launches", "last_inserted")
+             "blocks", "rehashes", "launches", "last_inserted", "host_waits", "host_wait_ns",
+             "allocs", "alloc_ns")
     return {k: int(v) for k, v in zip(names, out)}
 
 

@@ -28,8 +28,10 @@ __global__ void __launch_bounds__(256)
 bwd_probe_kernel(IdMap m, const long long* __restrict__ keys, long long n_keys,
                  const long long* __restrict__ bag_off, long long n_bags,
                  unsigned* __restrict__ rkey, unsigned* __restrict__ rval, unsigned sentinel,
-                 DevState* st) {
+                 unsigned* __restrict__ sort_zero, int sort_zero_words, DevState* st) {
   const int lane = threadIdx.x & 31;
+  if (blockIdx.x == 0)  // the sort's digit histograms and tile counters start at zero
+    for (int i = threadIdx.x; i < sort_zero_words; i += blockDim.x) sort_zero[i] = 0u;
   const long long nchunks = (n_bags + 31) / 32;
   const long long nw = ((long long)gridDim.x * blockDim.x) >> 5;
   for (long long c = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5; c < nchunks;
@@ -81,34 +83,48 @@ bwd_probe_kernel(IdMap m, const long long* __restrict__ keys, long long n_keys,
 }
 
 // ---------------------------------------------------------------------------
-// LSD radix sort of 32-bit keys with 32-bit values, 8-bit digits, stable
+// LSD radix sort of 32-bit keys with 32-bit values, 8-bit digits, stable,
+// one kernel per digit pass (decoupled look-back across tiles)
 // ---------------------------------------------------------------------------
 constexpr int kRadixThreads = 256;
-constexpr int kRadixItems = 16;
-constexpr int kRadixWarpItems = 32 * kRadixItems;                     // 512
-constexpr int kRadixTile = kRadixWarpItems * (kRadixThreads / 32);    // 4096
+constexpr int kRadixItems = 8;
+constexpr int kRadixWarpItems = 32 * kRadixItems;                     // 256
+constexpr int kRadixTile = kRadixWarpItems * (kRadixThreads / 32);    // 2048
 constexpr int kRadixBins = 256;
+constexpr int kRadixMaxPasses = 4;
+constexpr unsigned long long kLbAggregate = 1ull << 62;  // tile count published
+constexpr unsigned long long kLbPrefix = 2ull << 62;     // inclusive prefix published
+constexpr unsigned long long kLbCountMask = (1ull << 62) - 1;
+constexpr unsigned kLookbackSpins = 1u << 22;  // bounded wait for a predecessor tile
 
-// Per-tile digit counts, stored digit-major: hist[d * ntiles + tile].
-// Lanes holding the same digit are merged with match.any before the shared
-// counter is bumped, so a hot row costs one atomic per warp round.
+// Digit counts of every pass in one read of the keys (global atomics, one per
+// block and bin), and the look-back state of every pass cleared.  hist and
+// tile_ctr must be zero on entry (bwd_probe_kernel clears them).
 __global__ void __launch_bounds__(kRadixThreads)
-radix_hist_kernel(const unsigned* __restrict__ keys, long long n, int shift,
-                  unsigned* __restrict__ hist, long long ntiles) {
-  __shared__ unsigned h[kRadixBins];
-  h[threadIdx.x] = 0;
+radix_hist_all_kernel(const unsigned* __restrict__ keys, long long n, int passes,
+                      unsigned* __restrict__ hist, unsigned long long* __restrict__ status,
+                      long long status_words) {
+  __shared__ unsigned h[kRadixMaxPasses][kRadixBins];
+  for (int i = threadIdx.x; i < kRadixMaxPasses * kRadixBins; i += kRadixThreads) (&h[0][0])[i] = 0;
   __syncthreads();
-  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-  const long long base = (long long)blockIdx.x * kRadixTile + (long long)wid * kRadixWarpItems;
-#pragma unroll 4
-  for (int r = 0; r < kRadixItems; ++r) {
-    const long long p = base + r * 32 + lane;
-    const unsigned d = p < n ? ((__ldg(keys + p) >> shift) & 255u) : 256u;
-    const unsigned peers = __match_any_sync(0xffffffffu, d);
-    if (d < 256u && (__ffs(peers) - 1) == lane) atomicAdd(&h[d], (unsigned)__popc(peers));
+  const int lane = threadIdx.x & 31;
+  const long long stride = (long long)gridDim.x * kRadixThreads;
+  for (long long base = (long long)blockIdx.x * kRadixThreads; base < n; base += stride) {
+    const long long p = base + threadIdx.x;
+    const unsigned k = p < n ? __ldg(keys + p) : 0u;
+    for (int ps = 0; ps < passes; ++ps) {
+      const unsigned d = p < n ? ((k >> (8 * ps)) & 255u) : 256u;
+      const unsigned peers = __match_any_sync(0xffffffffu, d);
+      if (d < 256u && (__ffs(peers) - 1) == lane) atomicAdd(&h[ps][d], (unsigned)__popc(peers));
+    }
   }
   __syncthreads();
-  hist[(long long)threadIdx.x * ntiles + blockIdx.x] = h[threadIdx.x];
+  for (int i = threadIdx.x; i < passes * kRadixBins; i += kRadixThreads) {
+    const unsigned v = (&h[0][0])[i];
+    if (v) atomicAdd(hist + i, v);
+  }
+  for (long long i = (long long)blockIdx.x * kRadixThreads + threadIdx.x; i < status_words; i += stride)
+    status[i] = 0ull;
 }
 
 // Block-wide exclusive scan of one value per thread (256 threads).
@@ -135,52 +151,36 @@ __device__ __forceinline__ unsigned block_exclusive_scan_256(unsigned x, unsigne
   return pre + inc - x;
 }
 
-// In-place exclusive scan of one digit's row hist[d * ntiles, +ntiles); block
-// d also writes the digit total.
-__global__ void __launch_bounds__(256)
-radix_scan_kernel(unsigned* __restrict__ hist, long long ntiles, unsigned* __restrict__ totals) {
-  __shared__ unsigned wsum[8];
-  unsigned* row = hist + (long long)blockIdx.x * ntiles;
-  unsigned carry = 0;
-  for (long long b = 0; b < ntiles; b += 256) {
-    const long long i = b + threadIdx.x;
-    const unsigned x = i < ntiles ? row[i] : 0u;
-    unsigned tot;
-    const unsigned ex = block_exclusive_scan_256(x, wsum, tot);
-    if (i < ntiles) row[i] = carry + ex;
-    carry += tot;
-  }
-  if (threadIdx.x == 0) totals[blockIdx.x] = carry;
-}
-
-// Stable scatter of one tile.  Each warp ranks its 512 items in order (16
-// rounds of 32 lanes; match.any gives the rank among equal digits within a
-// round, a per-warp shared counter carries it across rounds), the block turns
-// per-warp counts into tile-local digit offsets, the items are placed in
-// digit order in shared memory and written out in runs, one run per digit,
-// to the tile's global offsets.
+// One stable digit pass.  Tiles are numbered in the order blocks start (an
+// atomic counter), so a tile only ever waits for tiles whose blocks are
+// already running.  Each warp ranks its 256 items in order (8 rounds of 32
+// lanes; match.any gives the rank among equal digits within a round, a
+// per-warp shared counter carries it across rounds); the tile publishes its
+// digit counts, adds up its predecessors' (decoupled look-back), publishes
+// its inclusive prefix, places its items in digit order in shared memory and
+// writes them out in runs.  A wait that exceeds its bound latches
+// kErrInternal and the pass goes on (its output is then undefined, never out
+// of bounds).
 __global__ void __launch_bounds__(kRadixThreads)
-radix_scatter_kernel(const unsigned* __restrict__ kin, const unsigned* __restrict__ vin,
-                     unsigned* __restrict__ kout, unsigned* __restrict__ vout, long long n,
-                     int shift, const unsigned* __restrict__ hist,
-                     const unsigned* __restrict__ totals, long long ntiles) {
+radix_onesweep_kernel(const unsigned* __restrict__ kin, const unsigned* __restrict__ vin,
+                      unsigned* __restrict__ kout, unsigned* __restrict__ vout, long long n,
+                      int shift, const unsigned* __restrict__ hist,
+                      unsigned long long* __restrict__ status, unsigned* __restrict__ tile_ctr,
+                      DevState* st) {
   __shared__ unsigned s_k[kRadixTile];
   __shared__ unsigned s_v[kRadixTile];
   __shared__ unsigned wc[8][kRadixBins + 1];
   __shared__ unsigned dstart[kRadixBins];
   __shared__ unsigned gbase[kRadixBins];
   __shared__ unsigned wsum[8];
+  __shared__ unsigned s_tile;
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-  const long long tile0 = (long long)blockIdx.x * kRadixTile;
-  const int tile_n = (int)min((long long)kRadixTile, n - tile0);
-
+  if (threadIdx.x == 0) s_tile = atomicAdd(tile_ctr, 1u);
   for (int i = threadIdx.x; i < 8 * (kRadixBins + 1); i += kRadixThreads) (&wc[0][0])[i] = 0;
-  {
-    unsigned tot;
-    const unsigned dpre = block_exclusive_scan_256(totals[threadIdx.x], wsum, tot);
-    gbase[threadIdx.x] = dpre + hist[(long long)threadIdx.x * ntiles + blockIdx.x];
-  }
   __syncthreads();
+  const long long tile = s_tile;
+  const long long tile0 = tile * kRadixTile;
+  const int tile_n = (int)max(0ll, min((long long)kRadixTile, n - tile0));
 
   unsigned k[kRadixItems], v[kRadixItems], lr[kRadixItems];
   const long long base = tile0 + (long long)wid * kRadixWarpItems;
@@ -204,25 +204,57 @@ radix_scatter_kernel(const unsigned* __restrict__ kin, const unsigned* __restric
     __syncwarp();
   }
   __syncthreads();
-  {
-    const int d = threadIdx.x;
-    unsigned pre = 0;
+  const int d = threadIdx.x;
+  unsigned cnt = 0;
 #pragma unroll
-    for (int w = 0; w < 8; ++w) {
-      const unsigned t = wc[w][d];
-      wc[w][d] = pre;
-      pre += t;
+  for (int w = 0; w < 8; ++w) {
+    const unsigned t = wc[w][d];
+    wc[w][d] = cnt;
+    cnt += t;
+  }
+  // publish this tile's count of digit d, then look back over the predecessors
+  volatile unsigned long long* sp = status + tile * kRadixBins + d;
+  if (tile == 0) {
+    *sp = kLbPrefix | cnt;
+  } else {
+    *sp = kLbAggregate | cnt;
+  }
+  unsigned long long excl = 0;
+  if (tile > 0) {
+    long long t = tile - 1;
+    unsigned spins = 0;
+    while (t >= 0) {
+      const unsigned long long sv = *(volatile unsigned long long*)(status + t * kRadixBins + d);
+      if (sv & kLbPrefix) {
+        excl += sv & kLbCountMask;
+        break;
+      }
+      if (sv & kLbAggregate) {
+        excl += sv & kLbCountMask;
+        --t;
+        continue;
+      }
+      if (++spins > kLookbackSpins) {
+        latch(st, kErrInternal);
+        break;
+      }
+      __nanosleep(32);
     }
+    *sp = kLbPrefix | (excl + cnt);
+  }
+  {
     unsigned tot;
-    dstart[d] = block_exclusive_scan_256(pre, wsum, tot);
+    const unsigned dpre = block_exclusive_scan_256(hist[d], wsum, tot);
+    gbase[d] = dpre + (unsigned)excl;
+    dstart[d] = block_exclusive_scan_256(cnt, wsum, tot);
   }
   __syncthreads();
 #pragma unroll
   for (int r = 0; r < kRadixItems; ++r) {
     const long long p = base + r * 32 + lane;
     if (p < n) {
-      const unsigned d = (k[r] >> shift) & 255u;
-      const unsigned pos = dstart[d] + wc[wid][d] + lr[r];
+      const unsigned dd = (k[r] >> shift) & 255u;
+      const unsigned pos = dstart[dd] + wc[wid][dd] + lr[r];
       s_k[pos] = k[r];
       s_v[pos] = v[r];
     }
@@ -230,8 +262,8 @@ radix_scatter_kernel(const unsigned* __restrict__ kin, const unsigned* __restric
   __syncthreads();
   for (int i = threadIdx.x; i < tile_n; i += kRadixThreads) {
     const unsigned key = s_k[i];
-    const unsigned d = (key >> shift) & 255u;
-    const unsigned o = gbase[d] + (unsigned)i - dstart[d];
+    const unsigned dd = (key >> shift) & 255u;
+    const unsigned o = gbase[dd] + (unsigned)i - dstart[dd];
     kout[o] = key;
     vout[o] = s_v[i];
   }
@@ -266,63 +298,69 @@ __device__ __forceinline__ void adam_step(float& w, float& m, float& v, float g,
   w = __fsub_rn(w, __fdiv_rn(__fmul_rn(o.lr, mhat), __fadd_rn(__fsqrt_rn(vhat), o.eps)));
 }
 
-// Group of G lanes, lane gl holding float4 columns gl + q*G (q < NV) of the
-// row gradient in fp64; rowwise_sq is the fp64 sum of g^2 over the row (only
-// used by row-wise Adagrad, computed by the caller over the group).
-template <int NV>
-__device__ __forceinline__ void update_row_vec(float* row, int dim, int gl, int G,
-                                               const double (&acc)[NV][4], const OptArgs& o,
-                                               double rowwise_sq) {
-  const int d4 = dim >> 2;
-  float4* w4 = reinterpret_cast<float4*>(row);
-  if (o.opt == 3) {
-    // one accumulator per row, stored at row[dim]; every lane computes the
-    // same new value, lane 0 stores it
-    const float G0 = row[dim];
-    const float Gn = __fadd_rn(G0, (float)(rowwise_sq / (double)dim));
-    const float den = __fadd_rn(__fsqrt_rn(Gn), o.eps);
+// The part of one row a lane owns: float4 columns gl + q*G (q < NV) of the
+// weights and of each per-element state array (Adagrad: G; Adam: m, v), plus
+// the row accumulator of row-wise Adagrad.  Loaded when a segment opens, so
+// the loads overlap the gradient sum; written back once when it closes.
+template <int OPT, int NV>
+struct RowBuf {
+  static constexpr int NS = OPT == 1 ? 1 : (OPT == 2 ? 2 : 0);
+  float4 w[NV];
+  float4 st[NS > 0 ? NS : 1][NV];
+  float acc_row;
+
+  __device__ __forceinline__ void load(const float* row, int dim, int gl, int G) {
+    const int d4 = dim >> 2;
+    const float4* r4 = reinterpret_cast<const float4*>(row);
+#pragma unroll
+    for (int q = 0; q < NV; ++q) {
+      const int c4 = gl + q * G;
+      if (c4 < d4) {
+        w[q] = r4[c4];
+#pragma unroll
+        for (int k = 0; k < NS; ++k) st[k][q] = r4[(k + 1) * d4 + c4];
+      }
+    }
+    if (OPT == 3) acc_row = row[dim];
+  }
+
+  // one optimizer step with the row gradient held in fp64 by this lane;
+  // rowwise_sq = sum over the whole row of g^2 (row-wise Adagrad only)
+  __device__ __forceinline__ void step_store(float* row, int dim, int gl, int G,
+                                             const double (&acc)[NV][4], const OptArgs& o,
+                                             double rowwise_sq) {
+    const int d4 = dim >> 2;
+    float4* r4 = reinterpret_cast<float4*>(row);
+    float den = 0.f, Gn = 0.f;
+    if (OPT == 3) {
+      Gn = __fadd_rn(acc_row, (float)(rowwise_sq / (double)dim));
+      den = __fadd_rn(__fsqrt_rn(Gn), o.eps);
+    }
 #pragma unroll
     for (int q = 0; q < NV; ++q) {
       const int c4 = gl + q * G;
       if (c4 >= d4) continue;
-      float4 w = w4[c4];
-      float* wp = &w.x;
+      float* wp = &w[q].x;
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const float g = (float)acc[q][e];
-        wp[e] = __fsub_rn(wp[e], __fdiv_rn(__fmul_rn(o.lr, g), den));
+        if (OPT == 0) {
+          wp[e] = sgd_w(wp[e], g, o.lr);
+        } else if (OPT == 1) {
+          adagrad_step(wp[e], (&st[0][q].x)[e], g, o.lr, o.eps);
+        } else if (OPT == 2) {
+          adam_step(wp[e], (&st[0][q].x)[e], (&st[NS - 1][q].x)[e], g, o);
+        } else {
+          wp[e] = __fsub_rn(wp[e], __fdiv_rn(__fmul_rn(o.lr, g), den));
+        }
       }
-      w4[c4] = w;
+      r4[c4] = w[q];
+#pragma unroll
+      for (int k = 0; k < NS; ++k) r4[(k + 1) * d4 + c4] = st[k][q];
     }
-    if (gl == 0) row[dim] = Gn;
-    return;
+    if (OPT == 3 && gl == 0) row[dim] = Gn;
   }
-#pragma unroll
-  for (int q = 0; q < NV; ++q) {
-    const int c4 = gl + q * G;
-    if (c4 >= d4) continue;
-    float4 w = w4[c4];
-    float* wp = &w.x;
-    if (o.opt == 0) {
-#pragma unroll
-      for (int e = 0; e < 4; ++e) wp[e] = sgd_w(wp[e], (float)acc[q][e], o.lr);
-    } else if (o.opt == 1) {
-      float4 Gs = w4[d4 + c4];
-      float* gp = &Gs.x;
-#pragma unroll
-      for (int e = 0; e < 4; ++e) adagrad_step(wp[e], gp[e], (float)acc[q][e], o.lr, o.eps);
-      w4[d4 + c4] = Gs;
-    } else {
-      float4 ms = w4[d4 + c4], vs = w4[2 * d4 + c4];
-      float *mp = &ms.x, *vp = &vs.x;
-#pragma unroll
-      for (int e = 0; e < 4; ++e) adam_step(wp[e], mp[e], vp[e], (float)acc[q][e], o);
-      w4[d4 + c4] = ms;
-      w4[2 * d4 + c4] = vs;
-    }
-    w4[c4] = w;
-  }
-}
+};
 
 // Scalar form for one column j (used by the combine kernel).
 __device__ __forceinline__ void update_col(float* row, int dim, int j, float g, const OptArgs& o,
@@ -358,30 +396,54 @@ enum : unsigned char { kPieceHead = 1, kPieceThrough = 2, kPieceTailStart = 4 };
 // starts here and ends in the next chunk is finished here (short overrun); one
 // that reaches chunk c + 2 is long: its piece up to the chunk end is written
 // as the starting partial and bwd_combine_kernel finishes it.
-template <int G, int NV>
-__global__ void __launch_bounds__(256)
+// Piece modes: 0 skip (owned by the previous chunk), 1 long head piece,
+// 2 owned short segment, 3 long segment starting here.
+template <int G, int NV, int OPT>
+__global__ void __launch_bounds__(256, NV == 1 ? 3 : (NV == 2 ? 2 : 1))
 bwd_seg_kernel(const unsigned* __restrict__ skey, const unsigned* __restrict__ sval, long long n,
                const float* __restrict__ grad, long long n_bags, int dim, RowSpace rs, OptArgs oa,
                double* __restrict__ part_head, double* __restrict__ part_tail,
                unsigned char* __restrict__ cflags, int C, DevState* st) {
-  constexpr int U = G < 8 ? G : 8;
+  constexpr int U = G < 4 ? G : 4;
   const int lane = threadIdx.x & 31;
   const int gl = lane & (G - 1);
   const int gw = lane / G;
   const unsigned gmask = (G == 32) ? 0xffffffffu : (((1u << G) - 1u) << (gw * G));
-  const long long gid = ((long long)blockIdx.x * blockDim.x + threadIdx.x) / G;
-  const long long ngroups = ((long long)gridDim.x * blockDim.x) / G;
-  const long long nchunks = (n + C - 1) / C;
-  const unsigned long long nrows = st->row_count;
+  // positions fit in 31 bits (the host rejects larger calls)
+  const int n32 = (int)n;
+  const int gid = (int)((blockIdx.x * blockDim.x + threadIdx.x) / G);
+  const int ngroups = (int)((gridDim.x * blockDim.x) / G);
+  const int nchunks = (n32 + C - 1) / C;
+  const unsigned nrows = (unsigned)min(st->row_count, 0xffffffffull);
   const int d4 = dim >> 2;
   const int pstride = NV * G * 4;  // doubles per partial vector
-  unsigned long long nseg_total = 0;
+  unsigned nseg_total = 0;
 
-  for (long long c = gid; c < nchunks; c += ngroups) {
-    const long long start = c * C;
-    const long long end = min(n, start + C);
+  for (int c = gid; c < nchunks; c += ngroups) {
+    const int start = c * C;
+    const int end = min(n32, start + C);
     unsigned char flags = 0;
     unsigned nseg = 0;
+
+    // the keys that decide who owns the chunk's first and last pieces
+    const unsigned cur0 = __ldg(skey + start);
+    const unsigned prev = start > 0 ? __ldg(skey + start - 1) : ~0u;
+    const unsigned back2 = c >= 2 ? __ldg(skey + (c - 1) * C - 1) : ~0u;
+    const unsigned fwd1 = (c + 1) * C < n32 ? __ldg(skey + (c + 1) * C) : ~0u;
+    const int p2 = (c + 2) * C;
+    const bool has2 = p2 < n32;
+    const unsigned fwd2 = has2 ? __ldg(skey + p2) : ~0u;
+
+    unsigned cur = cur0;
+    int mode;
+    if (start > 0 && prev == cur) {
+      mode = (back2 == cur || fwd1 == cur) ? 1 : 0;
+    } else {
+      ++nseg;
+      mode = (has2 && fwd2 == cur) ? 3 : 2;
+    }
+    RowBuf<OPT, NV> rb;
+    if (mode == 2 && cur < nrows) rb.load(rs.row(cur), dim, gl, G);
 
     double acc[NV][4];
 #pragma unroll
@@ -389,60 +451,33 @@ bwd_seg_kernel(const unsigned* __restrict__ skey, const unsigned* __restrict__ s
 #pragma unroll
       for (int e = 0; e < 4; ++e) acc[q][e] = 0.0;
 
-    // mode of the piece being read: 0 skip, 1 long head piece, 2 owned short
-    // segment, 3 long segment starting here
-    int mode;
-    unsigned cur = __ldg(skey + start);
-    if (start > 0 && __ldg(skey + start - 1) == cur) {
-      const bool head_long = (c >= 2 && __ldg(skey + (c - 1) * (long long)C - 1) == cur) ||
-                             ((c + 1) * (long long)C < n && __ldg(skey + (c + 1) * (long long)C) == cur);
-      mode = head_long ? 1 : 0;
-    } else {
-      ++nseg;
-      mode = ((c + 2) * (long long)C < n && __ldg(skey + (c + 2) * (long long)C) == cur) ? 3 : 2;
-    }
-
-    auto close_piece = [&](bool continues) {
-      if (mode == 1) {
-        double* o = part_head + c * (long long)pstride;
-#pragma unroll
-        for (int q = 0; q < NV; ++q)
-#pragma unroll
-          for (int e = 0; e < 4; ++e) o[(q * G + gl) * 4 + e] = acc[q][e];
-        flags |= continues ? kPieceThrough : kPieceHead;
-      } else if (mode == 3) {
-        double* o = part_tail + c * (long long)pstride;
-#pragma unroll
-        for (int q = 0; q < NV; ++q)
-#pragma unroll
-          for (int e = 0; e < 4; ++e) o[(q * G + gl) * 4 + e] = acc[q][e];
-        flags |= kPieceTailStart;
-      } else if (mode == 2 && cur < nrows) {
-        double sq = 0.0;
-        if (oa.opt == 3) {
-#pragma unroll
-          for (int q = 0; q < NV; ++q)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const double g = (double)(float)acc[q][e];
-              sq += g * g;
-            }
-#pragma unroll
-          for (int o = 1; o < G; o <<= 1) sq += __shfl_xor_sync(gmask, sq, o, G);
-        }
-        update_row_vec<NV>(rs.row(cur), dim, gl, G, acc, oa, sq);
+    // Window pipeline: the sorted (row, bag) pairs of window ws + G are loaded
+    // while window ws is processed, and each lane bulk-prefetches into L2 the
+    // gradient row of its pair and, where its pair opens a segment, the
+    // table row + state.  The register loads below then mostly hit L2.
+    const unsigned grad_bytes = (unsigned)dim * 4u;
+    const unsigned row_bytes = (unsigned)rs.stride * 4u;
+    auto prefetch_window = [&](int wsn, unsigned& kn, unsigned& vn, unsigned prev_last) {
+      const int cn = min(G, n32 - wsn);
+      kn = gl < cn ? __ldg(skey + wsn + gl) : 0u;
+      vn = gl < cn ? __ldg(sval + wsn + gl) : 0u;
+      const unsigned up = __shfl_up_sync(gmask, kn, 1, G);
+      const unsigned before = gl == 0 ? prev_last : up;
+      if (gl < cn && kn < nrows) {
+        if (vn < n_bags) prefetch_l2(grad + (long long)vn * dim, grad_bytes);
+        if (kn != before) prefetch_l2(rs.row(kn), row_bytes);
       }
-#pragma unroll
-      for (int q = 0; q < NV; ++q)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) acc[q][e] = 0.0;
     };
+    unsigned kk, vv, kk_next = 0u, vv_next = 0u;
+    prefetch_window(start, kk, vv, prev);
 
     bool done = false;
-    for (long long ws = start; ws < n && !done; ws += G) {
-      const int cnt = (int)min((long long)G, n - ws);
-      const unsigned kk = gl < cnt ? __ldg(skey + ws + gl) : 0u;
-      const unsigned vv = gl < cnt ? __ldg(sval + ws + gl) : 0u;
+    for (int ws = start; ws < n32 && !done; ws += G) {
+      const int cnt = min(G, n32 - ws);
+      const unsigned last = __shfl_sync(gmask, kk, (cnt - 1) & (G - 1), G);
+      // (a short segment may run to the first element of chunk c + 2, so the
+      // next window is always loaded while positions remain)
+      if (ws + G < n32) prefetch_window(ws + G, kk_next, vv_next, last);
       for (int t0 = 0; t0 < cnt && !done; t0 += U) {
         float4 x[U][NV];
 #pragma unroll
@@ -462,22 +497,50 @@ bwd_seg_kernel(const unsigned* __restrict__ skey, const unsigned* __restrict__ s
         for (int u = 0; u < U; ++u) {
           const int t = t0 + u;
           if (done || t >= cnt) break;
-          const long long p = ws + t;
+          const int p = ws + t;
           const unsigned kt = __shfl_sync(gmask, kk, t & (G - 1), G);
+          bool close = false, cont = false;
           if (kt != cur) {
-            close_piece(false);
-            if (p >= end) {
+            close = true;
+          } else if (p == end && mode != 2) {
+            close = true;  // a long piece stops at the chunk end
+            cont = true;
+          }
+          if (close) {
+            if (mode == 1 || mode == 3) {
+              double* o = (mode == 1 ? part_head : part_tail) + (long long)c * pstride;
+#pragma unroll
+              for (int q = 0; q < NV; ++q)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) o[(q * G + gl) * 4 + e] = acc[q][e];
+              flags |= mode == 3 ? kPieceTailStart : (cont ? kPieceThrough : kPieceHead);
+            } else if (mode == 2 && cur < nrows) {
+              double sq = 0.0;
+              if (OPT == 3) {
+#pragma unroll
+                for (int q = 0; q < NV; ++q)
+#pragma unroll
+                  for (int e = 0; e < 4; ++e) {
+                    const double g = (double)(float)acc[q][e];
+                    sq += g * g;
+                  }
+#pragma unroll
+                for (int o = 1; o < G; o <<= 1) sq += __shfl_xor_sync(gmask, sq, o, G);
+              }
+              rb.step_store(rs.row(cur), dim, gl, G, acc, oa, sq);
+            }
+#pragma unroll
+            for (int q = 0; q < NV; ++q)
+#pragma unroll
+              for (int e = 0; e < 4; ++e) acc[q][e] = 0.0;
+            if (cont || p >= end) {
               done = true;
               break;
             }
             cur = kt;
             ++nseg;
-            mode = ((c + 2) * (long long)C < n && __ldg(skey + (c + 2) * (long long)C) == cur) ? 3 : 2;
-          } else if (p == end && mode != 2) {
-            // a long piece (head or starting) stops at the chunk end
-            close_piece(true);
-            done = true;
-            break;
+            mode = (has2 && fwd2 == cur) ? 3 : 2;
+            if (mode == 2 && cur < nrows) rb.load(rs.row(cur), dim, gl, G);
           }
           if (mode != 0) {
 #pragma unroll
@@ -490,15 +553,40 @@ bwd_seg_kernel(const unsigned* __restrict__ skey, const unsigned* __restrict__ s
           }
         }
       }
+      kk = kk_next;
+      vv = vv_next;
     }
-    if (!done) close_piece(false);  // reached the end of the array
+    if (!done) {  // reached the end of the array with a piece open
+      if (mode == 1 || mode == 3) {
+        double* o = (mode == 1 ? part_head : part_tail) + (long long)c * pstride;
+#pragma unroll
+        for (int q = 0; q < NV; ++q)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) o[(q * G + gl) * 4 + e] = acc[q][e];
+        flags |= mode == 3 ? kPieceTailStart : kPieceHead;
+      } else if (mode == 2 && cur < nrows) {
+        double sq = 0.0;
+        if (OPT == 3) {
+#pragma unroll
+          for (int q = 0; q < NV; ++q)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const double g = (double)(float)acc[q][e];
+              sq += g * g;
+            }
+#pragma unroll
+          for (int o = 1; o < G; o <<= 1) sq += __shfl_xor_sync(gmask, sq, o, G);
+        }
+        rb.step_store(rs.row(cur), dim, gl, G, acc, oa, sq);
+      }
+    }
     if (gl == 0) {
       cflags[c] = flags;
-      if (cur >= nrows && nseg) --nseg;  // the sentinel run is not a row
+      if (cur >= nrows && nseg) --nseg;  // the missing-key run is not a row
       nseg_total += nseg;
     }
   }
-  if (gl == 0 && nseg_total) atomicAdd(&st->sum_unique, nseg_total);
+  if (gl == 0 && nseg_total) atomicAdd(&st->sum_unique, (unsigned long long)nseg_total);
 }
 
 #ifndef DHS_TEMPLATES_ONLY

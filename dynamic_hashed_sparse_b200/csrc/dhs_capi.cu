@@ -8,6 +8,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <chrono>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -29,7 +30,11 @@ constexpr long long kDefaultMaxRows = 1ll << 31;
 constexpr long long kMaxRowsLimit = (1ll << 32) - 2;
 constexpr unsigned long long kInitialSlots = 1ull << 16;
 constexpr double kMaxLoad = 0.5;
-constexpr int kSegChunk = 256;
+// Sort chunk of the segment-reduce kernel: big enough that a group's fixed
+// work per chunk stays small, small enough that every SM gets many chunks.
+int seg_chunk(long long n) {
+  return n > 4000000 ? 256 : n > 500000 ? 128 : n > 100000 ? 64 : 32;
+}
 constexpr int kSnapRing = 4;
 enum { PH_FWD_POOL = 0, PH_FWD_ASSIGN = 1, PH_BWD_PROBE = 2, PH_BWD_SORT = 3, PH_BWD_SEG = 4,
        PH_LOOKUP_INSERT = 5, PH_GROW = 6 };
@@ -86,6 +91,7 @@ struct dhs_table {
   long long max_blocks = 0;
   dhs_allocator alloc{};
   bool custom_alloc = false;
+  cudaMemPool_t pool = nullptr;  // table-owned stream-ordered pool (keeps freed memory)
   cudaStream_t last_stream = nullptr;
 
   Slot* slots = nullptr;
@@ -93,6 +99,8 @@ struct dhs_table {
   long long n_rehash = 0;
   long long n_insert_calls = 0;
   long long n_launches = 0;  // kernels launched by this table's calls
+  long long n_host_waits = 0, host_wait_ns = 0;  // host blocked on the device
+  long long n_allocs = 0, alloc_ns = 0;          // device allocations
 
   std::vector<float*> blocks_h;
   float** blocks_d = nullptr;
@@ -116,15 +124,33 @@ struct dhs_table {
 
 namespace {
 
+long long now_ns() {
+  return std::chrono::duration_cast<std::chrono::nanoseconds>(
+             std::chrono::steady_clock::now().time_since_epoch())
+      .count();
+}
+
 void* dalloc(dhs_table* t, size_t bytes, cudaStream_t s) {
   if (bytes == 0) bytes = 16;
-  if (t->custom_alloc) return t->alloc.alloc(bytes, (dhs_stream)s, t->alloc.ctx);
+  const long long t0 = now_ns();
   void* p = nullptr;
-  if (cudaMallocAsync(&p, bytes, s) != cudaSuccess) {
+  if (t->custom_alloc) {
+    p = t->alloc.alloc(bytes, (dhs_stream)s, t->alloc.ctx);
+  } else if (cudaMallocFromPoolAsync(&p, bytes, t->pool, s) != cudaSuccess) {
     cudaGetLastError();
-    return nullptr;
+    p = nullptr;
   }
+  t->n_allocs++;
+  t->alloc_ns += now_ns() - t0;
   return p;
+}
+
+cudaError_t host_wait(dhs_table* t, cudaEvent_t ev) {
+  const long long t0 = now_ns();
+  const cudaError_t e = cudaEventSynchronize(ev);
+  t->n_host_waits++;
+  t->host_wait_ns += now_ns() - t0;
+  return e;
 }
 
 void dfree(dhs_table* t, void* p, size_t bytes, cudaStream_t s) {
@@ -246,7 +272,7 @@ void refresh_ub(dhs_table* t, bool wait) {
     const int k = ((t->snap_next - 1 - i) % kSnapRing + kSnapRing) % kSnapRing;
     Snap& sn = t->snaps[k];
     if (!sn.valid) continue;
-    cudaError_t q = wait && i == 0 ? cudaEventSynchronize(sn.ev) : cudaEventQuery(sn.ev);
+    cudaError_t q = wait && i == 0 ? host_wait(t, sn.ev) : cudaEventQuery(sn.ev);
     if (q == cudaSuccess) {
       const long long ub = (long long)*sn.pinned + (t->cum_n - sn.cum_n);
       if (ub < t->rows_ub) t->rows_ub = ub;
@@ -258,7 +284,7 @@ void refresh_ub(dhs_table* t, bool wait) {
 
 void record_snapshot(dhs_table* t, cudaStream_t s) {
   Snap& sn = t->snaps[t->snap_next];
-  if (sn.valid) cudaEventSynchronize(sn.ev);  // ring slot reuse: at most kSnapRing in flight
+  if (sn.valid) host_wait(t, sn.ev);  // ring slot reuse: at most kSnapRing in flight
   cudaMemcpyAsync(sn.pinned, &t->st->row_count, sizeof(unsigned long long), cudaMemcpyDeviceToHost, s);
   cudaEventRecord(sn.ev, s);
   sn.cum_n = t->cum_n;
@@ -335,10 +361,10 @@ dhs_status ensure_ws(dhs_table* t, long long n, cudaStream_t s) {
   if (n <= t->ws_n) return DHS_OK;
   long long cap = std::max<long long>(n, t->ws_n > 0 ? t->ws_n + t->ws_n / 2 : 0);
   cap = std::max<long long>(cap, 4096);
-  const long long nwords = (cap + 31) / 32 + 32;
-  const long long ngroups = (cap + 1023) / 1024 + 1;
+  const long long ngroups = (cap + kGroupPositions - 1) / kGroupPositions + 1;
+  const long long nwords = ngroups * kGroupWords;
   const long long ntiles = (cap + kRadixTile - 1) / kRadixTile;
-  const long long nchunks = (cap + kSegChunk - 1) / kSegChunk;
+  const long long nchunks = (cap + seg_chunk(cap) - 1) / seg_chunk(cap) + (cap + 31) / 32;
   const int G = pick_group(t->dim), NV = pick_nv(t->dim, G);
   const long long pstride = (long long)NV * G * 4;
   DHS_TRY(bget(t, t->b_nbm, nwords * 4, s));
@@ -350,8 +376,9 @@ dhs_status ensure_ws(dhs_table* t, long long n, cudaStream_t s) {
   DHS_TRY(bget(t, t->b_va, cap * 4, s));
   DHS_TRY(bget(t, t->b_kb, cap * 4, s));
   DHS_TRY(bget(t, t->b_vb, cap * 4, s));
-  DHS_TRY(bget(t, t->b_hist, (size_t)kRadixBins * ntiles * 4, s));
-  DHS_TRY(bget(t, t->b_totals, kRadixBins * 4, s));
+  // digit histograms of every pass + one tile counter per pass; look-back state
+  DHS_TRY(bget(t, t->b_hist, (size_t)(kRadixMaxPasses * kRadixBins + kRadixMaxPasses) * 4, s));
+  DHS_TRY(bget(t, t->b_totals, (size_t)kRadixMaxPasses * ntiles * kRadixBins * 8, s));
   DHS_TRY(bget(t, t->b_ph, (size_t)nchunks * pstride * 8, s));
   DHS_TRY(bget(t, t->b_pt, (size_t)nchunks * pstride * 8, s));
   DHS_TRY(bget(t, t->b_cflags, nchunks, s));
@@ -377,9 +404,13 @@ dhs_status dispatch_pool(dhs_table* t, const long long* keys, long long n, const
 dhs_status dispatch_seg(dhs_table* t, const unsigned* sk, const unsigned* sv, long long n,
                         const float* grad, long long nb, const OptArgs& oa, cudaStream_t s) {
   const int G = pick_group(t->dim), NV = pick_nv(t->dim, G);
-  const cudaError_t e = launch_seg(G, NV, t->sm_count, sk, sv, n, grad, nb, t->dim, rowspace(t), oa,
-                                   (double*)t->b_ph.p, (double*)t->b_pt.p,
-                                   (unsigned char*)t->b_cflags.p, kSegChunk, t->st, s);
+  auto fn = t->opt == DHS_SGD ? launch_seg_sgd
+            : t->opt == DHS_ADAGRAD ? launch_seg_adagrad
+            : t->opt == DHS_ADAM ? launch_seg_adam
+                                 : launch_seg_rowwise;
+  const cudaError_t e = fn(G, NV, t->sm_count, sk, sv, n, grad, nb, t->dim, rowspace(t), oa,
+                           (double*)t->b_ph.p, (double*)t->b_pt.p, (unsigned char*)t->b_cflags.p,
+                           seg_chunk(n), t->st, s);
   t->n_launches++;
   if (e != cudaSuccess) cudaGetLastError();
   return e == cudaSuccess ? DHS_OK : DHS_ERR_CUDA;
@@ -388,13 +419,13 @@ dhs_status dispatch_seg(dhs_table* t, const unsigned* sk, const unsigned* sv, lo
 // offset assignment + row init for the new keys of an insert call
 dhs_status launch_assign(dhs_table* t, long long n, cudaStream_t s) {
   const long long nwords = (n + 31) / 32;
-  const long long ngroups = (n + 1023) / 1024;
-  fwd_mark_kernel<<<(unsigned)((nwords + 255) / 256), 256, 0, s>>>(
+  const long long ngroups = (n + kGroupPositions - 1) / kGroupPositions;
+  fwd_mark_kernel<<<(unsigned)ngroups, kGroupThreads, 0, s>>>(
       t->slots, (unsigned*)t->b_nbm.p, (unsigned*)t->b_fbm.p, (unsigned*)t->b_gcnt.p,
       (unsigned*)t->b_gpref.p, (const unsigned*)t->b_slotpos.p, nwords, ngroups, t->st);
   t->n_launches += 2;
   DHS_TRY(last_launch());
-  fwd_assign_kernel<<<(unsigned)((ngroups + kAssignWarps - 1) / kAssignWarps), kAssignWarps * 32, 0, s>>>(
+  fwd_assign_kernel<<<(unsigned)ngroups, kGroupThreads, 0, s>>>(
       t->slots, rowspace(t), t->dim, (const unsigned*)t->b_fbm.p, (const unsigned*)t->b_gpref.p,
       (const unsigned*)t->b_slotpos.p, nwords, ngroups, t->st);
   return last_launch();
@@ -423,6 +454,7 @@ const char* dhs_status_str(dhs_status s) {
     case DHS_ERR_TABLE_FULL: return "table full";
     case DHS_ERR_NOT_FOUND: return "key not found";
     case DHS_ERR_UNSUPPORTED: return "unsupported";
+    case DHS_ERR_INTERNAL: return "internal wait bound exceeded";
   }
   return "unknown status";
 }
@@ -482,6 +514,19 @@ dhs_status ht_create(int32_t dim, dhs_optimizer opt, int64_t block_rows, int64_t
   }
   cudaStream_t s = nullptr;
   dhs_status rc = DHS_OK;
+  if (!t->custom_alloc) {
+    cudaMemPoolProps props{};
+    props.allocType = cudaMemAllocationTypePinned;
+    props.location.type = cudaMemLocationTypeDevice;
+    props.location.id = t->device;
+    if (cudaMemPoolCreate(&t->pool, &props) != cudaSuccess) {
+      cudaGetLastError();
+      delete t;
+      return DHS_ERR_CUDA;
+    }
+    unsigned long long keep = ~0ull;  // never hand freed memory back to the driver
+    cudaMemPoolSetAttribute(t->pool, cudaMemPoolAttrReleaseThreshold, &keep);
+  }
   t->st = (DevState*)dalloc(t, sizeof(DevState), s);
   t->blocks_d = (float**)dalloc(t, sizeof(float*) * t->max_blocks, s);
   if (!t->st || !t->blocks_d) rc = DHS_ERR_OOM;
@@ -525,6 +570,7 @@ dhs_status ht_destroy(dhs_table* t) {
     if (sn.ev) cudaEventDestroy(sn.ev);
     if (sn.pinned) cudaFreeHost(sn.pinned);
   }
+  if (t->pool) cudaMemPoolDestroy(t->pool);
   for (auto& r : t->recs) {
     cudaEventDestroy(r.a);
     cudaEventDestroy(r.b);
@@ -543,6 +589,17 @@ dhs_status ht_reserve(dhs_table* t, int64_t n_keys, dhs_stream stream) {
   t->last_stream = s;
   if ((double)n_keys > kMaxLoad * (double)t->nslots)
     DHS_TRY(grow_map(t, (unsigned long long)std::ceil((double)n_keys / kMaxLoad), s));
+  const long long rows = std::min<long long>(n_keys, t->max_rows);
+  while ((long long)t->blocks_h.size() * t->block_rows < rows) {
+    const size_t bytes = (size_t)t->block_rows * t->stride * sizeof(float);
+    float* b = (float*)dalloc(t, bytes, s);
+    if (!b) return DHS_ERR_OOM;
+    t->blocks_h.push_back(b);
+    set_block_kernel<<<1, 1, 0, s>>>(t->blocks_d, (long long)t->blocks_h.size() - 1, b, t->st,
+                                     (unsigned long long)t->blocks_h.size());
+    t->n_launches++;
+    DHS_TRY(last_launch());
+  }
   return DHS_OK;
 }
 
@@ -642,7 +699,7 @@ dhs_status embbag_backward_update(dhs_table* t, const int64_t* d_keys, int64_t n
   const unsigned sentinel = (unsigned)t->rows_ub;
   int bits = 0;
   while (bits < 32 && (1ull << bits) <= (unsigned long long)sentinel) ++bits;
-  const int passes = std::max(1, (bits + 7) / 8);
+  const int passes = std::min(kRadixMaxPasses, std::max(1, (bits + 7) / 8));
 
   unsigned* ka = (unsigned*)t->b_ka.p;
   unsigned* va = (unsigned*)t->b_va.p;
@@ -656,23 +713,29 @@ dhs_status embbag_backward_update(dhs_table* t, const int64_t* d_keys, int64_t n
     const long long grid = grid_for((warps + 7) / 8, resident);
     bwd_probe_kernel<<<(unsigned)grid, 256, 0, s>>>(idmap(t), (const long long*)d_keys, n_keys,
                                                     (const long long*)d_bag_offsets, n_bags, ka, va,
-                                                    sentinel, t->st);
+                                                    sentinel, (unsigned*)t->b_hist.p,
+                                                    kRadixMaxPasses * kRadixBins + kRadixMaxPasses,
+                                                    t->st);
     t->n_launches++;
     DHS_TRY(last_launch());
   }
   {
     PhaseScope ph(t, PH_BWD_SORT, s);
     const long long ntiles = (n_keys + kRadixTile - 1) / kRadixTile;
+    unsigned* hist = (unsigned*)t->b_hist.p;
+    unsigned* tile_ctr = hist + kRadixMaxPasses * kRadixBins;
+    unsigned long long* status = (unsigned long long*)t->b_totals.p;
+    const long long hgrid = std::min<long long>((n_keys + kRadixThreads - 1) / kRadixThreads,
+                                                (long long)t->sm_count * 8);
+    radix_hist_all_kernel<<<(unsigned)hgrid, kRadixThreads, 0, s>>>(
+        ka, n_keys, passes, hist, status, (long long)passes * ntiles * kRadixBins);
+    t->n_launches++;
+    DHS_TRY(last_launch());
     for (int p = 0; p < passes; ++p) {
-      const int shift = 8 * p;
-      radix_hist_kernel<<<(unsigned)ntiles, kRadixThreads, 0, s>>>(ka, n_keys, shift,
-                                                                   (unsigned*)t->b_hist.p, ntiles);
-      radix_scan_kernel<<<kRadixBins, 256, 0, s>>>((unsigned*)t->b_hist.p, ntiles,
-                                                   (unsigned*)t->b_totals.p);
-      radix_scatter_kernel<<<(unsigned)ntiles, kRadixThreads, 0, s>>>(
-          ka, va, kb, vb, n_keys, shift, (const unsigned*)t->b_hist.p,
-          (const unsigned*)t->b_totals.p, ntiles);
-      t->n_launches += 3;
+      radix_onesweep_kernel<<<(unsigned)ntiles, kRadixThreads, 0, s>>>(
+          ka, va, kb, vb, n_keys, 8 * p, hist + p * kRadixBins, status + (long long)p * ntiles * kRadixBins,
+          tile_ctr + p, t->st);
+      t->n_launches++;
       DHS_TRY(last_launch());
       std::swap(ka, kb);
       std::swap(va, vb);
@@ -693,12 +756,13 @@ dhs_status embbag_backward_update(dhs_table* t, const int64_t* d_keys, int64_t n
     DHS_TRY(dispatch_seg(t, ka, va, n_keys, d_grad, n_bags, oa, s));
     const int G = pick_group(t->dim), NV = pick_nv(t->dim, G);
     const int pstride = NV * G * 4;
-    const long long nchunks = (n_keys + kSegChunk - 1) / kSegChunk;
+    const int chunk = seg_chunk(n_keys);
+    const long long nchunks = (n_keys + chunk - 1) / chunk;
     const size_t smem = (size_t)std::max(256, t->dim) * sizeof(double);
     const long long grid = std::min<long long>(nchunks, (long long)t->sm_count * 8);
     bwd_combine_kernel<<<(unsigned)grid, 256, smem, s>>>(ka, n_keys, t->dim, rowspace(t), oa,
                                                         (const double*)t->b_ph.p, (const double*)t->b_pt.p,
-                                                        (const unsigned char*)t->b_cflags.p, kSegChunk,
+                                                        (const unsigned char*)t->b_cflags.p, chunk,
                                                         pstride, t->st);
     t->n_launches++;
     DHS_TRY(last_launch());
@@ -749,7 +813,7 @@ dhs_status ht_size(dhs_table* t, int64_t* n_rows) {
   return rc;
 }
 
-dhs_status ht_counters(dhs_table* t, int64_t out[10]) {
+dhs_status ht_counters(dhs_table* t, int64_t out[14]) {
   DHS_TRY(check_table(t));
   if (!out) return DHS_ERR_INVALID_ARG;
   DeviceGuard g(t->device);
@@ -767,6 +831,10 @@ dhs_status ht_counters(dhs_table* t, int64_t out[10]) {
   out[7] = t->n_rehash;
   out[8] = t->n_launches;
   out[9] = (int64_t)h.m_last;
+  out[10] = t->n_host_waits;
+  out[11] = t->host_wait_ns;
+  out[12] = t->n_allocs;
+  out[13] = t->alloc_ns;
   return DHS_OK;
 }
 

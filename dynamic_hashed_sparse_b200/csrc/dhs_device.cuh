@@ -42,7 +42,7 @@ struct DevState {
   unsigned int pad;
 };
 
-enum : unsigned { kErrInvalid = 1u, kErrFull = 4u, kErrNotFound = 5u };
+enum : unsigned { kErrInvalid = 1u, kErrFull = 4u, kErrNotFound = 5u, kErrInternal = 7u };
 
 __device__ __forceinline__ void latch(DevState* st, unsigned code) {
   if (*(volatile unsigned*)&st->err == 0u) atomicCAS(&st->err, 0u, code);
@@ -158,6 +158,13 @@ __device__ __forceinline__ long long probe_find(IdMap m, unsigned long long key)
     w = (w + 1) & m.win_mask;
   }
   return -1;
+}
+
+// Bulk prefetch of `bytes` (a multiple of 16, 16-byte aligned) into L2: one
+// instruction per row, no register or shared-memory cost, so a warp can put a
+// whole window of upcoming rows in flight.
+__device__ __forceinline__ void prefetch_l2(const void* p, unsigned bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
 }
 
 __device__ __forceinline__ float4 f4add(float4 a, float4 b) {

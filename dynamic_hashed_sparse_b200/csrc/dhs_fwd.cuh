@@ -13,6 +13,8 @@
 // key stream.
 #pragma once
 
+#include <climits>
+
 #include "dhs_device.cuh"
 
 namespace dhs {
@@ -57,13 +59,13 @@ __device__ __forceinline__ long long load_bag_ends(const long long* __restrict__
 
 // Fused lookup-or-insert + gather + sum pooling.  A group of G lanes owns a
 // chunk of G consecutive bags; it probes the chunk's ids G at a time (one id
-// per lane), then walks those ids in order, each lane loading NV float4
-// columns of the row (16-byte vector loads), U rows in flight, and adds them
-// into the current bag's accumulator.  A new key's row is not read: its
-// initial value is computed from the key, exactly as the assignment kernel
-// will store it.
+// per lane; the probing lane also forms the row address), then walks those ids
+// in order, each lane loading NV float4 columns of the row (16-byte vector
+// loads), U rows in flight, and adds them into the current bag's accumulator.
+// A new key's row is not read: its initial value is computed from the key,
+// exactly as the assignment kernel will store it.
 template <int G, int NV>
-__global__ void __launch_bounds__(kFwdThreads)
+__global__ void __launch_bounds__(kFwdThreads, NV == 1 ? 4 : (NV == 2 ? 2 : 1))
 fwd_probe_pool_kernel(IdMap m, RowSpace rs, int dim, const long long* __restrict__ keys,
                       long long n_keys, const long long* __restrict__ bag_off, long long n_bags,
                       float* __restrict__ out, unsigned* __restrict__ nbm,
@@ -73,37 +75,49 @@ fwd_probe_pool_kernel(IdMap m, RowSpace rs, int dim, const long long* __restrict
   const int gl = lane & (G - 1);
   const int gw = lane / G;
   const unsigned gmask = (G == 32) ? 0xffffffffu : (((1u << G) - 1u) << (gw * G));
-  const long long gid = ((long long)blockIdx.x * kFwdThreads + threadIdx.x) / G;
-  const long long ngroups = ((long long)gridDim.x * kFwdThreads) / G;
-  const long long nchunks = (n_bags + G - 1) / G;
+  const int gid = (int)((blockIdx.x * kFwdThreads + threadIdx.x) / G);
+  const int ngroups = (int)((gridDim.x * kFwdThreads) / G);
+  // bags and positions fit in 31 bits (the host rejects larger calls)
+  const int nchunks = (int)((n_bags + G - 1) / G);
   const int d4 = dim >> 2;
 
-  for (long long c = gid; c < nchunks; c += ngroups) {
-    const long long b0 = c * G;
+  for (int c = gid; c < nchunks; c += ngroups) {
+    const long long b0 = (long long)c * G;
     const int nb = (int)min((long long)G, n_bags - b0);
-    long long s;
-    const long long e = load_bag_ends<G>(bag_off, b0, nb, n_keys, n_bags, s, gmask, gl, st);
-    const long long E = __shfl_sync(gmask, e, nb - 1, G);
+    long long s64;
+    const long long e64 = load_bag_ends<G>(bag_off, b0, nb, n_keys, n_bags, s64, gmask, gl, st);
+    const int e = e64 == LLONG_MAX ? INT_MAX : (int)e64;
+    const int s = (int)s64;
+    const int E = __shfl_sync(gmask, e, nb - 1, G);
     int cur = 0;
-    long long cur_end = __shfl_sync(gmask, e, 0, G);
+    int cur_end = __shfl_sync(gmask, e, 0, G);
     float4 acc[NV];
 #pragma unroll
     for (int q = 0; q < NV; ++q) acc[q] = make_float4(0.f, 0.f, 0.f, 0.f);
+    float* outb = out + b0 * (long long)dim;
 
-    for (long long ws = s; ws < E; ws += G) {
-      const int cnt = (int)min((long long)G, E - ws);
+    for (int ws = s; ws < E; ws += G) {
+      const int cnt = min(G, E - ws);
       // ---- probe: one id per lane ----
+      // ref: the row address of a hit, or the key itself for a new key
       int kind = kBad;
-      unsigned long long ref = 0, key = 0;
+      unsigned long long ref = 0;
       if (gl < cnt) {
-        const long long p = ws + gl;
+        const int p = ws + gl;
         const long long k = __ldg(keys + p);
-        key = (unsigned long long)k;
         if (k < 0) {
           latch(st, kErrInvalid);
         } else {
-          kind = probe_claim(m, key, (unsigned)p, ref, st);
-          if (kind == kNew) slotpos[p] = (unsigned)ref;
+          unsigned long long r;
+          kind = probe_claim(m, (unsigned long long)k, (unsigned)p, r, st);
+          if (kind == kHit) {
+            const float* rowp = rs.row(r);
+            ref = (unsigned long long)rowp;
+            prefetch_l2(rowp, (unsigned)dim * 4u);  // all G rows of the window in flight
+          } else if (kind == kNew) {
+            slotpos[p] = (unsigned)r;
+            ref = (unsigned long long)k;
+          }
         }
       }
       // mark the positions that carry a key new in this call (<= 2 words per window)
@@ -111,8 +125,8 @@ fwd_probe_pool_kernel(IdMap m, RowSpace rs, int dim, const long long* __restrict
         const unsigned bal = __ballot_sync(gmask, kind == kNew);
         const unsigned mine = (G == 32) ? bal : ((bal >> (gw * G)) & ((1u << G) - 1u));
         if (gl == 0 && mine) {
-          const unsigned long long p0 = (unsigned long long)ws;
-          const unsigned sh = (unsigned)(p0 & 31);
+          const unsigned p0 = (unsigned)ws;
+          const unsigned sh = p0 & 31u;
           atomicOr(&nbm[p0 >> 5], mine << sh);
           if (sh && (sh + G > 32)) {
             const unsigned hi = mine >> (32 - sh);
@@ -129,17 +143,15 @@ fwd_probe_pool_kernel(IdMap m, RowSpace rs, int dim, const long long* __restrict
           const int src = t & (G - 1);
           const int kt = __shfl_sync(gmask, kind, src, G);
           const unsigned long long rt = __shfl_sync(gmask, ref, src, G);
-          const unsigned long long keyt = __shfl_sync(gmask, key, src, G);
-          const float* rowp = (t < cnt && kt == kHit) ? rs.row(rt) : nullptr;
 #pragma unroll
           for (int q = 0; q < NV; ++q) {
             const int c4 = gl + q * G;
             float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
             if (t < cnt && c4 < d4) {
               if (kt == kHit)
-                x = __ldg(reinterpret_cast<const float4*>(rowp) + c4);
+                x = __ldg(reinterpret_cast<const float4*>(rt) + c4);
               else if (kt == kNew)
-                x = init_weight4(keyt, c4 * 4);
+                x = init_weight4(rt, c4 * 4);
             }
             v[u][q] = x;
           }
@@ -148,9 +160,9 @@ fwd_probe_pool_kernel(IdMap m, RowSpace rs, int dim, const long long* __restrict
         for (int u = 0; u < U; ++u) {
           const int t = t0 + u;
           if (t < cnt) {
-            const long long pos = ws + t;
+            const int pos = ws + t;
             while (pos >= cur_end) {
-              float4* o = reinterpret_cast<float4*>(out + (b0 + cur) * (long long)dim);
+              float4* o = reinterpret_cast<float4*>(outb + (long long)cur * dim);
 #pragma unroll
               for (int q = 0; q < NV; ++q) {
                 const int c4 = gl + q * G;
@@ -168,7 +180,7 @@ fwd_probe_pool_kernel(IdMap m, RowSpace rs, int dim, const long long* __restrict
     }
     // the bag in progress and any empty bags after it
     while (cur < nb) {
-      float4* o = reinterpret_cast<float4*>(out + (b0 + cur) * (long long)dim);
+      float4* o = reinterpret_cast<float4*>(outb + (long long)cur * dim);
 #pragma unroll
       for (int q = 0; q < NV; ++q) {
         const int c4 = gl + q * G;
@@ -222,38 +234,64 @@ __global__ void fwd_fixup_kernel(const Slot* __restrict__ slots, long long* __re
   }
 }
 
-// First-occurrence marking.  Thread per bitmap word (32 positions), warp per
-// group of 1024 positions.  A new position is a first occurrence iff its
-// slot holds PENDING | that position.  Writes the first-occurrence word,
-// clears the new-position word for the next call, and writes the group's
-// count.  The last block to finish scans the group counts, reserves the new
-// rows (row_base = row_count, row_count += M) and resets the ticket.
-__global__ void __launch_bounds__(256)
+// First-occurrence marking.  Block of 1024 threads per group of 4096 batch
+// positions (128 bitmap words), four positions per thread so that each thread
+// has four independent load chains in flight.  A position that carries a key
+// new in this call is its key's first occurrence iff the key's slot holds
+// PENDING | that position.  Writes the first-occurrence bitmap words, clears
+// the new-position words for the next call, and writes the group's count.
+// The last block to finish scans the group counts, reserves the new rows
+// (row_base = row_count, row_count += M) and resets the ticket.
+constexpr int kGroupThreads = 1024;
+constexpr int kGroupPerThread = 4;
+constexpr int kGroupPositions = kGroupThreads * kGroupPerThread;  // 4096
+constexpr int kGroupWords = kGroupPositions / 32;                  // 128
+
+__global__ void __launch_bounds__(kGroupThreads)
 fwd_mark_kernel(const Slot* __restrict__ slots, unsigned* __restrict__ nbm,
                 unsigned* __restrict__ fbm, unsigned* __restrict__ gcnt,
                 unsigned* __restrict__ gpref, const unsigned* __restrict__ slotpos,
                 long long nwords, long long ngroups, DevState* st) {
-  const long long w = (long long)blockIdx.x * 256 + threadIdx.x;
-  unsigned word = 0;
-  if (w < nwords) {
-    word = nbm[w];
-    if (word) nbm[w] = 0u;
-  }
-  unsigned fw = 0;
-  while (word) {
-    const int b = __ffs(word) - 1;
-    word &= word - 1;
-    const unsigned long long p = (unsigned long long)(w * 32 + b);
-    const unsigned s = slotpos[p];
-    const unsigned long long v = __ldcg(&slots[s].val);
-    if ((v & ~kPending) == p) fw |= 1u << b;
-  }
-  if (w < nwords) fbm[w] = fw;
-  const unsigned c = warp_sum_u32(__popc(fw));
-  const long long g = w >> 5;
-  if ((threadIdx.x & 31) == 0 && g < ngroups) gcnt[g] = c;
-
+  __shared__ unsigned wsum[32];
   __shared__ bool is_last;
+  __shared__ unsigned long long carry_s;
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  const long long g = blockIdx.x;
+  unsigned word[kGroupPerThread];
+  unsigned s[kGroupPerThread];
+  unsigned long long v[kGroupPerThread];
+#pragma unroll
+  for (int k = 0; k < kGroupPerThread; ++k) {
+    const long long w = g * kGroupWords + k * 32 + wid;
+    word[k] = w < nwords ? nbm[w] : 0u;
+  }
+#pragma unroll
+  for (int k = 0; k < kGroupPerThread; ++k) {
+    const unsigned long long p = (unsigned long long)(g * kGroupPositions + k * kGroupThreads + threadIdx.x);
+    s[k] = ((word[k] >> lane) & 1u) ? slotpos[p] : 0u;
+  }
+#pragma unroll
+  for (int k = 0; k < kGroupPerThread; ++k)
+    v[k] = ((word[k] >> lane) & 1u) ? __ldcg(&slots[s[k]].val) : 0ull;
+  unsigned cnt = 0;
+#pragma unroll
+  for (int k = 0; k < kGroupPerThread; ++k) {
+    const long long w = g * kGroupWords + k * 32 + wid;
+    const unsigned long long p = (unsigned long long)(g * kGroupPositions + k * kGroupThreads + threadIdx.x);
+    const bool first = ((word[k] >> lane) & 1u) && (v[k] & ~kPending) == p;
+    const unsigned fw = __ballot_sync(0xffffffffu, first);
+    if (lane == 0 && w < nwords) {
+      fbm[w] = fw;
+      if (word[k]) nbm[w] = 0u;
+    }
+    cnt += __popc(fw);
+  }
+  if (lane == 0) wsum[wid] = cnt;
+  __syncthreads();
+  if (wid == 0) {
+    const unsigned c = warp_sum_u32(wsum[lane]);
+    if (lane == 0) gcnt[g] = c;
+  }
   __threadfence();
   __syncthreads();
   if (threadIdx.x == 0) is_last = (atomicAdd(&st->ticket, 1u) == gridDim.x - 1);
@@ -261,13 +299,10 @@ fwd_mark_kernel(const Slot* __restrict__ slots, unsigned* __restrict__ nbm,
   if (!is_last) return;
   __threadfence();
 
-  // exclusive scan of gcnt[0, ngroups) by this block, 256 entries per pass
-  __shared__ unsigned wsum[8];
-  __shared__ unsigned long long carry_s;
+  // exclusive scan of gcnt[0, ngroups) by this block, 1024 entries per pass
   if (threadIdx.x == 0) carry_s = 0;
   __syncthreads();
-  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-  for (long long base = 0; base < ngroups; base += 256) {
+  for (long long base = 0; base < ngroups; base += kGroupThreads) {
     const long long i = base + threadIdx.x;
     const unsigned x = (i < ngroups) ? __ldcg(gcnt + i) : 0u;
     unsigned inc = x;
@@ -278,16 +313,21 @@ fwd_mark_kernel(const Slot* __restrict__ slots, unsigned* __restrict__ nbm,
     }
     if (lane == 31) wsum[wid] = inc;
     __syncthreads();
-    unsigned wpre = 0, tot = 0;
+    if (wid == 0) {
+      const unsigned vv = wsum[lane];
+      unsigned vi = vv;
 #pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      if (k < wid) wpre += wsum[k];
-      tot += wsum[k];
+      for (int o = 1; o < 32; o <<= 1) {
+        const unsigned y = __shfl_up_sync(0xffffffffu, vi, o);
+        if (lane >= o) vi += y;
+      }
+      wsum[lane] = vi - vv;  // exclusive prefix of the warp sums
     }
-    const unsigned long long carry = carry_s;
-    if (i < ngroups) gpref[i] = (unsigned)(carry + wpre + inc - x);
     __syncthreads();
-    if (threadIdx.x == 0) carry_s = carry + tot;
+    const unsigned long long carry = carry_s;
+    if (i < ngroups) gpref[i] = (unsigned)(carry + wsum[wid] + inc - x);
+    __syncthreads();
+    if (threadIdx.x == kGroupThreads - 1) carry_s = carry + wsum[wid] + inc;
     __syncthreads();
   }
   if (threadIdx.x == 0) {
@@ -302,60 +342,79 @@ fwd_mark_kernel(const Slot* __restrict__ slots, unsigned* __restrict__ nbm,
   }
 }
 
-// Offset assignment + row initialisation.  Warp per group of 1024 positions:
-// the group's new keys have consecutive ranks, so their rows are one
-// contiguous run (split only at a block edge).  Each new key's slot gets its
-// row offset; the run is then written with coalesced 16-byte stores (initial
-// weights from splitmix64(key), optimizer state zero).
-constexpr int kAssignWarps = 4;
-
-__global__ void __launch_bounds__(kAssignWarps * 32)
+// Offset assignment + row initialisation.  Block of 1024 threads per group of
+// 4096 positions, four per thread: the group's new keys have consecutive
+// ranks (the prefix over the group's 128 bitmap words plus the bit's place in
+// its word), so their rows are one contiguous run (split only at a block
+// edge).  Each first occurrence writes its key's row offset into the slot; the
+// block then writes the run with coalesced 16-byte stores (initial weights
+// from splitmix64(key), optimizer state zero).
+__global__ void __launch_bounds__(kGroupThreads)
 fwd_assign_kernel(Slot* __restrict__ slots, RowSpace rs, int dim,
                   const unsigned* __restrict__ fbm, const unsigned* __restrict__ gpref,
                   const unsigned* __restrict__ slotpos, long long nwords, long long ngroups,
                   DevState* st) {
-  __shared__ unsigned long long skey[kAssignWarps][1024];
+  __shared__ unsigned long long skey[kGroupPositions];  // 32 KB
+  __shared__ unsigned wpre[kGroupWords];
+  __shared__ unsigned s_total;
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-  const long long g = (long long)blockIdx.x * kAssignWarps + wid;
-  if (g >= ngroups) return;
-  const long long w = g * 32 + lane;
-  unsigned fw = (w < nwords) ? fbm[w] : 0u;
-  const unsigned c = __popc(fw);
-  unsigned inc = c;
+  const long long g = blockIdx.x;
+  if (threadIdx.x < 32) {
+    // exclusive prefix of the 128 words' counts (4 per lane, in word order)
+    unsigned c[4], t = 0;
 #pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const unsigned y = __shfl_up_sync(0xffffffffu, inc, o);
-    if (lane >= o) inc += y;
+    for (int k = 0; k < 4; ++k) {
+      const long long w = g * kGroupWords + lane * 4 + k;
+      c[k] = w < nwords ? __popc(fbm[w]) : 0u;
+      t += c[k];
+    }
+    unsigned inc = t;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const unsigned y = __shfl_up_sync(0xffffffffu, inc, o);
+      if (lane >= o) inc += y;
+    }
+    unsigned run = inc - t;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      wpre[lane * 4 + k] = run;
+      run += c[k];
+    }
+    if (lane == 31) s_total = inc;
   }
-  const unsigned total = __shfl_sync(0xffffffffu, inc, 31);
+  __syncthreads();
+  const unsigned total = s_total;
   if (total == 0) return;
   const unsigned long long row0 = st->row_base + gpref[g];
   const unsigned long long limit = st->n_blocks << rs.log2_br;
-  unsigned j = inc - c;
-  while (fw) {
-    const int b = __ffs(fw) - 1;
-    fw &= fw - 1;
-    const unsigned long long p = (unsigned long long)(w * 32 + b);
-    const unsigned s = slotpos[p];
-    const unsigned long long row = row0 + j;
-    skey[wid][j] = slots[s].key;
-    if (row < limit) {
-      slots[s].val = row;
-    } else {
-      latch(st, kErrFull);
-      slots[s].val = kPending;  // unusable; the table is reported full
+#pragma unroll
+  for (int k = 0; k < kGroupPerThread; ++k) {
+    const int wi = k * 32 + wid;
+    const long long w = g * kGroupWords + wi;
+    const unsigned fw = w < nwords ? fbm[w] : 0u;
+    if ((fw >> lane) & 1u) {
+      const unsigned j = wpre[wi] + __popc(fw & lanemask_lt());
+      const unsigned long long p = (unsigned long long)(g * kGroupPositions + k * kGroupThreads + threadIdx.x);
+      const unsigned sl = slotpos[p];
+      const unsigned long long row = row0 + j;
+      skey[j] = slots[sl].key;
+      if (row < limit) {
+        slots[sl].val = row;
+      } else {
+        latch(st, kErrFull);
+        slots[sl].val = kPending;  // unusable; the table is reported full
+      }
     }
-    ++j;
   }
-  __syncwarp();
+  __syncthreads();
   const int s4 = rs.stride >> 2, d4 = dim >> 2;
-  const long long work = (long long)total * s4;
-  for (long long idx = lane; idx < work; idx += 32) {
-    const unsigned r = (unsigned)(idx / s4);
-    const int c4 = (int)(idx - (long long)r * s4);
+  const int work = (int)total * s4;
+  for (int idx = threadIdx.x; idx < work; idx += kGroupThreads) {
+    const int r = idx / s4;
+    const int c4 = idx - r * s4;
     const unsigned long long row = row0 + r;
     if (row >= limit) continue;
-    const float4 x = (c4 < d4) ? init_weight4(skey[wid][r], c4 * 4) : make_float4(0.f, 0.f, 0.f, 0.f);
+    const float4 x = (c4 < d4) ? init_weight4(skey[r], c4 * 4) : make_float4(0.f, 0.f, 0.f, 0.f);
     reinterpret_cast<float4*>(rs.row(row))[c4] = x;
   }
 }

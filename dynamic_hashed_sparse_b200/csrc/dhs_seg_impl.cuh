@@ -1,0 +1,71 @@
+// Launcher of bwd_seg_kernel<G, NV, OPT> for one optimizer; included by one
+// translation unit per optimizer so that they compile in parallel.
+#pragma once
+
+#include <algorithm>
+
+#define DHS_TEMPLATES_ONLY
+#include "dhs_bwd.cuh"
+#include "dhs_launch.h"
+
+namespace dhs {
+namespace seg_impl {
+
+template <int G, int NV, int OPT>
+cudaError_t run(int sm_count, const unsigned* skey, const unsigned* sval, long long n,
+                const float* grad, long long n_bags, int dim, RowSpace rs, const OptArgs& oa,
+                double* part_head, double* part_tail, unsigned char* cflags, int chunk,
+                DevState* st, cudaStream_t s) {
+  static int resident = 0;
+  if (!resident) {
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, bwd_seg_kernel<G, NV, OPT>, 256, 0) !=
+            cudaSuccess || per_sm < 1) {
+      cudaGetLastError();
+      per_sm = 1;
+    }
+    resident = per_sm * sm_count;
+  }
+  const long long nchunks = (n + chunk - 1) / chunk;
+  const long long per_block = 256 / G;
+  const long long need = std::max<long long>(1, (nchunks + per_block - 1) / per_block);
+  const long long grid = std::min<long long>(need, resident);
+  bwd_seg_kernel<G, NV, OPT><<<(unsigned)grid, 256, 0, s>>>(skey, sval, n, grad, n_bags, dim, rs, oa,
+                                                           part_head, part_tail, cflags, chunk, st);
+  return cudaGetLastError();
+}
+
+template <int OPT>
+cudaError_t launch(int G, int NV, int sm_count, const unsigned* skey, const unsigned* sval,
+                   long long n, const float* grad, long long n_bags, int dim, RowSpace rs,
+                   const OptArgs& oa, double* part_head, double* part_tail, unsigned char* cflags,
+                   int chunk, DevState* st, cudaStream_t s) {
+#define DHS_RUN(g, v) \
+  run<g, v, OPT>(sm_count, skey, sval, n, grad, n_bags, dim, rs, oa, part_head, part_tail, cflags, chunk, st, s)
+  switch (G * 100 + NV) {
+    case 101: return DHS_RUN(1, 1);
+    case 201: return DHS_RUN(2, 1);
+    case 401: return DHS_RUN(4, 1);
+    case 801: return DHS_RUN(8, 1);
+    case 1601: return DHS_RUN(16, 1);
+    case 3201: return DHS_RUN(32, 1);
+    case 3202: return DHS_RUN(32, 2);
+    case 3204: return DHS_RUN(32, 4);
+  }
+#undef DHS_RUN
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace seg_impl
+}  // namespace dhs
+
+#define DHS_SEG_TU(OPT_, NAME_)                                                                  \
+  namespace dhs {                                                                                \
+  cudaError_t NAME_(int G, int NV, int sm_count, const unsigned* skey, const unsigned* sval,     \
+                    long long n, const float* grad, long long n_bags, int dim, RowSpace rs,      \
+                    const OptArgs& oa, double* part_head, double* part_tail,                     \
+                    unsigned char* cflags, int chunk, DevState* st, cudaStream_t s) {            \
+    return seg_impl::launch<OPT_>(G, NV, sm_count, skey, sval, n, grad, n_bags, dim, rs, oa,     \
+                                  part_head, part_tail, cflags, chunk, st, s);                   \
+  }                                                                                              \
+  }

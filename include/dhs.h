@@ -69,7 +69,8 @@ typedef enum {
   DHS_ERR_CUDA = 3,        /* a CUDA runtime call failed */
   DHS_ERR_TABLE_FULL = 4,  /* row limit (max_rows) or IDMap probe bound reached */
   DHS_ERR_NOT_FOUND = 5,   /* backward saw a key that is not in the table */
-  DHS_ERR_UNSUPPORTED = 6  /* configuration this build does not handle */
+  DHS_ERR_UNSUPPORTED = 6, /* configuration this build does not handle */
+  DHS_ERR_INTERNAL = 7     /* a bounded device-side wait gave up (results undefined) */
 } dhs_status;
 
 typedef enum {
@@ -120,8 +121,11 @@ dhs_status ht_create(int32_t dim, dhs_optimizer opt, int64_t block_rows, int64_t
 /* Wait for the table's work and release everything it owns.  NULL is a no-op. */
 dhs_status ht_destroy(dhs_table* t);
 
-/* Grow the IDMap now so that it holds n_keys keys without rehashing (e.g.
- * before a large pre-population).  Rows are untouched. */
+/* Reserve capacity for n_keys keys now: the IDMap is grown so that it holds
+ * them without rehashing, and EmbeddingBlocks covering n_keys rows (at most
+ * max_rows) are appended.  No key or row is added; existing rows are
+ * untouched.  Lets a caller keep allocation and rehash work out of its
+ * training steps. */
 dhs_status ht_reserve(dhs_table* t, int64_t n_keys, dhs_stream stream);
 
 /* Lookup-or-insert ([RecIS] IDMap: id -> offset; [BG] row lookup).
@@ -190,8 +194,10 @@ dhs_status ht_export(dhs_table* t, int64_t* h_keys, float* h_rows);
  * distinct keys updated, out[3] forward-type calls, out[4] backward calls,
  * out[5] IDMap slots, out[6] blocks allocated, out[7] IDMap rehashes,
  * out[8] kernels launched by the table's calls, out[9] keys inserted by the
- * last insert call. */
-dhs_status ht_counters(dhs_table* t, int64_t out[10]);
+ * last insert call, out[10] / out[11] times / ns the host waited for the
+ * device inside table calls, out[12] / out[13] device allocations / ns spent
+ * in them. */
+dhs_status ht_counters(dhs_table* t, int64_t out[14]);
 
 /* Per-phase device time, measured with CUDA events recorded on the call's
  * stream around each phase while enabled.  Phases: 0 forward probe + pool,

@@ -201,6 +201,39 @@ def test_hot_key_spanning_many_sort_chunks(occ):
             o.close()
 
 
+@pytest.mark.parametrize("n_target", [20_000, 150_000, 700_000])
+def test_segment_runs_at_every_chunk_alignment(n_target):
+    """Rows with run lengths that put segment starts and ends at every offset
+    of the sort chunks (the chunk size depends on the batch size: 32, 64, 128),
+    including runs of exactly C, 2C, 3C and one longer or shorter."""
+    rng = np.random.default_rng(n_target)
+    dim = 16
+    special = []
+    for C in (32, 64, 128, 256):
+        special += [C - 1, C, C + 1, 2 * C - 1, 2 * C, 2 * C + 1, 3 * C - 1, 3 * C, 3 * C + 1]
+    lens = []
+    while sum(lens) < n_target:
+        lens += list(rng.permutation(special + list(range(1, 40))))
+    lens = np.array(lens, np.int64)
+    keys_by_row = np.arange(lens.size, dtype=np.int64) * 7 + 11
+    for opt in ("adagrad", "adam"):
+        t, o = make_pair(dim, opt)
+        try:
+            dhs.ht_lookup_or_insert(t, dev(keys_by_row))
+            o.lookup_or_insert(keys_by_row)
+            keys = rng.permutation(np.repeat(keys_by_row, lens))
+            nb = keys.size // 3
+            cuts = np.sort(rng.integers(0, keys.size, size=nb - 1))
+            offs = np.concatenate([[0], cuts, [keys.size]]).astype(np.int64)
+            grad = rng.standard_normal((nb, dim)).astype(np.float32)
+            step_both(t, o, dev(keys), keys, offs, grad, 0.01)
+            assert dhs.ht_sync(t) == 0
+            compare_tables(t, o, f"runs {n_target} {opt}")
+        finally:
+            t.close()
+            o.close()
+
+
 def test_empty_inputs_and_empty_bags():
     t, o = make_pair(16, "adam")
     try:
