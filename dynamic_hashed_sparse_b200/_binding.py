@@ -191,6 +191,8 @@ def embbag_forward(t: Table, keys: torch.Tensor, bag_offsets: torch.Tensor,
         _dev(out, torch.float32, "out")
         if out.numel() != nb * t.dim:
             raise ValueError("out must hold n_bags * dim floats")
+        if out.data_ptr() % 16:
+            raise ValueError("out must be 16-byte aligned")
     _check("embbag_forward", _lib.embbag_forward(t.handle, keys.data_ptr(), keys.numel(),
                                                  bag_offsets.data_ptr(), nb, out.data_ptr(),
                                                  _stream(stream)))
@@ -202,6 +204,8 @@ def embbag_backward_update(t: Table, keys: torch.Tensor, bag_offsets: torch.Tens
     _dev(keys, torch.int64, "keys")
     _dev(bag_offsets, torch.int64, "bag_offsets")
     _dev(grad, torch.float32, "grad")
+    if grad.data_ptr() % 16:
+        raise ValueError("grad must be 16-byte aligned")
     nb = bag_offsets.numel() - 1
     if grad.numel() != nb * t.dim:
         raise ValueError("grad must hold n_bags * dim floats")

@@ -14,6 +14,28 @@
 
 #include "dhs_device.cuh"
 
+// Tuning constants (compile-time; -D overrides them when sweeping):
+//   DHS_SEG_PREFETCH  1: the segment kernel prefetches into L2 the table row of
+//                     each segment that opens among the pairs in flight; 0: not
+//   DHS_RADIX_ITEMS   keys per thread in a radix-sort tile
+#ifndef DHS_SEG_PREFETCH
+#define DHS_SEG_PREFETCH 0
+#endif
+#ifndef DHS_RADIX_ITEMS
+#define DHS_RADIX_ITEMS 8
+#endif
+//   DHS_SEG_MINB      resident 256-thread blocks per SM the segment kernel is
+//                     compiled for (register budget) when a lane holds one
+//                     float4 column
+#ifndef DHS_SEG_MINB
+#define DHS_SEG_MINB 4
+#endif
+//   DHS_SEG_RING      gradient rows in flight per group (shared-memory ring)
+//                     for a row of <= 128 floats; wider rows use fewer
+#ifndef DHS_SEG_RING
+#define DHS_SEG_RING 8
+#endif
+
 namespace dhs {
 
 // ---------------------------------------------------------------------------
@@ -87,9 +109,9 @@ bwd_probe_kernel(IdMap m, const long long* __restrict__ keys, long long n_keys,
 // one kernel per digit pass (decoupled look-back across tiles)
 // ---------------------------------------------------------------------------
 constexpr int kRadixThreads = 256;
-constexpr int kRadixItems = 8;
-constexpr int kRadixWarpItems = 32 * kRadixItems;                     // 256
-constexpr int kRadixTile = kRadixWarpItems * (kRadixThreads / 32);    // 2048
+constexpr int kRadixItems = DHS_RADIX_ITEMS;
+constexpr int kRadixWarpItems = 32 * kRadixItems;
+constexpr int kRadixTile = kRadixWarpItems * (kRadixThreads / 32);
 constexpr int kRadixBins = 256;
 constexpr int kRadixMaxPasses = 4;
 constexpr unsigned long long kLbAggregate = 1ull << 62;  // tile count published
@@ -298,13 +320,41 @@ __device__ __forceinline__ void adam_step(float& w, float& m, float& v, float g,
   w = __fsub_rn(w, __fdiv_rn(__fmul_rn(o.lr, mhat), __fadd_rn(__fsqrt_rn(vhat), o.eps)));
 }
 
+// Scalar form for one column j (used by the combine kernel).
+__device__ __forceinline__ void update_col(float* row, int dim, int j, float g, const OptArgs& o,
+                                           float rowwise_den) {
+  float w = row[j];
+  if (o.opt == 0) {
+    w = sgd_w(w, g, o.lr);
+  } else if (o.opt == 1) {
+    float G = row[dim + j];
+    adagrad_step(w, G, g, o.lr, o.eps);
+    row[dim + j] = G;
+  } else if (o.opt == 2) {
+    float m = row[dim + j], v = row[2 * dim + j];
+    adam_step(w, m, v, g, o);
+    row[dim + j] = m;
+    row[2 * dim + j] = v;
+  } else {
+    w = __fsub_rn(w, __fdiv_rn(__fmul_rn(o.lr, g), rowwise_den));
+  }
+  row[j] = w;
+}
+
+// ---------------------------------------------------------------------------
+// segment reduce + update
+// ---------------------------------------------------------------------------
+enum : unsigned char { kPieceHead = 1, kPieceThrough = 2, kPieceTailStart = 4 };
+
 // The part of one row a lane owns: float4 columns gl + q*G (q < NV) of the
 // weights and of each per-element state array (Adagrad: G; Adam: m, v), plus
 // the row accumulator of row-wise Adagrad.  Loaded when a segment opens, so
 // the loads overlap the gradient sum; written back once when it closes.
+__host__ __device__ constexpr int seg_state_arrays(int opt) { return opt == 1 ? 1 : (opt == 2 ? 2 : 0); }
+
 template <int OPT, int NV>
 struct RowBuf {
-  static constexpr int NS = OPT == 1 ? 1 : (OPT == 2 ? 2 : 0);
+  static constexpr int NS = seg_state_arrays(OPT);
   float4 w[NV];
   float4 st[NS > 0 ? NS : 1][NV];
   float acc_row;
@@ -362,31 +412,22 @@ struct RowBuf {
   }
 };
 
-// Scalar form for one column j (used by the combine kernel).
-__device__ __forceinline__ void update_col(float* row, int dim, int j, float g, const OptArgs& o,
-                                           float rowwise_den) {
-  float w = row[j];
-  if (o.opt == 0) {
-    w = sgd_w(w, g, o.lr);
-  } else if (o.opt == 1) {
-    float G = row[dim + j];
-    adagrad_step(w, G, g, o.lr, o.eps);
-    row[dim + j] = G;
-  } else if (o.opt == 2) {
-    float m = row[dim + j], v = row[2 * dim + j];
-    adam_step(w, m, v, g, o);
-    row[dim + j] = m;
-    row[2 * dim + j] = v;
-  } else {
-    w = __fsub_rn(w, __fdiv_rn(__fmul_rn(o.lr, g), rowwise_den));
-  }
-  row[j] = w;
+// Gradient rows in flight per group (ring of shared-memory slots, filled by
+// cp.async): DHS_SEG_RING for a row of <= 128 floats, fewer for wider rows,
+// so that a 256-thread block uses the same shared memory at every width.
+__host__ __device__ constexpr int seg_ring(int nv) { return DHS_SEG_RING / nv > 0 ? DHS_SEG_RING / nv : 1; }
+__host__ __device__ constexpr size_t seg_smem_bytes(int G, int NV) {
+  return (size_t)(256 / G) * seg_ring(NV) * NV * G * 16;
 }
 
-// ---------------------------------------------------------------------------
-// segment reduce + update
-// ---------------------------------------------------------------------------
-enum : unsigned char { kPieceHead = 1, kPieceThrough = 2, kPieceTailStart = 4 };
+__device__ __forceinline__ void cp_async16(unsigned dst, const void* src, unsigned src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
 // A group of G lanes owns sort chunk c = [cC, cC + C).  It sums, in fp64 and
 // in sorted (= batch) order, the gradients of every segment that starts in the
@@ -398,30 +439,42 @@ enum : unsigned char { kPieceHead = 1, kPieceThrough = 2, kPieceTailStart = 4 };
 // as the starting partial and bwd_combine_kernel finishes it.
 // Piece modes: 0 skip (owned by the previous chunk), 1 long head piece,
 // 2 owned short segment, 3 long segment starting here.
+// Data movement: the gradient row of pair i + R is copied into the group's
+// shared-memory ring (cp.async, each lane its own 16-byte columns, so no lane
+// reads another's data and no barrier is needed) while pair i is added; when
+// a segment starts among the pairs in flight, its table row is prefetched
+// into L2, so the row load at the segment's open mostly hits L2.
 template <int G, int NV, int OPT>
-__global__ void __launch_bounds__(256, NV == 1 ? 3 : (NV == 2 ? 2 : 1))
+__global__ void __launch_bounds__(256, NV == 1 ? DHS_SEG_MINB : (NV == 2 ? 2 : 1))
 bwd_seg_kernel(const unsigned* __restrict__ skey, const unsigned* __restrict__ sval, long long n,
                const float* __restrict__ grad, long long n_bags, int dim, RowSpace rs, OptArgs oa,
                double* __restrict__ part_head, double* __restrict__ part_tail,
                unsigned char* __restrict__ cflags, int C, DevState* st) {
-  constexpr int U = G < 4 ? G : 4;
+  constexpr int R = seg_ring(NV);
+  extern __shared__ float4 seg_ring_smem[];
   const int lane = threadIdx.x & 31;
   const int gl = lane & (G - 1);
   const int gw = lane / G;
   const unsigned gmask = (G == 32) ? 0xffffffffu : (((1u << G) - 1u) << (gw * G));
-  // positions fit in 31 bits (the host rejects larger calls)
+  const int grp = threadIdx.x / G;
+  float4* ring = seg_ring_smem + (size_t)grp * R * NV * G;
+  const unsigned ring_s = (unsigned)__cvta_generic_to_shared(ring);
+  // positions and bags fit in 31 bits (the host rejects larger calls)
   const int n32 = (int)n;
+  const unsigned nb32 = (unsigned)n_bags;
   const int gid = (int)((blockIdx.x * blockDim.x + threadIdx.x) / G);
   const int ngroups = (int)((gridDim.x * blockDim.x) / G);
   const int nchunks = (n32 + C - 1) / C;
   const unsigned nrows = (unsigned)min(st->row_count, 0xffffffffull);
   const int d4 = dim >> 2;
   const int pstride = NV * G * 4;  // doubles per partial vector
+  const unsigned row_bytes = (unsigned)rs.stride * 4u;
   unsigned nseg_total = 0;
 
   for (int c = gid; c < nchunks; c += ngroups) {
     const int start = c * C;
     const int end = min(n32, start + C);
+    const int limit = min(n32, end + C);  // an owned segment ends before chunk c + 2
     unsigned char flags = 0;
     unsigned nseg = 0;
 
@@ -433,6 +486,38 @@ bwd_seg_kernel(const unsigned* __restrict__ skey, const unsigned* __restrict__ s
     const int p2 = (c + 2) * C;
     const bool has2 = p2 < n32;
     const unsigned fwd2 = has2 ? __ldg(skey + p2) : ~0u;
+
+    // ---- producer: gradient rows of pairs start, start + 1, ... into the ring
+    int pf = start;          // next pair to copy
+    int pws = start - G;     // start of the producer's window of pairs
+    unsigned pk = 0u, pv = 0u, pprev = prev;
+    auto produce = [&]() {
+      if (pf < limit) {
+        if (pf >= pws + G) {
+          pws = pf;
+          pk = pws + gl < n32 ? __ldg(skey + pws + gl) : 0u;
+          pv = pws + gl < n32 ? __ldg(sval + pws + gl) : 0u;
+        }
+        const int t = pf - pws;
+        const unsigned b = __shfl_sync(gmask, pv, t, G);
+        const unsigned k = __shfl_sync(gmask, pk, t, G);
+        const bool ok = b < nb32 && k < nrows;
+        const float* src = grad + (size_t)(ok ? b : 0u) * dim;
+        const unsigned slot = ring_s + (unsigned)(((pf - start) % R) * NV * G) * 16u;
+#pragma unroll
+        for (int q = 0; q < NV; ++q) {
+          const int c4 = gl + q * G;
+          cp_async16(slot + (unsigned)(q * G + gl) * 16u, src + (c4 < d4 ? c4 * 4 : 0),
+                     ok && c4 < d4 ? 16u : 0u);
+        }
+        if (DHS_SEG_PREFETCH >= 1 && gl == 0 && ok && k != pprev) prefetch_l2(rs.row(k), row_bytes);
+        pprev = k;
+      }
+      cp_async_commit();  // one group per pair (empty past the limit)
+      ++pf;
+    };
+#pragma unroll
+    for (int j = 0; j < R; ++j) produce();
 
     unsigned cur = cur0;
     int mode;
@@ -451,119 +536,14 @@ bwd_seg_kernel(const unsigned* __restrict__ skey, const unsigned* __restrict__ s
 #pragma unroll
       for (int e = 0; e < 4; ++e) acc[q][e] = 0.0;
 
-    // Window pipeline: the sorted (row, bag) pairs of window ws + G are loaded
-    // while window ws is processed, and each lane bulk-prefetches into L2 the
-    // gradient row of its pair and, where its pair opens a segment, the
-    // table row + state.  The register loads below then mostly hit L2.
-    const unsigned grad_bytes = (unsigned)dim * 4u;
-    const unsigned row_bytes = (unsigned)rs.stride * 4u;
-    auto prefetch_window = [&](int wsn, unsigned& kn, unsigned& vn, unsigned prev_last) {
-      const int cn = min(G, n32 - wsn);
-      kn = gl < cn ? __ldg(skey + wsn + gl) : 0u;
-      vn = gl < cn ? __ldg(sval + wsn + gl) : 0u;
-      const unsigned up = __shfl_up_sync(gmask, kn, 1, G);
-      const unsigned before = gl == 0 ? prev_last : up;
-      if (gl < cn && kn < nrows) {
-        if (vn < n_bags) prefetch_l2(grad + (long long)vn * dim, grad_bytes);
-        if (kn != before) prefetch_l2(rs.row(kn), row_bytes);
-      }
-    };
-    unsigned kk, vv, kk_next = 0u, vv_next = 0u;
-    prefetch_window(start, kk, vv, prev);
-
-    bool done = false;
-    for (int ws = start; ws < n32 && !done; ws += G) {
-      const int cnt = min(G, n32 - ws);
-      const unsigned last = __shfl_sync(gmask, kk, (cnt - 1) & (G - 1), G);
-      // (a short segment may run to the first element of chunk c + 2, so the
-      // next window is always loaded while positions remain)
-      if (ws + G < n32) prefetch_window(ws + G, kk_next, vv_next, last);
-      for (int t0 = 0; t0 < cnt && !done; t0 += U) {
-        float4 x[U][NV];
-#pragma unroll
-        for (int u = 0; u < U; ++u) {
-          const int t = t0 + u;
-          const unsigned bt = __shfl_sync(gmask, vv, t & (G - 1), G);
-          const unsigned ktt = __shfl_sync(gmask, kk, t & (G - 1), G);
-          const bool ok = t < cnt && bt < n_bags && ktt < nrows;
-          const float4* gr = reinterpret_cast<const float4*>(grad + (long long)bt * dim);
-#pragma unroll
-          for (int q = 0; q < NV; ++q) {
-            const int c4 = gl + q * G;
-            x[u][q] = (ok && c4 < d4) ? __ldg(gr + c4) : make_float4(0.f, 0.f, 0.f, 0.f);
-          }
-        }
-#pragma unroll
-        for (int u = 0; u < U; ++u) {
-          const int t = t0 + u;
-          if (done || t >= cnt) break;
-          const int p = ws + t;
-          const unsigned kt = __shfl_sync(gmask, kk, t & (G - 1), G);
-          bool close = false, cont = false;
-          if (kt != cur) {
-            close = true;
-          } else if (p == end && mode != 2) {
-            close = true;  // a long piece stops at the chunk end
-            cont = true;
-          }
-          if (close) {
-            if (mode == 1 || mode == 3) {
-              double* o = (mode == 1 ? part_head : part_tail) + (long long)c * pstride;
-#pragma unroll
-              for (int q = 0; q < NV; ++q)
-#pragma unroll
-                for (int e = 0; e < 4; ++e) o[(q * G + gl) * 4 + e] = acc[q][e];
-              flags |= mode == 3 ? kPieceTailStart : (cont ? kPieceThrough : kPieceHead);
-            } else if (mode == 2 && cur < nrows) {
-              double sq = 0.0;
-              if (OPT == 3) {
-#pragma unroll
-                for (int q = 0; q < NV; ++q)
-#pragma unroll
-                  for (int e = 0; e < 4; ++e) {
-                    const double g = (double)(float)acc[q][e];
-                    sq += g * g;
-                  }
-#pragma unroll
-                for (int o = 1; o < G; o <<= 1) sq += __shfl_xor_sync(gmask, sq, o, G);
-              }
-              rb.step_store(rs.row(cur), dim, gl, G, acc, oa, sq);
-            }
-#pragma unroll
-            for (int q = 0; q < NV; ++q)
-#pragma unroll
-              for (int e = 0; e < 4; ++e) acc[q][e] = 0.0;
-            if (cont || p >= end) {
-              done = true;
-              break;
-            }
-            cur = kt;
-            ++nseg;
-            mode = (has2 && fwd2 == cur) ? 3 : 2;
-            if (mode == 2 && cur < nrows) rb.load(rs.row(cur), dim, gl, G);
-          }
-          if (mode != 0) {
-#pragma unroll
-            for (int q = 0; q < NV; ++q) {
-              acc[q][0] += (double)x[u][q].x;
-              acc[q][1] += (double)x[u][q].y;
-              acc[q][2] += (double)x[u][q].z;
-              acc[q][3] += (double)x[u][q].w;
-            }
-          }
-        }
-      }
-      kk = kk_next;
-      vv = vv_next;
-    }
-    if (!done) {  // reached the end of the array with a piece open
+    auto close_piece = [&](bool cont) {
       if (mode == 1 || mode == 3) {
         double* o = (mode == 1 ? part_head : part_tail) + (long long)c * pstride;
 #pragma unroll
         for (int q = 0; q < NV; ++q)
 #pragma unroll
           for (int e = 0; e < 4; ++e) o[(q * G + gl) * 4 + e] = acc[q][e];
-        flags |= mode == 3 ? kPieceTailStart : kPieceHead;
+        flags |= mode == 3 ? kPieceTailStart : (cont ? kPieceThrough : kPieceHead);
       } else if (mode == 2 && cur < nrows) {
         double sq = 0.0;
         if (OPT == 3) {
@@ -579,7 +559,53 @@ bwd_seg_kernel(const unsigned* __restrict__ skey, const unsigned* __restrict__ s
         }
         rb.step_store(rs.row(cur), dim, gl, G, acc, oa, sq);
       }
+#pragma unroll
+      for (int q = 0; q < NV; ++q)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) acc[q][e] = 0.0;
+    };
+
+    // ---- consumer: pairs in order
+    int cws = start - G;
+    unsigned ck = 0u;
+    bool done = false;
+    for (int i = start; i < n32; ++i) {
+      if (i >= cws + G) {
+        cws = i;
+        ck = i + gl < n32 ? __ldg(skey + i + gl) : 0u;
+      }
+      const unsigned kt = __shfl_sync(gmask, ck, i - cws, G);
+      if (kt != cur) {
+        close_piece(false);
+        if (i >= end) {
+          done = true;
+          break;
+        }
+        cur = kt;
+        ++nseg;
+        mode = (has2 && fwd2 == cur) ? 3 : 2;
+        if (mode == 2 && cur < nrows) rb.load(rs.row(cur), dim, gl, G);
+      } else if (i == end && mode != 2) {
+        close_piece(true);  // a long piece stops at the chunk end
+        done = true;
+        break;
+      }
+      cp_async_wait<R - 1>();  // pair i's columns have landed (this lane's own copy)
+      const float4* slot = ring + ((i - start) % R) * NV * G;
+      if (mode != 0) {
+#pragma unroll
+        for (int q = 0; q < NV; ++q) {
+          const float4 x = slot[q * G + gl];
+          acc[q][0] += (double)x.x;
+          acc[q][1] += (double)x.y;
+          acc[q][2] += (double)x.z;
+          acc[q][3] += (double)x.w;
+        }
+      }
+      produce();  // refill the slot just read with pair i + R
     }
+    if (!done) close_piece(false);  // reached the end of the array with a piece open
+    cp_async_wait_all();  // the ring is reused by the next chunk
     if (gl == 0) {
       cflags[c] = flags;
       if (cur >= nrows && nseg) --nseg;  // the missing-key run is not a row
@@ -592,7 +618,8 @@ bwd_seg_kernel(const unsigned* __restrict__ skey, const unsigned* __restrict__ s
 #ifndef DHS_TEMPLATES_ONLY
 // One thread block per long segment (chunks flagged kPieceTailStart): find the
 // run of partials (through pieces up to the first head piece), sum them in
-// fp64 in a fixed order, and apply the optimizer to the row.
+// fp64 in a fixed order, and apply the optimizer to the row.  Blocks scan the
+// chunk flags 256 at a time and only work on the owners they find.
 __global__ void __launch_bounds__(256)
 bwd_combine_kernel(const unsigned* __restrict__ skey, long long n, int dim, RowSpace rs,
                    OptArgs oa, const double* __restrict__ part_head,
@@ -601,72 +628,82 @@ bwd_combine_kernel(const unsigned* __restrict__ skey, long long n, int dim, RowS
   extern __shared__ double sacc[];  // [slices][dim]
   __shared__ long long s_end;
   __shared__ double s_sq;
+  __shared__ int s_owner[256];
+  __shared__ int s_nown;
   const long long nchunks = (n + C - 1) / C;
   const unsigned long long nrows = st->row_count;
   const int T = blockDim.x;
   const int slices = dim >= T ? 1 : T / dim;
-  for (long long c = blockIdx.x; c < nchunks; c += gridDim.x) {
-    if (!(cflags[c] & kPieceTailStart)) continue;
-    const unsigned key = skey[(c + 1) * (long long)C - 1];
-    // the run ends at the first chunk after c whose piece is a head piece
-    if (threadIdx.x == 0) s_end = nchunks - 1;
+  for (long long base = (long long)blockIdx.x * T; base < nchunks; base += (long long)gridDim.x * T) {
+    if (threadIdx.x == 0) s_nown = 0;
     __syncthreads();
-    for (long long b = c + 1; b < nchunks; b += T) {
-      const long long k = b + threadIdx.x;
-      const bool is_end = k < nchunks && (cflags[k] & kPieceHead);
-      const unsigned any = __syncthreads_or(is_end);
-      if (is_end) atomicMin((unsigned long long*)&s_end, (unsigned long long)k);
+    {
+      const long long cc = base + threadIdx.x;
+      if (cc < nchunks && (cflags[cc] & kPieceTailStart)) s_owner[atomicAdd(&s_nown, 1)] = (int)(cc - base);
+    }
+    __syncthreads();
+    const int nown = s_nown;
+    for (int oi = 0; oi < nown; ++oi) {
+      const long long c = base + s_owner[oi];
+      const unsigned key = skey[(c + 1) * (long long)C - 1];
+      // the run ends at the first chunk after c whose piece is a head piece
+      if (threadIdx.x == 0) s_end = nchunks - 1;
       __syncthreads();
-      if (any) break;
-    }
-    const long long kend = s_end;
-    // sums: slice s adds pieces s, s + slices, ... (piece 0 = starting partial)
-    const long long npieces = kend - c + 1;
-    for (int j0 = 0; j0 < dim; j0 += (slices == 1 ? T : dim)) {
-      const int sl = slices == 1 ? 0 : threadIdx.x / dim;
-      const int j = slices == 1 ? j0 + threadIdx.x : threadIdx.x % dim;
-      if (sl < slices && j < dim) {
-        double a = 0.0;
-        for (long long pc = sl; pc < npieces; pc += slices) {
-          const double* src = pc == 0 ? part_tail + c * (long long)pstride
-                                      : part_head + (c + pc) * (long long)pstride;
-          a += src[j];
-        }
-        sacc[sl * dim + j] = a;
+      for (long long b = c + 1; b < nchunks; b += T) {
+        const long long k = b + threadIdx.x;
+        const bool is_end = k < nchunks && (cflags[k] & kPieceHead);
+        const unsigned any = __syncthreads_or(is_end);
+        if (is_end) atomicMin((unsigned long long*)&s_end, (unsigned long long)k);
+        __syncthreads();
+        if (any) break;
       }
-      if (slices != 1) break;
-    }
-    __syncthreads();
-    // fold slices in order into slice 0
-    if (threadIdx.x < dim || slices == 1) {
+      const long long kend = s_end;
+      // sums: slice s adds pieces s, s + slices, ... (piece 0 = starting partial)
+      const long long npieces = kend - c + 1;
+      for (int j0 = 0; j0 < dim; j0 += (slices == 1 ? T : dim)) {
+        const int sl = slices == 1 ? 0 : threadIdx.x / dim;
+        const int j = slices == 1 ? j0 + threadIdx.x : threadIdx.x % dim;
+        if (sl < slices && j < dim) {
+          double a = 0.0;
+          for (long long pc = sl; pc < npieces; pc += slices) {
+            const double* src = pc == 0 ? part_tail + c * (long long)pstride
+                                        : part_head + (c + pc) * (long long)pstride;
+            a += src[j];
+          }
+          sacc[sl * dim + j] = a;
+        }
+        if (slices != 1) break;
+      }
+      __syncthreads();
+      // fold slices in order into slice 0
       for (int j = threadIdx.x; j < dim && slices > 1; j += T) {
         double a = sacc[j];
-        for (int s = 1; s < slices; ++s) a += sacc[s * dim + j];
+        for (int s2 = 1; s2 < slices; ++s2) a += sacc[s2 * dim + j];
         sacc[j] = a;
       }
-    }
-    __syncthreads();
-    if (key < nrows) {
-      float* row = rs.row(key);
-      float den = 0.f;
-      if (oa.opt == 3) {
-        if (threadIdx.x == 0) {
-          double sq = 0.0;
-          for (int j = 0; j < dim; ++j) {
-            const double g = (double)(float)sacc[j];
-            sq += g * g;
+      __syncthreads();
+      if (key < nrows) {
+        float* row = rs.row(key);
+        float den = 0.f;
+        if (oa.opt == 3) {
+          if (threadIdx.x == 0) {
+            double sq = 0.0;
+            for (int j = 0; j < dim; ++j) {
+              const double g = (double)(float)sacc[j];
+              sq += g * g;
+            }
+            s_sq = sq;
           }
-          s_sq = sq;
+          __syncthreads();
+          const float Gn = __fadd_rn(row[dim], (float)(s_sq / (double)dim));
+          den = __fadd_rn(__fsqrt_rn(Gn), oa.eps);
+          __syncthreads();
+          if (threadIdx.x == 0) row[dim] = Gn;
         }
-        __syncthreads();
-        const float Gn = __fadd_rn(row[dim], (float)(s_sq / (double)dim));
-        den = __fadd_rn(__fsqrt_rn(Gn), oa.eps);
-        __syncthreads();
-        if (threadIdx.x == 0) row[dim] = Gn;
+        for (int j = threadIdx.x; j < dim; j += T) update_col(row, dim, j, (float)sacc[j], oa, den);
       }
-      for (int j = threadIdx.x; j < dim; j += T) update_col(row, dim, j, (float)sacc[j], oa, den);
+      __syncthreads();
     }
-    __syncthreads();
   }
 }
 

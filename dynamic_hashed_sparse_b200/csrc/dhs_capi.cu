@@ -654,6 +654,7 @@ dhs_status embbag_forward(dhs_table* t, const int64_t* d_keys, int64_t n_keys,
     return DHS_ERR_INVALID_ARG;
   if (n_bags == 0) return n_keys == 0 ? DHS_OK : DHS_ERR_INVALID_ARG;
   if (!d_bag_offsets || !d_pooled_out || (n_keys > 0 && !d_keys)) return DHS_ERR_INVALID_ARG;
+  if ((uintptr_t)d_pooled_out % 16) return DHS_ERR_INVALID_ARG;
   DeviceGuard g(t->device);
   cudaStream_t s = (cudaStream_t)stream;
   t->last_stream = s;
@@ -685,6 +686,7 @@ dhs_status embbag_backward_update(dhs_table* t, const int64_t* d_keys, int64_t n
     return DHS_ERR_INVALID_ARG;
   if (n_bags == 0 && n_keys != 0) return DHS_ERR_INVALID_ARG;
   if (n_bags > 0 && (!d_bag_offsets || !d_grad)) return DHS_ERR_INVALID_ARG;
+  if ((uintptr_t)d_grad % 16) return DHS_ERR_INVALID_ARG;
   if (n_keys > 0 && !d_keys) return DHS_ERR_INVALID_ARG;
   if (!std::isfinite(lr)) return DHS_ERR_INVALID_ARG;
   DeviceGuard g(t->device);
@@ -759,7 +761,7 @@ dhs_status embbag_backward_update(dhs_table* t, const int64_t* d_keys, int64_t n
     const int chunk = seg_chunk(n_keys);
     const long long nchunks = (n_keys + chunk - 1) / chunk;
     const size_t smem = (size_t)std::max(256, t->dim) * sizeof(double);
-    const long long grid = std::min<long long>(nchunks, (long long)t->sm_count * 8);
+    const long long grid = std::min<long long>((nchunks + 255) / 256, (long long)t->sm_count * 8);
     bwd_combine_kernel<<<(unsigned)grid, 256, smem, s>>>(ka, n_keys, t->dim, rowspace(t), oa,
                                                         (const double*)t->b_ph.p, (const double*)t->b_pt.p,
                                                         (const unsigned char*)t->b_cflags.p, chunk,

@@ -17,9 +17,12 @@ cudaError_t run(int sm_count, const unsigned* skey, const unsigned* sval, long l
                 double* part_head, double* part_tail, unsigned char* cflags, int chunk,
                 DevState* st, cudaStream_t s) {
   static int resident = 0;
+  const size_t smem = seg_smem_bytes(G, NV);
   if (!resident) {
+    if (smem > 48 * 1024)
+      cudaFuncSetAttribute(bwd_seg_kernel<G, NV, OPT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     int per_sm = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, bwd_seg_kernel<G, NV, OPT>, 256, 0) !=
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, bwd_seg_kernel<G, NV, OPT>, 256, smem) !=
             cudaSuccess || per_sm < 1) {
       cudaGetLastError();
       per_sm = 1;
@@ -30,7 +33,7 @@ cudaError_t run(int sm_count, const unsigned* skey, const unsigned* sval, long l
   const long long per_block = 256 / G;
   const long long need = std::max<long long>(1, (nchunks + per_block - 1) / per_block);
   const long long grid = std::min<long long>(need, resident);
-  bwd_seg_kernel<G, NV, OPT><<<(unsigned)grid, 256, 0, s>>>(skey, sval, n, grad, n_bags, dim, rs, oa,
+  bwd_seg_kernel<G, NV, OPT><<<(unsigned)grid, 256, smem, s>>>(skey, sval, n, grad, n_bags, dim, rs, oa,
                                                            part_head, part_tail, cflags, chunk, st);
   return cudaGetLastError();
 }

@@ -148,8 +148,8 @@ dhs_status ht_lookup(dhs_table* t, const int64_t* d_keys, int64_t n, int64_t* d_
  *                        d_bag_offsets[b+1]) in that order, fp32.
  * d_keys int64[n_keys]; d_bag_offsets int64[n_bags + 1], non-decreasing,
  * [0] = 0, [n_bags] = n_keys (checked on the device); d_pooled_out
- * float[n_bags, dim] row-major.  An empty bag gives a zero row.  New keys get
- * rows exactly as in ht_lookup_or_insert. */
+ * float[n_bags, dim] row-major, 16-byte aligned.  An empty bag gives a zero
+ * row.  New keys get rows exactly as in ht_lookup_or_insert. */
 dhs_status embbag_forward(dhs_table* t, const int64_t* d_keys, int64_t n_keys,
                           const int64_t* d_bag_offsets, int64_t n_bags, float* d_pooled_out,
                           dhs_stream stream);
@@ -162,8 +162,8 @@ dhs_status embbag_forward(dhs_table* t, const int64_t* d_keys, int64_t n_keys,
  * with learning rate lr.  Rows not in d_keys are not read or written.  The
  * Adam step count advances by one per call.  Keys must be in the table
  * (missing ones are skipped and latch DHS_ERR_NOT_FOUND).
- * d_grad float[n_bags, dim] row-major; the other arguments as in
- * embbag_forward. */
+ * d_grad float[n_bags, dim] row-major, 16-byte aligned (rows are copied in
+ * 16-byte pieces); the other arguments as in embbag_forward. */
 dhs_status embbag_backward_update(dhs_table* t, const int64_t* d_keys, int64_t n_keys,
                                   const int64_t* d_bag_offsets, int64_t n_bags,
                                   const float* d_grad, float lr, dhs_stream stream);
