@@ -12,6 +12,8 @@ from ._binding import (  # noqa: F401
     dhs_pack_keys,
     dhs_status_str,
     embbag_backward_update,
+    embbag_backward_update_noalloc,
+    NOALLOC_MAX_KEYS,
     embbag_forward,
     ht_counters,
     ht_create,

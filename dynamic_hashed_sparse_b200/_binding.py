@@ -51,6 +51,7 @@ def _load() -> C.CDLL:
         "ht_lookup": (C.c_int, [vp, vp, i64, vp, vp]),
         "embbag_forward": (C.c_int, [vp, vp, i64, vp, i64, vp, vp]),
         "embbag_backward_update": (C.c_int, [vp, vp, i64, vp, i64, vp, f32, vp]),
+        "embbag_backward_update_noalloc": (C.c_int, [vp, vp, i64, vp, i64, vp, f32, vp]),
         "ht_get_rows": (C.c_int, [vp, vp, i64, vp, vp]),
         "ht_row_stride": (i64, [vp]),
         "ht_sync": (C.c_int, [vp]),
@@ -212,6 +213,27 @@ def embbag_backward_update(t: Table, keys: torch.Tensor, bag_offsets: torch.Tens
     _check("embbag_backward_update",
            _lib.embbag_backward_update(t.handle, keys.data_ptr(), keys.numel(), bag_offsets.data_ptr(),
                                        nb, grad.data_ptr(), float(lr), _stream(stream)))
+
+
+NOALLOC_MAX_KEYS = 131072
+
+
+def embbag_backward_update_noalloc(t: Table, keys: torch.Tensor, bag_offsets: torch.Tensor,
+                                   grad: torch.Tensor, lr: float, stream=None):
+    """embbag_backward_update for callers that cannot allocate device memory
+    during a step: the library uses a fixed device array as scratch (at most
+    NOALLOC_MAX_KEYS keys, dim <= 128); it allocates nothing.  Make the first
+    call on a device before any stream capture; calls that overlap on the GPU
+    race."""
+    _dev(keys, torch.int64, "keys")
+    _dev(bag_offsets, torch.int64, "bag_offsets")
+    _dev(grad, torch.float32, "grad")
+    nb = bag_offsets.numel() - 1
+    if grad.numel() != nb * t.dim:
+        raise ValueError("grad must hold n_bags * dim floats")
+    _check("embbag_backward_update_noalloc",
+           _lib.embbag_backward_update_noalloc(t.handle, keys.data_ptr(), keys.numel(), bag_offsets.data_ptr(),
+                                               nb, grad.data_ptr(), float(lr), _stream(stream)))
 
 
 def ht_get_rows(t: Table, keys: torch.Tensor, out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:

@@ -12,6 +12,7 @@
 #include <cmath>
 #include <cstdint>
 #include <cstring>
+#include <mutex>
 #include <new>
 #include <vector>
 
@@ -899,6 +900,151 @@ dhs_status ht_phase_times(dhs_table* t, double* ms_out, int64_t* count_out, int 
   t->recs.clear();
   cudaGetLastError();
   return rc;
+}
+
+
+// ---------------------------------------------------------------------------
+// Backward + update without any allocation
+// ---------------------------------------------------------------------------
+// For callers that cannot allocate device memory during a training step (for
+// example a runtime that forbids cudaMalloc once its steps are running, or
+// one that hands this library only the buffers it owns).  The scratch of the
+// sort and the segment reduce lives in one file-scope device array of fixed
+// size instead of the table's growable workspace.
+}  // extern "C"
+
+namespace {
+
+constexpr long long kNoAllocMaxKeys = 131072;
+constexpr int kNoAllocMaxDim = 128;
+constexpr int kNoAllocMinChunk = 32;  // seg_chunk() never goes below this
+
+constexpr size_t na_align(size_t x) { return (x + 255) & ~size_t(255); }
+constexpr size_t kNaPairs = na_align(kNoAllocMaxKeys * 4);  // one of ka, va, kb, vb
+constexpr size_t kNaSortZero = na_align((kRadixMaxPasses * kRadixBins + kRadixMaxPasses) * 4);
+constexpr size_t kNaStatus =
+    na_align((size_t)kRadixMaxPasses * ((kNoAllocMaxKeys + kRadixTile - 1) / kRadixTile) * kRadixBins * 8);
+constexpr size_t kNaChunks = (kNoAllocMaxKeys + kNoAllocMinChunk - 1) / kNoAllocMinChunk;
+constexpr size_t kNaPart = na_align(kNaChunks * kNoAllocMaxDim * 8);  // one of part_head, part_tail
+constexpr size_t kNaFlags = na_align(kNaChunks);
+constexpr size_t kNoAllocScratchBytes = 4 * kNaPairs + kNaSortZero + kNaStatus + 2 * kNaPart + kNaFlags;
+
+// Every GPU that loads this library holds this array until the process exits.
+__device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[128] = {};
+
+// Device address of the scratch array on `dev` (which must be current): looked
+// up once per device with cudaGetSymbolAddress, then cached.
+dhs_status noalloc_scratch(int dev, unsigned char** out) {
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (dev < 0 || dev >= 128) return DHS_ERR_UNSUPPORTED;
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) {
+      cudaGetLastError();
+      return DHS_ERR_CUDA;
+    }
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = (unsigned char*)g_noalloc_ptr[dev];
+  return DHS_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+dhs_status embbag_backward_update_noalloc(dhs_table* t, const int64_t* d_keys, int64_t n_keys,
+                                          const int64_t* d_bag_offsets, int64_t n_bags,
+                                          const float* d_grad, float lr, dhs_stream stream) {
+  DHS_TRY(check_table(t));
+  if (n_keys < 0 || n_bags < 0 || n_bags >= (1ll << 31)) return DHS_ERR_INVALID_ARG;
+  if (n_keys > kNoAllocMaxKeys || t->dim > kNoAllocMaxDim) return DHS_ERR_INVALID_ARG;
+  if (n_bags == 0 && n_keys != 0) return DHS_ERR_INVALID_ARG;
+  if (n_bags > 0 && (!d_bag_offsets || !d_grad)) return DHS_ERR_INVALID_ARG;
+  if ((uintptr_t)d_grad % 16) return DHS_ERR_INVALID_ARG;
+  if (n_keys > 0 && !d_keys) return DHS_ERR_INVALID_ARG;
+  if (!std::isfinite(lr)) return DHS_ERR_INVALID_ARG;
+  DeviceGuard g(t->device);
+  unsigned char* base = nullptr;
+  DHS_TRY(noalloc_scratch(t->device, &base));
+  cudaStream_t s = (cudaStream_t)stream;
+  t->last_stream = s;
+  t->adam_t += 1;
+  if (n_keys == 0) return DHS_OK;
+
+  unsigned* ka = (unsigned*)base;
+  unsigned* va = (unsigned*)(base + kNaPairs);
+  unsigned* kb = (unsigned*)(base + 2 * kNaPairs);
+  unsigned* vb = (unsigned*)(base + 3 * kNaPairs);
+  unsigned* hist = (unsigned*)(base + 4 * kNaPairs);
+  unsigned* tile_ctr = hist + kRadixMaxPasses * kRadixBins;
+  unsigned long long* status = (unsigned long long*)(base + 4 * kNaPairs + kNaSortZero);
+  double* part_head = (double*)(base + 4 * kNaPairs + kNaSortZero + kNaStatus);
+  double* part_tail = (double*)(base + 4 * kNaPairs + kNaSortZero + kNaStatus + kNaPart);
+  unsigned char* cflags = base + 4 * kNaPairs + kNaSortZero + kNaStatus + 2 * kNaPart;
+
+  refresh_ub(t, false);
+  const unsigned sentinel = (unsigned)t->rows_ub;
+  int bits = 0;
+  while (bits < 32 && (1ull << bits) <= (unsigned long long)sentinel) ++bits;
+  const int passes = std::min(kRadixMaxPasses, std::max(1, (bits + 7) / 8));
+
+  {
+    const long long warps = (n_bags + 31) / 32;
+    const long long grid = std::max<long long>(1, std::min<long long>((warps + 7) / 8, (long long)t->sm_count * 8));
+    bwd_probe_kernel<<<(unsigned)grid, 256, 0, s>>>(idmap(t), (const long long*)d_keys, n_keys,
+                                                    (const long long*)d_bag_offsets, n_bags, ka, va,
+                                                    sentinel, hist, kRadixMaxPasses * kRadixBins + kRadixMaxPasses,
+                                                    t->st);
+    DHS_TRY(last_launch());
+  }
+  const long long ntiles = (n_keys + kRadixTile - 1) / kRadixTile;
+  {
+    const long long hgrid = std::min<long long>((n_keys + kRadixThreads - 1) / kRadixThreads,
+                                                (long long)t->sm_count * 8);
+    radix_hist_all_kernel<<<(unsigned)hgrid, kRadixThreads, 0, s>>>(
+        ka, n_keys, passes, hist, status, (long long)passes * ntiles * kRadixBins);
+    DHS_TRY(last_launch());
+    for (int p = 0; p < passes; ++p) {
+      radix_onesweep_kernel<<<(unsigned)ntiles, kRadixThreads, 0, s>>>(
+          ka, va, kb, vb, n_keys, 8 * p, hist + p * kRadixBins, status + (long long)p * ntiles * kRadixBins,
+          tile_ctr + p, t->st);
+      DHS_TRY(last_launch());
+      std::swap(ka, kb);
+      std::swap(va, vb);
+    }
+  }
+  OptArgs oa;
+  oa.opt = t->opt;
+  oa.lr = lr;
+  oa.eps = t->eps;
+  oa.b1 = t->b1;
+  oa.b2 = t->b2;
+  oa.c1 = (float)(1.0 - (double)t->b1);
+  oa.c2 = (float)(1.0 - (double)t->b2);
+  oa.bc1 = (float)(1.0 - std::pow((double)t->b1, (double)t->adam_t));
+  oa.bc2 = (float)(1.0 - std::pow((double)t->b2, (double)t->adam_t));
+  const int G = pick_group(t->dim), NV = pick_nv(t->dim, G);
+  const int chunk = seg_chunk(n_keys);
+  auto fn = t->opt == DHS_SGD ? launch_seg_sgd
+            : t->opt == DHS_ADAGRAD ? launch_seg_adagrad
+            : t->opt == DHS_ADAM ? launch_seg_adam
+                                 : launch_seg_rowwise;
+  if (fn(G, NV, t->sm_count, ka, va, n_keys, d_grad, n_bags, t->dim, rowspace(t), oa, part_head, part_tail,
+         cflags, chunk, t->st, s) != cudaSuccess) {
+    cudaGetLastError();
+    return DHS_ERR_CUDA;
+  }
+  const long long nchunks = (n_keys + chunk - 1) / chunk;
+  const size_t smem = (size_t)std::max(256, t->dim) * sizeof(double);
+  const long long grid = std::min<long long>((nchunks + 255) / 256, (long long)t->sm_count * 8);
+  bwd_combine_kernel<<<(unsigned)grid, 256, smem, s>>>(ka, n_keys, t->dim, rowspace(t), oa, part_head,
+                                                      part_tail, cflags, chunk, NV * G * 4, t->st);
+  t->n_launches += 4 + passes;
+  return last_launch();
 }
 
 }  // extern "C"

@@ -168,6 +168,27 @@ dhs_status embbag_backward_update(dhs_table* t, const int64_t* d_keys, int64_t n
                                   const int64_t* d_bag_offsets, int64_t n_bags,
                                   const float* d_grad, float lr, dhs_stream stream);
 
+/* Allocation-free variant of embbag_backward_update (the pages have no
+ * counterpart: it exists for callers that cannot allocate device memory
+ * during a step, e.g. a runtime that forbids cudaMalloc once its training
+ * loop runs, or one that gives this library only the buffers it owns).
+ * Same arguments, same result as embbag_backward_update; the sort and
+ * segment-reduce scratch is one fixed file-scope device array (about 11 MB,
+ * held by every GPU that loads this library until the process exits)
+ * instead of the table's growable workspace, and no cudaMalloc, cudaFree or
+ * allocating library routine is called.
+ * Limits: n_keys <= DHS_NOALLOC_MAX_KEYS and a table dim <= 128; larger calls
+ * return DHS_ERR_INVALID_ARG and do nothing.
+ * The first call on a device looks the array's address up
+ * (cudaGetSymbolAddress) and caches it: make that first call before any
+ * stream capture.  All calls share the one array, so calls whose work
+ * overlaps on the GPU (different streams, or different tables on the same
+ * device without ordering) race; order them. */
+#define DHS_NOALLOC_MAX_KEYS 131072
+dhs_status embbag_backward_update_noalloc(dhs_table* t, const int64_t* d_keys, int64_t n_keys,
+                                          const int64_t* d_bag_offsets, int64_t n_bags,
+                                          const float* d_grad, float lr, dhs_stream stream);
+
 /* Copy the full rows (dim weights, then the state) of the given keys into
  * d_rows_out float[n, ht_row_stride(t)]; an absent key gives a NaN row. */
 dhs_status ht_get_rows(dhs_table* t, const int64_t* d_keys, int64_t n, float* d_rows_out,
