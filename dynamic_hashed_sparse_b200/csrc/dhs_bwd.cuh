@@ -28,7 +28,7 @@
 //                     compiled for (register budget) when a lane holds one
 //                     float4 column
 #ifndef DHS_SEG_MINB
-#define DHS_SEG_MINB 4
+#define DHS_SEG_MINB 3
 #endif
 //   DHS_SEG_RING      gradient rows in flight per group (shared-memory ring)
 //                     for a row of <= 128 floats; wider rows use fewer
@@ -118,6 +118,12 @@ constexpr unsigned long long kLbAggregate = 1ull << 62;  // tile count published
 constexpr unsigned long long kLbPrefix = 2ull << 62;     // inclusive prefix published
 constexpr unsigned long long kLbCountMask = (1ull << 62) - 1;
 constexpr unsigned kLookbackSpins = 1u << 22;  // bounded wait for a predecessor tile
+// words cleared by bwd_probe_kernel before a backward: digit histograms of
+// every pass, one tile counter per pass, the segment kernel's chunk counter
+// and the count of long-segment owner chunks
+constexpr int kSortZeroWords = kRadixMaxPasses * kRadixBins + kRadixMaxPasses + 2;
+constexpr int kSegChunkCtrWord = kRadixMaxPasses * kRadixBins + kRadixMaxPasses;
+constexpr int kSegOwnerCtrWord = kSegChunkCtrWord + 1;
 
 // Digit counts of every pass in one read of the keys (global atomics, one per
 // block and bin), and the look-back state of every pass cleared.  hist and
@@ -445,11 +451,12 @@ __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wai
 // a segment starts among the pairs in flight, its table row is prefetched
 // into L2, so the row load at the segment's open mostly hits L2.
 template <int G, int NV, int OPT>
-__global__ void __launch_bounds__(256, NV == 1 ? DHS_SEG_MINB : (NV == 2 ? 2 : 1))
+__global__ void __launch_bounds__(256, NV <= 2 ? DHS_SEG_MINB : 1)
 bwd_seg_kernel(const unsigned* __restrict__ skey, const unsigned* __restrict__ sval, long long n,
                const float* __restrict__ grad, long long n_bags, int dim, RowSpace rs, OptArgs oa,
                double* __restrict__ part_head, double* __restrict__ part_tail,
-               unsigned char* __restrict__ cflags, int C, DevState* st) {
+               unsigned char* __restrict__ cflags, int C, unsigned* __restrict__ chunk_ctr,
+               unsigned* __restrict__ owners, unsigned* __restrict__ owner_ctr, DevState* st) {
   constexpr int R = seg_ring(NV);
   extern __shared__ float4 seg_ring_smem[];
   const int lane = threadIdx.x & 31;
@@ -462,8 +469,6 @@ bwd_seg_kernel(const unsigned* __restrict__ skey, const unsigned* __restrict__ s
   // positions and bags fit in 31 bits (the host rejects larger calls)
   const int n32 = (int)n;
   const unsigned nb32 = (unsigned)n_bags;
-  const int gid = (int)((blockIdx.x * blockDim.x + threadIdx.x) / G);
-  const int ngroups = (int)((gridDim.x * blockDim.x) / G);
   const int nchunks = (n32 + C - 1) / C;
   const unsigned nrows = (unsigned)min(st->row_count, 0xffffffffull);
   const int d4 = dim >> 2;
@@ -471,7 +476,14 @@ bwd_seg_kernel(const unsigned* __restrict__ skey, const unsigned* __restrict__ s
   const unsigned row_bytes = (unsigned)rs.stride * 4u;
   unsigned nseg_total = 0;
 
-  for (int c = gid; c < nchunks; c += ngroups) {
+  // chunks are handed out one at a time (a counter), so groups that meet
+  // cheap chunks take more of them and none idles while others still work
+  auto next_chunk = [&]() {
+    int v = 0;
+    if (gl == 0) v = (int)atomicAdd(chunk_ctr, 1u);
+    return __shfl_sync(gmask, v, 0, G);
+  };
+  for (int c = next_chunk(); c < nchunks; c = next_chunk()) {
     const int start = c * C;
     const int end = min(n32, start + C);
     const int limit = min(n32, end + C);  // an owned segment ends before chunk c + 2
@@ -544,6 +556,7 @@ bwd_seg_kernel(const unsigned* __restrict__ skey, const unsigned* __restrict__ s
 #pragma unroll
           for (int e = 0; e < 4; ++e) o[(q * G + gl) * 4 + e] = acc[q][e];
         flags |= mode == 3 ? kPieceTailStart : (cont ? kPieceThrough : kPieceHead);
+        if (mode == 3 && gl == 0) owners[atomicAdd(owner_ctr, 1u)] = (unsigned)c;  // for the combine
       } else if (mode == 2 && cur < nrows) {
         double sq = 0.0;
         if (OPT == 3) {
@@ -616,94 +629,84 @@ bwd_seg_kernel(const unsigned* __restrict__ skey, const unsigned* __restrict__ s
 }
 
 #ifndef DHS_TEMPLATES_ONLY
-// One thread block per long segment (chunks flagged kPieceTailStart): find the
-// run of partials (through pieces up to the first head piece), sum them in
-// fp64 in a fixed order, and apply the optimizer to the row.  Blocks scan the
-// chunk flags 256 at a time and only work on the owners they find.
+// One thread block per long segment (the owner chunks the segment kernel
+// listed): find the run of partials (through pieces up to the first head
+// piece), sum them in fp64 in a fixed order, and apply the optimizer to the
+// row.
 __global__ void __launch_bounds__(256)
 bwd_combine_kernel(const unsigned* __restrict__ skey, long long n, int dim, RowSpace rs,
                    OptArgs oa, const double* __restrict__ part_head,
                    const double* __restrict__ part_tail, const unsigned char* __restrict__ cflags,
-                   int C, int pstride, DevState* st) {
+                   int C, int pstride, const unsigned* __restrict__ owners,
+                   const unsigned* __restrict__ owner_ctr, DevState* st) {
   extern __shared__ double sacc[];  // [slices][dim]
   __shared__ long long s_end;
   __shared__ double s_sq;
-  __shared__ int s_owner[256];
-  __shared__ int s_nown;
   const long long nchunks = (n + C - 1) / C;
   const unsigned long long nrows = st->row_count;
   const int T = blockDim.x;
   const int slices = dim >= T ? 1 : T / dim;
-  for (long long base = (long long)blockIdx.x * T; base < nchunks; base += (long long)gridDim.x * T) {
-    if (threadIdx.x == 0) s_nown = 0;
+  const unsigned n_own = *owner_ctr;
+  for (unsigned oi = blockIdx.x; oi < n_own; oi += gridDim.x) {
+    const long long c = owners[oi];
+    const unsigned key = skey[(c + 1) * (long long)C - 1];
+    // the run ends at the first chunk after c whose piece is a head piece
+    if (threadIdx.x == 0) s_end = nchunks - 1;
     __syncthreads();
-    {
-      const long long cc = base + threadIdx.x;
-      if (cc < nchunks && (cflags[cc] & kPieceTailStart)) s_owner[atomicAdd(&s_nown, 1)] = (int)(cc - base);
+    for (long long b = c + 1; b < nchunks; b += T) {
+      const long long k = b + threadIdx.x;
+      const bool is_end = k < nchunks && (cflags[k] & kPieceHead);
+      const unsigned any = __syncthreads_or(is_end);
+      if (is_end) atomicMin((unsigned long long*)&s_end, (unsigned long long)k);
+      __syncthreads();
+      if (any) break;
+    }
+    const long long kend = s_end;
+    // sums: slice s adds pieces s, s + slices, ... (piece 0 = starting partial)
+    const long long npieces = kend - c + 1;
+    for (int j0 = 0; j0 < dim; j0 += (slices == 1 ? T : dim)) {
+      const int sl = slices == 1 ? 0 : threadIdx.x / dim;
+      const int j = slices == 1 ? j0 + threadIdx.x : threadIdx.x % dim;
+      if (sl < slices && j < dim) {
+        double a = 0.0;
+        for (long long pc = sl; pc < npieces; pc += slices) {
+          const double* src = pc == 0 ? part_tail + c * (long long)pstride
+                                      : part_head + (c + pc) * (long long)pstride;
+          a += src[j];
+        }
+        sacc[sl * dim + j] = a;
+      }
+      if (slices != 1) break;
     }
     __syncthreads();
-    const int nown = s_nown;
-    for (int oi = 0; oi < nown; ++oi) {
-      const long long c = base + s_owner[oi];
-      const unsigned key = skey[(c + 1) * (long long)C - 1];
-      // the run ends at the first chunk after c whose piece is a head piece
-      if (threadIdx.x == 0) s_end = nchunks - 1;
-      __syncthreads();
-      for (long long b = c + 1; b < nchunks; b += T) {
-        const long long k = b + threadIdx.x;
-        const bool is_end = k < nchunks && (cflags[k] & kPieceHead);
-        const unsigned any = __syncthreads_or(is_end);
-        if (is_end) atomicMin((unsigned long long*)&s_end, (unsigned long long)k);
+    // fold slices in order into slice 0
+    for (int j = threadIdx.x; j < dim && slices > 1; j += T) {
+      double a = sacc[j];
+      for (int s2 = 1; s2 < slices; ++s2) a += sacc[s2 * dim + j];
+      sacc[j] = a;
+    }
+    __syncthreads();
+    if (key < nrows) {
+      float* row = rs.row(key);
+      float den = 0.f;
+      if (oa.opt == 3) {
+        if (threadIdx.x == 0) {
+          double sq = 0.0;
+          for (int j = 0; j < dim; ++j) {
+            const double g = (double)(float)sacc[j];
+            sq += g * g;
+          }
+          s_sq = sq;
+        }
         __syncthreads();
-        if (any) break;
+        const float Gn = __fadd_rn(row[dim], (float)(s_sq / (double)dim));
+        den = __fadd_rn(__fsqrt_rn(Gn), oa.eps);
+        __syncthreads();
+        if (threadIdx.x == 0) row[dim] = Gn;
       }
-      const long long kend = s_end;
-      // sums: slice s adds pieces s, s + slices, ... (piece 0 = starting partial)
-      const long long npieces = kend - c + 1;
-      for (int j0 = 0; j0 < dim; j0 += (slices == 1 ? T : dim)) {
-        const int sl = slices == 1 ? 0 : threadIdx.x / dim;
-        const int j = slices == 1 ? j0 + threadIdx.x : threadIdx.x % dim;
-        if (sl < slices && j < dim) {
-          double a = 0.0;
-          for (long long pc = sl; pc < npieces; pc += slices) {
-            const double* src = pc == 0 ? part_tail + c * (long long)pstride
-                                        : part_head + (c + pc) * (long long)pstride;
-            a += src[j];
-          }
-          sacc[sl * dim + j] = a;
-        }
-        if (slices != 1) break;
-      }
-      __syncthreads();
-      // fold slices in order into slice 0
-      for (int j = threadIdx.x; j < dim && slices > 1; j += T) {
-        double a = sacc[j];
-        for (int s2 = 1; s2 < slices; ++s2) a += sacc[s2 * dim + j];
-        sacc[j] = a;
-      }
-      __syncthreads();
-      if (key < nrows) {
-        float* row = rs.row(key);
-        float den = 0.f;
-        if (oa.opt == 3) {
-          if (threadIdx.x == 0) {
-            double sq = 0.0;
-            for (int j = 0; j < dim; ++j) {
-              const double g = (double)(float)sacc[j];
-              sq += g * g;
-            }
-            s_sq = sq;
-          }
-          __syncthreads();
-          const float Gn = __fadd_rn(row[dim], (float)(s_sq / (double)dim));
-          den = __fadd_rn(__fsqrt_rn(Gn), oa.eps);
-          __syncthreads();
-          if (threadIdx.x == 0) row[dim] = Gn;
-        }
-        for (int j = threadIdx.x; j < dim; j += T) update_col(row, dim, j, (float)sacc[j], oa, den);
-      }
-      __syncthreads();
+      for (int j = threadIdx.x; j < dim; j += T) update_col(row, dim, j, (float)sacc[j], oa, den);
     }
+    __syncthreads();
   }
 }
 

@@ -72,6 +72,19 @@ int pick_nv(int dim, int g) {
   return v;
 }
 
+// Segment-kernel lanes: 8 float columns per lane (two float4), so that a
+// warp holds two or more groups and the per-pair control work is shared;
+// rows wider than 256 floats use 16 columns per lane.
+int seg_group(int dim) {
+  if (dim > 256) return 32;
+  const int need = (dim + 7) / 8;
+  int g = 1;
+  while (g < need) g <<= 1;
+  return g;
+}
+
+int seg_nv(int dim) { return dim > 256 ? 4 : 2; }
+
 int log2_exact(long long x) {
   int l = 0;
   while ((1ll << l) < x) ++l;
@@ -116,7 +129,7 @@ struct dhs_table {
   // workspace, sized for ws_n positions
   long long ws_n = -1;
   Buf b_nbm, b_fbm, b_gcnt, b_gpref, b_slotpos, b_ka, b_va, b_kb, b_vb, b_hist, b_totals, b_ph,
-      b_pt, b_cflags;
+      b_pt, b_cflags, b_owners;
 
   bool timing = false;
   std::vector<PhaseRec> recs;
@@ -366,8 +379,7 @@ dhs_status ensure_ws(dhs_table* t, long long n, cudaStream_t s) {
   const long long nwords = ngroups * kGroupWords;
   const long long ntiles = (cap + kRadixTile - 1) / kRadixTile;
   const long long nchunks = (cap + seg_chunk(cap) - 1) / seg_chunk(cap) + (cap + 31) / 32;
-  const int G = pick_group(t->dim), NV = pick_nv(t->dim, G);
-  const long long pstride = (long long)NV * G * 4;
+  const long long pstride = (long long)seg_nv(t->dim) * seg_group(t->dim) * 4;
   DHS_TRY(bget(t, t->b_nbm, nwords * 4, s));
   DHS_TRY(bget(t, t->b_fbm, nwords * 4, s));
   DHS_TRY(bget(t, t->b_gcnt, ngroups * 4, s));
@@ -378,11 +390,12 @@ dhs_status ensure_ws(dhs_table* t, long long n, cudaStream_t s) {
   DHS_TRY(bget(t, t->b_kb, cap * 4, s));
   DHS_TRY(bget(t, t->b_vb, cap * 4, s));
   // digit histograms of every pass + one tile counter per pass; look-back state
-  DHS_TRY(bget(t, t->b_hist, (size_t)(kRadixMaxPasses * kRadixBins + kRadixMaxPasses) * 4, s));
+  DHS_TRY(bget(t, t->b_hist, (size_t)kSortZeroWords * 4, s));
   DHS_TRY(bget(t, t->b_totals, (size_t)kRadixMaxPasses * ntiles * kRadixBins * 8, s));
   DHS_TRY(bget(t, t->b_ph, (size_t)nchunks * pstride * 8, s));
   DHS_TRY(bget(t, t->b_pt, (size_t)nchunks * pstride * 8, s));
   DHS_TRY(bget(t, t->b_cflags, nchunks, s));
+  DHS_TRY(bget(t, t->b_owners, nchunks * 4, s));
   DHS_CUDA(cudaMemsetAsync(t->b_nbm.p, 0, t->b_nbm.bytes, s));
   t->ws_n = cap;
   return DHS_OK;
@@ -404,14 +417,15 @@ dhs_status dispatch_pool(dhs_table* t, const long long* keys, long long n, const
 
 dhs_status dispatch_seg(dhs_table* t, const unsigned* sk, const unsigned* sv, long long n,
                         const float* grad, long long nb, const OptArgs& oa, cudaStream_t s) {
-  const int G = pick_group(t->dim), NV = pick_nv(t->dim, G);
+  const int G = seg_group(t->dim), NV = seg_nv(t->dim);
   auto fn = t->opt == DHS_SGD ? launch_seg_sgd
             : t->opt == DHS_ADAGRAD ? launch_seg_adagrad
             : t->opt == DHS_ADAM ? launch_seg_adam
                                  : launch_seg_rowwise;
   const cudaError_t e = fn(G, NV, t->sm_count, sk, sv, n, grad, nb, t->dim, rowspace(t), oa,
                            (double*)t->b_ph.p, (double*)t->b_pt.p, (unsigned char*)t->b_cflags.p,
-                           seg_chunk(n), t->st, s);
+                           seg_chunk(n), (unsigned*)t->b_hist.p + kSegChunkCtrWord, (unsigned*)t->b_owners.p,
+                           (unsigned*)t->b_hist.p + kSegOwnerCtrWord, t->st, s);
   t->n_launches++;
   if (e != cudaSuccess) cudaGetLastError();
   return e == cudaSuccess ? DHS_OK : DHS_ERR_CUDA;
@@ -564,7 +578,8 @@ dhs_status ht_destroy(dhs_table* t) {
   dfree(t, t->blocks_d, sizeof(float*) * t->max_blocks, s);
   dfree(t, t->st, sizeof(DevState), s);
   Buf* bufs[] = {&t->b_nbm, &t->b_fbm, &t->b_gcnt, &t->b_gpref, &t->b_slotpos, &t->b_ka, &t->b_va,
-                 &t->b_kb, &t->b_vb, &t->b_hist, &t->b_totals, &t->b_ph, &t->b_pt, &t->b_cflags};
+                 &t->b_kb, &t->b_vb, &t->b_hist, &t->b_totals, &t->b_ph, &t->b_pt, &t->b_cflags,
+                 &t->b_owners};
   for (Buf* b : bufs) bfree(t, *b, s);
   cudaStreamSynchronize(s);
   for (auto& sn : t->snaps) {
@@ -716,8 +731,7 @@ dhs_status embbag_backward_update(dhs_table* t, const int64_t* d_keys, int64_t n
     const long long grid = grid_for((warps + 7) / 8, resident);
     bwd_probe_kernel<<<(unsigned)grid, 256, 0, s>>>(idmap(t), (const long long*)d_keys, n_keys,
                                                     (const long long*)d_bag_offsets, n_bags, ka, va,
-                                                    sentinel, (unsigned*)t->b_hist.p,
-                                                    kRadixMaxPasses * kRadixBins + kRadixMaxPasses,
+                                                    sentinel, (unsigned*)t->b_hist.p, kSortZeroWords,
                                                     t->st);
     t->n_launches++;
     DHS_TRY(last_launch());
@@ -757,16 +771,17 @@ dhs_status embbag_backward_update(dhs_table* t, const int64_t* d_keys, int64_t n
     oa.bc1 = (float)(1.0 - std::pow((double)t->b1, (double)t->adam_t));
     oa.bc2 = (float)(1.0 - std::pow((double)t->b2, (double)t->adam_t));
     DHS_TRY(dispatch_seg(t, ka, va, n_keys, d_grad, n_bags, oa, s));
-    const int G = pick_group(t->dim), NV = pick_nv(t->dim, G);
-    const int pstride = NV * G * 4;
+    const int pstride = seg_nv(t->dim) * seg_group(t->dim) * 4;
     const int chunk = seg_chunk(n_keys);
     const long long nchunks = (n_keys + chunk - 1) / chunk;
     const size_t smem = (size_t)std::max(256, t->dim) * sizeof(double);
-    const long long grid = std::min<long long>((nchunks + 255) / 256, (long long)t->sm_count * 8);
+    const long long grid = std::min<long long>(nchunks, (long long)t->sm_count * 4);
     bwd_combine_kernel<<<(unsigned)grid, 256, smem, s>>>(ka, n_keys, t->dim, rowspace(t), oa,
                                                         (const double*)t->b_ph.p, (const double*)t->b_pt.p,
                                                         (const unsigned char*)t->b_cflags.p, chunk,
-                                                        pstride, t->st);
+                                                        pstride, (const unsigned*)t->b_owners.p,
+                                                        (const unsigned*)t->b_hist.p + kSegOwnerCtrWord,
+                                                        t->st);
     t->n_launches++;
     DHS_TRY(last_launch());
   }
@@ -921,13 +936,15 @@ constexpr int kNoAllocMinChunk = 32;  // seg_chunk() never goes below this
 
 constexpr size_t na_align(size_t x) { return (x + 255) & ~size_t(255); }
 constexpr size_t kNaPairs = na_align(kNoAllocMaxKeys * 4);  // one of ka, va, kb, vb
-constexpr size_t kNaSortZero = na_align((kRadixMaxPasses * kRadixBins + kRadixMaxPasses) * 4);
+constexpr size_t kNaSortZero = na_align(kSortZeroWords * 4);
 constexpr size_t kNaStatus =
     na_align((size_t)kRadixMaxPasses * ((kNoAllocMaxKeys + kRadixTile - 1) / kRadixTile) * kRadixBins * 8);
 constexpr size_t kNaChunks = (kNoAllocMaxKeys + kNoAllocMinChunk - 1) / kNoAllocMinChunk;
 constexpr size_t kNaPart = na_align(kNaChunks * kNoAllocMaxDim * 8);  // one of part_head, part_tail
 constexpr size_t kNaFlags = na_align(kNaChunks);
-constexpr size_t kNoAllocScratchBytes = 4 * kNaPairs + kNaSortZero + kNaStatus + 2 * kNaPart + kNaFlags;
+constexpr size_t kNaOwners = na_align(kNaChunks * 4);
+constexpr size_t kNoAllocScratchBytes =
+    4 * kNaPairs + kNaSortZero + kNaStatus + 2 * kNaPart + kNaFlags + kNaOwners;
 
 // Every GPU that loads this library holds this array until the process exits.
 __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
@@ -985,6 +1002,7 @@ dhs_status embbag_backward_update_noalloc(dhs_table* t, const int64_t* d_keys, i
   double* part_head = (double*)(base + 4 * kNaPairs + kNaSortZero + kNaStatus);
   double* part_tail = (double*)(base + 4 * kNaPairs + kNaSortZero + kNaStatus + kNaPart);
   unsigned char* cflags = base + 4 * kNaPairs + kNaSortZero + kNaStatus + 2 * kNaPart;
+  unsigned* owners = (unsigned*)(base + 4 * kNaPairs + kNaSortZero + kNaStatus + 2 * kNaPart + kNaFlags);
 
   refresh_ub(t, false);
   const unsigned sentinel = (unsigned)t->rows_ub;
@@ -997,8 +1015,7 @@ dhs_status embbag_backward_update_noalloc(dhs_table* t, const int64_t* d_keys, i
     const long long grid = std::max<long long>(1, std::min<long long>((warps + 7) / 8, (long long)t->sm_count * 8));
     bwd_probe_kernel<<<(unsigned)grid, 256, 0, s>>>(idmap(t), (const long long*)d_keys, n_keys,
                                                     (const long long*)d_bag_offsets, n_bags, ka, va,
-                                                    sentinel, hist, kRadixMaxPasses * kRadixBins + kRadixMaxPasses,
-                                                    t->st);
+                                                    sentinel, hist, kSortZeroWords, t->st);
     DHS_TRY(last_launch());
   }
   const long long ntiles = (n_keys + kRadixTile - 1) / kRadixTile;
@@ -1027,22 +1044,23 @@ dhs_status embbag_backward_update_noalloc(dhs_table* t, const int64_t* d_keys, i
   oa.c2 = (float)(1.0 - (double)t->b2);
   oa.bc1 = (float)(1.0 - std::pow((double)t->b1, (double)t->adam_t));
   oa.bc2 = (float)(1.0 - std::pow((double)t->b2, (double)t->adam_t));
-  const int G = pick_group(t->dim), NV = pick_nv(t->dim, G);
+  const int G = seg_group(t->dim), NV = seg_nv(t->dim);
   const int chunk = seg_chunk(n_keys);
   auto fn = t->opt == DHS_SGD ? launch_seg_sgd
             : t->opt == DHS_ADAGRAD ? launch_seg_adagrad
             : t->opt == DHS_ADAM ? launch_seg_adam
                                  : launch_seg_rowwise;
   if (fn(G, NV, t->sm_count, ka, va, n_keys, d_grad, n_bags, t->dim, rowspace(t), oa, part_head, part_tail,
-         cflags, chunk, t->st, s) != cudaSuccess) {
+         cflags, chunk, hist + kSegChunkCtrWord, owners, hist + kSegOwnerCtrWord, t->st, s) != cudaSuccess) {
     cudaGetLastError();
     return DHS_ERR_CUDA;
   }
   const long long nchunks = (n_keys + chunk - 1) / chunk;
   const size_t smem = (size_t)std::max(256, t->dim) * sizeof(double);
-  const long long grid = std::min<long long>((nchunks + 255) / 256, (long long)t->sm_count * 8);
+  const long long grid = std::min<long long>(nchunks, (long long)t->sm_count * 4);
   bwd_combine_kernel<<<(unsigned)grid, 256, smem, s>>>(ka, n_keys, t->dim, rowspace(t), oa, part_head,
-                                                      part_tail, cflags, chunk, NV * G * 4, t->st);
+                                                      part_tail, cflags, chunk, NV * G * 4, owners,
+                                                      hist + kSegOwnerCtrWord, t->st);
   t->n_launches += 4 + passes;
   return last_launch();
 }

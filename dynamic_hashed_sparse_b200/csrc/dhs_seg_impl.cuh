@@ -15,7 +15,8 @@ template <int G, int NV, int OPT>
 cudaError_t run(int sm_count, const unsigned* skey, const unsigned* sval, long long n,
                 const float* grad, long long n_bags, int dim, RowSpace rs, const OptArgs& oa,
                 double* part_head, double* part_tail, unsigned char* cflags, int chunk,
-                DevState* st, cudaStream_t s) {
+                unsigned* chunk_ctr, unsigned* owners, unsigned* owner_ctr, DevState* st,
+                cudaStream_t s) {
   static int resident = 0;
   const size_t smem = seg_smem_bytes(G, NV);
   if (!resident) {
@@ -34,7 +35,8 @@ cudaError_t run(int sm_count, const unsigned* skey, const unsigned* sval, long l
   const long long need = std::max<long long>(1, (nchunks + per_block - 1) / per_block);
   const long long grid = std::min<long long>(need, resident);
   bwd_seg_kernel<G, NV, OPT><<<(unsigned)grid, 256, smem, s>>>(skey, sval, n, grad, n_bags, dim, rs, oa,
-                                                           part_head, part_tail, cflags, chunk, st);
+                                                              part_head, part_tail, cflags, chunk, chunk_ctr,
+                                                              owners, owner_ctr, st);
   return cudaGetLastError();
 }
 
@@ -42,16 +44,17 @@ template <int OPT>
 cudaError_t launch(int G, int NV, int sm_count, const unsigned* skey, const unsigned* sval,
                    long long n, const float* grad, long long n_bags, int dim, RowSpace rs,
                    const OptArgs& oa, double* part_head, double* part_tail, unsigned char* cflags,
-                   int chunk, DevState* st, cudaStream_t s) {
-#define DHS_RUN(g, v) \
-  run<g, v, OPT>(sm_count, skey, sval, n, grad, n_bags, dim, rs, oa, part_head, part_tail, cflags, chunk, st, s)
+                   int chunk, unsigned* chunk_ctr, unsigned* owners, unsigned* owner_ctr, DevState* st,
+                   cudaStream_t s) {
+#define DHS_RUN(g, v)                                                                                \
+  run<g, v, OPT>(sm_count, skey, sval, n, grad, n_bags, dim, rs, oa, part_head, part_tail, cflags, chunk, \
+                 chunk_ctr, owners, owner_ctr, st, s)
   switch (G * 100 + NV) {
-    case 101: return DHS_RUN(1, 1);
-    case 201: return DHS_RUN(2, 1);
-    case 401: return DHS_RUN(4, 1);
-    case 801: return DHS_RUN(8, 1);
-    case 1601: return DHS_RUN(16, 1);
-    case 3201: return DHS_RUN(32, 1);
+    case 102: return DHS_RUN(1, 2);
+    case 202: return DHS_RUN(2, 2);
+    case 402: return DHS_RUN(4, 2);
+    case 802: return DHS_RUN(8, 2);
+    case 1602: return DHS_RUN(16, 2);
     case 3202: return DHS_RUN(32, 2);
     case 3204: return DHS_RUN(32, 4);
   }
@@ -67,8 +70,10 @@ cudaError_t launch(int G, int NV, int sm_count, const unsigned* skey, const unsi
   cudaError_t NAME_(int G, int NV, int sm_count, const unsigned* skey, const unsigned* sval,     \
                     long long n, const float* grad, long long n_bags, int dim, RowSpace rs,      \
                     const OptArgs& oa, double* part_head, double* part_tail,                     \
-                    unsigned char* cflags, int chunk, DevState* st, cudaStream_t s) {            \
+                    unsigned char* cflags, int chunk, unsigned* chunk_ctr, unsigned* owners,     \
+                    unsigned* owner_ctr, DevState* st, cudaStream_t s) {                         \
     return seg_impl::launch<OPT_>(G, NV, sm_count, skey, sval, n, grad, n_bags, dim, rs, oa,     \
-                                  part_head, part_tail, cflags, chunk, st, s);                   \
+                                  part_head, part_tail, cflags, chunk, chunk_ctr, owners,        \
+                                  owner_ctr, st, s);                                             \
   }                                                                                              \
   }
