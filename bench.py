@@ -238,7 +238,7 @@ def run_reference(args):
     world, rank, _ = dist_env()
     if rank != 0:
         return 0
-    w = gen.full(args.workload)
+    w = make_workload(args.workload, 0, args.batch)
     frac = args.ref_frac
     ids, secs = time_oracle(w, args.warmup + args.steps, frac, timed_from=args.warmup)
     value = ids / secs if secs > 0 else 0.0
@@ -250,7 +250,7 @@ def run_reference(args):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * secs / max(1, args.steps),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f32", "data": "synthetic",
-        "config": workload_config(w),
+        "config": workload_config(w, 0, False),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": cpu_cores_used(), "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -259,19 +259,64 @@ def run_reference(args):
     return 0
 
 
-def workload_config(w) -> dict:
-    p = w.params
-    return {"workload": f"{w.name}: {p.get('tables', 1)} tables merged in one IDMap, batch {p.get('batch')} "
-                        f"samples x {p.get('tables')} ids (pooling 1), dim {w.dim} fp32, {w.optimizer} "
-                        f"lr {w.lr} eps {w.eps}, Zipf alpha {p.get('alpha')} per table, cardinalities "
-                        f"log-uniform in [1e3, 1e7]",
-            "ids_per_step": int(p.get("batch", 0)) * int(p.get("tables", 1)),
-            "batch": int(p.get("batch", 0)),
-            "bags_per_step": int(p.get("batch", 0)) * int(p.get("tables", 1)),
+L2_BYTES = 126 << 20
+
+DESCRIPTIONS = {
+    "tiny_uniform": "1024 bags x 1 id drawn uniformly from 65,536 distinct keys in [0, 2^40), one table, "
+                    "dim 16 fp32, SGD lr 0.01",
+    "dlrm_merged_26": "26 tables merged in one IDMap, {batch} samples x 26 ids (pooling 1), Zipf 1.05 per "
+                      "table over log-uniform [1e3, 1e7] cardinalities, dim 128 fp32, Adagrad lr 0.01 eps 1e-8",
+    "sequence_bags": "16,384 samples x 8 tables, bag length min(Poisson(50), 200), 20% of ids never seen "
+                     "before, the rest Zipf 1.2 over 1e6 ranks per table, dim 64 fp32, SGD lr 0.05",
+    "growth_stream": "one table from empty, 131,072 bags x 4 ids, 30% never-seen ids per step, the rest "
+                     "uniform over inserted ids, dim 32 fp32, Adam lr 1e-3 (b1 0.9, b2 0.999), blocks of 2^20 rows",
+    "hot_key": "5e7 keys pre-inserted (untimed), 262,144 bags x 20 ids, Zipf 1.4 over them, dim 64 fp32, "
+               "Adagrad lr 0.01 eps 1e-8",
+}
+
+
+def make_workload(name: str, rank: int = 0, batch: int = 0):
+    """The named workload; replicas (rank > 0) draw their own streams."""
+    if name == "dlrm_merged_26":
+        return gen.DlrmMerged(seed=1002 + 7919 * rank, batch=batch or 65536)
+    w = gen.full(name)
+    w.seed += 7919 * rank
+    return w
+
+
+def default_reserve(w, steps: int) -> int:
+    """Keys the stream holds after `steps` steps plus one batch of new keys."""
+    if w.name == "tiny_uniform":
+        return 65536
+    if w.name == "dlrm_merged_26":
+        return 6_000_000
+    if w.name == "sequence_bags":
+        return int(8e6 + (steps + 1) * 1.4e6)
+    if w.name == "growth_stream":
+        return w.inserted_before(steps) + 2 * 524288
+    return int(w.params["rows"]) + 1
+
+
+def workload_config(w, reserve: int, flush: bool) -> dict:
+    return {"workload": f"{w.name}: " + DESCRIPTIONS[w.name].format(batch=w.params.get("batch")),
             "dim": w.dim, "optimizer": w.optimizer,
-            "l2": "inputs larger than L2 (per-step gradients 872 MB, keys 13.6 MB; 126 MB L2)",
-            "table": "starts empty (capacity for 6M keys reserved before step 0 unless --reserve-keys "
-                     "says otherwise); warm-up = the stream's first steps"}
+            "l2": ("L2 flushed (512 MB written) before each timed step; each step is timed on its own"
+                   if flush else "inputs larger than L2 (per-step gradients and ids exceed 2 x 126 MB)"),
+            "table": f"starts as the workload defines it; capacity for {reserve} keys reserved before step 0; "
+                     "warm-up = the stream's first steps"}
+
+
+def setup_table(dhs, w, reserve: int):
+    """A table for the workload, capacity reserved and any pre-insertion done."""
+    import torch
+    t = dhs.ht_create(w.dim, w.optimizer, block_rows=w.block_rows, eps=w.eps, beta1=w.beta1, beta2=w.beta2)
+    if reserve:
+        dhs.ht_reserve(t, reserve)
+    for tids, ids in w.preinsert():
+        keys = dhs.dhs_pack_keys(torch.from_numpy(tids).cuda(), torch.from_numpy(ids).cuda())
+        dhs.ht_lookup_or_insert(t, keys)
+    torch.cuda.synchronize()
+    return t
 
 
 # ---------------------------------------------------------------------------
@@ -285,25 +330,27 @@ def run_dhs(args):
     dist = init_dist(world, "nccl")
     import dynamic_hashed_sparse_b200 as dhs
 
-    if args.workload == WORKLOAD:
-        w = gen.DlrmMerged(seed=1002 + 7919 * rank, batch=args.batch or 65536)
-    else:
-        w = gen.full(args.workload)
+    w = make_workload(args.workload, rank, args.batch)
     total = args.warmup + args.steps
+    reserve = default_reserve(w, total) if args.reserve_keys < 0 else args.reserve_keys
     # inputs for every step, resident in HBM before the timed region
     batches = []
     for s in range(total):
         b = w.batch(s)
         batches.append((torch.from_numpy(b.table_ids).to(device), torch.from_numpy(b.ids).to(device),
                         torch.from_numpy(b.bag_offsets).to(device), b.n, b.n_bags))
+    n_max = max(x[3] for x in batches)
+    nb_max = max(x[4] for x in batches)
     n_grad = min(total, args.grad_buffers)
-    grads = [w.torch_grads(s, batches[s][4], device) for s in range(n_grad)]
-    pooled = torch.empty((batches[0][4], w.dim), dtype=torch.float32, device=device)
-    keys = torch.empty(batches[0][3], dtype=torch.int64, device=device)
+    grads = [w.torch_grads(s, nb_max, device) for s in range(n_grad)]
+    pooled = torch.empty((nb_max, w.dim), dtype=torch.float32, device=device)
+    keys = torch.empty(max(1, n_max), dtype=torch.int64, device=device)
+    # a step whose inputs fit in twice the L2 gets the L2 flushed before it
+    step_bytes = n_max * 12 + (nb_max + 1) * 8 + nb_max * w.dim * 4
+    flush = step_bytes < 2 * L2_BYTES
+    fbuf = torch.empty(512 << 20, dtype=torch.uint8, device=device) if flush else None
 
-    t = dhs.ht_create(w.dim, w.optimizer, block_rows=w.block_rows, eps=w.eps, beta1=w.beta1, beta2=w.beta2)
-    if args.reserve_keys:
-        dhs.ht_reserve(t, args.reserve_keys)
+    t = setup_table(dhs, w, reserve)
     stream = torch.cuda.current_stream()
 
     def step(s):
@@ -311,7 +358,7 @@ def run_dhs(args):
         k = keys[:n]
         dhs.dhs_pack_keys(tids, ids, out=k)
         dhs.embbag_forward(t, k, offs, out=pooled[:nb])
-        dhs.embbag_backward_update(t, k, offs, grads[s % n_grad], w.lr)
+        dhs.embbag_backward_update(t, k, offs, grads[s % n_grad][:nb], w.lr)
 
     for s in range(args.warmup):
         step(s)
@@ -319,18 +366,29 @@ def run_dhs(args):
     c0 = dhs.ht_counters(t)
     dhs.ht_phase_times(t)  # clear
     dhs.ht_set_phase_timing(t, True)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(dist, device)
     torch.cuda.synchronize()
+    spans = []
     with ClockSampler(local) as clk:
-        e0.record(stream)
-        for s in range(args.warmup, total):
-            step(s)
-        e1.record(stream)
+        if not flush:
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for s in range(args.warmup, total):
+                step(s)
+            e1.record(stream)
+            spans.append((e0, e1))
+        else:
+            for s in range(args.warmup, total):
+                fbuf.zero_()
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                step(s)
+                e1.record(stream)
+                spans.append((e0, e1))
         torch.cuda.synchronize()
     barrier(dist, device)
     dhs.ht_set_phase_timing(t, False)
-    ms_local = e0.elapsed_time(e1)
+    ms_local = sum(a.elapsed_time(b) for a, b in spans)
     phases = dhs.ht_phase_times(t)
     c1 = dhs.ht_counters(t)
     status = dhs.ht_sync(t)
@@ -359,7 +417,7 @@ def run_dhs(args):
     dom_launch_ms = ph_ms[dom] / max(1, ph_cnt[dom])
     dom_bytes_per_launch = dom_bytes / max(1, ph_cnt[dom])
     achieved = dom_bytes_per_launch / (dom_launch_ms / 1e3) / 1e9
-    traffic = load_traffic(dom_kernel)
+    traffic = load_traffic(dom_kernel) if w.name == "dlrm_merged_26" else None
     roofline = {
         "bound": "hbm", "kernel": dom_kernel, "achieved": achieved, "peak": peaks["hbm_gbs"],
         "peak_source": peaks["source"], "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
@@ -368,24 +426,27 @@ def run_dhs(args):
         "alg_bytes_per_launch": dom_bytes_per_launch, "launch_ms": dom_launch_ms,
     }
 
+    def gbs(nbytes, t_ms):
+        return nbytes / (t_ms / 1e3) / 1e9 if t_ms else None
+
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
         "ms_per_step": ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "timing_valid": args.warmup >= 3,
-        "dtype": "f32", "data": "synthetic", "config": workload_config(w),
+        "dtype": "f32", "data": "synthetic", "config": workload_config(w, reserve, flush),
         "fwd": {"ids_per_s": n_ids / (fwd_ms / 1e3) if fwd_ms else None, "ms_per_step": fwd_ms / K,
-                "gbs": ab["fwd"] / (fwd_ms / 1e3) / 1e9 if fwd_ms else None,
-                "frac_of_peak": ab["fwd"] / (fwd_ms / 1e3) / 1e9 / peaks["hbm_gbs"] if fwd_ms else None},
+                "gbs": gbs(ab["fwd"], fwd_ms),
+                "frac_of_peak": gbs(ab["fwd"], fwd_ms) / peaks["hbm_gbs"] if fwd_ms else None},
         "bwd": {"ids_per_s": n_ids / (bwd_ms / 1e3) if bwd_ms else None, "ms_per_step": bwd_ms / K,
-                "gbs": ab["bwd"] / (bwd_ms / 1e3) / 1e9 if bwd_ms else None,
-                "frac_of_peak": ab["bwd"] / (bwd_ms / 1e3) / 1e9 / peaks["hbm_gbs"] if bwd_ms else None},
-        "step_gbs": (ab["fwd"] + ab["bwd"]) / (ms_local / 1e3) / 1e9,
+                "gbs": gbs(ab["bwd"], bwd_ms),
+                "frac_of_peak": gbs(ab["bwd"], bwd_ms) / peaks["hbm_gbs"] if bwd_ms else None},
+        "step_gbs": gbs(ab["fwd"] + ab["bwd"], ms_local),
         "phases_ms_per_step": {k: v / K for k, v in ph_ms.items() if ph_cnt[k]},
         "per_step": {"ids": n_ids / K, "bags": n_bags / K, "unique": U / K, "new": M / K},
         "roofline": roofline,
         "gpu_launches": launches,
         "table": {"rows": c1["rows"], "slots": c1["slots"], "blocks": c1["blocks"], "rehashes": c1["rehashes"],
-                  "reserved_keys": args.reserve_keys,
+                  "reserved_keys": reserve,
                   "timed_growth": {"rehashes": c1["rehashes"] - c0["rehashes"],
                                    "blocks_appended": c1["blocks"] - c0["blocks"],
                                    "device_allocs": c1["allocs"] - c0["allocs"],
@@ -393,16 +454,17 @@ def run_dhs(args):
     }
     line["clocks"] = clk.summary()
     t.close()
-    del grads, batches
+    del grads, batches, fbuf
     torch.cuda.empty_cache()
 
     if not args.no_e2e:
-        line["e2e"] = run_e2e(args, w, device, dist)
+        line["e2e"] = run_e2e(args, w, device, dist, reserve)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        ids, secs = time_oracle(gen.full(args.workload), args.cpu_steps, 1.0)
+        ids, secs = time_oracle(make_workload(args.workload, 0, args.batch), args.cpu_steps, args.cpu_frac)
         line["cpu_baseline"] = {"value": ids / secs, "unit": UNIT, "cores": cpu_cores_used(), "kind": "oracle",
-                                "sample": f"steps 0..{args.cpu_steps - 1} of {w.name}, full batches "
-                                          f"({ids} ids, {secs:.1f} s), oracle single-threaded"}
+                                "sample": f"steps 0..{args.cpu_steps - 1} of {w.name}, first {args.cpu_frac:g} "
+                                          f"of each batch's bags ({ids} ids, {secs:.1f} s), oracle "
+                                          "single-threaded, no pre-inserted keys"}
     if dist is not None:
         dist.destroy_process_group()
     if rank == 0:
@@ -410,7 +472,7 @@ def run_dhs(args):
     return 0
 
 
-def run_e2e(args, w, device, dist):
+def run_e2e(args, w, device, dist, reserve):
     """The same step through the public API with host inputs: per step, copy
     the ids, table ids, bag offsets and gradients from pinned host memory,
     run the step, and copy the pooled output back; all inside the timed
@@ -424,20 +486,18 @@ def run_e2e(args, w, device, dist):
         b = w.batch(s)
         hb.append((torch.from_numpy(b.table_ids).pin_memory(), torch.from_numpy(b.ids).pin_memory(),
                    torch.from_numpy(b.bag_offsets).pin_memory(), b.n, b.n_bags))
-    nb0 = hb[0][4]
+    n_max = max(x[3] for x in hb)
+    nb_max = max(x[4] for x in hb)
     n_grad = 2
-    hgrads = [w.torch_grads(s, nb0, device).cpu().pin_memory() for s in range(n_grad)]
-    hpooled = torch.empty((nb0, w.dim), dtype=torch.float32).pin_memory()
-    n0 = hb[0][3]
-    d_tids = torch.empty(n0, dtype=torch.int32, device=device)
-    d_ids = torch.empty(n0, dtype=torch.int64, device=device)
-    d_keys = torch.empty(n0, dtype=torch.int64, device=device)
-    d_offs = torch.empty(nb0 + 1, dtype=torch.int64, device=device)
-    d_grad = torch.empty((nb0, w.dim), dtype=torch.float32, device=device)
-    d_pooled = torch.empty((nb0, w.dim), dtype=torch.float32, device=device)
-    t = dhs.ht_create(w.dim, w.optimizer, block_rows=w.block_rows, eps=w.eps, beta1=w.beta1, beta2=w.beta2)
-    if args.reserve_keys:
-        dhs.ht_reserve(t, args.reserve_keys)
+    hgrads = [w.torch_grads(s, nb_max, device).cpu().pin_memory() for s in range(n_grad)]
+    hpooled = torch.empty((nb_max, w.dim), dtype=torch.float32).pin_memory()
+    d_tids = torch.empty(max(1, n_max), dtype=torch.int32, device=device)
+    d_ids = torch.empty(max(1, n_max), dtype=torch.int64, device=device)
+    d_keys = torch.empty(max(1, n_max), dtype=torch.int64, device=device)
+    d_offs = torch.empty(nb_max + 1, dtype=torch.int64, device=device)
+    d_grad = torch.empty((nb_max, w.dim), dtype=torch.float32, device=device)
+    d_pooled = torch.empty((nb_max, w.dim), dtype=torch.float32, device=device)
+    t = setup_table(dhs, w, reserve)
     h2d = d2h = 0
 
     def step(s):
@@ -491,8 +551,11 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-steps", type=int, default=5)
     ap.add_argument("--ref-frac", type=float, default=1.0 / 16)
-    ap.add_argument("--reserve-keys", type=int, default=6_000_000,
-                    help="capacity reserved (ht_reserve) before step 0; 0 = grow on demand")
+    ap.add_argument("--reserve-keys", type=int, default=-1,
+                    help="capacity reserved (ht_reserve) before step 0; -1 = what the workload reaches in "
+                         "the run plus one batch; 0 = grow on demand")
+    ap.add_argument("--cpu-frac", type=float, default=1.0,
+                    help="fraction of each batch's bags the CPU-baseline oracle processes")
     ap.add_argument("--batch", type=int, default=0,
                     help="samples per step (default: the workload's 65,536); smaller only for profiling")
     args = ap.parse_args(argv)

@@ -120,10 +120,13 @@ constexpr unsigned long long kLbCountMask = (1ull << 62) - 1;
 constexpr unsigned kLookbackSpins = 1u << 22;  // bounded wait for a predecessor tile
 // words cleared by bwd_probe_kernel before a backward: digit histograms of
 // every pass, one tile counter per pass, the segment kernel's chunk counter
-// and the count of long-segment owner chunks
-constexpr int kSortZeroWords = kRadixMaxPasses * kRadixBins + kRadixMaxPasses + 2;
+// the count of long-segment owner chunks and the combine's batch and slot
+// counters
+constexpr int kSortZeroWords = kRadixMaxPasses * kRadixBins + kRadixMaxPasses + 4;
 constexpr int kSegChunkCtrWord = kRadixMaxPasses * kRadixBins + kRadixMaxPasses;
 constexpr int kSegOwnerCtrWord = kSegChunkCtrWord + 1;
+constexpr int kCombineBatchCtrWord = kSegChunkCtrWord + 2;
+constexpr int kCombineSlotCtrWord = kSegChunkCtrWord + 3;
 
 // Digit counts of every pass in one read of the keys (global atomics, one per
 // block and bin), and the look-back state of every pass cleared.  hist and
@@ -350,7 +353,6 @@ __device__ __forceinline__ void update_col(float* row, int dim, int j, float g, 
 // ---------------------------------------------------------------------------
 // segment reduce + update
 // ---------------------------------------------------------------------------
-enum : unsigned char { kPieceHead = 1, kPieceThrough = 2, kPieceTailStart = 4 };
 
 // The part of one row a lane owns: float4 columns gl + q*G (q < NV) of the
 // weights and of each per-element state array (Adagrad: G; Adam: m, v), plus
@@ -455,7 +457,7 @@ __global__ void __launch_bounds__(256, NV <= 2 ? DHS_SEG_MINB : 1)
 bwd_seg_kernel(const unsigned* __restrict__ skey, const unsigned* __restrict__ sval, long long n,
                const float* __restrict__ grad, long long n_bags, int dim, RowSpace rs, OptArgs oa,
                double* __restrict__ part_head, double* __restrict__ part_tail,
-               unsigned char* __restrict__ cflags, int C, unsigned* __restrict__ chunk_ctr,
+               int C, unsigned* __restrict__ chunk_ctr,
                unsigned* __restrict__ owners, unsigned* __restrict__ owner_ctr, DevState* st) {
   constexpr int R = seg_ring(NV);
   extern __shared__ float4 seg_ring_smem[];
@@ -487,7 +489,6 @@ bwd_seg_kernel(const unsigned* __restrict__ skey, const unsigned* __restrict__ s
     const int start = c * C;
     const int end = min(n32, start + C);
     const int limit = min(n32, end + C);  // an owned segment ends before chunk c + 2
-    unsigned char flags = 0;
     unsigned nseg = 0;
 
     // the keys that decide who owns the chunk's first and last pieces
@@ -548,14 +549,13 @@ bwd_seg_kernel(const unsigned* __restrict__ skey, const unsigned* __restrict__ s
 #pragma unroll
       for (int e = 0; e < 4; ++e) acc[q][e] = 0.0;
 
-    auto close_piece = [&](bool cont) {
+    auto close_piece = [&]() {
       if (mode == 1 || mode == 3) {
         double* o = (mode == 1 ? part_head : part_tail) + (long long)c * pstride;
 #pragma unroll
         for (int q = 0; q < NV; ++q)
 #pragma unroll
           for (int e = 0; e < 4; ++e) o[(q * G + gl) * 4 + e] = acc[q][e];
-        flags |= mode == 3 ? kPieceTailStart : (cont ? kPieceThrough : kPieceHead);
         if (mode == 3 && gl == 0) owners[atomicAdd(owner_ctr, 1u)] = (unsigned)c;  // for the combine
       } else if (mode == 2 && cur < nrows) {
         double sq = 0.0;
@@ -589,7 +589,7 @@ bwd_seg_kernel(const unsigned* __restrict__ skey, const unsigned* __restrict__ s
       }
       const unsigned kt = __shfl_sync(gmask, ck, i - cws, G);
       if (kt != cur) {
-        close_piece(false);
+        close_piece();
         if (i >= end) {
           done = true;
           break;
@@ -599,7 +599,7 @@ bwd_seg_kernel(const unsigned* __restrict__ skey, const unsigned* __restrict__ s
         mode = (has2 && fwd2 == cur) ? 3 : 2;
         if (mode == 2 && cur < nrows) rb.load(rs.row(cur), dim, gl, G);
       } else if (i == end && mode != 2) {
-        close_piece(true);  // a long piece stops at the chunk end
+        close_piece();  // a long piece stops at the chunk end
         done = true;
         break;
       }
@@ -617,10 +617,9 @@ bwd_seg_kernel(const unsigned* __restrict__ skey, const unsigned* __restrict__ s
       }
       produce();  // refill the slot just read with pair i + R
     }
-    if (!done) close_piece(false);  // reached the end of the array with a piece open
+    if (!done) close_piece();  // reached the end of the array with a piece open
     cp_async_wait_all();  // the ring is reused by the next chunk
     if (gl == 0) {
-      cflags[c] = flags;
       if (cur >= nrows && nseg) --nseg;  // the missing-key run is not a row
       nseg_total += nseg;
     }
@@ -629,83 +628,161 @@ bwd_seg_kernel(const unsigned* __restrict__ skey, const unsigned* __restrict__ s
 }
 
 #ifndef DHS_TEMPLATES_ONLY
-// One thread block per long segment (the owner chunks the segment kernel
-// listed): find the run of partials (through pieces up to the first head
-// piece), sum them in fp64 in a fixed order, and apply the optimizer to the
-// row.
+// Long segments (the owner chunks the segment kernel listed) are finished in
+// two launches.  Plan: one warp per owner finds the chunk holding the
+// segment's last pair (the first pairs of the run's chunks all carry the key;
+// keys are sorted, so a 32-way search over chunk starts finds the last one),
+// cuts the run's pieces (the owner's starting partial, then one head piece
+// per following chunk) into batches of kCombinePieces and takes batch ids
+// (and, for runs of more than one batch, fp64 slots) from counters.
+// Combine: one block per batch adds its pieces in fp64; a one-batch run
+// updates its row directly, otherwise the batch stores its sum in its slot and
+// the last of the run's batches to finish (an atomic ticket; no block waits)
+// adds the slots in batch order and applies the optimizer once.  Every sum is
+// taken in an order fixed by the run alone.
+constexpr int kCombineThreads = 256;
+constexpr int kCombinePieces = 128;
+
+struct CombinePlan {
+  unsigned* kend;         // [owners] chunk holding the last pair
+  unsigned* boff;         // [owners] first batch id
+  unsigned* sbase;        // [owners] first slot (runs of more than one batch)
+  unsigned* ticket;       // [owners] batches finished
+  unsigned* batch_owner;  // [batch_cap] owner of each batch id
+  double* slots;          // [slot_cap][pstride]
+  unsigned batch_cap, slot_cap;
+  unsigned* batch_ctr;    // zeroed before the segment kernel
+  unsigned* slot_ctr;
+};
+
 __global__ void __launch_bounds__(256)
-bwd_combine_kernel(const unsigned* __restrict__ skey, long long n, int dim, RowSpace rs,
-                   OptArgs oa, const double* __restrict__ part_head,
-                   const double* __restrict__ part_tail, const unsigned char* __restrict__ cflags,
-                   int C, int pstride, const unsigned* __restrict__ owners,
-                   const unsigned* __restrict__ owner_ctr, DevState* st) {
-  extern __shared__ double sacc[];  // [slices][dim]
-  __shared__ long long s_end;
-  __shared__ double s_sq;
+bwd_combine_plan_kernel(const unsigned* __restrict__ skey, long long n, int C,
+                        const unsigned* __restrict__ owners, const unsigned* __restrict__ owner_ctr,
+                        CombinePlan pl, DevState* st) {
+  const int lane = threadIdx.x & 31;
   const long long nchunks = (n + C - 1) / C;
   const unsigned long long nrows = st->row_count;
-  const int T = blockDim.x;
-  const int slices = dim >= T ? 1 : T / dim;
   const unsigned n_own = *owner_ctr;
-  for (unsigned oi = blockIdx.x; oi < n_own; oi += gridDim.x) {
+  const long long warps = (long long)gridDim.x * (blockDim.x >> 5);
+  for (long long oi = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); oi < n_own;
+       oi += warps) {
     const long long c = owners[oi];
     const unsigned key = skey[(c + 1) * (long long)C - 1];
-    // the run ends at the first chunk after c whose piece is a head piece
-    if (threadIdx.x == 0) s_end = nchunks - 1;
-    __syncthreads();
-    for (long long b = c + 1; b < nchunks; b += T) {
-      const long long k = b + threadIdx.x;
-      const bool is_end = k < nchunks && (cflags[k] & kPieceHead);
-      const unsigned any = __syncthreads_or(is_end);
-      if (is_end) atomicMin((unsigned long long*)&s_end, (unsigned long long)k);
-      __syncthreads();
-      if (any) break;
+    long long lo = c + 1, hi = nchunks - 1;  // the last chunk is in [lo, hi]; chunk c + 1 is in the run
+    while (lo < hi) {
+      const long long stride = (hi - lo + 32) / 32;
+      const long long kk = lo + lane * stride;
+      const unsigned in_run = __ballot_sync(0xffffffffu, kk <= hi && skey[kk * C] == key);
+      lo += (long long)(31 - __clz(in_run)) * stride;  // lane 0 (chunk lo) is always in the run
+      hi = min(hi, lo + stride - 1);
+      if (stride == 1) break;
     }
-    const long long kend = s_end;
-    // sums: slice s adds pieces s, s + slices, ... (piece 0 = starting partial)
-    const long long npieces = kend - c + 1;
+    const long long npieces = lo - c + 1;
+    const unsigned nb = key < nrows ? (unsigned)((npieces + kCombinePieces - 1) / kCombinePieces) : 0u;
+    unsigned base = 0, sb = 0;
+    if (lane == 0) {
+      base = atomicAdd(pl.batch_ctr, nb);
+      if (nb > 1) sb = atomicAdd(pl.slot_ctr, nb);
+      if (base + nb > pl.batch_cap || (nb > 1 && sb + nb > pl.slot_cap)) {
+        latch(st, kErrInternal);  // the caps bound every run of sorted input
+        base = pl.batch_cap;
+      }
+      pl.kend[oi] = (unsigned)lo;
+      pl.boff[oi] = base;
+      pl.sbase[oi] = sb;
+      pl.ticket[oi] = 0u;
+    }
+    base = __shfl_sync(0xffffffffu, base, 0);
+    for (unsigned j = lane; j < nb && base + j < pl.batch_cap; j += 32) pl.batch_owner[base + j] = (unsigned)oi;
+  }
+}
+
+__global__ void __launch_bounds__(kCombineThreads)
+bwd_combine_kernel(const unsigned* __restrict__ skey, int dim, RowSpace rs, OptArgs oa,
+                   const double* __restrict__ part_head, const double* __restrict__ part_tail, int C,
+                   int pstride, const unsigned* __restrict__ owners,
+                   const unsigned* __restrict__ owner_ctr, CombinePlan pl) {
+  extern __shared__ double sacc[];  // [slices][dim]
+  __shared__ double s_sq;
+  __shared__ bool s_last;
+  const int T = blockDim.x;
+  const int slices = dim >= T ? 1 : T / dim;
+  const unsigned nbatch = min(*pl.batch_ctr, pl.batch_cap);
+  const unsigned n_own = *owner_ctr;
+  for (unsigned bid = blockIdx.x; bid < nbatch; bid += gridDim.x) {
+    const unsigned oi = pl.batch_owner[bid];
+    if (oi >= n_own) continue;  // only after a plan overflow, which the plan reported
+    const long long c = owners[oi];
+    const unsigned key = skey[(c + 1) * (long long)C - 1];
+    const long long npieces = (long long)pl.kend[oi] - c + 1;
+    const unsigned b = bid - pl.boff[oi];
+    const unsigned nb = (unsigned)((npieces + kCombinePieces - 1) / kCombinePieces);
+    if (b >= nb) continue;
+    const long long p0 = (long long)b * kCombinePieces;
+    const long long p1 = min(npieces, p0 + kCombinePieces);
+    // slice sl adds pieces p0 + sl, p0 + sl + slices, ... (piece 0 = starting partial)
     for (int j0 = 0; j0 < dim; j0 += (slices == 1 ? T : dim)) {
       const int sl = slices == 1 ? 0 : threadIdx.x / dim;
       const int j = slices == 1 ? j0 + threadIdx.x : threadIdx.x % dim;
       if (sl < slices && j < dim) {
-        double a = 0.0;
-        for (long long pc = sl; pc < npieces; pc += slices) {
+        auto piece = [&](long long pc) -> double {
           const double* src = pc == 0 ? part_tail + c * (long long)pstride
                                       : part_head + (c + pc) * (long long)pstride;
-          a += src[j];
+          return __ldcg(src + j);
+        };
+        double a[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+        long long pc = p0 + sl;
+        for (; pc + 7LL * slices < p1; pc += 8LL * slices) {
+#pragma unroll
+          for (int u = 0; u < 8; ++u) a[u] += piece(pc + (long long)u * slices);
         }
-        sacc[sl * dim + j] = a;
+        for (; pc < p1; pc += slices) a[0] += piece(pc);
+        sacc[sl * dim + j] = ((a[0] + a[1]) + (a[2] + a[3])) + ((a[4] + a[5]) + (a[6] + a[7]));
       }
       if (slices != 1) break;
     }
     __syncthreads();
-    // fold slices in order into slice 0
     for (int j = threadIdx.x; j < dim && slices > 1; j += T) {
       double a = sacc[j];
       for (int s2 = 1; s2 < slices; ++s2) a += sacc[s2 * dim + j];
       sacc[j] = a;
     }
     __syncthreads();
-    if (key < nrows) {
-      float* row = rs.row(key);
-      float den = 0.f;
-      if (oa.opt == 3) {
-        if (threadIdx.x == 0) {
-          double sq = 0.0;
-          for (int j = 0; j < dim; ++j) {
-            const double g = (double)(float)sacc[j];
-            sq += g * g;
-          }
-          s_sq = sq;
-        }
-        __syncthreads();
-        const float Gn = __fadd_rn(row[dim], (float)(s_sq / (double)dim));
-        den = __fadd_rn(__fsqrt_rn(Gn), oa.eps);
-        __syncthreads();
-        if (threadIdx.x == 0) row[dim] = Gn;
+    if (nb > 1) {
+      double* mine = pl.slots + (size_t)(pl.sbase[oi] + b) * pstride;
+      for (int j = threadIdx.x; j < dim; j += T) mine[j] = sacc[j];
+      __threadfence();
+      __syncthreads();
+      if (threadIdx.x == 0) s_last = atomicAdd(&pl.ticket[oi], 1u) == nb - 1u;
+      __syncthreads();
+      if (!s_last) continue;  // uniform across the block
+      __threadfence();
+      const double* all = pl.slots + (size_t)pl.sbase[oi] * pstride;
+      for (int j = threadIdx.x; j < dim; j += T) {
+        double a = 0.0;
+        for (unsigned k = 0; k < nb; ++k) a += __ldcg(all + (size_t)k * pstride + j);
+        sacc[j] = a;
       }
-      for (int j = threadIdx.x; j < dim; j += T) update_col(row, dim, j, (float)sacc[j], oa, den);
+      __syncthreads();
     }
+    float* row = rs.row(key);  // the plan gives no batch to a missing-key run
+    float den = 0.f;
+    if (oa.opt == 3) {
+      if (threadIdx.x == 0) {
+        double sq = 0.0;
+        for (int j = 0; j < dim; ++j) {
+          const double g = (double)(float)sacc[j];
+          sq += g * g;
+        }
+        s_sq = sq;
+      }
+      __syncthreads();
+      const float Gn = __fadd_rn(row[dim], (float)(s_sq / (double)dim));
+      den = __fadd_rn(__fsqrt_rn(Gn), oa.eps);
+      __syncthreads();
+      if (threadIdx.x == 0) row[dim] = Gn;
+    }
+    for (int j = threadIdx.x; j < dim; j += T) update_col(row, dim, j, (float)sacc[j], oa, den);
     __syncthreads();
   }
 }

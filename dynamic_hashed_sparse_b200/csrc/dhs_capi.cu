@@ -34,7 +34,10 @@ constexpr double kMaxLoad = 0.5;
 // Sort chunk of the segment-reduce kernel: big enough that a group's fixed
 // work per chunk stays small, small enough that every SM gets many chunks.
 int seg_chunk(long long n) {
-  return n > 4000000 ? 256 : n > 500000 ? 128 : n > 100000 ? 64 : 32;
+#ifdef DHS_SEG_CHUNK_FIXED  // tuning override (a power of two >= 32)
+  if (n > 100000) return DHS_SEG_CHUNK_FIXED;
+#endif
+  return n > 100000 ? 64 : 32;
 }
 constexpr int kSnapRing = 4;
 enum { PH_FWD_POOL = 0, PH_FWD_ASSIGN = 1, PH_BWD_PROBE = 2, PH_BWD_SORT = 3, PH_BWD_SEG = 4,
@@ -128,8 +131,9 @@ struct dhs_table {
 
   // workspace, sized for ws_n positions
   long long ws_n = -1;
+  long long ws_chunks = 0;  // chunk capacity of the segment and combine buffers
   Buf b_nbm, b_fbm, b_gcnt, b_gpref, b_slotpos, b_ka, b_va, b_kb, b_vb, b_hist, b_totals, b_ph,
-      b_pt, b_cflags, b_owners;
+      b_pt, b_owners, b_cplan, b_slots;
 
   bool timing = false;
   std::vector<PhaseRec> recs;
@@ -371,6 +375,32 @@ dhs_status ensure_capacity(dhs_table* t, long long n, cudaStream_t s) {
   return DHS_OK;
 }
 
+// Capacities of the long-segment combine for a workspace of `nchunks` chunks.
+// Owner chunks are at least two apart (a long segment reaches two chunks past
+// its owner), so there are at most nchunks / 2 + 1 of them; the runs overlap
+// in at most one chunk, so their pieces add up to at most 1.5 nchunks + 1.
+// Batch ids: one per run plus pieces / kCombinePieces.  Slots: only runs of
+// more than kCombinePieces pieces take them, fewer than two per
+// kCombinePieces of their pieces.
+constexpr long long combine_batch_cap(long long nchunks) { return nchunks / 2 + 2 * nchunks / kCombinePieces + 64; }
+constexpr long long combine_slot_cap(long long nchunks) { return 4 * nchunks / kCombinePieces + 64; }
+
+// The plan arrays cut from one buffer of 4 nchunks + batch cap words.
+CombinePlan combine_plan(unsigned* words, double* slots, long long nchunks, unsigned* zeroed) {
+  CombinePlan pl;
+  pl.kend = words;
+  pl.boff = words + nchunks;
+  pl.sbase = words + 2 * nchunks;
+  pl.ticket = words + 3 * nchunks;
+  pl.batch_owner = words + 4 * nchunks;
+  pl.slots = slots;
+  pl.batch_cap = (unsigned)combine_batch_cap(nchunks);
+  pl.slot_cap = (unsigned)combine_slot_cap(nchunks);
+  pl.batch_ctr = zeroed + kCombineBatchCtrWord;
+  pl.slot_ctr = zeroed + kCombineSlotCtrWord;
+  return pl;
+}
+
 dhs_status ensure_ws(dhs_table* t, long long n, cudaStream_t s) {
   if (n <= t->ws_n) return DHS_OK;
   long long cap = std::max<long long>(n, t->ws_n > 0 ? t->ws_n + t->ws_n / 2 : 0);
@@ -394,14 +424,33 @@ dhs_status ensure_ws(dhs_table* t, long long n, cudaStream_t s) {
   DHS_TRY(bget(t, t->b_totals, (size_t)kRadixMaxPasses * ntiles * kRadixBins * 8, s));
   DHS_TRY(bget(t, t->b_ph, (size_t)nchunks * pstride * 8, s));
   DHS_TRY(bget(t, t->b_pt, (size_t)nchunks * pstride * 8, s));
-  DHS_TRY(bget(t, t->b_cflags, nchunks, s));
   DHS_TRY(bget(t, t->b_owners, nchunks * 4, s));
+  DHS_TRY(bget(t, t->b_cplan, (size_t)(4 * nchunks + combine_batch_cap(nchunks)) * 4, s));
+  DHS_TRY(bget(t, t->b_slots, (size_t)combine_slot_cap(nchunks) * pstride * 8, s));
   DHS_CUDA(cudaMemsetAsync(t->b_nbm.p, 0, t->b_nbm.bytes, s));
   t->ws_n = cap;
+  t->ws_chunks = nchunks;
   return DHS_OK;
 }
 
 dhs_status check_table(const dhs_table* t) { return t ? DHS_OK : DHS_ERR_INVALID_ARG; }
+
+// Plan and combine launches for the long segments of one backward.
+dhs_status launch_combine(dhs_table* t, const unsigned* skey, long long n, const OptArgs& oa,
+                          const double* part_head, const double* part_tail, int chunk, int pstride,
+                          const unsigned* owners, unsigned* zeroed, const CombinePlan& pl,
+                          cudaStream_t s) {
+  const unsigned* owner_ctr = zeroed + kSegOwnerCtrWord;
+  bwd_combine_plan_kernel<<<(unsigned)t->sm_count * 2, 256, 0, s>>>(skey, n, chunk, owners, owner_ctr, pl,
+                                                                    t->st);
+  t->n_launches++;
+  DHS_TRY(last_launch());
+  const size_t smem = (size_t)std::max(kCombineThreads, t->dim) * sizeof(double);
+  bwd_combine_kernel<<<(unsigned)t->sm_count * 4, kCombineThreads, smem, s>>>(
+      skey, t->dim, rowspace(t), oa, part_head, part_tail, chunk, pstride, owners, owner_ctr, pl);
+  t->n_launches++;
+  return last_launch();
+}
 
 // ---- kernel dispatch on the row width ----
 dhs_status dispatch_pool(dhs_table* t, const long long* keys, long long n, const long long* bo,
@@ -423,7 +472,7 @@ dhs_status dispatch_seg(dhs_table* t, const unsigned* sk, const unsigned* sv, lo
             : t->opt == DHS_ADAM ? launch_seg_adam
                                  : launch_seg_rowwise;
   const cudaError_t e = fn(G, NV, t->sm_count, sk, sv, n, grad, nb, t->dim, rowspace(t), oa,
-                           (double*)t->b_ph.p, (double*)t->b_pt.p, (unsigned char*)t->b_cflags.p,
+                           (double*)t->b_ph.p, (double*)t->b_pt.p,
                            seg_chunk(n), (unsigned*)t->b_hist.p + kSegChunkCtrWord, (unsigned*)t->b_owners.p,
                            (unsigned*)t->b_hist.p + kSegOwnerCtrWord, t->st, s);
   t->n_launches++;
@@ -432,7 +481,7 @@ dhs_status dispatch_seg(dhs_table* t, const unsigned* sk, const unsigned* sv, lo
 }
 
 // offset assignment + row init for the new keys of an insert call
-dhs_status launch_assign(dhs_table* t, long long n, cudaStream_t s) {
+dhs_status launch_assign(dhs_table* t, const long long* keys, long long n, cudaStream_t s) {
   const long long nwords = (n + 31) / 32;
   const long long ngroups = (n + kGroupPositions - 1) / kGroupPositions;
   fwd_mark_kernel<<<(unsigned)ngroups, kGroupThreads, 0, s>>>(
@@ -441,7 +490,7 @@ dhs_status launch_assign(dhs_table* t, long long n, cudaStream_t s) {
   t->n_launches += 2;
   DHS_TRY(last_launch());
   fwd_assign_kernel<<<(unsigned)ngroups, kGroupThreads, 0, s>>>(
-      t->slots, rowspace(t), t->dim, (const unsigned*)t->b_fbm.p, (const unsigned*)t->b_gpref.p,
+      t->slots, rowspace(t), t->dim, keys, (const unsigned*)t->b_fbm.p, (const unsigned*)t->b_gpref.p,
       (const unsigned*)t->b_slotpos.p, nwords, ngroups, t->st);
   return last_launch();
 }
@@ -578,8 +627,8 @@ dhs_status ht_destroy(dhs_table* t) {
   dfree(t, t->blocks_d, sizeof(float*) * t->max_blocks, s);
   dfree(t, t->st, sizeof(DevState), s);
   Buf* bufs[] = {&t->b_nbm, &t->b_fbm, &t->b_gcnt, &t->b_gpref, &t->b_slotpos, &t->b_ka, &t->b_va,
-                 &t->b_kb, &t->b_vb, &t->b_hist, &t->b_totals, &t->b_ph, &t->b_pt, &t->b_cflags,
-                 &t->b_owners};
+                 &t->b_kb, &t->b_vb, &t->b_hist, &t->b_totals, &t->b_ph, &t->b_pt, &t->b_owners,
+                 &t->b_cplan, &t->b_slots};
   for (Buf* b : bufs) bfree(t, *b, s);
   cudaStreamSynchronize(s);
   for (auto& sn : t->snaps) {
@@ -636,7 +685,7 @@ dhs_status ht_lookup_or_insert(dhs_table* t, const int64_t* d_keys, int64_t n,
         (unsigned*)t->b_slotpos.p, t->st);
     t->n_launches += 2;
     DHS_TRY(last_launch());
-    DHS_TRY(launch_assign(t, n, s));
+    DHS_TRY(launch_assign(t, (const long long*)d_keys, n, s));
     const long long grid = std::min<long long>((n + 255) / 256, (long long)t->sm_count * 8);
     fwd_fixup_kernel<<<(unsigned)grid, 256, 0, s>>>(t->slots, (long long*)d_offsets_out, n);
     DHS_TRY(last_launch());
@@ -683,7 +732,7 @@ dhs_status embbag_forward(dhs_table* t, const int64_t* d_keys, int64_t n_keys,
   }
   if (n_keys > 0) {
     PhaseScope ph(t, PH_FWD_ASSIGN, s);
-    DHS_TRY(launch_assign(t, n_keys, s));
+    DHS_TRY(launch_assign(t, (const long long*)d_keys, n_keys, s));
   }
   t->n_insert_calls++;
   if (n_keys > 0) {
@@ -772,18 +821,11 @@ dhs_status embbag_backward_update(dhs_table* t, const int64_t* d_keys, int64_t n
     oa.bc2 = (float)(1.0 - std::pow((double)t->b2, (double)t->adam_t));
     DHS_TRY(dispatch_seg(t, ka, va, n_keys, d_grad, n_bags, oa, s));
     const int pstride = seg_nv(t->dim) * seg_group(t->dim) * 4;
-    const int chunk = seg_chunk(n_keys);
-    const long long nchunks = (n_keys + chunk - 1) / chunk;
-    const size_t smem = (size_t)std::max(256, t->dim) * sizeof(double);
-    const long long grid = std::min<long long>(nchunks, (long long)t->sm_count * 4);
-    bwd_combine_kernel<<<(unsigned)grid, 256, smem, s>>>(ka, n_keys, t->dim, rowspace(t), oa,
-                                                        (const double*)t->b_ph.p, (const double*)t->b_pt.p,
-                                                        (const unsigned char*)t->b_cflags.p, chunk,
-                                                        pstride, (const unsigned*)t->b_owners.p,
-                                                        (const unsigned*)t->b_hist.p + kSegOwnerCtrWord,
-                                                        t->st);
-    t->n_launches++;
-    DHS_TRY(last_launch());
+    DHS_TRY(launch_combine(t, ka, n_keys, oa, (const double*)t->b_ph.p, (const double*)t->b_pt.p,
+                           seg_chunk(n_keys), pstride, (const unsigned*)t->b_owners.p,
+                           (unsigned*)t->b_hist.p,
+                           combine_plan((unsigned*)t->b_cplan.p, (double*)t->b_slots.p, t->ws_chunks,
+                                        (unsigned*)t->b_hist.p), s));
   }
   return DHS_OK;
 }
@@ -941,10 +983,11 @@ constexpr size_t kNaStatus =
     na_align((size_t)kRadixMaxPasses * ((kNoAllocMaxKeys + kRadixTile - 1) / kRadixTile) * kRadixBins * 8);
 constexpr size_t kNaChunks = (kNoAllocMaxKeys + kNoAllocMinChunk - 1) / kNoAllocMinChunk;
 constexpr size_t kNaPart = na_align(kNaChunks * kNoAllocMaxDim * 8);  // one of part_head, part_tail
-constexpr size_t kNaFlags = na_align(kNaChunks);
 constexpr size_t kNaOwners = na_align(kNaChunks * 4);
+constexpr size_t kNaPlan = na_align((4 * kNaChunks + combine_batch_cap(kNaChunks)) * 4);
+constexpr size_t kNaSlots = na_align(combine_slot_cap(kNaChunks) * kNoAllocMaxDim * 8);
 constexpr size_t kNoAllocScratchBytes =
-    4 * kNaPairs + kNaSortZero + kNaStatus + 2 * kNaPart + kNaFlags + kNaOwners;
+    4 * kNaPairs + kNaSortZero + kNaStatus + 2 * kNaPart + kNaOwners + kNaPlan + kNaSlots;
 
 // Every GPU that loads this library holds this array until the process exits.
 __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
@@ -1001,8 +1044,10 @@ dhs_status embbag_backward_update_noalloc(dhs_table* t, const int64_t* d_keys, i
   unsigned long long* status = (unsigned long long*)(base + 4 * kNaPairs + kNaSortZero);
   double* part_head = (double*)(base + 4 * kNaPairs + kNaSortZero + kNaStatus);
   double* part_tail = (double*)(base + 4 * kNaPairs + kNaSortZero + kNaStatus + kNaPart);
-  unsigned char* cflags = base + 4 * kNaPairs + kNaSortZero + kNaStatus + 2 * kNaPart;
-  unsigned* owners = (unsigned*)(base + 4 * kNaPairs + kNaSortZero + kNaStatus + 2 * kNaPart + kNaFlags);
+  unsigned char* const tail = base + 4 * kNaPairs + kNaSortZero + kNaStatus + 2 * kNaPart;
+  unsigned* owners = (unsigned*)tail;
+  const CombinePlan plan =
+      combine_plan((unsigned*)(tail + kNaOwners), (double*)(tail + kNaOwners + kNaPlan), kNaChunks, hist);
 
   refresh_ub(t, false);
   const unsigned sentinel = (unsigned)t->rows_ub;
@@ -1051,18 +1096,12 @@ dhs_status embbag_backward_update_noalloc(dhs_table* t, const int64_t* d_keys, i
             : t->opt == DHS_ADAM ? launch_seg_adam
                                  : launch_seg_rowwise;
   if (fn(G, NV, t->sm_count, ka, va, n_keys, d_grad, n_bags, t->dim, rowspace(t), oa, part_head, part_tail,
-         cflags, chunk, hist + kSegChunkCtrWord, owners, hist + kSegOwnerCtrWord, t->st, s) != cudaSuccess) {
+         chunk, hist + kSegChunkCtrWord, owners, hist + kSegOwnerCtrWord, t->st, s) != cudaSuccess) {
     cudaGetLastError();
     return DHS_ERR_CUDA;
   }
-  const long long nchunks = (n_keys + chunk - 1) / chunk;
-  const size_t smem = (size_t)std::max(256, t->dim) * sizeof(double);
-  const long long grid = std::min<long long>(nchunks, (long long)t->sm_count * 4);
-  bwd_combine_kernel<<<(unsigned)grid, 256, smem, s>>>(ka, n_keys, t->dim, rowspace(t), oa, part_head,
-                                                      part_tail, cflags, chunk, NV * G * 4, owners,
-                                                      hist + kSegOwnerCtrWord, t->st);
-  t->n_launches += 4 + passes;
-  return last_launch();
+  t->n_launches += 3 + passes;
+  return launch_combine(t, ka, n_keys, oa, part_head, part_tail, chunk, NV * G * 4, owners, hist, plan, s);
 }
 
 }  // extern "C"

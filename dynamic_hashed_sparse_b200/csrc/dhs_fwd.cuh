@@ -166,7 +166,7 @@ fwd_probe_pool_kernel(IdMap m, RowSpace rs, int dim, const long long* __restrict
 #pragma unroll
               for (int q = 0; q < NV; ++q) {
                 const int c4 = gl + q * G;
-                if (c4 < d4) o[c4] = acc[q];
+                if (c4 < d4) __stcs(o + c4, acc[q]);  // streamed: not read again here
                 acc[q] = make_float4(0.f, 0.f, 0.f, 0.f);
               }
               ++cur;
@@ -184,7 +184,7 @@ fwd_probe_pool_kernel(IdMap m, RowSpace rs, int dim, const long long* __restrict
 #pragma unroll
       for (int q = 0; q < NV; ++q) {
         const int c4 = gl + q * G;
-        if (c4 < d4) o[c4] = acc[q];
+        if (c4 < d4) __stcs(o + c4, acc[q]);
         acc[q] = make_float4(0.f, 0.f, 0.f, 0.f);
       }
       ++cur;
@@ -350,7 +350,7 @@ fwd_mark_kernel(const Slot* __restrict__ slots, unsigned* __restrict__ nbm,
 // block then writes the run with coalesced 16-byte stores (initial weights
 // from splitmix64(key), optimizer state zero).
 __global__ void __launch_bounds__(kGroupThreads)
-fwd_assign_kernel(Slot* __restrict__ slots, RowSpace rs, int dim,
+fwd_assign_kernel(Slot* __restrict__ slots, RowSpace rs, int dim, const long long* __restrict__ keys,
                   const unsigned* __restrict__ fbm, const unsigned* __restrict__ gpref,
                   const unsigned* __restrict__ slotpos, long long nwords, long long ngroups,
                   DevState* st) {
@@ -397,7 +397,7 @@ fwd_assign_kernel(Slot* __restrict__ slots, RowSpace rs, int dim,
       const unsigned long long p = (unsigned long long)(g * kGroupPositions + k * kGroupThreads + threadIdx.x);
       const unsigned sl = slotpos[p];
       const unsigned long long row = row0 + j;
-      skey[j] = slots[sl].key;
+      skey[j] = (unsigned long long)__ldg(keys + p);  // the key first seen at p
       if (row < limit) {
         slots[sl].val = row;
       } else {
@@ -409,8 +409,12 @@ fwd_assign_kernel(Slot* __restrict__ slots, RowSpace rs, int dim,
   __syncthreads();
   const int s4 = rs.stride >> 2, d4 = dim >> 2;
   const int work = (int)total * s4;
+  // idx / s4 as a multiply-high by ceil(2^32 / s4) (s4 >= 2; that does not fit
+  // 32 bits for s4 = 1): exact while idx * s4 < 2^32 (here idx < 4096 * s4 and
+  // s4 <= 384)
+  const unsigned inv = s4 > 1 ? (unsigned)((0x100000000ull + (unsigned)s4 - 1) / (unsigned)s4) : 0u;
   for (int idx = threadIdx.x; idx < work; idx += kGroupThreads) {
-    const int r = idx / s4;
+    const int r = s4 > 1 ? (int)__umulhi((unsigned)idx, inv) : idx;
     const int c4 = idx - r * s4;
     const unsigned long long row = row0 + r;
     if (row >= limit) continue;

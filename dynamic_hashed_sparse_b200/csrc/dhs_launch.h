@@ -17,12 +17,12 @@ cudaError_t launch_probe_pool(int G, int NV, int sm_count, IdMap m, RowSpace rs,
                               DevState* st, cudaStream_t s);
 
 // bwd_seg_kernel<G, NV, OPT>, one entry point per optimizer
-#define DHS_SEG_DECL(NAME_)                                                                    \
-  cudaError_t NAME_(int G, int NV, int sm_count, const unsigned* skey, const unsigned* sval,   \
-                    long long n, const float* grad, long long n_bags, int dim, RowSpace rs,    \
-                    const OptArgs& oa, double* part_head, double* part_tail,                   \
-                    unsigned char* cflags, int chunk, unsigned* chunk_ctr, unsigned* owners,   \
-                    unsigned* owner_ctr, DevState* st, cudaStream_t s);
+#define DHS_SEG_DECL(NAME_)                                                                     \
+  cudaError_t NAME_(int G, int NV, int sm_count, const unsigned* skey, const unsigned* sval,    \
+                    long long n, const float* grad, long long n_bags, int dim, RowSpace rs,     \
+                    const OptArgs& oa, double* part_head, double* part_tail,                    \
+                    int chunk, unsigned* chunk_ctr, unsigned* owners, unsigned* owner_ctr,      \
+                    DevState* st, cudaStream_t s);
 DHS_SEG_DECL(launch_seg_sgd)
 DHS_SEG_DECL(launch_seg_adagrad)
 DHS_SEG_DECL(launch_seg_adam)

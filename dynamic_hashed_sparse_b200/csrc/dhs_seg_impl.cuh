@@ -14,7 +14,7 @@ namespace seg_impl {
 template <int G, int NV, int OPT>
 cudaError_t run(int sm_count, const unsigned* skey, const unsigned* sval, long long n,
                 const float* grad, long long n_bags, int dim, RowSpace rs, const OptArgs& oa,
-                double* part_head, double* part_tail, unsigned char* cflags, int chunk,
+                double* part_head, double* part_tail, int chunk,
                 unsigned* chunk_ctr, unsigned* owners, unsigned* owner_ctr, DevState* st,
                 cudaStream_t s) {
   static int resident = 0;
@@ -35,7 +35,7 @@ cudaError_t run(int sm_count, const unsigned* skey, const unsigned* sval, long l
   const long long need = std::max<long long>(1, (nchunks + per_block - 1) / per_block);
   const long long grid = std::min<long long>(need, resident);
   bwd_seg_kernel<G, NV, OPT><<<(unsigned)grid, 256, smem, s>>>(skey, sval, n, grad, n_bags, dim, rs, oa,
-                                                              part_head, part_tail, cflags, chunk, chunk_ctr,
+                                                              part_head, part_tail, chunk, chunk_ctr,
                                                               owners, owner_ctr, st);
   return cudaGetLastError();
 }
@@ -43,11 +43,11 @@ cudaError_t run(int sm_count, const unsigned* skey, const unsigned* sval, long l
 template <int OPT>
 cudaError_t launch(int G, int NV, int sm_count, const unsigned* skey, const unsigned* sval,
                    long long n, const float* grad, long long n_bags, int dim, RowSpace rs,
-                   const OptArgs& oa, double* part_head, double* part_tail, unsigned char* cflags,
+                   const OptArgs& oa, double* part_head, double* part_tail,
                    int chunk, unsigned* chunk_ctr, unsigned* owners, unsigned* owner_ctr, DevState* st,
                    cudaStream_t s) {
-#define DHS_RUN(g, v)                                                                                \
-  run<g, v, OPT>(sm_count, skey, sval, n, grad, n_bags, dim, rs, oa, part_head, part_tail, cflags, chunk, \
+#define DHS_RUN(g, v)                                                                           \
+  run<g, v, OPT>(sm_count, skey, sval, n, grad, n_bags, dim, rs, oa, part_head, part_tail, chunk, \
                  chunk_ctr, owners, owner_ctr, st, s)
   switch (G * 100 + NV) {
     case 102: return DHS_RUN(1, 2);
@@ -65,15 +65,14 @@ cudaError_t launch(int G, int NV, int sm_count, const unsigned* skey, const unsi
 }  // namespace seg_impl
 }  // namespace dhs
 
-#define DHS_SEG_TU(OPT_, NAME_)                                                                  \
-  namespace dhs {                                                                                \
-  cudaError_t NAME_(int G, int NV, int sm_count, const unsigned* skey, const unsigned* sval,     \
-                    long long n, const float* grad, long long n_bags, int dim, RowSpace rs,      \
-                    const OptArgs& oa, double* part_head, double* part_tail,                     \
-                    unsigned char* cflags, int chunk, unsigned* chunk_ctr, unsigned* owners,     \
-                    unsigned* owner_ctr, DevState* st, cudaStream_t s) {                         \
-    return seg_impl::launch<OPT_>(G, NV, sm_count, skey, sval, n, grad, n_bags, dim, rs, oa,     \
-                                  part_head, part_tail, cflags, chunk, chunk_ctr, owners,        \
-                                  owner_ctr, st, s);                                             \
-  }                                                                                              \
+#define DHS_SEG_TU(OPT_, NAME_)                                                                 \
+  namespace dhs {                                                                               \
+  cudaError_t NAME_(int G, int NV, int sm_count, const unsigned* skey, const unsigned* sval,    \
+                    long long n, const float* grad, long long n_bags, int dim, RowSpace rs,     \
+                    const OptArgs& oa, double* part_head, double* part_tail,                    \
+                    int chunk, unsigned* chunk_ctr, unsigned* owners, unsigned* owner_ctr,      \
+                    DevState* st, cudaStream_t s) {                                             \
+    return seg_impl::launch<OPT_>(G, NV, sm_count, skey, sval, n, grad, n_bags, dim, rs, oa,    \
+                                  part_head, part_tail, chunk, chunk_ctr, owners, owner_ctr, st, s); \
+  }                                                                                             \
   }
