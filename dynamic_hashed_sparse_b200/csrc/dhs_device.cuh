@@ -62,26 +62,39 @@ __device__ __forceinline__ unsigned long long hash_key(unsigned long long k) {
 // Output number n (n >= 1) of the splitmix64 generator seeded with `seed`
 // (Steele, Lea & Flood, OOPSLA 2014; Vigna's splitmix64.c): the state after n
 // steps is seed + n * golden gamma (mod 2^64), passed through the mixer.
-__device__ __forceinline__ unsigned long long splitmix64_output(unsigned long long seed,
-                                                                unsigned n) {
-  unsigned long long z = seed + (unsigned long long)n * 0x9E3779B97F4A7C15ull;
-  z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
-  z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
-  return z ^ (z >> 31);
+constexpr unsigned long long kSplitmixGamma = 0x9E3779B97F4A7C15ull;
+constexpr unsigned long long kSplitmixM1 = 0xBF58476D1CE4E5B9ull;
+constexpr unsigned long long kSplitmixM2 = 0x94D049BB133111EBull;
+
+// Bits 40..63 of splitmix64's output for the generator state z (the state
+// after its gamma step).  The finaliser's last step, x ^ (x >> 31), leaves
+// bits 40..63 of x unchanged, so they are the top 24 bits of the second
+// product, of which only the high word is formed:
+// hi32(lo64(a * m)) = hi32(alo * mlo) + alo * mhi + ahi * mlo (mod 2^32).
+__device__ __forceinline__ unsigned splitmix64_top24(unsigned long long z) {
+  z = (z ^ (z >> 30)) * kSplitmixM1;
+  z ^= z >> 27;
+  const unsigned lo = (unsigned)z, hi = (unsigned)(z >> 32);
+  const unsigned top = __umulhi(lo, (unsigned)kSplitmixM2) + lo * (unsigned)(kSplitmixM2 >> 32) +
+                       hi * (unsigned)kSplitmixM2;
+  return top >> 8;
 }
 
-// Initial weight j of the row of `key`: the top 24 bits of the (j+1)-th
-// splitmix64 output, centred, times 0.05 * 2^-23 (one rounded fp32 multiply
-// of exact operands), a value in [-0.05, 0.05).
-__device__ __forceinline__ float init_weight(unsigned long long key, int j) {
-  const unsigned long long z = splitmix64_output(key, (unsigned)j + 1u);
-  const int u = (int)(unsigned)(z >> 40) - (1 << 23);
-  return __fmul_rn((float)u, 0.05f * 0x1p-23f);
+// Initial weight from 24 random bits: centred, times 0.05 * 2^-23 (one
+// rounded fp32 multiply of exact operands), a value in [-0.05, 0.05).
+__device__ __forceinline__ float init_from_top24(unsigned t) {
+  return __fmul_rn((float)((int)t - (1 << 23)), 0.05f * 0x1p-23f);
 }
 
+// Initial weights j .. j+3 of the row of `key`: weight j comes from the
+// (j+1)-th splitmix64 output seeded with the key, whose state is
+// key + (j+1) * gamma.
 __device__ __forceinline__ float4 init_weight4(unsigned long long key, int j) {
-  return make_float4(init_weight(key, j), init_weight(key, j + 1), init_weight(key, j + 2),
-                     init_weight(key, j + 3));
+  const unsigned long long z = key + (unsigned long long)(j + 1) * kSplitmixGamma;
+  return make_float4(init_from_top24(splitmix64_top24(z)),
+                     init_from_top24(splitmix64_top24(z + kSplitmixGamma)),
+                     init_from_top24(splitmix64_top24(z + 2 * kSplitmixGamma)),
+                     init_from_top24(splitmix64_top24(z + 3 * kSplitmixGamma)));
 }
 
 struct IdMap {

@@ -413,13 +413,17 @@ fwd_assign_kernel(Slot* __restrict__ slots, RowSpace rs, int dim, const long lon
   // 32 bits for s4 = 1): exact while idx * s4 < 2^32 (here idx < 4096 * s4 and
   // s4 <= 384)
   const unsigned inv = s4 > 1 ? (unsigned)((0x100000000ull + (unsigned)s4 - 1) / (unsigned)s4) : 0u;
+  // rows before the first block edge share one base pointer
+  const unsigned long long in_block = (rs.br_mask + 1) - (row0 & rs.br_mask);
+  float4* const base = row0 < limit ? reinterpret_cast<float4*>(rs.row(row0)) : nullptr;
   for (int idx = threadIdx.x; idx < work; idx += kGroupThreads) {
     const int r = s4 > 1 ? (int)__umulhi((unsigned)idx, inv) : idx;
     const int c4 = idx - r * s4;
     const unsigned long long row = row0 + r;
     if (row >= limit) continue;
-    const float4 x = (c4 < d4) ? init_weight4(skey[r], c4 * 4) : make_float4(0.f, 0.f, 0.f, 0.f);
-    reinterpret_cast<float4*>(rs.row(row))[c4] = x;
+    float4* dst = (unsigned long long)r < in_block ? base + (size_t)r * s4
+                                                    : reinterpret_cast<float4*>(rs.row(row));
+    dst[c4] = (c4 < d4) ? init_weight4(skey[r], c4 * 4) : make_float4(0.f, 0.f, 0.f, 0.f);
   }
 }
 
