@@ -8,8 +8,8 @@
 // batch).  Occurrences are grouped by a stable sort on the row offset, so
 // each row's gradient is summed in batch order by one owner and written once:
 // there are no per-element atomics on rows.  A row whose run spans three or
-// more sort chunks (a hot key) is summed in pieces by every chunk it covers
-// and the pieces are combined by one thread block.
+// more sort chunks (a hot key) is summed in pieces by every chunk it covers;
+// the pieces are then added in batches and the batch sums in a fixed order.
 #pragma once
 
 #include "dhs_device.cuh"
@@ -34,6 +34,21 @@
 //                     for a row of <= 128 floats; wider rows use fewer
 #ifndef DHS_SEG_RING
 #define DHS_SEG_RING 8
+#endif
+//   DHS_RADIX_MINB    resident blocks per SM the one-sweep radix pass is
+//                     compiled for (register budget)
+//   DHS_SEGW_MIN_DIM  rows of at least this many floats use the warp-per-chunk
+//                     segment kernel; narrower rows the lane-group kernel
+#ifndef DHS_SEGW_MIN_DIM
+#define DHS_SEGW_MIN_DIM 32
+#endif
+#ifndef DHS_RADIX_MINB
+#define DHS_RADIX_MINB 5
+#endif
+//   DHS_HIST_MATCH    1: digit counts are combined per warp (match_any) before
+//                     the shared-memory atomic; 0: one atomic per key and pass
+#ifndef DHS_HIST_MATCH
+#define DHS_HIST_MATCH 0
 #endif
 
 namespace dhs {
@@ -138,16 +153,37 @@ radix_hist_all_kernel(const unsigned* __restrict__ keys, long long n, int passes
   __shared__ unsigned h[kRadixMaxPasses][kRadixBins];
   for (int i = threadIdx.x; i < kRadixMaxPasses * kRadixBins; i += kRadixThreads) (&h[0][0])[i] = 0;
   __syncthreads();
-  const int lane = threadIdx.x & 31;
   const long long stride = (long long)gridDim.x * kRadixThreads;
-  for (long long base = (long long)blockIdx.x * kRadixThreads; base < n; base += stride) {
-    const long long p = base + threadIdx.x;
-    const unsigned k = p < n ? __ldg(keys + p) : 0u;
+  // four keys per thread and step (one 16-byte load; the key array is 16-byte
+  // aligned), then the tail of n % 4 keys
+  const long long n4 = n >> 2;
+  const uint4* k4 = reinterpret_cast<const uint4*>(keys);
+  auto count = [&](unsigned k, bool ok) {
+#if DHS_HIST_MATCH
+    const int lane = threadIdx.x & 31;
     for (int ps = 0; ps < passes; ++ps) {
-      const unsigned d = p < n ? ((k >> (8 * ps)) & 255u) : 256u;
+      const unsigned d = ok ? ((k >> (8 * ps)) & 255u) : 256u;
       const unsigned peers = __match_any_sync(0xffffffffu, d);
       if (d < 256u && (__ffs(peers) - 1) == lane) atomicAdd(&h[ps][d], (unsigned)__popc(peers));
     }
+#else
+    if (ok)
+      for (int ps = 0; ps < passes; ++ps) atomicAdd(&h[ps][(k >> (8 * ps)) & 255u], 1u);
+#endif
+  };
+  for (long long base = (long long)blockIdx.x * kRadixThreads; base < n4; base += stride) {
+    const long long i = base + threadIdx.x;
+    const bool ok = i < n4;
+    const uint4 v = ok ? __ldg(k4 + i) : make_uint4(0u, 0u, 0u, 0u);
+    count(v.x, ok);
+    count(v.y, ok);
+    count(v.z, ok);
+    count(v.w, ok);
+  }
+  if (blockIdx.x == 0 && threadIdx.x < 32) {
+    const long long p = 4 * n4 + threadIdx.x;
+    const bool ok = p < n;  // at most 3 keys
+    count(ok ? __ldg(keys + p) : 0u, ok);
   }
   __syncthreads();
   for (int i = threadIdx.x; i < passes * kRadixBins; i += kRadixThreads) {
@@ -192,7 +228,7 @@ __device__ __forceinline__ unsigned block_exclusive_scan_256(unsigned x, unsigne
 // writes them out in runs.  A wait that exceeds its bound latches
 // kErrInternal and the pass goes on (its output is then undefined, never out
 // of bounds).
-__global__ void __launch_bounds__(kRadixThreads)
+__global__ void __launch_bounds__(kRadixThreads, DHS_RADIX_MINB)
 radix_onesweep_kernel(const unsigned* __restrict__ kin, const unsigned* __restrict__ vin,
                       unsigned* __restrict__ kout, unsigned* __restrict__ vout, long long n,
                       int shift, const unsigned* __restrict__ hist,
@@ -625,6 +661,320 @@ bwd_seg_kernel(const unsigned* __restrict__ skey, const unsigned* __restrict__ s
     }
   }
   if (gl == 0 && nseg_total) atomicAdd(&st->sum_unique, (unsigned long long)nseg_total);
+}
+
+// ---------------------------------------------------------------------------
+// Warp-per-chunk segment reduce: the same chunk ownership rules as
+// bwd_seg_kernel, but one whole warp walks a chunk's pairs, each lane holding
+// CPL consecutive columns of every row.  The chunk's keys (and those of the
+// next chunk, for an owned segment that runs past the chunk end) are loaded
+// once; run heads become four 32-bit masks, so finding a run's end, its
+// ownership and the pair range to stream are warp-uniform scalar steps and
+// no lane waits on another lane's control path.  Gradient rows of the next S
+// pairs are copied into this warp's shared-memory ring with cp.async (each
+// lane its own columns: no barrier), added in fp64 in sorted order; the
+// table row of an owned run is loaded into registers when the run opens and
+// written once when it closes.
+// ---------------------------------------------------------------------------
+__host__ __device__ constexpr int segw_slots(int cpl) { return 64 / cpl < 16 ? 64 / cpl : 16; }
+__host__ __device__ constexpr size_t segw_smem_bytes(int cpl) {
+  return (size_t)8 * segw_slots(cpl) * 32 * cpl * sizeof(float);
+}
+
+// This lane's CPL columns of one gradient row into shared memory (zero-filled
+// when !ok or past the row end).  dst and src are aligned to the copy size.
+template <int CPL>
+__device__ __forceinline__ void segw_copy(unsigned dst, const float* src, bool ok, int col0, int dim) {
+  if constexpr (CPL == 1) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(dst), "l"(src), "r"(ok ? 4u : 0u)
+                 : "memory");
+  } else if constexpr (CPL == 2) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 8, %2;" ::"r"(dst), "l"(src), "r"(ok ? 8u : 0u)
+                 : "memory");
+  } else {
+#pragma unroll
+    for (int k = 0; k < CPL / 4; ++k) {
+      const bool in = ok && col0 + 4 * k < dim;
+      cp_async16(dst + 16u * k, in ? src + 4 * k : src, in ? 16u : 0u);
+    }
+  }
+}
+
+// CPL columns of a row at p (p + col0 aligned to the vector width) into v and
+// back; columns at or past dim are neither read nor written.
+template <int CPL>
+__device__ __forceinline__ void segw_ld(float (&v)[CPL], const float* p, int col0, int dim) {
+  if constexpr (CPL == 1) {
+    v[0] = p[col0];
+  } else if constexpr (CPL == 2) {
+    const float2 x = *reinterpret_cast<const float2*>(p + col0);
+    v[0] = x.x;
+    v[1] = x.y;
+  } else {
+#pragma unroll
+    for (int k = 0; k < CPL / 4; ++k) {
+      if (col0 + 4 * k < dim) {
+        const float4 x = *reinterpret_cast<const float4*>(p + col0 + 4 * k);
+        v[4 * k] = x.x;
+        v[4 * k + 1] = x.y;
+        v[4 * k + 2] = x.z;
+        v[4 * k + 3] = x.w;
+      }
+    }
+  }
+}
+template <int CPL>
+__device__ __forceinline__ void segw_st(float* p, const float (&v)[CPL], int col0, int dim) {
+  if constexpr (CPL == 1) {
+    p[col0] = v[0];
+  } else if constexpr (CPL == 2) {
+    *reinterpret_cast<float2*>(p + col0) = make_float2(v[0], v[1]);
+  } else {
+#pragma unroll
+    for (int k = 0; k < CPL / 4; ++k)
+      if (col0 + 4 * k < dim)
+        *reinterpret_cast<float4*>(p + col0 + 4 * k) =
+            make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
+  }
+}
+
+template <int CPL, int OPT>
+__global__ void __launch_bounds__(256, CPL <= 4 ? 3 : 1)
+bwd_segw_kernel(const unsigned* __restrict__ skey, const unsigned* __restrict__ sval, long long n,
+                const float* __restrict__ grad, long long n_bags, int dim, RowSpace rs, OptArgs oa,
+                double* __restrict__ part_head, double* __restrict__ part_tail, int pstride, int C,
+                unsigned* __restrict__ chunk_ctr, unsigned* __restrict__ owners,
+                unsigned* __restrict__ owner_ctr, DevState* st) {
+  constexpr int S = segw_slots(CPL);
+  constexpr int NS = seg_state_arrays(OPT);
+  constexpr unsigned FULL = 0xffffffffu;
+  extern __shared__ float segw_smem[];
+  const int lane = threadIdx.x & 31;
+  const int wid = threadIdx.x >> 5;
+  const int col0 = lane * CPL;
+  const bool lane_on = col0 < dim;
+  float* ring = segw_smem + (size_t)wid * S * 32 * CPL + col0;  // this lane's columns of slot 0
+  const unsigned ring_s = (unsigned)__cvta_generic_to_shared(ring);
+  // positions and bags fit in 31 bits (the host rejects larger calls); C <= 64
+  const int n32 = (int)n;
+  const unsigned nb32 = (unsigned)n_bags;
+  const int nchunks = (n32 + C - 1) / C;
+  const unsigned nrows = (unsigned)min(st->row_count, 0xffffffffull);
+  unsigned nseg_total = 0;
+
+  for (;;) {
+    int c = 0;
+    if (lane == 0) c = (int)atomicAdd(chunk_ctr, 1u);
+    c = __shfl_sync(FULL, c, 0);
+    if (c >= nchunks) break;
+    const int start = c * C;
+    const int end = min(n32, start + C);
+    const int limit = min(n32, end + C);  // an owned run ends before chunk c + 2
+    const int lim = limit - start, cend = end - start;  // relative to start
+
+    // keys and bags of [start, limit), 32 per word
+    unsigned kw[4], vw[4];
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+      const int p = start + 32 * w + lane;
+      const bool in = p < limit;
+      kw[w] = in ? __ldg(skey + p) : ~0u;
+      vw[w] = in ? __ldg(sval + p) : 0u;
+    }
+    const unsigned prev = start > 0 ? __ldg(skey + start - 1) : ~0u;
+    const unsigned back2 = c >= 2 ? __ldg(skey + (c - 1) * C - 1) : ~0u;
+    const unsigned fwd1 = end < n32 ? __ldg(skey + end) : ~0u;
+    const bool has2 = (c + 2) * C < n32;
+    const unsigned fwd2 = has2 ? __ldg(skey + (c + 2) * C) : ~0u;
+    // run heads: bit q of word q / 32 set when position start + q starts a run
+    unsigned hm[4];
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+      unsigned before = __shfl_up_sync(FULL, kw[w], 1);
+      const unsigned carry = w == 0 ? prev : __shfl_sync(FULL, kw[w == 0 ? 0 : w - 1], 31);
+      if (lane == 0) before = carry;
+      hm[w] = __ballot_sync(FULL, 32 * w + lane < lim && kw[w] != before);
+    }
+    auto word = [&](const unsigned (&a)[4], int q) -> unsigned {
+      return q < 32 ? a[0] : (q < 64 ? a[1] : (q < 96 ? a[2] : a[3]));
+    };
+    auto key_at = [&](int q) -> unsigned { return __shfl_sync(FULL, word(kw, q), q & 31); };
+    // first head after relative position q, or lim
+    auto next_head = [&](int q) -> int {
+      int r = q + 1;
+#pragma unroll
+      for (int w = 0; w < 4; ++w) {
+        if (r < 32 * (w + 1) && r < lim) {
+          unsigned m = w == 0 ? hm[0] : (w == 1 ? hm[1] : (w == 2 ? hm[2] : hm[3]));
+          const int lo = r - 32 * w;
+          if (lo > 0) m &= 0xffffffffu << lo;
+          if (m) return 32 * w + __ffs(m) - 1;
+          r = 32 * (w + 1);
+        }
+      }
+      return lim;
+    };
+    // last head at or before relative position q (0 when the first run covers it)
+    auto last_head = [&](int q) -> int {
+#pragma unroll
+      for (int w = 3; w >= 0; --w) {
+        if (32 * w <= q) {
+          unsigned m = w == 0 ? hm[0] : (w == 1 ? hm[1] : (w == 2 ? hm[2] : hm[3]));
+          const int hi = q - 32 * w;
+          if (hi < 31) m &= (2u << hi) - 1u;
+          if (m) return 32 * w + 31 - __clz(m);
+        }
+      }
+      return 0;
+    };
+
+    // ownership: the first run continues one from the previous chunk unless a
+    // head sits at position 0; runs that reach chunk c + 2 are long
+    const unsigned k0 = key_at(0);
+    const bool first_here = hm[0] & 1u;
+    const int mode_first = first_here ? ((has2 && fwd2 == k0) ? 3 : 2)
+                                      : ((back2 == k0 || fwd1 == k0) ? 1 : 0);
+    const int s0 = mode_first == 0 ? next_head(0) : 0;
+    const int hl = last_head(cend - 1);
+    const unsigned kl = key_at(cend - 1);
+    const int mode_last = hl == 0 ? mode_first : ((has2 && fwd2 == kl) ? 3 : 2);
+    const int stop = mode_last == 2 ? next_head(cend - 1) : (mode_last == 0 ? s0 : cend);
+
+    // distinct rows started in this chunk; L2 prefetch of the owned runs' rows
+    {
+      unsigned cnt = 0;
+#pragma unroll
+      for (int w = 0; w < 4; ++w) {
+        const int q = 32 * w + lane;
+        const unsigned k = kw[w];
+        const bool head = (hm[w] >> lane) & 1u;
+        cnt += __popc(__ballot_sync(FULL, head && q < cend && k < nrows));
+        if (head && q >= s0 && q < stop && k < nrows && !(has2 && fwd2 == k))
+          prefetch_l2(rs.row(k), (unsigned)rs.stride * 4u);
+      }
+      nseg_total += cnt;
+    }
+    if (s0 >= stop) continue;
+
+    // ---- producer: gradient rows of stream pairs s0, s0 + 1, ... into the ring.
+    // A pair whose key has no row or whose bag is out of range copies zeros.
+#pragma unroll
+    for (int w = 0; w < 4; ++w) vw[w] = (kw[w] < nrows && vw[w] < nb32) ? vw[w] : ~0u;
+    constexpr unsigned kSlotBytes = 32u * CPL * 4u;
+    int pf = s0;
+    unsigned pword = word(vw, s0);  // bags of the 32-pair word holding pf
+    unsigned pslot = 0;             // byte offset of pf's slot
+    auto produce = [&]() {
+      if (pf < stop) {
+        if ((pf & 31) == 0) pword = word(vw, pf);
+        const unsigned b = __shfl_sync(FULL, pword, pf & 31);
+        const bool ok = lane_on && b != ~0u;
+        const float* src = grad + (size_t)(ok ? b : 0u) * dim + (lane_on ? col0 : 0);
+        segw_copy<CPL>(ring_s + pslot, src, ok, col0, dim);
+      }
+      cp_async_commit();  // one group per pair (empty past the stream end)
+      ++pf;
+      pslot = (pslot + kSlotBytes) & (S * kSlotBytes - 1u);
+    };
+#pragma unroll
+    for (int j = 0; j < S; ++j) produce();
+
+    // ---- consumer
+    double acc[CPL];
+#pragma unroll
+    for (int e = 0; e < CPL; ++e) acc[e] = 0.0;
+    float rw[CPL];
+    float rst[NS > 0 ? NS : 1][CPL];
+    float racc = 0.f;
+    unsigned kcur = 0;
+    int mode = 0, run_end = 0;
+    auto open = [&](int q) {
+      kcur = key_at(q);
+      mode = q == 0 ? mode_first : ((has2 && fwd2 == kcur) ? 3 : 2);
+      run_end = next_head(q);
+      if (mode != 2) run_end = min(run_end, cend);  // a long piece stops at the chunk end
+      if (mode == 2 && kcur < nrows) {
+        const float* row = rs.row(kcur);
+        if (lane_on) {
+          segw_ld<CPL>(rw, row, col0, dim);
+#pragma unroll
+          for (int k = 0; k < NS; ++k) segw_ld<CPL>(rst[k], row + (k + 1) * dim, col0, dim);
+        }
+        if (OPT == 3) racc = row[dim];
+      }
+    };
+    auto close = [&]() {
+      if (mode == 1 || mode == 3) {
+        double* o = (mode == 1 ? part_head : part_tail) + (long long)c * pstride + col0;
+        if (lane_on) {
+#pragma unroll
+          for (int e = 0; e < CPL; ++e)
+            if (col0 + e < dim) o[e] = acc[e];
+        }
+        if (mode == 3 && lane == 0) owners[atomicAdd(owner_ctr, 1u)] = (unsigned)c;  // for the combine
+      } else if (mode == 2 && kcur < nrows) {
+        float* row = rs.row(kcur);
+        float den = 0.f, Gn = 0.f;
+        if (OPT == 3) {
+          double sq = 0.0;
+#pragma unroll
+          for (int e = 0; e < CPL; ++e) {
+            if (lane_on && col0 + e < dim) {
+              const double g = (double)(float)acc[e];
+              sq += g * g;
+            }
+          }
+#pragma unroll
+          for (int o = 1; o < 32; o <<= 1) sq += __shfl_xor_sync(FULL, sq, o);
+          Gn = __fadd_rn(racc, (float)(sq / (double)dim));
+          den = __fadd_rn(__fsqrt_rn(Gn), oa.eps);
+        }
+        if (lane_on) {
+#pragma unroll
+          for (int e = 0; e < CPL; ++e) {
+            const float g = (float)acc[e];
+            if (OPT == 0) {
+              rw[e] = sgd_w(rw[e], g, oa.lr);
+            } else if (OPT == 1) {
+              adagrad_step(rw[e], rst[0][e], g, oa.lr, oa.eps);
+            } else if (OPT == 2) {
+              adam_step(rw[e], rst[0][e], rst[NS - 1][e], g, oa);
+            } else {
+              rw[e] = __fsub_rn(rw[e], __fdiv_rn(__fmul_rn(oa.lr, g), den));
+            }
+          }
+          segw_st<CPL>(row, rw, col0, dim);
+#pragma unroll
+          for (int k = 0; k < NS; ++k) segw_st<CPL>(row + (k + 1) * dim, rst[k], col0, dim);
+        }
+        if (OPT == 3 && lane == 0) row[dim] = Gn;
+      }
+#pragma unroll
+      for (int e = 0; e < CPL; ++e) acc[e] = 0.0;
+    };
+
+    open(s0);
+    int cslot = 0;  // float offset of pair q's slot
+    for (int q = s0; q < stop; ++q) {
+      cp_async_wait<S - 1>();  // pair q's columns have landed (this lane's own copy)
+      if (lane_on) {
+        float x[CPL];
+#pragma unroll
+        for (int e = 0; e < CPL; ++e) x[e] = 0.f;
+        segw_ld<CPL>(x, ring + cslot, 0, dim - col0);
+#pragma unroll
+        for (int e = 0; e < CPL; ++e) acc[e] += (double)x[e];
+      }
+      cslot = (cslot + 32 * CPL) & (S * 32 * CPL - 1);
+      produce();  // refill the slot just read with pair q + S
+      if (q + 1 == run_end) {
+        close();
+        if (q + 1 < stop) open(q + 1);
+      }
+    }
+    cp_async_wait_all();  // the ring is reused by the next chunk
+  }
+  if (lane == 0 && nseg_total) atomicAdd(&st->sum_unique, (unsigned long long)nseg_total);
 }
 
 #ifndef DHS_TEMPLATES_ONLY

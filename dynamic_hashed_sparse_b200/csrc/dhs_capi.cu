@@ -133,7 +133,7 @@ struct dhs_table {
   long long ws_n = -1;
   long long ws_chunks = 0;  // chunk capacity of the segment and combine buffers
   Buf b_nbm, b_fbm, b_gcnt, b_gpref, b_slotpos, b_ka, b_va, b_kb, b_vb, b_hist, b_totals, b_ph,
-      b_pt, b_owners, b_cplan, b_slots;
+      b_pt, b_owners, b_cplan, b_slots, b_refs;
 
   bool timing = false;
   std::vector<PhaseRec> recs;
@@ -415,6 +415,7 @@ dhs_status ensure_ws(dhs_table* t, long long n, cudaStream_t s) {
   DHS_TRY(bget(t, t->b_gcnt, ngroups * 4, s));
   DHS_TRY(bget(t, t->b_gpref, ngroups * 4, s));
   DHS_TRY(bget(t, t->b_slotpos, cap * 4, s));
+  DHS_TRY(bget(t, t->b_refs, cap * 8, s));
   DHS_TRY(bget(t, t->b_ka, cap * 4, s));
   DHS_TRY(bget(t, t->b_va, cap * 4, s));
   DHS_TRY(bget(t, t->b_kb, cap * 4, s));
@@ -464,20 +465,45 @@ dhs_status dispatch_pool(dhs_table* t, const long long* keys, long long n, const
   return e == cudaSuccess ? DHS_OK : DHS_ERR_CUDA;
 }
 
-dhs_status dispatch_seg(dhs_table* t, const unsigned* sk, const unsigned* sv, long long n,
-                        const float* grad, long long nb, const OptArgs& oa, cudaStream_t s) {
+// Segment kernel for one backward: the warp-per-chunk kernel for rows of at
+// least DHS_SEGW_MIN_DIM floats, the lane-group kernel below that.
+int segw_cpl(int dim) {
+  int c = 1;
+  while (32 * c < dim) c *= 2;
+  return c;
+}
+
+dhs_status launch_seg(dhs_table* t, const unsigned* sk, const unsigned* sv, long long n, const float* grad,
+                      long long nb, const OptArgs& oa, double* part_head, double* part_tail,
+                      unsigned* chunk_ctr, unsigned* owners, unsigned* owner_ctr, cudaStream_t s) {
   const int G = seg_group(t->dim), NV = seg_nv(t->dim);
-  auto fn = t->opt == DHS_SGD ? launch_seg_sgd
-            : t->opt == DHS_ADAGRAD ? launch_seg_adagrad
-            : t->opt == DHS_ADAM ? launch_seg_adam
-                                 : launch_seg_rowwise;
-  const cudaError_t e = fn(G, NV, t->sm_count, sk, sv, n, grad, nb, t->dim, rowspace(t), oa,
-                           (double*)t->b_ph.p, (double*)t->b_pt.p,
-                           seg_chunk(n), (unsigned*)t->b_hist.p + kSegChunkCtrWord, (unsigned*)t->b_owners.p,
-                           (unsigned*)t->b_hist.p + kSegOwnerCtrWord, t->st, s);
+  const int pstride = NV * G * 4;  // doubles per partial (>= dim)
+  cudaError_t e;
+  if (t->dim >= DHS_SEGW_MIN_DIM) {
+    auto fn = t->opt == DHS_SGD ? launch_seg_sgd_w
+              : t->opt == DHS_ADAGRAD ? launch_seg_adagrad_w
+              : t->opt == DHS_ADAM ? launch_seg_adam_w
+                                   : launch_seg_rowwise_w;
+    e = fn(segw_cpl(t->dim), t->sm_count, sk, sv, n, grad, nb, t->dim, rowspace(t), oa, part_head, part_tail,
+           pstride, seg_chunk(n), chunk_ctr, owners, owner_ctr, t->st, s);
+  } else {
+    auto fn = t->opt == DHS_SGD ? launch_seg_sgd
+              : t->opt == DHS_ADAGRAD ? launch_seg_adagrad
+              : t->opt == DHS_ADAM ? launch_seg_adam
+                                   : launch_seg_rowwise;
+    e = fn(G, NV, t->sm_count, sk, sv, n, grad, nb, t->dim, rowspace(t), oa, part_head, part_tail,
+           seg_chunk(n), chunk_ctr, owners, owner_ctr, t->st, s);
+  }
   t->n_launches++;
   if (e != cudaSuccess) cudaGetLastError();
   return e == cudaSuccess ? DHS_OK : DHS_ERR_CUDA;
+}
+
+dhs_status dispatch_seg(dhs_table* t, const unsigned* sk, const unsigned* sv, long long n,
+                        const float* grad, long long nb, const OptArgs& oa, cudaStream_t s) {
+  return launch_seg(t, sk, sv, n, grad, nb, oa, (double*)t->b_ph.p, (double*)t->b_pt.p,
+                    (unsigned*)t->b_hist.p + kSegChunkCtrWord, (unsigned*)t->b_owners.p,
+                    (unsigned*)t->b_hist.p + kSegOwnerCtrWord, s);
 }
 
 // offset assignment + row init for the new keys of an insert call
@@ -628,7 +654,7 @@ dhs_status ht_destroy(dhs_table* t) {
   dfree(t, t->st, sizeof(DevState), s);
   Buf* bufs[] = {&t->b_nbm, &t->b_fbm, &t->b_gcnt, &t->b_gpref, &t->b_slotpos, &t->b_ka, &t->b_va,
                  &t->b_kb, &t->b_vb, &t->b_hist, &t->b_totals, &t->b_ph, &t->b_pt, &t->b_owners,
-                 &t->b_cplan, &t->b_slots};
+                 &t->b_cplan, &t->b_slots, &t->b_refs};
   for (Buf* b : bufs) bfree(t, *b, s);
   cudaStreamSynchronize(s);
   for (auto& sn : t->snaps) {
@@ -727,8 +753,27 @@ dhs_status embbag_forward(dhs_table* t, const int64_t* d_keys, int64_t n_keys,
   DHS_TRY(ensure_ws(t, n_keys, s));
   {
     PhaseScope ph(t, PH_FWD_POOL, s);
-    DHS_TRY(dispatch_pool(t, (const long long*)d_keys, n_keys, (const long long*)d_bag_offsets,
-                          n_bags, d_pooled_out, s));
+    if (n_keys >= (long long)DHS_POOL_SPLIT_LEN * n_bags && n_keys > 0) {
+      // long bags: probe every id first (a thread per id), then gather
+      fwd_probe_offsets_kernel<<<(unsigned)((n_keys + kFwdThreads - 1) / kFwdThreads), kFwdThreads, 0, s>>>(
+          idmap(t), (const long long*)d_keys, n_keys, (long long*)t->b_refs.p, (unsigned*)t->b_nbm.p,
+          (unsigned*)t->b_slotpos.p, t->st);
+      t->n_launches++;
+      DHS_TRY(last_launch());
+      const int G = pick_group(t->dim), NV = pick_nv(t->dim, G);
+      const cudaError_t e =
+          launch_pool_refs(G, NV, t->sm_count, rowspace(t), t->dim, (const long long*)d_keys,
+                           (const long long*)t->b_refs.p, n_keys, (const long long*)d_bag_offsets, n_bags,
+                           d_pooled_out, t->st, s);
+      t->n_launches++;
+      if (e != cudaSuccess) {
+        cudaGetLastError();
+        return DHS_ERR_CUDA;
+      }
+    } else {
+      DHS_TRY(dispatch_pool(t, (const long long*)d_keys, n_keys, (const long long*)d_bag_offsets,
+                            n_bags, d_pooled_out, s));
+    }
   }
   if (n_keys > 0) {
     PhaseScope ph(t, PH_FWD_ASSIGN, s);
@@ -1091,16 +1136,9 @@ dhs_status embbag_backward_update_noalloc(dhs_table* t, const int64_t* d_keys, i
   oa.bc2 = (float)(1.0 - std::pow((double)t->b2, (double)t->adam_t));
   const int G = seg_group(t->dim), NV = seg_nv(t->dim);
   const int chunk = seg_chunk(n_keys);
-  auto fn = t->opt == DHS_SGD ? launch_seg_sgd
-            : t->opt == DHS_ADAGRAD ? launch_seg_adagrad
-            : t->opt == DHS_ADAM ? launch_seg_adam
-                                 : launch_seg_rowwise;
-  if (fn(G, NV, t->sm_count, ka, va, n_keys, d_grad, n_bags, t->dim, rowspace(t), oa, part_head, part_tail,
-         chunk, hist + kSegChunkCtrWord, owners, hist + kSegOwnerCtrWord, t->st, s) != cudaSuccess) {
-    cudaGetLastError();
-    return DHS_ERR_CUDA;
-  }
-  t->n_launches += 3 + passes;
+  DHS_TRY(launch_seg(t, ka, va, n_keys, d_grad, n_bags, oa, part_head, part_tail, hist + kSegChunkCtrWord, owners,
+                     hist + kSegOwnerCtrWord, s));
+  t->n_launches += 2 + passes;
   return launch_combine(t, ka, n_keys, oa, part_head, part_tail, chunk, NV * G * 4, owners, hist, plan, s);
 }
 

@@ -17,6 +17,13 @@
 
 #include "dhs_device.cuh"
 
+// Bags of at least DHS_POOL_SPLIT_LEN ids on average are pooled by the split
+// forward (a probe kernel with a thread per id, then fwd_pool_refs_kernel);
+// shorter bags by the fused fwd_probe_pool_kernel.
+#ifndef DHS_POOL_SPLIT_LEN
+#define DHS_POOL_SPLIT_LEN 4
+#endif
+
 namespace dhs {
 
 constexpr int kFwdThreads = 256;
@@ -57,6 +64,60 @@ __device__ __forceinline__ long long load_bag_ends(const long long* __restrict__
   return e;
 }
 
+// Gather + pool of one window of cnt ids (kind and ref held by lane t of the
+// group for id t of the window): each lane loads NV float4 columns of U rows
+// at a time, then adds them into the current bag's accumulator in id order,
+// writing out each bag as its end is passed.  A new key's row is computed
+// from the key, exactly as the assignment kernel will store it.
+template <int G, int NV>
+__device__ __forceinline__ void pool_window(int kind, unsigned long long ref, int cnt, int ws,
+                                            unsigned gmask, int gl, int d4, int dim, int e,
+                                            float4 (&acc)[NV], int& cur, int& cur_end, float* outb) {
+  constexpr int U = G < 8 ? G : 8;
+  for (int t0 = 0; t0 < cnt; t0 += U) {
+    float4 v[U][NV];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int t = t0 + u;
+      const int src = t & (G - 1);
+      const int kt = __shfl_sync(gmask, kind, src, G);
+      const unsigned long long rt = __shfl_sync(gmask, ref, src, G);
+#pragma unroll
+      for (int q = 0; q < NV; ++q) {
+        const int c4 = gl + q * G;
+        float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (t < cnt && c4 < d4) {
+          if (kt == kHit)
+            x = __ldg(reinterpret_cast<const float4*>(rt) + c4);
+          else if (kt == kNew)
+            x = init_weight4(rt, c4 * 4);
+        }
+        v[u][q] = x;
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int t = t0 + u;
+      if (t < cnt) {
+        const int pos = ws + t;
+        while (pos >= cur_end) {
+          float4* o = reinterpret_cast<float4*>(outb + (long long)cur * dim);
+#pragma unroll
+          for (int q = 0; q < NV; ++q) {
+            const int c4 = gl + q * G;
+            if (c4 < d4) __stcs(o + c4, acc[q]);  // streamed: not read again here
+            acc[q] = make_float4(0.f, 0.f, 0.f, 0.f);
+          }
+          ++cur;
+          cur_end = __shfl_sync(gmask, e, cur & (G - 1), G);
+        }
+#pragma unroll
+        for (int q = 0; q < NV; ++q) acc[q] = f4add(acc[q], v[u][q]);
+      }
+    }
+  }
+}
+
 // Fused lookup-or-insert + gather + sum pooling.  A group of G lanes owns a
 // chunk of G consecutive bags; it probes the chunk's ids G at a time (one id
 // per lane; the probing lane also forms the row address), then walks those ids
@@ -70,7 +131,6 @@ fwd_probe_pool_kernel(IdMap m, RowSpace rs, int dim, const long long* __restrict
                       long long n_keys, const long long* __restrict__ bag_off, long long n_bags,
                       float* __restrict__ out, unsigned* __restrict__ nbm,
                       unsigned* __restrict__ slotpos, DevState* st) {
-  constexpr int U = G < 8 ? G : 8;
   const int lane = threadIdx.x & 31;
   const int gl = lane & (G - 1);
   const int gw = lane / G;
@@ -134,51 +194,84 @@ fwd_probe_pool_kernel(IdMap m, RowSpace rs, int dim, const long long* __restrict
           }
         }
       }
-      // ---- gather + pool, in id order ----
-      for (int t0 = 0; t0 < cnt; t0 += U) {
-        float4 v[U][NV];
-#pragma unroll
-        for (int u = 0; u < U; ++u) {
-          const int t = t0 + u;
-          const int src = t & (G - 1);
-          const int kt = __shfl_sync(gmask, kind, src, G);
-          const unsigned long long rt = __shfl_sync(gmask, ref, src, G);
-#pragma unroll
-          for (int q = 0; q < NV; ++q) {
-            const int c4 = gl + q * G;
-            float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (t < cnt && c4 < d4) {
-              if (kt == kHit)
-                x = __ldg(reinterpret_cast<const float4*>(rt) + c4);
-              else if (kt == kNew)
-                x = init_weight4(rt, c4 * 4);
-            }
-            v[u][q] = x;
-          }
-        }
-#pragma unroll
-        for (int u = 0; u < U; ++u) {
-          const int t = t0 + u;
-          if (t < cnt) {
-            const int pos = ws + t;
-            while (pos >= cur_end) {
-              float4* o = reinterpret_cast<float4*>(outb + (long long)cur * dim);
-#pragma unroll
-              for (int q = 0; q < NV; ++q) {
-                const int c4 = gl + q * G;
-                if (c4 < d4) __stcs(o + c4, acc[q]);  // streamed: not read again here
-                acc[q] = make_float4(0.f, 0.f, 0.f, 0.f);
-              }
-              ++cur;
-              cur_end = __shfl_sync(gmask, e, cur & (G - 1), G);
-            }
-#pragma unroll
-            for (int q = 0; q < NV; ++q) acc[q] = f4add(acc[q], v[u][q]);
-          }
-        }
-      }
+      pool_window<G, NV>(kind, ref, cnt, ws, gmask, gl, d4, dim, e, acc, cur, cur_end, outb);
     }
     // the bag in progress and any empty bags after it
+    while (cur < nb) {
+      float4* o = reinterpret_cast<float4*>(outb + (long long)cur * dim);
+#pragma unroll
+      for (int q = 0; q < NV; ++q) {
+        const int c4 = gl + q * G;
+        if (c4 < d4) __stcs(o + c4, acc[q]);
+        acc[q] = make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+      ++cur;
+    }
+  }
+}
+
+// Gather + pool from per-id row references (the split forward for long bags):
+// refs[p] >= 0 is the row of a hit, <= -2 marks a key new in this call (its
+// row is computed from keys[p]), -1 an id without a row.  The references of
+// the window two ahead are loaded, and the rows of the next window prefetched
+// into L2, while the current window is gathered, so no window waits on a
+// probe.  Bags, windows and the order of additions are those of
+// fwd_probe_pool_kernel.
+template <int G, int NV>
+__global__ void __launch_bounds__(kFwdThreads, NV == 1 ? 4 : (NV == 2 ? 2 : 1))
+fwd_pool_refs_kernel(RowSpace rs, int dim, const long long* __restrict__ keys,
+                     const long long* __restrict__ refs, long long n_keys,
+                     const long long* __restrict__ bag_off, long long n_bags,
+                     float* __restrict__ out, DevState* st) {
+  const int lane = threadIdx.x & 31;
+  const int gl = lane & (G - 1);
+  const int gw = lane / G;
+  const unsigned gmask = (G == 32) ? 0xffffffffu : (((1u << G) - 1u) << (gw * G));
+  const int gid = (int)((blockIdx.x * kFwdThreads + threadIdx.x) / G);
+  const int ngroups = (int)((gridDim.x * kFwdThreads) / G);
+  const int nchunks = (int)((n_bags + G - 1) / G);
+  const int d4 = dim >> 2;
+  const unsigned row_bytes = (unsigned)dim * 4u;
+
+  for (int c = gid; c < nchunks; c += ngroups) {
+    const long long b0 = (long long)c * G;
+    const int nb = (int)min((long long)G, n_bags - b0);
+    long long s64;
+    const long long e64 = load_bag_ends<G>(bag_off, b0, nb, n_keys, n_bags, s64, gmask, gl, st);
+    const int e = e64 == LLONG_MAX ? INT_MAX : (int)e64;
+    const int s = (int)s64;
+    const int E = __shfl_sync(gmask, e, nb - 1, G);
+    int cur = 0;
+    int cur_end = __shfl_sync(gmask, e, 0, G);
+    float4 acc[NV];
+#pragma unroll
+    for (int q = 0; q < NV; ++q) acc[q] = make_float4(0.f, 0.f, 0.f, 0.f);
+    float* outb = out + b0 * (long long)dim;
+
+    auto ref_at = [&](int p) -> long long { return p < E ? __ldg(refs + p) : -1; };
+    long long r0 = ref_at(s + gl), r1 = ref_at(s + G + gl);
+    long long k0 = r0 <= -2 ? __ldg(keys + s + gl) : 0;
+    if (r0 >= 0) prefetch_l2(rs.row((unsigned long long)r0), row_bytes);
+    for (int ws = s; ws < E; ws += G) {
+      const int cnt = min(G, E - ws);
+      const long long rc = r0, kc = k0;
+      r0 = r1;
+      r1 = ref_at(ws + 2 * G + gl);
+      k0 = r0 <= -2 ? __ldg(keys + ws + G + gl) : 0;
+      if (r0 >= 0) prefetch_l2(rs.row((unsigned long long)r0), row_bytes);
+      int kind = kBad;
+      unsigned long long ref = 0;
+      if (gl < cnt) {
+        if (rc >= 0) {
+          kind = kHit;
+          ref = (unsigned long long)rs.row((unsigned long long)rc);
+        } else if (rc <= -2) {
+          kind = kNew;
+          ref = (unsigned long long)kc;
+        }
+      }
+      pool_window<G, NV>(kind, ref, cnt, ws, gmask, gl, d4, dim, e, acc, cur, cur_end, outb);
+    }
     while (cur < nb) {
       float4* o = reinterpret_cast<float4*>(outb + (long long)cur * dim);
 #pragma unroll

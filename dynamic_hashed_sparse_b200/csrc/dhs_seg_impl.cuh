@@ -62,6 +62,52 @@ cudaError_t launch(int G, int NV, int sm_count, const unsigned* skey, const unsi
   return cudaErrorInvalidValue;
 }
 
+template <int CPL, int OPT>
+cudaError_t run_w(int sm_count, const unsigned* skey, const unsigned* sval, long long n,
+                  const float* grad, long long n_bags, int dim, RowSpace rs, const OptArgs& oa,
+                  double* part_head, double* part_tail, int pstride, int chunk, unsigned* chunk_ctr,
+                  unsigned* owners, unsigned* owner_ctr, DevState* st, cudaStream_t s) {
+  static int resident = 0;
+  const size_t smem = segw_smem_bytes(CPL);
+  if (!resident) {
+    if (smem > 48 * 1024)
+      cudaFuncSetAttribute(bwd_segw_kernel<CPL, OPT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, bwd_segw_kernel<CPL, OPT>, 256, smem) !=
+            cudaSuccess || per_sm < 1) {
+      cudaGetLastError();
+      per_sm = 1;
+    }
+    resident = per_sm * sm_count;
+  }
+  const long long nchunks = (n + chunk - 1) / chunk;
+  const long long need = std::max<long long>(1, (nchunks + 7) / 8);  // a warp per chunk
+  const long long grid = std::min<long long>(need, resident);
+  bwd_segw_kernel<CPL, OPT><<<(unsigned)grid, 256, smem, s>>>(skey, sval, n, grad, n_bags, dim, rs, oa,
+                                                             part_head, part_tail, pstride, chunk,
+                                                             chunk_ctr, owners, owner_ctr, st);
+  return cudaGetLastError();
+}
+
+template <int OPT>
+cudaError_t launch_w(int cpl, int sm_count, const unsigned* skey, const unsigned* sval, long long n,
+                     const float* grad, long long n_bags, int dim, RowSpace rs, const OptArgs& oa,
+                     double* part_head, double* part_tail, int pstride, int chunk, unsigned* chunk_ctr,
+                     unsigned* owners, unsigned* owner_ctr, DevState* st, cudaStream_t s) {
+#define DHS_RUN(c)                                                                              \
+  run_w<c, OPT>(sm_count, skey, sval, n, grad, n_bags, dim, rs, oa, part_head, part_tail, pstride, \
+                chunk, chunk_ctr, owners, owner_ctr, st, s)
+  switch (cpl) {
+    case 1: return DHS_RUN(1);
+    case 2: return DHS_RUN(2);
+    case 4: return DHS_RUN(4);
+    case 8: return DHS_RUN(8);
+    case 16: return DHS_RUN(16);
+  }
+#undef DHS_RUN
+  return cudaErrorInvalidValue;
+}
+
 }  // namespace seg_impl
 }  // namespace dhs
 
@@ -74,5 +120,14 @@ cudaError_t launch(int G, int NV, int sm_count, const unsigned* skey, const unsi
                     DevState* st, cudaStream_t s) {                                             \
     return seg_impl::launch<OPT_>(G, NV, sm_count, skey, sval, n, grad, n_bags, dim, rs, oa,    \
                                   part_head, part_tail, chunk, chunk_ctr, owners, owner_ctr, st, s); \
+  }                                                                                             \
+  cudaError_t NAME_##_w(int cpl, int sm_count, const unsigned* skey, const unsigned* sval,       \
+                        long long n, const float* grad, long long n_bags, int dim, RowSpace rs,  \
+                        const OptArgs& oa, double* part_head, double* part_tail, int pstride,    \
+                        int chunk, unsigned* chunk_ctr, unsigned* owners, unsigned* owner_ctr,   \
+                        DevState* st, cudaStream_t s) {                                         \
+    return seg_impl::launch_w<OPT_>(cpl, sm_count, skey, sval, n, grad, n_bags, dim, rs, oa,    \
+                                    part_head, part_tail, pstride, chunk, chunk_ctr, owners,    \
+                                    owner_ctr, st, s);                                          \
   }                                                                                             \
   }

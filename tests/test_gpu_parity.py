@@ -143,7 +143,7 @@ def test_forward_is_bit_exact():
         o.close()
 
 
-DIMS = [4, 12, 16, 40, 64, 128, 200, 512]
+DIMS = [4, 12, 16, 32, 40, 64, 128, 132, 200, 260, 512]
 
 
 @pytest.mark.parametrize("opt", ["sgd", "adagrad", "adam", "adagrad_rowwise"])
@@ -171,11 +171,11 @@ def test_dims_and_optimizers(dim, opt):
 
 @pytest.mark.parametrize("occ", [255, 256, 257, 600, 5000, 40000])
 def test_hot_key_spanning_many_sort_chunks(occ):
-    """One key occurs `occ` times (runs over 1, 2, 3, ... sort chunks of 256),
-    mixed with a tail of other keys before and after it in row order."""
+    """One key occurs `occ` times (its run covers one sort chunk of 32 pairs up
+    to hundreds of them), mixed with a tail of other keys before and after it
+    in row order; both segment kernels (narrow and wide rows)."""
     rng = np.random.default_rng(occ)
-    dim = 32
-    for opt in ("adagrad", "adam", "adagrad_rowwise"):
+    for dim, opt in ((32, "adagrad"), (32, "adam"), (32, "adagrad_rowwise"), (12, "adagrad"), (128, "sgd")):
         t, o = make_pair(dim, opt)
         try:
             warm = np.arange(1, 600, dtype=np.int64)  # rows 0.. for the tail keys
@@ -201,13 +201,13 @@ def test_hot_key_spanning_many_sort_chunks(occ):
             o.close()
 
 
+@pytest.mark.parametrize("dim", [16, 64])
 @pytest.mark.parametrize("n_target", [20_000, 150_000, 700_000])
-def test_segment_runs_at_every_chunk_alignment(n_target):
+def test_segment_runs_at_every_chunk_alignment(n_target, dim):
     """Rows with run lengths that put segment starts and ends at every offset
-    of the sort chunks (the chunk size depends on the batch size: 32, 64, 128),
+    of the sort chunks (32 or 64 pairs, by batch size),
     including runs of exactly C, 2C, 3C and one longer or shorter."""
     rng = np.random.default_rng(n_target)
-    dim = 16
     special = []
     for C in (32, 64, 128, 256):
         special += [C - 1, C, C + 1, 2 * C - 1, 2 * C, 2 * C + 1, 3 * C - 1, 3 * C, 3 * C + 1]
