@@ -676,28 +676,39 @@ bwd_seg_kernel(const unsigned* __restrict__ skey, const unsigned* __restrict__ s
 // table row of an owned run is loaded into registers when the run opens and
 // written once when it closes.
 // ---------------------------------------------------------------------------
-__host__ __device__ constexpr int segw_slots(int cpl) { return 64 / cpl < 16 ? 64 / cpl : 16; }
+// Pairs per staged batch (two batches per warp in flight or being read): 8 KB
+// of rows per warp at every width.
+__host__ __device__ constexpr int segw_batch(int cpl) { return cpl <= 2 ? 16 : 32 / cpl; }
 __host__ __device__ constexpr size_t segw_smem_bytes(int cpl) {
-  return (size_t)8 * segw_slots(cpl) * 32 * cpl * sizeof(float);
+  return (size_t)8 * 2 * segw_batch(cpl) * 32 * cpl * sizeof(float);
 }
 
-// This lane's CPL columns of one gradient row into shared memory (zero-filled
-// when !ok or past the row end).  dst and src are aligned to the copy size.
-template <int CPL>
-__device__ __forceinline__ void segw_copy(unsigned dst, const float* src, bool ok, int col0, int dim) {
-  if constexpr (CPL == 1) {
-    asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(dst), "l"(src), "r"(ok ? 4u : 0u)
-                 : "memory");
-  } else if constexpr (CPL == 2) {
-    asm volatile("cp.async.ca.shared.global [%0], [%1], 8, %2;" ::"r"(dst), "l"(src), "r"(ok ? 8u : 0u)
-                 : "memory");
-  } else {
-#pragma unroll
-    for (int k = 0; k < CPL / 4; ++k) {
-      const bool in = ok && col0 + 4 * k < dim;
-      cp_async16(dst + 16u * k, in ? src + 4 * k : src, in ? 16u : 0u);
-    }
+__device__ __forceinline__ void mbar_init(unsigned bar, unsigned count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_arrive(unsigned bar, unsigned bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+// Waits (bounded) until the phase of the given parity has completed.
+constexpr unsigned kMbarSpins = 1u << 22;
+__device__ __forceinline__ bool mbar_wait(unsigned bar, unsigned parity) {
+  for (unsigned i = 0; i < kMbarSpins; ++i) {
+    unsigned done;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}"
+        : "=r"(done)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    if (done) return true;
   }
+  return false;
+}
+// One row (bytes a multiple of 16, both addresses 16-byte aligned) from
+// global into shared memory; completion is counted on the mbarrier.
+__device__ __forceinline__ void bulk_g2s(unsigned dst, const void* src, unsigned bytes, unsigned bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+               "l"(src), "r"(bytes), "r"(bar)
+               : "memory");
 }
 
 // CPL columns of a row at p (p + col0 aligned to the vector width) into v and
@@ -745,16 +756,28 @@ bwd_segw_kernel(const unsigned* __restrict__ skey, const unsigned* __restrict__ 
                 double* __restrict__ part_head, double* __restrict__ part_tail, int pstride, int C,
                 unsigned* __restrict__ chunk_ctr, unsigned* __restrict__ owners,
                 unsigned* __restrict__ owner_ctr, DevState* st) {
-  constexpr int S = segw_slots(CPL);
+  constexpr int B = segw_batch(CPL);
+  constexpr int PITCH = 32 * CPL;  // floats per staged row
   constexpr int NS = seg_state_arrays(OPT);
   constexpr unsigned FULL = 0xffffffffu;
-  extern __shared__ float segw_smem[];
+  extern __shared__ __align__(128) float segw_smem[];
+  __shared__ __align__(8) unsigned long long segw_bar[8][2];
+  __shared__ uint2 segw_runs[8][130];  // per warp: the stream's runs {key, start | mode << 16}
   const int lane = threadIdx.x & 31;
   const int wid = threadIdx.x >> 5;
   const int col0 = lane * CPL;
   const bool lane_on = col0 < dim;
-  float* ring = segw_smem + (size_t)wid * S * 32 * CPL + col0;  // this lane's columns of slot 0
-  const unsigned ring_s = (unsigned)__cvta_generic_to_shared(ring);
+  float* wbuf = segw_smem + (size_t)wid * 2 * B * PITCH;  // this warp's two batches of rows
+  const unsigned wbuf_s = (unsigned)__cvta_generic_to_shared(wbuf);
+  const unsigned bar_s = (unsigned)__cvta_generic_to_shared(&segw_bar[wid][0]);
+  if (lane == 0) {
+    mbar_init(bar_s, 1);
+    mbar_init(bar_s + 8, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncwarp();
+  unsigned parity = 0;  // bit b: parity of the next phase of batch buffer b
+  bool broken = false;
   // positions and bags fit in 31 bits (the host rejects larger calls); C <= 64
   const int n32 = (int)n;
   const unsigned nb32 = (unsigned)n_bags;
@@ -840,44 +863,74 @@ bwd_segw_kernel(const unsigned* __restrict__ skey, const unsigned* __restrict__ 
     const int mode_last = hl == 0 ? mode_first : ((has2 && fwd2 == kl) ? 3 : 2);
     const int stop = mode_last == 2 ? next_head(cend - 1) : (mode_last == 0 ? s0 : cend);
 
-    // distinct rows started in this chunk; L2 prefetch of the owned runs' rows
+    // distinct rows started in this chunk
     {
       unsigned cnt = 0;
 #pragma unroll
       for (int w = 0; w < 4; ++w) {
-        const int q = 32 * w + lane;
-        const unsigned k = kw[w];
         const bool head = (hm[w] >> lane) & 1u;
-        cnt += __popc(__ballot_sync(FULL, head && q < cend && k < nrows));
-        if (head && q >= s0 && q < stop && k < nrows && !(has2 && fwd2 == k))
-          prefetch_l2(rs.row(k), (unsigned)rs.stride * 4u);
+        cnt += __popc(__ballot_sync(FULL, head && 32 * w + lane < cend && kw[w] < nrows));
       }
       nseg_total += cnt;
     }
     if (s0 >= stop) continue;
 
-    // ---- producer: gradient rows of stream pairs s0, s0 + 1, ... into the ring.
-    // A pair whose key has no row or whose bag is out of range copies zeros.
+    // the stream's runs: entry 0 starts at s0, then one entry per head in
+    // (s0, stop), then a sentinel at stop; owned rows are prefetched into L2
+    uint2* runs = segw_runs[wid];
+    int nruns;
+    {
+      const unsigned ks0 = key_at(s0);
+      unsigned base = 1;
+#pragma unroll
+      for (int w = 0; w < 4; ++w) {
+        const int q = 32 * w + lane;
+        const bool h = ((hm[w] >> lane) & 1u) && q > s0 && q < stop;
+        const unsigned m = __ballot_sync(FULL, h);
+        if (h) {
+          const unsigned k = kw[w];
+          const unsigned md = (has2 && fwd2 == k) ? 3u : 2u;
+          runs[base + __popc(m & lanemask_lt())] = make_uint2(k, (unsigned)q | (md << 16));
+          if (md == 2u && k < nrows) prefetch_l2(rs.row(k), (unsigned)rs.stride * 4u);
+        }
+        base += __popc(m);
+      }
+      nruns = (int)base;
+      if (lane == 0) {
+        const unsigned md = s0 == 0 ? (unsigned)mode_first : ((has2 && fwd2 == ks0) ? 3u : 2u);
+        runs[0] = make_uint2(ks0, (unsigned)s0 | (md << 16));
+        runs[nruns] = make_uint2(0u, (unsigned)stop);
+        if (md == 2u && ks0 < nrows) prefetch_l2(rs.row(ks0), (unsigned)rs.stride * 4u);
+      }
+      __syncwarp();
+    }
+
+    // ---- producer: the gradient rows of stream batch j (pairs s0 + j B ...)
+    // into buffer j & 1, one bulk copy per row issued by the lane of that
+    // pair.  A pair whose key has no row or whose bag is out of range is not
+    // copied and not added.
 #pragma unroll
     for (int w = 0; w < 4; ++w) vw[w] = (kw[w] < nrows && vw[w] < nb32) ? vw[w] : ~0u;
-    constexpr unsigned kSlotBytes = 32u * CPL * 4u;
-    int pf = s0;
-    unsigned pword = word(vw, s0);  // bags of the 32-pair word holding pf
-    unsigned pslot = 0;             // byte offset of pf's slot
-    auto produce = [&]() {
-      if (pf < stop) {
-        if ((pf & 31) == 0) pword = word(vw, pf);
-        const unsigned b = __shfl_sync(FULL, pword, pf & 31);
-        const bool ok = lane_on && b != ~0u;
-        const float* src = grad + (size_t)(ok ? b : 0u) * dim + (lane_on ? col0 : 0);
-        segw_copy<CPL>(ring_s + pslot, src, ok, col0, dim);
-      }
-      cp_async_commit();  // one group per pair (empty past the stream end)
-      ++pf;
-      pslot = (pslot + kSlotBytes) & (S * kSlotBytes - 1u);
+    const int nbat = (stop - s0 + B - 1) / B;
+    const unsigned row_bytes = (unsigned)dim * 4u;
+    auto issue = [&](int j) -> unsigned {
+      const int q0 = s0 + j * B;
+      const int q = q0 + lane;
+      const int w0 = q0 >> 5;
+      const unsigned a0 = __shfl_sync(FULL, word(vw, 32 * w0), q & 31);
+      const unsigned a1 = __shfl_sync(FULL, word(vw, min(32 * w0 + 32, 127)), q & 31);
+      const unsigned bg = (q >> 5) == w0 ? a0 : a1;
+      const bool valid = lane < B && q < stop && bg != ~0u;
+      const unsigned vmask = __ballot_sync(FULL, valid);
+      const unsigned bar = bar_s + 8u * (j & 1);
+      // the buffer's previous rows were read by this warp's generic loads
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      if (lane == 0) mbar_expect_arrive(bar, (unsigned)__popc(vmask) * row_bytes);
+      __syncwarp();
+      if (valid)
+        bulk_g2s(wbuf_s + (unsigned)(((j & 1) * B + lane) * PITCH) * 4u, grad + (size_t)bg * dim, row_bytes, bar);
+      return vmask;
     };
-#pragma unroll
-    for (int j = 0; j < S; ++j) produce();
 
     // ---- consumer
     double acc[CPL];
@@ -888,19 +941,19 @@ bwd_segw_kernel(const unsigned* __restrict__ skey, const unsigned* __restrict__ 
     float racc = 0.f;
     unsigned kcur = 0;
     int mode = 0, run_end = 0;
-    auto open = [&](int q) {
-      kcur = key_at(q);
-      mode = q == 0 ? mode_first : ((has2 && fwd2 == kcur) ? 3 : 2);
-      run_end = next_head(q);
-      if (mode != 2) run_end = min(run_end, cend);  // a long piece stops at the chunk end
-      if (mode == 2 && kcur < nrows) {
-        const float* row = rs.row(kcur);
+    // the row of an owned run, loaded into the "next" registers one run ahead
+    float nw[CPL];
+    float nst[NS > 0 ? NS : 1][CPL];
+    float nra = 0.f;
+    auto fetch = [&](uint2 e) {
+      if ((e.y >> 16) == 2u && e.x < nrows) {
+        const float* row = rs.row(e.x);
         if (lane_on) {
-          segw_ld<CPL>(rw, row, col0, dim);
+          segw_ld<CPL>(nw, row, col0, dim);
 #pragma unroll
-          for (int k = 0; k < NS; ++k) segw_ld<CPL>(rst[k], row + (k + 1) * dim, col0, dim);
+          for (int k = 0; k < NS; ++k) segw_ld<CPL>(nst[k], row + (k + 1) * dim, col0, dim);
         }
-        if (OPT == 3) racc = row[dim];
+        if (OPT == 3) nra = row[dim];
       }
     };
     auto close = [&]() {
@@ -953,26 +1006,83 @@ bwd_segw_kernel(const unsigned* __restrict__ skey, const unsigned* __restrict__ 
       for (int e = 0; e < CPL; ++e) acc[e] = 0.0;
     };
 
-    open(s0);
-    int cslot = 0;  // float offset of pair q's slot
-    for (int q = s0; q < stop; ++q) {
-      cp_async_wait<S - 1>();  // pair q's columns have landed (this lane's own copy)
-      if (lane_on) {
-        float x[CPL];
-#pragma unroll
-        for (int e = 0; e < CPL; ++e) x[e] = 0.f;
-        segw_ld<CPL>(x, ring + cslot, 0, dim - col0);
-#pragma unroll
-        for (int e = 0; e < CPL; ++e) acc[e] += (double)x[e];
-      }
-      cslot = (cslot + 32 * CPL) & (S * 32 * CPL - 1);
-      produce();  // refill the slot just read with pair q + S
-      if (q + 1 == run_end) {
-        close();
-        if (q + 1 < stop) open(q + 1);
-      }
+    uint2 ecur = runs[0];
+    fetch(ecur);
+    unsigned vm[2];
+    vm[0] = issue(0);
+    vm[1] = nbat > 1 ? issue(1) : 0u;
+    // batch j holds stream pairs [q0, qbe); runs are the outer loop, the pairs
+    // of a run inside one batch a tight inner loop
+    int j = 0, q0 = s0, qbe = min(s0 + B, stop), q = s0;
+    unsigned vmask = vm[0];
+    const float* rows = wbuf + col0;
+    if (!mbar_wait(bar_s, parity & 1u)) {
+      latch(st, kErrInternal);  // a row copy never completed
+      broken = true;
+      break;
     }
-    cp_async_wait_all();  // the ring is reused by the next chunk
+    parity ^= 1u;
+    for (int r = 0; r < nruns && !broken; ++r) {
+      kcur = ecur.x;
+      mode = (int)(ecur.y >> 16);
+      const uint2 enext = runs[r + 1];
+      run_end = (int)(enext.y & 0xffffu);
+      if (mode != 2) run_end = min(run_end, cend);  // a long piece stops at the chunk end
+#pragma unroll
+      for (int e = 0; e < CPL; ++e) rw[e] = nw[e];
+#pragma unroll
+      for (int k = 0; k < NS; ++k)
+#pragma unroll
+        for (int e = 0; e < CPL; ++e) rst[k][e] = nst[k][e];
+      racc = nra;
+      if (r + 1 < nruns) fetch(enext);  // in flight while this run is summed
+      ecur = enext;
+      while (q < run_end) {
+        if (q == qbe) {
+          // next batch: refill the buffer just finished, wait for the other
+          __syncwarp();  // every lane has read this buffer
+          if (j + 2 < nbat) {
+            const unsigned m = issue(j + 2);
+            if (j & 1) vm[1] = m; else vm[0] = m;
+          }
+          ++j;
+          const int bsel = j & 1;
+          if (!mbar_wait(bar_s + 8u * bsel, (parity >> bsel) & 1u)) {
+            latch(st, kErrInternal);
+            broken = true;
+            break;
+          }
+          parity ^= 1u << bsel;
+          vmask = bsel ? vm[1] : vm[0];
+          rows = wbuf + bsel * B * PITCH + col0;
+          q0 = s0 + j * B;
+          qbe = min(q0 + B, stop);
+        }
+        const int qe = min(run_end, qbe);
+        if (lane_on) {
+          for (; q < qe; ++q) {
+            const int i = q - q0;
+            if ((vmask >> i) & 1u) {
+              float x[CPL];
+#pragma unroll
+              for (int e = 0; e < CPL; ++e) x[e] = 0.f;
+              segw_ld<CPL>(x, rows + i * PITCH, 0, dim - col0);
+#pragma unroll
+              for (int e = 0; e < CPL; ++e) acc[e] += (double)x[e];
+            }
+          }
+        } else {
+          q = qe;
+        }
+      }
+      if (broken) break;
+      close();
+    }
+    if (broken) break;
+  }
+  if (broken) {
+    // let the other buffer's copies (if any) land before the block exits
+    for (int b = 0; b < 2; ++b) (void)mbar_wait(bar_s + 8u * b, (parity >> b) & 1u);
   }
   if (lane == 0 && nseg_total) atomicAdd(&st->sum_unique, (unsigned long long)nseg_total);
 }

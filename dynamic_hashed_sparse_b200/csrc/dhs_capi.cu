@@ -751,33 +751,43 @@ dhs_status embbag_forward(dhs_table* t, const int64_t* d_keys, int64_t n_keys,
   t->last_stream = s;
   if (n_keys > 0) DHS_TRY(ensure_capacity(t, n_keys, s));
   DHS_TRY(ensure_ws(t, n_keys, s));
-  {
-    PhaseScope ph(t, PH_FWD_POOL, s);
-    if (n_keys >= (long long)DHS_POOL_SPLIT_LEN * n_bags && n_keys > 0) {
-      // long bags: probe every id first (a thread per id), then gather
+  if (n_keys >= (long long)DHS_POOL_SPLIT_LEN * n_bags && n_keys > 0) {
+    // long bags: probe every id (a thread per id), assign and write the new
+    // keys' rows, then gather every row from the table
+    {
+      PhaseScope ph(t, PH_FWD_POOL, s);
       fwd_probe_offsets_kernel<<<(unsigned)((n_keys + kFwdThreads - 1) / kFwdThreads), kFwdThreads, 0, s>>>(
           idmap(t), (const long long*)d_keys, n_keys, (long long*)t->b_refs.p, (unsigned*)t->b_nbm.p,
           (unsigned*)t->b_slotpos.p, t->st);
       t->n_launches++;
       DHS_TRY(last_launch());
+    }
+    {
+      PhaseScope ph(t, PH_FWD_ASSIGN, s);
+      DHS_TRY(launch_assign(t, (const long long*)d_keys, n_keys, s));
+    }
+    {
+      PhaseScope ph(t, PH_FWD_POOL, s);
       const int G = pick_group(t->dim), NV = pick_nv(t->dim, G);
       const cudaError_t e =
-          launch_pool_refs(G, NV, t->sm_count, rowspace(t), t->dim, (const long long*)d_keys,
-                           (const long long*)t->b_refs.p, n_keys, (const long long*)d_bag_offsets, n_bags,
-                           d_pooled_out, t->st, s);
+          launch_pool_refs(G, NV, t->sm_count, rowspace(t), t->dim, t->slots, (const long long*)t->b_refs.p,
+                           n_keys, (const long long*)d_bag_offsets, n_bags, d_pooled_out, t->st, s);
       t->n_launches++;
       if (e != cudaSuccess) {
         cudaGetLastError();
         return DHS_ERR_CUDA;
       }
-    } else {
+    }
+  } else {
+    {
+      PhaseScope ph(t, PH_FWD_POOL, s);
       DHS_TRY(dispatch_pool(t, (const long long*)d_keys, n_keys, (const long long*)d_bag_offsets,
                             n_bags, d_pooled_out, s));
     }
-  }
-  if (n_keys > 0) {
-    PhaseScope ph(t, PH_FWD_ASSIGN, s);
-    DHS_TRY(launch_assign(t, (const long long*)d_keys, n_keys, s));
+    if (n_keys > 0) {
+      PhaseScope ph(t, PH_FWD_ASSIGN, s);
+      DHS_TRY(launch_assign(t, (const long long*)d_keys, n_keys, s));
+    }
   }
   t->n_insert_calls++;
   if (n_keys > 0) {

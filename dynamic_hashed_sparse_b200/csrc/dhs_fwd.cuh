@@ -67,9 +67,9 @@ __device__ __forceinline__ long long load_bag_ends(const long long* __restrict__
 // Gather + pool of one window of cnt ids (kind and ref held by lane t of the
 // group for id t of the window): each lane loads NV float4 columns of U rows
 // at a time, then adds them into the current bag's accumulator in id order,
-// writing out each bag as its end is passed.  A new key's row is computed
-// from the key, exactly as the assignment kernel will store it.
-template <int G, int NV>
+// writing out each bag as its end is passed.  With NEW_KEYS, a new key's row
+// is computed from the key, exactly as the assignment kernel stores it.
+template <int G, int NV, bool NEW_KEYS>
 __device__ __forceinline__ void pool_window(int kind, unsigned long long ref, int cnt, int ws,
                                             unsigned gmask, int gl, int d4, int dim, int e,
                                             float4 (&acc)[NV], int& cur, int& cur_end, float* outb) {
@@ -89,7 +89,7 @@ __device__ __forceinline__ void pool_window(int kind, unsigned long long ref, in
         if (t < cnt && c4 < d4) {
           if (kt == kHit)
             x = __ldg(reinterpret_cast<const float4*>(rt) + c4);
-          else if (kt == kNew)
+          else if (NEW_KEYS && kt == kNew)
             x = init_weight4(rt, c4 * 4);
         }
         v[u][q] = x;
@@ -194,7 +194,7 @@ fwd_probe_pool_kernel(IdMap m, RowSpace rs, int dim, const long long* __restrict
           }
         }
       }
-      pool_window<G, NV>(kind, ref, cnt, ws, gmask, gl, d4, dim, e, acc, cur, cur_end, outb);
+      pool_window<G, NV, true>(kind, ref, cnt, ws, gmask, gl, d4, dim, e, acc, cur, cur_end, outb);
     }
     // the bag in progress and any empty bags after it
     while (cur < nb) {
@@ -210,16 +210,16 @@ fwd_probe_pool_kernel(IdMap m, RowSpace rs, int dim, const long long* __restrict
   }
 }
 
-// Gather + pool from per-id row references (the split forward for long bags):
-// refs[p] >= 0 is the row of a hit, <= -2 marks a key new in this call (its
-// row is computed from keys[p]), -1 an id without a row.  The references of
-// the window two ahead are loaded, and the rows of the next window prefetched
-// into L2, while the current window is gathered, so no window waits on a
-// probe.  Bags, windows and the order of additions are those of
-// fwd_probe_pool_kernel.
+// Gather + pool from per-id row references (the split forward for long bags,
+// run after the new keys' rows are assigned and written): refs[p] >= 0 is the
+// row of a hit, <= -2 the slot -(2 + refs[p]) of a key new in this call (its
+// row is the slot's value), -1 an id without a row.  The references of the
+// window two ahead (and the slot values of the next window's new ids) are
+// loaded while the current window is gathered, so no window waits on a probe.
+// Bags, windows and the order of additions are those of fwd_probe_pool_kernel.
 template <int G, int NV>
 __global__ void __launch_bounds__(kFwdThreads, NV == 1 ? 4 : (NV == 2 ? 2 : 1))
-fwd_pool_refs_kernel(RowSpace rs, int dim, const long long* __restrict__ keys,
+fwd_pool_refs_kernel(RowSpace rs, int dim, const Slot* __restrict__ slots,
                      const long long* __restrict__ refs, long long n_keys,
                      const long long* __restrict__ bag_off, long long n_bags,
                      float* __restrict__ out, DevState* st) {
@@ -231,7 +231,6 @@ fwd_pool_refs_kernel(RowSpace rs, int dim, const long long* __restrict__ keys,
   const int ngroups = (int)((gridDim.x * kFwdThreads) / G);
   const int nchunks = (int)((n_bags + G - 1) / G);
   const int d4 = dim >> 2;
-  const unsigned row_bytes = (unsigned)dim * 4u;
 
   for (int c = gid; c < nchunks; c += ngroups) {
     const long long b0 = (long long)c * G;
@@ -250,27 +249,30 @@ fwd_pool_refs_kernel(RowSpace rs, int dim, const long long* __restrict__ keys,
 
     auto ref_at = [&](int p) -> long long { return p < E ? __ldg(refs + p) : -1; };
     long long r0 = ref_at(s + gl), r1 = ref_at(s + G + gl);
-    long long k0 = r0 <= -2 ? __ldg(keys + s + gl) : 0;
-    if (r0 >= 0) prefetch_l2(rs.row((unsigned long long)r0), row_bytes);
+    // the row of a new key (PENDING if its assignment failed: the table is full)
+    auto new_row = [&](long long r) -> unsigned long long {
+      return r <= -2 ? __ldg(&slots[-2 - r].val) : kPending;
+    };
+    unsigned long long n0 = new_row(r0);
     for (int ws = s; ws < E; ws += G) {
       const int cnt = min(G, E - ws);
-      const long long rc = r0, kc = k0;
+      const long long rc = r0;
+      const unsigned long long nc = n0;
       r0 = r1;
       r1 = ref_at(ws + 2 * G + gl);
-      k0 = r0 <= -2 ? __ldg(keys + ws + G + gl) : 0;
-      if (r0 >= 0) prefetch_l2(rs.row((unsigned long long)r0), row_bytes);
+      n0 = new_row(r0);
       int kind = kBad;
       unsigned long long ref = 0;
       if (gl < cnt) {
         if (rc >= 0) {
           kind = kHit;
           ref = (unsigned long long)rs.row((unsigned long long)rc);
-        } else if (rc <= -2) {
-          kind = kNew;
-          ref = (unsigned long long)kc;
+        } else if (rc <= -2 && !(nc & kPending)) {
+          kind = kHit;
+          ref = (unsigned long long)rs.row(nc);
         }
       }
-      pool_window<G, NV>(kind, ref, cnt, ws, gmask, gl, d4, dim, e, acc, cur, cur_end, outb);
+      pool_window<G, NV, false>(kind, ref, cnt, ws, gmask, gl, d4, dim, e, acc, cur, cur_end, outb);
     }
     while (cur < nb) {
       float4* o = reinterpret_cast<float4*>(outb + (long long)cur * dim);

@@ -17,7 +17,7 @@ cudaError_t launch_probe_pool(int G, int NV, int sm_count, IdMap m, RowSpace rs,
                               DevState* st, cudaStream_t s);
 
 // fwd_pool_refs_kernel<G, NV> (gather + pool from per-id row references)
-cudaError_t launch_pool_refs(int G, int NV, int sm_count, RowSpace rs, int dim, const long long* keys,
+cudaError_t launch_pool_refs(int G, int NV, int sm_count, RowSpace rs, int dim, const Slot* slots,
                              const long long* refs, long long n_keys, const long long* bag_off,
                              long long n_bags, float* out, DevState* st, cudaStream_t s);
 

@@ -34,7 +34,7 @@ cudaError_t run(int sm_count, IdMap m, RowSpace rs, int dim, const long long* ke
 }
 
 template <int G, int NV>
-cudaError_t run_refs(int sm_count, RowSpace rs, int dim, const long long* keys, const long long* refs,
+cudaError_t run_refs(int sm_count, RowSpace rs, int dim, const Slot* slots, const long long* refs,
                      long long n_keys, const long long* bag_off, long long n_bags, float* out,
                      DevState* st, cudaStream_t s) {
   static int resident = 0;
@@ -51,7 +51,7 @@ cudaError_t run_refs(int sm_count, RowSpace rs, int dim, const long long* keys, 
   const long long per_block = kFwdThreads / G;
   const long long need = std::max<long long>(1, (nchunks + per_block - 1) / per_block);
   const long long grid = std::min<long long>(need, resident);
-  fwd_pool_refs_kernel<G, NV><<<(unsigned)grid, kFwdThreads, 0, s>>>(rs, dim, keys, refs, n_keys, bag_off,
+  fwd_pool_refs_kernel<G, NV><<<(unsigned)grid, kFwdThreads, 0, s>>>(rs, dim, slots, refs, n_keys, bag_off,
                                                                       n_bags, out, st);
   return cudaGetLastError();
 }
@@ -76,10 +76,10 @@ cudaError_t launch_probe_pool(int G, int NV, int sm_count, IdMap m, RowSpace rs,
   return cudaErrorInvalidValue;
 }
 
-cudaError_t launch_pool_refs(int G, int NV, int sm_count, RowSpace rs, int dim, const long long* keys,
+cudaError_t launch_pool_refs(int G, int NV, int sm_count, RowSpace rs, int dim, const Slot* slots,
                              const long long* refs, long long n_keys, const long long* bag_off,
                              long long n_bags, float* out, DevState* st, cudaStream_t s) {
-#define DHS_RUN(g, v) run_refs<g, v>(sm_count, rs, dim, keys, refs, n_keys, bag_off, n_bags, out, st, s)
+#define DHS_RUN(g, v) run_refs<g, v>(sm_count, rs, dim, slots, refs, n_keys, bag_off, n_bags, out, st, s)
   switch (G * 100 + NV) {
     case 101: return DHS_RUN(1, 1);
     case 201: return DHS_RUN(2, 1);
