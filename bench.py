@@ -33,6 +33,9 @@ from workloads import gen  # noqa: E402
 
 METRIC = "IDs/sec & HBM GB/s (% of peak): hashed lookup+bag-sum fwd, sparse update bwd"
 UNIT = "IDs/s"
+# kernel selection thresholds of the library (compile-time constants there)
+POOL_SPLIT_LEN = 4   # bags of >= 4 ids on average: probe kernel + gather from references
+SEGW_MIN_DIM = 32    # rows of >= 32 floats: warp-per-chunk segment kernel
 WORKLOAD = "dlrm_merged_26"
 
 
@@ -50,9 +53,12 @@ def alg_bytes(n: int, b: int, u: int, m: int, dim: int, opt: str) -> dict:
     pack = 4 * n + 8 * n + 8 * n
     fwd_pool = 8 * n + 8 * (b + 1) + 16 * u + 16 * m + R * (u - m) + 4 * dim * b
     fwd_assign = S * m + 16 * m
+    # the split forward (long bags) gathers every distinct row, new ones included,
+    # after the assignment wrote them
+    fwd_refs = 8 * (b + 1) + R * u + 4 * dim * b
     bwd = 8 * n + 8 * (b + 1) + 16 * u + 4 * dim * b + 2 * S * u
-    return dict(pack=pack, fwd_pool=fwd_pool, fwd_assign=fwd_assign,
-                fwd=pack + fwd_pool + fwd_assign, bwd=bwd,
+    return dict(pack=pack, fwd_pool=fwd_pool, fwd_refs=fwd_refs, fwd_assign=fwd_assign,
+                fwd=fwd_pool + fwd_assign, bwd=bwd,
                 bwd_seg=4 * dim * b + 2 * S * u + 8 * n)
 
 
@@ -409,11 +415,14 @@ def run_dhs(args):
     peaks = load_peaks()
     ph_ms = {k: v[0] for k, v in phases.items()}
     ph_cnt = {k: v[1] for k, v in phases.items()}
-    fwd_ms = ph_ms["fwd_probe_pool"] + ph_ms["fwd_assign"]
-    bwd_ms = ph_ms["bwd_probe"] + ph_ms["bwd_sort"] + ph_ms["bwd_seg_update"]
+    fwd_ms = ph_ms["fwd_probe"] + ph_ms["fwd_probe_pool"] + ph_ms["fwd_assign"]
+    bwd_ms = ph_ms["bwd_probe"] + ph_ms["bwd_sort"] + ph_ms["bwd_seg_update"] + ph_ms["bwd_combine"]
     dom = max(("fwd_probe_pool", "bwd_seg_update"), key=lambda k: ph_ms[k])
-    dom_kernel = {"fwd_probe_pool": "fwd_probe_pool_kernel", "bwd_seg_update": "bwd_seg_kernel"}[dom]
-    dom_bytes = ab["fwd_pool"] if dom == "fwd_probe_pool" else ab["bwd_seg"]
+    dom_kernel = {"fwd_probe_pool": ("fwd_pool_refs_kernel" if n_ids >= POOL_SPLIT_LEN * n_bags
+                                     else "fwd_probe_pool_kernel"),
+                  "bwd_seg_update": "bwd_segw_kernel" if w.dim >= SEGW_MIN_DIM else "bwd_seg_kernel"}[dom]
+    dom_bytes = ((ab["fwd_refs"] if dom_kernel == "fwd_pool_refs_kernel" else ab["fwd_pool"])
+                 if dom == "fwd_probe_pool" else ab["bwd_seg"])
     dom_launch_ms = ph_ms[dom] / max(1, ph_cnt[dom])
     dom_bytes_per_launch = dom_bytes / max(1, ph_cnt[dom])
     achieved = dom_bytes_per_launch / (dom_launch_ms / 1e3) / 1e9

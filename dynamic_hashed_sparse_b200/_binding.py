@@ -23,7 +23,7 @@ STATUS = {
 }
 OPT_CODES = {"sgd": 0, "adagrad": 1, "adam": 2, "adagrad_rowwise": 3}
 PHASES = ("fwd_probe_pool", "fwd_assign", "bwd_probe", "bwd_sort", "bwd_seg_update",
-          "lookup_or_insert", "idmap_growth")
+          "lookup_or_insert", "idmap_growth", "fwd_probe", "bwd_combine")
 
 
 class DhsError(RuntimeError):

@@ -42,6 +42,11 @@
 #ifndef DHS_SEGW_MIN_DIM
 #define DHS_SEGW_MIN_DIM 32
 #endif
+//   DHS_SEGW_EVICT_FIRST 1: gradient rows of calls with about one id per bag
+//                     are staged with an L2 evict-first policy; 0: normal
+#ifndef DHS_SEGW_EVICT_FIRST
+#define DHS_SEGW_EVICT_FIRST 1
+#endif
 #ifndef DHS_RADIX_MINB
 #define DHS_RADIX_MINB 5
 #endif
@@ -704,11 +709,24 @@ __device__ __forceinline__ bool mbar_wait(unsigned bar, unsigned parity) {
   return false;
 }
 // One row (bytes a multiple of 16, both addresses 16-byte aligned) from
-// global into shared memory; completion is counted on the mbarrier.
-__device__ __forceinline__ void bulk_g2s(unsigned dst, const void* src, unsigned bytes, unsigned bar) {
-  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
-               "l"(src), "r"(bytes), "r"(bar)
-               : "memory");
+// global into shared memory; completion is counted on the mbarrier.  The L2
+// policy marks rows read once as first to evict, so that they do not push out
+// the rows and keys the kernel reads again.
+__device__ __forceinline__ void bulk_g2s(unsigned dst, const void* src, unsigned bytes, unsigned bar,
+                                         unsigned long long policy) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;" ::"r"(
+          dst),
+      "l"(src), "r"(bytes), "r"(bar), "l"(policy)
+      : "memory");
+}
+__device__ __forceinline__ unsigned long long l2_policy(bool evict_first) {
+  unsigned long long p;
+  if (evict_first)
+    asm("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  else
+    asm("createpolicy.fractional.L2::evict_normal.b64 %0, 1.0;" : "=l"(p));
+  return p;
 }
 
 // CPL columns of a row at p (p + col0 aligned to the vector width) into v and
@@ -755,7 +773,7 @@ bwd_segw_kernel(const unsigned* __restrict__ skey, const unsigned* __restrict__ 
                 const float* __restrict__ grad, long long n_bags, int dim, RowSpace rs, OptArgs oa,
                 double* __restrict__ part_head, double* __restrict__ part_tail, int pstride, int C,
                 unsigned* __restrict__ chunk_ctr, unsigned* __restrict__ owners,
-                unsigned* __restrict__ owner_ctr, DevState* st) {
+                unsigned* __restrict__ owner_ctr, DevState* st, bool grad_once) {
   constexpr int B = segw_batch(CPL);
   constexpr int PITCH = 32 * CPL;  // floats per staged row
   constexpr int NS = seg_state_arrays(OPT);
@@ -778,6 +796,7 @@ bwd_segw_kernel(const unsigned* __restrict__ skey, const unsigned* __restrict__ 
   __syncwarp();
   unsigned parity = 0;  // bit b: parity of the next phase of batch buffer b
   bool broken = false;
+  const unsigned long long grad_policy = l2_policy(grad_once);
   // positions and bags fit in 31 bits (the host rejects larger calls); C <= 64
   const int n32 = (int)n;
   const unsigned nb32 = (unsigned)n_bags;
@@ -928,7 +947,8 @@ bwd_segw_kernel(const unsigned* __restrict__ skey, const unsigned* __restrict__ 
       if (lane == 0) mbar_expect_arrive(bar, (unsigned)__popc(vmask) * row_bytes);
       __syncwarp();
       if (valid)
-        bulk_g2s(wbuf_s + (unsigned)(((j & 1) * B + lane) * PITCH) * 4u, grad + (size_t)bg * dim, row_bytes, bar);
+        bulk_g2s(wbuf_s + (unsigned)(((j & 1) * B + lane) * PITCH) * 4u, grad + (size_t)bg * dim, row_bytes, bar,
+                 grad_policy);
       return vmask;
     };
 
@@ -1100,10 +1120,11 @@ bwd_segw_kernel(const unsigned* __restrict__ skey, const unsigned* __restrict__ 
 // the last of the run's batches to finish (an atomic ticket; no block waits)
 // adds the slots in batch order and applies the optimizer once.  Every sum is
 // taken in an order fixed by the run alone.
-constexpr int kCombineThreads = 256;
+constexpr int kCombineThreads = 128;
 constexpr int kCombinePieces = 128;
 
 struct CombinePlan {
+  unsigned* key;          // [owners] row of the run
   unsigned* kend;         // [owners] chunk holding the last pair
   unsigned* boff;         // [owners] first batch id
   unsigned* sbase;        // [owners] first slot (runs of more than one batch)
@@ -1147,6 +1168,7 @@ bwd_combine_plan_kernel(const unsigned* __restrict__ skey, long long n, int C,
         latch(st, kErrInternal);  // the caps bound every run of sorted input
         base = pl.batch_cap;
       }
+      pl.key[oi] = key;
       pl.kend[oi] = (unsigned)lo;
       pl.boff[oi] = base;
       pl.sbase[oi] = sb;
@@ -1173,7 +1195,7 @@ bwd_combine_kernel(const unsigned* __restrict__ skey, int dim, RowSpace rs, OptA
     const unsigned oi = pl.batch_owner[bid];
     if (oi >= n_own) continue;  // only after a plan overflow, which the plan reported
     const long long c = owners[oi];
-    const unsigned key = skey[(c + 1) * (long long)C - 1];
+    const unsigned key = pl.key[oi];
     const long long npieces = (long long)pl.kend[oi] - c + 1;
     const unsigned b = bid - pl.boff[oi];
     const unsigned nb = (unsigned)((npieces + kCombinePieces - 1) / kCombinePieces);

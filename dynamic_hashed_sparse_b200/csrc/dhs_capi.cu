@@ -41,7 +41,7 @@ int seg_chunk(long long n) {
 }
 constexpr int kSnapRing = 4;
 enum { PH_FWD_POOL = 0, PH_FWD_ASSIGN = 1, PH_BWD_PROBE = 2, PH_BWD_SORT = 3, PH_BWD_SEG = 4,
-       PH_LOOKUP_INSERT = 5, PH_GROW = 6 };
+       PH_LOOKUP_INSERT = 5, PH_GROW = 6, PH_FWD_PROBE = 7, PH_BWD_COMBINE = 8 };
 
 struct Snap {
   cudaEvent_t ev = nullptr;
@@ -385,14 +385,15 @@ dhs_status ensure_capacity(dhs_table* t, long long n, cudaStream_t s) {
 constexpr long long combine_batch_cap(long long nchunks) { return nchunks / 2 + 2 * nchunks / kCombinePieces + 64; }
 constexpr long long combine_slot_cap(long long nchunks) { return 4 * nchunks / kCombinePieces + 64; }
 
-// The plan arrays cut from one buffer of 4 nchunks + batch cap words.
+// The plan arrays cut from one buffer of 5 nchunks + batch cap words.
 CombinePlan combine_plan(unsigned* words, double* slots, long long nchunks, unsigned* zeroed) {
   CombinePlan pl;
-  pl.kend = words;
-  pl.boff = words + nchunks;
-  pl.sbase = words + 2 * nchunks;
-  pl.ticket = words + 3 * nchunks;
-  pl.batch_owner = words + 4 * nchunks;
+  pl.key = words;
+  pl.kend = words + nchunks;
+  pl.boff = words + 2 * nchunks;
+  pl.sbase = words + 3 * nchunks;
+  pl.ticket = words + 4 * nchunks;
+  pl.batch_owner = words + 5 * nchunks;
   pl.slots = slots;
   pl.batch_cap = (unsigned)combine_batch_cap(nchunks);
   pl.slot_cap = (unsigned)combine_slot_cap(nchunks);
@@ -426,7 +427,7 @@ dhs_status ensure_ws(dhs_table* t, long long n, cudaStream_t s) {
   DHS_TRY(bget(t, t->b_ph, (size_t)nchunks * pstride * 8, s));
   DHS_TRY(bget(t, t->b_pt, (size_t)nchunks * pstride * 8, s));
   DHS_TRY(bget(t, t->b_owners, nchunks * 4, s));
-  DHS_TRY(bget(t, t->b_cplan, (size_t)(4 * nchunks + combine_batch_cap(nchunks)) * 4, s));
+  DHS_TRY(bget(t, t->b_cplan, (size_t)(5 * nchunks + combine_batch_cap(nchunks)) * 4, s));
   DHS_TRY(bget(t, t->b_slots, (size_t)combine_slot_cap(nchunks) * pstride * 8, s));
   DHS_CUDA(cudaMemsetAsync(t->b_nbm.p, 0, t->b_nbm.bytes, s));
   t->ws_n = cap;
@@ -447,7 +448,7 @@ dhs_status launch_combine(dhs_table* t, const unsigned* skey, long long n, const
   t->n_launches++;
   DHS_TRY(last_launch());
   const size_t smem = (size_t)std::max(kCombineThreads, t->dim) * sizeof(double);
-  bwd_combine_kernel<<<(unsigned)t->sm_count * 4, kCombineThreads, smem, s>>>(
+  bwd_combine_kernel<<<(unsigned)t->sm_count * 16, kCombineThreads, smem, s>>>(
       skey, t->dim, rowspace(t), oa, part_head, part_tail, chunk, pstride, owners, owner_ctr, pl);
   t->n_launches++;
   return last_launch();
@@ -755,7 +756,7 @@ dhs_status embbag_forward(dhs_table* t, const int64_t* d_keys, int64_t n_keys,
     // long bags: probe every id (a thread per id), assign and write the new
     // keys' rows, then gather every row from the table
     {
-      PhaseScope ph(t, PH_FWD_POOL, s);
+      PhaseScope ph(t, PH_FWD_PROBE, s);
       fwd_probe_offsets_kernel<<<(unsigned)((n_keys + kFwdThreads - 1) / kFwdThreads), kFwdThreads, 0, s>>>(
           idmap(t), (const long long*)d_keys, n_keys, (long long*)t->b_refs.p, (unsigned*)t->b_nbm.p,
           (unsigned*)t->b_slotpos.p, t->st);
@@ -863,7 +864,6 @@ dhs_status embbag_backward_update(dhs_table* t, const int64_t* d_keys, int64_t n
     }
   }
   {
-    PhaseScope ph(t, PH_BWD_SEG, s);
     OptArgs oa;
     oa.opt = t->opt;
     oa.lr = lr;
@@ -874,7 +874,11 @@ dhs_status embbag_backward_update(dhs_table* t, const int64_t* d_keys, int64_t n
     oa.c2 = (float)(1.0 - (double)t->b2);
     oa.bc1 = (float)(1.0 - std::pow((double)t->b1, (double)t->adam_t));
     oa.bc2 = (float)(1.0 - std::pow((double)t->b2, (double)t->adam_t));
-    DHS_TRY(dispatch_seg(t, ka, va, n_keys, d_grad, n_bags, oa, s));
+    {
+      PhaseScope ph(t, PH_BWD_SEG, s);
+      DHS_TRY(dispatch_seg(t, ka, va, n_keys, d_grad, n_bags, oa, s));
+    }
+    PhaseScope ph(t, PH_BWD_COMBINE, s);
     const int pstride = seg_nv(t->dim) * seg_group(t->dim) * 4;
     DHS_TRY(launch_combine(t, ka, n_keys, oa, (const double*)t->b_ph.p, (const double*)t->b_pt.p,
                            seg_chunk(n_keys), pstride, (const unsigned*)t->b_owners.p,
@@ -1039,7 +1043,7 @@ constexpr size_t kNaStatus =
 constexpr size_t kNaChunks = (kNoAllocMaxKeys + kNoAllocMinChunk - 1) / kNoAllocMinChunk;
 constexpr size_t kNaPart = na_align(kNaChunks * kNoAllocMaxDim * 8);  // one of part_head, part_tail
 constexpr size_t kNaOwners = na_align(kNaChunks * 4);
-constexpr size_t kNaPlan = na_align((4 * kNaChunks + combine_batch_cap(kNaChunks)) * 4);
+constexpr size_t kNaPlan = na_align((5 * kNaChunks + combine_batch_cap(kNaChunks)) * 4);
 constexpr size_t kNaSlots = na_align(combine_slot_cap(kNaChunks) * kNoAllocMaxDim * 8);
 constexpr size_t kNoAllocScratchBytes =
     4 * kNaPairs + kNaSortZero + kNaStatus + 2 * kNaPart + kNaOwners + kNaPlan + kNaSlots;

@@ -83,9 +83,12 @@ cudaError_t run_w(int sm_count, const unsigned* skey, const unsigned* sval, long
   const long long nchunks = (n + chunk - 1) / chunk;
   const long long need = std::max<long long>(1, (nchunks + 7) / 8);  // a warp per chunk
   const long long grid = std::min<long long>(need, resident);
+  // gradient rows read about once per call (about one id per bag) are marked
+  // first to evict in L2
+  const bool grad_once = DHS_SEGW_EVICT_FIRST && 2 * n <= 3 * n_bags;
   bwd_segw_kernel<CPL, OPT><<<(unsigned)grid, 256, smem, s>>>(skey, sval, n, grad, n_bags, dim, rs, oa,
                                                              part_head, part_tail, pstride, chunk,
-                                                             chunk_ctr, owners, owner_ctr, st);
+                                                             chunk_ctr, owners, owner_ctr, st, grad_once);
   return cudaGetLastError();
 }
 

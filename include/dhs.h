@@ -221,9 +221,12 @@ dhs_status ht_export(dhs_table* t, int64_t* h_keys, float* h_rows);
 dhs_status ht_counters(dhs_table* t, int64_t out[14]);
 
 /* Per-phase device time, measured with CUDA events recorded on the call's
- * stream around each phase while enabled.  Phases: 0 forward probe + pool,
- * 1 forward offset assignment + row init, 2 backward probe, 3 backward sort,
- * 4 backward segment reduce + update, 5 lookup-or-insert, 6 IDMap growth.
+ * stream around each phase while enabled.  Phases: 0 forward pool (with the
+ * probe when bags are short), 1 forward offset assignment + row init,
+ * 2 backward probe, 3 backward sort, 4 backward segment reduce + update,
+ * 5 lookup-or-insert, 6 IDMap growth, 7 forward probe (long bags: the probe
+ * runs as its own kernel before the assignment), 8 backward combine of rows
+ * that span three or more sort chunks.
  * ht_phase_times synchronises, writes ms_out[p] = total ms and
  * count_out[p] = number of timed launches of phase p (p < n), then clears. */
 dhs_status ht_set_phase_timing(dhs_table* t, int enable);

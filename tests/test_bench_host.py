@@ -55,6 +55,8 @@ def test_algorithmic_bytes_formula():
     R, S = 32, 64
     assert ab["fwd_pool"] == 8 * 10 + 8 * 5 + 16 * 6 + 16 * 2 + R * 4 + 4 * 8 * 4
     assert ab["fwd_assign"] == S * 2 + 16 * 2
+    assert ab["fwd"] == ab["fwd_pool"] + ab["fwd_assign"]  # key packing is timed outside the forward
+    assert ab["fwd_refs"] == 8 * 5 + R * 6 + 4 * 8 * 4
     assert ab["bwd"] == 8 * 10 + 8 * 5 + 16 * 6 + 4 * 8 * 4 + 2 * S * 6
     assert bench.stride_floats(32, "adam") == 96 and bench.stride_floats(16, "adagrad_rowwise") == 20
 
