@@ -12,6 +12,8 @@
 // the pieces are then added in batches and the batch sums in a fixed order.
 #pragma once
 
+#include <climits>
+
 #include "dhs_device.cuh"
 
 // Tuning constants (compile-time; -D overrides them when sweeping):
@@ -22,7 +24,7 @@
 #define DHS_SEG_PREFETCH 0
 #endif
 #ifndef DHS_RADIX_ITEMS
-#define DHS_RADIX_ITEMS 8
+#define DHS_RADIX_ITEMS 16
 #endif
 //   DHS_SEG_MINB      resident 256-thread blocks per SM the segment kernel is
 //                     compiled for (register budget) when a lane holds one
@@ -48,7 +50,7 @@
 #define DHS_SEGW_EVICT_FIRST 1
 #endif
 #ifndef DHS_RADIX_MINB
-#define DHS_RADIX_MINB 5
+#define DHS_RADIX_MINB 3
 #endif
 //   DHS_HIST_MATCH    1: digit counts are combined per warp (match_any) before
 //                     the shared-memory atomic; 0: one atomic per key and pass
@@ -63,62 +65,108 @@ namespace dhs {
 // ---------------------------------------------------------------------------
 
 #ifndef DHS_TEMPLATES_ONLY
-// Warp per chunk of 32 bags; positions 32 at a time, one per lane.  A lane
-// finds its bag by counting the chunk's bag ends at or before its position.
-// Missing or negative keys get row `sentinel` (sorted last, never updated).
+// Warp per chunk of bpc bags (64 when bags are short, 32 when they are long,
+// so that long bags still spread over enough warps); positions 64 at a time,
+// two per lane, so that each lane has two probes in flight.  A position's bag
+// is the number of the chunk's bag ends at or before it (a binary search over
+// the ends held in the lanes' registers).  Missing or negative keys get row `sentinel` (sorted
+// last, never updated).
 __global__ void __launch_bounds__(256)
 bwd_probe_kernel(IdMap m, const long long* __restrict__ keys, long long n_keys,
                  const long long* __restrict__ bag_off, long long n_bags,
                  unsigned* __restrict__ rkey, unsigned* __restrict__ rval, unsigned sentinel,
-                 unsigned* __restrict__ sort_zero, int sort_zero_words, DevState* st) {
+                 unsigned* __restrict__ sort_zero, int sort_zero_words, int bpc, DevState* st) {
+  constexpr unsigned FULL = 0xffffffffu;
   const int lane = threadIdx.x & 31;
   if (blockIdx.x == 0)  // the sort's digit histograms and tile counters start at zero
     for (int i = threadIdx.x; i < sort_zero_words; i += blockDim.x) sort_zero[i] = 0u;
-  const long long nchunks = (n_bags + 31) / 32;
+  // positions and bags fit in 31 bits (the host rejects larger calls)
+  const int n = (int)n_keys;
+  const long long nchunks = (n_bags + bpc - 1) / bpc;
   const long long nw = ((long long)gridDim.x * blockDim.x) >> 5;
   for (long long c = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5; c < nchunks;
        c += nw) {
-    const long long b0 = c * 32;
-    const int nb = (int)min(32ll, n_bags - b0);
-    long long s = __ldg(bag_off + b0);
-    bool bad = (b0 == 0 && s != 0) || s < 0 || s > n_keys;
-    s = s < 0 ? 0 : (s > n_keys ? n_keys : s);
-    long long e = lane < nb ? __ldg(bag_off + b0 + lane + 1) : n_keys;
-    if (lane < nb && (e < s || e > n_keys || (b0 + lane + 1 == n_bags && e != n_keys))) bad = true;
-    e = e < s ? s : (e > n_keys ? n_keys : e);
+    // a chunk of bpc (32 or 64) bags: lane l holds the ends of bags b0 + l and
+    // b0 + 32 + l
+    const long long b0 = c * bpc;
+    const int nb = (int)min((long long)bpc, n_bags - b0);
+    long long s64 = __ldg(bag_off + b0);
+    long long x0 = lane < nb ? __ldg(bag_off + b0 + lane + 1) : n_keys;
+    long long x1 = lane + 32 < nb ? __ldg(bag_off + b0 + lane + 33) : n_keys;
+    bool bad = (b0 == 0 && s64 != 0) || s64 < 0 || s64 > n_keys;
+    s64 = s64 < 0 ? 0 : (s64 > n_keys ? n_keys : s64);
+    if (lane < nb && (x0 < s64 || x0 > n_keys || (b0 + lane + 1 == n_bags && x0 != n_keys))) bad = true;
+    if (lane + 32 < nb && (x1 < s64 || x1 > n_keys || (b0 + lane + 33 == n_bags && x1 != n_keys))) bad = true;
+    int s = (int)s64;
+    int e0 = (int)(x0 < s64 ? s64 : (x0 > n_keys ? n_keys : x0));
+    int e1 = (int)(x1 < s64 ? s64 : (x1 > n_keys ? n_keys : x1));
+    // running max, so that ends never decrease along the chunk
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
-      const long long x = __shfl_up_sync(0xffffffffu, e, o);
-      if (lane >= o && x > e) {
-        e = x;
+      const int y = __shfl_up_sync(FULL, e0, o);
+      if (lane >= o && y > e0) {
+        e0 = y;
+        bad = true;
+      }
+    }
+    {
+      const int carry = __shfl_sync(FULL, e0, 31);
+      if (carry > e1) {
+        e1 = carry;
+        if (lane + 32 < nb) bad = true;
+      }
+    }
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(FULL, e1, o);
+      if (lane >= o && y > e1) {
+        e1 = y;
         bad = true;
       }
     }
     // every position must get a (row, bag) pair even when the offsets are
     // malformed: the first bag starts at 0 and the last one ends at n_keys
     if (b0 == 0) s = 0;
-    if (lane == nb - 1 && b0 + nb == n_bags) e = n_keys;
-    if (lane >= nb) e = LLONG_MAX;
+    if (b0 + nb == n_bags) {
+      if (lane == nb - 1) e0 = n;
+      if (lane + 32 == nb - 1) e1 = n;
+    }
+    if (lane >= nb) e0 = INT_MAX;
+    if (lane + 32 >= nb) e1 = INT_MAX;
     if (bad) latch(st, kErrInvalid);
-    const long long E = __shfl_sync(0xffffffffu, e, nb - 1);
-    for (long long ws = s; ws < E; ws += 32) {
-      const long long p = ws + lane;
-      int cnt = 0;
-      for (int j = 0; j < nb; ++j) cnt += (__shfl_sync(0xffffffffu, e, j) <= p);
-      if (p < E) {
-        const long long k = __ldg(keys + p);
-        unsigned r = sentinel;
-        if (k < 0) {
-          latch(st, kErrInvalid);
-        } else {
-          const long long off = probe_find(m, (unsigned long long)k);
-          if (off < 0)
-            latch(st, kErrNotFound);
-          else
-            r = (unsigned)off;
-        }
-        rkey[p] = r;
-        rval[p] = (unsigned)(b0 + cnt);
+    const int E = nb > 32 ? __shfl_sync(FULL, e1, nb - 33) : __shfl_sync(FULL, e0, nb - 1);
+    // bag of position p: the number of bag ends <= p (binary search over the 64)
+    auto bag_of = [&](int p) -> int {
+      int lo = 0;
+#pragma unroll
+      for (int step = 32; step >= 1; step >>= 1) {
+        const int j = lo + step - 1;
+        const int a0 = __shfl_sync(FULL, e0, j & 31);
+        const int a1 = __shfl_sync(FULL, e1, j & 31);
+        if ((j < 32 ? a0 : a1) <= p) lo += step;
+      }
+      return lo;
+    };
+    for (int ws = s; ws < E; ws += 64) {
+      const int p0 = ws + lane, p1 = ws + 32 + lane;
+      // both positions' keys and probes are in flight together
+      const long long k0 = p0 < E ? __ldg(keys + p0) : 0;
+      const long long k1 = p1 < E ? __ldg(keys + p1) : 0;
+      long long f0 = -1, f1 = -1;
+      if (p0 < E && k0 >= 0) f0 = probe_find(m, (unsigned long long)k0);
+      if (p1 < E && k1 >= 0) f1 = probe_find(m, (unsigned long long)k1);
+      const int g0 = bag_of(p0), g1 = bag_of(p1);
+      if (p0 < E) {
+        if (k0 < 0) latch(st, kErrInvalid);
+        else if (f0 < 0) latch(st, kErrNotFound);
+        rkey[p0] = f0 >= 0 ? (unsigned)f0 : sentinel;
+        rval[p0] = (unsigned)(b0 + g0);
+      }
+      if (p1 < E) {
+        if (k1 < 0) latch(st, kErrInvalid);
+        else if (f1 < 0) latch(st, kErrNotFound);
+        rkey[p1] = f1 >= 0 ? (unsigned)f1 : sentinel;
+        rval[p1] = (unsigned)(b0 + g1);
       }
     }
   }

@@ -466,6 +466,10 @@ dhs_status dispatch_pool(dhs_table* t, const long long* keys, long long n, const
   return e == cudaSuccess ? DHS_OK : DHS_ERR_CUDA;
 }
 
+// Bags per warp of the backward probe: 64 when bags are short (two positions
+// per lane come from different bags), 32 when they are long (more warps).
+int bwd_probe_bags(long long n_keys, long long n_bags) { return n_keys < 4 * n_bags ? 64 : 32; }
+
 // Segment kernel for one backward: the warp-per-chunk kernel for rows of at
 // least DHS_SEGW_MIN_DIM floats, the lane-group kernel below that.
 int segw_cpl(int dim) {
@@ -832,12 +836,13 @@ dhs_status embbag_backward_update(dhs_table* t, const int64_t* d_keys, int64_t n
     PhaseScope ph(t, PH_BWD_PROBE, s);
     static int resident = 0;
     if (!resident) resident = resident_blocks(bwd_probe_kernel, 256, 0, t->sm_count);
-    const long long warps = (n_bags + 31) / 32;
+    const int bpc = bwd_probe_bags(n_keys, n_bags);
+    const long long warps = (n_bags + bpc - 1) / bpc;
     const long long grid = grid_for((warps + 7) / 8, resident);
     bwd_probe_kernel<<<(unsigned)grid, 256, 0, s>>>(idmap(t), (const long long*)d_keys, n_keys,
                                                     (const long long*)d_bag_offsets, n_bags, ka, va,
                                                     sentinel, (unsigned*)t->b_hist.p, kSortZeroWords,
-                                                    t->st);
+                                                    bpc, t->st);
     t->n_launches++;
     DHS_TRY(last_launch());
   }
@@ -1115,11 +1120,12 @@ dhs_status embbag_backward_update_noalloc(dhs_table* t, const int64_t* d_keys, i
   const int passes = std::min(kRadixMaxPasses, std::max(1, (bits + 7) / 8));
 
   {
-    const long long warps = (n_bags + 31) / 32;
+    const int bpc = bwd_probe_bags(n_keys, n_bags);
+    const long long warps = (n_bags + bpc - 1) / bpc;
     const long long grid = std::max<long long>(1, std::min<long long>((warps + 7) / 8, (long long)t->sm_count * 8));
     bwd_probe_kernel<<<(unsigned)grid, 256, 0, s>>>(idmap(t), (const long long*)d_keys, n_keys,
                                                     (const long long*)d_bag_offsets, n_bags, ka, va,
-                                                    sentinel, hist, kSortZeroWords, t->st);
+                                                    sentinel, hist, kSortZeroWords, bpc, t->st);
     DHS_TRY(last_launch());
   }
   const long long ntiles = (n_keys + kRadixTile - 1) / kRadixTile;
