@@ -645,7 +645,11 @@ bwd_seg_kernel(const unsigned* __restrict__ skey, const unsigned* __restrict__ s
         for (int q = 0; q < NV; ++q)
 #pragma unroll
           for (int e = 0; e < 4; ++e) o[(q * G + gl) * 4 + e] = acc[q][e];
-        if (mode == 3 && gl == 0) owners[atomicAdd(owner_ctr, 1u)] = (unsigned)c;  // for the combine
+        if (mode == 3 && gl == 0) {  // for the combine; at most one per chunk for sorted pairs
+          const unsigned slot = atomicAdd(owner_ctr, 1u);
+          if (slot < (unsigned)nchunks) owners[slot] = (unsigned)c;
+          else latch(st, kErrInternal);
+        }
       } else if (mode == 2 && cur < nrows) {
         double sq = 0.0;
         if (OPT == 3) {
@@ -1032,7 +1036,11 @@ bwd_segw_kernel(const unsigned* __restrict__ skey, const unsigned* __restrict__ 
           for (int e = 0; e < CPL; ++e)
             if (col0 + e < dim) o[e] = acc[e];
         }
-        if (mode == 3 && lane == 0) owners[atomicAdd(owner_ctr, 1u)] = (unsigned)c;  // for the combine
+        if (mode == 3 && lane == 0) {  // for the combine; at most one per chunk for sorted pairs
+          const unsigned slot = atomicAdd(owner_ctr, 1u);
+          if (slot < (unsigned)nchunks) owners[slot] = (unsigned)c;
+          else latch(st, kErrInternal);
+        }
       } else if (mode == 2 && kcur < nrows) {
         float* row = rs.row(kcur);
         float den = 0.f, Gn = 0.f;
@@ -1180,6 +1188,7 @@ struct CombinePlan {
   unsigned* batch_owner;  // [batch_cap] owner of each batch id
   double* slots;          // [slot_cap][pstride]
   unsigned batch_cap, slot_cap;
+  unsigned owner_cap;     // entries of the owner list and of the per-owner arrays
   unsigned* batch_ctr;    // zeroed before the segment kernel
   unsigned* slot_ctr;
 };
@@ -1191,7 +1200,7 @@ bwd_combine_plan_kernel(const unsigned* __restrict__ skey, long long n, int C,
   const int lane = threadIdx.x & 31;
   const long long nchunks = (n + C - 1) / C;
   const unsigned long long nrows = st->row_count;
-  const unsigned n_own = *owner_ctr;
+  const unsigned n_own = (unsigned)min((long long)*owner_ctr, nchunks);  // the seg kernel wrote [0, n_own)
   const long long warps = (long long)gridDim.x * (blockDim.x >> 5);
   for (long long oi = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); oi < n_own;
        oi += warps) {
@@ -1202,7 +1211,9 @@ bwd_combine_plan_kernel(const unsigned* __restrict__ skey, long long n, int C,
       const long long stride = (hi - lo + 32) / 32;
       const long long kk = lo + lane * stride;
       const unsigned in_run = __ballot_sync(0xffffffffu, kk <= hi && skey[kk * C] == key);
-      lo += (long long)(31 - __clz(in_run)) * stride;  // lane 0 (chunk lo) is always in the run
+      // lane 0 (chunk lo) is in the run when the pairs are sorted; counting it
+      // in regardless keeps lo >= c + 1 whatever the input
+      lo += (long long)(31 - __clz(in_run | 1u)) * stride;
       hi = min(hi, lo + stride - 1);
       if (stride == 1) break;
     }
@@ -1227,7 +1238,7 @@ bwd_combine_plan_kernel(const unsigned* __restrict__ skey, long long n, int C,
   }
 }
 
-__global__ void __launch_bounds__(kCombineThreads)
+__global__ void __launch_bounds__(kCombineThreads, 8)
 bwd_combine_kernel(const unsigned* __restrict__ skey, int dim, RowSpace rs, OptArgs oa,
                    const double* __restrict__ part_head, const double* __restrict__ part_tail, int C,
                    int pstride, const unsigned* __restrict__ owners,
@@ -1238,7 +1249,7 @@ bwd_combine_kernel(const unsigned* __restrict__ skey, int dim, RowSpace rs, OptA
   const int T = blockDim.x;
   const int slices = dim >= T ? 1 : T / dim;
   const unsigned nbatch = min(*pl.batch_ctr, pl.batch_cap);
-  const unsigned n_own = *owner_ctr;
+  const unsigned n_own = min(*owner_ctr, pl.owner_cap);  // the count may pass the list after a failed sort
   for (unsigned bid = blockIdx.x; bid < nbatch; bid += gridDim.x) {
     const unsigned oi = pl.batch_owner[bid];
     if (oi >= n_own) continue;  // only after a plan overflow, which the plan reported
@@ -1248,6 +1259,16 @@ bwd_combine_kernel(const unsigned* __restrict__ skey, int dim, RowSpace rs, OptA
     const unsigned b = bid - pl.boff[oi];
     const unsigned nb = (unsigned)((npieces + kCombinePieces - 1) / kCombinePieces);
     if (b >= nb) continue;
+    // the plan gives no batch to a missing-key run; this thread's column of
+    // the row (rows of at most T floats) is loaded while the pieces are summed
+    float* const row = rs.row(key);
+    const bool pre = dim <= T && (int)threadIdx.x < dim;
+    float pw = 0.f, ps0 = 0.f, ps1 = 0.f;
+    if (pre) {
+      pw = row[threadIdx.x];
+      if (oa.opt == 1 || oa.opt == 2) ps0 = row[dim + threadIdx.x];
+      if (oa.opt == 2) ps1 = row[2 * dim + threadIdx.x];
+    }
     const long long p0 = (long long)b * kCombinePieces;
     const long long p1 = min(npieces, p0 + kCombinePieces);
     // slice sl adds pieces p0 + sl, p0 + sl + slices, ... (piece 0 = starting partial)
@@ -1295,7 +1316,6 @@ bwd_combine_kernel(const unsigned* __restrict__ skey, int dim, RowSpace rs, OptA
       }
       __syncthreads();
     }
-    float* row = rs.row(key);  // the plan gives no batch to a missing-key run
     float den = 0.f;
     if (oa.opt == 3) {
       if (threadIdx.x == 0) {
@@ -1312,7 +1332,27 @@ bwd_combine_kernel(const unsigned* __restrict__ skey, int dim, RowSpace rs, OptA
       __syncthreads();
       if (threadIdx.x == 0) row[dim] = Gn;
     }
-    for (int j = threadIdx.x; j < dim; j += T) update_col(row, dim, j, (float)sacc[j], oa, den);
+    if (dim <= T) {
+      if (pre) {
+        const int j = threadIdx.x;
+        const float g = (float)sacc[j];
+        if (oa.opt == 0) {
+          pw = sgd_w(pw, g, oa.lr);
+        } else if (oa.opt == 1) {
+          adagrad_step(pw, ps0, g, oa.lr, oa.eps);
+          row[dim + j] = ps0;
+        } else if (oa.opt == 2) {
+          adam_step(pw, ps0, ps1, g, oa);
+          row[dim + j] = ps0;
+          row[2 * dim + j] = ps1;
+        } else {
+          pw = __fsub_rn(pw, __fdiv_rn(__fmul_rn(oa.lr, g), den));
+        }
+        row[j] = pw;
+      }
+    } else {
+      for (int j = threadIdx.x; j < dim; j += T) update_col(row, dim, j, (float)sacc[j], oa, den);
+    }
     __syncthreads();
   }
 }

@@ -397,6 +397,7 @@ CombinePlan combine_plan(unsigned* words, double* slots, long long nchunks, unsi
   pl.slots = slots;
   pl.batch_cap = (unsigned)combine_batch_cap(nchunks);
   pl.slot_cap = (unsigned)combine_slot_cap(nchunks);
+  pl.owner_cap = (unsigned)nchunks;
   pl.batch_ctr = zeroed + kCombineBatchCtrWord;
   pl.slot_ctr = zeroed + kCombineSlotCtrWord;
   return pl;
