@@ -69,7 +69,7 @@ typedef enum {
   DHS_ERR_CUDA = 3,        /* a CUDA runtime call failed */
   DHS_ERR_TABLE_FULL = 4,  /* row limit (max_rows) or IDMap probe bound reached */
   DHS_ERR_NOT_FOUND = 5,   /* backward saw a key that is not in the table */
-  DHS_ERR_UNSUPPORTED = 6, /* configuration this build does not handle */
+  DHS_ERR_UNSUPPORTED = 6, /* configuration the library does not handle */
   DHS_ERR_INTERNAL = 7     /* a bounded device-side wait gave up (results undefined) */
 } dhs_status;
 
