@@ -69,8 +69,8 @@ namespace dhs {
 // so that long bags still spread over enough warps); positions 64 at a time,
 // two per lane, so that each lane has two probes in flight.  A position's bag
 // is the number of the chunk's bag ends at or before it (a binary search over
-// the ends held in the lanes' registers).  Missing or negative keys get row `sentinel` (sorted
-// last, never updated).
+// the ends held in the lanes' registers).  Missing or negative keys get row
+// `sentinel` (sorted last, never updated).
 __global__ void __launch_bounds__(256)
 bwd_probe_kernel(IdMap m, const long long* __restrict__ keys, long long n_keys,
                  const long long* __restrict__ bag_off, long long n_bags,
@@ -273,14 +273,14 @@ __device__ __forceinline__ unsigned block_exclusive_scan_256(unsigned x, unsigne
 
 // One stable digit pass.  Tiles are numbered in the order blocks start (an
 // atomic counter), so a tile only ever waits for tiles whose blocks are
-// already running.  Each warp ranks its 256 items in order (8 rounds of 32
-// lanes; match.any gives the rank among equal digits within a round, a
-// per-warp shared counter carries it across rounds); the tile publishes its
-// digit counts, adds up its predecessors' (decoupled look-back), publishes
-// its inclusive prefix, places its items in digit order in shared memory and
-// writes them out in runs.  A wait that exceeds its bound latches
-// kErrInternal and the pass goes on (its output is then undefined, never out
-// of bounds).
+// already running.  Each warp ranks its 32 x kRadixItems items in order
+// (kRadixItems rounds of 32 lanes; match.any gives the rank among equal digits
+// within a round, a per-warp shared counter carries it across rounds); the
+// tile publishes its digit counts, adds up its predecessors' (decoupled
+// look-back), publishes its inclusive prefix, places its items in digit order
+// in shared memory and writes them out in runs.  A wait that exceeds its
+// bound latches kErrInternal and the pass goes on (its output is then
+// undefined, never out of bounds).
 __global__ void __launch_bounds__(kRadixThreads, DHS_RADIX_MINB)
 radix_onesweep_kernel(const unsigned* __restrict__ kin, const unsigned* __restrict__ vin,
                       unsigned* __restrict__ kout, unsigned* __restrict__ vout, long long n,
@@ -727,11 +727,12 @@ bwd_seg_kernel(const unsigned* __restrict__ skey, const unsigned* __restrict__ s
 // next chunk, for an owned segment that runs past the chunk end) are loaded
 // once; run heads become four 32-bit masks, so finding a run's end, its
 // ownership and the pair range to stream are warp-uniform scalar steps and
-// no lane waits on another lane's control path.  Gradient rows of the next S
-// pairs are copied into this warp's shared-memory ring with cp.async (each
-// lane its own columns: no barrier), added in fp64 in sorted order; the
-// table row of an owned run is loaded into registers when the run opens and
-// written once when it closes.
+// no lane waits on another lane's control path; the runs are listed once in
+// shared memory.  Gradient rows are staged a batch of pairs at a time into
+// this warp's two shared-memory buffers by cp.async.bulk (one copy per row,
+// issued by the lane of that pair; completion on the buffer's mbarrier, waits
+// bounded) and added in fp64 in sorted order; the table row of an owned run is
+// loaded into registers one run ahead and written once when the run closes.
 // ---------------------------------------------------------------------------
 // Pairs per staged batch (two batches per warp in flight or being read): 8 KB
 // of rows per warp at every width.
