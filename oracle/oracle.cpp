@@ -32,10 +32,20 @@
 //     position (nn.Embedding is a row lookup: the background article on RecIS,
 //     nn.Embedding section; EmbeddingBag mode="sum": DLRM practice article,
 //     section 2.1).
+//     EmbeddingBag's other forms (the same practice article names the module,
+//     whose "mean" mode and per-sample weights are part of its definition):
+//       weighted sum  pooled[b] = sum over i of fl(w_i * W[row_i]), each
+//                     product rounded to fp32, added in ascending position;
+//       mean          pooled[b] = fl(S_b / len_b), S_b the fp32 in-order sum,
+//                     one rounded division; an empty bag gives 0.
+//     Mean pooling with per-sample weights is rejected (as in PyTorch).
 //   * Backward: for each distinct key k of the batch, g_k = sum over the
 //     occurrences of k of grad[bag], accumulated in fp64 in ascending flat
 //     position and rounded once to fp32 (sum pooling sends each bag's output
-//     gradient to every id in the bag, duplicates counted).  Then one
+//     gradient to every id in the bag, duplicates counted).  With per-sample
+//     weights occurrence i contributes (double)w_i * (double)grad[bag] (an
+//     exact product); with mean pooling (double)grad[bag] / (double)len(bag).
+//     Then one
 //     optimizer step on the touched rows only (DLRM explainer, pitfall 4:
 //     sparse optimizer; background article: only row 23 is updated).
 //   * Optimizers, elementwise in fp32 with every operation rounded (this file
@@ -194,9 +204,12 @@ void orc_lookup(void* h, const int64_t* keys, int64_t n, int64_t* offsets_out) {
   }
 }
 
-int orc_forward(void* h, const int64_t* keys, const int64_t* bag_offsets, int64_t n_bags,
-                float* pooled) {
+// mode: 0 sum, 1 mean.  psw: per-sample weights float[n] or null.
+int orc_forward_ex(void* h, const int64_t* keys, const int64_t* bag_offsets, int64_t n_bags,
+                   const float* psw, int mode, float* pooled) {
   Table* t = (Table*)h;
+  if (mode != 0 && mode != 1) return ORC_ERR_INVALID;
+  if (mode == 1 && psw) return ORC_ERR_INVALID;
   int64_t n = n_bags > 0 ? bag_offsets[n_bags] : 0;
   std::vector<int64_t> off(n);
   int rc = orc_lookup_or_insert(h, keys, n, off.data());
@@ -206,16 +219,33 @@ int orc_forward(void* h, const int64_t* keys, const int64_t* bag_offsets, int64_
     for (int64_t i = bag_offsets[b]; i < bag_offsets[b + 1]; ++i) {
       if (off[i] < 0) continue;
       const float* w = t->row(off[i]);
-      for (int j = 0; j < t->dim; ++j) out[j] = out[j] + w[j];
+      if (psw) {
+        for (int j = 0; j < t->dim; ++j) {
+          const float prod = psw[i] * w[j];
+          out[j] = out[j] + prod;
+        }
+      } else {
+        for (int j = 0; j < t->dim; ++j) out[j] = out[j] + w[j];
+      }
     }
+    const int64_t len = bag_offsets[b + 1] - bag_offsets[b];
+    if (mode == 1 && len > 0)
+      for (int j = 0; j < t->dim; ++j) out[j] = out[j] / (float)len;
   }
   return rc;
 }
 
-int orc_backward_update(void* h, const int64_t* keys, const int64_t* bag_offsets, int64_t n_bags,
-                        const float* grad, float lr) {
+int orc_forward(void* h, const int64_t* keys, const int64_t* bag_offsets, int64_t n_bags,
+                float* pooled) {
+  return orc_forward_ex(h, keys, bag_offsets, n_bags, nullptr, 0, pooled);
+}
+
+int orc_backward_update_ex(void* h, const int64_t* keys, const int64_t* bag_offsets, int64_t n_bags,
+                           const float* psw, int mode, const float* grad, float lr) {
   Table* t = (Table*)h;
   const int d = t->dim;
+  if (mode != 0 && mode != 1) return ORC_ERR_INVALID;
+  if (mode == 1 && psw) return ORC_ERR_INVALID;
   int rc = ORC_OK;
   int64_t n = n_bags > 0 ? bag_offsets[n_bags] : 0;
   t->adam_t += 1;
@@ -250,7 +280,15 @@ int orc_backward_update(void* h, const int64_t* keys, const int64_t* bag_offsets
     std::fill(acc.begin(), acc.end(), 0.0);
     for (size_t q = a; q < e; ++q) {
       const float* gb = grad + occ[q].bag * d;
-      for (int j = 0; j < d; ++j) acc[j] += (double)gb[j];
+      if (psw) {
+        const double wq = (double)psw[occ[q].pos];
+        for (int j = 0; j < d; ++j) acc[j] += wq * (double)gb[j];
+      } else if (mode == 1) {
+        const double len = (double)(bag_offsets[occ[q].bag + 1] - bag_offsets[occ[q].bag]);
+        for (int j = 0; j < d; ++j) acc[j] += (double)gb[j] / len;
+      } else {
+        for (int j = 0; j < d; ++j) acc[j] += (double)gb[j];
+      }
     }
     for (int j = 0; j < d; ++j) g[j] = (float)acc[j];
 
@@ -292,6 +330,11 @@ int orc_backward_update(void* h, const int64_t* keys, const int64_t* bag_offsets
     a = e;
   }
   return rc;
+}
+
+int orc_backward_update(void* h, const int64_t* keys, const int64_t* bag_offsets, int64_t n_bags,
+                        const float* grad, float lr) {
+  return orc_backward_update_ex(h, keys, bag_offsets, n_bags, nullptr, 0, grad, lr);
 }
 
 // Export in row-offset order: keys[r] is the key whose offset is r; rows holds

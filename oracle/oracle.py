@@ -13,6 +13,7 @@ import numpy as np
 from . import build as _build
 
 OPT_CODES = {"sgd": 0, "adagrad": 1, "adam": 2, "adagrad_rowwise": 3}
+MODES = {"sum": 0, "mean": 1}
 _lib = None
 
 
@@ -41,6 +42,10 @@ def lib():
         L.orc_forward.argtypes = [vp, vp, vp, i64, vp]
         L.orc_backward_update.restype = C.c_int
         L.orc_backward_update.argtypes = [vp, vp, vp, i64, vp, f32]
+        L.orc_forward_ex.restype = C.c_int
+        L.orc_forward_ex.argtypes = [vp, vp, vp, i64, vp, C.c_int, vp]
+        L.orc_backward_update_ex.restype = C.c_int
+        L.orc_backward_update_ex.argtypes = [vp, vp, vp, i64, vp, C.c_int, vp, f32]
         L.orc_export.argtypes = [vp, vp, vp]
         L.orc_get_rows.restype = i64
         L.orc_get_rows.argtypes = [vp, vp, i64, vp]
@@ -113,21 +118,27 @@ class Oracle:
         lib().orc_lookup(self.h, _p(k), k.shape[0], _p(out))
         return out
 
-    def forward(self, keys, bag_offsets):
+    def forward(self, keys, bag_offsets, per_sample_weights=None, mode: str = "sum"):
+        """EmbeddingBag forward; mode "sum" or "mean"; optional per-sample
+        weights (float[n], sum mode only)."""
         k = np.ascontiguousarray(keys, np.int64)
         bo = np.ascontiguousarray(bag_offsets, np.int64)
         nb = bo.shape[0] - 1
         out = np.empty((nb, self.dim), np.float32)
-        rc = lib().orc_forward(self.h, _p(k), _p(bo), nb, _p(out))
+        w = None if per_sample_weights is None else np.ascontiguousarray(per_sample_weights, np.float32)
+        rc = lib().orc_forward_ex(self.h, _p(k), _p(bo), nb, _p(w) if w is not None else None,
+                                  MODES[mode], _p(out))
         return out, rc
 
-    def backward_update(self, keys, bag_offsets, grad, lr: float):
+    def backward_update(self, keys, bag_offsets, grad, lr: float, per_sample_weights=None, mode: str = "sum"):
         k = np.ascontiguousarray(keys, np.int64)
         bo = np.ascontiguousarray(bag_offsets, np.int64)
         g = np.ascontiguousarray(grad, np.float32)
         nb = bo.shape[0] - 1
         assert g.shape == (nb, self.dim)
-        return lib().orc_backward_update(self.h, _p(k), _p(bo), nb, _p(g), float(lr))
+        w = None if per_sample_weights is None else np.ascontiguousarray(per_sample_weights, np.float32)
+        return lib().orc_backward_update_ex(self.h, _p(k), _p(bo), nb, _p(w) if w is not None else None,
+                                            MODES[mode], _p(g), float(lr))
 
     def export(self):
         n = self.size

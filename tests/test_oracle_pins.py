@@ -95,6 +95,53 @@ def test_mapping_is_first_occurrence_order_brute_force():
         assert o.size == len(order)
 
 
+def test_read_only_lookup_brute_force():
+    """orc_lookup: a hit gives the offset the first-occurrence enumeration
+    assigned (computed here by a plain dict over the stream), an absent or
+    negative key gives -1, and nothing is inserted."""
+    rng = np.random.default_rng(11)
+    o = Oracle(4)
+    stream = []
+    for _ in range(4):
+        keys = rng.integers(0, 300, size=int(rng.integers(1, 120)), dtype=np.int64) * 13 + 5
+        o.lookup_or_insert(keys)
+        stream.extend(keys.tolist())
+    rank = {}
+    for k in stream:
+        rank.setdefault(k, len(rank))
+    size = o.size
+    probe = np.concatenate([np.array(stream[::3], np.int64),
+                            np.arange(0, 4000, 7, dtype=np.int64),  # mostly absent
+                            np.array([-1, -5, -(2 ** 62)], np.int64)])
+    got = o.lookup(probe)
+    want = [rank.get(int(k), -1) if k >= 0 else -1 for k in probe]
+    assert got.tolist() == want
+    assert (got == -1).sum() > 100 and (got >= 0).sum() > 100
+    assert o.size == size
+    # a hit is exactly what lookup_or_insert returns for the same key
+    off, _ = o.lookup_or_insert(np.array(stream[:50], np.int64))
+    np.testing.assert_array_equal(o.lookup(np.array(stream[:50], np.int64)), off)
+
+
+def test_get_rows_absent_keys_are_nan_and_counted():
+    o = Oracle(8, "adam")
+    present = np.array([3, 10, 77], np.int64)
+    o.lookup_or_insert(present)
+    _, rows = o.export()
+    ask = np.array([10, 999, 3, -4, 77, 1000], np.int64)
+    got, missing = o.get_rows(ask)
+    assert missing == 3
+    assert got.shape == (6, o.stride)
+    for i in (1, 3, 5):
+        assert np.all(np.isnan(got[i]))
+    # present rows are the stored rows (weights = init of the key, state 0)
+    np.testing.assert_array_equal(got[0], rows[1])
+    np.testing.assert_array_equal(got[2], rows[0])
+    np.testing.assert_array_equal(got[4], rows[2])
+    np.testing.assert_array_equal(got[0, :8], init_row(10, 8))
+    assert np.all(got[[0, 2, 4], 8:] == 0)
+
+
 def test_modulo_collision_ids_get_distinct_rows():
     g = _golden("modulo_collision.json")
     a, b = g["ids"]
@@ -135,6 +182,113 @@ def test_forward_matches_torch_embedding_bag_sum():
                                             torch.from_numpy(offs[:-1]), mode="sum").numpy()
     assert np.all(pooled[lens == 0] == 0)
     np.testing.assert_allclose(pooled, ref, rtol=1e-6, atol=1e-7)
+
+
+def _dense_case(d, seed, max_len=9):
+    """An oracle whose keys 0..63 map to rows 0..63, those rows as a torch
+    weight, and a batch of bags (empty ones included) over the 64 keys."""
+    o = Oracle(d)
+    o.lookup_or_insert(np.arange(64, dtype=np.int64))
+    _, rows = o.export()
+    rng = np.random.default_rng(seed)
+    lens = rng.integers(0, max_len, size=41)
+    lens[[0, 7, 40]] = 0
+    offs = np.concatenate([[0], np.cumsum(lens)]).astype(np.int64)
+    keys = rng.integers(0, 64, size=int(offs[-1]), dtype=np.int64)
+    psw = rng.uniform(-2.0, 2.0, size=keys.size).astype(np.float32)
+    return o, torch.from_numpy(rows[:, :d].copy()), lens, offs, keys, psw
+
+
+def test_mean_and_weighted_forward_match_torch_embedding_bag():
+    d = 12
+    o, weight, lens, offs, keys, psw = _dense_case(d, 2)
+    tk, to = torch.from_numpy(keys), torch.from_numpy(offs[:-1])
+    mean, rc = o.forward(keys, offs, mode="mean")
+    assert rc == 0
+    ref = torch.nn.functional.embedding_bag(tk, weight, to, mode="mean").numpy()
+    np.testing.assert_allclose(mean, ref, rtol=2e-6, atol=1e-7)
+    assert np.all(mean[lens == 0] == 0)
+    wsum, rc = o.forward(keys, offs, per_sample_weights=psw)
+    assert rc == 0
+    ref = torch.nn.functional.embedding_bag(tk, weight, to, mode="sum",
+                                            per_sample_weights=torch.from_numpy(psw)).numpy()
+    np.testing.assert_allclose(wsum, ref, rtol=2e-6, atol=2e-7)
+
+
+def test_pooling_mode_special_cases_are_exact():
+    d = 8
+    o, _, lens, offs, keys, psw = _dense_case(d, 3)
+    plain, _ = o.forward(keys, offs)
+    ones, _ = o.forward(keys, offs, per_sample_weights=np.ones(keys.size, np.float32))
+    assert np.array_equal(ones, plain)
+    # a power-of-two weight scales every product and every partial sum exactly
+    twos, _ = o.forward(keys, offs, per_sample_weights=np.full(keys.size, 2.0, np.float32))
+    assert np.array_equal(twos, 2 * plain)
+    # mean over bags of one id is the id's row
+    single = np.arange(keys.size + 1, dtype=np.int64)
+    a, _ = o.forward(keys, single, mode="mean")
+    b, _ = o.forward(keys, single)
+    assert np.array_equal(a, b)
+    # mean pooling takes no per-sample weights (rejected, nothing computed)
+    _, rc = o.forward(keys, offs, per_sample_weights=psw, mode="mean")
+    assert rc == 1
+    assert o.backward_update(keys, offs, np.ones((lens.size, d), np.float32), 0.1,
+                             per_sample_weights=psw, mode="mean") == 1
+
+
+@pytest.mark.parametrize("opt", ["sgd", "adagrad"])
+@pytest.mark.parametrize("form", ["mean", "weighted"])
+def test_mean_and_weighted_backward_match_torch_autograd(form, opt):
+    """A dense table's gradient from torch autograd through embedding_bag,
+    then torch's SGD / Adagrad step (rows without gradient do not move).
+    Torch sums a row's occurrence gradients in fp32 (the oracle sums them
+    exactly in fp64): with up to ~10 occurrences of |w g| <= ~4 per step the
+    fp32 sum is off by at most ~10 * 4 * 6e-8 = 2.4e-6, times lr 0.05 over
+    3 steps about 4e-7 on a weight, hence the absolute term next to the
+    relative bar.  A dropped weight or mean divisor moves weights by ~1e-2."""
+    d, lr = 12, 0.05
+    o = Oracle(d, opt)
+    o.lookup_or_insert(np.arange(64, dtype=np.int64))
+    _, rows = o.export()
+    _, _, lens, offs, keys, psw = _dense_case(d, 4)
+    rng = np.random.default_rng(5)
+    weight = torch.nn.Parameter(torch.from_numpy(rows[:, :d].copy()))
+    torch_opt = torch.optim.SGD([weight], lr=lr) if opt == "sgd" else \
+        torch.optim.Adagrad([weight], lr=lr, eps=1e-8)
+    for _ in range(3):
+        grad = rng.standard_normal((lens.size, d)).astype(np.float32)
+        kw = dict(mode="mean") if form == "mean" else dict(per_sample_weights=psw)
+        assert o.backward_update(keys, offs, grad, lr, **kw) == 0
+        tkw = dict(mode="mean") if form == "mean" else dict(mode="sum", per_sample_weights=torch.from_numpy(psw))
+        out = torch.nn.functional.embedding_bag(torch.from_numpy(keys), weight, torch.from_numpy(offs[:-1]), **tkw)
+        torch_opt.zero_grad()
+        (out * torch.from_numpy(grad)).sum().backward()
+        torch_opt.step()
+    _, got = o.export()
+    want = weight.detach().numpy()
+    assert np.all(np.abs(got[:, :d] - want) <= 1e-5 * np.abs(want) + 4e-7)
+    touched = np.unique(keys)
+    untouched = np.setdiff1d(np.arange(64), touched)
+    assert np.array_equal(got[untouched, :d], rows[untouched, :d])
+
+
+def test_mean_gradient_closed_form():
+    """Each key in exactly one bag of length L: its gradient is fl(g / L)
+    (the exact quotient, rounded once), so SGD moves it by fl(lr * fl(g / L))."""
+    d, lr = 4, 0.5
+    o = Oracle(d, "sgd")
+    lens = np.array([1, 3, 7, 2], np.int64)
+    keys = np.arange(lens.sum(), dtype=np.int64) + 100
+    offs = np.concatenate([[0], np.cumsum(lens)]).astype(np.int64)
+    o.lookup_or_insert(keys)
+    _, before = o.export()
+    g = np.array([[1.0, -3.0, 0.1, 7.0]] * lens.size, np.float32) * np.arange(1, 5, dtype=np.float32)[:, None]
+    assert o.backward_update(keys, offs, g, lr, mode="mean") == 0
+    _, after = o.export()
+    bag = np.repeat(np.arange(lens.size), lens)
+    gk = (g[bag].astype(np.float64) / lens[bag][:, None]).astype(np.float32)
+    want = before[:, :d] - np.float32(lr) * gk
+    assert np.array_equal(after[:, :d], want)
 
 
 def test_merged_tables_equal_separate_tables():
