@@ -61,6 +61,13 @@
 //                computed in fp64 and rounded to fp32; lazy: rows not in the
 //                batch keep their m and v).
 //
+//   * Row storage in bf16 (DLRM practice article, section 4.2: embedding
+//     matrices stored in 16-bit floats to halve their bytes), optimizer state
+//     in fp32: every stored weight is rounded to the nearest bf16 value, ties
+//     to even (the initial row and every optimizer step's result); the
+//     forward reads those values and sums in fp32; the optimizer computes in
+//     fp32 from them and the fp32 state, then rounds the new weight once.
+//
 // A missing key in the backward, or a negative key anywhere, is skipped and
 // reported through the return code; the other rows are processed normally.
 
@@ -87,6 +94,25 @@ uint64_t splitmix64_next(uint64_t* state) {
   return z ^ (z >> 31);
 }
 
+// Nearest bf16 value of x (the top 16 bits of an fp32 after rounding the low
+// 16 bits to nearest, ties to even), returned as the fp32 it widens to.  NaN
+// stays a NaN; values past the largest bf16 round to infinity.
+float round_bf16(float x) {
+  uint32_t u;
+  std::memcpy(&u, &x, 4);
+  if ((u & 0x7fffffffu) > 0x7f800000u) {  // NaN: keep it quiet
+    u = (u | 0x00400000u) & 0xffff0000u;
+  } else {
+    const uint32_t low = u & 0xffffu, half = 0x8000u;
+    const uint32_t keep_odd = (u >> 16) & 1u;
+    u &= 0xffff0000u;
+    if (low > half || (low == half && keep_odd)) u += 0x10000u;  // carries into the exponent as it should
+  }
+  float y;
+  std::memcpy(&y, &u, 4);
+  return y;
+}
+
 // Initial row of `key`: element j comes from the (j+1)-th output of the
 // splitmix64 stream seeded with the key.
 void init_row(int64_t key, int dim, float* w) {
@@ -102,6 +128,7 @@ void init_row(int64_t key, int dim, float* w) {
 struct Table {
   int dim;
   int opt;
+  bool bf16;     // weights stored as bf16 values
   int n_state;   // state floats per row
   float eps, beta1, beta2;
   int64_t adam_t;
@@ -120,9 +147,13 @@ struct Table {
     rows.resize((size_t)(r + 1) * stride(), 0.0f);
     float* w = row(r);
     init_row(key, dim, w);
+    for (int j = 0; j < dim; ++j) w[j] = store(w[j]);
     for (int64_t j = dim; j < stride(); ++j) w[j] = 0.0f;
     return r;
   }
+
+  // A weight as the table stores it.
+  float store(float v) const { return bf16 ? round_bf16(v) : v; }
 };
 
 int state_floats(int opt, int dim) {
@@ -158,11 +189,13 @@ int orc_pack_keys(const int32_t* table_ids, const int64_t* ids, int64_t n, int64
   return rc;
 }
 
-void* orc_create(int dim, int opt, float eps, float beta1, float beta2) {
-  if (dim <= 0 || state_floats(opt, dim) < 0) return nullptr;
+// storage: 0 fp32 weights, 1 bf16 weights (state fp32 either way)
+void* orc_create_ex(int dim, int opt, float eps, float beta1, float beta2, int storage) {
+  if (dim <= 0 || state_floats(opt, dim) < 0 || storage < 0 || storage > 1) return nullptr;
   Table* t = new Table();
   t->dim = dim;
   t->opt = opt;
+  t->bf16 = storage == 1;
   t->n_state = state_floats(opt, dim);
   t->eps = eps;
   t->beta1 = beta1;
@@ -170,6 +203,12 @@ void* orc_create(int dim, int opt, float eps, float beta1, float beta2) {
   t->adam_t = 0;
   return t;
 }
+
+void* orc_create(int dim, int opt, float eps, float beta1, float beta2) {
+  return orc_create_ex(dim, opt, eps, beta1, beta2, 0);
+}
+
+float orc_round_bf16(float x) { return round_bf16(x); }
 
 void orc_destroy(void* h) { delete (Table*)h; }
 
@@ -295,13 +334,13 @@ int orc_backward_update_ex(void* h, const int64_t* keys, const int64_t* bag_offs
     float* w = t->row(t->map[occ[a].key]);
     switch (t->opt) {
       case ORC_SGD:
-        for (int j = 0; j < d; ++j) w[j] = w[j] - lr * g[j];
+        for (int j = 0; j < d; ++j) w[j] = t->store(w[j] - lr * g[j]);
         break;
       case ORC_ADAGRAD: {
         float* G = w + d;
         for (int j = 0; j < d; ++j) {
           G[j] = G[j] + g[j] * g[j];
-          w[j] = w[j] - (lr * g[j]) / (std::sqrt(G[j]) + t->eps);
+          w[j] = t->store(w[j] - (lr * g[j]) / (std::sqrt(G[j]) + t->eps));
         }
         break;
       }
@@ -311,7 +350,7 @@ int orc_backward_update_ex(void* h, const int64_t* keys, const int64_t* bag_offs
         float* G = w + d;
         G[0] = G[0] + (float)(ss / d);
         float den = std::sqrt(G[0]) + t->eps;
-        for (int j = 0; j < d; ++j) w[j] = w[j] - (lr * g[j]) / den;
+        for (int j = 0; j < d; ++j) w[j] = t->store(w[j] - (lr * g[j]) / den);
         break;
       }
       case ORC_ADAM: {
@@ -322,7 +361,7 @@ int orc_backward_update_ex(void* h, const int64_t* keys, const int64_t* bag_offs
           v[j] = b2 * v[j] + c2 * (g[j] * g[j]);
           float mhat = m[j] / bc1;
           float vhat = v[j] / bc2;
-          w[j] = w[j] - (lr * mhat) / (std::sqrt(vhat) + t->eps);
+          w[j] = t->store(w[j] - (lr * mhat) / (std::sqrt(vhat) + t->eps));
         }
         break;
       }
@@ -344,6 +383,15 @@ void orc_export(void* h, int64_t* keys, float* rows) {
   int64_t n = (int64_t)t->key_of_row.size();
   if (keys) std::memcpy(keys, t->key_of_row.data(), sizeof(int64_t) * n);
   if (rows) std::memcpy(rows, t->rows.data(), sizeof(float) * n * t->stride());
+}
+
+// Overwrite the first n rows (stride floats each, weights then state) with
+// the given values, as stored (no rounding): lets a test start a step from
+// rows taken from another table.
+void orc_import_rows(void* h, const float* rows, int64_t n) {
+  Table* t = (Table*)h;
+  const int64_t m = std::min<int64_t>(n, (int64_t)t->key_of_row.size());
+  std::memcpy(t->rows.data(), rows, sizeof(float) * m * t->stride());
 }
 
 // Rows (weights then state) of the given keys; absent keys give NaN rows and

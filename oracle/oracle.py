@@ -14,6 +14,7 @@ from . import build as _build
 
 OPT_CODES = {"sgd": 0, "adagrad": 1, "adam": 2, "adagrad_rowwise": 3}
 MODES = {"sum": 0, "mean": 1}
+STORAGE = {"f32": 0, "bf16": 1}
 _lib = None
 
 
@@ -30,6 +31,10 @@ def lib():
         L.orc_pack_keys.argtypes = [vp, vp, i64, vp]
         L.orc_create.restype = vp
         L.orc_create.argtypes = [C.c_int, C.c_int, f32, f32, f32]
+        L.orc_create_ex.restype = vp
+        L.orc_create_ex.argtypes = [C.c_int, C.c_int, f32, f32, f32, C.c_int]
+        L.orc_round_bf16.restype = f32
+        L.orc_round_bf16.argtypes = [f32]
         L.orc_destroy.argtypes = [vp]
         L.orc_size.restype = i64
         L.orc_size.argtypes = [vp]
@@ -47,6 +52,7 @@ def lib():
         L.orc_backward_update_ex.restype = C.c_int
         L.orc_backward_update_ex.argtypes = [vp, vp, vp, i64, vp, C.c_int, vp, f32]
         L.orc_export.argtypes = [vp, vp, vp]
+        L.orc_import_rows.argtypes = [vp, vp, i64]
         L.orc_get_rows.restype = i64
         L.orc_get_rows.argtypes = [vp, vp, i64, vp]
         _lib = L
@@ -68,6 +74,13 @@ def init_row(key: int, dim: int) -> np.ndarray:
     return out
 
 
+def round_bf16(x: np.ndarray) -> np.ndarray:
+    """The oracle's fp32 -> nearest bf16 (widened back to fp32), elementwise."""
+    x = np.ascontiguousarray(x, np.float32)
+    f = lib().orc_round_bf16
+    return np.array([f(float(v)) for v in x.ravel()], np.float32).reshape(x.shape)
+
+
 def pack_keys(table_ids: np.ndarray, ids: np.ndarray):
     t = np.ascontiguousarray(table_ids, np.int32)
     i = np.ascontiguousarray(ids, np.int64)
@@ -80,10 +93,11 @@ class Oracle:
     """std::unordered_map IDMap + one row vector; sequential loops."""
 
     def __init__(self, dim: int, optimizer: str = "sgd", eps: float = 1e-8,
-                 beta1: float = 0.9, beta2: float = 0.999):
+                 beta1: float = 0.9, beta2: float = 0.999, storage: str = "f32"):
         self.dim = int(dim)
         self.optimizer = optimizer
-        self.h = lib().orc_create(self.dim, OPT_CODES[optimizer], eps, beta1, beta2)
+        self.storage = storage
+        self.h = lib().orc_create_ex(self.dim, OPT_CODES[optimizer], eps, beta1, beta2, STORAGE[storage])
         if not self.h:
             raise ValueError("bad oracle arguments")
 

@@ -13,7 +13,7 @@ import numpy as np
 import pytest
 import torch
 
-from oracle import Oracle, init_row, pack_keys, splitmix64_outputs
+from oracle import Oracle, init_row, pack_keys, round_bf16, splitmix64_outputs
 from tests.conftest import GOLDEN
 
 SCALE = np.float32(0.05) * np.float32(2.0 ** -23)
@@ -538,3 +538,86 @@ def test_bytes_per_row_arithmetic():
     for c in g["cases"]:
         gb = c["rows"] * c["dim"] * c["bytes_per_float"] / 1e9
         assert abs(gb - c["stated_gb"]) / c["stated_gb"] < 0.03
+
+
+# --- bf16 row storage -----------------------------------------------------------------
+
+def _torch_bf16(x):
+    return torch.from_numpy(np.ascontiguousarray(x, np.float32)).to(torch.bfloat16).to(torch.float32).numpy()
+
+
+def test_round_bf16_matches_torch_conversion():
+    """Round to nearest, ties to even, against torch's float -> bfloat16 cast:
+    random values over the whole exponent range, exact ties (both parities),
+    subnormals, signed zeros, infinities, the largest finite values, NaN."""
+    rng = np.random.default_rng(17)
+    rand = rng.integers(0, 2 ** 32, size=20000, dtype=np.uint64).astype(np.uint32).view(np.float32)
+    hi = rng.integers(0, 2 ** 16, size=2000, dtype=np.uint64).astype(np.uint32) << np.uint32(16)
+    ties = (hi | np.uint32(0x8000)).view(np.float32)            # exactly half way
+    near = np.concatenate([(hi | np.uint32(0x7fff)), (hi | np.uint32(0x8001))]).view(np.float32)
+    special = np.array([0.0, -0.0, np.inf, -np.inf, 1e-45, -1e-45, 1e-40, 3.4028235e38, -3.4028235e38,
+                        3.3961776e38, 1.0, 1.00390625, 1.005859375, 0.05, -0.05], np.float32)
+    x = np.concatenate([rand, ties, near, special])
+    got, want = round_bf16(x), _torch_bf16(x)
+    nan = np.isnan(want)
+    assert np.array_equal(np.isnan(got), nan)
+    assert np.array_equal(got[~nan].view(np.uint32), want[~nan].view(np.uint32))
+    assert np.isnan(round_bf16(np.array([np.nan], np.float32)))[0]
+
+
+@pytest.mark.parametrize("opt", ["sgd", "adagrad", "adam", "adagrad_rowwise"])
+def test_bf16_table_rounds_every_stored_weight(opt):
+    """A bf16 table keeps every weight on the bf16 grid (initial rows and each
+    step's result), its state in fp32, and equals the fp32 table's arithmetic
+    with one rounding (torch's cast) per stored weight: checked step by step
+    from the same pre-step rows."""
+    d, lr = 8, 0.05
+    rng = np.random.default_rng(23)
+    o = Oracle(d, opt, storage="bf16")
+    keys = np.arange(40, dtype=np.int64) * 3 + 1
+    o.lookup_or_insert(keys)
+    _, rows = o.export()
+    assert np.array_equal(rows[:, :d], _torch_bf16(np.stack([init_row(int(k), d) for k in keys])))
+    for step in range(3):
+        offs = np.arange(0, 41, 4, dtype=np.int64)
+        grad = rng.standard_normal((10, d)).astype(np.float32)
+        _, before = o.export()
+        assert o.backward_update(keys, offs, grad, lr) == 0
+        _, after = o.export()
+        # the same step on an fp32 table holding the pre-step rows, then one cast
+        ref = Oracle(d, opt)
+        ref.lookup_or_insert(keys)
+        _set_rows(ref, before)
+        for _ in range(step):  # Adam's step count: empty calls advance it
+            ref.backward_update(np.zeros(0, np.int64), np.zeros(1, np.int64), np.zeros((0, d), np.float32), lr)
+        ref.backward_update(keys, offs, grad, lr)
+        _, r32 = ref.export()
+        ref.close()
+        assert np.array_equal(after[:, :d], _torch_bf16(r32[:, :d]))
+        assert np.array_equal(after[:, d:], r32[:, d:])  # fp32 state, unrounded
+    assert np.array_equal(after[:, :d], _torch_bf16(after[:, :d]))
+
+
+def _set_rows(o, rows):
+    """Overwrite an oracle table's stored rows with `rows` (row order)."""
+    import ctypes as C
+    from oracle.oracle import lib
+    n, s = rows.shape
+    buf = np.ascontiguousarray(rows, np.float32)
+    lib().orc_import_rows(o.h, buf.ctypes.data_as(C.c_void_p), n)
+
+
+def test_bf16_forward_sums_the_stored_values():
+    d = 8
+    o = Oracle(d, "sgd", storage="bf16")
+    o.lookup_or_insert(np.arange(64, dtype=np.int64))
+    _, rows = o.export()
+    weight = torch.from_numpy(rows[:, :d].copy())  # the stored (bf16-exact) values
+    rng = np.random.default_rng(29)
+    lens = rng.integers(0, 9, size=30)
+    offs = np.concatenate([[0], np.cumsum(lens)]).astype(np.int64)
+    keys = rng.integers(0, 64, size=int(offs[-1]), dtype=np.int64)
+    pooled, _ = o.forward(keys, offs)
+    ref = torch.nn.functional.embedding_bag(torch.from_numpy(keys), weight, torch.from_numpy(offs[:-1]),
+                                            mode="sum").numpy()
+    np.testing.assert_allclose(pooled, ref, rtol=1e-6, atol=1e-7)
