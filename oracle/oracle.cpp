@@ -68,11 +68,32 @@
 //     forward reads those values and sums in fp32; the optimizer computes in
 //     fp32 from them and the fp32 state, then rounds the new weight once.
 //
+//   * Feature admission and eviction (RecIS overview, code layout: the
+//     HashtableHook admission / eviction strategy of the embedding engine;
+//     the pages give only its name, so these are the plainest readings):
+//       admission  a key gets a row in the first insert call in which its
+//                  occurrences over all insert calls so far, this call's
+//                  included, reach the threshold (1 = at first sight).  A key
+//                  without a row contributes nothing to pooled sums, its
+//                  gradients are dropped, and its count is kept.  Keys
+//                  admitted in one call get rows in the order of their first
+//                  occurrence in that call.
+//       eviction   every insert call is one step; a key's stamp is the last
+//                  step it occurred in.  evict(max_idle) removes every key
+//                  (with or without a row) last seen before step
+//                  current - max_idle; their rows become free, and later
+//                  admitted keys take free rows in ascending order before new
+//                  ones are appended (a reused row starts from the new key's
+//                  initial values, state 0).  An evicted key that comes back
+//                  is a new key.
+//
 // A missing key in the backward, or a negative key anywhere, is skipped and
 // reported through the return code; the other rows are processed normally.
+// A key that is known but not yet admitted is skipped silently.
 
 #include <algorithm>
 #include <cmath>
+#include <set>
 #include <cstdint>
 #include <cstring>
 #include <unordered_map>
@@ -133,18 +154,32 @@ struct Table {
   float eps, beta1, beta2;
   int64_t adam_t;
   std::unordered_map<int64_t, int64_t> map;
-  std::vector<int64_t> key_of_row;
+  std::vector<int64_t> key_of_row;  // -1 for a free (evicted) row
   std::vector<float> rows;  // row r at r * stride: dim weights then state
+  // admission / eviction
+  int64_t admit_threshold = 1;
+  bool track = false;                                // stamp keys (needed by evict)
+  int64_t step = 0;                                  // insert calls so far
+  std::unordered_map<int64_t, int64_t> pending;      // occurrences of keys without a row
+  std::unordered_map<int64_t, int64_t> last_seen;    // step of each known key's last occurrence
+  std::set<int64_t> free_rows;
 
   int64_t stride() const { return (int64_t)dim + n_state; }
 
   float* row(int64_t r) { return rows.data() + r * stride(); }
 
   int64_t insert_new(int64_t key) {
-    int64_t r = (int64_t)key_of_row.size();
+    int64_t r;
+    if (!free_rows.empty()) {  // the smallest free row first
+      r = *free_rows.begin();
+      free_rows.erase(free_rows.begin());
+      key_of_row[r] = key;
+    } else {
+      r = (int64_t)key_of_row.size();
+      key_of_row.push_back(key);
+      rows.resize((size_t)(r + 1) * stride(), 0.0f);
+    }
     map.emplace(key, r);
-    key_of_row.push_back(key);
-    rows.resize((size_t)(r + 1) * stride(), 0.0f);
     float* w = row(r);
     init_row(key, dim, w);
     for (int j = 0; j < dim; ++j) w[j] = store(w[j]);
@@ -216,23 +251,78 @@ int64_t orc_size(void* h) { return (int64_t)((Table*)h)->key_of_row.size(); }
 
 int64_t orc_stride(void* h) { return ((Table*)h)->stride(); }
 
-// Sequential in i: a key not yet in the map gets the next row.
+// One insert call (lookup_or_insert, forward).  Without admission (threshold
+// 1) this is: sequential in i, a key not yet in the map gets the next row.
+// With admission: the call's occurrences of each key without a row are added
+// to its count first; keys whose count reaches the threshold are admitted in
+// the order of their first occurrence in the call; then every position's row
+// is read (-1 for a key still without a row).
 int orc_lookup_or_insert(void* h, const int64_t* keys, int64_t n, int64_t* offsets_out) {
   Table* t = (Table*)h;
   int rc = ORC_OK;
+  t->step += 1;
+  std::vector<int64_t> first;  // keys without a row, by first occurrence in the call
+  std::unordered_map<int64_t, int64_t> here;
   for (int64_t i = 0; i < n; ++i) {
-    int64_t k = keys[i];
+    const int64_t k = keys[i];
     if (k < 0) {
       rc = ORC_ERR_INVALID;
-      if (offsets_out) offsets_out[i] = -1;
       continue;
     }
-    auto it = t->map.find(k);
-    int64_t r = (it == t->map.end()) ? t->insert_new(k) : it->second;
-    if (offsets_out) offsets_out[i] = r;
+    if (t->track) t->last_seen[k] = t->step;
+    if (t->map.count(k)) continue;
+    if (here[k]++ == 0) first.push_back(k);
+  }
+  for (int64_t k : first) {
+    const int64_t total = t->pending[k] + here[k];
+    if (total >= t->admit_threshold) {
+      t->pending.erase(k);
+      t->insert_new(k);
+    } else {
+      t->pending[k] = total;
+    }
+  }
+  for (int64_t i = 0; i < n; ++i) {
+    const int64_t k = keys[i];
+    auto it = k < 0 ? t->map.end() : t->map.find(k);
+    if (offsets_out) offsets_out[i] = it == t->map.end() ? -1 : it->second;
   }
   return rc;
 }
+
+// Admission threshold (occurrences before a key gets a row; <= 1: at once)
+// and access tracking (stamps for evict); set before the first insert call.
+void orc_set_hooks(void* h, int64_t threshold, int track) {
+  Table* t = (Table*)h;
+  t->admit_threshold = std::max<int64_t>(1, threshold);
+  t->track = track != 0;
+}
+
+// Evict every key last seen before step (current - max_idle); returns the
+// number of rows freed.
+int64_t orc_evict(void* h, int64_t max_idle) {
+  Table* t = (Table*)h;
+  const int64_t keep_from = t->step - max_idle;
+  int64_t freed = 0;
+  std::vector<int64_t> gone;
+  for (const auto& kv : t->last_seen)
+    if (kv.second < keep_from) gone.push_back(kv.first);
+  for (int64_t k : gone) {
+    t->last_seen.erase(k);
+    t->pending.erase(k);
+    auto it = t->map.find(k);
+    if (it != t->map.end()) {
+      t->key_of_row[it->second] = -1;
+      t->free_rows.insert(it->second);
+      t->map.erase(it);
+      ++freed;
+    }
+  }
+  return freed;
+}
+
+// Keys with a row.
+int64_t orc_live(void* h) { return (int64_t)((Table*)h)->map.size(); }
 
 // Read-only lookup: -1 where the key is absent.
 void orc_lookup(void* h, const int64_t* keys, int64_t n, int64_t* offsets_out) {
@@ -297,7 +387,10 @@ int orc_backward_update_ex(void* h, const int64_t* keys, const int64_t* bag_offs
     for (int64_t i = bag_offsets[b]; i < bag_offsets[b + 1]; ++i) {
       int64_t k = keys[i];
       if (k < 0) { rc = ORC_ERR_INVALID; continue; }
-      if (t->map.find(k) == t->map.end()) { rc = rc ? rc : ORC_ERR_NOT_FOUND; continue; }
+      if (t->map.find(k) == t->map.end()) {
+        if (!t->pending.count(k)) rc = rc ? rc : ORC_ERR_NOT_FOUND;  // a key not admitted yet: skipped
+        continue;
+      }
       occ.push_back({k, i, b});
     }
   std::sort(occ.begin(), occ.end(), [](const Occ& a, const Occ& b) {

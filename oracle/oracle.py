@@ -53,6 +53,11 @@ def lib():
         L.orc_backward_update_ex.argtypes = [vp, vp, vp, i64, vp, C.c_int, vp, f32]
         L.orc_export.argtypes = [vp, vp, vp]
         L.orc_import_rows.argtypes = [vp, vp, i64]
+        L.orc_set_hooks.argtypes = [vp, i64, C.c_int]
+        L.orc_evict.restype = i64
+        L.orc_evict.argtypes = [vp, i64]
+        L.orc_live.restype = i64
+        L.orc_live.argtypes = [vp]
         L.orc_get_rows.restype = i64
         L.orc_get_rows.argtypes = [vp, vp, i64, vp]
         _lib = L
@@ -114,7 +119,20 @@ class Oracle:
 
     @property
     def size(self) -> int:
+        """Rows allocated (free rows included)."""
         return int(lib().orc_size(self.h))
+
+    @property
+    def live(self) -> int:
+        """Keys with a row."""
+        return int(lib().orc_live(self.h))
+
+    def set_hooks(self, admit_threshold: int = 1, track_access: bool = False):
+        """Admission threshold and access tracking (before the first insert)."""
+        lib().orc_set_hooks(self.h, int(admit_threshold), int(bool(track_access)))
+
+    def evict(self, max_idle: int) -> int:
+        return int(lib().orc_evict(self.h, int(max_idle)))
 
     @property
     def stride(self) -> int:

@@ -621,3 +621,103 @@ def test_bf16_forward_sums_the_stored_values():
     ref = torch.nn.functional.embedding_bag(torch.from_numpy(keys), weight, torch.from_numpy(offs[:-1]),
                                             mode="sum").numpy()
     np.testing.assert_allclose(pooled, ref, rtol=1e-6, atol=1e-7)
+
+
+# --- admission / eviction (readings of the hook the pages only name) --------------------
+
+def _same_tables(a, b, d):
+    ka, ra = a.export()
+    kb, rb = b.export()
+    assert np.array_equal(ka, kb) and np.array_equal(ra[:, :d], rb[:, :d]) and np.array_equal(ra, rb)
+
+
+def test_admission_threshold_one_is_the_plain_table():
+    rng = np.random.default_rng(41)
+    a, b = Oracle(8, "adagrad"), Oracle(8, "adagrad")
+    b.set_hooks(admit_threshold=1, track_access=True)
+    for _ in range(4):
+        lens = rng.integers(0, 6, size=50)
+        offs = np.concatenate([[0], np.cumsum(lens)]).astype(np.int64)
+        keys = rng.integers(0, 120, size=int(offs[-1])).astype(np.int64)
+        pa, _ = a.forward(keys, offs)
+        pb, _ = b.forward(keys, offs)
+        assert np.array_equal(pa, pb)
+        g = rng.standard_normal((50, 8)).astype(np.float32)
+        assert a.backward_update(keys, offs, g, 0.1) == b.backward_update(keys, offs, g, 0.1) == 0
+    _same_tables(a, b, 8)
+
+
+def test_admission_closed_form_and_zero_contribution():
+    """A key occurring c times in every call is admitted in call ceil(A / c)
+    with its initial row; until then each of its ids pools as if it were
+    absent from its bag (the pooled rows equal those of a plain table fed the
+    batch without those ids) and its gradients are dropped."""
+    A, d = 5, 4
+    o = Oracle(d, "sgd")
+    o.set_hooks(admit_threshold=A)
+    counts = {100: 1, 200: 2, 300: 3, 400: 5, 500: 7}
+    keys = np.array([k for k, c in counts.items() for _ in range(c)], np.int64)
+    rng = np.random.default_rng(43)
+    for call in range(1, 7):
+        keys_c = rng.permutation(keys)
+        offs = np.array([0, keys_c.size // 2, keys_c.size], np.int64)
+        before = {k for k in counts if -(-A // counts[k]) < call}  # admitted in an earlier call
+        now = {k for k in counts if -(-A // counts[k]) <= call}
+        pooled, _ = o.forward(keys_c, offs)
+        # reference: a plain table holding only the admitted keys, same values
+        ref = Oracle(d, "sgd")
+        keep = np.array([k in now for k in keys_c])
+        ref_off = np.concatenate([[0], np.cumsum([keep[:keys_c.size // 2].sum(), keep[keys_c.size // 2:].sum()])])
+        ref_keys = keys_c[keep]
+        got_rows, missing = o.get_rows(np.array(sorted(now), np.int64)) if now else (None, 0)
+        assert missing == 0
+        ref.lookup_or_insert(np.array(sorted(now), np.int64))
+        if now:
+            _set_rows(ref, got_rows)
+        rp, _ = ref.forward(ref_keys, ref_off.astype(np.int64))
+        np.testing.assert_array_equal(pooled, rp)
+        for k in now - before:  # admitted in this call: the initial row
+            r, _ = o.get_rows(np.array([k], np.int64))
+            assert np.array_equal(r[0, :d], init_row(k, d))
+        assert o.live == len(now)
+        g = np.ones((2, d), np.float32)
+        assert o.backward_update(keys_c, offs, g, 0.5) == 0  # keys not admitted: skipped, no error
+        ref.close()
+
+
+def test_eviction_live_set_and_row_reuse():
+    """After evict(max_idle) the live keys are exactly those seen in the last
+    max_idle + 1 calls (a set computed from the stream); freed rows are handed
+    to the next admitted keys smallest first, with their initial values; rows
+    of surviving keys are bit-identical."""
+    d = 4
+    o = Oracle(d, "adam")
+    o.set_hooks(track_access=True)
+    rng = np.random.default_rng(47)
+    calls = [rng.choice(60, size=25, replace=False).astype(np.int64) * 7 + 1 for _ in range(6)]
+    for ks in calls:
+        o.forward(ks, np.array([0, ks.size], np.int64))
+        o.backward_update(ks, np.array([0, ks.size], np.int64), rng.standard_normal((1, d)).astype(np.float32), 0.1)
+    keys_before, rows_before = o.export()
+    max_idle = 2
+    recent = set(np.concatenate(calls[-(max_idle + 1):]).tolist())
+    freed = o.evict(max_idle)
+    keys_after, rows_after = o.export()
+    live = set(keys_after[keys_after >= 0].tolist())
+    assert live == recent and o.live == len(recent)
+    free_rows = sorted(np.nonzero(keys_after < 0)[0].tolist())
+    assert freed == len(free_rows) and freed == len(set(keys_before.tolist()) - recent)
+    surv = keys_after >= 0
+    assert np.array_equal(rows_after[surv], rows_before[surv])
+    # new keys take the free rows smallest first, then appended rows
+    fresh = np.array([10_001, 10_002, 10_003] + [20_000 + i for i in range(len(free_rows))], np.int64)
+    off, _ = o.lookup_or_insert(fresh)
+    expect = free_rows + list(range(len(keys_after), len(keys_after) + fresh.size - len(free_rows)))
+    assert off.tolist() == expect
+    r, _ = o.get_rows(fresh[:1])
+    assert np.array_equal(r[0, :d], init_row(int(fresh[0]), d)) and np.all(r[0, d:] == 0)
+    # an evicted key that returns is a new key: a fresh initial row
+    gone = sorted(set(keys_before.tolist()) - recent)[0]
+    o.lookup_or_insert(np.array([gone], np.int64))
+    r, _ = o.get_rows(np.array([gone], np.int64))
+    assert np.array_equal(r[0, :d], init_row(int(gone), d)) and np.all(r[0, d:] == 0)
