@@ -5,7 +5,14 @@ One step = key packing, embbag_forward and embbag_backward_update over one
 batch of the 26-table DLRM-style merged workload (65,536 samples x 26 ids,
 pooling 1, dim 128 fp32, Adagrad, Zipf 1.05 ids; synthetic, seeded).  The
 table starts empty: warm-up steps are the stream's first steps, timed steps
-the ones after.  Prints one JSON line.
+the ones after.  After the headline, the other four workloads (tiny uniform,
+sequence bags, growth stream, hot key) and the headline's stream on a table
+with bf16 weights are each run whole with their own step counts and reported
+under "workloads", with capacity reserved before step 0; the growth stream
+runs a second time with its table growing on demand inside the timed steps
+("growth_stream:on-demand").  "e2e" repeats the headline steps through the public
+API from pinned host buffers, with the copies pipelined against the compute.
+Prints one JSON line.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl dhs|reference]
 
@@ -46,10 +53,16 @@ def stride_floats(dim: int, opt: str) -> int:
     return dim + {"sgd": 0, "adagrad": dim, "adam": 2 * dim, "adagrad_rowwise": 4}[opt]
 
 
-def alg_bytes(n: int, b: int, u: int, m: int, dim: int, opt: str) -> dict:
+def row_bytes(dim: int, opt: str, weights: str = "f32"):
+    """(R, S): bytes of a row's weights, and of the whole row with its fp32
+    optimizer state."""
+    r = (2 if weights == "bf16" else 4) * dim
+    return r, r + 4 * (stride_floats(dim, opt) - dim)
+
+
+def alg_bytes(n: int, b: int, u: int, m: int, dim: int, opt: str, weights: str = "f32") -> dict:
     """Per step.  n ids, b bags, u distinct keys, m of them new."""
-    R = 4 * dim
-    S = 4 * stride_floats(dim, opt)
+    R, S = row_bytes(dim, opt, weights)
     pack = 4 * n + 8 * n + 8 * n
     fwd_pool = 8 * n + 8 * (b + 1) + 16 * u + 16 * m + R * (u - m) + 4 * dim * b
     fwd_assign = S * m + 16 * m
@@ -303,19 +316,33 @@ def default_reserve(w, steps: int) -> int:
     return int(w.params["rows"]) + 1
 
 
+def resolve_reserve(w, steps: int, policy) -> int:
+    """Keys reserved before step 0: an explicit count, -1 for the workload's
+    default, or "on-demand" (0: the table grows inside the timed steps; a
+    pre-populated table still gets room for its pre-inserted keys)."""
+    if policy == "on-demand":
+        return int(w.params["rows"]) + 1 if w.name == "hot_key" else 0
+    policy = int(policy)
+    return default_reserve(w, steps) if policy < 0 else policy
+
+
 def workload_config(w, reserve: int, flush: bool) -> dict:
+    table = ("starts as the workload defines it; "
+             + (f"capacity for {reserve} keys reserved before step 0" if reserve
+                else "grows on demand inside the timed steps (no reservation)")
+             + "; warm-up = the stream's first steps")
     return {"workload": f"{w.name}: " + DESCRIPTIONS[w.name].format(batch=w.params.get("batch")),
             "dim": w.dim, "optimizer": w.optimizer,
             "l2": ("L2 flushed (512 MB written) before each timed step; each step is timed on its own"
                    if flush else "inputs larger than L2 (per-step gradients and ids exceed 2 x 126 MB)"),
-            "table": f"starts as the workload defines it; capacity for {reserve} keys reserved before step 0; "
-                     "warm-up = the stream's first steps"}
+            "table": table}
 
 
-def setup_table(dhs, w, reserve: int):
+def setup_table(dhs, w, reserve: int, weights: str = "f32"):
     """A table for the workload, capacity reserved and any pre-insertion done."""
     import torch
-    t = dhs.ht_create(w.dim, w.optimizer, block_rows=w.block_rows, eps=w.eps, beta1=w.beta1, beta2=w.beta2)
+    t = dhs.ht_create(w.dim, w.optimizer, block_rows=w.block_rows, eps=w.eps, beta1=w.beta1, beta2=w.beta2,
+                      weights=weights)
     if reserve:
         dhs.ht_reserve(t, reserve)
     for tids, ids in w.preinsert():
@@ -326,28 +353,61 @@ def setup_table(dhs, w, reserve: int):
 
 
 # ---------------------------------------------------------------------------
+# host inputs, generated in a process pool started before the first CUDA call
+# ---------------------------------------------------------------------------
+_WORKLOAD_CACHE = {}
+
+
+def _gen_batch(job):
+    name, rank, batch, step = job
+    key = (name, rank, batch)
+    if key not in _WORKLOAD_CACHE:
+        _WORKLOAD_CACHE[key] = make_workload(name, rank, batch)
+    b = _WORKLOAD_CACHE[key].batch(step)
+    return step, b.table_ids, b.ids, b.bag_offsets
+
+
+class BatchSource:
+    """Seeded host batches of a workload's steps.  Generation runs in a
+    `spawn` process pool (no CUDA state is inherited), so that the long
+    streams' inputs are ready in seconds."""
+
+    def __init__(self, procs: int):
+        self.pool = None
+        if procs > 1:
+            import multiprocessing as mp
+            self.pool = mp.get_context("spawn").Pool(procs)
+
+    def batches(self, name: str, rank: int, batch: int, steps: int):
+        jobs = [(name, rank, batch, s) for s in range(steps)]
+        out = self.pool.map(_gen_batch, jobs, chunksize=1) if self.pool else [_gen_batch(j) for j in jobs]
+        out.sort(key=lambda x: x[0])
+        return [gen.Batch(t, i, o) for _, t, i, o in out]
+
+    def close(self):
+        if self.pool:
+            self.pool.close()
+            self.pool.join()
+            self.pool = None
+
+
+# ---------------------------------------------------------------------------
 # the device run
 # ---------------------------------------------------------------------------
-def run_dhs(args):
+def measure(dhs, w, host_batches, device, dist, warmup: int, reserve: int, grad_buffers: int,
+            clock_index: int, want_traffic: bool, weights: str = "f32") -> dict:
+    """Run the workload's first warmup + K steps (K = len(host_batches) -
+    warmup) with every input resident in HBM, timing the last K with CUDA
+    events on the launching stream (one event per step boundary; the time is
+    the max over ranks).  Returns the measured quantities."""
     import torch
-    world, rank, local = dist_env()
-    torch.cuda.set_device(local)
-    device = torch.device("cuda", local)
-    dist = init_dist(world, "nccl")
-    import dynamic_hashed_sparse_b200 as dhs
-
-    w = make_workload(args.workload, rank, args.batch)
-    total = args.warmup + args.steps
-    reserve = default_reserve(w, total) if args.reserve_keys < 0 else args.reserve_keys
-    # inputs for every step, resident in HBM before the timed region
-    batches = []
-    for s in range(total):
-        b = w.batch(s)
-        batches.append((torch.from_numpy(b.table_ids).to(device), torch.from_numpy(b.ids).to(device),
-                        torch.from_numpy(b.bag_offsets).to(device), b.n, b.n_bags))
+    total = len(host_batches)
+    K = total - warmup
+    batches = [(torch.from_numpy(b.table_ids).to(device), torch.from_numpy(b.ids).to(device),
+                torch.from_numpy(b.bag_offsets).to(device), b.n, b.n_bags) for b in host_batches]
     n_max = max(x[3] for x in batches)
     nb_max = max(x[4] for x in batches)
-    n_grad = min(total, args.grad_buffers)
+    n_grad = min(total, grad_buffers)
     grads = [w.torch_grads(s, nb_max, device) for s in range(n_grad)]
     pooled = torch.empty((nb_max, w.dim), dtype=torch.float32, device=device)
     keys = torch.empty(max(1, n_max), dtype=torch.int64, device=device)
@@ -356,7 +416,7 @@ def run_dhs(args):
     flush = step_bytes < 2 * L2_BYTES
     fbuf = torch.empty(512 << 20, dtype=torch.uint8, device=device) if flush else None
 
-    t = setup_table(dhs, w, reserve)
+    t = setup_table(dhs, w, reserve, weights)
     stream = torch.cuda.current_stream()
 
     def step(s):
@@ -366,7 +426,7 @@ def run_dhs(args):
         dhs.embbag_forward(t, k, offs, out=pooled[:nb])
         dhs.embbag_backward_update(t, k, offs, grads[s % n_grad][:nb], w.lr)
 
-    for s in range(args.warmup):
+    for s in range(warmup):
         step(s)
     torch.cuda.synchronize()
     c0 = dhs.ht_counters(t)
@@ -375,43 +435,45 @@ def run_dhs(args):
     barrier(dist, device)
     torch.cuda.synchronize()
     spans = []
-    with ClockSampler(local) as clk:
+    with ClockSampler(clock_index) as clk:
         if not flush:
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record(stream)
-            for s in range(args.warmup, total):
+            ev = [torch.cuda.Event(enable_timing=True) for _ in range(K + 1)]
+            ev[0].record(stream)
+            for i, s in enumerate(range(warmup, total)):
                 step(s)
-            e1.record(stream)
-            spans.append((e0, e1))
+                ev[i + 1].record(stream)
+            torch.cuda.synchronize()
+            spans = [ev[i].elapsed_time(ev[i + 1]) for i in range(K)]
+            ms_local = ev[0].elapsed_time(ev[K])
         else:
-            for s in range(args.warmup, total):
+            pairs = []
+            for s in range(warmup, total):
                 fbuf.zero_()
                 e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
                 e0.record(stream)
                 step(s)
                 e1.record(stream)
-                spans.append((e0, e1))
-        torch.cuda.synchronize()
+                pairs.append((e0, e1))
+            torch.cuda.synchronize()
+            spans = [a.elapsed_time(b) for a, b in pairs]
+            ms_local = sum(spans)
     barrier(dist, device)
     dhs.ht_set_phase_timing(t, False)
-    ms_local = sum(a.elapsed_time(b) for a, b in spans)
     phases = dhs.ht_phase_times(t)
     c1 = dhs.ht_counters(t)
     status = dhs.ht_sync(t)
     if status != 0:
-        raise RuntimeError(f"device status {status} ({dhs.dhs_status_str(status)}) after the timed steps")
+        raise RuntimeError(f"{w.name}: device status {status} ({dhs.dhs_status_str(status)}) after the timed steps")
 
-    K = args.steps
-    n_ids = sum(batches[s][3] for s in range(args.warmup, total))
-    n_bags = sum(batches[s][4] for s in range(args.warmup, total))
+    n_ids = sum(batches[s][3] for s in range(warmup, total))
+    n_bags = sum(batches[s][4] for s in range(warmup, total))
     U = c1["unique_updated"] - c0["unique_updated"]
     M = c1["inserted"] - c0["inserted"]
     launches = c1["launches"] - c0["launches"] + K  # + one key-packing kernel per step
     ms = max_over_ranks(ms_local, dist, device)
     ids_all = sum_over_ranks(float(n_ids), dist, device)
-    value = ids_all / (ms / 1e3)
 
-    ab = alg_bytes(n_ids, n_bags, U, M, w.dim, w.optimizer)
+    ab = alg_bytes(n_ids, n_bags, U, M, w.dim, w.optimizer, weights)
     peaks = load_peaks()
     ph_ms = {k: v[0] for k, v in phases.items()}
     ph_cnt = {k: v[1] for k, v in phases.items()}
@@ -425,8 +487,8 @@ def run_dhs(args):
                  if dom == "fwd_probe_pool" else ab["bwd_seg"])
     dom_launch_ms = ph_ms[dom] / max(1, ph_cnt[dom])
     dom_bytes_per_launch = dom_bytes / max(1, ph_cnt[dom])
-    achieved = dom_bytes_per_launch / (dom_launch_ms / 1e3) / 1e9
-    traffic = load_traffic(dom_kernel) if w.name == "dlrm_merged_26" else None
+    achieved = dom_bytes_per_launch / (dom_launch_ms / 1e3) / 1e9 if dom_launch_ms else 0.0
+    traffic = load_traffic(dom_kernel) if want_traffic else None
     roofline = {
         "bound": "hbm", "kernel": dom_kernel, "achieved": achieved, "peak": peaks["hbm_gbs"],
         "peak_source": peaks["source"], "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
@@ -438,17 +500,18 @@ def run_dhs(args):
     def gbs(nbytes, t_ms):
         return nbytes / (t_ms / 1e3) / 1e9 if t_ms else None
 
-    line = {
-        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
-        "ms_per_step": ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "timing_valid": args.warmup >= 3,
-        "dtype": "f32", "data": "synthetic", "config": workload_config(w, reserve, flush),
+    def frac(nbytes, t_ms):
+        g = gbs(nbytes, t_ms)
+        return g / peaks["hbm_gbs"] if g is not None else None
+
+    res = {
+        "value": ids_all / (ms / 1e3), "ms_per_step": ms / K, "steps": K, "warmup": warmup,
+        "median_step_ms": statistics.median(spans) if spans else None,
+        "flush": flush, "reserve": reserve,
         "fwd": {"ids_per_s": n_ids / (fwd_ms / 1e3) if fwd_ms else None, "ms_per_step": fwd_ms / K,
-                "gbs": gbs(ab["fwd"], fwd_ms),
-                "frac_of_peak": gbs(ab["fwd"], fwd_ms) / peaks["hbm_gbs"] if fwd_ms else None},
+                "gbs": gbs(ab["fwd"], fwd_ms), "frac_of_peak": frac(ab["fwd"], fwd_ms)},
         "bwd": {"ids_per_s": n_ids / (bwd_ms / 1e3) if bwd_ms else None, "ms_per_step": bwd_ms / K,
-                "gbs": gbs(ab["bwd"], bwd_ms),
-                "frac_of_peak": gbs(ab["bwd"], bwd_ms) / peaks["hbm_gbs"] if bwd_ms else None},
+                "gbs": gbs(ab["bwd"], bwd_ms), "frac_of_peak": frac(ab["bwd"], bwd_ms)},
         "step_gbs": gbs(ab["fwd"] + ab["bwd"], ms_local),
         "phases_ms_per_step": {k: v / K for k, v in ph_ms.items() if ph_cnt[k]},
         "per_step": {"ids": n_ids / K, "bags": n_bags / K, "unique": U / K, "new": M / K},
@@ -459,15 +522,82 @@ def run_dhs(args):
                   "timed_growth": {"rehashes": c1["rehashes"] - c0["rehashes"],
                                    "blocks_appended": c1["blocks"] - c0["blocks"],
                                    "device_allocs": c1["allocs"] - c0["allocs"],
+                                   "alloc_ms": (c1["alloc_ns"] - c0["alloc_ns"]) / 1e6,
+                                   "idmap_growth_ms": ph_ms.get("idmap_growth", 0.0),
+                                   "host_waits": c1["host_waits"] - c0["host_waits"],
                                    "host_wait_ms": (c1["host_wait_ns"] - c0["host_wait_ns"]) / 1e6}},
+        "clocks": clk.summary(),
+        "config": dict(workload_config(w, reserve, flush), weights=weights),
     }
-    line["clocks"] = clk.summary()
     t.close()
-    del grads, batches, fbuf
+    del grads, batches, fbuf, pooled, keys
     torch.cuda.empty_cache()
+    return res
+
+
+# the other configs, each run whole: (label, workload, weight storage, capacity policy)
+EXTRA_WORKLOADS = (
+    ("tiny_uniform", "tiny_uniform", "f32", "-1"),
+    ("sequence_bags", "sequence_bags", "f32", "-1"),
+    ("growth_stream", "growth_stream", "f32", "-1"),
+    ("growth_stream:on-demand", "growth_stream", "f32", "on-demand"),
+    ("hot_key", "hot_key", "f32", "-1"),
+    ("dlrm_merged_26:bf16", "dlrm_merged_26", "bf16", "-1"),
+)
+
+
+def run_dhs(args):
+    world, rank, local = dist_env()
+    procs = max(1, min(16, (os.cpu_count() or 2) // max(1, world) - 1))
+    src = BatchSource(procs)  # before the first CUDA call
+    import torch
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    dist = init_dist(world, "nccl")
+    import dynamic_hashed_sparse_b200 as dhs
+
+    w = make_workload(args.workload, rank, args.batch)
+    total = args.warmup + args.steps
+    reserve = resolve_reserve(w, total, args.reserve_keys)
+    host_batches = src.batches(args.workload, rank, args.batch, total)
+    head = measure(dhs, w, host_batches, device, dist, args.warmup, reserve, args.grad_buffers, local,
+                   want_traffic=(w.name == "dlrm_merged_26" and not args.batch))
+    K = args.steps
+    line = {
+        "metric": METRIC, "value": head["value"], "unit": UNIT, "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": head["ms_per_step"], "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "timing_valid": args.warmup >= 3,
+        "dtype": "f32", "data": "synthetic", "config": head["config"],
+    }
+    for k in ("fwd", "bwd", "step_gbs", "median_step_ms", "phases_ms_per_step", "per_step", "roofline",
+              "gpu_launches", "table", "clocks"):
+        line[k] = head[k]
+
+    # the other configs, each run whole with its own step count
+    wanted = [] if args.workloads == "none" else (
+        [e for e in EXTRA_WORKLOADS if not (e[0] == args.workload)] if args.workloads == "all"
+        else [e for e in EXTRA_WORKLOADS if e[0] in args.workloads.split(",")])
+    if wanted:
+        extra = {}
+        for label, name, weights, policy in wanted:
+            wx = make_workload(name, rank)
+            wsteps = wx.steps
+            wwarm = min(3, wsteps - 1)
+            hb = src.batches(name, rank, 0, wsteps)
+            r = measure(dhs, wx, hb, device, dist, wwarm, resolve_reserve(wx, wsteps, policy),
+                        args.grad_buffers, local, want_traffic=False, weights=weights)
+            extra[label] = {"ids_per_s": r["value"], "ms_per_step": r["ms_per_step"],
+                            "median_step_ms": r["median_step_ms"], "steps": r["steps"], "warmup": r["warmup"],
+                            "fwd": r["fwd"], "bwd": r["bwd"], "roofline": r["roofline"],
+                            "phases_ms_per_step": r["phases_ms_per_step"], "per_step": r["per_step"],
+                            "table": r["table"], "clocks": r["clocks"], "config": r["config"]}
+            del hb
+        line["workloads"] = extra
+    src.close()
 
     if not args.no_e2e:
-        line["e2e"] = run_e2e(args, w, device, dist, reserve)
+        line["e2e"] = run_e2e(dhs, w, host_batches, device, dist, reserve, args.warmup)
+    del host_batches
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         ids, secs = time_oracle(make_workload(args.workload, 0, args.batch), args.cpu_steps, args.cpu_frac)
         line["cpu_baseline"] = {"value": ids / secs, "unit": UNIT, "cores": cpu_cores_used(), "kind": "oracle",
@@ -481,71 +611,104 @@ def run_dhs(args):
     return 0
 
 
-def run_e2e(args, w, device, dist, reserve):
-    """The same step through the public API with host inputs: per step, copy
-    the ids, table ids, bag offsets and gradients from pinned host memory,
-    run the step, and copy the pooled output back; all inside the timed
-    region."""
+def run_e2e(dhs, w, host_batches, device, dist, reserve, warmup):
+    """The same steps through the public API with host inputs.  Every step
+    copies its ids, table ids, bag offsets and gradients in from pinned host
+    memory and copies its pooled output back, all inside the timed region.
+    The copies are pipelined: step s+2's inputs go in on one copy stream and
+    step s's pooled output comes back on another while step s computes
+    (device inputs and outputs double-buffered, ordered by events), so a step
+    costs about its larger transfer rather than the sum of both."""
     import torch
 
-    import dynamic_hashed_sparse_b200 as dhs
-    total = args.warmup + args.steps
-    hb = []
-    for s in range(total):
-        b = w.batch(s)
-        hb.append((torch.from_numpy(b.table_ids).pin_memory(), torch.from_numpy(b.ids).pin_memory(),
-                   torch.from_numpy(b.bag_offsets).pin_memory(), b.n, b.n_bags))
+    total = len(host_batches)
+    K = total - warmup
+    hb = [(torch.from_numpy(b.table_ids).pin_memory(), torch.from_numpy(b.ids).pin_memory(),
+           torch.from_numpy(b.bag_offsets).pin_memory(), b.n, b.n_bags) for b in host_batches]
     n_max = max(x[3] for x in hb)
     nb_max = max(x[4] for x in hb)
-    n_grad = 2
-    hgrads = [w.torch_grads(s, nb_max, device).cpu().pin_memory() for s in range(n_grad)]
-    hpooled = torch.empty((nb_max, w.dim), dtype=torch.float32).pin_memory()
-    d_tids = torch.empty(max(1, n_max), dtype=torch.int32, device=device)
-    d_ids = torch.empty(max(1, n_max), dtype=torch.int64, device=device)
-    d_keys = torch.empty(max(1, n_max), dtype=torch.int64, device=device)
-    d_offs = torch.empty(nb_max + 1, dtype=torch.int64, device=device)
-    d_grad = torch.empty((nb_max, w.dim), dtype=torch.float32, device=device)
-    d_pooled = torch.empty((nb_max, w.dim), dtype=torch.float32, device=device)
+    hgrads = [w.torch_grads(s, nb_max, device).cpu().pin_memory() for s in range(2)]
+    hpooled = [torch.empty((nb_max, w.dim), dtype=torch.float32).pin_memory() for _ in range(2)]
+
+    def dbuf():
+        return {"tids": torch.empty(max(1, n_max), dtype=torch.int32, device=device),
+                "ids": torch.empty(max(1, n_max), dtype=torch.int64, device=device),
+                "keys": torch.empty(max(1, n_max), dtype=torch.int64, device=device),
+                "offs": torch.empty(nb_max + 1, dtype=torch.int64, device=device),
+                "grad": torch.empty((nb_max, w.dim), dtype=torch.float32, device=device),
+                "pooled": torch.empty((nb_max, w.dim), dtype=torch.float32, device=device)}
+
+    bufs = [dbuf(), dbuf()]
     t = setup_table(dhs, w, reserve)
-    h2d = d2h = 0
+    s_in, s_cmp, s_out = torch.cuda.Stream(device), torch.cuda.Stream(device), torch.cuda.Stream(device)
+    ev_in = [torch.cuda.Event() for _ in range(2)]
+    ev_cmp = [torch.cuda.Event() for _ in range(2)]
+    ev_out = [torch.cuda.Event() for _ in range(2)]
+    moved = {"h2d": 0, "d2h": 0}
 
-    def step(s):
-        nonlocal h2d, d2h
+    def h2d(s):
+        k = s % 2
         tids, ids, offs, n, nb = hb[s]
-        g = hgrads[s % n_grad]
-        d_tids[:n].copy_(tids, non_blocking=True)
-        d_ids[:n].copy_(ids, non_blocking=True)
-        d_offs[: nb + 1].copy_(offs, non_blocking=True)
-        d_grad[:nb].copy_(g[:nb], non_blocking=True)
-        k = d_keys[:n]
-        dhs.dhs_pack_keys(d_tids[:n], d_ids[:n], out=k)
-        dhs.embbag_forward(t, k, d_offs[: nb + 1], out=d_pooled[:nb])
-        dhs.embbag_backward_update(t, k, d_offs[: nb + 1], d_grad[:nb], w.lr)
-        hpooled[:nb].copy_(d_pooled[:nb], non_blocking=True)
-        h2d += tids.numel() * 4 + ids.numel() * 8 + (nb + 1) * 8 + nb * w.dim * 4
-        d2h += nb * w.dim * 4
+        d = bufs[k]
+        with torch.cuda.stream(s_in):
+            s_in.wait_event(ev_cmp[k])  # step s-2 has finished reading this buffer
+            d["tids"][:n].copy_(tids, non_blocking=True)
+            d["ids"][:n].copy_(ids, non_blocking=True)
+            d["offs"][: nb + 1].copy_(offs, non_blocking=True)
+            d["grad"][:nb].copy_(hgrads[s % 2][:nb], non_blocking=True)
+            ev_in[k].record(s_in)
+        moved["h2d"] += tids.numel() * 4 + ids.numel() * 8 + (nb + 1) * 8 + nb * w.dim * 4
 
-    for s in range(args.warmup):
-        step(s)
+    def compute_and_d2h(s):
+        k = s % 2
+        _, _, _, n, nb = hb[s]
+        d = bufs[k]
+        with torch.cuda.stream(s_cmp):
+            s_cmp.wait_event(ev_in[k])
+            s_cmp.wait_event(ev_out[k])  # step s-2's output has left this buffer
+            kk = d["keys"][:n]
+            dhs.dhs_pack_keys(d["tids"][:n], d["ids"][:n], out=kk, stream=s_cmp)
+            dhs.embbag_forward(t, kk, d["offs"][: nb + 1], out=d["pooled"][:nb], stream=s_cmp)
+            dhs.embbag_backward_update(t, kk, d["offs"][: nb + 1], d["grad"][:nb], w.lr, stream=s_cmp)
+            ev_cmp[k].record(s_cmp)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(ev_cmp[k])
+            hpooled[k][:nb].copy_(d["pooled"][:nb], non_blocking=True)
+            ev_out[k].record(s_out)
+        moved["d2h"] += nb * w.dim * 4
+
+    def run(first, last):
+        for s in range(first, min(first + 2, last)):
+            h2d(s)
+        for s in range(first, last):
+            compute_and_d2h(s)
+            if s + 2 < last:
+                h2d(s + 2)
+
+    run(0, warmup)
     torch.cuda.synchronize()
-    h2d = d2h = 0
+    moved["h2d"] = moved["d2h"] = 0
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(dist, device)
     torch.cuda.synchronize()
-    e0.record()
-    for s in range(args.warmup, total):
-        step(s)
-    e1.record()
+    e0.record(s_in)
+    run(warmup, total)
+    s_out.wait_stream(s_cmp)
+    s_out.wait_stream(s_in)
+    e1.record(s_out)
     torch.cuda.synchronize()
     ms = max_over_ranks(e0.elapsed_time(e1), dist, device)
-    ids = sum_over_ranks(float(sum(hb[s][3] for s in range(args.warmup, total))), dist, device)
+    ids = sum_over_ranks(float(sum(hb[s][3] for s in range(warmup, total))), dist, device)
     status = dhs.ht_sync(t)
     t.close()
+    del bufs, hb, hgrads, hpooled
+    torch.cuda.empty_cache()
     if status != 0:
         raise RuntimeError(f"device status {status} in the end-to-end run")
-    K = args.steps
-    return {"value": ids / (ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d // K,
-            "d2h_bytes_per_step": d2h // K, "ms_per_step": ms / K}
+    return {"value": ids / (ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": moved["h2d"] // K,
+            "d2h_bytes_per_step": moved["d2h"] // K, "ms_per_step": ms / K,
+            "pipeline": "H2D of step s+2 and D2H of step s overlap the compute of step s (3 streams, "
+                        "double-buffered device inputs/outputs)"}
 
 
 def main(argv=None):
@@ -555,14 +718,17 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="dhs", choices=["dhs", "reference"])
     ap.add_argument("--workload", default=WORKLOAD, choices=list(gen.NAMES))
+    ap.add_argument("--workloads", default="all",
+                    help="other configs measured after the headline, each run whole: 'all', 'none' or a "
+                         "comma-separated list of labels (" + ", ".join(e[0] for e in EXTRA_WORKLOADS) + ")")
     ap.add_argument("--grad-buffers", type=int, default=32)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-steps", type=int, default=5)
     ap.add_argument("--ref-frac", type=float, default=1.0 / 16)
-    ap.add_argument("--reserve-keys", type=int, default=-1,
-                    help="capacity reserved (ht_reserve) before step 0; -1 = what the workload reaches in "
-                         "the run plus one batch; 0 = grow on demand")
+    ap.add_argument("--reserve-keys", default="-1",
+                    help="headline: capacity reserved (ht_reserve) before step 0; -1 = what the workload "
+                         "reaches in the run plus one batch; 0 or 'on-demand' = grow inside the timed steps")
     ap.add_argument("--cpu-frac", type=float, default=1.0,
                     help="fraction of each batch's bags the CPU-baseline oracle processes")
     ap.add_argument("--batch", type=int, default=0,

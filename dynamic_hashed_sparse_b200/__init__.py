@@ -9,12 +9,17 @@ from ._binding import (  # noqa: F401
     OPT_CODES,
     PHASES,
     Table,
+    TorchAllocator,
     dhs_pack_keys,
     dhs_status_str,
     embbag_backward_update,
     embbag_backward_update_noalloc,
     NOALLOC_MAX_KEYS,
     embbag_forward,
+    embbag_forward_ex,
+    embbag_backward_update_ex,
+    POOL_MODES,
+    ROW_DTYPES,
     ht_counters,
     ht_create,
     ht_destroy,
@@ -24,6 +29,9 @@ from ._binding import (  # noqa: F401
     ht_lookup_or_insert,
     ht_phase_times,
     ht_reserve,
+    ht_set_hooks,
+    ht_evict,
+    ht_live_rows,
     ht_row_stride,
     ht_set_phase_timing,
     ht_size,

@@ -10,6 +10,7 @@ from __future__ import annotations
 
 import ctypes as C
 import os
+import re
 from typing import Optional, Tuple
 
 import numpy as np
@@ -22,6 +23,8 @@ STATUS = {
     4: "table full", 5: "key not found", 6: "unsupported", 7: "internal wait bound exceeded",
 }
 OPT_CODES = {"sgd": 0, "adagrad": 1, "adam": 2, "adagrad_rowwise": 3}
+POOL_MODES = {"sum": 0, "mean": 1}
+ROW_DTYPES = {"f32": 0, "bf16": 1}
 PHASES = ("fwd_probe_pool", "fwd_assign", "bwd_probe", "bwd_sort", "bwd_seg_update",
           "lookup_or_insert", "idmap_growth", "fwd_probe", "bwd_combine")
 
@@ -45,14 +48,20 @@ def _load() -> C.CDLL:
         "dhs_status_str": (C.c_char_p, [C.c_int]),
         "dhs_pack_keys": (C.c_int, [vp, vp, i64, vp, vp]),
         "ht_create": (C.c_int, [i32, C.c_int, i64, i64, vp, vp, C.POINTER(vp)]),
+        "ht_create_ex": (C.c_int, [i32, C.c_int, C.c_int, i64, i64, vp, vp, C.POINTER(vp)]),
         "ht_destroy": (C.c_int, [vp]),
         "ht_reserve": (C.c_int, [vp, i64, vp]),
         "ht_lookup_or_insert": (C.c_int, [vp, vp, i64, vp, vp]),
         "ht_lookup": (C.c_int, [vp, vp, i64, vp, vp]),
         "embbag_forward": (C.c_int, [vp, vp, i64, vp, i64, vp, vp]),
         "embbag_backward_update": (C.c_int, [vp, vp, i64, vp, i64, vp, f32, vp]),
+        "embbag_forward_ex": (C.c_int, [vp, vp, i64, vp, i64, vp, C.c_int, vp, vp]),
+        "embbag_backward_update_ex": (C.c_int, [vp, vp, i64, vp, i64, vp, C.c_int, vp, f32, vp]),
         "embbag_backward_update_noalloc": (C.c_int, [vp, vp, i64, vp, i64, vp, f32, vp]),
         "ht_get_rows": (C.c_int, [vp, vp, i64, vp, vp]),
+        "ht_set_hooks": (C.c_int, [vp, i64, C.c_int]),
+        "ht_evict": (C.c_int, [vp, i64, C.POINTER(i64), vp]),
+        "ht_live_rows": (C.c_int, [vp, C.POINTER(i64)]),
         "ht_row_stride": (i64, [vp]),
         "ht_sync": (C.c_int, [vp]),
         "ht_size": (C.c_int, [vp, C.POINTER(i64)]),
@@ -77,6 +86,49 @@ def lib() -> C.CDLL:
 
 class _OptParams(C.Structure):
     _fields_ = [("eps", C.c_float), ("beta1", C.c_float), ("beta2", C.c_float)]
+
+
+# dhs_allocator: alloc(bytes, stream, ctx) -> device pointer or NULL;
+# free(ptr, bytes, stream, ctx)
+ALLOC_FN = C.CFUNCTYPE(C.c_void_p, C.c_size_t, C.c_void_p, C.c_void_p)
+FREE_FN = C.CFUNCTYPE(None, C.c_void_p, C.c_size_t, C.c_void_p, C.c_void_p)
+
+
+class _Allocator(C.Structure):
+    _fields_ = [("alloc", ALLOC_FN), ("free", FREE_FN), ("ctx", C.c_void_p)]
+
+
+class TorchAllocator:
+    """A dhs_allocator backed by torch's caching allocator, counting its calls
+    (alloc_calls, free_calls, live_bytes).  The ctypes callbacks are kept
+    alive by this object, which must outlive every table created with it."""
+
+    def __init__(self, device=None):
+        self.device = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+        self.alloc_calls = 0
+        self.free_calls = 0
+        self.live_bytes = 0
+        self._sizes = {}
+
+        def _alloc(nbytes, stream, ctx):
+            try:
+                p = torch.cuda.caching_allocator_alloc(int(nbytes), self.device, int(stream or 0))
+            except RuntimeError:
+                return None
+            self.alloc_calls += 1
+            self.live_bytes += int(nbytes)
+            self._sizes[int(p)] = int(nbytes)
+            return int(p)
+
+        def _free(ptr, nbytes, stream, ctx):
+            if ptr:
+                self.free_calls += 1
+                self.live_bytes -= self._sizes.pop(int(ptr), 0)
+                torch.cuda.caching_allocator_delete(int(ptr))
+
+        self._c_alloc = ALLOC_FN(_alloc)
+        self._c_free = FREE_FN(_free)
+        self.struct = _Allocator(self._c_alloc, self._c_free, None)
 
 
 def _check(fn: str, rc: int):
@@ -105,12 +157,13 @@ def _dev(t: torch.Tensor, dtype, name: str) -> torch.Tensor:
 class Table:
     """Handle of one library-owned table (IDMap + EmbeddingBlocks)."""
 
-    def __init__(self, handle: int, dim: int, optimizer: str, device: torch.device):
+    def __init__(self, handle: int, dim: int, optimizer: str, device: torch.device, weights: str = "f32"):
         self.handle = handle
         self.dim = dim
         self.optimizer = optimizer
         self.device = device
-        self.stride = int(_lib.ht_row_stride(handle))
+        self.weights = weights
+        self.stride = int(_lib.ht_row_stride(handle))  # floats per exported row
 
     def close(self):
         if self.handle:
@@ -143,15 +196,20 @@ def dhs_pack_keys(table_ids: torch.Tensor, ids: torch.Tensor, out: Optional[torc
 
 def ht_create(dim: int, optimizer: str = "sgd", block_rows: int = 0, max_rows: int = 0,
               eps: float = 1e-8, beta1: float = 0.9, beta2: float = 0.999,
-              device=None) -> Table:
+              device=None, allocator: Optional[TorchAllocator] = None, weights: str = "f32") -> Table:
+    """A new table; weights "f32" or "bf16" (bf16 weights, fp32 optimizer
+    state: ht_create_ex)."""
     device = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
     p = _OptParams(eps, beta1, beta2)
     h = C.c_void_p()
     with torch.cuda.device(device):
-        rc = _lib.ht_create(int(dim), OPT_CODES[optimizer], int(block_rows), int(max_rows),
-                            C.byref(p), None, C.byref(h))
+        rc = _lib.ht_create_ex(int(dim), OPT_CODES[optimizer], ROW_DTYPES[weights], int(block_rows),
+                               int(max_rows), C.byref(p),
+                               C.byref(allocator.struct) if allocator is not None else None, C.byref(h))
     _check("ht_create", rc)
-    return Table(h.value, int(dim), optimizer, device)
+    t = Table(h.value, int(dim), optimizer, device, weights)
+    t.allocator = allocator  # keeps the callbacks alive as long as the table
+    return t
 
 
 def ht_destroy(t: Table):
@@ -215,7 +273,64 @@ def embbag_backward_update(t: Table, keys: torch.Tensor, bag_offsets: torch.Tens
                                        nb, grad.data_ptr(), float(lr), _stream(stream)))
 
 
-NOALLOC_MAX_KEYS = 131072
+def _header_define(name: str) -> int:
+    with open(os.path.join(_build.INCLUDE, "dhs.h")) as f:
+        m = re.search(rf"#define\s+{name}\s+(\d+)", f.read())
+    if not m:
+        raise ImportError(f"{name} is not defined in include/dhs.h")
+    return int(m.group(1))
+
+
+def _psw(per_sample_weights, keys: torch.Tensor) -> int:
+    if per_sample_weights is None:
+        return 0
+    _dev(per_sample_weights, torch.float32, "per_sample_weights")
+    if per_sample_weights.numel() != keys.numel():
+        raise ValueError("per_sample_weights needs one weight per key")
+    return per_sample_weights.data_ptr()
+
+
+def embbag_forward_ex(t: Table, keys: torch.Tensor, bag_offsets: torch.Tensor,
+                      per_sample_weights: Optional[torch.Tensor] = None, mode: str = "sum",
+                      out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """EmbeddingBag forward with mode "sum" (optionally weighted per id) or
+    "mean"."""
+    _dev(keys, torch.int64, "keys")
+    _dev(bag_offsets, torch.int64, "bag_offsets")
+    nb = bag_offsets.numel() - 1
+    if nb < 0:
+        raise ValueError("bag_offsets needs n_bags + 1 entries")
+    if out is None:
+        out = torch.empty((nb, t.dim), dtype=torch.float32, device=keys.device)
+    else:
+        _dev(out, torch.float32, "out")
+        if out.numel() != nb * t.dim:
+            raise ValueError("out must hold n_bags * dim floats")
+    _check("embbag_forward_ex",
+           _lib.embbag_forward_ex(t.handle, keys.data_ptr(), keys.numel(), bag_offsets.data_ptr(), nb,
+                                  _psw(per_sample_weights, keys), POOL_MODES[mode], out.data_ptr(),
+                                  _stream(stream)))
+    return out
+
+
+def embbag_backward_update_ex(t: Table, keys: torch.Tensor, bag_offsets: torch.Tensor, grad: torch.Tensor,
+                              lr: float, per_sample_weights: Optional[torch.Tensor] = None, mode: str = "sum",
+                              stream=None):
+    """Backward + update for the pooling forms of embbag_forward_ex (same
+    weights and mode as the forward)."""
+    _dev(keys, torch.int64, "keys")
+    _dev(bag_offsets, torch.int64, "bag_offsets")
+    _dev(grad, torch.float32, "grad")
+    nb = bag_offsets.numel() - 1
+    if grad.numel() != nb * t.dim:
+        raise ValueError("grad must hold n_bags * dim floats")
+    _check("embbag_backward_update_ex",
+           _lib.embbag_backward_update_ex(t.handle, keys.data_ptr(), keys.numel(), bag_offsets.data_ptr(), nb,
+                                          _psw(per_sample_weights, keys), POOL_MODES[mode], grad.data_ptr(),
+                                          float(lr), _stream(stream)))
+
+
+NOALLOC_MAX_KEYS = _header_define("DHS_NOALLOC_MAX_KEYS")
 
 
 def embbag_backward_update_noalloc(t: Table, keys: torch.Tensor, bag_offsets: torch.Tensor,
@@ -245,6 +360,25 @@ def ht_get_rows(t: Table, keys: torch.Tensor, out: Optional[torch.Tensor] = None
     return out
 
 
+def ht_set_hooks(t: Table, admit_threshold: int = 1, track_access: bool = False):
+    """Feature admission threshold and access tracking (before the first insert)."""
+    _check("ht_set_hooks", _lib.ht_set_hooks(t.handle, int(admit_threshold), int(bool(track_access))))
+
+
+def ht_evict(t: Table, max_idle: int, stream=None) -> int:
+    """Evict keys idle for more than max_idle insert calls; returns the rows freed."""
+    n = C.c_int64()
+    _check("ht_evict", _lib.ht_evict(t.handle, int(max_idle), C.byref(n), _stream(stream)))
+    return int(n.value)
+
+
+def ht_live_rows(t: Table) -> Tuple[int, int]:
+    """(rows held by keys, latched status)."""
+    n = C.c_int64()
+    rc = _lib.ht_live_rows(t.handle, C.byref(n))
+    return int(n.value), int(rc)
+
+
 def ht_row_stride(t: Table) -> int:
     return int(_lib.ht_row_stride(t.handle))
 
@@ -260,12 +394,14 @@ def ht_size(t: Table) -> Tuple[int, int]:
     return int(n.value), int(rc)
 
 
-def ht_export(t: Table) -> Tuple[np.ndarray, np.ndarray, int]:
+def ht_export(t: Table, rows: bool = True) -> Tuple[np.ndarray, Optional[np.ndarray], int]:
+    """(keys by row, rows or None, latched status).  rows=False exports the
+    key -> row map only."""
     n, rc = ht_size(t)
     keys = np.empty(n, np.int64)
-    rows = np.empty((n, t.stride), np.float32)
-    rc2 = _lib.ht_export(t.handle, keys.ctypes.data, rows.ctypes.data)
-    return keys, rows, int(rc or rc2)
+    r = np.empty((n, t.stride), np.float32) if rows else None
+    rc2 = _lib.ht_export(t.handle, keys.ctypes.data, r.ctypes.data if rows else None)
+    return keys, r, int(rc or rc2)
 
 
 def ht_counters(t: Table) -> dict:

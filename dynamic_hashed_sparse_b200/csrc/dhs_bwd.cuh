@@ -71,11 +71,18 @@ namespace dhs {
 // is the number of the chunk's bag ends at or before it (a binary search over
 // the ends held in the lanes' registers).  Missing or negative keys get row
 // `sentinel` (sorted last, never updated).
+// Extended pooling (per-sample weights psw, or mean pooling): the sort value
+// is the position instead of the bag; bagpos[p] = its bag and mult[p] = the
+// factor its bag's gradient is scaled by (psw[p], or 1 / the bag's length).
+template <bool EXT>
 __global__ void __launch_bounds__(256)
 bwd_probe_kernel(IdMap m, const long long* __restrict__ keys, long long n_keys,
                  const long long* __restrict__ bag_off, long long n_bags,
                  unsigned* __restrict__ rkey, unsigned* __restrict__ rval, unsigned sentinel,
-                 unsigned* __restrict__ sort_zero, int sort_zero_words, int bpc, DevState* st) {
+                 unsigned* __restrict__ sort_zero, int sort_zero_words, int bpc,
+                 const float* __restrict__ psw, bool mean, unsigned* __restrict__ bagpos,
+                 double* __restrict__ mult, DevState* st) {
+  constexpr bool ext = EXT;
   constexpr unsigned FULL = 0xffffffffu;
   const int lane = threadIdx.x & 31;
   if (blockIdx.x == 0)  // the sort's digit histograms and tile counters start at zero
@@ -156,17 +163,38 @@ bwd_probe_kernel(IdMap m, const long long* __restrict__ keys, long long n_keys,
       if (p0 < E && k0 >= 0) f0 = probe_find(m, (unsigned long long)k0);
       if (p1 < E && k1 >= 0) f1 = probe_find(m, (unsigned long long)k1);
       const int g0 = bag_of(p0), g1 = bag_of(p1);
+      // f < 0: no row (-1 absent: an error; -2 known but not admitted: skipped)
       if (p0 < E) {
         if (k0 < 0) latch(st, kErrInvalid);
-        else if (f0 < 0) latch(st, kErrNotFound);
+        else if (f0 == -1) latch(st, kErrNotFound);
         rkey[p0] = f0 >= 0 ? (unsigned)f0 : sentinel;
-        rval[p0] = (unsigned)(b0 + g0);
+        rval[p0] = ext ? (unsigned)p0 : (unsigned)(b0 + g0);
       }
       if (p1 < E) {
         if (k1 < 0) latch(st, kErrInvalid);
-        else if (f1 < 0) latch(st, kErrNotFound);
+        else if (f1 == -1) latch(st, kErrNotFound);
         rkey[p1] = f1 >= 0 ? (unsigned)f1 : sentinel;
-        rval[p1] = (unsigned)(b0 + g1);
+        rval[p1] = ext ? (unsigned)p1 : (unsigned)(b0 + g1);
+      }
+      if constexpr (EXT) {
+        // bag g of the chunk spans [end(g - 1), end(g)), end(-1) = s
+        auto bag_end = [&](int g) -> int {
+          const int a0 = __shfl_sync(FULL, e0, g & 31);
+          const int a1 = __shfl_sync(FULL, e1, g & 31);
+          return g < 32 ? a0 : a1;
+        };
+        // every lane takes part in every shuffle (no shuffle under a condition)
+        const int end0 = bag_end(g0), prev0 = bag_end(max(g0 - 1, 0));
+        const int end1 = bag_end(g1), prev1 = bag_end(max(g1 - 1, 0));
+        const int beg0 = g0 > 0 ? prev0 : s, beg1 = g1 > 0 ? prev1 : s;
+        if (p0 < E) {
+          bagpos[p0] = (unsigned)(b0 + g0);
+          mult[p0] = psw ? (double)__ldg(psw + p0) : 1.0 / (double)(end0 - beg0);
+        }
+        if (p1 < E) {
+          bagpos[p1] = (unsigned)(b0 + g1);
+          mult[p1] = psw ? (double)__ldg(psw + p1) : 1.0 / (double)(end1 - beg1);
+        }
       }
     }
   }
@@ -418,25 +446,39 @@ __device__ __forceinline__ void adam_step(float& w, float& m, float& v, float g,
   w = __fsub_rn(w, __fdiv_rn(__fmul_rn(o.lr, mhat), __fadd_rn(__fsqrt_rn(vhat), o.eps)));
 }
 
-// Scalar form for one column j (used by the combine kernel).
-__device__ __forceinline__ void update_col(float* row, int dim, int j, float g, const OptArgs& o,
+// Weight j of a row: fp32, or bf16 widened (wfl < dim).
+__device__ __forceinline__ float load_w(const float* row, int j, bool bf16) {
+  if (!bf16) return row[j];
+  return __uint_as_float((unsigned)reinterpret_cast<const unsigned short*>(row)[j] << 16);
+}
+__device__ __forceinline__ void store_w(float* row, int j, float w, bool bf16) {
+  if (!bf16)
+    row[j] = w;
+  else
+    reinterpret_cast<__nv_bfloat16*>(row)[j] = __float2bfloat16_rn(w);
+}
+
+// Scalar form for one column j (used by the combine kernel); the state
+// starts wfl floats into the row.
+__device__ __forceinline__ void update_col(float* row, int dim, int wfl, int j, float g, const OptArgs& o,
                                            float rowwise_den) {
-  float w = row[j];
+  const bool bf16 = wfl != dim;
+  float w = load_w(row, j, bf16);
   if (o.opt == 0) {
     w = sgd_w(w, g, o.lr);
   } else if (o.opt == 1) {
-    float G = row[dim + j];
+    float G = row[wfl + j];
     adagrad_step(w, G, g, o.lr, o.eps);
-    row[dim + j] = G;
+    row[wfl + j] = G;
   } else if (o.opt == 2) {
-    float m = row[dim + j], v = row[2 * dim + j];
+    float m = row[wfl + j], v = row[wfl + dim + j];
     adam_step(w, m, v, g, o);
-    row[dim + j] = m;
-    row[2 * dim + j] = v;
+    row[wfl + j] = m;
+    row[wfl + dim + j] = v;
   } else {
     w = __fsub_rn(w, __fdiv_rn(__fmul_rn(o.lr, g), rowwise_den));
   }
-  row[j] = w;
+  store_w(row, j, w, bf16);
 }
 
 // ---------------------------------------------------------------------------
@@ -541,13 +583,16 @@ __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wai
 // reads another's data and no barrier is needed) while pair i is added; when
 // a segment starts among the pairs in flight, its table row is prefetched
 // into L2, so the row load at the segment's open mostly hits L2.
-template <int G, int NV, int OPT>
+// EXT: as in bwd_segw_kernel (positions as sort values, bags and factors
+// gathered from bagpos and mult).
+template <int G, int NV, int OPT, bool EXT>
 __global__ void __launch_bounds__(256, NV <= 2 ? DHS_SEG_MINB : 1)
 bwd_seg_kernel(const unsigned* __restrict__ skey, const unsigned* __restrict__ sval, long long n,
                const float* __restrict__ grad, long long n_bags, int dim, RowSpace rs, OptArgs oa,
                double* __restrict__ part_head, double* __restrict__ part_tail,
                int C, unsigned* __restrict__ chunk_ctr,
-               unsigned* __restrict__ owners, unsigned* __restrict__ owner_ctr, DevState* st) {
+               unsigned* __restrict__ owners, unsigned* __restrict__ owner_ctr, DevState* st,
+               const unsigned* __restrict__ bagpos, const double* __restrict__ mult) {
   constexpr int R = seg_ring(NV);
   extern __shared__ float4 seg_ring_smem[];
   const int lane = threadIdx.x & 31;
@@ -599,6 +644,7 @@ bwd_seg_kernel(const unsigned* __restrict__ skey, const unsigned* __restrict__ s
           pws = pf;
           pk = pws + gl < n32 ? __ldg(skey + pws + gl) : 0u;
           pv = pws + gl < n32 ? __ldg(sval + pws + gl) : 0u;
+          if (EXT && pws + gl < n32) pv = __ldg(bagpos + pv);  // position -> bag
         }
         const int t = pf - pws;
         const unsigned b = __shfl_sync(gmask, pv, t, G);
@@ -674,11 +720,13 @@ bwd_seg_kernel(const unsigned* __restrict__ skey, const unsigned* __restrict__ s
     // ---- consumer: pairs in order
     int cws = start - G;
     unsigned ck = 0u;
+    double cm = 0.0;  // EXT: the factor of pair cws + gl
     bool done = false;
     for (int i = start; i < n32; ++i) {
       if (i >= cws + G) {
         cws = i;
         ck = i + gl < n32 ? __ldg(skey + i + gl) : 0u;
+        if (EXT) cm = i + gl < n32 ? __ldg(mult + __ldg(sval + i + gl)) : 0.0;
       }
       const unsigned kt = __shfl_sync(gmask, ck, i - cws, G);
       if (kt != cur) {
@@ -698,14 +746,22 @@ bwd_seg_kernel(const unsigned* __restrict__ skey, const unsigned* __restrict__ s
       }
       cp_async_wait<R - 1>();  // pair i's columns have landed (this lane's own copy)
       const float4* slot = ring + ((i - start) % R) * NV * G;
+      const double f = EXT ? __shfl_sync(gmask, cm, i - cws, G) : 1.0;
       if (mode != 0) {
 #pragma unroll
         for (int q = 0; q < NV; ++q) {
           const float4 x = slot[q * G + gl];
-          acc[q][0] += (double)x.x;
-          acc[q][1] += (double)x.y;
-          acc[q][2] += (double)x.z;
-          acc[q][3] += (double)x.w;
+          if (EXT) {
+            acc[q][0] += (double)x.x * f;
+            acc[q][1] += (double)x.y * f;
+            acc[q][2] += (double)x.z * f;
+            acc[q][3] += (double)x.w * f;
+          } else {
+            acc[q][0] += (double)x.x;
+            acc[q][1] += (double)x.y;
+            acc[q][2] += (double)x.z;
+            acc[q][3] += (double)x.w;
+          }
         }
       }
       produce();  // refill the slot just read with pair i + R
@@ -805,6 +861,53 @@ __device__ __forceinline__ void segw_ld(float (&v)[CPL], const float* p, int col
     }
   }
 }
+// CPL consecutive bf16 weights at element col0 of the row at p, widened to
+// fp32 and back (rounded to nearest even); as segw_ld / segw_st, columns at or
+// past dim are neither read nor written (dim is a multiple of 8).
+template <int CPL>
+__device__ __forceinline__ void segw_ld_bf(float (&v)[CPL], const float* p, int col0, int dim) {
+  const unsigned short* h = reinterpret_cast<const unsigned short*>(p) + col0;
+  if constexpr (CPL == 1) {
+    v[0] = __uint_as_float((unsigned)h[0] << 16);
+  } else if constexpr (CPL == 2) {
+    const unsigned u = *reinterpret_cast<const unsigned*>(h);
+    v[0] = bf16_lo(u);
+    v[1] = bf16_hi(u);
+  } else if constexpr (CPL == 4) {
+    const uint2 u = *reinterpret_cast<const uint2*>(h);
+    v[0] = bf16_lo(u.x); v[1] = bf16_hi(u.x); v[2] = bf16_lo(u.y); v[3] = bf16_hi(u.y);
+  } else {
+#pragma unroll
+    for (int k = 0; k < CPL / 8; ++k) {
+      if (col0 + 8 * k < dim) {
+        const uint4 u = *reinterpret_cast<const uint4*>(h + 8 * k);
+        v[8 * k + 0] = bf16_lo(u.x); v[8 * k + 1] = bf16_hi(u.x);
+        v[8 * k + 2] = bf16_lo(u.y); v[8 * k + 3] = bf16_hi(u.y);
+        v[8 * k + 4] = bf16_lo(u.z); v[8 * k + 5] = bf16_hi(u.z);
+        v[8 * k + 6] = bf16_lo(u.w); v[8 * k + 7] = bf16_hi(u.w);
+      }
+    }
+  }
+}
+template <int CPL>
+__device__ __forceinline__ void segw_st_bf(float* p, const float (&v)[CPL], int col0, int dim) {
+  unsigned short* h = reinterpret_cast<unsigned short*>(p) + col0;
+  if constexpr (CPL == 1) {
+    *reinterpret_cast<__nv_bfloat16*>(h) = __float2bfloat16_rn(v[0]);
+  } else if constexpr (CPL == 2) {
+    *reinterpret_cast<unsigned*>(h) = pack_bf16x2(v[0], v[1]);
+  } else if constexpr (CPL == 4) {
+    *reinterpret_cast<uint2*>(h) = make_uint2(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]));
+  } else {
+#pragma unroll
+    for (int k = 0; k < CPL / 8; ++k)
+      if (col0 + 8 * k < dim)
+        *reinterpret_cast<uint4*>(h + 8 * k) =
+            make_uint4(pack_bf16x2(v[8 * k], v[8 * k + 1]), pack_bf16x2(v[8 * k + 2], v[8 * k + 3]),
+                       pack_bf16x2(v[8 * k + 4], v[8 * k + 5]), pack_bf16x2(v[8 * k + 6], v[8 * k + 7]));
+  }
+}
+
 template <int CPL>
 __device__ __forceinline__ void segw_st(float* p, const float (&v)[CPL], int col0, int dim) {
   if constexpr (CPL == 1) {
@@ -820,13 +923,19 @@ __device__ __forceinline__ void segw_st(float* p, const float (&v)[CPL], int col
   }
 }
 
-template <int CPL, int OPT>
+// EXT (extended pooling): sort values are positions; the pair's bag is
+// bagpos[position] and its gradient row is scaled by mult[position] (a
+// per-sample weight, or 1 / the bag's length), both gathered once per chunk.
+// BF: the table's weights are bf16 (state fp32): loaded widened, updated in
+// fp32, stored rounded to nearest even.
+template <int CPL, int OPT, bool EXT, bool BF>
 __global__ void __launch_bounds__(256, CPL <= 4 ? 3 : 1)
 bwd_segw_kernel(const unsigned* __restrict__ skey, const unsigned* __restrict__ sval, long long n,
                 const float* __restrict__ grad, long long n_bags, int dim, RowSpace rs, OptArgs oa,
                 double* __restrict__ part_head, double* __restrict__ part_tail, int pstride, int C,
                 unsigned* __restrict__ chunk_ctr, unsigned* __restrict__ owners,
-                unsigned* __restrict__ owner_ctr, DevState* st, bool grad_once) {
+                unsigned* __restrict__ owner_ctr, DevState* st, bool grad_once,
+                const unsigned* __restrict__ bagpos, const double* __restrict__ mult) {
   constexpr int B = segw_batch(CPL);
   constexpr int PITCH = 32 * CPL;  // floats per staged row
   constexpr int NS = seg_state_arrays(OPT);
@@ -834,6 +943,7 @@ bwd_segw_kernel(const unsigned* __restrict__ skey, const unsigned* __restrict__ 
   extern __shared__ __align__(128) float segw_smem[];
   __shared__ __align__(8) unsigned long long segw_bar[8][2];
   __shared__ uint2 segw_runs[8][130];  // per warp: the stream's runs {key, start | mode << 16}
+  __shared__ double segw_mult[EXT ? 8 : 1][EXT ? 128 : 1];  // per warp: each pair's factor
   const int lane = threadIdx.x & 31;
   const int wid = threadIdx.x >> 5;
   const int col0 = lane * CPL;
@@ -875,6 +985,18 @@ bwd_segw_kernel(const unsigned* __restrict__ skey, const unsigned* __restrict__ 
       const bool in = p < limit;
       kw[w] = in ? __ldg(skey + p) : ~0u;
       vw[w] = in ? __ldg(sval + p) : 0u;
+    }
+    if constexpr (EXT) {
+      // positions -> bags, and each pair's factor into this warp's list (the
+      // previous chunk's readers passed the warp-wide shuffle at the loop top)
+#pragma unroll
+      for (int w = 0; w < 4; ++w) {
+        const bool in = start + 32 * w + lane < limit;
+        const unsigned pos = vw[w];
+        segw_mult[wid][32 * w + lane] = in ? __ldg(mult + pos) : 0.0;
+        vw[w] = in ? __ldg(bagpos + pos) : 0u;
+      }
+      __syncwarp();
     }
     const unsigned prev = start > 0 ? __ldg(skey + start - 1) : ~0u;
     const unsigned back2 = c >= 2 ? __ldg(skey + (c - 1) * C - 1) : ~0u;
@@ -1018,15 +1140,19 @@ bwd_segw_kernel(const unsigned* __restrict__ skey, const unsigned* __restrict__ 
     float nw[CPL];
     float nst[NS > 0 ? NS : 1][CPL];
     float nra = 0.f;
+    const int wfl = rs.wfl;  // the state starts wfl floats into the row
     auto fetch = [&](uint2 e) {
       if ((e.y >> 16) == 2u && e.x < nrows) {
         const float* row = rs.row(e.x);
         if (lane_on) {
-          segw_ld<CPL>(nw, row, col0, dim);
+          if constexpr (BF)
+            segw_ld_bf<CPL>(nw, row, col0, dim);
+          else
+            segw_ld<CPL>(nw, row, col0, dim);
 #pragma unroll
-          for (int k = 0; k < NS; ++k) segw_ld<CPL>(nst[k], row + (k + 1) * dim, col0, dim);
+          for (int k = 0; k < NS; ++k) segw_ld<CPL>(nst[k], row + wfl + k * dim, col0, dim);
         }
-        if (OPT == 3) nra = row[dim];
+        if (OPT == 3) nra = row[wfl];
       }
     };
     auto close = [&]() {
@@ -1073,11 +1199,14 @@ bwd_segw_kernel(const unsigned* __restrict__ skey, const unsigned* __restrict__ 
               rw[e] = __fsub_rn(rw[e], __fdiv_rn(__fmul_rn(oa.lr, g), den));
             }
           }
-          segw_st<CPL>(row, rw, col0, dim);
+          if constexpr (BF)
+            segw_st_bf<CPL>(row, rw, col0, dim);
+          else
+            segw_st<CPL>(row, rw, col0, dim);
 #pragma unroll
-          for (int k = 0; k < NS; ++k) segw_st<CPL>(row + (k + 1) * dim, rst[k], col0, dim);
+          for (int k = 0; k < NS; ++k) segw_st<CPL>(row + wfl + k * dim, rst[k], col0, dim);
         }
-        if (OPT == 3 && lane == 0) row[dim] = Gn;
+        if (OPT == 3 && lane == 0) row[wfl] = Gn;
       }
 #pragma unroll
       for (int e = 0; e < CPL; ++e) acc[e] = 0.0;
@@ -1144,8 +1273,14 @@ bwd_segw_kernel(const unsigned* __restrict__ skey, const unsigned* __restrict__ 
 #pragma unroll
               for (int e = 0; e < CPL; ++e) x[e] = 0.f;
               segw_ld<CPL>(x, rows + i * PITCH, 0, dim - col0);
+              if constexpr (EXT) {
+                const double f = segw_mult[wid][q];
 #pragma unroll
-              for (int e = 0; e < CPL; ++e) acc[e] += (double)x[e];
+                for (int e = 0; e < CPL; ++e) acc[e] += (double)x[e] * f;
+              } else {
+#pragma unroll
+                for (int e = 0; e < CPL; ++e) acc[e] += (double)x[e];
+              }
             }
           }
         } else {
@@ -1170,15 +1305,63 @@ bwd_segw_kernel(const unsigned* __restrict__ skey, const unsigned* __restrict__ 
 // segment's last pair (the first pairs of the run's chunks all carry the key;
 // keys are sorted, so a 32-way search over chunk starts finds the last one),
 // cuts the run's pieces (the owner's starting partial, then one head piece
-// per following chunk) into batches of kCombinePieces and takes batch ids
-// (and, for runs of more than one batch, fp64 slots) from counters.
+// per following chunk) into batches of about sqrt(pieces) each and takes
+// batch ids (and, for runs of more than one batch, fp64 slots) from counters.
 // Combine: one block per batch adds its pieces in fp64; a one-batch run
 // updates its row directly, otherwise the batch stores its sum in its slot and
 // the last of the run's batches to finish (an atomic ticket; no block waits)
 // adds the slots in batch order and applies the optimizer once.  Every sum is
-// taken in an order fixed by the run alone.
-constexpr int kCombineThreads = 128;
-constexpr int kCombinePieces = 128;
+// taken in an order fixed by the run alone.  With batches of about sqrt(pieces)
+// both the batch sums and the final sum over the slots are short chains of
+// loads, for a run of a few hundred pieces as for one of tens of thousands.
+constexpr int kCombineThreads = 256;
+constexpr int kCombineMinPieces = 16;
+
+// Pieces per batch of a run of npieces pieces: the smallest power of two of
+// at least kCombineMinPieces whose square reaches npieces.
+__host__ __device__ inline unsigned combine_batch_pieces(long long npieces) {
+  unsigned p = kCombineMinPieces;
+  while ((long long)p * p < npieces) p <<= 1;
+  return p;
+}
+
+// Runs of at most this many pieces are finished by the plan kernel's warp.
+constexpr int kWarpFinishPieces = 16;
+
+// One warp finishes a run of npieces pieces: piece 0 at first, piece k >= 1
+// at rest + (k - 1) * pstride; lane l owns columns l + 32 i (dim <= 512).
+__device__ __forceinline__ void finish_run_warp(float* row, int dim, int wfl, const OptArgs& oa,
+                                                const double* first, const double* rest, int pstride,
+                                                long long npieces, int lane) {
+  constexpr int kCols = 16;  // columns per lane at dim 512
+  float g[kCols];
+  double sq = 0.0;
+#pragma unroll
+  for (int i = 0; i < kCols; ++i) {
+    const int j = lane + 32 * i;
+    g[i] = 0.f;
+    if (j < dim) {
+      double a = __ldcg(first + j);
+      for (long long k = 1; k < npieces; ++k) a += __ldcg(rest + (k - 1) * pstride + j);
+      g[i] = (float)a;
+      const double gd = (double)g[i];
+      sq += gd * gd;
+    }
+  }
+  float den = 0.f, Gn = 0.f;
+  if (oa.opt == 3) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
+    Gn = __fadd_rn(row[wfl], (float)(sq / (double)dim));
+    den = __fadd_rn(__fsqrt_rn(Gn), oa.eps);
+  }
+#pragma unroll
+  for (int i = 0; i < kCols; ++i) {
+    const int j = lane + 32 * i;
+    if (j < dim) update_col(row, dim, wfl, j, g[i], oa, den);
+  }
+  if (oa.opt == 3 && lane == 0) row[wfl] = Gn;
+}
 
 struct CombinePlan {
   unsigned* key;          // [owners] row of the run
@@ -1186,6 +1369,7 @@ struct CombinePlan {
   unsigned* boff;         // [owners] first batch id
   unsigned* sbase;        // [owners] first slot (runs of more than one batch)
   unsigned* ticket;       // [owners] batches finished
+  unsigned* ppb;          // [owners] pieces per batch
   unsigned* batch_owner;  // [batch_cap] owner of each batch id
   double* slots;          // [slot_cap][pstride]
   unsigned batch_cap, slot_cap;
@@ -1197,7 +1381,9 @@ struct CombinePlan {
 __global__ void __launch_bounds__(256)
 bwd_combine_plan_kernel(const unsigned* __restrict__ skey, long long n, int C,
                         const unsigned* __restrict__ owners, const unsigned* __restrict__ owner_ctr,
-                        CombinePlan pl, DevState* st) {
+                        CombinePlan pl, int dim, RowSpace rs, OptArgs oa,
+                        const double* __restrict__ part_head, const double* __restrict__ part_tail,
+                        int pstride, DevState* st) {
   const int lane = threadIdx.x & 31;
   const long long nchunks = (n + C - 1) / C;
   const unsigned long long nrows = st->row_count;
@@ -1219,7 +1405,16 @@ bwd_combine_plan_kernel(const unsigned* __restrict__ skey, long long n, int C,
       if (stride == 1) break;
     }
     const long long npieces = lo - c + 1;
-    const unsigned nb = key < nrows ? (unsigned)((npieces + kCombinePieces - 1) / kCombinePieces) : 0u;
+    const unsigned P = combine_batch_pieces(npieces);
+    unsigned nb = key < nrows ? (unsigned)((npieces + P - 1) / P) : 0u;
+    if (key < nrows && npieces <= kWarpFinishPieces) {
+      // a short run is finished here by this warp: lane l sums columns l,
+      // l + 32, ... over the pieces in order (piece 0 = the owner's starting
+      // partial), then applies the optimizer; no batch is planned for it
+      finish_run_warp(rs.row(key), dim, rs.wfl, oa, part_tail + c * (long long)pstride,
+                      part_head + (c + 1) * (long long)pstride, pstride, npieces, lane);
+      nb = 0;
+    }
     unsigned base = 0, sb = 0;
     if (lane == 0) {
       base = atomicAdd(pl.batch_ctr, nb);
@@ -1233,13 +1428,14 @@ bwd_combine_plan_kernel(const unsigned* __restrict__ skey, long long n, int C,
       pl.boff[oi] = base;
       pl.sbase[oi] = sb;
       pl.ticket[oi] = 0u;
+      pl.ppb[oi] = P;
     }
     base = __shfl_sync(0xffffffffu, base, 0);
     for (unsigned j = lane; j < nb && base + j < pl.batch_cap; j += 32) pl.batch_owner[base + j] = (unsigned)oi;
   }
 }
 
-__global__ void __launch_bounds__(kCombineThreads, 8)
+__global__ void __launch_bounds__(kCombineThreads, 4)
 bwd_combine_kernel(const unsigned* __restrict__ skey, int dim, RowSpace rs, OptArgs oa,
                    const double* __restrict__ part_head, const double* __restrict__ part_tail, int C,
                    int pstride, const unsigned* __restrict__ owners,
@@ -1258,20 +1454,23 @@ bwd_combine_kernel(const unsigned* __restrict__ skey, int dim, RowSpace rs, OptA
     const unsigned key = pl.key[oi];
     const long long npieces = (long long)pl.kend[oi] - c + 1;
     const unsigned b = bid - pl.boff[oi];
-    const unsigned nb = (unsigned)((npieces + kCombinePieces - 1) / kCombinePieces);
+    const unsigned P = pl.ppb[oi];
+    const unsigned nb = (unsigned)((npieces + P - 1) / P);
     if (b >= nb) continue;
     // the plan gives no batch to a missing-key run; this thread's column of
     // the row (rows of at most T floats) is loaded while the pieces are summed
     float* const row = rs.row(key);
+    const int wfl = rs.wfl;
+    const bool bf16 = wfl != dim;
     const bool pre = dim <= T && (int)threadIdx.x < dim;
     float pw = 0.f, ps0 = 0.f, ps1 = 0.f;
     if (pre) {
-      pw = row[threadIdx.x];
-      if (oa.opt == 1 || oa.opt == 2) ps0 = row[dim + threadIdx.x];
-      if (oa.opt == 2) ps1 = row[2 * dim + threadIdx.x];
+      pw = load_w(row, threadIdx.x, bf16);
+      if (oa.opt == 1 || oa.opt == 2) ps0 = row[wfl + threadIdx.x];
+      if (oa.opt == 2) ps1 = row[wfl + dim + threadIdx.x];
     }
-    const long long p0 = (long long)b * kCombinePieces;
-    const long long p1 = min(npieces, p0 + kCombinePieces);
+    const long long p0 = (long long)b * P;
+    const long long p1 = min(npieces, p0 + (long long)P);
     // slice sl adds pieces p0 + sl, p0 + sl + slices, ... (piece 0 = starting partial)
     for (int j0 = 0; j0 < dim; j0 += (slices == 1 ? T : dim)) {
       const int sl = slices == 1 ? 0 : threadIdx.x / dim;
@@ -1328,10 +1527,10 @@ bwd_combine_kernel(const unsigned* __restrict__ skey, int dim, RowSpace rs, OptA
         s_sq = sq;
       }
       __syncthreads();
-      const float Gn = __fadd_rn(row[dim], (float)(s_sq / (double)dim));
+      const float Gn = __fadd_rn(row[wfl], (float)(s_sq / (double)dim));
       den = __fadd_rn(__fsqrt_rn(Gn), oa.eps);
       __syncthreads();
-      if (threadIdx.x == 0) row[dim] = Gn;
+      if (threadIdx.x == 0) row[wfl] = Gn;
     }
     if (dim <= T) {
       if (pre) {
@@ -1341,18 +1540,18 @@ bwd_combine_kernel(const unsigned* __restrict__ skey, int dim, RowSpace rs, OptA
           pw = sgd_w(pw, g, oa.lr);
         } else if (oa.opt == 1) {
           adagrad_step(pw, ps0, g, oa.lr, oa.eps);
-          row[dim + j] = ps0;
+          row[wfl + j] = ps0;
         } else if (oa.opt == 2) {
           adam_step(pw, ps0, ps1, g, oa);
-          row[dim + j] = ps0;
-          row[2 * dim + j] = ps1;
+          row[wfl + j] = ps0;
+          row[wfl + dim + j] = ps1;
         } else {
           pw = __fsub_rn(pw, __fdiv_rn(__fmul_rn(oa.lr, g), den));
         }
-        row[j] = pw;
+        store_w(row, j, pw, bf16);
       }
     } else {
-      for (int j = threadIdx.x; j < dim; j += T) update_col(row, dim, j, (float)sacc[j], oa, den);
+      for (int j = threadIdx.x; j < dim; j += T) update_col(row, dim, wfl, j, (float)sacc[j], oa, den);
     }
     __syncthreads();
   }

@@ -12,7 +12,9 @@
 #include <cmath>
 #include <cstdint>
 #include <cstring>
+#include <map>
 #include <mutex>
+#include <tuple>
 #include <new>
 #include <vector>
 
@@ -23,6 +25,31 @@
 #include "dhs_launch.h"
 
 using namespace dhs;
+
+namespace dhs {
+
+int blocks_per_sm(const void* kernel, int threads, size_t smem) {
+  static std::mutex mu;
+  static std::map<std::tuple<const void*, int, int, size_t>, int> cache;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  const auto key = std::make_tuple(kernel, dev, threads, smem);
+  std::lock_guard<std::mutex> lock(mu);
+  const auto it = cache.find(key);
+  if (it != cache.end()) return it->second;
+  // opt in to the dynamic size asked for: static + dynamic shared memory above
+  // 48 KB needs it even when the dynamic part alone is below
+  if (smem > 0) cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, threads, smem) != cudaSuccess || per_sm < 1) {
+    cudaGetLastError();
+    per_sm = 1;
+  }
+  cache.emplace(key, per_sm);
+  return per_sm;
+}
+
+}  // namespace dhs
 
 namespace {
 
@@ -45,7 +72,7 @@ enum { PH_FWD_POOL = 0, PH_FWD_ASSIGN = 1, PH_BWD_PROBE = 2, PH_BWD_SORT = 3, PH
 
 struct Snap {
   cudaEvent_t ev = nullptr;
-  unsigned long long* pinned = nullptr;  // row_count copied here
+  unsigned long long* pinned = nullptr;  // row_count, keys_used copied here
   long long cum_n = 0;                   // inserted-key upper bound counter at record time
   bool valid = false;
 };
@@ -100,6 +127,8 @@ struct dhs_table {
   int device = 0;
   int sm_count = 148;
   int dim = 0, opt = 0, stride = 0;
+  int wfl = 0;          // floats per row holding the weights (dim, or dim / 2 for bf16 weights)
+  bool wbf16 = false;   // weights stored as bf16
   float eps = 1e-8f, b1 = 0.9f, b2 = 0.999f;
   long long adam_t = 0;
   long long block_rows = kDefaultBlockRows;
@@ -125,6 +154,22 @@ struct dhs_table {
 
   // upper bound on the device row count after all enqueued work
   long long rows_ub = 0;
+  // with hooks: upper bound on the IDMap slots in use (keys with or without a
+  // row, and tombstones until the next rehash)
+  long long keys_ub = 0;
+
+  // admission / eviction (ht_set_hooks)
+  bool has_hooks_set = false;
+  unsigned admit = 1;
+  bool track = false;
+  long long step = 0;          // insert calls so far
+  unsigned* cnt = nullptr;     // [nslots]
+  unsigned* stamp = nullptr;   // [nslots]
+  unsigned* free_bm = nullptr; // bit per row
+  long long free_words = 0;
+  unsigned* free_list = nullptr;
+  long long free_list_cap = 0;
+  Buf b_fcnt, b_freed;
   long long cum_n = 0;  // sum of key counts of all insert calls
   Snap snaps[kSnapRing];
   int snap_next = 0;
@@ -133,7 +178,7 @@ struct dhs_table {
   long long ws_n = -1;
   long long ws_chunks = 0;  // chunk capacity of the segment and combine buffers
   Buf b_nbm, b_fbm, b_gcnt, b_gpref, b_slotpos, b_ka, b_va, b_kb, b_vb, b_hist, b_totals, b_ph,
-      b_pt, b_owners, b_cplan, b_slots, b_refs;
+      b_pt, b_owners, b_cplan, b_slots, b_refs, b_bagpos, b_mult;
 
   bool timing = false;
   std::vector<PhaseRec> recs;
@@ -193,6 +238,8 @@ void bfree(dhs_table* t, Buf& b, cudaStream_t s) {
   b.bytes = 0;
 }
 
+size_t block_bytes(const dhs_table* t) { return (size_t)t->block_rows * t->stride * sizeof(float); }
+
 struct DeviceGuard {
   int prev = -1;
   explicit DeviceGuard(int dev) {
@@ -230,7 +277,14 @@ dhs_status last_launch() {
 IdMap idmap(const dhs_table* t) { return IdMap{t->slots, t->nslots / 2 - 1}; }
 
 RowSpace rowspace(const dhs_table* t) {
-  return RowSpace{t->blocks_d, (unsigned long long)t->block_rows - 1, t->log2_br, t->stride};
+  return RowSpace{t->blocks_d, (unsigned long long)t->block_rows - 1, t->log2_br, t->stride, t->wfl};
+}
+
+bool has_hooks(const dhs_table* t) { return t->admit > 1 || t->track; }
+
+Hooks hooks(const dhs_table* t) {
+  return Hooks{t->admit > 1 ? t->cnt : nullptr, t->track ? t->stamp : nullptr, t->admit, (unsigned)t->step,
+               t->free_list, t->free_bm};
 }
 
 // ---- phase timing ----
@@ -268,13 +322,7 @@ struct PhaseScope {
 // ---- grid sizing ----
 template <typename K>
 int resident_blocks(K kernel, int threads, size_t smem, int sm_count) {
-  int per_sm = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, threads, smem) != cudaSuccess ||
-      per_sm < 1) {
-    cudaGetLastError();
-    per_sm = 1;
-  }
-  return per_sm * sm_count;
+  return blocks_per_sm((const void*)kernel, threads, smem) * sm_count;
 }
 
 long long grid_for(long long units_per_block_needed, int resident) {
@@ -292,8 +340,10 @@ void refresh_ub(dhs_table* t, bool wait) {
     if (!sn.valid) continue;
     cudaError_t q = wait && i == 0 ? host_wait(t, sn.ev) : cudaEventQuery(sn.ev);
     if (q == cudaSuccess) {
-      const long long ub = (long long)*sn.pinned + (t->cum_n - sn.cum_n);
+      const long long ub = (long long)sn.pinned[0] + (t->cum_n - sn.cum_n);
       if (ub < t->rows_ub) t->rows_ub = ub;
+      const long long kb = (long long)sn.pinned[1] + (t->cum_n - sn.cum_n);
+      if (kb < t->keys_ub) t->keys_ub = kb;
       return;
     }
     cudaGetLastError();
@@ -303,7 +353,8 @@ void refresh_ub(dhs_table* t, bool wait) {
 void record_snapshot(dhs_table* t, cudaStream_t s) {
   Snap& sn = t->snaps[t->snap_next];
   if (sn.valid) host_wait(t, sn.ev);  // ring slot reuse: at most kSnapRing in flight
-  cudaMemcpyAsync(sn.pinned, &t->st->row_count, sizeof(unsigned long long), cudaMemcpyDeviceToHost, s);
+  // row_count and keys_used are adjacent
+  cudaMemcpyAsync(sn.pinned, &t->st->row_count, 2 * sizeof(unsigned long long), cudaMemcpyDeviceToHost, s);
   cudaEventRecord(sn.ev, s);
   sn.cum_n = t->cum_n;
   sn.valid = true;
@@ -320,50 +371,69 @@ dhs_status grow_map(dhs_table* t, unsigned long long want_slots, cudaStream_t s)
   PhaseScope ph(t, PH_GROW, s);
   unsigned long long ns = std::max<unsigned long long>(t->nslots * 2, kInitialSlots);
   while (ns < want_slots) ns <<= 1;
+  const int thr = 256;
   Slot* fresh = (Slot*)dalloc(t, ns * sizeof(Slot), s);
   if (!fresh) return DHS_ERR_OOM;
-  const int thr = 256;
   const long long g = std::min<long long>((long long)((ns + thr - 1) / thr), (long long)t->sm_count * 16);
   fill_empty_kernel<<<(unsigned)g, thr, 0, s>>>(fresh, ns);
   t->n_launches++;
+  // per-slot counts and stamps of the new map (hooks), zero until the rehash
+  // moves the keys' values over
+  unsigned* ncnt = nullptr;
+  unsigned* nstamp = nullptr;
+  if (t->cnt) {
+    ncnt = (unsigned*)dalloc(t, ns * 4, s);
+    if (!ncnt) return DHS_ERR_OOM;
+    DHS_CUDA(cudaMemsetAsync(ncnt, 0, ns * 4, s));
+  }
+  if (t->stamp) {
+    nstamp = (unsigned*)dalloc(t, ns * 4, s);
+    if (!nstamp) return DHS_ERR_OOM;
+    DHS_CUDA(cudaMemsetAsync(nstamp, 0, ns * 4, s));
+  }
   if (t->slots) {
     IdMap to{fresh, ns / 2 - 1};
+    if (has_hooks(t)) DHS_CUDA(cudaMemsetAsync(&t->st->keys_used, 0, sizeof(unsigned long long), s));
     const long long g2 = std::min<long long>((long long)((t->nslots + thr - 1) / thr), (long long)t->sm_count * 16);
-    rehash_kernel<<<(unsigned)g2, thr, 0, s>>>(t->slots, t->nslots, to, t->st);
+    rehash_kernel<<<(unsigned)g2, thr, 0, s>>>(t->slots, t->nslots, to, t->cnt, ncnt, t->stamp, nstamp, t->st);
     t->n_launches++;
     dfree(t, t->slots, t->nslots * sizeof(Slot), s);
     t->n_rehash++;
   }
+  if (t->cnt) dfree(t, t->cnt, t->nslots * 4, s);
+  if (t->stamp) dfree(t, t->stamp, t->nslots * 4, s);
+  t->cnt = ncnt;
+  t->stamp = nstamp;
   t->slots = fresh;
   t->nslots = ns;
   return last_launch();
 }
 
 // Make room for up to `n` new keys: IDMap load <= kMaxLoad and blocks
-// covering the row upper bound.
+// covering the row upper bound.  The bound is the newest row-count snapshot
+// that has finished plus every key of the insert calls enqueued since.  When
+// that bound says the table might have to grow (or cross max_rows), the host
+// first waits for the newest snapshot (the previous insert call's row count)
+// and grows only if the tightened bound still needs it: growth, which maps
+// fresh device memory, happens only for rows that can really arrive.
 dhs_status ensure_capacity(dhs_table* t, long long n, cudaStream_t s) {
   refresh_ub(t, false);
   long long need = t->rows_ub + n;
-  if (need > t->max_rows) {
+  // slots: with hooks, keys without a row and tombstones take slots too
+  long long need_slots = has_hooks(t) ? t->keys_ub + n : need;
+  const long long have_rows = (long long)t->blocks_h.size() * t->block_rows;
+  if (need > t->max_rows || (double)need_slots > kMaxLoad * (double)t->nslots || need > have_rows) {
     refresh_ub(t, true);
     need = t->rows_ub + n;
+    need_slots = has_hooks(t) ? t->keys_ub + n : need;
     if (need > t->max_rows) return DHS_ERR_TABLE_FULL;
   }
-  if ((double)need > kMaxLoad * (double)t->nslots) {
-    refresh_ub(t, true);
-    need = t->rows_ub + n;
-    if ((double)need > kMaxLoad * (double)t->nslots)
-      DHS_TRY(grow_map(t, (unsigned long long)std::ceil((double)need / kMaxLoad), s));
-  }
+  if ((double)need_slots > kMaxLoad * (double)t->nslots)
+    DHS_TRY(grow_map(t, (unsigned long long)std::ceil((double)need_slots / kMaxLoad), s));
   long long have = (long long)t->blocks_h.size() * t->block_rows;
-  if (need > have) {
-    refresh_ub(t, true);
-    need = t->rows_ub + n;
-  }
   while (need > have) {
     if ((long long)t->blocks_h.size() >= t->max_blocks) return DHS_ERR_TABLE_FULL;
-    const size_t bytes = (size_t)t->block_rows * t->stride * sizeof(float);
-    float* b = (float*)dalloc(t, bytes, s);
+    float* b = (float*)dalloc(t, block_bytes(t), s);
     if (!b) return DHS_ERR_OOM;
     t->blocks_h.push_back(b);
     set_block_kernel<<<1, 1, 0, s>>>(t->blocks_d, (long long)t->blocks_h.size() - 1, b, t->st,
@@ -379,13 +449,15 @@ dhs_status ensure_capacity(dhs_table* t, long long n, cudaStream_t s) {
 // Owner chunks are at least two apart (a long segment reaches two chunks past
 // its owner), so there are at most nchunks / 2 + 1 of them; the runs overlap
 // in at most one chunk, so their pieces add up to at most 1.5 nchunks + 1.
-// Batch ids: one per run plus pieces / kCombinePieces.  Slots: only runs of
-// more than kCombinePieces pieces take them, fewer than two per
-// kCombinePieces of their pieces.
-constexpr long long combine_batch_cap(long long nchunks) { return nchunks / 2 + 2 * nchunks / kCombinePieces + 64; }
-constexpr long long combine_slot_cap(long long nchunks) { return 4 * nchunks / kCombinePieces + 64; }
+// A run of n pieces gets ceil(n / P) batches, P >= kCombineMinPieces: batch
+// ids are at most one per run plus pieces / kCombineMinPieces.  Slots: only
+// runs of more than one batch take them (n > P), fewer than 2 n / P each.
+constexpr long long combine_batch_cap(long long nchunks) {
+  return nchunks / 2 + 2 * nchunks / kCombineMinPieces + 64;
+}
+constexpr long long combine_slot_cap(long long nchunks) { return 4 * nchunks / kCombineMinPieces + 64; }
 
-// The plan arrays cut from one buffer of 5 nchunks + batch cap words.
+// The plan arrays cut from one buffer of 6 nchunks + batch cap words.
 CombinePlan combine_plan(unsigned* words, double* slots, long long nchunks, unsigned* zeroed) {
   CombinePlan pl;
   pl.key = words;
@@ -393,7 +465,8 @@ CombinePlan combine_plan(unsigned* words, double* slots, long long nchunks, unsi
   pl.boff = words + 2 * nchunks;
   pl.sbase = words + 3 * nchunks;
   pl.ticket = words + 4 * nchunks;
-  pl.batch_owner = words + 5 * nchunks;
+  pl.ppb = words + 5 * nchunks;
+  pl.batch_owner = words + 6 * nchunks;
   pl.slots = slots;
   pl.batch_cap = (unsigned)combine_batch_cap(nchunks);
   pl.slot_cap = (unsigned)combine_slot_cap(nchunks);
@@ -428,7 +501,7 @@ dhs_status ensure_ws(dhs_table* t, long long n, cudaStream_t s) {
   DHS_TRY(bget(t, t->b_ph, (size_t)nchunks * pstride * 8, s));
   DHS_TRY(bget(t, t->b_pt, (size_t)nchunks * pstride * 8, s));
   DHS_TRY(bget(t, t->b_owners, nchunks * 4, s));
-  DHS_TRY(bget(t, t->b_cplan, (size_t)(5 * nchunks + combine_batch_cap(nchunks)) * 4, s));
+  DHS_TRY(bget(t, t->b_cplan, (size_t)(6 * nchunks + combine_batch_cap(nchunks)) * 4, s));
   DHS_TRY(bget(t, t->b_slots, (size_t)combine_slot_cap(nchunks) * pstride * 8, s));
   DHS_CUDA(cudaMemsetAsync(t->b_nbm.p, 0, t->b_nbm.bytes, s));
   t->ws_n = cap;
@@ -436,7 +509,18 @@ dhs_status ensure_ws(dhs_table* t, long long n, cudaStream_t s) {
   return DHS_OK;
 }
 
+// The per-position bag and factor arrays of an extended-pooling backward
+// (allocated on first use, sized like the rest of the workspace).
+dhs_status ensure_ws_ext(dhs_table* t, cudaStream_t s) {
+  DHS_TRY(bget(t, t->b_bagpos, (size_t)t->ws_n * 4, s));
+  return bget(t, t->b_mult, (size_t)t->ws_n * 8, s);
+}
+
 dhs_status check_table(const dhs_table* t) { return t ? DHS_OK : DHS_ERR_INVALID_ARG; }
+
+// Floats per row as ht_get_rows / ht_export return it: dim weights (widened
+// from bf16 where stored so) followed by the fp32 state.
+int export_stride(const dhs_table* t) { return t->dim + (t->stride - t->wfl); }
 
 // Plan and combine launches for the long segments of one backward.
 dhs_status launch_combine(dhs_table* t, const unsigned* skey, long long n, const OptArgs& oa,
@@ -444,12 +528,12 @@ dhs_status launch_combine(dhs_table* t, const unsigned* skey, long long n, const
                           const unsigned* owners, unsigned* zeroed, const CombinePlan& pl,
                           cudaStream_t s) {
   const unsigned* owner_ctr = zeroed + kSegOwnerCtrWord;
-  bwd_combine_plan_kernel<<<(unsigned)t->sm_count * 2, 256, 0, s>>>(skey, n, chunk, owners, owner_ctr, pl,
-                                                                    t->st);
+  bwd_combine_plan_kernel<<<(unsigned)t->sm_count * 2, 256, 0, s>>>(
+      skey, n, chunk, owners, owner_ctr, pl, t->dim, rowspace(t), oa, part_head, part_tail, pstride, t->st);
   t->n_launches++;
   DHS_TRY(last_launch());
   const size_t smem = (size_t)std::max(kCombineThreads, t->dim) * sizeof(double);
-  bwd_combine_kernel<<<(unsigned)t->sm_count * 16, kCombineThreads, smem, s>>>(
+  bwd_combine_kernel<<<(unsigned)t->sm_count * 8, kCombineThreads, smem, s>>>(
       skey, t->dim, rowspace(t), oa, part_head, part_tail, chunk, pstride, owners, owner_ctr, pl);
   t->n_launches++;
   return last_launch();
@@ -457,11 +541,15 @@ dhs_status launch_combine(dhs_table* t, const unsigned* skey, long long n, const
 
 // ---- kernel dispatch on the row width ----
 dhs_status dispatch_pool(dhs_table* t, const long long* keys, long long n, const long long* bo,
-                         long long nb, float* out, cudaStream_t s) {
-  const int G = pick_group(t->dim), NV = pick_nv(t->dim, G);
-  const cudaError_t e = launch_probe_pool(G, NV, t->sm_count, idmap(t), rowspace(t), t->dim, keys, n,
-                                          bo, nb, out, (unsigned*)t->b_nbm.p,
-                                          (unsigned*)t->b_slotpos.p, t->st, s);
+                         long long nb, const float* psw, bool mean, float* out, cudaStream_t s) {
+  // a lane's 16-byte unit holds 4 fp32 or 8 bf16 weights
+  const int wd = t->wbf16 ? t->dim / 2 : t->dim;
+  const int G = pick_group(wd), NV = pick_nv(wd, G);
+  const cudaError_t e =
+      (t->wbf16 ? launch_probe_pool_bf16 : launch_probe_pool)(G, NV, t->sm_count, idmap(t), rowspace(t), t->dim,
+                                                              keys, n, bo, nb, psw, mean, out,
+                                                              (unsigned*)t->b_nbm.p, (unsigned*)t->b_slotpos.p,
+                                                              t->st, s);
   t->n_launches++;
   if (e != cudaSuccess) cudaGetLastError();
   return e == cudaSuccess ? DHS_OK : DHS_ERR_CUDA;
@@ -479,26 +567,29 @@ int segw_cpl(int dim) {
   return c;
 }
 
+// bagpos / mult non-null: extended pooling (sort values are positions).
 dhs_status launch_seg(dhs_table* t, const unsigned* sk, const unsigned* sv, long long n, const float* grad,
                       long long nb, const OptArgs& oa, double* part_head, double* part_tail,
-                      unsigned* chunk_ctr, unsigned* owners, unsigned* owner_ctr, cudaStream_t s) {
+                      unsigned* chunk_ctr, unsigned* owners, unsigned* owner_ctr, const unsigned* bagpos,
+                      const double* mult, cudaStream_t s) {
   const int G = seg_group(t->dim), NV = seg_nv(t->dim);
   const int pstride = NV * G * 4;  // doubles per partial (>= dim)
+  const bool ext = mult != nullptr;
   cudaError_t e;
   if (t->dim >= DHS_SEGW_MIN_DIM) {
-    auto fn = t->opt == DHS_SGD ? launch_seg_sgd_w
-              : t->opt == DHS_ADAGRAD ? launch_seg_adagrad_w
-              : t->opt == DHS_ADAM ? launch_seg_adam_w
-                                   : launch_seg_rowwise_w;
-    e = fn(segw_cpl(t->dim), t->sm_count, sk, sv, n, grad, nb, t->dim, rowspace(t), oa, part_head, part_tail,
-           pstride, seg_chunk(n), chunk_ctr, owners, owner_ctr, t->st, s);
+    auto fn = t->opt == DHS_SGD ? (ext ? launch_seg_sgd_ext_w : launch_seg_sgd_w)
+              : t->opt == DHS_ADAGRAD ? (ext ? launch_seg_adagrad_ext_w : launch_seg_adagrad_w)
+              : t->opt == DHS_ADAM ? (ext ? launch_seg_adam_ext_w : launch_seg_adam_w)
+                                   : (ext ? launch_seg_rowwise_ext_w : launch_seg_rowwise_w);
+    e = fn(segw_cpl(t->dim), t->wbf16, t->sm_count, sk, sv, n, grad, nb, t->dim, rowspace(t), oa, part_head,
+           part_tail, pstride, seg_chunk(n), chunk_ctr, owners, owner_ctr, t->st, bagpos, mult, s);
   } else {
-    auto fn = t->opt == DHS_SGD ? launch_seg_sgd
-              : t->opt == DHS_ADAGRAD ? launch_seg_adagrad
-              : t->opt == DHS_ADAM ? launch_seg_adam
-                                   : launch_seg_rowwise;
+    auto fn = t->opt == DHS_SGD ? (ext ? launch_seg_sgd_ext : launch_seg_sgd)
+              : t->opt == DHS_ADAGRAD ? (ext ? launch_seg_adagrad_ext : launch_seg_adagrad)
+              : t->opt == DHS_ADAM ? (ext ? launch_seg_adam_ext : launch_seg_adam)
+                                   : (ext ? launch_seg_rowwise_ext : launch_seg_rowwise);
     e = fn(G, NV, t->sm_count, sk, sv, n, grad, nb, t->dim, rowspace(t), oa, part_head, part_tail,
-           seg_chunk(n), chunk_ctr, owners, owner_ctr, t->st, s);
+           seg_chunk(n), chunk_ctr, owners, owner_ctr, t->st, bagpos, mult, s);
   }
   t->n_launches++;
   if (e != cudaSuccess) cudaGetLastError();
@@ -506,10 +597,11 @@ dhs_status launch_seg(dhs_table* t, const unsigned* sk, const unsigned* sv, long
 }
 
 dhs_status dispatch_seg(dhs_table* t, const unsigned* sk, const unsigned* sv, long long n,
-                        const float* grad, long long nb, const OptArgs& oa, cudaStream_t s) {
+                        const float* grad, long long nb, const OptArgs& oa, bool ext, cudaStream_t s) {
   return launch_seg(t, sk, sv, n, grad, nb, oa, (double*)t->b_ph.p, (double*)t->b_pt.p,
                     (unsigned*)t->b_hist.p + kSegChunkCtrWord, (unsigned*)t->b_owners.p,
-                    (unsigned*)t->b_hist.p + kSegOwnerCtrWord, s);
+                    (unsigned*)t->b_hist.p + kSegOwnerCtrWord, ext ? (const unsigned*)t->b_bagpos.p : nullptr,
+                    ext ? (const double*)t->b_mult.p : nullptr, s);
 }
 
 // offset assignment + row init for the new keys of an insert call
@@ -518,12 +610,12 @@ dhs_status launch_assign(dhs_table* t, const long long* keys, long long n, cudaS
   const long long ngroups = (n + kGroupPositions - 1) / kGroupPositions;
   fwd_mark_kernel<<<(unsigned)ngroups, kGroupThreads, 0, s>>>(
       t->slots, (unsigned*)t->b_nbm.p, (unsigned*)t->b_fbm.p, (unsigned*)t->b_gcnt.p,
-      (unsigned*)t->b_gpref.p, (const unsigned*)t->b_slotpos.p, nwords, ngroups, t->st);
+      (unsigned*)t->b_gpref.p, (const unsigned*)t->b_slotpos.p, nwords, ngroups, hooks(t), t->st);
   t->n_launches += 2;
   DHS_TRY(last_launch());
-  fwd_assign_kernel<<<(unsigned)ngroups, kGroupThreads, 0, s>>>(
+  fwd_assign_kernel<<<(unsigned)(ngroups * kAssignSplit), kGroupThreads, 0, s>>>(
       t->slots, rowspace(t), t->dim, keys, (const unsigned*)t->b_fbm.p, (const unsigned*)t->b_gpref.p,
-      (const unsigned*)t->b_slotpos.p, nwords, ngroups, t->st);
+      (const unsigned*)t->b_slotpos.p, nwords, ngroups, hooks(t), t->st);
   return last_launch();
 }
 
@@ -568,11 +660,15 @@ dhs_status dhs_pack_keys(const int32_t* d_table_ids, const int64_t* d_ids, int64
   return last_launch();
 }
 
-dhs_status ht_create(int32_t dim, dhs_optimizer opt, int64_t block_rows, int64_t max_rows,
-                     const dhs_opt_params* params, const dhs_allocator* alloc, dhs_table** out) {
+dhs_status ht_create_ex(int32_t dim, dhs_optimizer opt, dhs_row_dtype weights, int64_t block_rows,
+                        int64_t max_rows, const dhs_opt_params* params, const dhs_allocator* alloc,
+                        dhs_table** out) {
   if (!out) return DHS_ERR_INVALID_ARG;
   *out = nullptr;
   if (dim < 4 || dim > 512 || dim % 4) return DHS_ERR_INVALID_ARG;
+  if (weights != DHS_ROWS_F32 && weights != DHS_ROWS_BF16) return DHS_ERR_INVALID_ARG;
+  // bf16 rows: 8 weights per 16-byte unit, warp segment kernel (dim >= 32)
+  if (weights == DHS_ROWS_BF16 && (dim % 8 || dim < DHS_SEGW_MIN_DIM)) return DHS_ERR_UNSUPPORTED;
   if (state_floats(opt, dim) < 0) return DHS_ERR_INVALID_ARG;
   if (block_rows == 0) block_rows = kDefaultBlockRows;
   if (block_rows < 1 || (block_rows & (block_rows - 1)) || block_rows > (1ll << 30))
@@ -594,7 +690,9 @@ dhs_status ht_create(int32_t dim, dhs_optimizer opt, int64_t block_rows, int64_t
   cudaDeviceGetAttribute(&t->sm_count, cudaDevAttrMultiProcessorCount, t->device);
   t->dim = dim;
   t->opt = opt;
-  t->stride = dim + state_floats(opt, dim);
+  t->wbf16 = weights == DHS_ROWS_BF16;
+  t->wfl = t->wbf16 ? dim / 2 : dim;
+  t->stride = t->wfl + state_floats(opt, dim);
   if (params) {
     t->eps = params->eps;
     t->b1 = params->beta1;
@@ -631,7 +729,7 @@ dhs_status ht_create(int32_t dim, dhs_optimizer opt, int64_t block_rows, int64_t
     rc = DHS_ERR_CUDA;
   for (int i = 0; rc == DHS_OK && i < kSnapRing; ++i) {
     if (cudaEventCreateWithFlags(&t->snaps[i].ev, cudaEventDisableTiming) != cudaSuccess ||
-        cudaHostAlloc((void**)&t->snaps[i].pinned, sizeof(unsigned long long), cudaHostAllocDefault) != cudaSuccess)
+        cudaHostAlloc((void**)&t->snaps[i].pinned, 2 * sizeof(unsigned long long), cudaHostAllocDefault) != cudaSuccess)
       rc = DHS_ERR_CUDA;
   }
   if (rc == DHS_OK) rc = grow_map(t, kInitialSlots, s);
@@ -646,6 +744,11 @@ dhs_status ht_create(int32_t dim, dhs_optimizer opt, int64_t block_rows, int64_t
   return DHS_OK;
 }
 
+dhs_status ht_create(int32_t dim, dhs_optimizer opt, int64_t block_rows, int64_t max_rows,
+                     const dhs_opt_params* params, const dhs_allocator* alloc, dhs_table** out) {
+  return ht_create_ex(dim, opt, DHS_ROWS_F32, block_rows, max_rows, params, alloc, out);
+}
+
 dhs_status ht_destroy(dhs_table* t) {
   if (!t) return DHS_OK;
   DeviceGuard g(t->device);
@@ -658,9 +761,13 @@ dhs_status ht_destroy(dhs_table* t) {
   dfree(t, t->slots, t->nslots * sizeof(Slot), s);
   dfree(t, t->blocks_d, sizeof(float*) * t->max_blocks, s);
   dfree(t, t->st, sizeof(DevState), s);
-  Buf* bufs[] = {&t->b_nbm, &t->b_fbm, &t->b_gcnt, &t->b_gpref, &t->b_slotpos, &t->b_ka, &t->b_va,
+  if (t->cnt) dfree(t, t->cnt, t->nslots * 4, s);
+  if (t->stamp) dfree(t, t->stamp, t->nslots * 4, s);
+  if (t->free_bm) dfree(t, t->free_bm, (size_t)t->free_words * 4, s);
+  if (t->free_list) dfree(t, t->free_list, (size_t)t->free_list_cap * 4, s);
+  Buf* bufs[] = {&t->b_fcnt, &t->b_freed, &t->b_nbm, &t->b_fbm, &t->b_gcnt, &t->b_gpref, &t->b_slotpos, &t->b_ka, &t->b_va,
                  &t->b_kb, &t->b_vb, &t->b_hist, &t->b_totals, &t->b_ph, &t->b_pt, &t->b_owners,
-                 &t->b_cplan, &t->b_slots, &t->b_refs};
+                 &t->b_cplan, &t->b_slots, &t->b_refs, &t->b_bagpos, &t->b_mult};
   for (Buf* b : bufs) bfree(t, *b, s);
   cudaStreamSynchronize(s);
   for (auto& sn : t->snaps) {
@@ -704,17 +811,21 @@ dhs_status ht_lookup_or_insert(dhs_table* t, const int64_t* d_keys, int64_t n,
                                int64_t* d_offsets_out, dhs_stream stream) {
   DHS_TRY(check_table(t));
   if (n < 0 || n >= (1ll << 31) || (n > 0 && (!d_keys || !d_offsets_out))) return DHS_ERR_INVALID_ARG;
-  if (n == 0) return DHS_OK;
+  if (n == 0) {
+    t->step++;  // every insert call is a step of the access stamps
+    return DHS_OK;
+  }
   DeviceGuard g(t->device);
   cudaStream_t s = (cudaStream_t)stream;
   t->last_stream = s;
   DHS_TRY(ensure_capacity(t, n, s));
   DHS_TRY(ensure_ws(t, n, s));
+  t->step++;
   {
     PhaseScope ph(t, PH_LOOKUP_INSERT, s);
     fwd_probe_offsets_kernel<<<(unsigned)((n + kFwdThreads - 1) / kFwdThreads), kFwdThreads, 0, s>>>(
         idmap(t), (const long long*)d_keys, n, (long long*)d_offsets_out, (unsigned*)t->b_nbm.p,
-        (unsigned*)t->b_slotpos.p, t->st);
+        (unsigned*)t->b_slotpos.p, hooks(t), t->st);
     t->n_launches += 2;
     DHS_TRY(last_launch());
     DHS_TRY(launch_assign(t, (const long long*)d_keys, n, s));
@@ -723,6 +834,7 @@ dhs_status ht_lookup_or_insert(dhs_table* t, const int64_t* d_keys, int64_t n,
     DHS_TRY(last_launch());
   }
   t->rows_ub += n;
+  t->keys_ub += n;
   t->cum_n += n;
   t->n_insert_calls++;
   record_snapshot(t, s);
@@ -743,13 +855,21 @@ dhs_status ht_lookup(dhs_table* t, const int64_t* d_keys, int64_t n, int64_t* d_
   return last_launch();
 }
 
-dhs_status embbag_forward(dhs_table* t, const int64_t* d_keys, int64_t n_keys,
-                          const int64_t* d_bag_offsets, int64_t n_bags, float* d_pooled_out,
-                          dhs_stream stream) {
+dhs_status embbag_forward_ex(dhs_table* t, const int64_t* d_keys, int64_t n_keys,
+                             const int64_t* d_bag_offsets, int64_t n_bags, const float* d_per_sample_weights,
+                             dhs_pool_mode mode, float* d_pooled_out, dhs_stream stream) {
   DHS_TRY(check_table(t));
   if (n_keys < 0 || n_keys >= (1ll << 31) || n_bags < 0 || n_bags >= (1ll << 31))
     return DHS_ERR_INVALID_ARG;
-  if (n_bags == 0) return n_keys == 0 ? DHS_OK : DHS_ERR_INVALID_ARG;
+  if (mode != DHS_POOL_SUM && mode != DHS_POOL_MEAN) return DHS_ERR_INVALID_ARG;
+  if (mode == DHS_POOL_MEAN && d_per_sample_weights) return DHS_ERR_INVALID_ARG;
+  const bool mean = mode == DHS_POOL_MEAN;
+  const float* psw = n_keys > 0 ? d_per_sample_weights : nullptr;
+  if (n_bags == 0) {
+    if (n_keys != 0) return DHS_ERR_INVALID_ARG;
+    t->step++;  // every insert call is a step of the access stamps
+    return DHS_OK;
+  }
   if (!d_bag_offsets || !d_pooled_out || (n_keys > 0 && !d_keys)) return DHS_ERR_INVALID_ARG;
   if ((uintptr_t)d_pooled_out % 16) return DHS_ERR_INVALID_ARG;
   DeviceGuard g(t->device);
@@ -757,14 +877,17 @@ dhs_status embbag_forward(dhs_table* t, const int64_t* d_keys, int64_t n_keys,
   t->last_stream = s;
   if (n_keys > 0) DHS_TRY(ensure_capacity(t, n_keys, s));
   DHS_TRY(ensure_ws(t, n_keys, s));
-  if (n_keys >= (long long)DHS_POOL_SPLIT_LEN * n_bags && n_keys > 0) {
+  t->step++;
+  // admission and eviction need the split forward (the probe counts and
+  // stamps, the assignment decides which keys get a row before the gather)
+  if (n_keys > 0 && (n_keys >= (long long)DHS_POOL_SPLIT_LEN * n_bags || has_hooks(t))) {
     // long bags: probe every id (a thread per id), assign and write the new
     // keys' rows, then gather every row from the table
     {
       PhaseScope ph(t, PH_FWD_PROBE, s);
       fwd_probe_offsets_kernel<<<(unsigned)((n_keys + kFwdThreads - 1) / kFwdThreads), kFwdThreads, 0, s>>>(
           idmap(t), (const long long*)d_keys, n_keys, (long long*)t->b_refs.p, (unsigned*)t->b_nbm.p,
-          (unsigned*)t->b_slotpos.p, t->st);
+          (unsigned*)t->b_slotpos.p, hooks(t), t->st);
       t->n_launches++;
       DHS_TRY(last_launch());
     }
@@ -774,10 +897,11 @@ dhs_status embbag_forward(dhs_table* t, const int64_t* d_keys, int64_t n_keys,
     }
     {
       PhaseScope ph(t, PH_FWD_POOL, s);
-      const int G = pick_group(t->dim), NV = pick_nv(t->dim, G);
-      const cudaError_t e =
-          launch_pool_refs(G, NV, t->sm_count, rowspace(t), t->dim, t->slots, (const long long*)t->b_refs.p,
-                           n_keys, (const long long*)d_bag_offsets, n_bags, d_pooled_out, t->st, s);
+      const int wd = t->wbf16 ? t->dim / 2 : t->dim;
+      const int G = pick_group(wd), NV = pick_nv(wd, G);
+      const cudaError_t e = (t->wbf16 ? launch_pool_refs_bf16 : launch_pool_refs)(
+          G, NV, t->sm_count, rowspace(t), t->dim, t->slots, (const long long*)t->b_refs.p, n_keys,
+          (const long long*)d_bag_offsets, n_bags, psw, mean, d_pooled_out, t->st, s);
       t->n_launches++;
       if (e != cudaSuccess) {
         cudaGetLastError();
@@ -788,7 +912,7 @@ dhs_status embbag_forward(dhs_table* t, const int64_t* d_keys, int64_t n_keys,
     {
       PhaseScope ph(t, PH_FWD_POOL, s);
       DHS_TRY(dispatch_pool(t, (const long long*)d_keys, n_keys, (const long long*)d_bag_offsets,
-                            n_bags, d_pooled_out, s));
+                            n_bags, psw, mean, d_pooled_out, s));
     }
     if (n_keys > 0) {
       PhaseScope ph(t, PH_FWD_ASSIGN, s);
@@ -798,18 +922,31 @@ dhs_status embbag_forward(dhs_table* t, const int64_t* d_keys, int64_t n_keys,
   t->n_insert_calls++;
   if (n_keys > 0) {
     t->rows_ub += n_keys;
+    t->keys_ub += n_keys;
     t->cum_n += n_keys;
     record_snapshot(t, s);
   }
   return DHS_OK;
 }
 
-dhs_status embbag_backward_update(dhs_table* t, const int64_t* d_keys, int64_t n_keys,
-                                  const int64_t* d_bag_offsets, int64_t n_bags,
-                                  const float* d_grad, float lr, dhs_stream stream) {
+dhs_status embbag_forward(dhs_table* t, const int64_t* d_keys, int64_t n_keys,
+                          const int64_t* d_bag_offsets, int64_t n_bags, float* d_pooled_out,
+                          dhs_stream stream) {
+  return embbag_forward_ex(t, d_keys, n_keys, d_bag_offsets, n_bags, nullptr, DHS_POOL_SUM, d_pooled_out, stream);
+}
+
+dhs_status embbag_backward_update_ex(dhs_table* t, const int64_t* d_keys, int64_t n_keys,
+                                     const int64_t* d_bag_offsets, int64_t n_bags,
+                                     const float* d_per_sample_weights, dhs_pool_mode mode,
+                                     const float* d_grad, float lr, dhs_stream stream) {
   DHS_TRY(check_table(t));
   if (n_keys < 0 || n_keys >= (1ll << 31) || n_bags < 0 || n_bags >= (1ll << 31))
     return DHS_ERR_INVALID_ARG;
+  if (mode != DHS_POOL_SUM && mode != DHS_POOL_MEAN) return DHS_ERR_INVALID_ARG;
+  if (mode == DHS_POOL_MEAN && d_per_sample_weights) return DHS_ERR_INVALID_ARG;
+  const bool mean = mode == DHS_POOL_MEAN;
+  const float* psw = n_keys > 0 ? d_per_sample_weights : nullptr;
+  const bool ext = psw != nullptr || mean;
   if (n_bags == 0 && n_keys != 0) return DHS_ERR_INVALID_ARG;
   if (n_bags > 0 && (!d_bag_offsets || !d_grad)) return DHS_ERR_INVALID_ARG;
   if ((uintptr_t)d_grad % 16) return DHS_ERR_INVALID_ARG;
@@ -821,6 +958,7 @@ dhs_status embbag_backward_update(dhs_table* t, const int64_t* d_keys, int64_t n
   t->adam_t += 1;
   if (n_keys == 0) return DHS_OK;
   DHS_TRY(ensure_ws(t, n_keys, s));
+  if (ext) DHS_TRY(ensure_ws_ext(t, s));
 
   // rows of the table are < rows_ub; rows_ub itself marks a missing key
   refresh_ub(t, false);
@@ -835,15 +973,15 @@ dhs_status embbag_backward_update(dhs_table* t, const int64_t* d_keys, int64_t n
   unsigned* vb = (unsigned*)t->b_vb.p;
   {
     PhaseScope ph(t, PH_BWD_PROBE, s);
-    static int resident = 0;
-    if (!resident) resident = resident_blocks(bwd_probe_kernel, 256, 0, t->sm_count);
+    // a warp per chunk of bags, all launched at once: the SMs overlap the
+    // chunks' dependent loads (bag ends, keys, slots) across many warps
     const int bpc = bwd_probe_bags(n_keys, n_bags);
     const long long warps = (n_bags + bpc - 1) / bpc;
-    const long long grid = grid_for((warps + 7) / 8, resident);
-    bwd_probe_kernel<<<(unsigned)grid, 256, 0, s>>>(idmap(t), (const long long*)d_keys, n_keys,
-                                                    (const long long*)d_bag_offsets, n_bags, ka, va,
-                                                    sentinel, (unsigned*)t->b_hist.p, kSortZeroWords,
-                                                    bpc, t->st);
+    const long long grid = std::max<long long>(1, (warps + 7) / 8);
+    (ext ? bwd_probe_kernel<true> : bwd_probe_kernel<false>)<<<(unsigned)grid, 256, 0, s>>>(
+        idmap(t), (const long long*)d_keys, n_keys, (const long long*)d_bag_offsets, n_bags, ka, va, sentinel,
+        (unsigned*)t->b_hist.p, kSortZeroWords, bpc, psw, mean, (unsigned*)t->b_bagpos.p, (double*)t->b_mult.p,
+        t->st);
     t->n_launches++;
     DHS_TRY(last_launch());
   }
@@ -882,7 +1020,7 @@ dhs_status embbag_backward_update(dhs_table* t, const int64_t* d_keys, int64_t n
     oa.bc2 = (float)(1.0 - std::pow((double)t->b2, (double)t->adam_t));
     {
       PhaseScope ph(t, PH_BWD_SEG, s);
-      DHS_TRY(dispatch_seg(t, ka, va, n_keys, d_grad, n_bags, oa, s));
+      DHS_TRY(dispatch_seg(t, ka, va, n_keys, d_grad, n_bags, oa, ext, s));
     }
     PhaseScope ph(t, PH_BWD_COMBINE, s);
     const int pstride = seg_nv(t->dim) * seg_group(t->dim) * 4;
@@ -895,6 +1033,13 @@ dhs_status embbag_backward_update(dhs_table* t, const int64_t* d_keys, int64_t n
   return DHS_OK;
 }
 
+dhs_status embbag_backward_update(dhs_table* t, const int64_t* d_keys, int64_t n_keys,
+                                  const int64_t* d_bag_offsets, int64_t n_bags,
+                                  const float* d_grad, float lr, dhs_stream stream) {
+  return embbag_backward_update_ex(t, d_keys, n_keys, d_bag_offsets, n_bags, nullptr, DHS_POOL_SUM, d_grad, lr,
+                                   stream);
+}
+
 dhs_status ht_get_rows(dhs_table* t, const int64_t* d_keys, int64_t n, float* d_rows_out,
                        dhs_stream stream) {
   DHS_TRY(check_table(t));
@@ -904,12 +1049,103 @@ dhs_status ht_get_rows(dhs_table* t, const int64_t* d_keys, int64_t n, float* d_
   cudaStream_t s = (cudaStream_t)stream;
   t->last_stream = s;
   const long long grid = std::min<long long>((n + 7) / 8, (long long)t->sm_count * 16);
-  get_rows_kernel<<<(unsigned)grid, 256, 0, s>>>(idmap(t), rowspace(t), (const long long*)d_keys, n, d_rows_out);
+  get_rows_kernel<<<(unsigned)grid, 256, 0, s>>>(idmap(t), rowspace(t), t->dim, export_stride(t),
+                                                 (const long long*)d_keys, n, d_rows_out);
   t->n_launches++;
   return last_launch();
 }
 
-int64_t ht_row_stride(const dhs_table* t) { return t ? t->stride : -1; }
+dhs_status ht_set_hooks(dhs_table* t, int64_t admit_threshold, int track_access) {
+  DHS_TRY(check_table(t));
+  if (admit_threshold < 0 || admit_threshold > 0x7fffffff) return DHS_ERR_INVALID_ARG;
+  if (t->step > 0 || t->rows_ub > 0 || t->has_hooks_set) return DHS_ERR_INVALID_ARG;  // before the first insert, once
+  DeviceGuard g(t->device);
+  cudaStream_t s = t->last_stream;
+  t->admit = (unsigned)std::max<int64_t>(1, admit_threshold);
+  t->track = track_access != 0;
+  t->has_hooks_set = true;
+  if (t->admit > 1) {
+    t->cnt = (unsigned*)dalloc(t, t->nslots * 4, s);
+    if (!t->cnt) return DHS_ERR_OOM;
+    DHS_CUDA(cudaMemsetAsync(t->cnt, 0, t->nslots * 4, s));
+  }
+  if (t->track) {
+    t->stamp = (unsigned*)dalloc(t, t->nslots * 4, s);
+    if (!t->stamp) return DHS_ERR_OOM;
+    DHS_CUDA(cudaMemsetAsync(t->stamp, 0, t->nslots * 4, s));
+  }
+  DHS_CUDA(cudaMemsetAsync(&t->st->keys_used, 0, sizeof(unsigned long long), s));
+  return DHS_OK;
+}
+
+dhs_status ht_evict(dhs_table* t, int64_t max_idle, int64_t* n_freed, dhs_stream stream) {
+  DHS_TRY(check_table(t));
+  if (!t->track || max_idle < 0 || !n_freed) return DHS_ERR_INVALID_ARG;
+  DeviceGuard g(t->device);
+  cudaStream_t s = (cudaStream_t)stream;
+  t->last_stream = s;
+  *n_freed = 0;
+  const long long keep_from = t->step - max_idle;  // keys last seen before this step go
+  if (keep_from <= 1) return DHS_OK;                // every stamp is >= 1
+  DHS_CUDA(cudaStreamSynchronize(s));
+  unsigned long long rows = 0;
+  DHS_CUDA(cudaMemcpy(&rows, &t->st->row_count, sizeof(rows), cudaMemcpyDeviceToHost));
+  // the free-row bitmap covers every row; the list can hold them all
+  const long long words = (long long)((rows + 31) / 32);
+  if (words > t->free_words) {
+    const long long nw = std::max<long long>(words, t->free_words * 2);
+    unsigned* nb = (unsigned*)dalloc(t, (size_t)nw * 4, s);
+    if (!nb) return DHS_ERR_OOM;
+    DHS_CUDA(cudaMemsetAsync(nb, 0, (size_t)nw * 4, s));
+    if (t->free_bm) {
+      DHS_CUDA(cudaMemcpyAsync(nb, t->free_bm, (size_t)t->free_words * 4, cudaMemcpyDeviceToDevice, s));
+      dfree(t, t->free_bm, (size_t)t->free_words * 4, s);
+    }
+    t->free_bm = nb;
+    t->free_words = nw;
+  }
+  if ((long long)rows > t->free_list_cap) {
+    const long long cap = std::max<long long>((long long)rows, t->free_list_cap * 2);
+    unsigned* nl = (unsigned*)dalloc(t, (size_t)cap * 4, s);
+    if (!nl) return DHS_ERR_OOM;
+    if (t->free_list) dfree(t, t->free_list, (size_t)t->free_list_cap * 4, s);
+    t->free_list = nl;
+    t->free_list_cap = cap;
+  }
+  const long long nblocks = std::max<long long>(1, (words + kFreeWords - 1) / kFreeWords);
+  DHS_TRY(bget(t, t->b_fcnt, (size_t)nblocks * 4, s));
+  DHS_TRY(bget(t, t->b_freed, sizeof(unsigned long long), s));
+  DHS_CUDA(cudaMemsetAsync(t->b_freed.p, 0, sizeof(unsigned long long), s));
+  const int thr = 256;
+  const long long g1 = std::min<long long>((long long)((t->nslots + thr - 1) / thr), (long long)t->sm_count * 16);
+  evict_kernel<<<(unsigned)g1, thr, 0, s>>>(t->slots, t->nslots, t->stamp, (unsigned)keep_from, t->free_bm,
+                                            (unsigned long long*)t->b_freed.p);
+  free_count_kernel<<<(unsigned)nblocks, kFreeThreads, 0, s>>>(t->free_bm, words, (unsigned*)t->b_fcnt.p,
+                                                                nblocks, t->st);
+  free_scatter_kernel<<<(unsigned)nblocks, kFreeThreads, 0, s>>>(t->free_bm, words, (const unsigned*)t->b_fcnt.p,
+                                                                  t->free_list);
+  t->n_launches += 3;
+  DHS_TRY(last_launch());
+  unsigned long long freed = 0;
+  DHS_CUDA(cudaMemcpyAsync(&freed, t->b_freed.p, sizeof(freed), cudaMemcpyDeviceToHost, s));
+  DHS_CUDA(cudaStreamSynchronize(s));
+  *n_freed = (int64_t)freed;
+  return DHS_OK;
+}
+
+dhs_status ht_live_rows(dhs_table* t, int64_t* n_live) {
+  DHS_TRY(check_table(t));
+  if (!n_live) return DHS_ERR_INVALID_ARG;
+  const dhs_status rc = ht_sync(t);
+  if (rc == DHS_ERR_CUDA) return rc;
+  DeviceGuard g(t->device);
+  DevState h;
+  DHS_CUDA(cudaMemcpy(&h, t->st, sizeof(h), cudaMemcpyDeviceToHost));
+  *n_live = (int64_t)(h.row_count - (h.free_count - h.free_head));
+  return rc;
+}
+
+int64_t ht_row_stride(const dhs_table* t) { return t ? export_stride(t) : -1; }
 
 dhs_status ht_sync(dhs_table* t) {
   DHS_TRY(check_table(t));
@@ -974,6 +1210,7 @@ dhs_status ht_export(dhs_table* t, int64_t* h_keys, float* h_rows) {
     long long* kb = (long long*)dalloc(t, sizeof(long long) * rows, s);
     if (!kb) return DHS_ERR_OOM;
     const long long grid = std::min<long long>((long long)((t->nslots + 255) / 256), (long long)t->sm_count * 16);
+    DHS_CUDA(cudaMemsetAsync(kb, 0xff, sizeof(long long) * rows, s));  // a free (evicted) row has key -1
     keys_by_row_kernel<<<(unsigned)grid, 256, 0, s>>>(t->slots, t->nslots, kb, (unsigned long long)rows);
     dhs_status lr = last_launch();
     if (lr == DHS_OK && cudaMemcpyAsync(h_keys, kb, sizeof(long long) * rows, cudaMemcpyDeviceToHost, s) != cudaSuccess)
@@ -983,11 +1220,32 @@ dhs_status ht_export(dhs_table* t, int64_t* h_keys, float* h_rows) {
     cudaStreamSynchronize(s);
     DHS_TRY(lr);
   }
-  if (h_rows) {
+  if (h_rows && !t->wbf16) {
     for (long long r0 = 0; r0 < rows; r0 += t->block_rows) {
       const long long cnt = std::min<long long>(t->block_rows, rows - r0);
       DHS_CUDA(cudaMemcpy(h_rows + r0 * t->stride, t->blocks_h[r0 >> t->log2_br],
                           sizeof(float) * cnt * t->stride, cudaMemcpyDeviceToHost));
+    }
+  } else if (h_rows) {
+    // bf16 weights: each block's raw rows, widened on the host to the fp32
+    // export layout (dim weights, then the state)
+    const int es = export_stride(t);
+    std::vector<float> raw;
+    for (long long r0 = 0; r0 < rows; r0 += t->block_rows) {
+      const long long cnt = std::min<long long>(t->block_rows, rows - r0);
+      raw.resize((size_t)cnt * t->stride);
+      DHS_CUDA(cudaMemcpy(raw.data(), t->blocks_h[r0 >> t->log2_br], sizeof(float) * cnt * t->stride,
+                          cudaMemcpyDeviceToHost));
+      for (long long r = 0; r < cnt; ++r) {
+        const float* src = raw.data() + r * t->stride;
+        float* dst = h_rows + (r0 + r) * es;
+        const uint16_t* w = reinterpret_cast<const uint16_t*>(src);
+        for (int j = 0; j < t->dim; ++j) {
+          const uint32_t u = (uint32_t)w[j] << 16;
+          std::memcpy(dst + j, &u, 4);
+        }
+        std::memcpy(dst + t->dim, src + t->wfl, sizeof(float) * (t->stride - t->wfl));
+      }
     }
   }
   return rc;
@@ -1037,7 +1295,7 @@ dhs_status ht_phase_times(dhs_table* t, double* ms_out, int64_t* count_out, int 
 
 namespace {
 
-constexpr long long kNoAllocMaxKeys = 131072;
+constexpr long long kNoAllocMaxKeys = DHS_NOALLOC_MAX_KEYS;
 constexpr int kNoAllocMaxDim = 128;
 constexpr int kNoAllocMinChunk = 32;  // seg_chunk() never goes below this
 
@@ -1049,7 +1307,7 @@ constexpr size_t kNaStatus =
 constexpr size_t kNaChunks = (kNoAllocMaxKeys + kNoAllocMinChunk - 1) / kNoAllocMinChunk;
 constexpr size_t kNaPart = na_align(kNaChunks * kNoAllocMaxDim * 8);  // one of part_head, part_tail
 constexpr size_t kNaOwners = na_align(kNaChunks * 4);
-constexpr size_t kNaPlan = na_align((5 * kNaChunks + combine_batch_cap(kNaChunks)) * 4);
+constexpr size_t kNaPlan = na_align((6 * kNaChunks + combine_batch_cap(kNaChunks)) * 4);
 constexpr size_t kNaSlots = na_align(combine_slot_cap(kNaChunks) * kNoAllocMaxDim * 8);
 constexpr size_t kNoAllocScratchBytes =
     4 * kNaPairs + kNaSortZero + kNaStatus + 2 * kNaPart + kNaOwners + kNaPlan + kNaSlots;
@@ -1087,6 +1345,8 @@ dhs_status embbag_backward_update_noalloc(dhs_table* t, const int64_t* d_keys, i
   DHS_TRY(check_table(t));
   if (n_keys < 0 || n_bags < 0 || n_bags >= (1ll << 31)) return DHS_ERR_INVALID_ARG;
   if (n_keys > kNoAllocMaxKeys || t->dim > kNoAllocMaxDim) return DHS_ERR_INVALID_ARG;
+  // the partial vectors are sized for kNoAllocMaxDim doubles each
+  if (seg_nv(t->dim) * seg_group(t->dim) * 4 > kNoAllocMaxDim) return DHS_ERR_INVALID_ARG;
   if (n_bags == 0 && n_keys != 0) return DHS_ERR_INVALID_ARG;
   if (n_bags > 0 && (!d_bag_offsets || !d_grad)) return DHS_ERR_INVALID_ARG;
   if ((uintptr_t)d_grad % 16) return DHS_ERR_INVALID_ARG;
@@ -1124,9 +1384,10 @@ dhs_status embbag_backward_update_noalloc(dhs_table* t, const int64_t* d_keys, i
     const int bpc = bwd_probe_bags(n_keys, n_bags);
     const long long warps = (n_bags + bpc - 1) / bpc;
     const long long grid = std::max<long long>(1, std::min<long long>((warps + 7) / 8, (long long)t->sm_count * 8));
-    bwd_probe_kernel<<<(unsigned)grid, 256, 0, s>>>(idmap(t), (const long long*)d_keys, n_keys,
+    bwd_probe_kernel<false><<<(unsigned)grid, 256, 0, s>>>(idmap(t), (const long long*)d_keys, n_keys,
                                                     (const long long*)d_bag_offsets, n_bags, ka, va,
-                                                    sentinel, hist, kSortZeroWords, bpc, t->st);
+                                                    sentinel, hist, kSortZeroWords, bpc, nullptr, false,
+                                                    nullptr, nullptr, t->st);
     DHS_TRY(last_launch());
   }
   const long long ntiles = (n_keys + kRadixTile - 1) / kRadixTile;
@@ -1158,7 +1419,7 @@ dhs_status embbag_backward_update_noalloc(dhs_table* t, const int64_t* d_keys, i
   const int G = seg_group(t->dim), NV = seg_nv(t->dim);
   const int chunk = seg_chunk(n_keys);
   DHS_TRY(launch_seg(t, ka, va, n_keys, d_grad, n_bags, oa, part_head, part_tail, hist + kSegChunkCtrWord, owners,
-                     hist + kSegOwnerCtrWord, s));
+                     hist + kSegOwnerCtrWord, nullptr, nullptr, s));
   t->n_launches += 2 + passes;
   return launch_combine(t, ka, n_keys, oa, part_head, part_tail, chunk, NV * G * 4, owners, hist, plan, s);
 }

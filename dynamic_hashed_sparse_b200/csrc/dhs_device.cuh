@@ -11,17 +11,26 @@
 // EmbeddingBlocks ([RecIS] overview, second level: contiguous blocks holding
 // parameters and optimizer state, appended as the table grows): a device
 // array of block pointers; row r lives at blocks[r >> log2_block_rows] +
-// (r & (block_rows - 1)) * stride, stride = dim weights + optimizer state,
-// a multiple of 4 floats so every row is 16-byte aligned.
+// (r & (block_rows - 1)) * stride, stride = the weights (wfl floats: dim
+// fp32 values, or dim bf16 values in dim / 2 floats) + the optimizer state
+// (fp32), a multiple of 4 floats so every row is 16-byte aligned.
 #pragma once
 
 #include <cstdint>
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
 namespace dhs {
 
 constexpr unsigned long long kEmptyKey = ~0ull;
+// An evicted key's slot: probes step over it (the chain goes on), and it is
+// never claimed again (so no key can sit behind an empty slot in its chain);
+// a rehash drops it.
+constexpr unsigned long long kTombKey = ~1ull;
 constexpr unsigned long long kPending = 1ull << 63;
+// Between calls, the value of a key that is known but has no row yet (not
+// admitted): above every PENDING | position, so a claim's atomicMin replaces it.
+constexpr unsigned long long kCounting = ~1ull;
 
 struct __align__(16) Slot {
   unsigned long long key;
@@ -31,14 +40,19 @@ struct __align__(16) Slot {
 // Device-resident scalars of one table.
 struct DevState {
   unsigned long long row_count;  // rows assigned so far
-  unsigned long long row_base;   // first row of the current call's new keys
+  unsigned long long keys_used;  // slots claimed since the last rehash (with admission / eviction)
+  unsigned long long row_base;   // first appended row of the current call's new keys
   unsigned long long m_last;     // new rows of the last insert call
   unsigned long long n_blocks;   // blocks the host has appended
   unsigned long long sum_new;    // total inserted rows
   unsigned long long sum_unique; // total distinct keys updated by backward calls
+  unsigned long long free_count; // rows in the free list (evicted rows)
+  unsigned long long free_head;  // free-list rows handed out so far
+  unsigned long long free_base;  // free_head before the current call
+  unsigned long long m_free;     // rows of the current call taken from the free list
   unsigned int err;              // first latched error code, 0 = none
   unsigned int ticket;           // last-block-done counter (mark kernel)
-  unsigned int ticket2;          // spare
+  unsigned int ticket2;          // last-block-done counter (free-list compaction)
   unsigned int pad;
 };
 
@@ -107,6 +121,7 @@ struct RowSpace {
   unsigned long long br_mask;  // block_rows - 1
   int log2_br;
   int stride;  // floats per row
+  int wfl;     // floats holding the weights (dim, or dim / 2 for bf16 weights); the state starts there
   __device__ __forceinline__ float* row(unsigned long long r) const {
     float* b = (float*)__ldg((const unsigned long long*)(blocks + (r >> log2_br)));
     return b + (r & br_mask) * (unsigned long long)stride;
@@ -115,15 +130,31 @@ struct RowSpace {
 
 enum : int { kHit = 0, kNew = 1, kBad = 2 };
 
+// Admission / eviction state of a table (null pointers and zeros when the
+// table uses neither).
+struct Hooks {
+  unsigned* cnt;              // [slots] occurrences of keys without a row (admission)
+  unsigned* stamp;            // [slots] last insert call a key occurred in (eviction)
+  unsigned admit;             // admission threshold (<= 1: a row at first sight)
+  unsigned step;              // this insert call's number (1, 2, ...)
+  const unsigned* free_list;  // rows freed by evictions, ascending
+  unsigned* free_bm;          // bit per row: the row is free
+};
+
 // Find `key`, claiming an empty slot if it is absent.  Returns kHit with the
-// row offset in `out`, or kNew with the slot index in `out` (the key is new in
-// this call; the slot's val becomes PENDING | min position).  No thread ever
-// waits on another: a claimed key is usable at once, its offset is assigned
-// by a later kernel.  The probe visits at most every window once.
+// row offset in `out`, or kNew with the slot index in `out` (the key has no
+// row yet: new in this call, or known but not admitted; the slot's val
+// becomes PENDING | min position).  `slot` receives the key's slot index.
+// No thread ever waits on another: a claimed key is usable at once, its
+// offset is assigned by a later kernel.  The probe visits at most every
+// window once; tombstones are stepped over and never claimed.  `claimed`
+// is set when this thread took an empty slot.
 __device__ __forceinline__ int probe_claim(IdMap m, unsigned long long key, unsigned pos,
-                                           unsigned long long& out, DevState* st) {
+                                           unsigned long long& out, unsigned long long& slot,
+                                           bool& claimed, DevState* st) {
   unsigned long long w = hash_key(key) & m.win_mask;
   const unsigned long long mine = kPending | (unsigned long long)pos;
+  claimed = false;
   for (unsigned long long step = 0; step <= m.win_mask; ++step) {
     Slot* ws = m.slots + 2 * w;
     const ulonglong2 a = *reinterpret_cast<const ulonglong2*>(ws);
@@ -133,19 +164,22 @@ __device__ __forceinline__ int probe_claim(IdMap m, unsigned long long key, unsi
       const unsigned long long k = j ? b.x : a.x;
       const unsigned long long v = j ? b.y : a.y;
       if (k == key) {
+        slot = 2 * w + j;
         if (!(v & kPending)) {
           out = v;
           return kHit;
         }
         if (mine < v) atomicMin(&ws[j].val, mine);
-        out = 2 * w + j;
+        out = slot;
         return kNew;
       }
       if (k == kEmptyKey) {
         const unsigned long long old = atomicCAS(&ws[j].key, kEmptyKey, key);
         if (old == kEmptyKey || old == key) {
           atomicMin(&ws[j].val, mine);
-          out = 2 * w + j;
+          slot = 2 * w + j;
+          out = slot;
+          claimed = old == kEmptyKey;
           return kNew;
         }
       }
@@ -156,17 +190,25 @@ __device__ __forceinline__ int probe_claim(IdMap m, unsigned long long key, unsi
   return kBad;
 }
 
-// Read-only probe (no concurrent writers): row offset, or -1 if absent (or
-// left without a row by a failed assignment).
+__device__ __forceinline__ int probe_claim(IdMap m, unsigned long long key, unsigned pos,
+                                           unsigned long long& out, DevState* st) {
+  unsigned long long slot;
+  bool claimed;
+  return probe_claim(m, key, pos, out, slot, claimed, st);
+}
+
+// Read-only probe (no concurrent writers): the row offset; -1 if the key is
+// absent; -2 if it is known but has no row (not admitted yet, or left
+// without a row by a failed assignment).  Tombstones are stepped over.
 __device__ __forceinline__ long long probe_find(IdMap m, unsigned long long key) {
   unsigned long long w = hash_key(key) & m.win_mask;
   for (unsigned long long step = 0; step <= m.win_mask; ++step) {
     const ulonglong2* ws = reinterpret_cast<const ulonglong2*>(m.slots + 2 * w);
     const ulonglong2 a = __ldg(ws);
     const ulonglong2 b = __ldg(ws + 1);
-    if (a.x == key) return (a.y & kPending) ? -1 : (long long)a.y;
+    if (a.x == key) return (a.y & kPending) ? -2 : (long long)a.y;
     if (a.x == kEmptyKey) return -1;
-    if (b.x == key) return (b.y & kPending) ? -1 : (long long)b.y;
+    if (b.x == key) return (b.y & kPending) ? -2 : (long long)b.y;
     if (b.x == kEmptyKey) return -1;
     w = (w + 1) & m.win_mask;
   }
@@ -178,6 +220,22 @@ __device__ __forceinline__ long long probe_find(IdMap m, unsigned long long key)
 // whole window of upcoming rows in flight.
 __device__ __forceinline__ void prefetch_l2(const void* p, unsigned bytes) {
   asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+
+// bf16 weights.  A bf16 value is the top half of an fp32, so widening is
+// exact; storing rounds to nearest, ties to even.
+__device__ __forceinline__ float bf16_lo(unsigned w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(unsigned w) { return __uint_as_float(w & 0xffff0000u); }
+__device__ __forceinline__ float round_bf16(float a) { return __bfloat162float(__float2bfloat16_rn(a)); }
+// two values rounded to bf16, a in the low half
+__device__ __forceinline__ unsigned pack_bf16x2(float a, float b) {
+  const __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<const unsigned*>(&v);
+}
+// 8 bf16 weights (one 16-byte unit) widened to fp32
+__device__ __forceinline__ void unpack_bf16x8(const uint4 u, float4& a, float4& b) {
+  a = make_float4(bf16_lo(u.x), bf16_hi(u.x), bf16_lo(u.y), bf16_hi(u.y));
+  b = make_float4(bf16_lo(u.z), bf16_hi(u.z), bf16_lo(u.w), bf16_hi(u.w));
 }
 
 __device__ __forceinline__ float4 f4add(float4 a, float4 b) {

@@ -1,3 +1,3 @@
-// bwd_seg_kernel instantiations for Adagrad (per-element accumulator).
+// Segment-kernel instantiations for Adagrad (per-element accumulator), sum pooling.
 #include "dhs_seg_impl.cuh"
-DHS_SEG_TU(1, launch_seg_adagrad)
+DHS_SEG_TU(1, false, launch_seg_adagrad)

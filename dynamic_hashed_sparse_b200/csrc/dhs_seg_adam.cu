@@ -1,3 +1,3 @@
-// bwd_seg_kernel instantiations for Adam.
+// Segment-kernel instantiations for Adam, sum pooling.
 #include "dhs_seg_impl.cuh"
-DHS_SEG_TU(2, launch_seg_adam)
+DHS_SEG_TU(2, false, launch_seg_adam)

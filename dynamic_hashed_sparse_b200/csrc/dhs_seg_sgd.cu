@@ -1,3 +1,3 @@
-// bwd_seg_kernel instantiations for SGD.
+// Segment-kernel instantiations for SGD, sum pooling.
 #include "dhs_seg_impl.cuh"
-DHS_SEG_TU(0, launch_seg_sgd)
+DHS_SEG_TU(0, false, launch_seg_sgd)

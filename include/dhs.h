@@ -80,6 +80,13 @@ typedef enum {
   DHS_ADAGRAD_ROWWISE = 3  /* one accumulator per row: G += mean(g^2)           */
 } dhs_optimizer;
 
+/* EmbeddingBag pooling ([DLRM-P] 2.1, nn.EmbeddingBag): the sum of a bag's
+ * rows (optionally weighted per id), or their mean. */
+typedef enum {
+  DHS_POOL_SUM = 0,
+  DHS_POOL_MEAN = 1
+} dhs_pool_mode;
+
 typedef struct {
   float eps;   /* default 1e-8 */
   float beta1; /* Adam, default 0.9 */
@@ -118,6 +125,26 @@ dhs_status ht_create(int32_t dim, dhs_optimizer opt, int64_t block_rows, int64_t
                      const dhs_opt_params* params, const dhs_allocator* alloc,
                      dhs_table** out);
 
+/* Storage type of the weights ([DLRM-P] 4.2: embedding matrices stored in
+ * 16-bit floats to halve their bytes); the optimizer state is fp32 either way. */
+typedef enum {
+  DHS_ROWS_F32 = 0,
+  DHS_ROWS_BF16 = 1  /* dim a multiple of 8 in [32, 512] */
+} dhs_row_dtype;
+
+/* ht_create with a weight storage type.  DHS_ROWS_BF16: each stored weight
+ * (the initial row and every optimizer step's result) is rounded to the
+ * nearest bf16 value, ties to even; the forward sums the stored values in
+ * fp32; the optimizer computes in fp32 and rounds once on store; the state
+ * stays fp32.  A bf16 row holds dim bf16 weights then the state (dim / 2 +
+ * state floats, 16-byte aligned).  bf16 with dim not a multiple of 8 or below
+ * 32 returns DHS_ERR_UNSUPPORTED.  ht_get_rows and ht_export return bf16
+ * weights widened to fp32, so their rows have dim + state floats for both
+ * types (ht_row_stride). */
+dhs_status ht_create_ex(int32_t dim, dhs_optimizer opt, dhs_row_dtype weights, int64_t block_rows,
+                        int64_t max_rows, const dhs_opt_params* params, const dhs_allocator* alloc,
+                        dhs_table** out);
+
 /* Wait for the table's work and release everything it owns.  NULL is a no-op. */
 dhs_status ht_destroy(dhs_table* t);
 
@@ -138,7 +165,8 @@ dhs_status ht_reserve(dhs_table* t, int64_t n_keys, dhs_stream stream);
 dhs_status ht_lookup_or_insert(dhs_table* t, const int64_t* d_keys, int64_t n,
                                int64_t* d_offsets_out, dhs_stream stream);
 
-/* Read-only lookup (no insert): offset, or -1 for an absent or negative key. */
+/* Read-only lookup (no insert): offset, or -1 for an absent or negative key
+ * (or one not admitted yet). */
 dhs_status ht_lookup(dhs_table* t, const int64_t* d_keys, int64_t n, int64_t* d_offsets_out,
                      dhs_stream stream);
 
@@ -168,12 +196,38 @@ dhs_status embbag_backward_update(dhs_table* t, const int64_t* d_keys, int64_t n
                                   const int64_t* d_bag_offsets, int64_t n_bags,
                                   const float* d_grad, float lr, dhs_stream stream);
 
+/* embbag_forward with EmbeddingBag's other forms ([DLRM-P] 2.1: the module
+ * nn.EmbeddingBag, whose definition includes mode="mean" and per-sample
+ * weights).  d_per_sample_weights: NULL, or float[n_keys] (device), one
+ * weight per id, allowed with DHS_POOL_SUM only:
+ *   DHS_POOL_SUM   pooled[b] = sum of fl(w_i * row(key_i)) in bag order
+ *                  (no weights: the plain sum of embbag_forward);
+ *   DHS_POOL_MEAN  pooled[b] = fl(sum of rows / (float)len_b), one rounded
+ *                  division of the fp32 in-order sum; an empty bag gives 0.
+ * Mean pooling with weights, or an unknown mode, returns
+ * DHS_ERR_INVALID_ARG at once.  Everything else as in embbag_forward. */
+dhs_status embbag_forward_ex(dhs_table* t, const int64_t* d_keys, int64_t n_keys,
+                             const int64_t* d_bag_offsets, int64_t n_bags, const float* d_per_sample_weights,
+                             dhs_pool_mode mode, float* d_pooled_out, dhs_stream stream);
+
+/* embbag_backward_update for the forms of embbag_forward_ex: the pooled
+ * output's gradient reaches occurrence i scaled by w_i (per-sample weights)
+ * or by 1 / len(bag of i) (mean pooling), so
+ *   g_k = sum over the positions i holding k of f_i * d_grad[bag(i), :],
+ * with f_i * grad formed and summed in fp64 and rounded once to fp32, then
+ * one optimizer step as in embbag_backward_update.  The weights and mode must
+ * be those of the forward.  Same argument rules as embbag_forward_ex. */
+dhs_status embbag_backward_update_ex(dhs_table* t, const int64_t* d_keys, int64_t n_keys,
+                                     const int64_t* d_bag_offsets, int64_t n_bags,
+                                     const float* d_per_sample_weights, dhs_pool_mode mode,
+                                     const float* d_grad, float lr, dhs_stream stream);
+
 /* Allocation-free variant of embbag_backward_update (the pages have no
  * counterpart: it exists for callers that cannot allocate device memory
  * during a step, e.g. a runtime that forbids cudaMalloc once its training
  * loop runs, or one that gives this library only the buffers it owns).
  * Same arguments, same result as embbag_backward_update; the sort and
- * segment-reduce scratch is one fixed file-scope device array (about 11 MB,
+ * segment-reduce scratch is one fixed file-scope device array (about 12 MB,
  * held by every GPU that loads this library until the process exits)
  * instead of the table's growable workspace, and no cudaMalloc, cudaFree or
  * allocating library routine is called.
@@ -189,12 +243,44 @@ dhs_status embbag_backward_update_noalloc(dhs_table* t, const int64_t* d_keys, i
                                           const int64_t* d_bag_offsets, int64_t n_bags,
                                           const float* d_grad, float lr, dhs_stream stream);
 
+/* Feature admission and eviction ([RecIS] code-layout section: the
+ * HashtableHook admission / eviction strategy of the embedding engine; the
+ * pages give only its name, so the behaviour below is this library's
+ * reading).  Call on a new table, before its first insert call, at most once.
+ *   admit_threshold: a key gets a row in the first insert call (forward or
+ *     lookup-or-insert) in which its occurrences over all such calls, this
+ *     call's included, reach the threshold (0 or 1: at first sight).  Until
+ *     then it pools as a zero row, lookups give -1, its gradients are skipped
+ *     (not an error) and its count is kept.  Keys admitted by one call get
+ *     rows in the order of their first position in it.
+ *   track_access: every insert call is one step and stamps the keys that
+ *     occur in it; needed by ht_evict.
+ * With either set, forward calls always take the split forward (probe,
+ * assignment, gather).  Returns DHS_ERR_INVALID_ARG on a used table. */
+dhs_status ht_set_hooks(dhs_table* t, int64_t admit_threshold, int track_access);
+
+/* Evict every key (with or without a row) whose last occurrence is more than
+ * max_idle insert calls back (stamp < calls so far - max_idle): its IDMap
+ * slot becomes a tombstone (skipped by probes, dropped by the next rehash)
+ * and its row becomes free.  Later new keys take the free rows in ascending
+ * order before rows are appended; a reused row starts from its new key's
+ * initial values and zero state.  An evicted key that occurs again is a new
+ * key.  Synchronous: waits for the stream, then *n_freed = rows freed.
+ * Needs track_access (else DHS_ERR_INVALID_ARG).  ht_size still counts
+ * every row ever appended; ht_export gives key -1 for a free row. */
+dhs_status ht_evict(dhs_table* t, int64_t max_idle, int64_t* n_freed, dhs_stream stream);
+
+/* *n_live = rows held by keys (appended rows minus free ones).  Synchronises
+ * like ht_sync and returns its status. */
+dhs_status ht_live_rows(dhs_table* t, int64_t* n_live);
+
 /* Copy the full rows (dim weights, then the state) of the given keys into
  * d_rows_out float[n, ht_row_stride(t)]; an absent key gives a NaN row. */
 dhs_status ht_get_rows(dhs_table* t, const int64_t* d_keys, int64_t n, float* d_rows_out,
                        dhs_stream stream);
 
-/* Floats per row (weights + optimizer state), or -1 for a NULL handle. */
+/* Floats per row as ht_get_rows / ht_export return it (dim weights as fp32,
+ * then the optimizer state), or -1 for a NULL handle. */
 int64_t ht_row_stride(const dhs_table* t);
 
 /* Wait for all the table's work; return the first latched device error (and

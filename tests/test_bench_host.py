@@ -59,6 +59,10 @@ def test_algorithmic_bytes_formula():
     assert ab["fwd_refs"] == 8 * 5 + R * 6 + 4 * 8 * 4
     assert ab["bwd"] == 8 * 10 + 8 * 5 + 16 * 6 + 4 * 8 * 4 + 2 * S * 6
     assert bench.stride_floats(32, "adam") == 96 and bench.stride_floats(16, "adagrad_rowwise") == 20
+    # bf16 weights: 2 bytes per weight, fp32 state
+    assert bench.row_bytes(8, "adagrad", "bf16") == (16, 16 + 32)
+    bf = bench.alg_bytes(n=10, b=4, u=6, m=2, dim=8, opt="adagrad", weights="bf16")
+    assert bf["fwd_pool"] == ab["fwd_pool"] - 16 * 4 and bf["bwd"] == ab["bwd"] - 2 * 16 * 6
 
 
 def test_reference_arm_line_on_cpu():
@@ -70,3 +74,34 @@ def test_reference_arm_line_on_cpu():
     assert line["impl"] == "reference" and line["unit"] == "IDs/s" and line["value"] > 0
     assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] == 1
     assert line["e2e"]["h2d_bytes_per_step"] == 0
+
+
+def test_pooled_generation_equals_serial_generation():
+    """The bench's spawn-pool input generation yields the same seeded batches,
+    in step order, as generating them one by one."""
+    sys.path.insert(0, ROOT)
+    import numpy as np
+
+    import bench
+    src = bench.BatchSource(2)
+    try:
+        got = src.batches("growth_stream", 0, 0, 3)
+    finally:
+        src.close()
+    w = bench.make_workload("growth_stream", 0)
+    for s, b in enumerate(got):
+        ref = w.batch(s)
+        assert np.array_equal(b.ids, ref.ids) and np.array_equal(b.table_ids, ref.table_ids)
+        assert np.array_equal(b.bag_offsets, ref.bag_offsets)
+
+
+def test_reserve_policy():
+    sys.path.insert(0, ROOT)
+    import bench
+    w = bench.make_workload("growth_stream", 0)
+    assert bench.resolve_reserve(w, 200, "on-demand") == 0
+    assert bench.resolve_reserve(w, 200, "0") == 0
+    assert bench.resolve_reserve(w, 200, "12345") == 12345
+    assert bench.resolve_reserve(w, 10, "-1") == bench.default_reserve(w, 10)
+    hot = bench.make_workload("hot_key", 0)
+    assert bench.resolve_reserve(hot, 20, "on-demand") == 50_000_001

@@ -56,7 +56,13 @@ def test_host_side_argument_errors_return_before_cuda():
     assert L.ht_lookup_or_insert(None, None, 0, None, None) == 1
     assert L.embbag_forward(None, None, 0, None, 0, None, None) == 1
     assert L.embbag_backward_update(None, None, 0, None, 0, None, C.c_float(0.1), None) == 1
+    assert L.embbag_forward_ex(None, None, 0, None, 0, None, 0, None, None) == 1
+    assert L.embbag_backward_update_ex(None, None, 0, None, 0, None, 1, None, C.c_float(0.1), None) == 1
     assert L.ht_sync(None) == 1
+    assert L.ht_set_hooks(None, 2, 1) == 1
+    n = C.c_int64()
+    assert L.ht_evict(None, 3, C.byref(n), None) == 1
+    assert L.ht_live_rows(None, C.byref(n)) == 1
     assert L.ht_row_stride(None) == -1
     # negative sizes
     assert L.dhs_pack_keys(None, None, -1, None, None) == 1

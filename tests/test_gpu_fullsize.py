@@ -67,6 +67,39 @@ def test_growth_stream_full_size():
     _run(gen.full("growth_stream"), steps=8, reserve=0)
 
 
+def test_growth_stream_all_steps_key_map():
+    """All 200 steps of the growth stream (forward + backward per step, the
+    table growing on demand from empty to about 3.2e7 rows: many IDMap
+    doublings and block appends) against the oracle's key -> row map over the
+    same key stream.  The map depends on the keys alone, not on dim or on the
+    optimizer, so the oracle runs at dim 4 and only its map is compared."""
+    w = gen.full("growth_stream")
+    t = dhs.ht_create(w.dim, w.optimizer, block_rows=w.block_rows, eps=w.eps, beta1=w.beta1, beta2=w.beta2)
+    o = Oracle(4, "sgd")
+    try:
+        for s in range(w.steps):
+            b = w.batch(s)
+            kg, ko = _pack(b)
+            og = dev(b.bag_offsets)
+            dhs.embbag_forward(t, kg, og)
+            dhs.embbag_backward_update(t, kg, og, w.torch_grads(s, b.n_bags, "cuda"), w.lr)
+            o.lookup_or_insert(ko)
+            if s % 50 == 49:
+                assert dhs.ht_sync(t) == 0, f"step {s}"
+        gk, _, rc = dhs.ht_export(t, rows=False)
+        assert rc == 0
+        ok_, _ = o.export()
+        assert gk.size == ok_.size == w.inserted_before(w.steps)
+        np.testing.assert_array_equal(gk, ok_)
+        c = dhs.ht_counters(t)
+        # the IDMap grew to hold the keys at load <= 0.5, and blocks cover every row
+        assert c["slots"] >= 2 * gk.size and c["rehashes"] >= 5
+        assert c["blocks"] >= -(-gk.size // w.block_rows)
+    finally:
+        t.close()
+        o.close()
+
+
 def test_tiny_uniform_full_size():
     _run(gen.full("tiny_uniform"), steps=10, reserve=0)
 

@@ -143,18 +143,25 @@ def test_forward_is_bit_exact():
         o.close()
 
 
-DIMS = [4, 12, 16, 32, 40, 64, 128, 132, 200, 260, 512]
+DIMS = [4, 8, 12, 16, 32, 40, 64, 128, 132, 200, 260, 512]
 
 
+@pytest.mark.parametrize("bags", ["long", "short"])
 @pytest.mark.parametrize("opt", ["sgd", "adagrad", "adam", "adagrad_rowwise"])
 @pytest.mark.parametrize("dim", DIMS)
-def test_dims_and_optimizers(dim, opt):
-    rng = np.random.default_rng(dim * 7 + len(opt))
+def test_dims_and_optimizers(dim, opt, bags):
+    """Every row width the kernels are instantiated for, with every optimizer.
+    Long bags (about 5.5 ids each) take the split forward (probe kernel, then
+    the gather from row references); short bags (about 1.5 ids each) the fused
+    probe + pool kernel.  Together the widths reach each (group, columns)
+    instantiation of both forward kernels and of both segment kernels."""
+    rng = np.random.default_rng(dim * 7 + len(opt) + (0 if bags == "long" else 1000))
     t, o = make_pair(dim, opt, block_rows=256)
     try:
+        dhs.ht_set_phase_timing(t, True)
         for s in range(3):
             nb = int(rng.integers(300, 900))
-            lens = rng.integers(0, 12, size=nb)
+            lens = rng.integers(0, 12 if bags == "long" else 4, size=nb)
             lens[rng.integers(0, nb, size=5)] = 0
             offs = np.concatenate([[0], np.cumsum(lens)]).astype(np.int64)
             n = int(offs[-1])
@@ -163,7 +170,10 @@ def test_dims_and_optimizers(dim, opt):
             grad = rng.standard_normal((nb, dim)).astype(np.float32)
             step_both(t, o, dev(keys), keys, offs, grad, 0.05)
         assert dhs.ht_sync(t) == 0
-        compare_tables(t, o, f"dim {dim} {opt}")
+        ph = dhs.ht_phase_times(t)
+        # the split forward runs its probe as a phase of its own; the fused one does not
+        assert (ph["fwd_probe"][1] == 3) == (bags == "long"), ph
+        compare_tables(t, o, f"dim {dim} {opt} {bags} bags")
     finally:
         t.close()
         o.close()
