@@ -6,8 +6,8 @@ batch of the 26-table DLRM-style merged workload (65,536 samples x 26 ids,
 pooling 1, dim 128 fp32, Adagrad, Zipf 1.05 ids; synthetic, seeded).  The
 table starts empty: warm-up steps are the stream's first steps, timed steps
 the ones after.  After the headline, the other four workloads (tiny uniform,
-sequence bags, growth stream, hot key) and the headline's stream on a table
-with bf16 weights are each run whole with their own step counts and reported
+sequence bags, growth stream, hot key) and the headline's and the sequence
+stream on tables with bf16 weights are each run whole with their own step counts and reported
 under "workloads", with capacity reserved before step 0; the growth stream
 runs a second time with its table growing on demand inside the timed steps
 ("growth_stream:on-demand").  "e2e" repeats the headline steps through the public
@@ -543,6 +543,7 @@ EXTRA_WORKLOADS = (
     ("growth_stream:on-demand", "growth_stream", "f32", "on-demand"),
     ("hot_key", "hot_key", "f32", "-1"),
     ("dlrm_merged_26:bf16", "dlrm_merged_26", "bf16", "-1"),
+    ("sequence_bags:bf16", "sequence_bags", "bf16", "-1"),
 )
 
 

@@ -72,8 +72,9 @@ namespace dhs {
 // the ends held in the lanes' registers).  Missing or negative keys get row
 // `sentinel` (sorted last, never updated).
 // Extended pooling (per-sample weights psw, or mean pooling): the sort value
-// is the position instead of the bag; bagpos[p] = its bag and mult[p] = the
-// factor its bag's gradient is scaled by (psw[p], or 1 / the bag's length).
+// is the position instead of the bag; bagpos[p] = its bag and mult[p] = its
+// weight psw[p] (the bag's gradient is multiplied by it) or, for mean
+// pooling, the bag's length (the gradient is divided by it).
 template <bool EXT>
 __global__ void __launch_bounds__(256)
 bwd_probe_kernel(IdMap m, const long long* __restrict__ keys, long long n_keys,
@@ -189,11 +190,11 @@ bwd_probe_kernel(IdMap m, const long long* __restrict__ keys, long long n_keys,
         const int beg0 = g0 > 0 ? prev0 : s, beg1 = g1 > 0 ? prev1 : s;
         if (p0 < E) {
           bagpos[p0] = (unsigned)(b0 + g0);
-          mult[p0] = psw ? (double)__ldg(psw + p0) : 1.0 / (double)(end0 - beg0);
+          mult[p0] = psw ? (double)__ldg(psw + p0) : (double)(end0 - beg0);
         }
         if (p1 < E) {
           bagpos[p1] = (unsigned)(b0 + g1);
-          mult[p1] = psw ? (double)__ldg(psw + p1) : 1.0 / (double)(end1 - beg1);
+          mult[p1] = psw ? (double)__ldg(psw + p1) : (double)(end1 - beg1);
         }
       }
     }
@@ -419,6 +420,13 @@ radix_onesweep_kernel(const unsigned* __restrict__ kin, const unsigned* __restri
 
 #endif  // DHS_TEMPLATES_ONLY
 
+// One occurrence's gradient term added in fp64 for extended pooling: x times
+// the weight, or x divided by the bag length (mean), each operation rounded
+// on its own (no fused multiply-add), as the plain definition computes it.
+__device__ __forceinline__ double ext_add(double acc, float x, double f, bool mean) {
+  return __dadd_rn(acc, mean ? __ddiv_rn((double)x, f) : __dmul_rn((double)x, f));
+}
+
 // ---------------------------------------------------------------------------
 // optimizer step on one row (fp32, each operation rounded)
 // ---------------------------------------------------------------------------
@@ -592,7 +600,7 @@ bwd_seg_kernel(const unsigned* __restrict__ skey, const unsigned* __restrict__ s
                double* __restrict__ part_head, double* __restrict__ part_tail,
                int C, unsigned* __restrict__ chunk_ctr,
                unsigned* __restrict__ owners, unsigned* __restrict__ owner_ctr, DevState* st,
-               const unsigned* __restrict__ bagpos, const double* __restrict__ mult) {
+               const unsigned* __restrict__ bagpos, const double* __restrict__ mult, bool mean) {
   constexpr int R = seg_ring(NV);
   extern __shared__ float4 seg_ring_smem[];
   const int lane = threadIdx.x & 31;
@@ -752,10 +760,10 @@ bwd_seg_kernel(const unsigned* __restrict__ skey, const unsigned* __restrict__ s
         for (int q = 0; q < NV; ++q) {
           const float4 x = slot[q * G + gl];
           if (EXT) {
-            acc[q][0] += (double)x.x * f;
-            acc[q][1] += (double)x.y * f;
-            acc[q][2] += (double)x.z * f;
-            acc[q][3] += (double)x.w * f;
+            acc[q][0] = ext_add(acc[q][0], x.x, f, mean);
+            acc[q][1] = ext_add(acc[q][1], x.y, f, mean);
+            acc[q][2] = ext_add(acc[q][2], x.z, f, mean);
+            acc[q][3] = ext_add(acc[q][3], x.w, f, mean);
           } else {
             acc[q][0] += (double)x.x;
             acc[q][1] += (double)x.y;
@@ -924,8 +932,9 @@ __device__ __forceinline__ void segw_st(float* p, const float (&v)[CPL], int col
 }
 
 // EXT (extended pooling): sort values are positions; the pair's bag is
-// bagpos[position] and its gradient row is scaled by mult[position] (a
-// per-sample weight, or 1 / the bag's length), both gathered once per chunk.
+// bagpos[position] and its gradient row is multiplied by mult[position] (a
+// per-sample weight) or, with mean, divided by it (the bag's length), both
+// gathered once per chunk.
 // BF: the table's weights are bf16 (state fp32): loaded widened, updated in
 // fp32, stored rounded to nearest even.
 template <int CPL, int OPT, bool EXT, bool BF>
@@ -935,7 +944,7 @@ bwd_segw_kernel(const unsigned* __restrict__ skey, const unsigned* __restrict__ 
                 double* __restrict__ part_head, double* __restrict__ part_tail, int pstride, int C,
                 unsigned* __restrict__ chunk_ctr, unsigned* __restrict__ owners,
                 unsigned* __restrict__ owner_ctr, DevState* st, bool grad_once,
-                const unsigned* __restrict__ bagpos, const double* __restrict__ mult) {
+                const unsigned* __restrict__ bagpos, const double* __restrict__ mult, bool mean) {
   constexpr int B = segw_batch(CPL);
   constexpr int PITCH = 32 * CPL;  // floats per staged row
   constexpr int NS = seg_state_arrays(OPT);
@@ -1276,7 +1285,7 @@ bwd_segw_kernel(const unsigned* __restrict__ skey, const unsigned* __restrict__ 
               if constexpr (EXT) {
                 const double f = segw_mult[wid][q];
 #pragma unroll
-                for (int e = 0; e < CPL; ++e) acc[e] += (double)x[e] * f;
+                for (int e = 0; e < CPL; ++e) acc[e] = ext_add(acc[e], x[e], f, mean);
               } else {
 #pragma unroll
                 for (int e = 0; e < CPL; ++e) acc[e] += (double)x[e];

@@ -571,7 +571,7 @@ int segw_cpl(int dim) {
 dhs_status launch_seg(dhs_table* t, const unsigned* sk, const unsigned* sv, long long n, const float* grad,
                       long long nb, const OptArgs& oa, double* part_head, double* part_tail,
                       unsigned* chunk_ctr, unsigned* owners, unsigned* owner_ctr, const unsigned* bagpos,
-                      const double* mult, cudaStream_t s) {
+                      const double* mult, bool mean, cudaStream_t s) {
   const int G = seg_group(t->dim), NV = seg_nv(t->dim);
   const int pstride = NV * G * 4;  // doubles per partial (>= dim)
   const bool ext = mult != nullptr;
@@ -582,14 +582,14 @@ dhs_status launch_seg(dhs_table* t, const unsigned* sk, const unsigned* sv, long
               : t->opt == DHS_ADAM ? (ext ? launch_seg_adam_ext_w : launch_seg_adam_w)
                                    : (ext ? launch_seg_rowwise_ext_w : launch_seg_rowwise_w);
     e = fn(segw_cpl(t->dim), t->wbf16, t->sm_count, sk, sv, n, grad, nb, t->dim, rowspace(t), oa, part_head,
-           part_tail, pstride, seg_chunk(n), chunk_ctr, owners, owner_ctr, t->st, bagpos, mult, s);
+           part_tail, pstride, seg_chunk(n), chunk_ctr, owners, owner_ctr, t->st, bagpos, mult, mean, s);
   } else {
     auto fn = t->opt == DHS_SGD ? (ext ? launch_seg_sgd_ext : launch_seg_sgd)
               : t->opt == DHS_ADAGRAD ? (ext ? launch_seg_adagrad_ext : launch_seg_adagrad)
               : t->opt == DHS_ADAM ? (ext ? launch_seg_adam_ext : launch_seg_adam)
                                    : (ext ? launch_seg_rowwise_ext : launch_seg_rowwise);
     e = fn(G, NV, t->sm_count, sk, sv, n, grad, nb, t->dim, rowspace(t), oa, part_head, part_tail,
-           seg_chunk(n), chunk_ctr, owners, owner_ctr, t->st, bagpos, mult, s);
+           seg_chunk(n), chunk_ctr, owners, owner_ctr, t->st, bagpos, mult, mean, s);
   }
   t->n_launches++;
   if (e != cudaSuccess) cudaGetLastError();
@@ -597,11 +597,11 @@ dhs_status launch_seg(dhs_table* t, const unsigned* sk, const unsigned* sv, long
 }
 
 dhs_status dispatch_seg(dhs_table* t, const unsigned* sk, const unsigned* sv, long long n,
-                        const float* grad, long long nb, const OptArgs& oa, bool ext, cudaStream_t s) {
+                        const float* grad, long long nb, const OptArgs& oa, bool ext, bool mean, cudaStream_t s) {
   return launch_seg(t, sk, sv, n, grad, nb, oa, (double*)t->b_ph.p, (double*)t->b_pt.p,
                     (unsigned*)t->b_hist.p + kSegChunkCtrWord, (unsigned*)t->b_owners.p,
                     (unsigned*)t->b_hist.p + kSegOwnerCtrWord, ext ? (const unsigned*)t->b_bagpos.p : nullptr,
-                    ext ? (const double*)t->b_mult.p : nullptr, s);
+                    ext ? (const double*)t->b_mult.p : nullptr, mean, s);
 }
 
 // offset assignment + row init for the new keys of an insert call
@@ -1020,7 +1020,7 @@ dhs_status embbag_backward_update_ex(dhs_table* t, const int64_t* d_keys, int64_
     oa.bc2 = (float)(1.0 - std::pow((double)t->b2, (double)t->adam_t));
     {
       PhaseScope ph(t, PH_BWD_SEG, s);
-      DHS_TRY(dispatch_seg(t, ka, va, n_keys, d_grad, n_bags, oa, ext, s));
+      DHS_TRY(dispatch_seg(t, ka, va, n_keys, d_grad, n_bags, oa, ext, mean, s));
     }
     PhaseScope ph(t, PH_BWD_COMBINE, s);
     const int pstride = seg_nv(t->dim) * seg_group(t->dim) * 4;
@@ -1419,7 +1419,7 @@ dhs_status embbag_backward_update_noalloc(dhs_table* t, const int64_t* d_keys, i
   const int G = seg_group(t->dim), NV = seg_nv(t->dim);
   const int chunk = seg_chunk(n_keys);
   DHS_TRY(launch_seg(t, ka, va, n_keys, d_grad, n_bags, oa, part_head, part_tail, hist + kSegChunkCtrWord, owners,
-                     hist + kSegOwnerCtrWord, nullptr, nullptr, s));
+                     hist + kSegOwnerCtrWord, nullptr, nullptr, false, s));
   t->n_launches += 2 + passes;
   return launch_combine(t, ka, n_keys, oa, part_head, part_tail, chunk, NV * G * 4, owners, hist, plan, s);
 }

@@ -41,14 +41,15 @@ cudaError_t launch_pool_refs_bf16(int G, int NV, int sm_count, RowSpace rs, int 
                                   cudaStream_t s);
 
 // bwd_seg_kernel<G, NV, OPT, EXT>, one entry point per optimizer and pooling
-// form (_ext: per-sample weights or mean pooling; bagpos / mult are used only
-// there)
+// form (_ext: per-sample weights or mean pooling; bagpos / mult / mean are
+// used only there)
 #define DHS_SEG_DECL(NAME_)                                                                     \
   cudaError_t NAME_(int G, int NV, int sm_count, const unsigned* skey, const unsigned* sval,    \
                     long long n, const float* grad, long long n_bags, int dim, RowSpace rs,     \
                     const OptArgs& oa, double* part_head, double* part_tail,                    \
                     int chunk, unsigned* chunk_ctr, unsigned* owners, unsigned* owner_ctr,      \
-                    DevState* st, const unsigned* bagpos, const double* mult, cudaStream_t s);
+                    DevState* st, const unsigned* bagpos, const double* mult, bool mean,        \
+                    cudaStream_t s);
 DHS_SEG_DECL(launch_seg_sgd)
 DHS_SEG_DECL(launch_seg_adagrad)
 DHS_SEG_DECL(launch_seg_adam)
@@ -66,7 +67,8 @@ DHS_SEG_DECL(launch_seg_rowwise_ext)
                     long long n, const float* grad, long long n_bags, int dim, RowSpace rs,     \
                     const OptArgs& oa, double* part_head, double* part_tail, int pstride,       \
                     int chunk, unsigned* chunk_ctr, unsigned* owners, unsigned* owner_ctr,      \
-                    DevState* st, const unsigned* bagpos, const double* mult, cudaStream_t s);
+                    DevState* st, const unsigned* bagpos, const double* mult, bool mean,        \
+                    cudaStream_t s);
 DHS_SEGW_DECL(launch_seg_sgd_w)
 DHS_SEGW_DECL(launch_seg_adagrad_w)
 DHS_SEGW_DECL(launch_seg_adam_w)

@@ -92,9 +92,14 @@ def test_eviction_and_row_reuse(dim, opt, admit):
     try:
         base = 0
         for step in range(12):
-            keys, offs = _batch(rng, 4000, 3000, short=step % 2 == 0)
-            keys = keys + base  # the key range drifts: old keys go idle
-            base += 4000 * 7919 // 3
+            # a drifting key range, so that old keys go idle; small calls
+            # until the first eviction (step 3) leaves tombstones, then calls
+            # whose claimed slots outgrow the initial IDMap of 32,768 keys,
+            # so that the rehash meets tombstones, counts and stamps
+            universe, bags = (3000, 1000) if step <= 3 else (30000, 6000)
+            keys, offs = _batch(rng, universe, bags, short=step % 2 == 0)
+            keys = keys + base
+            base += universe * 7919 // 3
             _step(t, o, keys, offs, dim, rng)
             if step in (3, 6, 9, 10):
                 max_idle = {3: 1, 6: 2, 9: 0, 10: 3}[step]
