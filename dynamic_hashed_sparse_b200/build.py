@@ -25,6 +25,9 @@ NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-I", INCLUDE,
          "--expt-relaxed-constexpr", "-diag-suppress", "177"]
+# Tuning overrides: DHS_DEFINES="DHS_RADIX_ITEMS=8 DHS_LOOKBACK_WINDOW=4" compiles
+# every source with those macros (the documented tuning macros of the kernels).
+DEFINES = ["-D" + d for d in os.environ.get("DHS_DEFINES", "").split()]
 
 
 def _sources():
@@ -38,6 +41,7 @@ def _deps():
 
 def _digest() -> str:
     h = hashlib.sha256()
+    h.update(" ".join(DEFINES).encode())
     for p in sorted(_deps()):
         h.update(os.path.basename(p).encode())
         with open(p, "rb") as f:
@@ -57,7 +61,7 @@ def up_to_date() -> bool:
 
 def _compile(src: str, verbose: bool) -> str:
     obj = os.path.join(OBJDIR, os.path.basename(src) + ".o")
-    cmd = [NVCC, *ARCH, *FLAGS, "-c", src, "-o", obj]
+    cmd = [NVCC, *ARCH, *FLAGS, *DEFINES, "-c", src, "-o", obj]
     if verbose:
         cmd.insert(1, "-Xptxas=-v")
     r = subprocess.run(cmd, capture_output=True, text=True)

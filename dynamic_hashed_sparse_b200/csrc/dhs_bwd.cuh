@@ -52,10 +52,9 @@
 #ifndef DHS_RADIX_MINB
 #define DHS_RADIX_MINB 3
 #endif
-//   DHS_HIST_MATCH    1: digit counts are combined per warp (match_any) before
-//                     the shared-memory atomic; 0: one atomic per key and pass
-#ifndef DHS_HIST_MATCH
-#define DHS_HIST_MATCH 0
+//   DHS_LOOKBACK_WINDOW predecessor tiles a radix pass's look-back reads at once
+#ifndef DHS_LOOKBACK_WINDOW
+#define DHS_LOOKBACK_WINDOW 8
 #endif
 
 namespace dhs {
@@ -65,6 +64,31 @@ namespace dhs {
 // ---------------------------------------------------------------------------
 
 #ifndef DHS_TEMPLATES_ONLY
+// ---------------------------------------------------------------------------
+// LSD radix sort of 32-bit keys with 32-bit values, 8-bit digits, stable,
+// one kernel per digit pass (decoupled look-back across tiles)
+// ---------------------------------------------------------------------------
+constexpr int kRadixThreads = 256;
+constexpr int kRadixItems = DHS_RADIX_ITEMS;
+constexpr int kRadixWarpItems = 32 * kRadixItems;
+constexpr int kRadixTile = kRadixWarpItems * (kRadixThreads / 32);
+constexpr int kRadixBins = 256;
+constexpr int kRadixMaxPasses = 4;
+constexpr unsigned long long kLbAggregate = 1ull << 62;  // tile count published
+constexpr unsigned long long kLbPrefix = 2ull << 62;     // inclusive prefix published
+constexpr unsigned long long kLbCountMask = (1ull << 62) - 1;
+constexpr unsigned kLookbackSpins = 1u << 22;  // bounded wait for a predecessor tile
+constexpr int kLookbackWindow = DHS_LOOKBACK_WINDOW;  // predecessors read per look-back step
+// words cleared (one memset) before a backward's probe: digit histograms of
+// every pass, one tile counter per pass, the segment kernel's chunk counter,
+// the count of long-segment owner chunks and the combine's batch and slot
+// counters
+constexpr int kSortZeroWords = kRadixMaxPasses * kRadixBins + kRadixMaxPasses + 4;
+constexpr int kSegChunkCtrWord = kRadixMaxPasses * kRadixBins + kRadixMaxPasses;
+constexpr int kSegOwnerCtrWord = kSegChunkCtrWord + 1;
+constexpr int kCombineBatchCtrWord = kSegChunkCtrWord + 2;
+constexpr int kCombineSlotCtrWord = kSegChunkCtrWord + 3;
+
 // Warp per chunk of bpc bags (64 when bags are short, 32 when they are long,
 // so that long bags still spread over enough warps); positions 64 at a time,
 // two per lane, so that each lane has two probes in flight.  A position's bag
@@ -80,14 +104,25 @@ __global__ void __launch_bounds__(256)
 bwd_probe_kernel(IdMap m, const long long* __restrict__ keys, long long n_keys,
                  const long long* __restrict__ bag_off, long long n_bags,
                  unsigned* __restrict__ rkey, unsigned* __restrict__ rval, unsigned sentinel,
-                 unsigned* __restrict__ sort_zero, int sort_zero_words, int bpc,
+                 unsigned* __restrict__ hist, int passes, unsigned long long* __restrict__ status0,
+                 long long status0_words, int bpc,
                  const float* __restrict__ psw, bool mean, unsigned* __restrict__ bagpos,
                  double* __restrict__ mult, DevState* st) {
   constexpr bool ext = EXT;
   constexpr unsigned FULL = 0xffffffffu;
   const int lane = threadIdx.x & 31;
-  if (blockIdx.x == 0)  // the sort's digit histograms and tile counters start at zero
-    for (int i = threadIdx.x; i < sort_zero_words; i += blockDim.x) sort_zero[i] = 0u;
+  // the sort's digit counts of every pass, taken here from the rows this
+  // kernel writes (hist is zero on entry); and the first pass's look-back
+  // words cleared
+  __shared__ unsigned h[kRadixMaxPasses][kRadixBins];
+  for (int i = threadIdx.x; i < kRadixMaxPasses * kRadixBins; i += blockDim.x) (&h[0][0])[i] = 0u;
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < status0_words;
+       i += (long long)gridDim.x * blockDim.x)
+    status0[i] = 0ull;
+  __syncthreads();
+  auto count = [&](unsigned k) {
+    for (int ps = 0; ps < passes; ++ps) atomicAdd(&h[ps][(k >> (8 * ps)) & 255u], 1u);
+  };
   // positions and bags fit in 31 bits (the host rejects larger calls)
   const int n = (int)n_keys;
   const long long nchunks = (n_bags + bpc - 1) / bpc;
@@ -170,12 +205,14 @@ bwd_probe_kernel(IdMap m, const long long* __restrict__ keys, long long n_keys,
         else if (f0 == -1) latch(st, kErrNotFound);
         rkey[p0] = f0 >= 0 ? (unsigned)f0 : sentinel;
         rval[p0] = ext ? (unsigned)p0 : (unsigned)(b0 + g0);
+        count(f0 >= 0 ? (unsigned)f0 : sentinel);
       }
       if (p1 < E) {
         if (k1 < 0) latch(st, kErrInvalid);
         else if (f1 == -1) latch(st, kErrNotFound);
         rkey[p1] = f1 >= 0 ? (unsigned)f1 : sentinel;
         rval[p1] = ext ? (unsigned)p1 : (unsigned)(b0 + g1);
+        count(f1 >= 0 ? (unsigned)f1 : sentinel);
       }
       if constexpr (EXT) {
         // bag g of the chunk spans [end(g - 1), end(g)), end(-1) = s
@@ -199,82 +236,13 @@ bwd_probe_kernel(IdMap m, const long long* __restrict__ keys, long long n_keys,
       }
     }
   }
-}
-
-// ---------------------------------------------------------------------------
-// LSD radix sort of 32-bit keys with 32-bit values, 8-bit digits, stable,
-// one kernel per digit pass (decoupled look-back across tiles)
-// ---------------------------------------------------------------------------
-constexpr int kRadixThreads = 256;
-constexpr int kRadixItems = DHS_RADIX_ITEMS;
-constexpr int kRadixWarpItems = 32 * kRadixItems;
-constexpr int kRadixTile = kRadixWarpItems * (kRadixThreads / 32);
-constexpr int kRadixBins = 256;
-constexpr int kRadixMaxPasses = 4;
-constexpr unsigned long long kLbAggregate = 1ull << 62;  // tile count published
-constexpr unsigned long long kLbPrefix = 2ull << 62;     // inclusive prefix published
-constexpr unsigned long long kLbCountMask = (1ull << 62) - 1;
-constexpr unsigned kLookbackSpins = 1u << 22;  // bounded wait for a predecessor tile
-// words cleared by bwd_probe_kernel before a backward: digit histograms of
-// every pass, one tile counter per pass, the segment kernel's chunk counter
-// the count of long-segment owner chunks and the combine's batch and slot
-// counters
-constexpr int kSortZeroWords = kRadixMaxPasses * kRadixBins + kRadixMaxPasses + 4;
-constexpr int kSegChunkCtrWord = kRadixMaxPasses * kRadixBins + kRadixMaxPasses;
-constexpr int kSegOwnerCtrWord = kSegChunkCtrWord + 1;
-constexpr int kCombineBatchCtrWord = kSegChunkCtrWord + 2;
-constexpr int kCombineSlotCtrWord = kSegChunkCtrWord + 3;
-
-// Digit counts of every pass in one read of the keys (global atomics, one per
-// block and bin), and the look-back state of every pass cleared.  hist and
-// tile_ctr must be zero on entry (bwd_probe_kernel clears them).
-__global__ void __launch_bounds__(kRadixThreads)
-radix_hist_all_kernel(const unsigned* __restrict__ keys, long long n, int passes,
-                      unsigned* __restrict__ hist, unsigned long long* __restrict__ status,
-                      long long status_words) {
-  __shared__ unsigned h[kRadixMaxPasses][kRadixBins];
-  for (int i = threadIdx.x; i < kRadixMaxPasses * kRadixBins; i += kRadixThreads) (&h[0][0])[i] = 0;
   __syncthreads();
-  const long long stride = (long long)gridDim.x * kRadixThreads;
-  // four keys per thread and step (one 16-byte load; the key array is 16-byte
-  // aligned), then the tail of n % 4 keys
-  const long long n4 = n >> 2;
-  const uint4* k4 = reinterpret_cast<const uint4*>(keys);
-  auto count = [&](unsigned k, bool ok) {
-#if DHS_HIST_MATCH
-    const int lane = threadIdx.x & 31;
-    for (int ps = 0; ps < passes; ++ps) {
-      const unsigned d = ok ? ((k >> (8 * ps)) & 255u) : 256u;
-      const unsigned peers = __match_any_sync(0xffffffffu, d);
-      if (d < 256u && (__ffs(peers) - 1) == lane) atomicAdd(&h[ps][d], (unsigned)__popc(peers));
-    }
-#else
-    if (ok)
-      for (int ps = 0; ps < passes; ++ps) atomicAdd(&h[ps][(k >> (8 * ps)) & 255u], 1u);
-#endif
-  };
-  for (long long base = (long long)blockIdx.x * kRadixThreads; base < n4; base += stride) {
-    const long long i = base + threadIdx.x;
-    const bool ok = i < n4;
-    const uint4 v = ok ? __ldg(k4 + i) : make_uint4(0u, 0u, 0u, 0u);
-    count(v.x, ok);
-    count(v.y, ok);
-    count(v.z, ok);
-    count(v.w, ok);
-  }
-  if (blockIdx.x == 0 && threadIdx.x < 32) {
-    const long long p = 4 * n4 + threadIdx.x;
-    const bool ok = p < n;  // at most 3 keys
-    count(ok ? __ldg(keys + p) : 0u, ok);
-  }
-  __syncthreads();
-  for (int i = threadIdx.x; i < passes * kRadixBins; i += kRadixThreads) {
+  for (int i = threadIdx.x; i < passes * kRadixBins; i += blockDim.x) {
     const unsigned v = (&h[0][0])[i];
     if (v) atomicAdd(hist + i, v);
   }
-  for (long long i = (long long)blockIdx.x * kRadixThreads + threadIdx.x; i < status_words; i += stride)
-    status[i] = 0ull;
 }
+
 
 // Block-wide exclusive scan of one value per thread (256 threads).
 __device__ __forceinline__ unsigned block_exclusive_scan_256(unsigned x, unsigned* wsum,
@@ -315,7 +283,7 @@ radix_onesweep_kernel(const unsigned* __restrict__ kin, const unsigned* __restri
                       unsigned* __restrict__ kout, unsigned* __restrict__ vout, long long n,
                       int shift, const unsigned* __restrict__ hist,
                       unsigned long long* __restrict__ status, unsigned* __restrict__ tile_ctr,
-                      DevState* st) {
+                      unsigned long long* __restrict__ next_status, long long next_words, DevState* st) {
   __shared__ unsigned s_k[kRadixTile];
   __shared__ unsigned s_v[kRadixTile];
   __shared__ unsigned wc[8][kRadixBins + 1];
@@ -325,26 +293,29 @@ radix_onesweep_kernel(const unsigned* __restrict__ kin, const unsigned* __restri
   __shared__ unsigned s_tile;
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
   if (threadIdx.x == 0) s_tile = atomicAdd(tile_ctr, 1u);
+  // the next pass's look-back words start at zero (that pass runs after this one)
+  for (long long i = (long long)blockIdx.x * kRadixThreads + threadIdx.x; i < next_words;
+       i += (long long)gridDim.x * kRadixThreads)
+    next_status[i] = 0ull;
   for (int i = threadIdx.x; i < 8 * (kRadixBins + 1); i += kRadixThreads) (&wc[0][0])[i] = 0;
   __syncthreads();
-  const long long tile = s_tile;
-  const long long tile0 = tile * kRadixTile;
-  const int tile_n = (int)max(0ll, min((long long)kRadixTile, n - tile0));
+  // positions fit in 31 bits (the host rejects larger calls)
+  const int tile = (int)s_tile;
+  const int tile0 = tile * kRadixTile;
+  const int tile_n = max(0, min(kRadixTile, (int)n - tile0));
+  // items r * 32 + lane of this warp are in range below rem
+  const int rem = tile_n - wid * kRadixWarpItems;
 
-  unsigned k[kRadixItems], v[kRadixItems], lr[kRadixItems];
-  const long long base = tile0 + (long long)wid * kRadixWarpItems;
+  // keys now; values only when they are placed (fewer registers held)
+  unsigned k[kRadixItems], lr[kRadixItems];
+  const unsigned* kb = kin + tile0 + wid * kRadixWarpItems + lane;
+  const unsigned* vb = vin + tile0 + wid * kRadixWarpItems + lane;
 #pragma unroll
-  for (int r = 0; r < kRadixItems; ++r) {
-    const long long p = base + r * 32 + lane;
-    const bool ok = p < n;
-    k[r] = ok ? __ldg(kin + p) : 0u;
-    v[r] = ok ? __ldg(vin + p) : 0u;
-  }
+  for (int r = 0; r < kRadixItems; ++r) k[r] = r * 32 + lane < rem ? __ldg(kb + r * 32) : 0u;
   const unsigned lt = lanemask_lt();
 #pragma unroll
   for (int r = 0; r < kRadixItems; ++r) {
-    const long long p = base + r * 32 + lane;
-    const unsigned d = p < n ? ((k[r] >> shift) & 255u) : 256u;
+    const unsigned d = r * 32 + lane < rem ? ((k[r] >> shift) & 255u) : 256u;
     const unsigned peers = __match_any_sync(0xffffffffu, d);
     const unsigned before = wc[wid][d];
     lr[r] = before + __popc(peers & lt);
@@ -361,53 +332,67 @@ radix_onesweep_kernel(const unsigned* __restrict__ kin, const unsigned* __restri
     wc[w][d] = cnt;
     cnt += t;
   }
-  // publish this tile's count of digit d, then look back over the predecessors
-  volatile unsigned long long* sp = status + tile * kRadixBins + d;
+  // publish this tile's count of digit d at once; the tile's items go to
+  // shared memory in digit order before the look-back, so that no item is
+  // held in registers while it waits
+  volatile unsigned long long* sp = status + (long long)tile * kRadixBins + d;
   if (tile == 0) {
     *sp = kLbPrefix | cnt;
   } else {
     *sp = kLbAggregate | cnt;
   }
-  unsigned long long excl = 0;
-  if (tile > 0) {
-    long long t = tile - 1;
-    unsigned spins = 0;
-    while (t >= 0) {
-      const unsigned long long sv = *(volatile unsigned long long*)(status + t * kRadixBins + d);
-      if (sv & kLbPrefix) {
-        excl += sv & kLbCountMask;
-        break;
-      }
-      if (sv & kLbAggregate) {
-        excl += sv & kLbCountMask;
-        --t;
-        continue;
-      }
-      if (++spins > kLookbackSpins) {
-        latch(st, kErrInternal);
-        break;
-      }
-      __nanosleep(32);
-    }
-    *sp = kLbPrefix | (excl + cnt);
-  }
+  unsigned dpre;
   {
     unsigned tot;
-    const unsigned dpre = block_exclusive_scan_256(hist[d], wsum, tot);
-    gbase[d] = dpre + (unsigned)excl;
+    dpre = block_exclusive_scan_256(hist[d], wsum, tot);
     dstart[d] = block_exclusive_scan_256(cnt, wsum, tot);
   }
   __syncthreads();
 #pragma unroll
   for (int r = 0; r < kRadixItems; ++r) {
-    const long long p = base + r * 32 + lane;
-    if (p < n) {
+    if (r * 32 + lane < rem) {
       const unsigned dd = (k[r] >> shift) & 255u;
       const unsigned pos = dstart[dd] + wc[wid][dd] + lr[r];
       s_k[pos] = k[r];
-      s_v[pos] = v[r];
+      s_v[pos] = __ldg(vb + r * 32);
     }
   }
+  unsigned long long excl = 0;
+  if (tile > 0) {
+    // kLookbackWindow predecessors are read at once (independent loads in
+    // flight together) and taken in order until a prefix, or a tile that has
+    // not published yet, is met; tile 0 always publishes a prefix, so the
+    // walk never passes it
+    int t = tile - 1;
+    unsigned spins = 0;
+    for (;;) {
+      unsigned long long sv[kLookbackWindow];
+#pragma unroll
+      for (int i = 0; i < kLookbackWindow; ++i)
+        sv[i] = t - i >= 0 ? *(volatile unsigned long long*)(status + (long long)(t - i) * kRadixBins + d) : 0ull;
+      int used = 0;
+      bool done = false;
+#pragma unroll
+      for (int i = 0; i < kLookbackWindow; ++i) {
+        if (!done && used == i && (sv[i] & (kLbPrefix | kLbAggregate))) {
+          excl += sv[i] & kLbCountMask;
+          if (sv[i] & kLbPrefix) done = true;
+          else used = i + 1;
+        }
+      }
+      if (done) break;
+      t -= used;
+      if (used == 0) {
+        if (++spins > kLookbackSpins || t < 0) {
+          latch(st, kErrInternal);
+          break;
+        }
+        __nanosleep(32);
+      }
+    }
+    *sp = kLbPrefix | (excl + cnt);
+  }
+  gbase[d] = dpre + (unsigned)excl;
   __syncthreads();
   for (int i = threadIdx.x; i < tile_n; i += kRadixThreads) {
     const unsigned key = s_k[i];
@@ -1350,8 +1335,15 @@ __device__ __forceinline__ void finish_run_warp(float* row, int dim, int wfl, co
     const int j = lane + 32 * i;
     g[i] = 0.f;
     if (j < dim) {
-      double a = __ldcg(first + j);
-      for (long long k = 1; k < npieces; ++k) a += __ldcg(rest + (k - 1) * pstride + j);
+      // every piece of the column in flight at once, then added in order
+      double v[kWarpFinishPieces];
+      v[0] = __ldcg(first + j);
+#pragma unroll
+      for (int k = 1; k < kWarpFinishPieces; ++k) v[k] = k < npieces ? __ldcg(rest + (k - 1) * pstride + j) : 0.0;
+      double a = v[0];
+#pragma unroll
+      for (int k = 1; k < kWarpFinishPieces; ++k)
+        if (k < npieces) a += v[k];
       g[i] = (float)a;
       const double gd = (double)g[i];
       sq += gd * gd;

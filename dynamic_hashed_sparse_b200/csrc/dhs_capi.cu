@@ -973,15 +973,21 @@ dhs_status embbag_backward_update_ex(dhs_table* t, const int64_t* d_keys, int64_
   unsigned* vb = (unsigned*)t->b_vb.p;
   {
     PhaseScope ph(t, PH_BWD_PROBE, s);
-    // a warp per chunk of bags, all launched at once: the SMs overlap the
-    // chunks' dependent loads (bag ends, keys, slots) across many warps
+    // one resident wave of blocks, each warp taking chunks of bags in turn:
+    // each block flushes its digit counts with one atomic per nonzero bin,
+    // so fewer blocks mean fewer atomics on the shared counters
+    const int resident = resident_blocks(ext ? bwd_probe_kernel<true> : bwd_probe_kernel<false>, 256, 0,
+                                         t->sm_count);
     const int bpc = bwd_probe_bags(n_keys, n_bags);
     const long long warps = (n_bags + bpc - 1) / bpc;
-    const long long grid = std::max<long long>(1, (warps + 7) / 8);
+    const long long grid = grid_for((warps + 7) / 8, resident);
+    const long long ntiles = (n_keys + kRadixTile - 1) / kRadixTile;
+    // the counters the probe and the sort accumulate into start at zero
+    DHS_CUDA(cudaMemsetAsync(t->b_hist.p, 0, (size_t)kSortZeroWords * 4, s));
     (ext ? bwd_probe_kernel<true> : bwd_probe_kernel<false>)<<<(unsigned)grid, 256, 0, s>>>(
         idmap(t), (const long long*)d_keys, n_keys, (const long long*)d_bag_offsets, n_bags, ka, va, sentinel,
-        (unsigned*)t->b_hist.p, kSortZeroWords, bpc, psw, mean, (unsigned*)t->b_bagpos.p, (double*)t->b_mult.p,
-        t->st);
+        (unsigned*)t->b_hist.p, passes, (unsigned long long*)t->b_totals.p, ntiles * kRadixBins, bpc, psw, mean,
+        (unsigned*)t->b_bagpos.p, (double*)t->b_mult.p, t->st);
     t->n_launches++;
     DHS_TRY(last_launch());
   }
@@ -991,16 +997,11 @@ dhs_status embbag_backward_update_ex(dhs_table* t, const int64_t* d_keys, int64_
     unsigned* hist = (unsigned*)t->b_hist.p;
     unsigned* tile_ctr = hist + kRadixMaxPasses * kRadixBins;
     unsigned long long* status = (unsigned long long*)t->b_totals.p;
-    const long long hgrid = std::min<long long>((n_keys + kRadixThreads - 1) / kRadixThreads,
-                                                (long long)t->sm_count * 8);
-    radix_hist_all_kernel<<<(unsigned)hgrid, kRadixThreads, 0, s>>>(
-        ka, n_keys, passes, hist, status, (long long)passes * ntiles * kRadixBins);
-    t->n_launches++;
-    DHS_TRY(last_launch());
     for (int p = 0; p < passes; ++p) {
+      const long long words = ntiles * kRadixBins;
       radix_onesweep_kernel<<<(unsigned)ntiles, kRadixThreads, 0, s>>>(
-          ka, va, kb, vb, n_keys, 8 * p, hist + p * kRadixBins, status + (long long)p * ntiles * kRadixBins,
-          tile_ctr + p, t->st);
+          ka, va, kb, vb, n_keys, 8 * p, hist + p * kRadixBins, status + (long long)p * words, tile_ctr + p,
+          status + (long long)(p + 1) * words, p + 1 < passes ? words : 0, t->st);
       t->n_launches++;
       DHS_TRY(last_launch());
       std::swap(ka, kb);
@@ -1383,24 +1384,23 @@ dhs_status embbag_backward_update_noalloc(dhs_table* t, const int64_t* d_keys, i
   {
     const int bpc = bwd_probe_bags(n_keys, n_bags);
     const long long warps = (n_bags + bpc - 1) / bpc;
-    const long long grid = std::max<long long>(1, std::min<long long>((warps + 7) / 8, (long long)t->sm_count * 8));
+    const long long grid = grid_for((warps + 7) / 8, resident_blocks(bwd_probe_kernel<false>, 256, 0, t->sm_count));
+    const long long ntiles = (n_keys + kRadixTile - 1) / kRadixTile;
+    // the shared array keeps the last call's counters: they start at zero
+    DHS_CUDA(cudaMemsetAsync(hist, 0, (size_t)kSortZeroWords * 4, s));
     bwd_probe_kernel<false><<<(unsigned)grid, 256, 0, s>>>(idmap(t), (const long long*)d_keys, n_keys,
                                                     (const long long*)d_bag_offsets, n_bags, ka, va,
-                                                    sentinel, hist, kSortZeroWords, bpc, nullptr, false,
-                                                    nullptr, nullptr, t->st);
+                                                    sentinel, hist, passes, status, ntiles * kRadixBins, bpc,
+                                                    nullptr, false, nullptr, nullptr, t->st);
     DHS_TRY(last_launch());
   }
   const long long ntiles = (n_keys + kRadixTile - 1) / kRadixTile;
   {
-    const long long hgrid = std::min<long long>((n_keys + kRadixThreads - 1) / kRadixThreads,
-                                                (long long)t->sm_count * 8);
-    radix_hist_all_kernel<<<(unsigned)hgrid, kRadixThreads, 0, s>>>(
-        ka, n_keys, passes, hist, status, (long long)passes * ntiles * kRadixBins);
-    DHS_TRY(last_launch());
     for (int p = 0; p < passes; ++p) {
+      const long long words = ntiles * kRadixBins;
       radix_onesweep_kernel<<<(unsigned)ntiles, kRadixThreads, 0, s>>>(
-          ka, va, kb, vb, n_keys, 8 * p, hist + p * kRadixBins, status + (long long)p * ntiles * kRadixBins,
-          tile_ctr + p, t->st);
+          ka, va, kb, vb, n_keys, 8 * p, hist + p * kRadixBins, status + (long long)p * words, tile_ctr + p,
+          status + (long long)(p + 1) * words, p + 1 < passes ? words : 0, t->st);
       DHS_TRY(last_launch());
       std::swap(ka, kb);
       std::swap(va, vb);
@@ -1420,7 +1420,7 @@ dhs_status embbag_backward_update_noalloc(dhs_table* t, const int64_t* d_keys, i
   const int chunk = seg_chunk(n_keys);
   DHS_TRY(launch_seg(t, ka, va, n_keys, d_grad, n_bags, oa, part_head, part_tail, hist + kSegChunkCtrWord, owners,
                      hist + kSegOwnerCtrWord, nullptr, nullptr, false, s));
-  t->n_launches += 2 + passes;
+  t->n_launches += 1 + passes;
   return launch_combine(t, ka, n_keys, oa, part_head, part_tail, chunk, NV * G * 4, owners, hist, plan, s);
 }
 
