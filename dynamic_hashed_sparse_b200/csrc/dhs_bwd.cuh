@@ -52,6 +52,11 @@
 #ifndef DHS_RADIX_MINB
 #define DHS_RADIX_MINB 3
 #endif
+//   DHS_SEG_FINISH_PIECES pieces of a long segment the segment kernel's warp
+//                     adds itself (longer ones go to the combine kernels)
+#ifndef DHS_SEG_FINISH_PIECES
+#define DHS_SEG_FINISH_PIECES 256
+#endif
 //   DHS_LOOKBACK_WINDOW predecessor tiles a radix pass's look-back reads at once
 #ifndef DHS_LOOKBACK_WINDOW
 #define DHS_LOOKBACK_WINDOW 8
@@ -105,20 +110,23 @@ bwd_probe_kernel(IdMap m, const long long* __restrict__ keys, long long n_keys,
                  const long long* __restrict__ bag_off, long long n_bags,
                  unsigned* __restrict__ rkey, unsigned* __restrict__ rval, unsigned sentinel,
                  unsigned* __restrict__ hist, int passes, unsigned long long* __restrict__ status0,
-                 long long status0_words, int bpc,
+                 long long status0_words, unsigned* __restrict__ zero32, long long zero32_words, int bpc,
                  const float* __restrict__ psw, bool mean, unsigned* __restrict__ bagpos,
                  double* __restrict__ mult, DevState* st) {
   constexpr bool ext = EXT;
   constexpr unsigned FULL = 0xffffffffu;
   const int lane = threadIdx.x & 31;
   // the sort's digit counts of every pass, taken here from the rows this
-  // kernel writes (hist is zero on entry); and the first pass's look-back
-  // words cleared
+  // kernel writes (hist is zero on entry); the first pass's look-back words
+  // and the segment kernel's arrival table (zero32) cleared
   __shared__ unsigned h[kRadixMaxPasses][kRadixBins];
   for (int i = threadIdx.x; i < kRadixMaxPasses * kRadixBins; i += blockDim.x) (&h[0][0])[i] = 0u;
   for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < status0_words;
        i += (long long)gridDim.x * blockDim.x)
     status0[i] = 0ull;
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < zero32_words;
+       i += (long long)gridDim.x * blockDim.x)
+    zero32[i] = 0u;
   __syncthreads();
   auto count = [&](unsigned k) {
     for (int ps = 0; ps < passes; ++ps) atomicAdd(&h[ps][(k >> (8 * ps)) & 255u], 1u);
@@ -916,6 +924,23 @@ __device__ __forceinline__ void segw_st(float* p, const float (&v)[CPL], int col
   }
 }
 
+// Arrival sums of long segments: see the segment kernel's close step.
+constexpr unsigned kRunBias = 1u << 30;
+
+// Entry of row in the arrival table (inserted when absent); ~0u after
+// latching kErrInternal when the table is full (it is sized for every long
+// segment of sorted input, so only a failed sort gets there).
+__device__ __forceinline__ unsigned run_slot(const RunTable& rt, unsigned row, DevState* st) {
+  unsigned h = (row * 0x9E3779B1u) & rt.mask;  // Fibonacci hashing of the row
+  for (unsigned i = 0; i <= rt.mask; ++i) {
+    const unsigned old = atomicCAS(rt.key + h, 0u, row + 1u);
+    if (old == 0u || old == row + 1u) return h;
+    h = (h + 1u) & rt.mask;
+  }
+  latch(st, kErrInternal);
+  return ~0u;
+}
+
 // EXT (extended pooling): sort values are positions; the pair's bag is
 // bagpos[position] and its gradient row is multiplied by mult[position] (a
 // per-sample weight) or, with mean, divided by it (the bag's length), both
@@ -929,7 +954,8 @@ bwd_segw_kernel(const unsigned* __restrict__ skey, const unsigned* __restrict__ 
                 double* __restrict__ part_head, double* __restrict__ part_tail, int pstride, int C,
                 unsigned* __restrict__ chunk_ctr, unsigned* __restrict__ owners,
                 unsigned* __restrict__ owner_ctr, DevState* st, bool grad_once,
-                const unsigned* __restrict__ bagpos, const double* __restrict__ mult, bool mean) {
+                const unsigned* __restrict__ bagpos, const double* __restrict__ mult, bool mean,
+                RunTable rt) {
   constexpr int B = segw_batch(CPL);
   constexpr int PITCH = 32 * CPL;  // floats per staged row
   constexpr int NS = seg_state_arrays(OPT);
@@ -1149,6 +1175,98 @@ bwd_segw_kernel(const unsigned* __restrict__ skey, const unsigned* __restrict__ 
         if (OPT == 3) nra = row[wfl];
       }
     };
+    // the optimizer step on the row of kcur with the gradient in acc and the
+    // row's values in rw / rst / racc
+    auto update_row = [&](float* row) {
+      float den = 0.f, Gn = 0.f;
+      if (OPT == 3) {
+        double sq = 0.0;
+#pragma unroll
+        for (int e = 0; e < CPL; ++e) {
+          if (lane_on && col0 + e < dim) {
+            const double g = (double)(float)acc[e];
+            sq += g * g;
+          }
+        }
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) sq += __shfl_xor_sync(FULL, sq, o);
+        Gn = __fadd_rn(racc, (float)(sq / (double)dim));
+        den = __fadd_rn(__fsqrt_rn(Gn), oa.eps);
+      }
+      if (lane_on) {
+#pragma unroll
+        for (int e = 0; e < CPL; ++e) {
+          const float g = (float)acc[e];
+          if (OPT == 0) {
+            rw[e] = sgd_w(rw[e], g, oa.lr);
+          } else if (OPT == 1) {
+            adagrad_step(rw[e], rst[0][e], g, oa.lr, oa.eps);
+          } else if (OPT == 2) {
+            adam_step(rw[e], rst[0][e], rst[NS - 1][e], g, oa);
+          } else {
+            rw[e] = __fsub_rn(rw[e], __fdiv_rn(__fmul_rn(oa.lr, g), den));
+          }
+        }
+        if constexpr (BF)
+          segw_st_bf<CPL>(row, rw, col0, dim);
+        else
+          segw_st<CPL>(row, rw, col0, dim);
+#pragma unroll
+        for (int k = 0; k < NS; ++k) segw_st<CPL>(row + wfl + k * dim, rst[k], col0, dim);
+      }
+      if (OPT == 3 && lane == 0) row[wfl] = Gn;
+    };
+    // the warp that brings the last piece of a long segment finishes it: the
+    // pieces (the first chunk's tail partial, then each later chunk's head
+    // partial) added in chunk order into acc, then the optimizer step
+    auto finish_long = [&](unsigned f0, unsigned np) {
+      constexpr int FB = CPL <= 2 ? 8 : (CPL == 4 ? 4 : (CPL == 8 ? 2 : 1));  // pieces in flight
+#pragma unroll
+      for (int e = 0; e < CPL; ++e) acc[e] = 0.0;
+      if (lane_on) {
+        for (unsigned k0 = 0; k0 < np; k0 += FB) {
+          double v[FB][CPL];
+#pragma unroll
+          for (int i = 0; i < FB; ++i) {
+            const unsigned k = k0 + (unsigned)i;
+            const double* src =
+                (k == 0 ? part_tail + (long long)f0 * pstride : part_head + (long long)(f0 + k) * pstride) + col0;
+            if constexpr (CPL == 1) {
+              v[i][0] = k < np ? __ldcg(src) : 0.0;
+            } else {
+#pragma unroll
+              for (int e = 0; e < CPL; e += 2) {
+                const double2 x = k < np && col0 + e < dim ? __ldcg(reinterpret_cast<const double2*>(src + e))
+                                                           : make_double2(0.0, 0.0);
+                v[i][e] = x.x;
+                v[i][e + 1] = x.y;
+              }
+            }
+          }
+#pragma unroll
+          for (int i = 0; i < FB; ++i)
+            if (k0 + (unsigned)i < np)
+#pragma unroll
+              for (int e = 0; e < CPL; ++e) acc[e] += v[i][e];
+        }
+      }
+      float* row = rs.row(kcur);
+      if (lane_on) {
+        if constexpr (BF)
+          segw_ld_bf<CPL>(rw, row, col0, dim);
+        else
+          segw_ld<CPL>(rw, row, col0, dim);
+#pragma unroll
+        for (int k = 0; k < NS; ++k) segw_ld<CPL>(rst[k], row + wfl + k * dim, col0, dim);
+      }
+      if (OPT == 3) racc = row[wfl];
+      update_row(row);
+    };
+    auto add_owner = [&](unsigned oc) {  // for the combine kernels
+      const unsigned slot = atomicAdd(owner_ctr, 1u);
+      if (slot < (unsigned)nchunks) owners[slot] = oc;
+      else latch(st, kErrInternal);
+    };
     auto close = [&]() {
       if (mode == 1 || mode == 3) {
         double* o = (mode == 1 ? part_head : part_tail) + (long long)c * pstride + col0;
@@ -1157,50 +1275,47 @@ bwd_segw_kernel(const unsigned* __restrict__ skey, const unsigned* __restrict__ 
           for (int e = 0; e < CPL; ++e)
             if (col0 + e < dim) o[e] = acc[e];
         }
-        if (mode == 3 && lane == 0) {  // for the combine; at most one per chunk for sorted pairs
-          const unsigned slot = atomicAdd(owner_ctr, 1u);
-          if (slot < (unsigned)nchunks) owners[slot] = (unsigned)c;
-          else latch(st, kErrInternal);
+        if (rt.key != nullptr && kcur < nrows) {
+          // arrival: the owner adds 1 + c + bias, the chunk where the segment
+          // ends 1 + bias - c, every other piece 1; the sum reaches
+          // 1 + 2 bias exactly when all c1 - c0 + 1 pieces have arrived, in
+          // whatever order (no partial sum can reach it: chunks < 2^26)
+          __threadfence();  // this lane's partial before the arrival
+          __syncwarp();
+          unsigned fin = 0, slot = 0;
+          if (lane == 0) {
+            const bool is_end = mode == 1 && (run_end < cend || fwd1 != kcur);
+            unsigned add = 1u;
+            if (mode == 3) add += (unsigned)c + kRunBias;
+            if (is_end) add += kRunBias - (unsigned)c;
+            slot = run_slot(rt, kcur, st);
+            if (slot != ~0u) {
+              if (mode == 3) *(volatile unsigned*)(rt.c0 + slot) = (unsigned)c;
+              if (is_end) *(volatile unsigned*)(rt.c1 + slot) = (unsigned)c;
+              __threadfence();
+              const unsigned old = atomicAdd(rt.ctr + slot, add);
+              fin = old + add == 1u + 2u * kRunBias ? 1u : 0u;
+            }
+          }
+          fin = __shfl_sync(FULL, fin, 0);
+          if (fin) {
+            slot = __shfl_sync(FULL, slot, 0);
+            __threadfence();
+            const unsigned f0 = *(volatile unsigned*)(rt.c0 + slot);
+            const unsigned f1 = *(volatile unsigned*)(rt.c1 + slot);
+            if (f1 < f0 || f1 >= (unsigned)nchunks) {
+              if (lane == 0) latch(st, kErrInternal);
+            } else if (f1 - f0 + 1u <= rt.max_pieces) {
+              finish_long(f0, f1 - f0 + 1u);
+            } else if (lane == 0) {
+              add_owner(f0);
+            }
+          }
+        } else if (mode == 3 && lane == 0) {  // at most one per chunk for sorted pairs
+          add_owner((unsigned)c);
         }
       } else if (mode == 2 && kcur < nrows) {
-        float* row = rs.row(kcur);
-        float den = 0.f, Gn = 0.f;
-        if (OPT == 3) {
-          double sq = 0.0;
-#pragma unroll
-          for (int e = 0; e < CPL; ++e) {
-            if (lane_on && col0 + e < dim) {
-              const double g = (double)(float)acc[e];
-              sq += g * g;
-            }
-          }
-#pragma unroll
-          for (int o = 1; o < 32; o <<= 1) sq += __shfl_xor_sync(FULL, sq, o);
-          Gn = __fadd_rn(racc, (float)(sq / (double)dim));
-          den = __fadd_rn(__fsqrt_rn(Gn), oa.eps);
-        }
-        if (lane_on) {
-#pragma unroll
-          for (int e = 0; e < CPL; ++e) {
-            const float g = (float)acc[e];
-            if (OPT == 0) {
-              rw[e] = sgd_w(rw[e], g, oa.lr);
-            } else if (OPT == 1) {
-              adagrad_step(rw[e], rst[0][e], g, oa.lr, oa.eps);
-            } else if (OPT == 2) {
-              adam_step(rw[e], rst[0][e], rst[NS - 1][e], g, oa);
-            } else {
-              rw[e] = __fsub_rn(rw[e], __fdiv_rn(__fmul_rn(oa.lr, g), den));
-            }
-          }
-          if constexpr (BF)
-            segw_st_bf<CPL>(row, rw, col0, dim);
-          else
-            segw_st<CPL>(row, rw, col0, dim);
-#pragma unroll
-          for (int k = 0; k < NS; ++k) segw_st<CPL>(row + wfl + k * dim, rst[k], col0, dim);
-        }
-        if (OPT == 3 && lane == 0) row[wfl] = Gn;
+        update_row(rs.row(kcur));
       }
 #pragma unroll
       for (int e = 0; e < CPL; ++e) acc[e] = 0.0;

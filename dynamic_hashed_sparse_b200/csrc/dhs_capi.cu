@@ -178,7 +178,8 @@ struct dhs_table {
   long long ws_n = -1;
   long long ws_chunks = 0;  // chunk capacity of the segment and combine buffers
   Buf b_nbm, b_fbm, b_gcnt, b_gpref, b_slotpos, b_ka, b_va, b_kb, b_vb, b_hist, b_totals, b_ph,
-      b_pt, b_owners, b_cplan, b_slots, b_refs, b_bagpos, b_mult;
+      b_pt, b_owners, b_cplan, b_slots, b_refs, b_bagpos, b_mult, b_runs;
+  long long ws_run_cap = 0;  // entries of the long-segment arrival table
 
   bool timing = false;
   std::vector<PhaseRec> recs;
@@ -457,6 +458,19 @@ constexpr long long combine_batch_cap(long long nchunks) {
 }
 constexpr long long combine_slot_cap(long long nchunks) { return 4 * nchunks / kCombineMinPieces + 64; }
 
+// Entries of the arrival table of a backward over nchunks sort chunks: a
+// power of two of at least nchunks + 2, so that the long segments (each spans
+// three chunks or more, so there are at most nchunks / 2 + 1) fill at most
+// about half of it.
+long long run_table_cap(long long nchunks) {
+  long long c = 64;
+  while (c < nchunks + 2) c <<= 1;
+  return c;
+}
+// Pieces of a long segment that the segment kernel's warp adds itself; longer
+// segments go to the combine kernels.
+constexpr unsigned kSegFinishPieces = DHS_SEG_FINISH_PIECES;
+
 // The plan arrays cut from one buffer of 6 nchunks + batch cap words.
 CombinePlan combine_plan(unsigned* words, double* slots, long long nchunks, unsigned* zeroed) {
   CombinePlan pl;
@@ -503,6 +517,10 @@ dhs_status ensure_ws(dhs_table* t, long long n, cudaStream_t s) {
   DHS_TRY(bget(t, t->b_owners, nchunks * 4, s));
   DHS_TRY(bget(t, t->b_cplan, (size_t)(6 * nchunks + combine_batch_cap(nchunks)) * 4, s));
   DHS_TRY(bget(t, t->b_slots, (size_t)combine_slot_cap(nchunks) * pstride * 8, s));
+  // arrival table: key, ctr, c0, c1 arrays of run_table_cap entries each
+  const long long rcap = run_table_cap(nchunks);
+  DHS_TRY(bget(t, t->b_runs, (size_t)4 * rcap * 4, s));
+  t->ws_run_cap = rcap;
   DHS_CUDA(cudaMemsetAsync(t->b_nbm.p, 0, t->b_nbm.bytes, s));
   t->ws_n = cap;
   t->ws_chunks = nchunks;
@@ -571,7 +589,7 @@ int segw_cpl(int dim) {
 dhs_status launch_seg(dhs_table* t, const unsigned* sk, const unsigned* sv, long long n, const float* grad,
                       long long nb, const OptArgs& oa, double* part_head, double* part_tail,
                       unsigned* chunk_ctr, unsigned* owners, unsigned* owner_ctr, const unsigned* bagpos,
-                      const double* mult, bool mean, cudaStream_t s) {
+                      const double* mult, bool mean, const RunTable& rt, cudaStream_t s) {
   const int G = seg_group(t->dim), NV = seg_nv(t->dim);
   const int pstride = NV * G * 4;  // doubles per partial (>= dim)
   const bool ext = mult != nullptr;
@@ -582,7 +600,7 @@ dhs_status launch_seg(dhs_table* t, const unsigned* sk, const unsigned* sv, long
               : t->opt == DHS_ADAM ? (ext ? launch_seg_adam_ext_w : launch_seg_adam_w)
                                    : (ext ? launch_seg_rowwise_ext_w : launch_seg_rowwise_w);
     e = fn(segw_cpl(t->dim), t->wbf16, t->sm_count, sk, sv, n, grad, nb, t->dim, rowspace(t), oa, part_head,
-           part_tail, pstride, seg_chunk(n), chunk_ctr, owners, owner_ctr, t->st, bagpos, mult, mean, s);
+           part_tail, pstride, seg_chunk(n), chunk_ctr, owners, owner_ctr, t->st, bagpos, mult, mean, rt, s);
   } else {
     auto fn = t->opt == DHS_SGD ? (ext ? launch_seg_sgd_ext : launch_seg_sgd)
               : t->opt == DHS_ADAGRAD ? (ext ? launch_seg_adagrad_ext : launch_seg_adagrad)
@@ -596,12 +614,27 @@ dhs_status launch_seg(dhs_table* t, const unsigned* sk, const unsigned* sv, long
   return e == cudaSuccess ? DHS_OK : DHS_ERR_CUDA;
 }
 
+// The arrival table of a backward of n ids (its key and ctr arrays are
+// cleared by the probe kernel: the first 2 * (mask + 1) words of b_runs).
+RunTable run_table(dhs_table* t, long long n) {
+  RunTable rt;
+  const long long cap = std::min(run_table_cap((n + seg_chunk(n) - 1) / seg_chunk(n)), t->ws_run_cap);
+  unsigned* w = (unsigned*)t->b_runs.p;
+  rt.key = w;
+  rt.ctr = w + cap;
+  rt.c0 = w + 2 * cap;
+  rt.c1 = w + 3 * cap;
+  rt.mask = (unsigned)(cap - 1);
+  rt.max_pieces = kSegFinishPieces;
+  return rt;
+}
+
 dhs_status dispatch_seg(dhs_table* t, const unsigned* sk, const unsigned* sv, long long n,
                         const float* grad, long long nb, const OptArgs& oa, bool ext, bool mean, cudaStream_t s) {
   return launch_seg(t, sk, sv, n, grad, nb, oa, (double*)t->b_ph.p, (double*)t->b_pt.p,
                     (unsigned*)t->b_hist.p + kSegChunkCtrWord, (unsigned*)t->b_owners.p,
                     (unsigned*)t->b_hist.p + kSegOwnerCtrWord, ext ? (const unsigned*)t->b_bagpos.p : nullptr,
-                    ext ? (const double*)t->b_mult.p : nullptr, mean, s);
+                    ext ? (const double*)t->b_mult.p : nullptr, mean, run_table(t, n), s);
 }
 
 // offset assignment + row init for the new keys of an insert call
@@ -767,7 +800,7 @@ dhs_status ht_destroy(dhs_table* t) {
   if (t->free_list) dfree(t, t->free_list, (size_t)t->free_list_cap * 4, s);
   Buf* bufs[] = {&t->b_fcnt, &t->b_freed, &t->b_nbm, &t->b_fbm, &t->b_gcnt, &t->b_gpref, &t->b_slotpos, &t->b_ka, &t->b_va,
                  &t->b_kb, &t->b_vb, &t->b_hist, &t->b_totals, &t->b_ph, &t->b_pt, &t->b_owners,
-                 &t->b_cplan, &t->b_slots, &t->b_refs, &t->b_bagpos, &t->b_mult};
+                 &t->b_cplan, &t->b_slots, &t->b_refs, &t->b_bagpos, &t->b_mult, &t->b_runs};
   for (Buf* b : bufs) bfree(t, *b, s);
   cudaStreamSynchronize(s);
   for (auto& sn : t->snaps) {
@@ -986,7 +1019,8 @@ dhs_status embbag_backward_update_ex(dhs_table* t, const int64_t* d_keys, int64_
     DHS_CUDA(cudaMemsetAsync(t->b_hist.p, 0, (size_t)kSortZeroWords * 4, s));
     (ext ? bwd_probe_kernel<true> : bwd_probe_kernel<false>)<<<(unsigned)grid, 256, 0, s>>>(
         idmap(t), (const long long*)d_keys, n_keys, (const long long*)d_bag_offsets, n_bags, ka, va, sentinel,
-        (unsigned*)t->b_hist.p, passes, (unsigned long long*)t->b_totals.p, ntiles * kRadixBins, bpc, psw, mean,
+        (unsigned*)t->b_hist.p, passes, (unsigned long long*)t->b_totals.p, ntiles * kRadixBins,
+        (unsigned*)t->b_runs.p, 2 * ((long long)run_table(t, n_keys).mask + 1), bpc, psw, mean,
         (unsigned*)t->b_bagpos.p, (double*)t->b_mult.p, t->st);
     t->n_launches++;
     DHS_TRY(last_launch());
@@ -1390,8 +1424,8 @@ dhs_status embbag_backward_update_noalloc(dhs_table* t, const int64_t* d_keys, i
     DHS_CUDA(cudaMemsetAsync(hist, 0, (size_t)kSortZeroWords * 4, s));
     bwd_probe_kernel<false><<<(unsigned)grid, 256, 0, s>>>(idmap(t), (const long long*)d_keys, n_keys,
                                                     (const long long*)d_bag_offsets, n_bags, ka, va,
-                                                    sentinel, hist, passes, status, ntiles * kRadixBins, bpc,
-                                                    nullptr, false, nullptr, nullptr, t->st);
+                                                    sentinel, hist, passes, status, ntiles * kRadixBins,
+                                                    nullptr, 0, bpc, nullptr, false, nullptr, nullptr, t->st);
     DHS_TRY(last_launch());
   }
   const long long ntiles = (n_keys + kRadixTile - 1) / kRadixTile;
@@ -1418,8 +1452,9 @@ dhs_status embbag_backward_update_noalloc(dhs_table* t, const int64_t* d_keys, i
   oa.bc2 = (float)(1.0 - std::pow((double)t->b2, (double)t->adam_t));
   const int G = seg_group(t->dim), NV = seg_nv(t->dim);
   const int chunk = seg_chunk(n_keys);
+  RunTable no_table{};  // the owner chunks go to the combine kernels as they close
   DHS_TRY(launch_seg(t, ka, va, n_keys, d_grad, n_bags, oa, part_head, part_tail, hist + kSegChunkCtrWord, owners,
-                     hist + kSegOwnerCtrWord, nullptr, nullptr, false, s));
+                     hist + kSegOwnerCtrWord, nullptr, nullptr, false, no_table, s));
   t->n_launches += 1 + passes;
   return launch_combine(t, ka, n_keys, oa, part_head, part_tail, chunk, NV * G * 4, owners, hist, plan, s);
 }

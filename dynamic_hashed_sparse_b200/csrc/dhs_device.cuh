@@ -128,6 +128,20 @@ struct RowSpace {
   }
 };
 
+// Arrivals of the pieces of the long segments of one backward: open
+// addressing on the row (mask + 1 entries, a power of two).  key = row + 1
+// (0: empty), ctr = the pieces' arrival sum, c0 / c1 = the segment's first and
+// last sort chunk.  key and ctr start at zero.  key == nullptr: no table (the
+// owner chunks go to the combine kernels as they close).
+struct RunTable {
+  unsigned* key;
+  unsigned* ctr;
+  unsigned* c0;
+  unsigned* c1;
+  unsigned mask;
+  unsigned max_pieces;  // longer segments are finished by the combine kernels
+};
+
 enum : int { kHit = 0, kNew = 1, kBad = 2 };
 
 // Admission / eviction state of a table (null pointers and zeros when the

@@ -61,14 +61,15 @@ DHS_SEG_DECL(launch_seg_rowwise_ext)
 #undef DHS_SEG_DECL
 
 // bwd_segw_kernel<CPL, OPT, EXT, BF> (a warp per chunk, CPL columns per
-// lane; bf16: the table's weights are bf16)
+// lane; bf16: the table's weights are bf16; rt: the arrival table of the
+// long segments, or key == nullptr)
 #define DHS_SEGW_DECL(NAME_)                                                                    \
   cudaError_t NAME_(int cpl, bool bf16, int sm_count, const unsigned* skey, const unsigned* sval, \
                     long long n, const float* grad, long long n_bags, int dim, RowSpace rs,     \
                     const OptArgs& oa, double* part_head, double* part_tail, int pstride,       \
                     int chunk, unsigned* chunk_ctr, unsigned* owners, unsigned* owner_ctr,      \
                     DevState* st, const unsigned* bagpos, const double* mult, bool mean,        \
-                    cudaStream_t s);
+                    const RunTable& rt, cudaStream_t s);
 DHS_SEGW_DECL(launch_seg_sgd_w)
 DHS_SEGW_DECL(launch_seg_adagrad_w)
 DHS_SEGW_DECL(launch_seg_adam_w)

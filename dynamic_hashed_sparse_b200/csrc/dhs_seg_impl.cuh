@@ -57,7 +57,7 @@ cudaError_t run_w(int sm_count, const unsigned* skey, const unsigned* sval, long
                   const float* grad, long long n_bags, int dim, RowSpace rs, const OptArgs& oa,
                   double* part_head, double* part_tail, int pstride, int chunk, unsigned* chunk_ctr,
                   unsigned* owners, unsigned* owner_ctr, DevState* st, const unsigned* bagpos,
-                  const double* mult, bool mean, cudaStream_t s) {
+                  const double* mult, bool mean, const RunTable& rt, cudaStream_t s) {
   const size_t smem = segw_smem_bytes(CPL);
   const int resident = blocks_per_sm((const void*)bwd_segw_kernel<CPL, OPT, EXT, BF>, 256, smem) * sm_count;
   const long long nchunks = (n + chunk - 1) / chunk;
@@ -69,7 +69,7 @@ cudaError_t run_w(int sm_count, const unsigned* skey, const unsigned* sval, long
   bwd_segw_kernel<CPL, OPT, EXT, BF><<<(unsigned)grid, 256, smem, s>>>(skey, sval, n, grad, n_bags, dim, rs, oa,
                                                                   part_head, part_tail, pstride, chunk,
                                                                   chunk_ctr, owners, owner_ctr, st, grad_once,
-                                                                  bagpos, mult, mean);
+                                                                  bagpos, mult, mean, rt);
   return cudaGetLastError();
 }
 
@@ -78,12 +78,12 @@ cudaError_t launch_w(int cpl, bool bf16, int sm_count, const unsigned* skey, con
                      const float* grad, long long n_bags, int dim, RowSpace rs, const OptArgs& oa,
                      double* part_head, double* part_tail, int pstride, int chunk, unsigned* chunk_ctr,
                      unsigned* owners, unsigned* owner_ctr, DevState* st, const unsigned* bagpos,
-                     const double* mult, bool mean, cudaStream_t s) {
+                     const double* mult, bool mean, const RunTable& rt, cudaStream_t s) {
 #define DHS_RUN(c)                                                                                       \
   (bf16 ? run_w<c, OPT, EXT, true>(sm_count, skey, sval, n, grad, n_bags, dim, rs, oa, part_head, part_tail,  \
-                                   pstride, chunk, chunk_ctr, owners, owner_ctr, st, bagpos, mult, mean, s)   \
+                                   pstride, chunk, chunk_ctr, owners, owner_ctr, st, bagpos, mult, mean, rt, s) \
         : run_w<c, OPT, EXT, false>(sm_count, skey, sval, n, grad, n_bags, dim, rs, oa, part_head, part_tail, \
-                                    pstride, chunk, chunk_ctr, owners, owner_ctr, st, bagpos, mult, mean, s))
+                                    pstride, chunk, chunk_ctr, owners, owner_ctr, st, bagpos, mult, mean, rt, s))
   switch (cpl) {
     case 1: return DHS_RUN(1);
     case 2: return DHS_RUN(2);
@@ -115,9 +115,9 @@ cudaError_t launch_w(int cpl, bool bf16, int sm_count, const unsigned* skey, con
                         const OptArgs& oa, double* part_head, double* part_tail, int pstride,    \
                         int chunk, unsigned* chunk_ctr, unsigned* owners, unsigned* owner_ctr,   \
                         DevState* st, const unsigned* bagpos, const double* mult, bool mean,    \
-                        cudaStream_t s) {                                                       \
+                        const RunTable& rt, cudaStream_t s) {                                   \
     return seg_impl::launch_w<OPT_, EXT_>(cpl, bf16, sm_count, skey, sval, n, grad, n_bags, dim, rs, oa, \
                                           part_head, part_tail, pstride, chunk, chunk_ctr, owners, \
-                                          owner_ctr, st, bagpos, mult, mean, s);                \
+                                          owner_ctr, st, bagpos, mult, mean, rt, s);            \
   }                                                                                             \
   }

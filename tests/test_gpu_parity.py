@@ -179,11 +179,14 @@ def test_dims_and_optimizers(dim, opt, bags):
         o.close()
 
 
-@pytest.mark.parametrize("occ", [255, 256, 257, 600, 5000, 40000])
+@pytest.mark.parametrize("occ", [255, 256, 257, 600, 5000, 8150, 8200, 8250, 40000])
 def test_hot_key_spanning_many_sort_chunks(occ):
     """One key occurs `occ` times (its run covers one sort chunk of 32 pairs up
     to hundreds of them), mixed with a tail of other keys before and after it
-    in row order; both segment kernels (narrow and wide rows)."""
+    in row order; both segment kernels (narrow and wide rows).  Runs of about
+    256 chunks (8,150 to 8,250 occurrences) sit at the boundary between a long
+    segment that the wide segment kernel's warp finishes and one that goes to
+    the combine kernels."""
     rng = np.random.default_rng(occ)
     for dim, opt in ((32, "adagrad"), (32, "adam"), (32, "adagrad_rowwise"), (12, "adagrad"), (128, "sgd")):
         t, o = make_pair(dim, opt)
