@@ -14,6 +14,14 @@ runs a second time with its table growing on demand inside the timed steps
 API from pinned host buffers, with the copies pipelined against the compute.
 Prints one JSON line.
 
+Timing: CUDA events on the launching stream at each step's start, at the
+forward / backward boundary and at its end, nothing else inside the timed
+steps but the IDMap growth phase's own events; "fwd" is key packing +
+embbag_forward, "bwd" is embbag_backward_update.  "phases_ms_per_step" (and
+the roofline's kernel time) come from a replay of the timed steps on the same
+table with an event around every phase; a replay inserts no keys, so its
+forward assignment phase is empty.
+
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl dhs|reference]
 
 --impl reference times the CPU oracle (single core) on a bounded sample of
@@ -70,8 +78,9 @@ def alg_bytes(n: int, b: int, u: int, m: int, dim: int, opt: str, weights: str =
     # after the assignment wrote them
     fwd_refs = 8 * (b + 1) + R * u + 4 * dim * b
     bwd = 8 * n + 8 * (b + 1) + 16 * u + 4 * dim * b + 2 * S * u
+    # the timed forward is key packing + embbag_forward
     return dict(pack=pack, fwd_pool=fwd_pool, fwd_refs=fwd_refs, fwd_assign=fwd_assign,
-                fwd=fwd_pool + fwd_assign, bwd=bwd,
+                fwd=pack + fwd_pool + fwd_assign, bwd=bwd,
                 bwd_seg=4 * dim * b + 2 * S * u + 8 * n)
 
 
@@ -279,6 +288,7 @@ def run_reference(args):
 
 
 L2_BYTES = 126 << 20
+PHASE_TIMING = True  # per-phase events inside the timed steps (--no-phases: off)
 
 DESCRIPTIONS = {
     "tiny_uniform": "1024 bags x 1 id drawn uniformly from 65,536 distinct keys in [0, 2^40), one table, "
@@ -419,51 +429,75 @@ def measure(dhs, w, host_batches, device, dist, warmup: int, reserve: int, grad_
     t = setup_table(dhs, w, reserve, weights)
     stream = torch.cuda.current_stream()
 
-    def step(s):
+    def fwd(s):
         tids, ids, offs, n, nb = batches[s]
         k = keys[:n]
         dhs.dhs_pack_keys(tids, ids, out=k)
         dhs.embbag_forward(t, k, offs, out=pooled[:nb])
-        dhs.embbag_backward_update(t, k, offs, grads[s % n_grad][:nb], w.lr)
+
+    def bwd(s):
+        tids, ids, offs, n, nb = batches[s]
+        dhs.embbag_backward_update(t, keys[:n], offs, grads[s % n_grad][:nb], w.lr)
 
     for s in range(warmup):
-        step(s)
+        fwd(s)
+        bwd(s)
     torch.cuda.synchronize()
     c0 = dhs.ht_counters(t)
     dhs.ht_phase_times(t)  # clear
-    dhs.ht_set_phase_timing(t, True)
+    dhs.ht_set_phase_timing(t, 2)  # IDMap growth inside the timed steps, reported on its own
     barrier(dist, device)
     torch.cuda.synchronize()
-    spans = []
+    # timed steps: events at each step's start, forward / backward boundary
+    # and end only (per-phase events would perturb the launches they sit
+    # between)
+    E = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+    marks = []
     with ClockSampler(clock_index) as clk:
-        if not flush:
-            ev = [torch.cuda.Event(enable_timing=True) for _ in range(K + 1)]
-            ev[0].record(stream)
-            for i, s in enumerate(range(warmup, total)):
-                step(s)
-                ev[i + 1].record(stream)
-            torch.cuda.synchronize()
-            spans = [ev[i].elapsed_time(ev[i + 1]) for i in range(K)]
-            ms_local = ev[0].elapsed_time(ev[K])
-        else:
-            pairs = []
-            for s in range(warmup, total):
-                fbuf.zero_()
-                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                e0.record(stream)
-                step(s)
-                e1.record(stream)
-                pairs.append((e0, e1))
-            torch.cuda.synchronize()
-            spans = [a.elapsed_time(b) for a, b in pairs]
-            ms_local = sum(spans)
+        prev = None
+        for s in range(warmup, total):
+            if flush or prev is None:
+                if flush:
+                    fbuf.zero_()
+                prev = E()
+                prev.record(stream)
+            mid, end = E(), E()
+            fwd(s)
+            mid.record(stream)
+            bwd(s)
+            end.record(stream)
+            marks.append((prev, mid, end))
+            prev = end
+        torch.cuda.synchronize()
+    spans = [a.elapsed_time(c) for a, _, c in marks]
+    fwd_spans = [a.elapsed_time(b) for a, b, _ in marks]
+    bwd_spans = [b.elapsed_time(c) for _, b, c in marks]
+    ms_local = sum(spans)
     barrier(dist, device)
-    dhs.ht_set_phase_timing(t, False)
-    phases = dhs.ht_phase_times(t)
+    dhs.ht_set_phase_timing(t, 0)
+    growth = dhs.ht_phase_times(t)
     c1 = dhs.ht_counters(t)
     status = dhs.ht_sync(t)
     if status != 0:
         raise RuntimeError(f"{w.name}: device status {status} ({dhs.dhs_status_str(status)}) after the timed steps")
+    # phase breakdown: the timed steps replayed on the same table with an
+    # event around every phase (the replay inserts no keys: its forward
+    # assignment phase is empty; the other phases do the timed steps' work)
+    phases = {}
+    if PHASE_TIMING:
+        dhs.ht_phase_times(t)  # clear
+        dhs.ht_set_phase_timing(t, True)
+        for s in range(warmup, total):
+            if flush:
+                fbuf.zero_()
+            fwd(s)
+            bwd(s)
+        torch.cuda.synchronize()
+        dhs.ht_set_phase_timing(t, False)
+        phases = dhs.ht_phase_times(t)
+        status = dhs.ht_sync(t)
+        if status != 0:
+            raise RuntimeError(f"{w.name}: device status {status} after the phase replay")
 
     n_ids = sum(batches[s][3] for s in range(warmup, total))
     n_bags = sum(batches[s][4] for s in range(warmup, total))
@@ -477,16 +511,16 @@ def measure(dhs, w, host_batches, device, dist, warmup: int, reserve: int, grad_
     peaks = load_peaks()
     ph_ms = {k: v[0] for k, v in phases.items()}
     ph_cnt = {k: v[1] for k, v in phases.items()}
-    fwd_ms = ph_ms["fwd_probe"] + ph_ms["fwd_probe_pool"] + ph_ms["fwd_assign"]
-    bwd_ms = ph_ms["bwd_probe"] + ph_ms["bwd_sort"] + ph_ms["bwd_seg_update"] + ph_ms["bwd_combine"]
-    dom = max(("fwd_probe_pool", "bwd_seg_update"), key=lambda k: ph_ms[k])
+    fwd_ms = max_over_ranks(sum(fwd_spans), dist, device)
+    bwd_ms = max_over_ranks(sum(bwd_spans), dist, device)
+    dom = max(("fwd_probe_pool", "bwd_seg_update"), key=lambda k: ph_ms.get(k, 0.0))
     dom_kernel = {"fwd_probe_pool": ("fwd_pool_refs_kernel" if n_ids >= POOL_SPLIT_LEN * n_bags
                                      else "fwd_probe_pool_kernel"),
                   "bwd_seg_update": "bwd_segw_kernel" if w.dim >= SEGW_MIN_DIM else "bwd_seg_kernel"}[dom]
     dom_bytes = ((ab["fwd_refs"] if dom_kernel == "fwd_pool_refs_kernel" else ab["fwd_pool"])
                  if dom == "fwd_probe_pool" else ab["bwd_seg"])
-    dom_launch_ms = ph_ms[dom] / max(1, ph_cnt[dom])
-    dom_bytes_per_launch = dom_bytes / max(1, ph_cnt[dom])
+    dom_launch_ms = ph_ms.get(dom, 0.0) / max(1, ph_cnt.get(dom, 0))
+    dom_bytes_per_launch = dom_bytes / max(1, ph_cnt.get(dom, 0))
     achieved = dom_bytes_per_launch / (dom_launch_ms / 1e3) / 1e9 if dom_launch_ms else 0.0
     traffic = load_traffic(dom_kernel) if want_traffic else None
     roofline = {
@@ -513,7 +547,7 @@ def measure(dhs, w, host_batches, device, dist, warmup: int, reserve: int, grad_
         "bwd": {"ids_per_s": n_ids / (bwd_ms / 1e3) if bwd_ms else None, "ms_per_step": bwd_ms / K,
                 "gbs": gbs(ab["bwd"], bwd_ms), "frac_of_peak": frac(ab["bwd"], bwd_ms)},
         "step_gbs": gbs(ab["fwd"] + ab["bwd"], ms_local),
-        "phases_ms_per_step": {k: v / K for k, v in ph_ms.items() if ph_cnt[k]},
+        "phases_ms_per_step": {k: v / K for k, v in ph_ms.items() if ph_cnt[k] and k != "idmap_growth"},
         "per_step": {"ids": n_ids / K, "bags": n_bags / K, "unique": U / K, "new": M / K},
         "roofline": roofline,
         "gpu_launches": launches,
@@ -523,7 +557,7 @@ def measure(dhs, w, host_batches, device, dist, warmup: int, reserve: int, grad_
                                    "blocks_appended": c1["blocks"] - c0["blocks"],
                                    "device_allocs": c1["allocs"] - c0["allocs"],
                                    "alloc_ms": (c1["alloc_ns"] - c0["alloc_ns"]) / 1e6,
-                                   "idmap_growth_ms": ph_ms.get("idmap_growth", 0.0),
+                                   "idmap_growth_ms": growth.get("idmap_growth", (0.0, 0))[0],
                                    "host_waits": c1["host_waits"] - c0["host_waits"],
                                    "host_wait_ms": (c1["host_wait_ns"] - c0["host_wait_ns"]) / 1e6}},
         "clocks": clk.summary(),
@@ -724,6 +758,8 @@ def main(argv=None):
                          "comma-separated list of labels (" + ", ".join(e[0] for e in EXTRA_WORKLOADS) + ")")
     ap.add_argument("--grad-buffers", type=int, default=32)
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-phases", action="store_true",
+                    help="time the steps without the per-phase events (no phase breakdown)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-steps", type=int, default=5)
     ap.add_argument("--ref-frac", type=float, default=1.0 / 16)
@@ -735,6 +771,8 @@ def main(argv=None):
     ap.add_argument("--batch", type=int, default=0,
                     help="samples per step (default: the workload's 65,536); smaller only for profiling")
     args = ap.parse_args(argv)
+    global PHASE_TIMING
+    PHASE_TIMING = not args.no_phases
     if args.warmup < 0 or args.steps < 1:
         ap.error("--steps must be >= 1 and --warmup >= 0")
     if args.impl == "reference":

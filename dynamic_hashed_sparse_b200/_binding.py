@@ -413,8 +413,9 @@ def ht_counters(t: Table) -> dict:
     return {k: int(v) for k, v in zip(names, out)}
 
 
-def ht_set_phase_timing(t: Table, enable: bool):
-    _check("ht_set_phase_timing", _lib.ht_set_phase_timing(t.handle, int(bool(enable))))
+def ht_set_phase_timing(t: Table, enable):
+    """enable: False / 0 off, True / 1 every phase, 2 the IDMap growth phase only."""
+    _check("ht_set_phase_timing", _lib.ht_set_phase_timing(t.handle, int(enable)))
 
 
 def ht_phase_times(t: Table) -> dict:

@@ -52,6 +52,12 @@
 #ifndef DHS_RADIX_MINB
 #define DHS_RADIX_MINB 3
 #endif
+//   DHS_SEG_RUN_TABLE 1: long segments are finished by the segment kernel's
+//                     warp that brings the last piece; 0: all go to the
+//                     combine kernels
+#ifndef DHS_SEG_RUN_TABLE
+#define DHS_SEG_RUN_TABLE 1
+#endif
 //   DHS_SEG_FINISH_PIECES pieces of a long segment the segment kernel's warp
 //                     adds itself (longer ones go to the combine kernels)
 #ifndef DHS_SEG_FINISH_PIECES
@@ -105,20 +111,23 @@ constexpr int kCombineSlotCtrWord = kSegChunkCtrWord + 3;
 // weight psw[p] (the bag's gradient is multiplied by it) or, for mean
 // pooling, the bag's length (the gradient is divided by it).
 template <bool EXT>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(256, 4)
 bwd_probe_kernel(IdMap m, const long long* __restrict__ keys, long long n_keys,
                  const long long* __restrict__ bag_off, long long n_bags,
                  unsigned* __restrict__ rkey, unsigned* __restrict__ rval, unsigned sentinel,
                  unsigned* __restrict__ hist, int passes, unsigned long long* __restrict__ status0,
-                 long long status0_words, unsigned* __restrict__ zero32, long long zero32_words, int bpc,
+                 long long status0_words, unsigned* __restrict__ zero32, long long zero32_words,
+                 unsigned* __restrict__ next_ctr, long long next_ctr_words, int bpc,
                  const float* __restrict__ psw, bool mean, unsigned* __restrict__ bagpos,
                  double* __restrict__ mult, DevState* st) {
+  pdl_enter();
   constexpr bool ext = EXT;
   constexpr unsigned FULL = 0xffffffffu;
   const int lane = threadIdx.x & 31;
   // the sort's digit counts of every pass, taken here from the rows this
   // kernel writes (hist is zero on entry); the first pass's look-back words
-  // and the segment kernel's arrival table (zero32) cleared
+  // and the segment kernel's arrival table (zero32) cleared, and the counters
+  // of the next backward (next_ctr, another area than this one's)
   __shared__ unsigned h[kRadixMaxPasses][kRadixBins];
   for (int i = threadIdx.x; i < kRadixMaxPasses * kRadixBins; i += blockDim.x) (&h[0][0])[i] = 0u;
   for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < status0_words;
@@ -127,6 +136,9 @@ bwd_probe_kernel(IdMap m, const long long* __restrict__ keys, long long n_keys,
   for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < zero32_words;
        i += (long long)gridDim.x * blockDim.x)
     zero32[i] = 0u;
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < next_ctr_words;
+       i += (long long)gridDim.x * blockDim.x)
+    next_ctr[i] = 0u;
   __syncthreads();
   auto count = [&](unsigned k) {
     for (int ps = 0; ps < passes; ++ps) atomicAdd(&h[ps][(k >> (8 * ps)) & 255u], 1u);
@@ -182,6 +194,10 @@ bwd_probe_kernel(IdMap m, const long long* __restrict__ keys, long long n_keys,
       if (lane == nb - 1) e0 = n;
       if (lane + 32 == nb - 1) e1 = n;
     }
+    // one id per bag throughout the chunk (a common case): a position's bag
+    // is its offset from the chunk's start, no search needed
+    const bool singles =
+        __all_sync(FULL, (lane >= nb || e0 == s + lane + 1) && (lane + 32 >= nb || e1 == s + lane + 33));
     if (lane >= nb) e0 = INT_MAX;
     if (lane + 32 >= nb) e1 = INT_MAX;
     if (bad) latch(st, kErrInvalid);
@@ -206,7 +222,7 @@ bwd_probe_kernel(IdMap m, const long long* __restrict__ keys, long long n_keys,
       long long f0 = -1, f1 = -1;
       if (p0 < E && k0 >= 0) f0 = probe_find(m, (unsigned long long)k0);
       if (p1 < E && k1 >= 0) f1 = probe_find(m, (unsigned long long)k1);
-      const int g0 = bag_of(p0), g1 = bag_of(p1);
+      const int g0 = singles ? p0 - s : bag_of(p0), g1 = singles ? p1 - s : bag_of(p1);
       // f < 0: no row (-1 absent: an error; -2 known but not admitted: skipped)
       if (p0 < E) {
         if (k0 < 0) latch(st, kErrInvalid);
@@ -292,6 +308,7 @@ radix_onesweep_kernel(const unsigned* __restrict__ kin, const unsigned* __restri
                       int shift, const unsigned* __restrict__ hist,
                       unsigned long long* __restrict__ status, unsigned* __restrict__ tile_ctr,
                       unsigned long long* __restrict__ next_status, long long next_words, DevState* st) {
+  pdl_enter();
   __shared__ unsigned s_k[kRadixTile];
   __shared__ unsigned s_v[kRadixTile];
   __shared__ unsigned wc[8][kRadixBins + 1];
@@ -594,6 +611,7 @@ bwd_seg_kernel(const unsigned* __restrict__ skey, const unsigned* __restrict__ s
                int C, unsigned* __restrict__ chunk_ctr,
                unsigned* __restrict__ owners, unsigned* __restrict__ owner_ctr, DevState* st,
                const unsigned* __restrict__ bagpos, const double* __restrict__ mult, bool mean) {
+  pdl_enter();
   constexpr int R = seg_ring(NV);
   extern __shared__ float4 seg_ring_smem[];
   const int lane = threadIdx.x & 31;
@@ -956,6 +974,7 @@ bwd_segw_kernel(const unsigned* __restrict__ skey, const unsigned* __restrict__ 
                 unsigned* __restrict__ owner_ctr, DevState* st, bool grad_once,
                 const unsigned* __restrict__ bagpos, const double* __restrict__ mult, bool mean,
                 RunTable rt) {
+  pdl_enter();
   constexpr int B = segw_batch(CPL);
   constexpr int PITCH = 32 * CPL;  // floats per staged row
   constexpr int NS = seg_state_arrays(OPT);
@@ -1156,6 +1175,7 @@ bwd_segw_kernel(const unsigned* __restrict__ skey, const unsigned* __restrict__ 
     float racc = 0.f;
     unsigned kcur = 0;
     int mode = 0, run_end = 0;
+    unsigned rslot = 0;  // lane 0: arrival entry of the current piece
     // the row of an owned run, loaded into the "next" registers one run ahead
     float nw[CPL];
     float nst[NS > 0 ? NS : 1][CPL];
@@ -1280,22 +1300,21 @@ bwd_segw_kernel(const unsigned* __restrict__ skey, const unsigned* __restrict__ 
           // ends 1 + bias - c, every other piece 1; the sum reaches
           // 1 + 2 bias exactly when all c1 - c0 + 1 pieces have arrived, in
           // whatever order (no partial sum can reach it: chunks < 2^26)
-          __threadfence();  // this lane's partial before the arrival
+          const unsigned slot0 = rslot;
+          const bool is_end = mode == 1 && (run_end < cend || fwd1 != kcur);
+          if (lane == 0 && slot0 != ~0u) {
+            if (mode == 3) *(volatile unsigned*)(rt.c0 + slot0) = (unsigned)c;
+            if (is_end) *(volatile unsigned*)(rt.c1 + slot0) = (unsigned)c;
+          }
+          __threadfence();  // this lane's partial (and lane 0's chunk index) before the arrival
           __syncwarp();
-          unsigned fin = 0, slot = 0;
-          if (lane == 0) {
-            const bool is_end = mode == 1 && (run_end < cend || fwd1 != kcur);
+          unsigned fin = 0, slot = slot0;
+          if (lane == 0 && slot0 != ~0u) {
             unsigned add = 1u;
             if (mode == 3) add += (unsigned)c + kRunBias;
             if (is_end) add += kRunBias - (unsigned)c;
-            slot = run_slot(rt, kcur, st);
-            if (slot != ~0u) {
-              if (mode == 3) *(volatile unsigned*)(rt.c0 + slot) = (unsigned)c;
-              if (is_end) *(volatile unsigned*)(rt.c1 + slot) = (unsigned)c;
-              __threadfence();
-              const unsigned old = atomicAdd(rt.ctr + slot, add);
-              fin = old + add == 1u + 2u * kRunBias ? 1u : 0u;
-            }
+            const unsigned old = atomicAdd(rt.ctr + slot0, add);
+            fin = old + add == 1u + 2u * kRunBias ? 1u : 0u;
           }
           fin = __shfl_sync(FULL, fin, 0);
           if (fin) {
@@ -1343,6 +1362,10 @@ bwd_segw_kernel(const unsigned* __restrict__ skey, const unsigned* __restrict__ 
       const uint2 enext = runs[r + 1];
       run_end = (int)(enext.y & 0xffffu);
       if (mode != 2) run_end = min(run_end, cend);  // a long piece stops at the chunk end
+      // a piece of a long segment finds its arrival entry now, so that the
+      // lookup's latency passes while the piece is summed
+      if ((mode == 1 || mode == 3) && lane == 0 && rt.key != nullptr && kcur < nrows)
+        rslot = run_slot(rt, kcur, st);
 #pragma unroll
       for (int e = 0; e < CPL; ++e) rw[e] = nw[e];
 #pragma unroll
@@ -1500,6 +1523,7 @@ bwd_combine_plan_kernel(const unsigned* __restrict__ skey, long long n, int C,
                         CombinePlan pl, int dim, RowSpace rs, OptArgs oa,
                         const double* __restrict__ part_head, const double* __restrict__ part_tail,
                         int pstride, DevState* st) {
+  pdl_enter();
   const int lane = threadIdx.x & 31;
   const long long nchunks = (n + C - 1) / C;
   const unsigned long long nrows = st->row_count;
@@ -1556,6 +1580,7 @@ bwd_combine_kernel(const unsigned* __restrict__ skey, int dim, RowSpace rs, OptA
                    const double* __restrict__ part_head, const double* __restrict__ part_tail, int C,
                    int pstride, const unsigned* __restrict__ owners,
                    const unsigned* __restrict__ owner_ctr, CombinePlan pl) {
+  pdl_enter();
   extern __shared__ double sacc[];  // [slices][dim]
   __shared__ double s_sq;
   __shared__ bool s_last;

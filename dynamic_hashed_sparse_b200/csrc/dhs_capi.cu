@@ -72,7 +72,8 @@ enum { PH_FWD_POOL = 0, PH_FWD_ASSIGN = 1, PH_BWD_PROBE = 2, PH_BWD_SORT = 3, PH
 
 struct Snap {
   cudaEvent_t ev = nullptr;
-  unsigned long long* pinned = nullptr;  // row_count, keys_used copied here
+  unsigned long long* pinned = nullptr;  // row_count, keys_used written here (mapped)
+  unsigned long long* pinned_dev = nullptr;  // the same memory as the device addresses it
   long long cum_n = 0;                   // inserted-key upper bound counter at record time
   bool valid = false;
 };
@@ -180,8 +181,9 @@ struct dhs_table {
   Buf b_nbm, b_fbm, b_gcnt, b_gpref, b_slotpos, b_ka, b_va, b_kb, b_vb, b_hist, b_totals, b_ph,
       b_pt, b_owners, b_cplan, b_slots, b_refs, b_bagpos, b_mult, b_runs;
   long long ws_run_cap = 0;  // entries of the long-segment arrival table
+  int hist_sel = 0;          // which half of b_hist the next backward uses (the probe clears the other)
 
-  bool timing = false;
+  int timing = 0;  // 0 off, 1 every phase, 2 the IDMap growth phase only
   std::vector<PhaseRec> recs;
   std::vector<cudaEvent_t> ev_pool;
 };
@@ -306,7 +308,7 @@ struct PhaseScope {
   cudaStream_t s;
   cudaEvent_t a = nullptr;
   PhaseScope(dhs_table* t_, int ph, cudaStream_t s_) : t(t_), phase(ph), s(s_) {
-    if (t->timing) {
+    if (t->timing == 1 || (t->timing == 2 && ph == PH_GROW)) {
       a = ev_get(t);
       cudaEventRecord(a, s);
     }
@@ -351,11 +353,22 @@ void refresh_ub(dhs_table* t, bool wait) {
   }
 }
 
+// The device's row count and key count written straight into mapped pinned
+// host memory (no copy-engine transfer on the stream: a one-warp kernel).
+__global__ void snapshot_kernel(const DevState* st, volatile unsigned long long* host) {
+  pdl_enter();
+  if (threadIdx.x == 0) {
+    host[0] = st->row_count;
+    host[1] = st->keys_used;
+    __threadfence_system();
+  }
+}
+
 void record_snapshot(dhs_table* t, cudaStream_t s) {
   Snap& sn = t->snaps[t->snap_next];
   if (sn.valid) host_wait(t, sn.ev);  // ring slot reuse: at most kSnapRing in flight
-  // row_count and keys_used are adjacent
-  cudaMemcpyAsync(sn.pinned, &t->st->row_count, 2 * sizeof(unsigned long long), cudaMemcpyDeviceToHost, s);
+  launch_k(snapshot_kernel, 1, 32, 0, s, t->st, sn.pinned_dev);
+  t->n_launches++;
   cudaEventRecord(sn.ev, s);
   sn.cum_n = t->cum_n;
   sn.valid = true;
@@ -510,7 +523,12 @@ dhs_status ensure_ws(dhs_table* t, long long n, cudaStream_t s) {
   DHS_TRY(bget(t, t->b_kb, cap * 4, s));
   DHS_TRY(bget(t, t->b_vb, cap * 4, s));
   // digit histograms of every pass + one tile counter per pass; look-back state
-  DHS_TRY(bget(t, t->b_hist, (size_t)kSortZeroWords * 4, s));
+  // two areas of counters (digit histograms, tile and chunk counters): a
+  // backward uses one while its probe clears the other for the next backward
+  if (!t->b_hist.p) {
+    DHS_TRY(bget(t, t->b_hist, (size_t)2 * kSortZeroWords * 4, s));
+    DHS_CUDA(cudaMemsetAsync(t->b_hist.p, 0, t->b_hist.bytes, s));
+  }
   DHS_TRY(bget(t, t->b_totals, (size_t)kRadixMaxPasses * ntiles * kRadixBins * 8, s));
   DHS_TRY(bget(t, t->b_ph, (size_t)nchunks * pstride * 8, s));
   DHS_TRY(bget(t, t->b_pt, (size_t)nchunks * pstride * 8, s));
@@ -546,12 +564,12 @@ dhs_status launch_combine(dhs_table* t, const unsigned* skey, long long n, const
                           const unsigned* owners, unsigned* zeroed, const CombinePlan& pl,
                           cudaStream_t s) {
   const unsigned* owner_ctr = zeroed + kSegOwnerCtrWord;
-  bwd_combine_plan_kernel<<<(unsigned)t->sm_count * 2, 256, 0, s>>>(
+  launch_k(bwd_combine_plan_kernel, (unsigned)t->sm_count * 2, 256, 0, s,
       skey, n, chunk, owners, owner_ctr, pl, t->dim, rowspace(t), oa, part_head, part_tail, pstride, t->st);
   t->n_launches++;
   DHS_TRY(last_launch());
   const size_t smem = (size_t)std::max(kCombineThreads, t->dim) * sizeof(double);
-  bwd_combine_kernel<<<(unsigned)t->sm_count * 8, kCombineThreads, smem, s>>>(
+  launch_k(bwd_combine_kernel, (unsigned)t->sm_count * 8, kCombineThreads, smem, s,
       skey, t->dim, rowspace(t), oa, part_head, part_tail, chunk, pstride, owners, owner_ctr, pl);
   t->n_launches++;
   return last_launch();
@@ -626,14 +644,19 @@ RunTable run_table(dhs_table* t, long long n) {
   rt.c1 = w + 3 * cap;
   rt.mask = (unsigned)(cap - 1);
   rt.max_pieces = kSegFinishPieces;
+  if (!DHS_SEG_RUN_TABLE) rt.key = nullptr;
   return rt;
 }
 
+// The counters of the current backward (zero when it starts).
+unsigned* hist_words(dhs_table* t) { return (unsigned*)t->b_hist.p + (size_t)t->hist_sel * kSortZeroWords; }
+
 dhs_status dispatch_seg(dhs_table* t, const unsigned* sk, const unsigned* sv, long long n,
-                        const float* grad, long long nb, const OptArgs& oa, bool ext, bool mean, cudaStream_t s) {
+                        const float* grad, long long nb, const OptArgs& oa, bool ext, bool mean, unsigned* ctr,
+                        cudaStream_t s) {
   return launch_seg(t, sk, sv, n, grad, nb, oa, (double*)t->b_ph.p, (double*)t->b_pt.p,
-                    (unsigned*)t->b_hist.p + kSegChunkCtrWord, (unsigned*)t->b_owners.p,
-                    (unsigned*)t->b_hist.p + kSegOwnerCtrWord, ext ? (const unsigned*)t->b_bagpos.p : nullptr,
+                    ctr + kSegChunkCtrWord, (unsigned*)t->b_owners.p,
+                    ctr + kSegOwnerCtrWord, ext ? (const unsigned*)t->b_bagpos.p : nullptr,
                     ext ? (const double*)t->b_mult.p : nullptr, mean, run_table(t, n), s);
 }
 
@@ -641,12 +664,12 @@ dhs_status dispatch_seg(dhs_table* t, const unsigned* sk, const unsigned* sv, lo
 dhs_status launch_assign(dhs_table* t, const long long* keys, long long n, cudaStream_t s) {
   const long long nwords = (n + 31) / 32;
   const long long ngroups = (n + kGroupPositions - 1) / kGroupPositions;
-  fwd_mark_kernel<<<(unsigned)ngroups, kGroupThreads, 0, s>>>(
+  launch_k(fwd_mark_kernel, (unsigned)ngroups, kGroupThreads, 0, s, 
       t->slots, (unsigned*)t->b_nbm.p, (unsigned*)t->b_fbm.p, (unsigned*)t->b_gcnt.p,
       (unsigned*)t->b_gpref.p, (const unsigned*)t->b_slotpos.p, nwords, ngroups, hooks(t), t->st);
   t->n_launches += 2;
   DHS_TRY(last_launch());
-  fwd_assign_kernel<<<(unsigned)(ngroups * kAssignSplit), kGroupThreads, 0, s>>>(
+  launch_k(fwd_assign_kernel, (unsigned)(ngroups * kAssignSplit), kGroupThreads, 0, s, 
       t->slots, rowspace(t), t->dim, keys, (const unsigned*)t->b_fbm.p, (const unsigned*)t->b_gpref.p,
       (const unsigned*)t->b_slotpos.p, nwords, ngroups, hooks(t), t->st);
   return last_launch();
@@ -688,7 +711,7 @@ dhs_status dhs_pack_keys(const int32_t* d_table_ids, const int64_t* d_ids, int64
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const long long grid = std::min<long long>((n + 255) / 256, (long long)sms * 8);
-  pack_keys_kernel<<<(unsigned)grid, 256, 0, (cudaStream_t)stream>>>(
+  launch_k(pack_keys_kernel, (unsigned)grid, 256, 0, (cudaStream_t)stream, 
       d_table_ids, (const long long*)d_ids, n, (long long*)d_keys_out);
   return last_launch();
 }
@@ -762,7 +785,9 @@ dhs_status ht_create_ex(int32_t dim, dhs_optimizer opt, dhs_row_dtype weights, i
     rc = DHS_ERR_CUDA;
   for (int i = 0; rc == DHS_OK && i < kSnapRing; ++i) {
     if (cudaEventCreateWithFlags(&t->snaps[i].ev, cudaEventDisableTiming) != cudaSuccess ||
-        cudaHostAlloc((void**)&t->snaps[i].pinned, 2 * sizeof(unsigned long long), cudaHostAllocDefault) != cudaSuccess)
+        cudaHostAlloc((void**)&t->snaps[i].pinned, 2 * sizeof(unsigned long long), cudaHostAllocMapped) !=
+            cudaSuccess ||
+        cudaHostGetDevicePointer((void**)&t->snaps[i].pinned_dev, t->snaps[i].pinned, 0) != cudaSuccess)
       rc = DHS_ERR_CUDA;
   }
   if (rc == DHS_OK) rc = grow_map(t, kInitialSlots, s);
@@ -856,14 +881,14 @@ dhs_status ht_lookup_or_insert(dhs_table* t, const int64_t* d_keys, int64_t n,
   t->step++;
   {
     PhaseScope ph(t, PH_LOOKUP_INSERT, s);
-    fwd_probe_offsets_kernel<<<(unsigned)((n + kFwdThreads - 1) / kFwdThreads), kFwdThreads, 0, s>>>(
+    launch_k(fwd_probe_offsets_kernel, (unsigned)((n + kFwdThreads - 1) / kFwdThreads), kFwdThreads, 0, s, 
         idmap(t), (const long long*)d_keys, n, (long long*)d_offsets_out, (unsigned*)t->b_nbm.p,
         (unsigned*)t->b_slotpos.p, hooks(t), t->st);
     t->n_launches += 2;
     DHS_TRY(last_launch());
     DHS_TRY(launch_assign(t, (const long long*)d_keys, n, s));
     const long long grid = std::min<long long>((n + 255) / 256, (long long)t->sm_count * 8);
-    fwd_fixup_kernel<<<(unsigned)grid, 256, 0, s>>>(t->slots, (long long*)d_offsets_out, n);
+    launch_k(fwd_fixup_kernel, (unsigned)grid, 256, 0, s, t->slots, (long long*)d_offsets_out, n);
     DHS_TRY(last_launch());
   }
   t->rows_ub += n;
@@ -883,7 +908,7 @@ dhs_status ht_lookup(dhs_table* t, const int64_t* d_keys, int64_t n, int64_t* d_
   cudaStream_t s = (cudaStream_t)stream;
   t->last_stream = s;
   const long long grid = std::min<long long>((n + 255) / 256, (long long)t->sm_count * 16);
-  lookup_kernel<<<(unsigned)grid, 256, 0, s>>>(idmap(t), (const long long*)d_keys, n, (long long*)d_offsets_out);
+  launch_k(lookup_kernel, (unsigned)grid, 256, 0, s, idmap(t), (const long long*)d_keys, n, (long long*)d_offsets_out);
   t->n_launches++;
   return last_launch();
 }
@@ -918,7 +943,7 @@ dhs_status embbag_forward_ex(dhs_table* t, const int64_t* d_keys, int64_t n_keys
     // keys' rows, then gather every row from the table
     {
       PhaseScope ph(t, PH_FWD_PROBE, s);
-      fwd_probe_offsets_kernel<<<(unsigned)((n_keys + kFwdThreads - 1) / kFwdThreads), kFwdThreads, 0, s>>>(
+      launch_k(fwd_probe_offsets_kernel, (unsigned)((n_keys + kFwdThreads - 1) / kFwdThreads), kFwdThreads, 0, s, 
           idmap(t), (const long long*)d_keys, n_keys, (long long*)t->b_refs.p, (unsigned*)t->b_nbm.p,
           (unsigned*)t->b_slotpos.p, hooks(t), t->st);
       t->n_launches++;
@@ -1004,6 +1029,7 @@ dhs_status embbag_backward_update_ex(dhs_table* t, const int64_t* d_keys, int64_
   unsigned* va = (unsigned*)t->b_va.p;
   unsigned* kb = (unsigned*)t->b_kb.p;
   unsigned* vb = (unsigned*)t->b_vb.p;
+  unsigned* const ctr = hist_words(t);  // this backward's counters
   {
     PhaseScope ph(t, PH_BWD_PROBE, s);
     // one resident wave of blocks, each warp taking chunks of bags in turn:
@@ -1015,25 +1041,29 @@ dhs_status embbag_backward_update_ex(dhs_table* t, const int64_t* d_keys, int64_
     const long long warps = (n_bags + bpc - 1) / bpc;
     const long long grid = grid_for((warps + 7) / 8, resident);
     const long long ntiles = (n_keys + kRadixTile - 1) / kRadixTile;
-    // the counters the probe and the sort accumulate into start at zero
-    DHS_CUDA(cudaMemsetAsync(t->b_hist.p, 0, (size_t)kSortZeroWords * 4, s));
-    (ext ? bwd_probe_kernel<true> : bwd_probe_kernel<false>)<<<(unsigned)grid, 256, 0, s>>>(
-        idmap(t), (const long long*)d_keys, n_keys, (const long long*)d_bag_offsets, n_bags, ka, va, sentinel,
-        (unsigned*)t->b_hist.p, passes, (unsigned long long*)t->b_totals.p, ntiles * kRadixBins,
-        (unsigned*)t->b_runs.p, 2 * ((long long)run_table(t, n_keys).mask + 1), bpc, psw, mean,
-        (unsigned*)t->b_bagpos.p, (double*)t->b_mult.p, t->st);
+    // the counters this backward accumulates into are zero (cleared by the
+    // previous backward's probe, or at allocation); this probe clears the
+    // other area for the next one
+    unsigned* next_hist = (unsigned*)t->b_hist.p + (size_t)(1 - t->hist_sel) * kSortZeroWords;
+    (void)launch_k(ext ? bwd_probe_kernel<true> : bwd_probe_kernel<false>, (unsigned)grid, 256, 0, s, idmap(t),
+                   (const long long*)d_keys, n_keys, (const long long*)d_bag_offsets, n_bags, ka, va, sentinel,
+                   ctr, passes, (unsigned long long*)t->b_totals.p, ntiles * kRadixBins,
+                   (unsigned*)t->b_runs.p, 2 * ((long long)run_table(t, n_keys).mask + 1), next_hist,
+                   (long long)kSortZeroWords, bpc, psw, mean, (unsigned*)t->b_bagpos.p, (double*)t->b_mult.p,
+                   t->st);
     t->n_launches++;
     DHS_TRY(last_launch());
+    t->hist_sel ^= 1;  // the next backward uses the area this probe cleared
   }
   {
     PhaseScope ph(t, PH_BWD_SORT, s);
     const long long ntiles = (n_keys + kRadixTile - 1) / kRadixTile;
-    unsigned* hist = (unsigned*)t->b_hist.p;
+    unsigned* hist = ctr;
     unsigned* tile_ctr = hist + kRadixMaxPasses * kRadixBins;
     unsigned long long* status = (unsigned long long*)t->b_totals.p;
     for (int p = 0; p < passes; ++p) {
       const long long words = ntiles * kRadixBins;
-      radix_onesweep_kernel<<<(unsigned)ntiles, kRadixThreads, 0, s>>>(
+      launch_k(radix_onesweep_kernel, (unsigned)ntiles, kRadixThreads, 0, s, 
           ka, va, kb, vb, n_keys, 8 * p, hist + p * kRadixBins, status + (long long)p * words, tile_ctr + p,
           status + (long long)(p + 1) * words, p + 1 < passes ? words : 0, t->st);
       t->n_launches++;
@@ -1055,15 +1085,15 @@ dhs_status embbag_backward_update_ex(dhs_table* t, const int64_t* d_keys, int64_
     oa.bc2 = (float)(1.0 - std::pow((double)t->b2, (double)t->adam_t));
     {
       PhaseScope ph(t, PH_BWD_SEG, s);
-      DHS_TRY(dispatch_seg(t, ka, va, n_keys, d_grad, n_bags, oa, ext, mean, s));
+      DHS_TRY(dispatch_seg(t, ka, va, n_keys, d_grad, n_bags, oa, ext, mean, ctr, s));
     }
     PhaseScope ph(t, PH_BWD_COMBINE, s);
     const int pstride = seg_nv(t->dim) * seg_group(t->dim) * 4;
     DHS_TRY(launch_combine(t, ka, n_keys, oa, (const double*)t->b_ph.p, (const double*)t->b_pt.p,
                            seg_chunk(n_keys), pstride, (const unsigned*)t->b_owners.p,
-                           (unsigned*)t->b_hist.p,
-                           combine_plan((unsigned*)t->b_cplan.p, (double*)t->b_slots.p, t->ws_chunks,
-                                        (unsigned*)t->b_hist.p), s));
+                           ctr,
+                           combine_plan((unsigned*)t->b_cplan.p, (double*)t->b_slots.p, t->ws_chunks, ctr),
+                           s));
   }
   return DHS_OK;
 }
@@ -1084,7 +1114,7 @@ dhs_status ht_get_rows(dhs_table* t, const int64_t* d_keys, int64_t n, float* d_
   cudaStream_t s = (cudaStream_t)stream;
   t->last_stream = s;
   const long long grid = std::min<long long>((n + 7) / 8, (long long)t->sm_count * 16);
-  get_rows_kernel<<<(unsigned)grid, 256, 0, s>>>(idmap(t), rowspace(t), t->dim, export_stride(t),
+  launch_k(get_rows_kernel, (unsigned)grid, 256, 0, s, idmap(t), rowspace(t), t->dim, export_stride(t),
                                                  (const long long*)d_keys, n, d_rows_out);
   t->n_launches++;
   return last_launch();
@@ -1288,7 +1318,8 @@ dhs_status ht_export(dhs_table* t, int64_t* h_keys, float* h_rows) {
 
 dhs_status ht_set_phase_timing(dhs_table* t, int enable) {
   DHS_TRY(check_table(t));
-  t->timing = enable != 0;
+  if (enable < 0 || enable > 2) return DHS_ERR_INVALID_ARG;
+  t->timing = enable;
   return DHS_OK;
 }
 
@@ -1425,14 +1456,15 @@ dhs_status embbag_backward_update_noalloc(dhs_table* t, const int64_t* d_keys, i
     bwd_probe_kernel<false><<<(unsigned)grid, 256, 0, s>>>(idmap(t), (const long long*)d_keys, n_keys,
                                                     (const long long*)d_bag_offsets, n_bags, ka, va,
                                                     sentinel, hist, passes, status, ntiles * kRadixBins,
-                                                    nullptr, 0, bpc, nullptr, false, nullptr, nullptr, t->st);
+                                                    nullptr, 0, nullptr, 0, bpc, nullptr, false, nullptr, nullptr,
+                                                    t->st);
     DHS_TRY(last_launch());
   }
   const long long ntiles = (n_keys + kRadixTile - 1) / kRadixTile;
   {
     for (int p = 0; p < passes; ++p) {
       const long long words = ntiles * kRadixBins;
-      radix_onesweep_kernel<<<(unsigned)ntiles, kRadixThreads, 0, s>>>(
+      launch_k(radix_onesweep_kernel, (unsigned)ntiles, kRadixThreads, 0, s, 
           ka, va, kb, vb, n_keys, 8 * p, hist + p * kRadixBins, status + (long long)p * words, tile_ctr + p,
           status + (long long)(p + 1) * words, p + 1 < passes ? words : 0, t->st);
       DHS_TRY(last_launch());

@@ -20,7 +20,24 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+//   DHS_PDL 1: the hot-path kernels are launched as programmatic dependents of
+//           the kernel before them in the stream (their launch overlaps its
+//           tail); 0: plain launches
+#ifndef DHS_PDL
+#define DHS_PDL 1
+#endif
+
 namespace dhs {
+
+// First statement of a hot-path kernel.  Launched as a programmatic
+// dependent, the kernel waits here until the kernel before it in the stream
+// has finished and its writes are visible (a no-op after a plain launch);
+// then it lets the kernel after it begin launching, whose blocks in turn wait
+// at their own first statement.
+__device__ __forceinline__ void pdl_enter() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
 
 constexpr unsigned long long kEmptyKey = ~0ull;
 // An evicted key's slot: probes step over it (the chain goes on), and it is

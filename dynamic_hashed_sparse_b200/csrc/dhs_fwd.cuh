@@ -211,6 +211,7 @@ fwd_probe_pool_kernel(IdMap m, RowSpace rs, int dim, const long long* __restrict
                       const float* __restrict__ psw,
                       float* __restrict__ out, unsigned* __restrict__ nbm,
                       unsigned* __restrict__ slotpos, DevState* st) {
+  pdl_enter();
   constexpr bool W = PM == 1, MEAN = PM == 2;
   const int lane = threadIdx.x & 31;
   const int gl = lane & (G - 1);
@@ -301,6 +302,7 @@ fwd_pool_refs_kernel(RowSpace rs, int dim, const Slot* __restrict__ slots,
                      const long long* __restrict__ bag_off, long long n_bags,
                      const float* __restrict__ psw,
                      float* __restrict__ out, DevState* st) {
+  pdl_enter();
   constexpr bool W = PM == 1, MEAN = PM == 2;
   const int lane = threadIdx.x & 31;
   const int gl = lane & (G - 1);
@@ -374,6 +376,7 @@ __global__ void __launch_bounds__(kFwdThreads)
 fwd_probe_offsets_kernel(IdMap m, const long long* __restrict__ keys, long long n,
                          long long* __restrict__ offsets_out, unsigned* __restrict__ nbm,
                          unsigned* __restrict__ slotpos, Hooks hk, DevState* st) {
+  pdl_enter();
   const long long p = (long long)blockIdx.x * kFwdThreads + threadIdx.x;
   bool is_new = false, claimed = false;
   if (p < n) {
@@ -407,6 +410,7 @@ fwd_probe_offsets_kernel(IdMap m, const long long* __restrict__ keys, long long 
 
 __global__ void fwd_fixup_kernel(const Slot* __restrict__ slots, long long* __restrict__ offsets,
                                  long long n) {
+  pdl_enter();
   for (long long p = (long long)blockIdx.x * blockDim.x + threadIdx.x; p < n;
        p += (long long)gridDim.x * blockDim.x) {
     const long long o = offsets[p];
@@ -438,6 +442,7 @@ fwd_mark_kernel(Slot* __restrict__ slots, unsigned* __restrict__ nbm,
                 unsigned* __restrict__ fbm, unsigned* __restrict__ gcnt,
                 unsigned* __restrict__ gpref, const unsigned* __restrict__ slotpos,
                 long long nwords, long long ngroups, Hooks hk, DevState* st) {
+  pdl_enter();
   __shared__ unsigned wsum[32];
   __shared__ bool is_last;
   __shared__ unsigned long long carry_s;
@@ -556,6 +561,7 @@ fwd_assign_kernel(Slot* __restrict__ slots, RowSpace rs, int dim, const long lon
                   const unsigned* __restrict__ fbm, const unsigned* __restrict__ gpref,
                   const unsigned* __restrict__ slotpos, long long nwords, long long ngroups,
                   Hooks hk, DevState* st) {
+  pdl_enter();
   __shared__ unsigned long long skey[kGroupPositions];  // 32 KB
   __shared__ unsigned wpre[kGroupWords];
   __shared__ unsigned s_total;
@@ -830,6 +836,7 @@ free_scatter_kernel(const unsigned* __restrict__ free_bm, long long nwords, cons
 
 __global__ void lookup_kernel(IdMap m, const long long* __restrict__ keys, long long n,
                               long long* __restrict__ out) {
+  pdl_enter();
   for (long long p = (long long)blockIdx.x * blockDim.x + threadIdx.x; p < n;
        p += (long long)gridDim.x * blockDim.x) {
     const long long k = __ldg(keys + p);
@@ -843,6 +850,7 @@ __global__ void lookup_kernel(IdMap m, const long long* __restrict__ keys, long 
 // key, NaN for an absent key.
 __global__ void get_rows_kernel(IdMap m, RowSpace rs, int dim, int ostride, const long long* __restrict__ keys,
                                 long long n, float* __restrict__ out) {
+  pdl_enter();
   const int lane = threadIdx.x & 31;
   const long long nw = ((long long)gridDim.x * blockDim.x) >> 5;
   const bool bf = rs.wfl != dim;
@@ -877,6 +885,7 @@ __global__ void keys_by_row_kernel(const Slot* __restrict__ slots, unsigned long
 
 __global__ void pack_keys_kernel(const int* __restrict__ tids, const long long* __restrict__ ids,
                                  long long n, long long* __restrict__ keys) {
+  pdl_enter();
   for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n;
        i += (long long)gridDim.x * blockDim.x) {
     const long long t = tids[i], id = ids[i];

@@ -4,11 +4,32 @@
 
 #include <cuda_runtime.h>
 
+#include <utility>
+
 #include "dhs_device.cuh"
 
 namespace dhs {
 
 struct OptArgs;
+
+// Launch of a hot-path kernel (one whose first statement is pdl_enter()):
+// with DHS_PDL, as a programmatic dependent of the work before it in the
+// stream.  Returns the launch's error.
+template <typename... P, typename... A>
+cudaError_t launch_k(void (*kernel)(P...), unsigned grid, unsigned block, size_t smem, cudaStream_t s,
+                     A&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(block);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = DHS_PDL ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<A>(args)...);
+}
 
 // Blocks of `kernel` (launched with `threads` threads and `smem` bytes of
 // dynamic shared memory) that fit on one SM of the current device, at least

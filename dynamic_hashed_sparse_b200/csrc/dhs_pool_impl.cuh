@@ -24,7 +24,7 @@ cudaError_t run(int sm_count, IdMap m, RowSpace rs, int dim, const long long* ke
   const long long per_block = kFwdThreads / G;
   const long long need = std::max<long long>(1, (nchunks + per_block - 1) / per_block);
   const long long grid = std::min<long long>(need, resident);
-  fwd_probe_pool_kernel<G, NV, PM, BF><<<(unsigned)grid, kFwdThreads, 0, s>>>(
+  launch_k(fwd_probe_pool_kernel<G, NV, PM, BF>, (unsigned)grid, kFwdThreads, 0, s, 
       m, rs, dim, keys, n_keys, bag_off, n_bags, psw, out, nbm, slotpos, st);
   return cudaGetLastError();
 }
@@ -39,7 +39,7 @@ cudaError_t run_refs(int sm_count, RowSpace rs, int dim, const Slot* slots, cons
   const long long per_block = kFwdThreads / G;
   const long long need = std::max<long long>(1, (nchunks + per_block - 1) / per_block);
   const long long grid = std::min<long long>(need, resident);
-  fwd_pool_refs_kernel<G, NV, PM, BF><<<(unsigned)grid, kFwdThreads, 0, s>>>(rs, dim, slots, refs, n_keys,
+  launch_k(fwd_pool_refs_kernel<G, NV, PM, BF>, (unsigned)grid, kFwdThreads, 0, s, rs, dim, slots, refs, n_keys,
                                                                              bag_off, n_bags, psw, out, st);
   return cudaGetLastError();
 }

@@ -24,7 +24,7 @@ cudaError_t run(int sm_count, const unsigned* skey, const unsigned* sval, long l
   const long long per_block = 256 / G;
   const long long need = std::max<long long>(1, (nchunks + per_block - 1) / per_block);
   const long long grid = std::min<long long>(need, resident);
-  bwd_seg_kernel<G, NV, OPT, EXT><<<(unsigned)grid, 256, smem, s>>>(skey, sval, n, grad, n_bags, dim, rs, oa,
+  launch_k(bwd_seg_kernel<G, NV, OPT, EXT>, (unsigned)grid, 256, smem, s, skey, sval, n, grad, n_bags, dim, rs, oa,
                                                                    part_head, part_tail, chunk, chunk_ctr,
                                                                    owners, owner_ctr, st, bagpos, mult, mean);
   return cudaGetLastError();
@@ -66,7 +66,7 @@ cudaError_t run_w(int sm_count, const unsigned* skey, const unsigned* sval, long
   // gradient rows read about once per call (about one id per bag) are marked
   // first to evict in L2
   const bool grad_once = DHS_SEGW_EVICT_FIRST && 2 * n <= 3 * n_bags;
-  bwd_segw_kernel<CPL, OPT, EXT, BF><<<(unsigned)grid, 256, smem, s>>>(skey, sval, n, grad, n_bags, dim, rs, oa,
+  launch_k(bwd_segw_kernel<CPL, OPT, EXT, BF>, (unsigned)grid, 256, smem, s, skey, sval, n, grad, n_bags, dim, rs, oa,
                                                                   part_head, part_tail, pstride, chunk,
                                                                   chunk_ctr, owners, owner_ctr, st, grad_once,
                                                                   bagpos, mult, mean, rt);

@@ -313,6 +313,9 @@ dhs_status ht_counters(dhs_table* t, int64_t out[14]);
  * 5 lookup-or-insert, 6 IDMap growth, 7 forward probe (long bags: the probe
  * runs as its own kernel before the assignment), 8 backward combine of rows
  * that span three or more sort chunks.
+ * enable: 0 off, 1 every phase, 2 the IDMap growth phase only (rare; its
+ * events stay out of the launches of the steady-state phases, between which
+ * an event delays the next kernel's launch).  Other values: invalid.
  * ht_phase_times synchronises, writes ms_out[p] = total ms and
  * count_out[p] = number of timed launches of phase p (p < n), then clears. */
 dhs_status ht_set_phase_timing(dhs_table* t, int enable);

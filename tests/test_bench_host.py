@@ -55,7 +55,9 @@ def test_algorithmic_bytes_formula():
     R, S = 32, 64
     assert ab["fwd_pool"] == 8 * 10 + 8 * 5 + 16 * 6 + 16 * 2 + R * 4 + 4 * 8 * 4
     assert ab["fwd_assign"] == S * 2 + 16 * 2
-    assert ab["fwd"] == ab["fwd_pool"] + ab["fwd_assign"]  # key packing is timed outside the forward
+    # the timed forward includes key packing (table ids 4 B + ids 8 B read, keys 8 B written)
+    assert ab["pack"] == 20 * 10
+    assert ab["fwd"] == ab["pack"] + ab["fwd_pool"] + ab["fwd_assign"]
     assert ab["fwd_refs"] == 8 * 5 + R * 6 + 4 * 8 * 4
     assert ab["bwd"] == 8 * 10 + 8 * 5 + 16 * 6 + 4 * 8 * 4 + 2 * S * 6
     assert bench.stride_floats(32, "adam") == 96 and bench.stride_floats(16, "adagrad_rowwise") == 20
