@@ -36,5 +36,9 @@ from ._binding import (  # noqa: F401
     ht_set_phase_timing,
     ht_size,
     ht_sync,
+    ht_shard_route,
+    ht_shard_pool,
+    ht_shard_grads,
     lib,
 )
+from .sharded import NcclExchange, ShardedTable, run_lockstep  # noqa: F401,E402

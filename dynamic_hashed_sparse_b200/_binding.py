@@ -23,7 +23,7 @@ STATUS = {
     4: "table full", 5: "key not found", 6: "unsupported", 7: "internal wait bound exceeded",
 }
 OPT_CODES = {"sgd": 0, "adagrad": 1, "adam": 2, "adagrad_rowwise": 3}
-POOL_MODES = {"sum": 0, "mean": 1}
+POOL_MODES = {"sum": 0, "mean": 1, "divide": 2}  # "divide": backward only (sharded owners)
 ROW_DTYPES = {"f32": 0, "bf16": 1}
 PHASES = ("fwd_probe_pool", "fwd_assign", "bwd_probe", "bwd_sort", "bwd_seg_update",
           "lookup_or_insert", "idmap_growth", "fwd_probe", "bwd_combine")
@@ -69,6 +69,9 @@ def _load() -> C.CDLL:
         "ht_counters": (C.c_int, [vp, vp]),
         "ht_set_phase_timing": (C.c_int, [vp, C.c_int]),
         "ht_phase_times": (C.c_int, [vp, vp, vp, C.c_int]),
+        "ht_shard_route": (C.c_int, [vp, vp, i64, i32, vp, vp, vp, vp]),
+        "ht_shard_pool": (C.c_int, [vp, vp, vp, i64, vp, i64, vp, C.c_int, vp, vp]),
+        "ht_shard_grads": (C.c_int, [vp, vp, vp, i64, i64, vp, vp, C.c_int, vp, vp, vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -423,3 +426,66 @@ def ht_phase_times(t: Table) -> dict:
     cnt = np.zeros(len(PHASES), np.int64)
     _check("ht_phase_times", _lib.ht_phase_times(t.handle, ms.ctypes.data, cnt.ctypes.data, len(PHASES)))
     return {p: (float(m), int(c)) for p, m, c in zip(PHASES, ms, cnt)}
+
+
+# ---- hash-sharded engine (see the header's section on it) ----
+
+def ht_shard_route(t: Table, keys: torch.Tensor, world: int, stream=None):
+    """Group the batch's keys by owner rank: (send_keys int64[n], slot_of
+    int32[n], counts list[world]).  Synchronises the stream."""
+    _dev(keys, torch.int64, "keys")
+    n = keys.numel()
+    send = torch.empty(n, dtype=torch.int64, device=keys.device)
+    slot = torch.empty(n, dtype=torch.int32, device=keys.device)
+    counts = np.zeros(world, np.int64)
+    _check("ht_shard_route", _lib.ht_shard_route(t.handle, keys.data_ptr(), n, int(world), send.data_ptr(),
+                                                 slot.data_ptr(), counts.ctypes.data, _stream(stream)))
+    return send, slot, [int(c) for c in counts]
+
+
+def ht_shard_pool(t: Table, rows: torch.Tensor, slot_of: torch.Tensor, bag_offsets: torch.Tensor,
+                  per_sample_weights: Optional[torch.Tensor] = None, mode: str = "sum",
+                  out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Pool the owners' rows (rows[slot_of[i]] is the row of id i)."""
+    _dev(rows, torch.float32, "rows")
+    _dev(slot_of, torch.int32, "slot_of")
+    _dev(bag_offsets, torch.int64, "bag_offsets")
+    n = slot_of.numel()
+    nb = bag_offsets.numel() - 1
+    if rows.numel() != n * t.dim:
+        raise ValueError("rows must hold n_keys * dim floats")
+    if out is None:
+        out = torch.empty((nb, t.dim), dtype=torch.float32, device=rows.device)
+    psw = 0
+    if per_sample_weights is not None:
+        _dev(per_sample_weights, torch.float32, "per_sample_weights")
+        if per_sample_weights.numel() != n:
+            raise ValueError("per_sample_weights needs one weight per key")
+        psw = per_sample_weights.data_ptr()
+    _check("ht_shard_pool", _lib.ht_shard_pool(t.handle, rows.data_ptr(), slot_of.data_ptr(), n,
+                                               bag_offsets.data_ptr(), nb, psw, POOL_MODES[mode], out.data_ptr(),
+                                               _stream(stream)))
+    return out
+
+
+def ht_shard_grads(t: Table, grad: torch.Tensor, bag_offsets: torch.Tensor, slot_of: torch.Tensor,
+                   per_sample_weights: Optional[torch.Tensor] = None, mode: str = "sum", stream=None):
+    """Per-id gradient rows in routed order (and their factors, or None for
+    plain sum pooling): (send_grads float[n, dim], send_fact float[n] or None)."""
+    _dev(grad, torch.float32, "grad")
+    _dev(bag_offsets, torch.int64, "bag_offsets")
+    _dev(slot_of, torch.int32, "slot_of")
+    n = slot_of.numel()
+    nb = bag_offsets.numel() - 1
+    if grad.numel() != nb * t.dim:
+        raise ValueError("grad must hold n_bags * dim floats")
+    send = torch.empty((n, t.dim), dtype=torch.float32, device=grad.device)
+    psw = 0
+    if per_sample_weights is not None:
+        _dev(per_sample_weights, torch.float32, "per_sample_weights")
+        psw = per_sample_weights.data_ptr()
+    fact = torch.empty(n, dtype=torch.float32, device=grad.device) if (psw or mode == "mean") else None
+    _check("ht_shard_grads", _lib.ht_shard_grads(t.handle, grad.data_ptr(), bag_offsets.data_ptr(), nb, n,
+                                                 slot_of.data_ptr(), psw, POOL_MODES[mode], send.data_ptr(),
+                                                 fact.data_ptr() if fact is not None else 0, _stream(stream)))
+    return send, fact

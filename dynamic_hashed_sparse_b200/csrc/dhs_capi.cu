@@ -23,6 +23,7 @@
 #include "dhs_device.cuh"
 #include "dhs_fwd.cuh"
 #include "dhs_launch.h"
+#include "dhs_shard.cuh"
 
 using namespace dhs;
 
@@ -179,7 +180,7 @@ struct dhs_table {
   long long ws_n = -1;
   long long ws_chunks = 0;  // chunk capacity of the segment and combine buffers
   Buf b_nbm, b_fbm, b_gcnt, b_gpref, b_slotpos, b_ka, b_va, b_kb, b_vb, b_hist, b_totals, b_ph,
-      b_pt, b_owners, b_cplan, b_slots, b_refs, b_bagpos, b_mult, b_runs;
+      b_pt, b_owners, b_cplan, b_slots, b_refs, b_bagpos, b_mult, b_runs, b_shard;
   long long ws_run_cap = 0;  // entries of the long-segment arrival table
   int hist_sel = 0;          // which half of b_hist the next backward uses (the probe clears the other)
 
@@ -825,7 +826,7 @@ dhs_status ht_destroy(dhs_table* t) {
   if (t->free_list) dfree(t, t->free_list, (size_t)t->free_list_cap * 4, s);
   Buf* bufs[] = {&t->b_fcnt, &t->b_freed, &t->b_nbm, &t->b_fbm, &t->b_gcnt, &t->b_gpref, &t->b_slotpos, &t->b_ka, &t->b_va,
                  &t->b_kb, &t->b_vb, &t->b_hist, &t->b_totals, &t->b_ph, &t->b_pt, &t->b_owners,
-                 &t->b_cplan, &t->b_slots, &t->b_refs, &t->b_bagpos, &t->b_mult, &t->b_runs};
+                 &t->b_cplan, &t->b_slots, &t->b_refs, &t->b_bagpos, &t->b_mult, &t->b_runs, &t->b_shard};
   for (Buf* b : bufs) bfree(t, *b, s);
   cudaStreamSynchronize(s);
   for (auto& sn : t->snaps) {
@@ -1000,9 +1001,12 @@ dhs_status embbag_backward_update_ex(dhs_table* t, const int64_t* d_keys, int64_
   DHS_TRY(check_table(t));
   if (n_keys < 0 || n_keys >= (1ll << 31) || n_bags < 0 || n_bags >= (1ll << 31))
     return DHS_ERR_INVALID_ARG;
-  if (mode != DHS_POOL_SUM && mode != DHS_POOL_MEAN) return DHS_ERR_INVALID_ARG;
+  if (mode != DHS_POOL_SUM && mode != DHS_POOL_MEAN && mode != DHS_POOL_DIVIDE) return DHS_ERR_INVALID_ARG;
   if (mode == DHS_POOL_MEAN && d_per_sample_weights) return DHS_ERR_INVALID_ARG;
-  const bool mean = mode == DHS_POOL_MEAN;
+  if (mode == DHS_POOL_DIVIDE && n_keys > 0 && !d_per_sample_weights) return DHS_ERR_INVALID_ARG;
+  // mean pooling divides each id's term by its bag's length (DHS_POOL_DIVIDE:
+  // by the per-id value given)
+  const bool mean = mode == DHS_POOL_MEAN || mode == DHS_POOL_DIVIDE;
   const float* psw = n_keys > 0 ? d_per_sample_weights : nullptr;
   const bool ext = psw != nullptr || mean;
   if (n_bags == 0 && n_keys != 0) return DHS_ERR_INVALID_ARG;
@@ -1489,6 +1493,97 @@ dhs_status embbag_backward_update_noalloc(dhs_table* t, const int64_t* d_keys, i
                      hist + kSegOwnerCtrWord, nullptr, nullptr, false, no_table, s));
   t->n_launches += 1 + passes;
   return launch_combine(t, ka, n_keys, oa, part_head, part_tail, chunk, NV * G * 4, owners, hist, plan, s);
+}
+
+// ---- hash-sharded engine ----
+
+dhs_status ht_shard_route(dhs_table* t, const int64_t* d_keys, int64_t n_keys, int32_t world,
+                          int64_t* d_send_keys, int32_t* d_slot_of, int64_t* h_send_counts, dhs_stream stream) {
+  DHS_TRY(check_table(t));
+  if (world < 1 || world > kRadixBins || n_keys < 0 || n_keys >= (1ll << 31) || !h_send_counts)
+    return DHS_ERR_INVALID_ARG;
+  if (n_keys > 0 && (!d_keys || !d_send_keys || !d_slot_of)) return DHS_ERR_INVALID_ARG;
+  for (int r = 0; r < world; ++r) h_send_counts[r] = 0;
+  if (n_keys == 0) return DHS_OK;
+  DeviceGuard g(t->device);
+  cudaStream_t s = (cudaStream_t)stream;
+  t->last_stream = s;
+  DHS_TRY(ensure_ws(t, n_keys, s));
+  // owner histogram (256 bins) and the routing pass's tile counter
+  DHS_TRY(bget(t, t->b_shard, (size_t)(kRadixBins + 1) * 4, s));
+  unsigned* hist = (unsigned*)t->b_shard.p;
+  DHS_CUDA(cudaMemsetAsync(hist, 0, t->b_shard.bytes, s));
+  unsigned* okey = (unsigned*)t->b_ka.p;
+  unsigned* opos = (unsigned*)t->b_va.p;
+  unsigned* skey = (unsigned*)t->b_kb.p;
+  unsigned* spos = (unsigned*)t->b_vb.p;
+  const long long ntiles = (n_keys + kRadixTile - 1) / kRadixTile;
+  unsigned long long* status = (unsigned long long*)t->b_totals.p;
+  const unsigned grid = (unsigned)std::min<long long>((n_keys + 255) / 256, (long long)t->sm_count * 8);
+  // owners + positions, one stable digit pass by owner, then the gather
+  (void)launch_k(shard_count_kernel, grid, 256, 0, s, (const long long*)d_keys, (long long)n_keys,
+                 (unsigned)world, okey, opos, hist, status, ntiles * kRadixBins);
+  DHS_TRY(last_launch());
+  (void)launch_k(radix_onesweep_kernel, (unsigned)ntiles, kRadixThreads, 0, s, (const unsigned*)okey,
+                 (const unsigned*)opos, skey, spos, (long long)n_keys, 0, (const unsigned*)hist, status,
+                 hist + kRadixBins, (unsigned long long*)nullptr, 0ll, t->st);
+  DHS_TRY(last_launch());
+  (void)launch_k(shard_gather_kernel, grid, 256, 0, s, (const long long*)d_keys, (const unsigned*)spos,
+                 (long long)n_keys, (long long*)d_send_keys, (int*)d_slot_of);
+  DHS_TRY(last_launch());
+  t->n_launches += 3;
+  std::vector<unsigned> counts(world);
+  DHS_CUDA(cudaMemcpyAsync(counts.data(), hist, world * sizeof(unsigned), cudaMemcpyDeviceToHost, s));
+  DHS_CUDA(cudaStreamSynchronize(s));
+  for (int r = 0; r < world; ++r) h_send_counts[r] = counts[r];
+  return DHS_OK;
+}
+
+dhs_status ht_shard_pool(dhs_table* t, const float* d_rows, const int32_t* d_slot_of, int64_t n_keys,
+                         const int64_t* d_bag_offsets, int64_t n_bags, const float* d_per_sample_weights,
+                         dhs_pool_mode mode, float* d_pooled_out, dhs_stream stream) {
+  DHS_TRY(check_table(t));
+  if (n_keys < 0 || n_keys >= (1ll << 31) || n_bags < 0 || n_bags >= (1ll << 31)) return DHS_ERR_INVALID_ARG;
+  if (mode != DHS_POOL_SUM && mode != DHS_POOL_MEAN) return DHS_ERR_INVALID_ARG;
+  if (mode == DHS_POOL_MEAN && d_per_sample_weights) return DHS_ERR_INVALID_ARG;
+  if (n_bags == 0) return n_keys == 0 ? DHS_OK : DHS_ERR_INVALID_ARG;
+  if (!d_bag_offsets || !d_pooled_out || (n_keys > 0 && (!d_rows || !d_slot_of))) return DHS_ERR_INVALID_ARG;
+  if ((uintptr_t)d_pooled_out % 16 || (uintptr_t)d_rows % 16) return DHS_ERR_INVALID_ARG;
+  DeviceGuard g(t->device);
+  cudaStream_t s = (cudaStream_t)stream;
+  t->last_stream = s;
+  const float* psw = n_keys > 0 ? d_per_sample_weights : nullptr;
+  const unsigned grid = (unsigned)std::min<long long>((n_bags + 7) / 8, (long long)t->sm_count * 8);
+  auto k = psw ? shard_pool_kernel<true, false>
+               : (mode == DHS_POOL_MEAN ? shard_pool_kernel<false, true> : shard_pool_kernel<false, false>);
+  (void)launch_k(k, grid, 256, 0, s, d_rows, (const int*)d_slot_of, (long long)n_keys,
+                 (const long long*)d_bag_offsets, (long long)n_bags, t->dim, psw, d_pooled_out, t->st);
+  t->n_launches++;
+  return last_launch();
+}
+
+dhs_status ht_shard_grads(dhs_table* t, const float* d_grad, const int64_t* d_bag_offsets, int64_t n_bags,
+                          int64_t n_keys, const int32_t* d_slot_of, const float* d_per_sample_weights,
+                          dhs_pool_mode mode, float* d_send_grads, float* d_send_fact, dhs_stream stream) {
+  DHS_TRY(check_table(t));
+  if (n_keys < 0 || n_keys >= (1ll << 31) || n_bags < 0 || n_bags >= (1ll << 31)) return DHS_ERR_INVALID_ARG;
+  if (mode != DHS_POOL_SUM && mode != DHS_POOL_MEAN) return DHS_ERR_INVALID_ARG;
+  if (mode == DHS_POOL_MEAN && d_per_sample_weights) return DHS_ERR_INVALID_ARG;
+  if (n_bags == 0) return n_keys == 0 ? DHS_OK : DHS_ERR_INVALID_ARG;
+  if (!d_bag_offsets || !d_grad || (n_keys > 0 && (!d_slot_of || !d_send_grads))) return DHS_ERR_INVALID_ARG;
+  if ((uintptr_t)d_grad % 16 || (uintptr_t)d_send_grads % 16) return DHS_ERR_INVALID_ARG;
+  const float* psw = n_keys > 0 ? d_per_sample_weights : nullptr;
+  const int fact = psw ? 1 : (mode == DHS_POOL_MEAN ? 2 : 0);
+  if (fact && n_keys > 0 && !d_send_fact) return DHS_ERR_INVALID_ARG;
+  DeviceGuard g(t->device);
+  cudaStream_t s = (cudaStream_t)stream;
+  t->last_stream = s;
+  const unsigned grid = (unsigned)std::min<long long>((n_bags + 7) / 8, (long long)t->sm_count * 8);
+  auto k = fact == 1 ? shard_expand_kernel<1> : (fact == 2 ? shard_expand_kernel<2> : shard_expand_kernel<0>);
+  (void)launch_k(k, grid, 256, 0, s, d_grad, (const long long*)d_bag_offsets, (long long)n_bags, (long long)n_keys,
+                 (const int*)d_slot_of, psw, t->dim, d_send_grads, d_send_fact, t->st);
+  t->n_launches++;
+  return last_launch();
 }
 
 }  // extern "C"

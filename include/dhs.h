@@ -84,7 +84,12 @@ typedef enum {
  * rows (optionally weighted per id), or their mean. */
 typedef enum {
   DHS_POOL_SUM = 0,
-  DHS_POOL_MEAN = 1
+  DHS_POOL_MEAN = 1,
+  /* Backward only: mean pooling carried to a key's owner by the sharded
+   * engine, each id its own bag: d_per_sample_weights holds the length of
+   * the id's original bag, and the id's gradient row is divided by it (in
+   * fp64, as DHS_POOL_MEAN does). */
+  DHS_POOL_DIVIDE = 2
 } dhs_pool_mode;
 
 typedef struct {
@@ -320,6 +325,54 @@ dhs_status ht_counters(dhs_table* t, int64_t out[14]);
  * count_out[p] = number of timed launches of phase p (p < n), then clears. */
 dhs_status ht_set_phase_timing(dhs_table* t, int enable);
 dhs_status ht_phase_times(dhs_table* t, double* ms_out, int64_t* count_out, int n);
+
+/* ---- hash-sharded engine ([RecIS] code-architecture section: collective
+ * All-to-All for parameter aggregation; [DLRM-E] practice cases 1 and 2: rows
+ * split across cards, lookups exchanged by all-to-all) ----
+ * Each of `world` ranks holds one table; key k belongs to rank
+ *   owner(k) = floor(hi32(mix(k XOR 0x5DEECE66D)) * world / 2^32),
+ * mix = the splitmix64 finaliser (Steele, Lea & Flood; Vigna), hi32 = its
+ * upper 32 bits, so that the owner is independent of the IDMap's bucket
+ * hash.  One step on a rank:
+ *   forward:  ht_shard_route -> exchange the keys (all-to-all) -> each owner
+ *             embbag_forward_ex(received keys, one id per bag) gives their
+ *             rows -> exchange the rows back -> ht_shard_pool;
+ *   backward: ht_shard_grads -> exchange gradient rows and factors -> each
+ *             owner embbag_backward_update_ex(received keys, one id per bag,
+ *             factors, DHS_POOL_SUM or DHS_POOL_DIVIDE).
+ * The exchange is the caller's (NCCL all-to-all in the Python engine).
+ * Owners receive the ids in (source rank, position) order, so every sum runs
+ * over the terms of the global batch (rank 0's ids first) in that order:
+ * pooled outputs are formed as one table forms them (bit for bit from the
+ * same rows), and each key's gradient is the fp64 sum one table fed the
+ * concatenated batches forms, up to the association of its partial sums. */
+
+/* Route the ids of one batch: d_send_keys int64[n_keys] (device) gets the
+ * keys grouped by owner (rank 0's first), in position order within a
+ * group; d_slot_of int32[n_keys] (device) gets each position's index in
+ * d_send_keys; h_send_counts int64[world] (host) the group sizes.  world in
+ * [1, 256]; n_keys < 2^31.  Synchronises the stream (the counts are read on
+ * the host).  Uses the table's backward workspace (stream-ordered). */
+dhs_status ht_shard_route(dhs_table* t, const int64_t* d_keys, int64_t n_keys, int32_t world,
+                          int64_t* d_send_keys, int32_t* d_slot_of, int64_t* h_send_counts, dhs_stream stream);
+
+/* Pool the rows returned by the owners: d_rows float[n_keys, dim] in
+ * d_send_keys order; pooled[b] is formed from d_rows[d_slot_of[i]] for the
+ * positions i of bag b exactly as embbag_forward_ex forms it from the
+ * table's rows (same order, same rounding; mode DHS_POOL_SUM with optional
+ * d_per_sample_weights, or DHS_POOL_MEAN).  d_pooled_out float[n_bags, dim]. */
+dhs_status ht_shard_pool(dhs_table* t, const float* d_rows, const int32_t* d_slot_of, int64_t n_keys,
+                         const int64_t* d_bag_offsets, int64_t n_bags, const float* d_per_sample_weights,
+                         dhs_pool_mode mode, float* d_pooled_out, dhs_stream stream);
+
+/* The per-id gradient rows to send to the owners: d_send_grads[d_slot_of[i]]
+ * = d_grad[bag(i)] (float[n_keys, dim], copied exactly) and, unless d_send_fact
+ * is NULL, d_send_fact[d_slot_of[i]] = the id's factor: its per-sample weight
+ * (DHS_POOL_SUM with weights) or its bag's length (DHS_POOL_MEAN, which the
+ * owner passes on as DHS_POOL_DIVIDE).  Plain sum pooling needs no factors. */
+dhs_status ht_shard_grads(dhs_table* t, const float* d_grad, const int64_t* d_bag_offsets, int64_t n_bags,
+                          int64_t n_keys, const int32_t* d_slot_of, const float* d_per_sample_weights,
+                          dhs_pool_mode mode, float* d_send_grads, float* d_send_fact, dhs_stream stream);
 
 #ifdef __cplusplus
 }

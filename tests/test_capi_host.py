@@ -64,6 +64,11 @@ def test_host_side_argument_errors_return_before_cuda():
     assert L.ht_evict(None, 3, C.byref(n), None) == 1
     assert L.ht_live_rows(None, C.byref(n)) == 1
     assert L.ht_row_stride(None) == -1
+    # sharded engine calls
+    counts = (C.c_int64 * 4)()
+    assert L.ht_shard_route(None, None, 0, 4, None, None, counts, None) == 1
+    assert L.ht_shard_pool(None, None, None, 0, None, 0, None, 0, None, None) == 1
+    assert L.ht_shard_grads(None, None, None, 0, 0, None, None, 0, None, None, None) == 1
     # negative sizes
     assert L.dhs_pack_keys(None, None, -1, None, None) == 1
     assert L.dhs_pack_keys(None, None, 0, None, None) == 0
