@@ -44,6 +44,17 @@
 #ifndef DHS_SEGW_MIN_DIM
 #define DHS_SEGW_MIN_DIM 32
 #endif
+//   DHS_SEG_NARROW_MAX_DIM, DHS_SEG_NARROW_RUN  fp32 rows of more than
+//                     DHS_SEGW_MIN_DIM and at most DHS_SEG_NARROW_MAX_DIM
+//                     floats use the lane-group kernel while the table's
+//                     backward calls have averaged fewer than
+//                     DHS_SEG_NARROW_RUN ids per distinct row
+#ifndef DHS_SEG_NARROW_MAX_DIM
+#define DHS_SEG_NARROW_MAX_DIM 64
+#endif
+#ifndef DHS_SEG_NARROW_RUN
+#define DHS_SEG_NARROW_RUN 8
+#endif
 //   DHS_SEGW_EVICT_FIRST 1: gradient rows of calls with about one id per bag
 //                     are staged with an L2 evict-first policy; 0: normal
 #ifndef DHS_SEGW_EVICT_FIRST
@@ -62,6 +73,11 @@
 //                     adds itself (longer ones go to the combine kernels)
 #ifndef DHS_SEG_FINISH_PIECES
 #define DHS_SEG_FINISH_PIECES 256
+#endif
+//   DHS_PROBE_DEDUP   1: the backward probe probes a key held by several lanes
+//                     of a warp once (match.any); 0: every lane probes
+#ifndef DHS_PROBE_DEDUP
+#define DHS_PROBE_DEDUP 0
 #endif
 //   DHS_LOOKBACK_WINDOW predecessor tiles a radix pass's look-back reads at once
 #ifndef DHS_LOOKBACK_WINDOW
@@ -220,8 +236,20 @@ bwd_probe_kernel(IdMap m, const long long* __restrict__ keys, long long n_keys,
       const long long k0 = p0 < E ? __ldg(keys + p0) : 0;
       const long long k1 = p1 < E ? __ldg(keys + p1) : 0;
       long long f0 = -1, f1 = -1;
+#if DHS_PROBE_DEDUP
+      // a key held by several lanes is probed once, by the lowest of them
+      const unsigned long long q0 = p0 < E && k0 >= 0 ? (unsigned long long)k0 : ~0ull;
+      const unsigned long long q1 = p1 < E && k1 >= 0 ? (unsigned long long)k1 : ~0ull;
+      const unsigned m0 = __match_any_sync(FULL, q0), m1 = __match_any_sync(FULL, q1);
+      const int l0 = __ffs(m0) - 1, l1 = __ffs(m1) - 1;
+      if (l0 == lane && q0 != ~0ull) f0 = probe_find(m, q0);
+      if (l1 == lane && q1 != ~0ull) f1 = probe_find(m, q1);
+      f0 = __shfl_sync(FULL, f0, l0);
+      f1 = __shfl_sync(FULL, f1, l1);
+#else
       if (p0 < E && k0 >= 0) f0 = probe_find(m, (unsigned long long)k0);
       if (p1 < E && k1 >= 0) f1 = probe_find(m, (unsigned long long)k1);
+#endif
       const int g0 = singles ? p0 - s : bag_of(p0), g1 = singles ? p1 - s : bag_of(p1);
       // f < 0: no row (-1 absent: an error; -2 known but not admitted: skipped)
       if (p0 < E) {

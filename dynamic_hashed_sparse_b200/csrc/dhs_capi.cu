@@ -73,9 +73,10 @@ enum { PH_FWD_POOL = 0, PH_FWD_ASSIGN = 1, PH_BWD_PROBE = 2, PH_BWD_SORT = 3, PH
 
 struct Snap {
   cudaEvent_t ev = nullptr;
-  unsigned long long* pinned = nullptr;  // row_count, keys_used written here (mapped)
+  unsigned long long* pinned = nullptr;  // row_count, keys_used, sum_unique written here (mapped)
   unsigned long long* pinned_dev = nullptr;  // the same memory as the device addresses it
   long long cum_n = 0;                   // inserted-key upper bound counter at record time
+  long long bwd_n = 0;                   // ids of all backward calls enqueued before it
   bool valid = false;
 };
 
@@ -173,6 +174,10 @@ struct dhs_table {
   long long free_list_cap = 0;
   Buf b_fcnt, b_freed;
   long long cum_n = 0;  // sum of key counts of all insert calls
+  long long bwd_n = 0;  // sum of key counts of all backward calls
+  // from the newest finished snapshot: ids of the backward calls before it
+  // and the distinct rows they updated (their ratio is the mean segment length)
+  long long seen_bwd_n = 0, seen_unique = 0;
   Snap snaps[kSnapRing];
   int snap_next = 0;
 
@@ -348,6 +353,8 @@ void refresh_ub(dhs_table* t, bool wait) {
       if (ub < t->rows_ub) t->rows_ub = ub;
       const long long kb = (long long)sn.pinned[1] + (t->cum_n - sn.cum_n);
       if (kb < t->keys_ub) t->keys_ub = kb;
+      t->seen_bwd_n = sn.bwd_n;
+      t->seen_unique = (long long)sn.pinned[2];
       return;
     }
     cudaGetLastError();
@@ -361,6 +368,7 @@ __global__ void snapshot_kernel(const DevState* st, volatile unsigned long long*
   if (threadIdx.x == 0) {
     host[0] = st->row_count;
     host[1] = st->keys_used;
+    host[2] = st->sum_unique;
     __threadfence_system();
   }
 }
@@ -372,6 +380,7 @@ void record_snapshot(dhs_table* t, cudaStream_t s) {
   t->n_launches++;
   cudaEventRecord(sn.ev, s);
   sn.cum_n = t->cum_n;
+  sn.bwd_n = t->bwd_n;
   sn.valid = true;
   t->snap_next = (t->snap_next + 1) % kSnapRing;
 }
@@ -604,6 +613,18 @@ int segw_cpl(int dim) {
   return c;
 }
 
+// The segment kernel for a backward: the lane-group kernel for rows of fewer
+// than DHS_SEGW_MIN_DIM floats, and for fp32 rows of more than that and at
+// most DHS_SEG_NARROW_MAX_DIM floats while the table's segments have been
+// short (fewer than DHS_SEG_NARROW_RUN ids per distinct row over its backward
+// calls so far): a warp per chunk spends most of its issue slots on
+// per-segment work there.  Otherwise the warp-per-chunk kernel.
+bool use_narrow_seg(const dhs_table* t) {
+  if (t->dim < DHS_SEGW_MIN_DIM) return true;
+  return !t->wbf16 && t->dim > DHS_SEGW_MIN_DIM && t->dim <= DHS_SEG_NARROW_MAX_DIM && t->seen_unique > 0 &&
+         t->seen_bwd_n < (long long)DHS_SEG_NARROW_RUN * t->seen_unique;
+}
+
 // bagpos / mult non-null: extended pooling (sort values are positions).
 dhs_status launch_seg(dhs_table* t, const unsigned* sk, const unsigned* sv, long long n, const float* grad,
                       long long nb, const OptArgs& oa, double* part_head, double* part_tail,
@@ -613,7 +634,7 @@ dhs_status launch_seg(dhs_table* t, const unsigned* sk, const unsigned* sv, long
   const int pstride = NV * G * 4;  // doubles per partial (>= dim)
   const bool ext = mult != nullptr;
   cudaError_t e;
-  if (t->dim >= DHS_SEGW_MIN_DIM) {
+  if (!use_narrow_seg(t)) {
     auto fn = t->opt == DHS_SGD ? (ext ? launch_seg_sgd_ext_w : launch_seg_sgd_w)
               : t->opt == DHS_ADAGRAD ? (ext ? launch_seg_adagrad_ext_w : launch_seg_adagrad_w)
               : t->opt == DHS_ADAM ? (ext ? launch_seg_adam_ext_w : launch_seg_adam_w)
@@ -786,7 +807,7 @@ dhs_status ht_create_ex(int32_t dim, dhs_optimizer opt, dhs_row_dtype weights, i
     rc = DHS_ERR_CUDA;
   for (int i = 0; rc == DHS_OK && i < kSnapRing; ++i) {
     if (cudaEventCreateWithFlags(&t->snaps[i].ev, cudaEventDisableTiming) != cudaSuccess ||
-        cudaHostAlloc((void**)&t->snaps[i].pinned, 2 * sizeof(unsigned long long), cudaHostAllocMapped) !=
+        cudaHostAlloc((void**)&t->snaps[i].pinned, 3 * sizeof(unsigned long long), cudaHostAllocMapped) !=
             cudaSuccess ||
         cudaHostGetDevicePointer((void**)&t->snaps[i].pinned_dev, t->snaps[i].pinned, 0) != cudaSuccess)
       rc = DHS_ERR_CUDA;
@@ -1018,6 +1039,7 @@ dhs_status embbag_backward_update_ex(dhs_table* t, const int64_t* d_keys, int64_
   cudaStream_t s = (cudaStream_t)stream;
   t->last_stream = s;
   t->adam_t += 1;
+  t->bwd_n += n_keys;
   if (n_keys == 0) return DHS_OK;
   DHS_TRY(ensure_ws(t, n_keys, s));
   if (ext) DHS_TRY(ensure_ws_ext(t, s));
@@ -1428,6 +1450,7 @@ dhs_status embbag_backward_update_noalloc(dhs_table* t, const int64_t* d_keys, i
   cudaStream_t s = (cudaStream_t)stream;
   t->last_stream = s;
   t->adam_t += 1;
+  t->bwd_n += n_keys;
   if (n_keys == 0) return DHS_OK;
 
   unsigned* ka = (unsigned*)base;
