@@ -159,3 +159,49 @@ def test_shard_key_to_row_maps_follow_the_global_order():
             s.close()
         for o in oracles:
             o.close()
+
+
+def test_sharded_engine_through_nccl_with_one_rank():
+    """ShardedTable's own driver over a real NCCL process group (one rank on
+    this GPU: every call on this pool gets one GPU), against the oracle."""
+    import datetime
+    import socket
+
+    import torch.distributed as tdist
+    with socket.socket() as so:
+        so.bind(("127.0.0.1", 0))
+        port = so.getsockname()[1]
+    tdist.init_process_group("nccl", init_method=f"tcp://127.0.0.1:{port}", world_size=1, rank=0,
+                             timeout=datetime.timedelta(seconds=60))
+    rng = np.random.default_rng(3)
+    dim, lr = 32, 0.05
+    s = o = None
+    try:
+        s = ShardedTable(dim, "adagrad", block_rows=1024)
+        assert (s.world, s.rank) == (1, 0)
+        o = Oracle(dim, "adagrad")
+        for step in range(3):
+            keys, offs = _batch(rng, 600, 6, 5000)
+            pooled = host(s.forward(dev(keys), dev(offs), mode="mean"))
+            grad = rng.standard_normal((offs.size - 1, dim)).astype(np.float32)
+            s.backward_update(dev(grad), lr)
+            ref, rc = o.forward(keys, offs, None, "mean")
+            assert rc == 0
+            assert o.backward_update(keys, offs, grad, lr, None, "mean") == 0
+            if step == 0:
+                np.testing.assert_array_equal(pooled, ref)
+            else:
+                assert_close(pooled, ref, f"step {step} pooled")
+        assert dhs.ht_sync(s.table) == 0
+        gk, grows, rc = dhs.ht_export(s.table)
+        ok, orows = o.export()
+        assert rc == 0
+        np.testing.assert_array_equal(gk, ok)  # one rank owns every key, in stream order
+        assert_close(grows[:, :dim], orows[:, :dim], "weights")
+        assert_close(grows[:, dim:], orows[:, dim:], "state")
+    finally:
+        if s is not None:
+            s.close()
+        if o is not None:
+            o.close()
+        tdist.destroy_process_group()
