@@ -247,6 +247,61 @@ def test_segment_runs_at_every_chunk_alignment(n_target, dim):
             o.close()
 
 
+@pytest.mark.parametrize("dim,opt,short", [(64, "adagrad", True), (16, "adam", False), (128, "sgd", True)])
+def test_backward_with_keys_other_than_the_last_forward(dim, opt, short):
+    """Backward calls whose keys are not those of the forward just before:
+    the keys of an older forward, the same keys at other positions, a third
+    of them replaced by other known keys, more positions than the forward
+    before, and after a lookup-or-insert and growth, all against the
+    oracle."""
+    rng = np.random.default_rng(dim + (7 if short else 0))
+    t, o = make_pair(dim, opt, block_rows=512)
+    try:
+        def batch(n_bags, universe):
+            lens = rng.integers(0, 3 if short else 9, size=n_bags)
+            offs = np.concatenate([[0], np.cumsum(lens)]).astype(np.int64)
+            keys = (rng.integers(0, universe, size=int(offs[-1])) * 7 + 5).astype(np.int64)
+            return keys, offs
+
+        def fwd(keys, offs):
+            pg = host(dhs.embbag_forward(t, dev(keys), dev(offs)))
+            po, rc = o.forward(keys, offs)
+            assert rc == 0
+            assert_close(pg, po, "pooled")
+
+        def bwd(keys, offs):
+            grad = rng.standard_normal((offs.size - 1, dim)).astype(np.float32)
+            dhs.embbag_backward_update(t, dev(keys), dev(offs), dev(grad), 0.03)
+            assert o.backward_update(keys, offs, grad, 0.03) == 0
+
+        a, b = batch(800, 3000), batch(900, 3000)
+        fwd(*a)
+        fwd(*b)
+        bwd(*a)  # keys of an older forward
+        c = batch(700, 5000)
+        fwd(*c)
+        kc, oc = c
+        perm = rng.permutation(kc.size)
+        bwd(kc[perm], oc)  # same keys, other positions
+        fwd(*c)
+        mixed = kc.copy()
+        mixed[::3] = a[0][: mixed[::3].size]  # a third replaced by other known keys
+        bwd(mixed, oc)
+        d = batch(1500, 20000)  # more positions than the last forward, with growth
+        fwd(d[0][:-100], np.minimum(d[1], d[0].size - 100))
+        fwd(*d)
+        bwd(*d)
+        e = batch(400, 3000)
+        dhs.ht_lookup_or_insert(t, dev(e[0]))
+        o.lookup_or_insert(e[0])
+        bwd(*e)  # after a lookup-or-insert
+        assert dhs.ht_sync(t) == 0
+        compare_tables(t, o, f"dim {dim} {opt}")
+    finally:
+        t.close()
+        o.close()
+
+
 def test_empty_inputs_and_empty_bags():
     t, o = make_pair(16, "adam")
     try:
