@@ -106,10 +106,11 @@ constexpr unsigned long long kLbPrefix = 2ull << 62;     // inclusive prefix pub
 constexpr unsigned long long kLbCountMask = (1ull << 62) - 1;
 constexpr unsigned kLookbackSpins = 1u << 22;  // bounded wait for a predecessor tile
 constexpr int kLookbackWindow = DHS_LOOKBACK_WINDOW;  // predecessors read per look-back step
-// words cleared (one memset) before a backward's probe: digit histograms of
-// every pass, one tile counter per pass, the segment kernel's chunk counter,
-// the count of long-segment owner chunks and the combine's batch and slot
-// counters
+// the counters a backward starts from zero (cleared by the previous
+// backward's probe, or by a memset before the allocation-free backward's):
+// digit histograms of every pass, one tile counter per pass, the segment
+// kernel's chunk counter, the count of long-segment owner chunks and the
+// combine's batch and slot counters
 constexpr int kSortZeroWords = kRadixMaxPasses * kRadixBins + kRadixMaxPasses + 4;
 constexpr int kSegChunkCtrWord = kRadixMaxPasses * kRadixBins + kRadixMaxPasses;
 constexpr int kSegOwnerCtrWord = kSegChunkCtrWord + 1;
