@@ -6,8 +6,9 @@ batch of the 26-table DLRM-style merged workload (65,536 samples x 26 ids,
 pooling 1, dim 128 fp32, Adagrad, Zipf 1.05 ids; synthetic, seeded).  The
 table starts empty: warm-up steps are the stream's first steps, timed steps
 the ones after.  After the headline, the other four workloads (tiny uniform,
-sequence bags, growth stream, hot key) and the headline's and the sequence
-stream on tables with bf16 weights are each run whole with their own step counts and reported
+sequence bags, growth stream, hot key), the headline's and the sequence
+stream on tables with bf16 weights, and the headline with row-wise Adagrad
+are each run whole with their own step counts and reported
 under "workloads", with capacity reserved before step 0; the growth stream
 runs a second time with its table growing on demand inside the timed steps
 ("growth_stream:on-demand").  "e2e" repeats the headline steps through the public
@@ -115,7 +116,7 @@ def load_traffic(kernel: str):
 # ---------------------------------------------------------------------------
 class ClockSampler:
     """SM clock and clock-event reasons of this process's GPU, sampled every
-    ~10 ms by a thread through NVML while the timed region runs (two cheap
+    ~2 ms by a thread through NVML while the timed region runs (two cheap
     queries per sample, so the sampling does not stall the driver)."""
 
     REASONS = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
@@ -124,7 +125,7 @@ class ClockSampler:
                ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap"),
                ("hw_power_brake", "nvmlClocksEventReasonHwPowerBrakeSlowdown"))
 
-    def __init__(self, cuda_index: int, period_s: float = 0.01):
+    def __init__(self, cuda_index: int, period_s: float = 0.002):
         self.idx = cuda_index
         self.period = period_s
         self.samples = []
@@ -569,16 +570,54 @@ def measure(dhs, w, host_batches, device, dist, warmup: int, reserve: int, grad_
     return res
 
 
-# the other configs, each run whole: (label, workload, weight storage, capacity policy)
+# the other configs, each run whole: (label, workload, weight storage,
+# capacity policy, optimizer in place of the workload's or None)
 EXTRA_WORKLOADS = (
-    ("tiny_uniform", "tiny_uniform", "f32", "-1"),
-    ("sequence_bags", "sequence_bags", "f32", "-1"),
-    ("growth_stream", "growth_stream", "f32", "-1"),
-    ("growth_stream:on-demand", "growth_stream", "f32", "on-demand"),
-    ("hot_key", "hot_key", "f32", "-1"),
-    ("dlrm_merged_26:bf16", "dlrm_merged_26", "bf16", "-1"),
-    ("sequence_bags:bf16", "sequence_bags", "bf16", "-1"),
+    ("tiny_uniform", "tiny_uniform", "f32", "-1", None),
+    ("sequence_bags", "sequence_bags", "f32", "-1", None),
+    ("growth_stream", "growth_stream", "f32", "-1", None),
+    ("growth_stream:on-demand", "growth_stream", "f32", "on-demand", None),
+    ("hot_key", "hot_key", "f32", "-1", None),
+    ("dlrm_merged_26:bf16", "dlrm_merged_26", "bf16", "-1", None),
+    # the headline config with Adagrad's row-wise form (one accumulator per row)
+    ("dlrm_merged_26:rowwise", "dlrm_merged_26", "f32", "-1", "adagrad_rowwise"),
+    ("sequence_bags:bf16", "sequence_bags", "bf16", "-1", None),
 )
+
+
+def run_l2_peak(mib: int = 32, copies: int = 100, replays: int = 5):
+    """Copy bandwidth of buffers that stay in L2 (two 32 MiB buffers, half
+    the 126 MB L2): read + write bytes per second of `copies` back-to-back
+    copies captured in one CUDA graph (no host launch gaps), replayed
+    `replays` times after a warm-up and timed with CUDA events.  Prints one
+    JSON line."""
+    import torch
+    n = mib << 20
+    a = torch.empty(n, dtype=torch.uint8, device="cuda").fill_(1)
+    b = torch.empty_like(a)
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        for _ in range(4):
+            b.copy_(a)
+    torch.cuda.current_stream().wait_stream(s)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for i in range(copies):
+            (b if i % 2 == 0 else a).copy_(a if i % 2 == 0 else b)
+    g.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(replays):
+        g.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1)
+    del g
+    print(json.dumps({"l2_copy_gbs": 2.0 * n * copies * replays / (ms / 1e3) / 1e9, "buffer_bytes": n,
+                      "copies": copies * replays, "ms": ms, "method": "torch copy kernels in one CUDA graph"}))
+    return 0
 
 
 def run_dhs(args):
@@ -614,8 +653,10 @@ def run_dhs(args):
         else [e for e in EXTRA_WORKLOADS if e[0] in args.workloads.split(",")])
     if wanted:
         extra = {}
-        for label, name, weights, policy in wanted:
+        for label, name, weights, policy, opt in wanted:
             wx = make_workload(name, rank)
+            if opt:
+                wx.optimizer = opt
             wsteps = wx.steps
             wwarm = min(3, wsteps - 1)
             hb = src.batches(name, rank, 0, wsteps)
@@ -752,6 +793,8 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=40)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="dhs", choices=["dhs", "reference"])
+    ap.add_argument("--l2-peak", action="store_true",
+                    help="only measure the L2-resident copy bandwidth (the yardstick of L2-bound workloads)")
     ap.add_argument("--workload", default=WORKLOAD, choices=list(gen.NAMES))
     ap.add_argument("--workloads", default="all",
                     help="other configs measured after the headline, each run whole: 'all', 'none' or a "
@@ -775,6 +818,8 @@ def main(argv=None):
     PHASE_TIMING = not args.no_phases
     if args.warmup < 0 or args.steps < 1:
         ap.error("--steps must be >= 1 and --warmup >= 0")
+    if args.l2_peak:
+        return run_l2_peak()
     if args.impl == "reference":
         return run_reference(args)
     return run_dhs(args)
