@@ -55,6 +55,16 @@
 #ifndef DHS_SEG_NARROW_RUN
 #define DHS_SEG_NARROW_RUN 8
 #endif
+//   DHS_SEGW_MINB     resident blocks per SM the warp segment kernel is
+//                     compiled for (register budget) with up to 4 columns per
+//                     lane; DHS_SEGW_BATCH4 gradient rows a warp stages per
+//                     batch at 4 columns per lane (two batches in flight)
+#ifndef DHS_SEGW_MINB
+#define DHS_SEGW_MINB 3
+#endif
+#ifndef DHS_SEGW_BATCH4
+#define DHS_SEGW_BATCH4 8
+#endif
 //   DHS_SEGW_EVICT_FIRST 1: gradient rows of calls with about one id per bag
 //                     are staged with an L2 evict-first policy; 0: normal
 #ifndef DHS_SEGW_EVICT_FIRST
@@ -840,7 +850,9 @@ bwd_seg_kernel(const unsigned* __restrict__ skey, const unsigned* __restrict__ s
 // ---------------------------------------------------------------------------
 // Pairs per staged batch (two batches per warp in flight or being read): 8 KB
 // of rows per warp at every width.
-__host__ __device__ constexpr int segw_batch(int cpl) { return cpl <= 2 ? 16 : 32 / cpl; }
+__host__ __device__ constexpr int segw_batch(int cpl) {
+  return cpl <= 2 ? 16 : (cpl == 4 ? DHS_SEGW_BATCH4 : 32 / cpl);
+}
 __host__ __device__ constexpr size_t segw_smem_bytes(int cpl) {
   return (size_t)8 * 2 * segw_batch(cpl) * 32 * cpl * sizeof(float);
 }
@@ -995,7 +1007,7 @@ __device__ __forceinline__ unsigned run_slot(const RunTable& rt, unsigned row, D
 // BF: the table's weights are bf16 (state fp32): loaded widened, updated in
 // fp32, stored rounded to nearest even.
 template <int CPL, int OPT, bool EXT, bool BF>
-__global__ void __launch_bounds__(256, CPL <= 4 ? 3 : 1)
+__global__ void __launch_bounds__(256, CPL <= 4 ? DHS_SEGW_MINB : 1)
 bwd_segw_kernel(const unsigned* __restrict__ skey, const unsigned* __restrict__ sval, long long n,
                 const float* __restrict__ grad, long long n_bags, int dim, RowSpace rs, OptArgs oa,
                 double* __restrict__ part_head, double* __restrict__ part_tail, int pstride, int C,
