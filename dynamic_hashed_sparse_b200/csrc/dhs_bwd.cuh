@@ -89,6 +89,17 @@
 #ifndef DHS_PROBE_DEDUP
 #define DHS_PROBE_DEDUP 0
 #endif
+//   DHS_RADIX_MATCH   how a radix pass finds the lanes of equal digit:
+//                     0 match.any when the warp's first 32 items hold at most
+//                     DHS_RADIX_MATCH_DISTINCT distinct digits, else one
+//                     ballot per digit bit; 1 match.any always; 2 ballots
+//                     always
+#ifndef DHS_RADIX_MATCH
+#define DHS_RADIX_MATCH 0
+#endif
+#ifndef DHS_RADIX_MATCH_DISTINCT
+#define DHS_RADIX_MATCH_DISTINCT 16
+#endif
 //   DHS_LOOKBACK_WINDOW predecessor tiles a radix pass's look-back reads at once
 #ifndef DHS_LOOKBACK_WINDOW
 #define DHS_LOOKBACK_WINDOW 8
@@ -116,6 +127,7 @@ constexpr unsigned long long kLbPrefix = 2ull << 62;     // inclusive prefix pub
 constexpr unsigned long long kLbCountMask = (1ull << 62) - 1;
 constexpr unsigned kLookbackSpins = 1u << 22;  // bounded wait for a predecessor tile
 constexpr int kLookbackWindow = DHS_LOOKBACK_WINDOW;  // predecessors read per look-back step
+constexpr int kRadixMatchDistinct = DHS_RADIX_MATCH_DISTINCT;
 // the counters a backward starts from zero (cleared by the previous
 // backward's probe, or by a memset before the allocation-free backward's):
 // digit histograms of every pass, one tile counter per pass, the segment
@@ -334,7 +346,7 @@ __device__ __forceinline__ unsigned block_exclusive_scan_256(unsigned x, unsigne
 // One stable digit pass.  Tiles are numbered in the order blocks start (an
 // atomic counter), so a tile only ever waits for tiles whose blocks are
 // already running.  Each warp ranks its 32 x kRadixItems items in order
-// (kRadixItems rounds of 32 lanes; match.any gives the rank among equal digits
+// (kRadixItems rounds of 32 lanes; the lanes of equal digit give the rank
 // within a round, a per-warp shared counter carries it across rounds); the
 // tile publishes its digit counts, adds up its predecessors' (decoupled
 // look-back), publishes its inclusive prefix, places its items in digit order
@@ -377,10 +389,33 @@ radix_onesweep_kernel(const unsigned* __restrict__ kin, const unsigned* __restri
 #pragma unroll
   for (int r = 0; r < kRadixItems; ++r) k[r] = r * 32 + lane < rem ? __ldg(kb + r * 32) : 0u;
   const unsigned lt = lanemask_lt();
+  // the lanes of equal digit: match.any costs about as many steps as there
+  // are distinct digits among the 32 lanes, one ballot per digit bit a fixed
+  // nine; the number of distinct digits in the warp's first round decides
+  // for all its rounds
+  bool use_match = DHS_RADIX_MATCH == 1;
+  if (DHS_RADIX_MATCH == 0) {
+    const unsigned d0 = lane < rem ? ((k[0] >> shift) & 255u) : 256u;
+    const unsigned p0 = __match_any_sync(0xffffffffu, d0);
+    const int distinct = __popc(__ballot_sync(0xffffffffu, (__ffs(p0) - 1) == lane));
+    use_match = distinct <= kRadixMatchDistinct;
+  }
 #pragma unroll
   for (int r = 0; r < kRadixItems; ++r) {
     const unsigned d = r * 32 + lane < rem ? ((k[r] >> shift) & 255u) : 256u;
-    const unsigned peers = __match_any_sync(0xffffffffu, d);
+    // (9 bits: 256 marks an item past the end)
+    unsigned peers;
+    if (use_match) {
+      peers = __match_any_sync(0xffffffffu, d);
+    } else {
+      peers = 0xffffffffu;
+#pragma unroll
+      for (int b = 0; b < 9; ++b) {
+        const bool bit = (d >> b) & 1u;
+        const unsigned m = __ballot_sync(0xffffffffu, bit);
+        peers &= bit ? m : ~m;
+      }
+    }
     const unsigned before = wc[wid][d];
     lr[r] = before + __popc(peers & lt);
     __syncwarp();
