@@ -497,8 +497,14 @@ radix_onesweep_kernel(const unsigned* __restrict__ kin, const unsigned* __restri
     const unsigned key = s_k[i];
     const unsigned dd = (key >> shift) & 255u;
     const unsigned o = gbase[dd] + (unsigned)i - dstart[dd];
-    kout[o] = key;
-    vout[o] = s_v[i];
+    // o < n for counts that match the items; malformed bag offsets (already
+    // reported) can count a position twice, so the bound is checked
+    if (o < (unsigned)n) {
+      kout[o] = key;
+      vout[o] = s_v[i];
+    } else {
+      latch(st, kErrInvalid);
+    }
   }
 }
 

@@ -1058,25 +1058,25 @@ dhs_status embbag_backward_update_ex(dhs_table* t, const int64_t* d_keys, int64_
   unsigned* const ctr = hist_words(t);  // this backward's counters
   {
     PhaseScope ph(t, PH_BWD_PROBE, s);
-    // one resident wave of blocks, each warp taking chunks of bags in turn:
-    // each block flushes its digit counts with one atomic per nonzero bin,
-    // so fewer blocks mean fewer atomics on the shared counters
-    const int resident = resident_blocks(ext ? bwd_probe_kernel<true> : bwd_probe_kernel<false>, 256, 0,
-                                         t->sm_count);
     const int bpc = bwd_probe_bags(n_keys, n_bags);
-    const long long warps = (n_bags + bpc - 1) / bpc;
-    const long long grid = grid_for((warps + 7) / 8, resident);
     const long long ntiles = (n_keys + kRadixTile - 1) / kRadixTile;
     // the counters this backward accumulates into are zero (cleared by the
     // previous backward's probe, or at allocation); this probe clears the
     // other area for the next one
     unsigned* next_hist = (unsigned*)t->b_hist.p + (size_t)(1 - t->hist_sel) * kSortZeroWords;
+    const long long zero_runs = 2 * ((long long)run_table(t, n_keys).mask + 1);
+    // one resident wave of blocks, each warp taking chunks of bags in turn:
+    // each block flushes its digit counts with one atomic per nonzero bin,
+    // so fewer blocks mean fewer atomics on the shared counters
+    const int resident = resident_blocks(ext ? bwd_probe_kernel<true> : bwd_probe_kernel<false>, 256, 0,
+                                         t->sm_count);
+    const long long warps = (n_bags + bpc - 1) / bpc;
+    const long long grid = grid_for((warps + 7) / 8, resident);
     (void)launch_k(ext ? bwd_probe_kernel<true> : bwd_probe_kernel<false>, (unsigned)grid, 256, 0, s, idmap(t),
-                   (const long long*)d_keys, n_keys, (const long long*)d_bag_offsets, n_bags, ka, va, sentinel,
-                   ctr, passes, (unsigned long long*)t->b_totals.p, ntiles * kRadixBins,
-                   (unsigned*)t->b_runs.p, 2 * ((long long)run_table(t, n_keys).mask + 1), next_hist,
-                   (long long)kSortZeroWords, bpc, psw, mean, (unsigned*)t->b_bagpos.p, (double*)t->b_mult.p,
-                   t->st);
+                   (const long long*)d_keys, n_keys, (const long long*)d_bag_offsets, n_bags, ka, va, sentinel, ctr,
+                   passes, (unsigned long long*)t->b_totals.p, ntiles * kRadixBins, (unsigned*)t->b_runs.p,
+                   zero_runs, next_hist, (long long)kSortZeroWords, bpc, psw, mean, (unsigned*)t->b_bagpos.p,
+                   (double*)t->b_mult.p, t->st);
     t->n_launches++;
     DHS_TRY(last_launch());
     t->hist_sel ^= 1;  // the next backward uses the area this probe cleared
