@@ -65,6 +65,11 @@
 #ifndef DHS_SEGW_BATCH4
 #define DHS_SEGW_BATCH4 8
 #endif
+//   DHS_SEGW_REVERSE  1: the warp segment kernel takes its chunks from the
+//                     last to the first; 0: in order
+#ifndef DHS_SEGW_REVERSE
+#define DHS_SEGW_REVERSE 1
+#endif
 //   DHS_SEGW_EVICT_FIRST 1: gradient rows of calls with about one id per bag
 //                     are staged with an L2 evict-first policy; 0: normal
 #ifndef DHS_SEGW_EVICT_FIRST
@@ -82,7 +87,7 @@
 //   DHS_SEG_FINISH_PIECES pieces of a long segment the segment kernel's warp
 //                     adds itself (longer ones go to the combine kernels)
 #ifndef DHS_SEG_FINISH_PIECES
-#define DHS_SEG_FINISH_PIECES 256
+#define DHS_SEG_FINISH_PIECES 32
 #endif
 //   DHS_PROBE_DEDUP   1: the backward probe probes a key held by several lanes
 //                     of a warp once (match.any); 0: every lane probes
@@ -1093,6 +1098,11 @@ bwd_segw_kernel(const unsigned* __restrict__ skey, const unsigned* __restrict__ 
     if (lane == 0) c = (int)atomicAdd(chunk_ctr, 1u);
     c = __shfl_sync(FULL, c, 0);
     if (c >= nchunks) break;
+    // chunks are handed out from the end of the sorted pairs: rows sort in
+    // the order they were created, so the high rows (keys seen recently, in
+    // short segments, a row update every few pairs: the slow chunks) go
+    // first and the chunks inside long segments of old hot rows last
+    if (DHS_SEGW_REVERSE) c = nchunks - 1 - c;
     const int start = c * C;
     const int end = min(n32, start + C);
     const int limit = min(n32, end + C);  // an owned run ends before chunk c + 2

@@ -179,12 +179,12 @@ def test_dims_and_optimizers(dim, opt, bags):
         o.close()
 
 
-@pytest.mark.parametrize("occ", [255, 256, 257, 600, 5000, 8150, 8200, 8250, 40000])
+@pytest.mark.parametrize("occ", [255, 256, 257, 600, 1000, 1030, 1060, 5000, 8200, 40000])
 def test_hot_key_spanning_many_sort_chunks(occ):
     """One key occurs `occ` times (its run covers one sort chunk of 32 pairs up
     to hundreds of them), mixed with a tail of other keys before and after it
     in row order; both segment kernels (narrow and wide rows).  Runs of about
-    256 chunks (8,150 to 8,250 occurrences) sit at the boundary between a long
+    32 chunks (1,000 to 1,060 occurrences) sit at the boundary between a long
     segment that the wide segment kernel's warp finishes and one that goes to
     the combine kernels."""
     rng = np.random.default_rng(occ)
