@@ -147,6 +147,7 @@ struct dhs_table {
   unsigned long long nslots = 0;
   long long n_rehash = 0;
   long long n_insert_calls = 0;
+  long long n_pool_calls = 0;  // fused pool launches (their chunk counters alternate)
   long long n_launches = 0;  // kernels launched by this table's calls
   long long n_host_waits = 0, host_wait_ns = 0;  // host blocked on the device
   long long n_allocs = 0, alloc_ns = 0;          // device allocations
@@ -595,10 +596,14 @@ dhs_status dispatch_pool(dhs_table* t, const long long* keys, long long n, const
       (t->wbf16 ? launch_probe_pool_bf16 : launch_probe_pool)(G, NV, t->sm_count, idmap(t), rowspace(t), t->dim,
                                                               keys, n, bo, nb, psw, mean, out,
                                                               (unsigned*)t->b_nbm.p, (unsigned*)t->b_slotpos.p,
-                                                              t->st, s);
+                                                              (int)(t->n_pool_calls & 1), t->st, s);
   t->n_launches++;
-  if (e != cudaSuccess) cudaGetLastError();
-  return e == cudaSuccess ? DHS_OK : DHS_ERR_CUDA;
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return DHS_ERR_CUDA;
+  }
+  t->n_pool_calls++;  // the launch cleared the other counter for the next one
+  return DHS_OK;
 }
 
 // Bags per warp of the backward probe: 64 when bags are short (two positions

@@ -71,6 +71,7 @@ struct DevState {
   unsigned int ticket;           // last-block-done counter (mark kernel)
   unsigned int ticket2;          // last-block-done counter (free-list compaction)
   unsigned int pad;
+  unsigned int fwd_ctr[2];       // chunk counters of the forward's pool kernels (one per call, alternating)
 };
 
 enum : unsigned { kErrInvalid = 1u, kErrFull = 4u, kErrNotFound = 5u, kErrInternal = 7u };

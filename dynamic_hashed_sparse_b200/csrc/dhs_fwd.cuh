@@ -195,6 +195,19 @@ __device__ __forceinline__ void flush_bags(float4 (&acc)[NV * RowUnit<BF>::CV], 
   }
 }
 
+//   DHS_POOL_DYNAMIC  1: the fused pool kernel's groups take chunks of bags
+//                     from a counter; 0: every ngroups-th chunk
+#ifndef DHS_POOL_DYNAMIC
+#define DHS_POOL_DYNAMIC 1
+#endif
+
+// The next chunk for a group of G lanes, from the call's counter.
+__device__ __forceinline__ int pool_fetch(unsigned* ctr, unsigned gmask, int gl, int G) {
+  unsigned c = 0;
+  if (gl == 0) c = atomicAdd(ctr, 1u);
+  return (int)__shfl_sync(gmask, c, 0, G);
+}
+
 // Fused lookup-or-insert + gather + sum pooling.  A group of G lanes owns a
 // chunk of G consecutive bags; it probes the chunk's ids G at a time (one id
 // per lane; the probing lane also forms the row address), then walks those ids
@@ -210,7 +223,7 @@ fwd_probe_pool_kernel(IdMap m, RowSpace rs, int dim, const long long* __restrict
                       long long n_keys, const long long* __restrict__ bag_off, long long n_bags,
                       const float* __restrict__ psw,
                       float* __restrict__ out, unsigned* __restrict__ nbm,
-                      unsigned* __restrict__ slotpos, DevState* st) {
+                      unsigned* __restrict__ slotpos, int ctr_sel, DevState* st) {
   pdl_enter();
   constexpr bool W = PM == 1, MEAN = PM == 2;
   const int lane = threadIdx.x & 31;
@@ -224,7 +237,15 @@ fwd_probe_pool_kernel(IdMap m, RowSpace rs, int dim, const long long* __restrict
   constexpr int CV = RowUnit<BF>::CV;
   const int du = BF ? dim >> 3 : dim >> 2;  // 16-byte units of a row's weights
 
+#if DHS_POOL_DYNAMIC
+  // chunks handed out one at a time from this call's counter, so that groups
+  // whose chunks take longer take fewer; the next call's counter is cleared
+  unsigned* const ctr = &st->fwd_ctr[ctr_sel];
+  if (blockIdx.x == 0 && threadIdx.x == 0) st->fwd_ctr[ctr_sel ^ 1] = 0u;
+  for (int c = pool_fetch(ctr, gmask, gl, G); c < nchunks; c = pool_fetch(ctr, gmask, gl, G)) {
+#else
   for (int c = gid; c < nchunks; c += ngroups) {
+#endif
     const long long b0 = (long long)c * G;
     const int nb = (int)min((long long)G, n_bags - b0);
     long long s64;

@@ -43,7 +43,7 @@ int blocks_per_sm(const void* kernel, int threads, size_t smem);
 cudaError_t launch_probe_pool(int G, int NV, int sm_count, IdMap m, RowSpace rs, int dim,
                               const long long* keys, long long n_keys, const long long* bag_off,
                               long long n_bags, const float* psw, bool mean, float* out, unsigned* nbm,
-                              unsigned* slotpos, DevState* st, cudaStream_t s);
+                              unsigned* slotpos, int ctr_sel, DevState* st, cudaStream_t s);
 
 // fwd_pool_refs_kernel<G, NV, PM> (gather + pool from per-id row references)
 cudaError_t launch_pool_refs(int G, int NV, int sm_count, RowSpace rs, int dim, const Slot* slots,
@@ -55,7 +55,7 @@ cudaError_t launch_pool_refs(int G, int NV, int sm_count, RowSpace rs, int dim, 
 cudaError_t launch_probe_pool_bf16(int G, int NV, int sm_count, IdMap m, RowSpace rs, int dim,
                                    const long long* keys, long long n_keys, const long long* bag_off,
                                    long long n_bags, const float* psw, bool mean, float* out, unsigned* nbm,
-                                   unsigned* slotpos, DevState* st, cudaStream_t s);
+                                   unsigned* slotpos, int ctr_sel, DevState* st, cudaStream_t s);
 cudaError_t launch_pool_refs_bf16(int G, int NV, int sm_count, RowSpace rs, int dim, const Slot* slots,
                                   const long long* refs, long long n_keys, const long long* bag_off,
                                   long long n_bags, const float* psw, bool mean, float* out, DevState* st,

@@ -7,9 +7,9 @@ namespace dhs {
 cudaError_t launch_probe_pool(int G, int NV, int sm_count, IdMap m, RowSpace rs, int dim,
                               const long long* keys, long long n_keys, const long long* bag_off,
                               long long n_bags, const float* psw, bool mean, float* out, unsigned* nbm,
-                              unsigned* slotpos, DevState* st, cudaStream_t s) {
+                              unsigned* slotpos, int ctr_sel, DevState* st, cudaStream_t s) {
 #define DHS_RUN(g, v) \
-  pool_impl::run_form<g, v, false>(sm_count, m, rs, dim, keys, n_keys, bag_off, n_bags, psw, mean, out, nbm, slotpos, st, s)
+  pool_impl::run_form<g, v, false>(sm_count, m, rs, dim, keys, n_keys, bag_off, n_bags, psw, mean, out, nbm, slotpos, ctr_sel, st, s)
   switch (G * 100 + NV) {
     case 101: return DHS_RUN(1, 1);
     case 201: return DHS_RUN(2, 1);
