@@ -51,7 +51,9 @@ METRIC = "IDs/sec & HBM GB/s (% of peak): hashed lookup+bag-sum fwd, sparse upda
 UNIT = "IDs/s"
 # kernel selection thresholds of the library (compile-time constants there)
 POOL_SPLIT_LEN = 4   # bags of >= 4 ids on average: probe kernel + gather from references
-SEGW_MIN_DIM = 32    # rows of >= 32 floats: warp-per-chunk segment kernel
+SEGW_MIN_DIM = 32    # rows of >= 32 floats: warp-per-chunk segment kernel ...
+NARROW_MAX_DIM = 64  # ... except fp32 rows of 33-64 floats with fewer than
+NARROW_RUN = 8       # 8 ids per updated row on average: the lane-group kernel
 WORKLOAD = "dlrm_merged_26"
 
 
@@ -92,6 +94,15 @@ def load_peaks() -> dict:
             d = json.load(f)
         return dict(hbm_gbs=float(d["hbm_gbs"]), source="measured")
     return dict(hbm_gbs=6650.0, source="fallback")
+
+
+def narrow_seg(dim: int, weights: str, n_ids: int, unique: int) -> bool:
+    """Which segment kernel the library runs (the lane-group one for narrow
+    rows, and for fp32 rows of 33-64 floats whose rows get few ids)."""
+    if dim < SEGW_MIN_DIM:
+        return True
+    return (weights == "f32" and SEGW_MIN_DIM < dim <= NARROW_MAX_DIM and unique > 0
+            and n_ids < NARROW_RUN * unique)
 
 
 def load_traffic(kernel: str):
@@ -517,7 +528,8 @@ def measure(dhs, w, host_batches, device, dist, warmup: int, reserve: int, grad_
     dom = max(("fwd_probe_pool", "bwd_seg_update"), key=lambda k: ph_ms.get(k, 0.0))
     dom_kernel = {"fwd_probe_pool": ("fwd_pool_refs_kernel" if n_ids >= POOL_SPLIT_LEN * n_bags
                                      else "fwd_probe_pool_kernel"),
-                  "bwd_seg_update": "bwd_segw_kernel" if w.dim >= SEGW_MIN_DIM else "bwd_seg_kernel"}[dom]
+                  "bwd_seg_update": "bwd_seg_kernel" if narrow_seg(w.dim, weights, n_ids, U)
+                  else "bwd_segw_kernel"}[dom]
     dom_bytes = ((ab["fwd_refs"] if dom_kernel == "fwd_pool_refs_kernel" else ab["fwd_pool"])
                  if dom == "fwd_probe_pool" else ab["bwd_seg"])
     dom_launch_ms = ph_ms.get(dom, 0.0) / max(1, ph_cnt.get(dom, 0))
