@@ -576,8 +576,11 @@ fwd_mark_kernel(Slot* __restrict__ slots, unsigned* __restrict__ nbm,
 // fastest (more blocks per group repeat the prefix and the key gathering for
 // fewer rows each).
 constexpr int kAssignSplit = 1;
+#ifndef DHS_ASSIGN_COLUMNS
+#define DHS_ASSIGN_COLUMNS 1  // column-per-thread row initialisation (0: flat index loop only)
+#endif
 
-__global__ void __launch_bounds__(kGroupThreads)
+__global__ void __launch_bounds__(kGroupThreads, 2)
 fwd_assign_kernel(Slot* __restrict__ slots, RowSpace rs, int dim, const long long* __restrict__ keys,
                   const unsigned* __restrict__ fbm, const unsigned* __restrict__ gpref,
                   const unsigned* __restrict__ slotpos, long long nwords, long long ngroups,
@@ -662,6 +665,38 @@ fwd_assign_kernel(Slot* __restrict__ slots, RowSpace rs, int dim, const long lon
   const unsigned long long qfirst = rank0 + r_lo;
   const bool contiguous = qfirst >= m_free;
   const unsigned long long rfirst = contiguous ? row_of(qfirst) : 0;
+#if DHS_ASSIGN_COLUMNS
+  // Common case: appended rows, all below the limit, and a row's 16-byte
+  // units (weights, then state) dividing the block's threads.  Each thread
+  // then keeps one column of the run (its hash offset loop-invariant) and
+  // steps over rows, one EmbeddingBlock piece of the run at a time.
+  const int nrows = (int)(r_hi - r_lo), sd = s4 - du;
+  if (contiguous && rfirst + (unsigned long long)nrows <= limit && du <= kGroupThreads &&
+      kGroupThreads % du == 0 && (sd == 0 || (sd <= kGroupThreads && kGroupThreads % sd == 0))) {
+    const int wc = threadIdx.x % du, wstep = kGroupThreads / du;
+    for (int r0 = 0; r0 < nrows;) {
+      const unsigned long long row0 = rfirst + (unsigned long long)r0;
+      const int len = (int)min((unsigned long long)(nrows - r0), (rs.br_mask + 1) - (row0 & rs.br_mask));
+      float4* const b = reinterpret_cast<float4*>(rs.row(row0));
+      const unsigned long long* const kr = skey + r_lo + r0;
+      if (!bf) {
+        for (int r = threadIdx.x / du; r < len; r += wstep) b[(size_t)r * s4 + wc] = init_weight4(kr[r], wc * 4);
+      } else {
+        for (int r = threadIdx.x / du; r < len; r += wstep) {
+          const float4 a = init_weight4(kr[r], wc * 8), c = init_weight4(kr[r], wc * 8 + 4);
+          reinterpret_cast<uint4*>(b)[(size_t)r * s4 + wc] =
+              make_uint4(pack_bf16x2(a.x, a.y), pack_bf16x2(a.z, a.w), pack_bf16x2(c.x, c.y), pack_bf16x2(c.z, c.w));
+        }
+      }
+      if (sd > 0) {
+        const int sc = threadIdx.x % sd, sstep = kGroupThreads / sd;
+        for (int r = threadIdx.x / sd; r < len; r += sstep) b[(size_t)r * s4 + du + sc] = make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+      r0 += len;
+    }
+    return;
+  }
+#endif
   const unsigned long long in_block = (rs.br_mask + 1) - (rfirst & rs.br_mask);
   float4* const base = contiguous && rfirst < limit ? reinterpret_cast<float4*>(rs.row(rfirst)) : nullptr;
   for (int idx = threadIdx.x; idx < work; idx += kGroupThreads) {
