@@ -106,6 +106,12 @@
 #define DHS_RADIX_MATCH_DISTINCT 16
 #endif
 //   DHS_LOOKBACK_WINDOW predecessor tiles a radix pass's look-back reads at once
+//   DHS_BWD_RECORD   1: the backward probe reads the rows a split forward
+//                    recorded per position where the keys are the same; 0:
+//                    it always probes the IDMap
+#ifndef DHS_BWD_RECORD
+#define DHS_BWD_RECORD 1
+#endif
 #ifndef DHS_LOOKBACK_WINDOW
 #define DHS_LOOKBACK_WINDOW 8
 #endif
@@ -150,6 +156,10 @@ constexpr int kCombineSlotCtrWord = kSegChunkCtrWord + 3;
 // is the number of the chunk's bag ends at or before it (a binary search over
 // the ends held in the lanes' registers).  Missing or negative keys get row
 // `sentinel` (sorted last, never updated).
+// rec_keys / rec_rows (both null, or both set): the last forward's keys and
+// rows per position (a split forward over the same number of positions);
+// a position whose key equals the recorded one takes the recorded row
+// without probing the IDMap.
 // Extended pooling (per-sample weights psw, or mean pooling): the sort value
 // is the position instead of the bag; bagpos[p] = its bag and mult[p] = its
 // weight psw[p] (the bag's gradient is multiplied by it) or, for mean
@@ -163,7 +173,8 @@ bwd_probe_kernel(IdMap m, const long long* __restrict__ keys, long long n_keys,
                  long long status0_words, unsigned* __restrict__ zero32, long long zero32_words,
                  unsigned* __restrict__ next_ctr, long long next_ctr_words, int bpc,
                  const float* __restrict__ psw, bool mean, unsigned* __restrict__ bagpos,
-                 double* __restrict__ mult, DevState* st) {
+                 double* __restrict__ mult, const long long* __restrict__ rec_keys,
+                 const long long* __restrict__ rec_rows, DevState* st) {
   pdl_enter();
   constexpr bool ext = EXT;
   constexpr unsigned FULL = 0xffffffffu;
@@ -264,6 +275,16 @@ bwd_probe_kernel(IdMap m, const long long* __restrict__ keys, long long n_keys,
       const long long k0 = p0 < E ? __ldg(keys + p0) : 0;
       const long long k1 = p1 < E ? __ldg(keys + p1) : 0;
       long long f0 = -1, f1 = -1;
+      if (rec_keys) {
+        // the forward's record of these positions: where its key is this
+        // key, its row (or no row) stands, and only other keys are probed
+        const long long q0 = p0 < E ? __ldg(rec_keys + p0) : 0, r0 = p0 < E ? __ldg(rec_rows + p0) : 0;
+        const long long q1 = p1 < E ? __ldg(rec_keys + p1) : 0, r1 = p1 < E ? __ldg(rec_rows + p1) : 0;
+        if (p0 < E && k0 >= 0)
+          f0 = q0 == k0 && r0 >= 0 ? r0 : (q0 == k0 && r0 == kRecNoRow ? -2 : probe_find(m, (unsigned long long)k0));
+        if (p1 < E && k1 >= 0)
+          f1 = q1 == k1 && r1 >= 0 ? r1 : (q1 == k1 && r1 == kRecNoRow ? -2 : probe_find(m, (unsigned long long)k1));
+      } else {
 #if DHS_PROBE_DEDUP
       // a key held by several lanes is probed once, by the lowest of them
       const unsigned long long q0 = p0 < E && k0 >= 0 ? (unsigned long long)k0 : ~0ull;
@@ -278,6 +299,7 @@ bwd_probe_kernel(IdMap m, const long long* __restrict__ keys, long long n_keys,
       if (p0 < E && k0 >= 0) f0 = probe_find(m, (unsigned long long)k0);
       if (p1 < E && k1 >= 0) f1 = probe_find(m, (unsigned long long)k1);
 #endif
+      }
       const int g0 = singles ? p0 - s : bag_of(p0), g1 = singles ? p1 - s : bag_of(p1);
       // f < 0: no row (-1 absent: an error; -2 known but not admitted: skipped)
       if (p0 < E) {

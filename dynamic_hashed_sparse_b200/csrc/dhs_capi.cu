@@ -186,8 +186,11 @@ struct dhs_table {
   long long ws_n = -1;
   long long ws_chunks = 0;  // chunk capacity of the segment and combine buffers
   Buf b_nbm, b_fbm, b_gcnt, b_gpref, b_slotpos, b_ka, b_va, b_kb, b_vb, b_hist, b_totals, b_ph,
-      b_pt, b_owners, b_cplan, b_slots, b_refs, b_bagpos, b_mult, b_runs, b_shard;
+      b_pt, b_owners, b_cplan, b_slots, b_refs, b_bagpos, b_mult, b_runs, b_shard, b_reckey;
   long long ws_run_cap = 0;  // entries of the long-segment arrival table
+  // positions of the last insert call when it was a split forward, whose
+  // keys (b_reckey) and rows (b_refs) are recorded per position; -1: none
+  long long rec_n = -1;
   int hist_sel = 0;          // which half of b_hist the next backward uses (the probe clears the other)
 
   int timing = 0;  // 0 off, 1 every phase, 2 the IDMap growth phase only
@@ -516,6 +519,7 @@ CombinePlan combine_plan(unsigned* words, double* slots, long long nchunks, unsi
 
 dhs_status ensure_ws(dhs_table* t, long long n, cudaStream_t s) {
   if (n <= t->ws_n) return DHS_OK;
+  t->rec_n = -1;  // the record does not survive a reallocation
   long long cap = std::max<long long>(n, t->ws_n > 0 ? t->ws_n + t->ws_n / 2 : 0);
   cap = std::max<long long>(cap, 4096);
   const long long ngroups = (cap + kGroupPositions - 1) / kGroupPositions + 1;
@@ -529,6 +533,7 @@ dhs_status ensure_ws(dhs_table* t, long long n, cudaStream_t s) {
   DHS_TRY(bget(t, t->b_gpref, ngroups * 4, s));
   DHS_TRY(bget(t, t->b_slotpos, cap * 4, s));
   DHS_TRY(bget(t, t->b_refs, cap * 8, s));
+  DHS_TRY(bget(t, t->b_reckey, cap * 8, s));
   DHS_TRY(bget(t, t->b_ka, cap * 4, s));
   DHS_TRY(bget(t, t->b_va, cap * 4, s));
   DHS_TRY(bget(t, t->b_kb, cap * 4, s));
@@ -852,7 +857,8 @@ dhs_status ht_destroy(dhs_table* t) {
   if (t->free_list) dfree(t, t->free_list, (size_t)t->free_list_cap * 4, s);
   Buf* bufs[] = {&t->b_fcnt, &t->b_freed, &t->b_nbm, &t->b_fbm, &t->b_gcnt, &t->b_gpref, &t->b_slotpos, &t->b_ka, &t->b_va,
                  &t->b_kb, &t->b_vb, &t->b_hist, &t->b_totals, &t->b_ph, &t->b_pt, &t->b_owners,
-                 &t->b_cplan, &t->b_slots, &t->b_refs, &t->b_bagpos, &t->b_mult, &t->b_runs, &t->b_shard};
+                 &t->b_cplan, &t->b_slots, &t->b_refs, &t->b_bagpos, &t->b_mult, &t->b_runs, &t->b_shard,
+                 &t->b_reckey};
   for (Buf* b : bufs) bfree(t, *b, s);
   cudaStreamSynchronize(s);
   for (auto& sn : t->snaps) {
@@ -873,6 +879,7 @@ dhs_status ht_destroy(dhs_table* t) {
 dhs_status ht_reserve(dhs_table* t, int64_t n_keys, dhs_stream stream) {
   DHS_TRY(check_table(t));
   if (n_keys < 0) return DHS_ERR_INVALID_ARG;
+  t->rec_n = -1;
   DeviceGuard g(t->device);
   cudaStream_t s = (cudaStream_t)stream;
   t->last_stream = s;
@@ -896,6 +903,7 @@ dhs_status ht_lookup_or_insert(dhs_table* t, const int64_t* d_keys, int64_t n,
                                int64_t* d_offsets_out, dhs_stream stream) {
   DHS_TRY(check_table(t));
   if (n < 0 || n >= (1ll << 31) || (n > 0 && (!d_keys || !d_offsets_out))) return DHS_ERR_INVALID_ARG;
+  t->rec_n = -1;
   if (n == 0) {
     t->step++;  // every insert call is a step of the access stamps
     return DHS_OK;
@@ -910,7 +918,7 @@ dhs_status ht_lookup_or_insert(dhs_table* t, const int64_t* d_keys, int64_t n,
     PhaseScope ph(t, PH_LOOKUP_INSERT, s);
     launch_k(fwd_probe_offsets_kernel, (unsigned)((n + kFwdThreads - 1) / kFwdThreads), kFwdThreads, 0, s, 
         idmap(t), (const long long*)d_keys, n, (long long*)d_offsets_out, (unsigned*)t->b_nbm.p,
-        (unsigned*)t->b_slotpos.p, hooks(t), t->st);
+        (unsigned*)t->b_slotpos.p, (long long*)nullptr, hooks(t), t->st);
     t->n_launches += 2;
     DHS_TRY(last_launch());
     DHS_TRY(launch_assign(t, (const long long*)d_keys, n, s));
@@ -950,6 +958,7 @@ dhs_status embbag_forward_ex(dhs_table* t, const int64_t* d_keys, int64_t n_keys
   if (mode == DHS_POOL_MEAN && d_per_sample_weights) return DHS_ERR_INVALID_ARG;
   const bool mean = mode == DHS_POOL_MEAN;
   const float* psw = n_keys > 0 ? d_per_sample_weights : nullptr;
+  t->rec_n = -1;
   if (n_bags == 0) {
     if (n_keys != 0) return DHS_ERR_INVALID_ARG;
     t->step++;  // every insert call is a step of the access stamps
@@ -972,7 +981,7 @@ dhs_status embbag_forward_ex(dhs_table* t, const int64_t* d_keys, int64_t n_keys
       PhaseScope ph(t, PH_FWD_PROBE, s);
       launch_k(fwd_probe_offsets_kernel, (unsigned)((n_keys + kFwdThreads - 1) / kFwdThreads), kFwdThreads, 0, s, 
           idmap(t), (const long long*)d_keys, n_keys, (long long*)t->b_refs.p, (unsigned*)t->b_nbm.p,
-          (unsigned*)t->b_slotpos.p, hooks(t), t->st);
+          (unsigned*)t->b_slotpos.p, (long long*)t->b_reckey.p, hooks(t), t->st);
       t->n_launches++;
       DHS_TRY(last_launch());
     }
@@ -985,7 +994,7 @@ dhs_status embbag_forward_ex(dhs_table* t, const int64_t* d_keys, int64_t n_keys
       const int wd = t->wbf16 ? t->dim / 2 : t->dim;
       const int G = pick_group(wd), NV = pick_nv(wd, G);
       const cudaError_t e = (t->wbf16 ? launch_pool_refs_bf16 : launch_pool_refs)(
-          G, NV, t->sm_count, rowspace(t), t->dim, t->slots, (const long long*)t->b_refs.p, n_keys,
+          G, NV, t->sm_count, rowspace(t), t->dim, t->slots, (long long*)t->b_refs.p, n_keys,
           (const long long*)d_bag_offsets, n_bags, psw, mean, d_pooled_out, t->st, s);
       t->n_launches++;
       if (e != cudaSuccess) {
@@ -993,6 +1002,7 @@ dhs_status embbag_forward_ex(dhs_table* t, const int64_t* d_keys, int64_t n_keys
         return DHS_ERR_CUDA;
       }
     }
+    t->rec_n = n_keys;  // keys and rows of every position recorded
   } else {
     {
       PhaseScope ph(t, PH_FWD_POOL, s);
@@ -1065,6 +1075,9 @@ dhs_status embbag_backward_update_ex(dhs_table* t, const int64_t* d_keys, int64_
     PhaseScope ph(t, PH_BWD_PROBE, s);
     const int bpc = bwd_probe_bags(n_keys, n_bags);
     const long long ntiles = (n_keys + kRadixTile - 1) / kRadixTile;
+    // the last insert call was a split forward over as many positions: its
+    // record of keys and rows stands in for the probe where the keys agree
+    const bool rec = DHS_BWD_RECORD && t->rec_n == n_keys;
     // the counters this backward accumulates into are zero (cleared by the
     // previous backward's probe, or at allocation); this probe clears the
     // other area for the next one
@@ -1081,7 +1094,8 @@ dhs_status embbag_backward_update_ex(dhs_table* t, const int64_t* d_keys, int64_
                    (const long long*)d_keys, n_keys, (const long long*)d_bag_offsets, n_bags, ka, va, sentinel, ctr,
                    passes, (unsigned long long*)t->b_totals.p, ntiles * kRadixBins, (unsigned*)t->b_runs.p,
                    zero_runs, next_hist, (long long)kSortZeroWords, bpc, psw, mean, (unsigned*)t->b_bagpos.p,
-                   (double*)t->b_mult.p, t->st);
+                   (double*)t->b_mult.p, rec ? (const long long*)t->b_reckey.p : nullptr,
+                   rec ? (const long long*)t->b_refs.p : nullptr, t->st);
     t->n_launches++;
     DHS_TRY(last_launch());
     t->hist_sel ^= 1;  // the next backward uses the area this probe cleared
@@ -1177,6 +1191,7 @@ dhs_status ht_set_hooks(dhs_table* t, int64_t admit_threshold, int track_access)
 dhs_status ht_evict(dhs_table* t, int64_t max_idle, int64_t* n_freed, dhs_stream stream) {
   DHS_TRY(check_table(t));
   if (!t->track || max_idle < 0 || !n_freed) return DHS_ERR_INVALID_ARG;
+  t->rec_n = -1;  // evicted keys lose their rows
   DeviceGuard g(t->device);
   cudaStream_t s = (cudaStream_t)stream;
   t->last_stream = s;
@@ -1489,7 +1504,7 @@ dhs_status embbag_backward_update_noalloc(dhs_table* t, const int64_t* d_keys, i
                                                     (const long long*)d_bag_offsets, n_bags, ka, va,
                                                     sentinel, hist, passes, status, ntiles * kRadixBins,
                                                     nullptr, 0, nullptr, 0, bpc, nullptr, false, nullptr, nullptr,
-                                                    t->st);
+                                                    nullptr, nullptr, t->st);
     DHS_TRY(last_launch());
   }
   const long long ntiles = (n_keys + kRadixTile - 1) / kRadixTile;

@@ -16,6 +16,7 @@
 // (fp32), a multiple of 4 floats so every row is 16-byte aligned.
 #pragma once
 
+#include <climits>
 #include <cstdint>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -48,6 +49,9 @@ constexpr unsigned long long kPending = 1ull << 63;
 // Between calls, the value of a key that is known but has no row yet (not
 // admitted): above every PENDING | position, so a claim's atomicMin replaces it.
 constexpr unsigned long long kCounting = ~1ull;
+// The forward's per-position record of a key without a row (known but not
+// admitted, or not placed because the table was full).
+constexpr long long kRecNoRow = LLONG_MIN;
 
 struct __align__(16) Slot {
   unsigned long long key;

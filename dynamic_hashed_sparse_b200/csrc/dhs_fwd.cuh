@@ -315,11 +315,13 @@ fwd_probe_pool_kernel(IdMap m, RowSpace rs, int dim, const long long* __restrict
 // window two ahead (and the slot values of the next window's new ids) are
 // loaded while the current window is gathered, so no window waits on a probe.
 // Bags, windows and the order of additions are those of fwd_probe_pool_kernel,
-// and so is the pooling form PM.
+// and so is the pooling form PM.  The reference of a new key's position is
+// replaced by its row (kRecNoRow: none), so that after the call refs[p] is
+// the row of position p for every key that has one.
 template <int G, int NV, int PM, bool BF>
 __global__ void __launch_bounds__(kFwdThreads, NV == 1 ? 4 : (NV == 2 ? 2 : 1))
 fwd_pool_refs_kernel(RowSpace rs, int dim, const Slot* __restrict__ slots,
-                     const long long* __restrict__ refs, long long n_keys,
+                     long long* __restrict__ refs, long long n_keys,
                      const long long* __restrict__ bag_off, long long n_bags,
                      const float* __restrict__ psw,
                      float* __restrict__ out, DevState* st) {
@@ -350,7 +352,7 @@ fwd_pool_refs_kernel(RowSpace rs, int dim, const Slot* __restrict__ slots,
     for (int q = 0; q < NV * CV; ++q) acc[q] = make_float4(0.f, 0.f, 0.f, 0.f);
     float* outb = out + b0 * (long long)dim;
 
-    auto ref_at = [&](int p) -> long long { return p < E ? __ldg(refs + p) : -1; };
+    auto ref_at = [&](int p) -> long long { return p < E ? refs[p] : -1; };
     auto w_at = [&](int p) -> float { return (W && p < E) ? __ldg(psw + p) : 0.f; };
     long long r0 = ref_at(s + gl), r1 = ref_at(s + G + gl);
     float w0 = w_at(s + gl);
@@ -374,9 +376,13 @@ fwd_pool_refs_kernel(RowSpace rs, int dim, const Slot* __restrict__ slots,
         if (rc >= 0) {
           kind = kHit;
           ref = (unsigned long long)rs.row((unsigned long long)rc);
-        } else if (rc <= -2 && !(nc & kPending)) {
-          kind = kHit;
-          ref = (unsigned long long)rs.row(nc);
+        } else if (rc <= -2) {
+          if (!(nc & kPending)) {
+            kind = kHit;
+            ref = (unsigned long long)rs.row(nc);
+          }
+          // the reference left for the backward: the row, or no row
+          refs[ws + gl] = (nc & kPending) ? kRecNoRow : (long long)nc;
         }
       }
       pool_window<G, NV, false, W, MEAN, BF>(kind, ref, wc, cnt, ws, gmask, gl, du, dim, e, acc, cur, cur_end,
@@ -392,16 +398,21 @@ fwd_pool_refs_kernel(RowSpace rs, int dim, const Slot* __restrict__ slots,
 // this call, or not admitted: resolved by fwd_fixup_kernel or by the gather)
 // and -1 for a negative key.  With hooks, every key's slot is stamped with
 // the call's step, a key without a row has its occurrence counted, and the
-// slots taken from empty are counted in keys_used.
+// slots taken from empty are counted in keys_used.  rec_keys (may be null)
+// gets a copy of the keys: with offsets_out (once fwd_pool_refs_kernel has
+// put the new keys' rows in) it is the call's record of key and row per
+// position, which a backward on the same keys reads instead of probing.
 __global__ void __launch_bounds__(kFwdThreads)
 fwd_probe_offsets_kernel(IdMap m, const long long* __restrict__ keys, long long n,
                          long long* __restrict__ offsets_out, unsigned* __restrict__ nbm,
-                         unsigned* __restrict__ slotpos, Hooks hk, DevState* st) {
+                         unsigned* __restrict__ slotpos, long long* __restrict__ rec_keys, Hooks hk,
+                         DevState* st) {
   pdl_enter();
   const long long p = (long long)blockIdx.x * kFwdThreads + threadIdx.x;
   bool is_new = false, claimed = false;
   if (p < n) {
     const long long k = __ldg(keys + p);
+    if (rec_keys) rec_keys[p] = k;
     long long o = -1;
     if (k < 0) {
       latch(st, kErrInvalid);

@@ -47,7 +47,7 @@ cudaError_t launch_probe_pool(int G, int NV, int sm_count, IdMap m, RowSpace rs,
 
 // fwd_pool_refs_kernel<G, NV, PM> (gather + pool from per-id row references)
 cudaError_t launch_pool_refs(int G, int NV, int sm_count, RowSpace rs, int dim, const Slot* slots,
-                             const long long* refs, long long n_keys, const long long* bag_off,
+                             long long* refs, long long n_keys, const long long* bag_off,
                              long long n_bags, const float* psw, bool mean, float* out, DevState* st,
                              cudaStream_t s);
 
@@ -57,7 +57,7 @@ cudaError_t launch_probe_pool_bf16(int G, int NV, int sm_count, IdMap m, RowSpac
                                    long long n_bags, const float* psw, bool mean, float* out, unsigned* nbm,
                                    unsigned* slotpos, int ctr_sel, DevState* st, cudaStream_t s);
 cudaError_t launch_pool_refs_bf16(int G, int NV, int sm_count, RowSpace rs, int dim, const Slot* slots,
-                                  const long long* refs, long long n_keys, const long long* bag_off,
+                                  long long* refs, long long n_keys, const long long* bag_off,
                                   long long n_bags, const float* psw, bool mean, float* out, DevState* st,
                                   cudaStream_t s);
 

@@ -25,7 +25,7 @@ cudaError_t launch_probe_pool(int G, int NV, int sm_count, IdMap m, RowSpace rs,
 }
 
 cudaError_t launch_pool_refs(int G, int NV, int sm_count, RowSpace rs, int dim, const Slot* slots,
-                             const long long* refs, long long n_keys, const long long* bag_off,
+                             long long* refs, long long n_keys, const long long* bag_off,
                              long long n_bags, const float* psw, bool mean, float* out, DevState* st,
                              cudaStream_t s) {
 #define DHS_RUN(g, v) \

@@ -23,7 +23,7 @@ cudaError_t launch_probe_pool_bf16(int G, int NV, int sm_count, IdMap m, RowSpac
 }
 
 cudaError_t launch_pool_refs_bf16(int G, int NV, int sm_count, RowSpace rs, int dim, const Slot* slots,
-                                  const long long* refs, long long n_keys, const long long* bag_off,
+                                  long long* refs, long long n_keys, const long long* bag_off,
                                   long long n_bags, const float* psw, bool mean, float* out, DevState* st,
                                   cudaStream_t s) {
 #define DHS_RUN(g, v) \

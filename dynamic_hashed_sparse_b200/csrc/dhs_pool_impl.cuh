@@ -30,7 +30,7 @@ cudaError_t run(int sm_count, IdMap m, RowSpace rs, int dim, const long long* ke
 }
 
 template <int G, int NV, int PM, bool BF>
-cudaError_t run_refs(int sm_count, RowSpace rs, int dim, const Slot* slots, const long long* refs,
+cudaError_t run_refs(int sm_count, RowSpace rs, int dim, const Slot* slots, long long* refs,
                      long long n_keys, const long long* bag_off, long long n_bags, const float* psw,
                      float* out, DevState* st, cudaStream_t s) {
   const int resident =
@@ -55,7 +55,7 @@ cudaError_t run_form(int sm_count, IdMap m, RowSpace rs, int dim, const long lon
 }
 
 template <int G, int NV, bool BF>
-cudaError_t run_refs_form(int sm_count, RowSpace rs, int dim, const Slot* slots, const long long* refs,
+cudaError_t run_refs_form(int sm_count, RowSpace rs, int dim, const Slot* slots, long long* refs,
                           long long n_keys, const long long* bag_off, long long n_bags, const float* psw,
                           bool mean, float* out, DevState* st, cudaStream_t s) {
   if (psw) return run_refs<G, NV, 1, BF>(sm_count, rs, dim, slots, refs, n_keys, bag_off, n_bags, psw, out, st, s);

@@ -196,7 +196,11 @@ dhs_status embbag_forward(dhs_table* t, const int64_t* d_keys, int64_t n_keys,
  * Adam step count advances by one per call.  Keys must be in the table
  * (missing ones are skipped and latch DHS_ERR_NOT_FOUND).
  * d_grad float[n_bags, dim] row-major, 16-byte aligned (rows are copied in
- * 16-byte pieces); the other arguments as in embbag_forward. */
+ * 16-byte pieces); the other arguments as in embbag_forward.
+ * Performance note: when the table's last insert call was a forward whose
+ * bags averaged at least 4 ids, over as many positions as this call, the
+ * rows that forward found are reused at every position holding the same key
+ * (other positions are looked up); the result does not depend on it. */
 dhs_status embbag_backward_update(dhs_table* t, const int64_t* d_keys, int64_t n_keys,
                                   const int64_t* d_bag_offsets, int64_t n_bags,
                                   const float* d_grad, float lr, dhs_stream stream);

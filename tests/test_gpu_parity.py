@@ -247,7 +247,8 @@ def test_segment_runs_at_every_chunk_alignment(n_target, dim):
             o.close()
 
 
-@pytest.mark.parametrize("dim,opt,short", [(64, "adagrad", True), (16, "adam", False), (128, "sgd", True)])
+@pytest.mark.parametrize("dim,opt,short", [(64, "adagrad", True), (16, "adam", False), (128, "sgd", True),
+                                           (64, "adagrad", False), (128, "sgd", False)])
 def test_backward_with_keys_other_than_the_last_forward(dim, opt, short):
     """Backward calls whose keys are not those of the forward just before:
     the keys of an older forward, the same keys at other positions, a third
@@ -258,7 +259,10 @@ def test_backward_with_keys_other_than_the_last_forward(dim, opt, short):
     t, o = make_pair(dim, opt, block_rows=512)
     try:
         def batch(n_bags, universe):
-            lens = rng.integers(0, 3 if short else 9, size=n_bags)
+            # short bags run the fused forward; long ones (at least 4 ids per
+            # bag on average) the split forward, whose record of keys and rows
+            # the backward reads where its keys are the forward's
+            lens = rng.integers(0, 3, size=n_bags) if short else rng.integers(2, 12, size=n_bags)
             offs = np.concatenate([[0], np.cumsum(lens)]).astype(np.int64)
             keys = (rng.integers(0, universe, size=int(offs[-1])) * 7 + 5).astype(np.int64)
             return keys, offs
@@ -287,6 +291,8 @@ def test_backward_with_keys_other_than_the_last_forward(dim, opt, short):
         mixed = kc.copy()
         mixed[::3] = a[0][: mixed[::3].size]  # a third replaced by other known keys
         bwd(mixed, oc)
+        bwd(*c)  # the keys of the last forward, after another backward
+        bwd(*c)
         d = batch(1500, 20000)  # more positions than the last forward, with growth
         fwd(d[0][:-100], np.minimum(d[1], d[0].size - 100))
         fwd(*d)
