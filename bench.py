@@ -632,6 +632,51 @@ def run_l2_peak(mib: int = 32, copies: int = 100, replays: int = 5):
     return 0
 
 
+def run_pcie_peak(mib: int = 896, reps: int = 5):
+    """Host <-> device copy rates from pinned memory: each direction alone
+    and both at once on two streams (the bound of the end-to-end leg, whose
+    steps copy their inputs in while the previous outputs come back).
+    Prints one JSON line."""
+    import torch
+    n = mib << 20
+    h_in = torch.empty(n, dtype=torch.uint8).pin_memory()
+    h_out = torch.empty(n, dtype=torch.uint8).pin_memory()
+    d_in = torch.empty(n, dtype=torch.uint8, device="cuda")
+    d_out = torch.empty(n, dtype=torch.uint8, device="cuda")
+    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+
+    def h2d():
+        s_in.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s_in):
+            d_in.copy_(h_in, non_blocking=True)
+
+    def d2h():
+        s_out.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s_out):
+            h_out.copy_(d_out, non_blocking=True)
+
+    def timed(fns):
+        for f in fns:
+            f()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(reps):
+            for f in fns:
+                f()
+        torch.cuda.current_stream().wait_stream(s_in)
+        torch.cuda.current_stream().wait_stream(s_out)
+        e1.record()
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / reps
+
+    out = {"buffer_bytes": n, "method": "pinned host buffers, cudaMemcpyAsync through torch, CUDA events"}
+    for name, fns in (("h2d_gbs", [h2d]), ("d2h_gbs", [d2h]), ("both_gbs_per_direction", [h2d, d2h])):
+        out[name] = n / (timed(fns) / 1e3) / 1e9
+    print(json.dumps(out))
+    return 0
+
+
 def run_dhs(args):
     world, rank, local = dist_env()
     procs = max(1, min(16, (os.cpu_count() or 2) // max(1, world) - 1))
@@ -807,6 +852,8 @@ def main(argv=None):
     ap.add_argument("--impl", default="dhs", choices=["dhs", "reference"])
     ap.add_argument("--l2-peak", action="store_true",
                     help="only measure the L2-resident copy bandwidth (the yardstick of L2-bound workloads)")
+    ap.add_argument("--pcie-peak", action="store_true",
+                    help="only measure host <-> device copy rates (the yardstick of the end-to-end leg)")
     ap.add_argument("--workload", default=WORKLOAD, choices=list(gen.NAMES))
     ap.add_argument("--workloads", default="all",
                     help="other configs measured after the headline, each run whole: 'all', 'none' or a "
@@ -832,6 +879,8 @@ def main(argv=None):
         ap.error("--steps must be >= 1 and --warmup >= 0")
     if args.l2_peak:
         return run_l2_peak()
+    if args.pcie_peak:
+        return run_pcie_peak()
     if args.impl == "reference":
         return run_reference(args)
     return run_dhs(args)
