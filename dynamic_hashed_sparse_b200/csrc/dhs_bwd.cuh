@@ -84,6 +84,10 @@
 #ifndef DHS_SEG_RUN_TABLE
 #define DHS_SEG_RUN_TABLE 1
 #endif
+//   DHS_SEG_RUN_TABLE_NARROW the same for the lane-group segment kernel
+#ifndef DHS_SEG_RUN_TABLE_NARROW
+#define DHS_SEG_RUN_TABLE_NARROW 1
+#endif
 //   DHS_SEG_FINISH_PIECES pieces of a long segment the segment kernel's warp
 //                     adds itself (longer ones go to the combine kernels)
 #ifndef DHS_SEG_FINISH_PIECES
@@ -676,6 +680,23 @@ struct RowBuf {
   }
 };
 
+// Arrival sums of long segments: see the segment kernel's close step.
+constexpr unsigned kRunBias = 1u << 30;
+
+// Entry of row in the arrival table (inserted when absent); ~0u after
+// latching kErrInternal when the table is full (it is sized for every long
+// segment of sorted input, so only a failed sort gets there).
+__device__ __forceinline__ unsigned run_slot(const RunTable& rt, unsigned row, DevState* st) {
+  unsigned h = (row * 0x9E3779B1u) & rt.mask;  // Fibonacci hashing of the row
+  for (unsigned i = 0; i <= rt.mask; ++i) {
+    const unsigned old = atomicCAS(rt.key + h, 0u, row + 1u);
+    if (old == 0u || old == row + 1u) return h;
+    h = (h + 1u) & rt.mask;
+  }
+  latch(st, kErrInternal);
+  return ~0u;
+}
+
 // Gradient rows in flight per group (ring of shared-memory slots, filled by
 // cp.async): DHS_SEG_RING for a row of <= 128 floats, fewer for wider rows,
 // so that a 256-thread block uses the same shared memory at every width.
@@ -717,7 +738,8 @@ bwd_seg_kernel(const unsigned* __restrict__ skey, const unsigned* __restrict__ s
                double* __restrict__ part_head, double* __restrict__ part_tail,
                int C, unsigned* __restrict__ chunk_ctr,
                unsigned* __restrict__ owners, unsigned* __restrict__ owner_ctr, DevState* st,
-               const unsigned* __restrict__ bagpos, const double* __restrict__ mult, bool mean) {
+               const unsigned* __restrict__ bagpos, const double* __restrict__ mult, bool mean,
+               RunTable rt) {
   pdl_enter();
   constexpr int R = seg_ring(NV);
   extern __shared__ float4 seg_ring_smem[];
@@ -810,32 +832,123 @@ bwd_seg_kernel(const unsigned* __restrict__ skey, const unsigned* __restrict__ s
 #pragma unroll
       for (int e = 0; e < 4; ++e) acc[q][e] = 0.0;
 
-    auto close_piece = [&]() {
+    // the optimizer step on row `key` with the gradient in acc (rb holds the row)
+    auto update = [&](unsigned key) {
+      double sq = 0.0;
+      if (OPT == 3) {
+#pragma unroll
+        for (int q = 0; q < NV; ++q)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const double g = (double)(float)acc[q][e];
+            sq += g * g;
+          }
+#pragma unroll
+        for (int o = 1; o < G; o <<= 1) sq += __shfl_xor_sync(gmask, sq, o, G);
+      }
+      rb.step_store(rs.row(key), dim, gl, G, acc, oa, sq);
+    };
+    auto add_owner = [&](unsigned oc) {  // for the combine kernels
+      const unsigned slot = atomicAdd(owner_ctr, 1u);
+      if (slot < (unsigned)nchunks) owners[slot] = oc;
+      else latch(st, kErrInternal);
+    };
+    // Arrival of a long segment's piece (its partial written), as in
+    // bwd_segw_kernel: the owner adds 1 + c + bias, the piece where the
+    // segment ends 1 + bias - c, any other piece 1; the group whose addition
+    // completes 1 + 2 bias adds the pieces up in chunk order and steps the row
+    // (or, past max_pieces, hands the segment to the combine kernels).  A
+    // chunk has at most two such pieces, its first (mode 1) and its last
+    // (mode 3); their arrivals wait until the chunk's pairs are done, which
+    // keeps this code out of the loop over pairs.
+    auto arrive = [&](unsigned key, int pmode, bool is_end) {
+      unsigned slot = ~0u, fin = 0u;
+      if (gl == 0) {
+        slot = run_slot(rt, key, st);
+        if (slot != ~0u) {
+          if (pmode == 3) *(volatile unsigned*)(rt.c0 + slot) = (unsigned)c;
+          if (is_end) *(volatile unsigned*)(rt.c1 + slot) = (unsigned)c;
+        }
+      }
+      __threadfence();  // this lane's partial (and the chunk index) before the arrival
+      __syncwarp(gmask);
+      if (gl == 0 && slot != ~0u) {
+        unsigned add = 1u;
+        if (pmode == 3) add += (unsigned)c + kRunBias;
+        if (is_end) add += kRunBias - (unsigned)c;
+        const unsigned old = atomicAdd(rt.ctr + slot, add);
+        fin = old + add == 1u + 2u * kRunBias ? 1u : 0u;
+      }
+      fin = __shfl_sync(gmask, fin, 0, G);
+      if (!fin) return;
+      slot = __shfl_sync(gmask, slot, 0, G);
+      __threadfence();
+      const unsigned f0 = *(volatile unsigned*)(rt.c0 + slot);
+      const unsigned f1 = *(volatile unsigned*)(rt.c1 + slot);
+      if (f1 < f0 || f1 >= (unsigned)nchunks) {
+        if (gl == 0) latch(st, kErrInternal);
+      } else if (f1 - f0 + 1u <= rt.max_pieces) {
+        // the first chunk's tail partial, then each later chunk's head
+        // partial, added in chunk order (PF pieces in flight)
+        constexpr int PF = NV >= 2 ? (OPT == 1 ? 4 : 2) : 4;  // (registers: no spills)
+        const unsigned np = f1 - f0 + 1u;
+#pragma unroll
+        for (int q = 0; q < NV; ++q)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) acc[q][e] = 0.0;
+        for (unsigned k0 = 0; k0 < np; k0 += PF) {
+          double v[PF][NV][4];
+#pragma unroll
+          for (int u = 0; u < PF; ++u) {
+            const unsigned k = k0 + (unsigned)u;
+            const double* src = k == 0 ? part_tail + (long long)f0 * pstride
+                                       : part_head + (long long)(f0 + k) * pstride;
+#pragma unroll
+            for (int q = 0; q < NV; ++q)
+#pragma unroll
+              for (int e = 0; e < 4; e += 2) {
+                const double2 x = k < np ? __ldcg(reinterpret_cast<const double2*>(src + (q * G + gl) * 4 + e))
+                                         : make_double2(0.0, 0.0);
+                v[u][q][e] = x.x;
+                v[u][q][e + 1] = x.y;
+              }
+          }
+#pragma unroll
+          for (int u = 0; u < PF; ++u)
+            if (k0 + (unsigned)u < np)
+#pragma unroll
+              for (int q = 0; q < NV; ++q)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) acc[q][e] += v[u][q][e];
+        }
+        rb.load(rs.row(key), dim, gl, G);
+        update(key);
+      } else if (gl == 0) {
+        add_owner(f0);
+      }
+    };
+    unsigned pend1 = ~0u, pend3 = ~0u;  // rows of the chunk's long pieces awaiting arrival
+    bool pend1_end = false;
+    // ended: the segment's last pair is in this piece
+    auto close_piece = [&](bool ended) {
       if (mode == 1 || mode == 3) {
         double* o = (mode == 1 ? part_head : part_tail) + (long long)c * pstride;
 #pragma unroll
         for (int q = 0; q < NV; ++q)
 #pragma unroll
           for (int e = 0; e < 4; ++e) o[(q * G + gl) * 4 + e] = acc[q][e];
-        if (mode == 3 && gl == 0) {  // for the combine; at most one per chunk for sorted pairs
-          const unsigned slot = atomicAdd(owner_ctr, 1u);
-          if (slot < (unsigned)nchunks) owners[slot] = (unsigned)c;
-          else latch(st, kErrInternal);
+        if (rt.key != nullptr && cur < nrows) {
+          if (mode == 1) {
+            pend1 = cur;
+            pend1_end = ended;
+          } else {
+            pend3 = cur;
+          }
+        } else if (mode == 3 && gl == 0) {  // for the combine; at most one per chunk for sorted pairs
+          add_owner((unsigned)c);
         }
       } else if (mode == 2 && cur < nrows) {
-        double sq = 0.0;
-        if (OPT == 3) {
-#pragma unroll
-          for (int q = 0; q < NV; ++q)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const double g = (double)(float)acc[q][e];
-              sq += g * g;
-            }
-#pragma unroll
-          for (int o = 1; o < G; o <<= 1) sq += __shfl_xor_sync(gmask, sq, o, G);
-        }
-        rb.step_store(rs.row(cur), dim, gl, G, acc, oa, sq);
+        update(cur);
       }
 #pragma unroll
       for (int q = 0; q < NV; ++q)
@@ -856,7 +969,7 @@ bwd_seg_kernel(const unsigned* __restrict__ skey, const unsigned* __restrict__ s
       }
       const unsigned kt = __shfl_sync(gmask, ck, i - cws, G);
       if (kt != cur) {
-        close_piece();
+        close_piece(true);
         if (i >= end) {
           done = true;
           break;
@@ -866,7 +979,7 @@ bwd_seg_kernel(const unsigned* __restrict__ skey, const unsigned* __restrict__ s
         mode = (has2 && fwd2 == cur) ? 3 : 2;
         if (mode == 2 && cur < nrows) rb.load(rs.row(cur), dim, gl, G);
       } else if (i == end && mode != 2) {
-        close_piece();  // a long piece stops at the chunk end
+        close_piece(false);  // a long piece stops at the chunk end
         done = true;
         break;
       }
@@ -892,8 +1005,10 @@ bwd_seg_kernel(const unsigned* __restrict__ skey, const unsigned* __restrict__ s
       }
       produce();  // refill the slot just read with pair i + R
     }
-    if (!done) close_piece();  // reached the end of the array with a piece open
+    if (!done) close_piece(true);  // reached the end of the array with a piece open
     cp_async_wait_all();  // the ring is reused by the next chunk
+    if (pend1 != ~0u) arrive(pend1, 1, pend1_end);
+    if (pend3 != ~0u) arrive(pend3, 3, false);
     if (gl == 0) {
       if (cur >= nrows && nseg) --nseg;  // the missing-key run is not a row
       nseg_total += nseg;
@@ -1049,23 +1164,6 @@ __device__ __forceinline__ void segw_st(float* p, const float (&v)[CPL], int col
         *reinterpret_cast<float4*>(p + col0 + 4 * k) =
             make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
   }
-}
-
-// Arrival sums of long segments: see the segment kernel's close step.
-constexpr unsigned kRunBias = 1u << 30;
-
-// Entry of row in the arrival table (inserted when absent); ~0u after
-// latching kErrInternal when the table is full (it is sized for every long
-// segment of sorted input, so only a failed sort gets there).
-__device__ __forceinline__ unsigned run_slot(const RunTable& rt, unsigned row, DevState* st) {
-  unsigned h = (row * 0x9E3779B1u) & rt.mask;  // Fibonacci hashing of the row
-  for (unsigned i = 0; i <= rt.mask; ++i) {
-    const unsigned old = atomicCAS(rt.key + h, 0u, row + 1u);
-    if (old == 0u || old == row + 1u) return h;
-    h = (h + 1u) & rt.mask;
-  }
-  latch(st, kErrInternal);
-  return ~0u;
 }
 
 // EXT (extended pooling): sort values are positions; the pair's bag is

@@ -657,7 +657,8 @@ dhs_status launch_seg(dhs_table* t, const unsigned* sk, const unsigned* sv, long
               : t->opt == DHS_ADAM ? (ext ? launch_seg_adam_ext : launch_seg_adam)
                                    : (ext ? launch_seg_rowwise_ext : launch_seg_rowwise);
     e = fn(G, NV, t->sm_count, sk, sv, n, grad, nb, t->dim, rowspace(t), oa, part_head, part_tail,
-           seg_chunk(n), chunk_ctr, owners, owner_ctr, t->st, bagpos, mult, mean, s);
+           seg_chunk(n), chunk_ctr, owners, owner_ctr, t->st, bagpos, mult, mean,
+           DHS_SEG_RUN_TABLE_NARROW ? rt : RunTable{}, s);
   }
   t->n_launches++;
   if (e != cudaSuccess) cudaGetLastError();

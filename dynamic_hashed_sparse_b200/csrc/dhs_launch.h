@@ -70,7 +70,7 @@ cudaError_t launch_pool_refs_bf16(int G, int NV, int sm_count, RowSpace rs, int 
                     const OptArgs& oa, double* part_head, double* part_tail,                    \
                     int chunk, unsigned* chunk_ctr, unsigned* owners, unsigned* owner_ctr,      \
                     DevState* st, const unsigned* bagpos, const double* mult, bool mean,        \
-                    cudaStream_t s);
+                    const RunTable& rt, cudaStream_t s);
 DHS_SEG_DECL(launch_seg_sgd)
 DHS_SEG_DECL(launch_seg_adagrad)
 DHS_SEG_DECL(launch_seg_adam)

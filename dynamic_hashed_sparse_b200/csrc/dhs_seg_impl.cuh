@@ -17,7 +17,7 @@ cudaError_t run(int sm_count, const unsigned* skey, const unsigned* sval, long l
                 const float* grad, long long n_bags, int dim, RowSpace rs, const OptArgs& oa,
                 double* part_head, double* part_tail, int chunk,
                 unsigned* chunk_ctr, unsigned* owners, unsigned* owner_ctr, DevState* st,
-                const unsigned* bagpos, const double* mult, bool mean, cudaStream_t s) {
+                const unsigned* bagpos, const double* mult, bool mean, const RunTable& rt, cudaStream_t s) {
   const size_t smem = seg_smem_bytes(G, NV);
   const int resident = blocks_per_sm((const void*)bwd_seg_kernel<G, NV, OPT, EXT>, 256, smem) * sm_count;
   const long long nchunks = (n + chunk - 1) / chunk;
@@ -26,7 +26,7 @@ cudaError_t run(int sm_count, const unsigned* skey, const unsigned* sval, long l
   const long long grid = std::min<long long>(need, resident);
   launch_k(bwd_seg_kernel<G, NV, OPT, EXT>, (unsigned)grid, 256, smem, s, skey, sval, n, grad, n_bags, dim, rs, oa,
                                                                    part_head, part_tail, chunk, chunk_ctr,
-                                                                   owners, owner_ctr, st, bagpos, mult, mean);
+                                                                   owners, owner_ctr, st, bagpos, mult, mean, rt);
   return cudaGetLastError();
 }
 
@@ -35,10 +35,10 @@ cudaError_t launch(int G, int NV, int sm_count, const unsigned* skey, const unsi
                    long long n, const float* grad, long long n_bags, int dim, RowSpace rs,
                    const OptArgs& oa, double* part_head, double* part_tail,
                    int chunk, unsigned* chunk_ctr, unsigned* owners, unsigned* owner_ctr, DevState* st,
-                   const unsigned* bagpos, const double* mult, bool mean, cudaStream_t s) {
+                   const unsigned* bagpos, const double* mult, bool mean, const RunTable& rt, cudaStream_t s) {
 #define DHS_RUN(g, v)                                                                                \
   run<g, v, OPT, EXT>(sm_count, skey, sval, n, grad, n_bags, dim, rs, oa, part_head, part_tail, chunk, \
-                      chunk_ctr, owners, owner_ctr, st, bagpos, mult, mean, s)
+                      chunk_ctr, owners, owner_ctr, st, bagpos, mult, mean, rt, s)
   switch (G * 100 + NV) {
     case 102: return DHS_RUN(1, 2);
     case 202: return DHS_RUN(2, 2);
@@ -105,10 +105,10 @@ cudaError_t launch_w(int cpl, bool bf16, int sm_count, const unsigned* skey, con
                     const OptArgs& oa, double* part_head, double* part_tail,                    \
                     int chunk, unsigned* chunk_ctr, unsigned* owners, unsigned* owner_ctr,      \
                     DevState* st, const unsigned* bagpos, const double* mult, bool mean,        \
-                    cudaStream_t s) {                                                           \
+                    const RunTable& rt, cudaStream_t s) {                                       \
     return seg_impl::launch<OPT_, EXT_>(G, NV, sm_count, skey, sval, n, grad, n_bags, dim, rs, oa, \
                                         part_head, part_tail, chunk, chunk_ctr, owners, owner_ctr, \
-                                        st, bagpos, mult, mean, s);                             \
+                                        st, bagpos, mult, mean, rt, s);                         \
   }                                                                                             \
   cudaError_t NAME_##_w(int cpl, bool bf16, int sm_count, const unsigned* skey, const unsigned* sval, \
                         long long n, const float* grad, long long n_bags, int dim, RowSpace rs,  \

@@ -183,12 +183,13 @@ def test_dims_and_optimizers(dim, opt, bags):
 def test_hot_key_spanning_many_sort_chunks(occ):
     """One key occurs `occ` times (its run covers one sort chunk of 32 pairs up
     to hundreds of them), mixed with a tail of other keys before and after it
-    in row order; both segment kernels (narrow and wide rows).  Runs of about
-    32 chunks (1,000 to 1,060 occurrences) sit at the boundary between a long
-    segment that the wide segment kernel's warp finishes and one that goes to
-    the combine kernels."""
+    in row order; both segment kernels (narrow and wide rows), every
+    optimizer.  Runs of about 32 chunks (1,000 to 1,060 occurrences) sit at
+    the boundary between a long segment that the segment kernel's warp or
+    lane group finishes and one that goes to the combine kernels."""
     rng = np.random.default_rng(occ)
-    for dim, opt in ((32, "adagrad"), (32, "adam"), (32, "adagrad_rowwise"), (12, "adagrad"), (128, "sgd")):
+    for dim, opt in ((32, "adagrad"), (32, "adam"), (32, "adagrad_rowwise"), (12, "adagrad"), (128, "sgd"),
+                     (16, "sgd"), (20, "adam"), (16, "adagrad_rowwise")):
         t, o = make_pair(dim, opt)
         try:
             warm = np.arange(1, 600, dtype=np.int64)  # rows 0.. for the tail keys
