@@ -702,7 +702,7 @@ dhs_status launch_assign(dhs_table* t, const long long* keys, long long n, cudaS
       (unsigned*)t->b_gpref.p, (const unsigned*)t->b_slotpos.p, nwords, ngroups, hooks(t), t->st);
   t->n_launches += 2;
   DHS_TRY(last_launch());
-  launch_k(fwd_assign_kernel, (unsigned)(ngroups * kAssignSplit), kGroupThreads, 0, s, 
+  launch_k(fwd_assign_kernel, (unsigned)ngroups, kGroupThreads, 0, s, 
       t->slots, rowspace(t), t->dim, keys, (const unsigned*)t->b_fbm.p, (const unsigned*)t->b_gpref.p,
       (const unsigned*)t->b_slotpos.p, nwords, ngroups, hooks(t), t->st);
   return last_launch();

@@ -576,40 +576,34 @@ fwd_mark_kernel(Slot* __restrict__ slots, unsigned* __restrict__ nbm,
   }
 }
 
-// Offset assignment + row initialisation.  kAssignSplit blocks of 1024
-// threads per group of 4096 positions: the group's new keys have consecutive
-// ranks (the prefix over the group's 128 bitmap words plus the bit's place in
-// its word), so their rows are one contiguous run (split only at a block
-// edge).  Every block of a group recomputes the word prefix; block part 0
-// writes each first occurrence's row offset into its slot; block `part`
-// writes its share of the run with coalesced 16-byte stores (initial weights
-// from splitmix64(key), optimizer state zero).  One block per group measured
-// fastest (more blocks per group repeat the prefix and the key gathering for
-// fewer rows each).
-constexpr int kAssignSplit = 1;
+// Offset assignment + row initialisation of group g (4096 batch positions,
+// 1024 threads): the group's new keys have consecutive ranks from rank0 (the
+// prefix over the group's 128 first-occurrence words, fw_of(word), plus the
+// bit's place in its word), so their rows are one contiguous run.  Each
+// first occurrence's row offset goes into its slot; the run is written with
+// coalesced 16-byte stores (initial weights from splitmix64(key), optimizer
+// state zero).  Rank q takes free-list row free_list[free_base + q] while
+// q < m_free, else appended row row_base + (q - m_free).
 #ifndef DHS_ASSIGN_COLUMNS
 #define DHS_ASSIGN_COLUMNS 1  // column-per-thread row initialisation (0: flat index loop only)
 #endif
 
-__global__ void __launch_bounds__(kGroupThreads, 2)
-fwd_assign_kernel(Slot* __restrict__ slots, RowSpace rs, int dim, const long long* __restrict__ keys,
-                  const unsigned* __restrict__ fbm, const unsigned* __restrict__ gpref,
-                  const unsigned* __restrict__ slotpos, long long nwords, long long ngroups,
-                  Hooks hk, DevState* st) {
-  pdl_enter();
-  __shared__ unsigned long long skey[kGroupPositions];  // 32 KB
-  __shared__ unsigned wpre[kGroupWords];
-  __shared__ unsigned s_total;
+template <class FW>
+__device__ __forceinline__ void assign_group(long long g, FW fw_of, unsigned long long rank0,
+                                             unsigned long long m_free, unsigned long long free_base,
+                                             unsigned long long row_base, Slot* __restrict__ slots,
+                                             RowSpace rs, int dim, const long long* __restrict__ keys,
+                                             const unsigned* __restrict__ slotpos, long long nwords, Hooks hk,
+                                             DevState* st, unsigned long long* skey, unsigned* wpre,
+                                             unsigned* s_total) {
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-  const long long g = blockIdx.x / kAssignSplit;
-  const int part = (int)(blockIdx.x % kAssignSplit);
   if (threadIdx.x < 32) {
     // exclusive prefix of the 128 words' counts (4 per lane, in word order)
     unsigned c[4], t = 0;
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
       const long long w = g * kGroupWords + lane * 4 + k;
-      c[k] = w < nwords ? __popc(fbm[w]) : 0u;
+      c[k] = w < nwords ? __popc(fw_of(w)) : 0u;
       t += c[k];
     }
     unsigned inc = t;
@@ -624,32 +618,27 @@ fwd_assign_kernel(Slot* __restrict__ slots, RowSpace rs, int dim, const long lon
       wpre[lane * 4 + k] = run;
       run += c[k];
     }
-    if (lane == 31) s_total = inc;
+    if (lane == 31) *s_total = inc;
   }
   __syncthreads();
-  const unsigned total = s_total;
-  // this block's share of the group's rows: [r_lo, r_hi)
-  const unsigned r_lo = (unsigned)(((unsigned long long)total * part) / kAssignSplit);
-  const unsigned r_hi = (unsigned)(((unsigned long long)total * (part + 1)) / kAssignSplit);
-  if (r_lo >= r_hi && part != 0) return;
+  const unsigned total = *s_total;
+  const unsigned r_lo = 0, r_hi = total;  // the group's rows
   // rank q of the call's new keys: free-list row q while q < m_free, else
   // appended row row_base + (q - m_free)
-  const unsigned long long m_free = st->m_free, free_base = st->free_base, row_base = st->row_base;
   auto row_of = [&](unsigned long long q) -> unsigned long long {
     return q < m_free ? (unsigned long long)hk.free_list[free_base + q] : row_base + (q - m_free);
   };
-  const unsigned long long rank0 = gpref[g];  // the group's first rank
   const unsigned long long limit = st->n_blocks << rs.log2_br;
 #pragma unroll
   for (int k = 0; k < kGroupPerThread; ++k) {
     const int wi = k * 32 + wid;
     const long long w = g * kGroupWords + wi;
-    const unsigned fw = w < nwords ? fbm[w] : 0u;
+    const unsigned fw = w < nwords ? fw_of(w) : 0u;
     if ((fw >> lane) & 1u) {
       const unsigned j = wpre[wi] + __popc(fw & lanemask_lt());
       const unsigned long long p = (unsigned long long)(g * kGroupPositions + k * kGroupThreads + threadIdx.x);
       if (j >= r_lo && j < r_hi) skey[j] = (unsigned long long)__ldg(keys + p);  // the key first seen at p
-      if (part == 0) {
+      {
         const unsigned sl = slotpos[p];
         const unsigned long long row = row_of(rank0 + j);
         if (rank0 + j < m_free) atomicAnd(hk.free_bm + (row >> 5), ~(1u << (row & 31)));  // no longer free
@@ -727,6 +716,25 @@ fwd_assign_kernel(Slot* __restrict__ slots, RowSpace rs, int dim, const long lon
           make_uint4(pack_bf16x2(a.x, a.y), pack_bf16x2(a.z, a.w), pack_bf16x2(b.x, b.y), pack_bf16x2(b.z, b.w));
     }
   }
+}
+
+// The two-kernel form (first-occurrence marking by fwd_mark_kernel, whose
+// last block scans the group counts and reserves the rows): one block per
+// group.  More blocks per group (each writing a share of the run) measured
+// slower: each repeated the prefix and the key gathering for fewer rows.
+__global__ void __launch_bounds__(kGroupThreads, 2)
+fwd_assign_kernel(Slot* __restrict__ slots, RowSpace rs, int dim, const long long* __restrict__ keys,
+                  const unsigned* __restrict__ fbm, const unsigned* __restrict__ gpref,
+                  const unsigned* __restrict__ slotpos, long long nwords, long long ngroups,
+                  Hooks hk, DevState* st) {
+  pdl_enter();
+  __shared__ unsigned long long skey[kGroupPositions];  // 32 KB
+  __shared__ unsigned wpre[kGroupWords];
+  __shared__ unsigned s_total;
+  const long long g = blockIdx.x;
+  auto fw_of = [&](long long w) -> unsigned { return fbm[w]; };
+  assign_group(g, fw_of, (unsigned long long)gpref[g], st->m_free, st->free_base, st->row_base, slots, rs, dim,
+               keys, slotpos, nwords, hk, st, skey, wpre, &s_total);
 }
 
 // ---- IDMap maintenance and read-only access ----
