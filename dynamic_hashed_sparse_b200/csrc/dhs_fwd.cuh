@@ -23,6 +23,12 @@
 #ifndef DHS_POOL_SPLIT_LEN
 #define DHS_POOL_SPLIT_LEN 4
 #endif
+// Blocks per SM the fused pool kernel is compiled for with 32-lane groups
+// and one 16-byte unit per lane (rows of 128 fp32 or 256 bf16 weights;
+// register budget 65536 / (256 * blocks)); 4 at the other widths
+#ifndef DHS_POOL_MINB
+#define DHS_POOL_MINB 4
+#endif
 
 namespace dhs {
 
@@ -218,7 +224,7 @@ __device__ __forceinline__ int pool_fetch(unsigned* ctr, unsigned gmask, int gl,
 // 1 sum with per-sample weights psw[position] scaling each row, 2 mean
 // (each bag divided by its length).  BF: the table's weights are bf16.
 template <int G, int NV, int PM, bool BF>
-__global__ void __launch_bounds__(kFwdThreads, NV == 1 ? 4 : (NV == 2 ? 2 : 1))
+__global__ void __launch_bounds__(kFwdThreads, NV == 1 ? (G == 32 ? DHS_POOL_MINB : 4) : (NV == 2 ? 2 : 1))
 fwd_probe_pool_kernel(IdMap m, RowSpace rs, int dim, const long long* __restrict__ keys,
                       long long n_keys, const long long* __restrict__ bag_off, long long n_bags,
                       const float* __restrict__ psw,
