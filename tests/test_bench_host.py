@@ -107,3 +107,18 @@ def test_reserve_policy():
     assert bench.resolve_reserve(w, 10, "-1") == bench.default_reserve(w, 10)
     hot = bench.make_workload("hot_key", 0)
     assert bench.resolve_reserve(hot, 20, "on-demand") == 50_000_001
+
+
+def test_segment_kernel_label_follows_the_library_rule():
+    """The roofline names the segment kernel the library runs: the lane-group
+    kernel below 32 floats, and for fp32 rows of 33-64 floats while rows get
+    fewer than 8 ids on average; the warp kernel otherwise."""
+    sys.path.insert(0, ROOT)
+    import bench
+    assert bench.narrow_seg(16, "f32", 1000, 10)
+    assert not bench.narrow_seg(32, "f32", 1000, 999)          # 32 floats: the warp kernel
+    assert bench.narrow_seg(64, "f32", 6_550_000, 1_780_000)   # sequence_bags: 3.7 ids per row
+    assert not bench.narrow_seg(64, "f32", 5_240_000, 85_000)  # hot_key: 62 ids per row
+    assert not bench.narrow_seg(64, "bf16", 6_550_000, 1_780_000)
+    assert not bench.narrow_seg(128, "f32", 1_700_000, 380_000)
+    assert not bench.narrow_seg(64, "f32", 100, 0)             # no backward seen yet
