@@ -128,7 +128,8 @@ def load_traffic(kernel: str):
 class ClockSampler:
     """SM clock and clock-event reasons of this process's GPU, sampled every
     ~2 ms by a thread through NVML while the timed region runs (two cheap
-    queries per sample, so the sampling does not stall the driver)."""
+    queries per sample, so the sampling does not hold up the GPU driver or
+    the launching thread)."""
 
     REASONS = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
                ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
